@@ -1,0 +1,303 @@
+"""Plain CPU oracle for the MACAQ W4A4 MXFP4 linear (dense and grouped).
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / reference leg of ``bench.py`` may import this package.  It
+shares no code with the CUDA library and never imports it.
+
+The arithmetic lives in ``macaq_oracle.c`` (plain C, built with
+``-ffp-contract=off`` so every float operation is one IEEE rounding); this
+module only loads it with ctypes and marshals numpy arrays.  Every function
+cites what it follows on the pages:
+
+* "MACAQ W4A4 fused dense and grouped matmul for Ascend 950", summary: channel
+  scaling, block-32 BF16 Hadamard rotation, MXFP4 activation quantisation,
+  matmul with BF16 output; weight transform offline.
+* same page, "Latency against existing native CANN operators": the MX
+  quantisation is block32 E2M1, round-to-even, scale_alg=0.
+* "torch_npu.npu_grouped_matmul", function description and the group_list /
+  group_list_type parameters: grouped y_i = x_i @ weight_i.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "macaq_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+OK = 0
+ERR_SHAPE = -3
+ERR_TOO_MANY_GROUPS = -6
+ERR_GROUP_LIST_TYPE = -7
+ERR_GROUP_LIST_INVALID = -10
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (no FMA contraction, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call([
+            "gcc", "-O2", "-std=gnu11", "-ffp-contract=off", "-fno-fast-math",
+            "-fopenmp", "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+_lib = None
+
+
+def _L():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        I64 = ctypes.c_int64
+        I = ctypes.c_int
+        sig = {
+            "oracle_f32_to_bf16": (ctypes.c_uint16, [ctypes.c_float]),
+            "oracle_bf16_to_f64": (ctypes.c_double, [ctypes.c_uint16]),
+            "oracle_fwht32": (None, [P, P, I64]),
+            "oracle_e8m0_from_amax": (I, [ctypes.c_float]),
+            "oracle_e2m1_decode": (ctypes.c_double, [I]),
+            "oracle_e2m1_encode": (I, [ctypes.c_double]),
+            "oracle_mx_quantize_blocks": (None, [P, I64, P, P]),
+            "oracle_act_rotate": (None, [P, P, I64, I64, P]),
+            "oracle_quantize_act": (I, [P, P, I64, I64, P, P, I]),
+            "oracle_quantize_weights": (I, [P, P, I64, I64, P, P, I]),
+            "oracle_gemm": (I, [P, P, P, P, I64, I64, I64, P, I]),
+            "oracle_gemm_at": (I, [P, P, P, P, I64, P, P, I64, P]),
+            "oracle_group_offsets": (I, [P, I, I64, I64, P]),
+            "oracle_grouped_mm": (I, [P, P, P, P, I, I64, I64, I64, I64, P, I]),
+            "oracle_linear_f64": (None, [P, P, I64, I64, I64, P]),
+            "oracle_transform_f64": (None, [P, P, P, I64, I64, I64, P]),
+            "oracle_dequantize": (None, [P, P, I64, I64, P]),
+            "oracle_quantize_plain": (I, [P, I64, I64, P, P]),
+            "oracle_num_threads": (I, []),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(lib, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = lib
+    return _lib
+
+
+def _p(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# --------------------------------------------------------------------------
+# element-level pieces
+# --------------------------------------------------------------------------
+
+def f32_to_bf16(v) -> np.ndarray:
+    """binary32 -> bf16 bit pattern, round-to-nearest-even (the BF16 rounding
+    the summary's "BF16 Hadamard rotation" implies)."""
+    v = _c(v, np.float32).ravel()
+    f = _L().oracle_f32_to_bf16
+    return np.array([f(float(x)) for x in v], dtype=np.uint16)
+
+
+def bf16_to_f64(h) -> np.ndarray:
+    h = _c(h, np.uint16)
+    return (h.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def fwht32(v) -> np.ndarray:
+    """Unnormalised block-32 Sylvester Hadamard transform in FP32 (summary:
+    "block-32 BF16 Hadamard rotation"; butterfly order h = 1..16)."""
+    v = _c(v, np.float32)
+    assert v.size % 32 == 0
+    out = np.empty_like(v)
+    _L().oracle_fwht32(_p(v), _p(out), v.size // 32)
+    return out
+
+
+def e8m0_from_amax(amax: float) -> int:
+    """Shared scale code, OCP MX scale_alg=0 (latency section: scale_alg=0)."""
+    return int(_L().oracle_e8m0_from_amax(float(amax)))
+
+
+def e2m1_encode(v: float) -> int:
+    """E2M1 round-to-nearest-even with saturation (latency section: E2M1,
+    round-to-even)."""
+    return int(_L().oracle_e2m1_encode(float(v)))
+
+
+def e2m1_decode(code: int) -> float:
+    return float(_L().oracle_e2m1_decode(int(code)))
+
+
+def mx_quantize_blocks(v) -> tuple[np.ndarray, np.ndarray]:
+    """MX quantisation of consecutive 32-element blocks of fp32 values."""
+    v = _c(v, np.float32).ravel()
+    assert v.size % 32 == 0
+    nb = v.size // 32
+    codes = np.empty(nb * 16, np.uint8)
+    scales = np.empty(nb, np.uint8)
+    _L().oracle_mx_quantize_blocks(_p(v), nb, _p(codes), _p(scales))
+    return codes, scales
+
+
+def unpack_codes(codes: np.ndarray) -> np.ndarray:
+    """[..., K/2] packed bytes -> [..., K] 4-bit codes (element 2j = low nibble)."""
+    lo = codes & 0xF
+    hi = codes >> 4
+    return np.stack([lo, hi], axis=-1).reshape(*codes.shape[:-1], codes.shape[-1] * 2)
+
+
+# --------------------------------------------------------------------------
+# activation and weight paths
+# --------------------------------------------------------------------------
+
+def act_rotate(x_bf16: np.ndarray, D: np.ndarray) -> np.ndarray:
+    """u = RNE_bf16(FWHT32(RNE_bf16(x * RN32(1/D)))) as bf16 bits [M, K]
+    (summary: channel scaling, then block-32 BF16 Hadamard rotation)."""
+    x = _c(x_bf16, np.uint16)
+    D = _c(D, np.float32)
+    M, K = x.shape
+    u = np.empty_like(x)
+    _L().oracle_act_rotate(_p(x), _p(D), M, K, _p(u))
+    return u
+
+
+def quantize_act(x_bf16: np.ndarray, D: np.ndarray, nthreads: int = 0):
+    """Activation codes [M, K/2] and E8M0 scales [M, K/32] (summary: scaling,
+    rotation, MXFP4 activation quantisation)."""
+    x = _c(x_bf16, np.uint16)
+    D = _c(D, np.float32)
+    M, K = x.shape
+    codes = np.empty((M, K // 2), np.uint8)
+    scales = np.empty((M, K // 32), np.uint8)
+    st = _L().oracle_quantize_act(_p(x), _p(D), M, K, _p(codes), _p(scales), nthreads)
+    assert st == OK, st
+    return codes, scales
+
+
+def quantize_weights(W: np.ndarray, D: np.ndarray, nthreads: int = 0):
+    """Offline weight codes/scales from FWHT32(RN32(W*D)) in FP32 (summary:
+    weight transformation is offline).  W [N, K] or [E, N, K]; D [K] or [E, K]."""
+    W = _c(W, np.float32)
+    D = _c(D, np.float32)
+    if W.ndim == 3:
+        outs = [quantize_weights(W[e], D[e], nthreads) for e in range(W.shape[0])]
+        return np.stack([o[0] for o in outs]), np.stack([o[1] for o in outs])
+    N, K = W.shape
+    codes = np.empty((N, K // 2), np.uint8)
+    scales = np.empty((N, K // 32), np.uint8)
+    st = _L().oracle_quantize_weights(_p(W), _p(D), N, K, _p(codes), _p(scales), nthreads)
+    assert st == OK, st
+    return codes, scales
+
+
+def gemm(qa, sa, qw, sw, nthreads: int = 0) -> np.ndarray:
+    """Exact block-scaled product, y = RNE_bf16(2^-5 * sum) as bf16 bits [M, N]
+    (summary: matrix multiplication producing BF16 output)."""
+    qa, sa, qw, sw = (_c(a, np.uint8) for a in (qa, sa, qw, sw))
+    M, K = qa.shape[0], qa.shape[1] * 2
+    N = qw.shape[0]
+    y = np.empty((M, N), np.uint16)
+    st = _L().oracle_gemm(_p(qa), _p(sa), _p(qw), _p(sw), M, N, K, _p(y), nthreads)
+    assert st == OK, st
+    return y
+
+
+def gemm_at(qa, sa, qw, sw, rows, cols) -> np.ndarray:
+    """Exact outputs at the given (row, col) pairs only."""
+    qa, sa, qw, sw = (_c(a, np.uint8) for a in (qa, sa, qw, sw))
+    K = qa.shape[1] * 2
+    rows = _c(rows, np.int64)
+    cols = _c(cols, np.int64)
+    out = np.empty(rows.size, np.uint16)
+    st = _L().oracle_gemm_at(_p(qa), _p(sa), _p(qw), _p(sw), K, _p(rows), _p(cols), rows.size,
+                             _p(out))
+    assert st == OK, st
+    return out
+
+
+def dense_mm(x_bf16, D, W, nthreads: int = 0) -> np.ndarray:
+    """Whole dense MACAQ linear: bf16 bits [M, N]."""
+    qa, sa = quantize_act(x_bf16, D, nthreads)
+    qw, sw = quantize_weights(W, D, nthreads)
+    return gemm(qa, sa, qw, sw, nthreads)
+
+
+def group_offsets(group_list, group_list_type: int, M: int):
+    """Row offsets [E+1] from group_list (npu_grouped_matmul, group_list and
+    group_list_type).  Returns (status, offsets)."""
+    gl = _c(group_list, np.int64)
+    E = gl.size
+    off = np.zeros(max(E + 1, 2), np.int64)
+    st = _L().oracle_group_offsets(_p(gl), int(group_list_type), E, M, _p(off))
+    return int(st), off[:E + 1]
+
+
+def grouped_mm(x_bf16, D, W, group_list, group_list_type: int, nthreads: int = 0):
+    """Grouped MACAQ linear (npu_grouped_matmul, single x / single 3-D weight /
+    single y).  Returns (status, y bf16 bits [M, N])."""
+    x = _c(x_bf16, np.uint16)
+    D = _c(D, np.float32)
+    W = _c(W, np.float32)
+    gl = _c(group_list, np.int64)
+    M, K = x.shape
+    E, N, _ = W.shape
+    y = np.zeros((M, N), np.uint16)
+    st = _L().oracle_grouped_mm(_p(x), _p(D), _p(W), _p(gl), int(group_list_type), E, M, N, K,
+                                _p(y), nthreads)
+    return int(st), y
+
+
+def linear_f64(x_bf16, W) -> np.ndarray:
+    x = _c(x_bf16, np.uint16)
+    W = _c(W, np.float32)
+    M, K = x.shape
+    N = W.shape[0]
+    out = np.empty((M, N), np.float64)
+    _L().oracle_linear_f64(_p(x), _p(W), M, N, K, _p(out))
+    return out
+
+
+def transform_f64(x_bf16, D, W) -> np.ndarray:
+    """((x/D)H).((W*D)H)^T / 32 in binary64, with no rounding to BF16 or MXFP4."""
+    x = _c(x_bf16, np.uint16)
+    D = _c(D, np.float32)
+    W = _c(W, np.float32)
+    M, K = x.shape
+    N = W.shape[0]
+    out = np.empty((M, N), np.float64)
+    _L().oracle_transform_f64(_p(x), _p(D), _p(W), M, N, K, _p(out))
+    return out
+
+
+def dequantize(codes, scales) -> np.ndarray:
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.uint8)
+    R, K = codes.shape[0], codes.shape[1] * 2
+    out = np.empty((R, K), np.float64)
+    _L().oracle_dequantize(_p(codes), _p(scales), R, K, _p(out))
+    return out
+
+
+def quantize_plain(v) -> tuple[np.ndarray, np.ndarray]:
+    """Plain MXFP4 of [R, K] fp32 values, no D and no H (the pages' native
+    baseline, npu_dynamic_mx_quant)."""
+    v = _c(v, np.float32)
+    R, K = v.shape
+    codes = np.empty((R, K // 2), np.uint8)
+    scales = np.empty((R, K // 32), np.uint8)
+    st = _L().oracle_quantize_plain(_p(v), R, K, _p(codes), _p(scales))
+    assert st == OK, st
+    return codes, scales
+
+
+def num_threads() -> int:
+    return int(_L().oracle_num_threads())

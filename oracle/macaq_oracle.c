@@ -1,0 +1,635 @@
+/*
+ * MACAQ W4A4 MXFP4 linear -- plain CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or
+ * call this file; only the tests, the smoke check and the benchmark's CPU
+ * baseline do.  It shares no code, header, table or constant with the CUDA
+ * library.
+ *
+ * What it computes follows the page "MACAQ W4A4 fused dense and grouped
+ * matmul for Ascend 950" (gitcode.com/cann/ops-nn/pull/12568), summary
+ * section: channel scaling, a block-32 BF16 Hadamard rotation, MXFP4
+ * activation quantisation (block32 E2M1, round-to-even, scale_alg=0) and a
+ * matrix multiplication with BF16 output; the weight transform (W, D, H) is
+ * offline.  The grouped form follows the torch_npu npu_grouped_matmul page
+ * (function description: y_i = x_i @ weight_i; parameters: group_list,
+ * group_list_type 0 = cumulative sum, 1 = per-group counts).
+ *
+ * Readings taken where the pages are silent (each one is listed, with the
+ * reason, in the design notes of the repository):
+ *   R1  activations are divided by D and weights multiplied by D, so that
+ *       (x/D)H . ((W.D)H)^T / 32 == x.W^T without quantisation;
+ *   R2  H is the unnormalised +-1 Sylvester matrix, H.H^T = 32 I, and the
+ *       1/32 is applied to the FP32 sum as an exact power of two;
+ *   R3  activation arithmetic: r = RN32(1/D); xs = RNE_bf16(RN32(x*r));
+ *       u = RNE_bf16(FWHT32(xs)) with an FP32 butterfly in the fixed order
+ *       h = 1, 2, 4, 8, 16;
+ *   R4  E8M0 scale = floor(log2(amax)) - 2 + 127 clamped to [0, 254]; an
+ *       amax of zero or below the smallest normal gives 0; non-finite gives
+ *       255 (finite input is a precondition);
+ *   R5  E2M1 element = round-to-nearest-even with saturation at +-6 of
+ *       v * 2^(127 - scale); the sign bit copies the sign of v;
+ *   R6  weights take the same steps on t = FWHT32(RN32(W*D)) in FP32 with
+ *       no BF16 rounding (offline preparation);
+ *   R7  y = RNE_bf16(2^-5 * exact sum of the decoded block-scaled products).
+ *
+ * Build:  gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fopenmp -shared -fPIC
+ * (no FMA contraction: every float operation is one IEEE binary32 rounding).
+ */
+#include <stdint.h>
+#include <string.h>
+#include <math.h>
+#include <stdlib.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* status codes returned by the grouped oracle; values match the ones the
+ * library documents for the same conditions, written out independently */
+#define ORACLE_OK 0
+#define ORACLE_ERR_SHAPE (-3)
+#define ORACLE_ERR_TOO_MANY_GROUPS (-6)
+#define ORACLE_ERR_GROUP_LIST_TYPE (-7)
+#define ORACLE_ERR_GROUP_LIST_INVALID (-10)
+
+/* ------------------------------------------------------------------ */
+/* binary16-brain (bf16) <-> binary32                                  */
+/* ------------------------------------------------------------------ */
+
+double oracle_bf16_to_f64(uint16_t h);
+
+static float bf16_bits_to_float(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* Round a binary32 to bf16 by the definition of round-to-nearest-even on
+ * the 16 discarded bits.  NaN stays NaN (quiet). */
+static uint16_t float_to_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7fffffffu) > 0x7f800000u)
+        return (uint16_t)((u >> 16) | 0x0040u);
+    uint32_t keep = u >> 16;
+    uint32_t dropped = u & 0xffffu;
+    if (dropped > 0x8000u || (dropped == 0x8000u && (keep & 1u)))
+        keep += 1u; /* a carry into the exponent is the correct result */
+    return (uint16_t)keep;
+}
+
+uint16_t oracle_f32_to_bf16(float f) { return float_to_bf16_rne(f); }
+double oracle_bf16_to_f64(uint16_t h) { return (double)bf16_bits_to_float(h); }
+
+/* ------------------------------------------------------------------ */
+/* Block-32 Sylvester Hadamard transform, FP32 butterfly (R2, R3)      */
+/* ------------------------------------------------------------------ */
+
+/* In-place unnormalised Walsh-Hadamard transform of 32 floats.  At stage h
+ * every pair (i, i+h) with bit h of i clear becomes (v[i]+v[i+h],
+ * v[i]-v[i+h]), each a single binary32 rounding. */
+static void fwht32_f32(float v[32])
+{
+    for (int h = 1; h < 32; h <<= 1) {
+        for (int i = 0; i < 32; i++) {
+            if (i & h)
+                continue;
+            float a = v[i];
+            float b = v[i + h];
+            v[i] = a + b;
+            v[i + h] = a - b;
+        }
+    }
+}
+
+void oracle_fwht32(const float *in, float *out, int64_t nblocks)
+{
+    for (int64_t b = 0; b < nblocks; b++) {
+        float v[32];
+        memcpy(v, in + 32 * b, sizeof v);
+        fwht32_f32(v);
+        memcpy(out + 32 * b, v, sizeof v);
+    }
+}
+
+/* The same transform in binary64 (used only by the unquantised convention
+ * check, where sums of products must not round). */
+static void fwht32_f64(double v[32])
+{
+    for (int h = 1; h < 32; h <<= 1)
+        for (int i = 0; i < 32; i++) {
+            if (i & h)
+                continue;
+            double a = v[i], b = v[i + h];
+            v[i] = a + b;
+            v[i + h] = a - b;
+        }
+}
+
+/* ------------------------------------------------------------------ */
+/* MX scale (E8M0) and element (E2M1) encodings (R4, R5)               */
+/* ------------------------------------------------------------------ */
+
+/* OCP MX scale_alg=0: shared exponent = floor(log2(amax)) - emax_elem with
+ * emax_elem = 2 for E2M1 (largest magnitude 6 = 1.5 * 2^2). */
+int oracle_e8m0_from_amax(float amax)
+{
+    double a = fabs((double)amax);
+    if (isnan(a) || isinf(a))
+        return 255;
+    if (a == 0.0)
+        return 0;
+    int e;
+    (void)frexp(a, &e);          /* a = f * 2^e with f in [0.5, 1) */
+    int floor_log2 = e - 1;
+    int c = floor_log2 - 2 + 127;
+    if (c < 0)
+        c = 0;
+    if (c > 254)
+        c = 254;
+    return c;
+}
+
+/* Decoded magnitude of the three E2M1 magnitude bits (exponent bias 1,
+ * one mantissa bit, code 1 is the subnormal 0.5). */
+static double e2m1_magnitude(int m)
+{
+    int e = (m >> 1) & 3;
+    int f = m & 1;
+    if (e == 0)
+        return 0.5 * f;
+    return ldexp(1.0 + 0.5 * f, e - 1);
+}
+
+double oracle_e2m1_decode(int code)
+{
+    double m = e2m1_magnitude(code & 7);
+    return (code & 8) ? -m : m;
+}
+
+/* Round-to-nearest-even onto {0, .5, 1, 1.5, 2, 3, 4, 6} with saturation,
+ * written as the interval table that the rule produces.  The tie points
+ * (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5) go to the code whose mantissa bit
+ * is 0. */
+int oracle_e2m1_encode(double v)
+{
+    int s = signbit(v) ? 8 : 0;
+    double a = fabs(v);
+    int m;
+    if (a <= 0.25)
+        m = 0;
+    else if (a < 0.75)
+        m = 1;
+    else if (a <= 1.25)
+        m = 2;
+    else if (a < 1.75)
+        m = 3;
+    else if (a <= 2.5)
+        m = 4;
+    else if (a < 3.5)
+        m = 5;
+    else if (a <= 5.0)
+        m = 6;
+    else
+        m = 7; /* (5, inf): 6, saturating */
+    return s | m;
+}
+
+/* Quantise one block of 32 values given as doubles that are exact copies
+ * of binary32 values: E8M0 from the block amax, then E2M1 of each value
+ * scaled by 2^(127 - c) (exact in binary64). codes: 16 bytes, element 2j in
+ * the low nibble of byte j. */
+static void mx_quantize_block(const double v[32], uint8_t codes[16], uint8_t *scale)
+{
+    float amax = 0.0f;
+    for (int i = 0; i < 32; i++) {
+        float a = (float)fabs(v[i]);
+        if (a > amax || isnan(a))
+            amax = a;
+    }
+    int c = oracle_e8m0_from_amax(amax);
+    *scale = (uint8_t)c;
+    for (int j = 0; j < 16; j++) {
+        int lo = oracle_e2m1_encode(ldexp(v[2 * j], 127 - c));
+        int hi = oracle_e2m1_encode(ldexp(v[2 * j + 1], 127 - c));
+        codes[j] = (uint8_t)(lo | (hi << 4));
+    }
+}
+
+void oracle_mx_quantize_blocks(const float *v, int64_t nblocks, uint8_t *codes, uint8_t *scales)
+{
+    for (int64_t b = 0; b < nblocks; b++) {
+        double d[32];
+        for (int i = 0; i < 32; i++)
+            d[i] = (double)v[32 * b + i];
+        mx_quantize_block(d, codes + 16 * b, scales + b);
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Activation path (R1, R3): x bf16 [M,K], D fp32 [K]                  */
+/* ------------------------------------------------------------------ */
+
+/* Rotated BF16 activations u for one row: writes K bf16 bit patterns. */
+static void act_rotate_row(const uint16_t *xrow, const float *D, int64_t K, uint16_t *urow)
+{
+    for (int64_t b = 0; b < K / 32; b++) {
+        float v[32];
+        for (int i = 0; i < 32; i++) {
+            int64_t k = 32 * b + i;
+            float r = 1.0f / D[k];                            /* RN32(1/D) */
+            float prod = bf16_bits_to_float(xrow[k]) * r;     /* RN32(x*r) */
+            v[i] = bf16_bits_to_float(float_to_bf16_rne(prod));
+        }
+        fwht32_f32(v);
+        for (int i = 0; i < 32; i++)
+            urow[32 * b + i] = float_to_bf16_rne(v[i]);
+    }
+}
+
+void oracle_act_rotate(const uint16_t *x, const float *D, int64_t M, int64_t K, uint16_t *u)
+{
+    for (int64_t m = 0; m < M; m++)
+        act_rotate_row(x + m * K, D, K, u + m * K);
+}
+
+/* codes: [M, K/2] (element 2j low nibble), scales: [M, K/32] */
+int oracle_quantize_act(const uint16_t *x, const float *D, int64_t M, int64_t K,
+                        uint8_t *codes, uint8_t *scales, int nthreads)
+{
+    if (K <= 0 || K % 32 != 0 || M < 0)
+        return ORACLE_ERR_SHAPE;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t m = 0; m < M; m++) {
+        uint16_t *u = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)K);
+        act_rotate_row(x + m * K, D, K, u);
+        for (int64_t b = 0; b < K / 32; b++) {
+            double d[32];
+            for (int i = 0; i < 32; i++)
+                d[i] = (double)bf16_bits_to_float(u[32 * b + i]);
+            mx_quantize_block(d, codes + m * (K / 2) + 16 * b, scales + m * (K / 32) + b);
+        }
+        free(u);
+    }
+    (void)nthreads;
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Weight path (R1, R6): W fp32 [N,K], D fp32 [K]                      */
+/* ------------------------------------------------------------------ */
+
+int oracle_quantize_weights(const float *W, const float *D, int64_t N, int64_t K,
+                            uint8_t *codes, uint8_t *scales, int nthreads)
+{
+    if (K <= 0 || K % 32 != 0 || N < 0)
+        return ORACLE_ERR_SHAPE;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t n = 0; n < N; n++) {
+        for (int64_t b = 0; b < K / 32; b++) {
+            float t[32];
+            for (int i = 0; i < 32; i++) {
+                int64_t k = 32 * b + i;
+                t[i] = W[n * K + k] * D[k]; /* RN32(W*D) */
+            }
+            fwht32_f32(t);
+            double d[32];
+            for (int i = 0; i < 32; i++)
+                d[i] = (double)t[i];
+            mx_quantize_block(d, codes + n * (K / 2) + 16 * b, scales + n * (K / 32) + b);
+        }
+    }
+    (void)nthreads;
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Exact block-scaled dot product and BF16 rounding (R7)               */
+/* ------------------------------------------------------------------ */
+
+/* A signed fixed-point accumulator wide enough for any sum that can occur:
+ * every term is an integer times 2^E with E in [-256, 252]; the accumulator
+ * holds the sum in units of 2^-256 as a two's complement integer of
+ * NLIMB*64 bits. */
+#define NLIMB 10
+typedef struct {
+    uint64_t w[NLIMB];
+} wide_t;
+
+static void wide_add_shifted(wide_t *acc, int64_t p, int shift)
+{
+    /* add p * 2^shift, p a signed 64-bit integer, 0 <= shift < 576 */
+    if (p == 0)
+        return;
+    uint64_t ext = p < 0 ? ~(uint64_t)0 : 0;
+    uint64_t lo = (uint64_t)p;
+    int limb = shift / 64, bit = shift % 64;
+    uint64_t parts[NLIMB];
+    for (int i = 0; i < NLIMB; i++)
+        parts[i] = ext;
+    for (int i = 0; i < limb; i++)
+        parts[i] = 0;
+    if (bit == 0) {
+        parts[limb] = lo;
+    } else {
+        parts[limb] = lo << bit;
+        if (limb + 1 < NLIMB)
+            parts[limb + 1] = (lo >> (64 - bit)) | (ext << bit);
+    }
+    unsigned carry = 0;
+    for (int i = 0; i < NLIMB; i++) {
+        uint64_t s = acc->w[i] + parts[i];
+        unsigned c1 = s < acc->w[i];
+        uint64_t s2 = s + carry;
+        unsigned c2 = s2 < s;
+        acc->w[i] = s2;
+        carry = c1 | c2;
+    }
+}
+
+static int wide_bit(const wide_t *a, int i)
+{
+    if (i < 0 || i >= NLIMB * 64)
+        return 0;
+    return (int)((a->w[i / 64] >> (i % 64)) & 1);
+}
+
+/* 1 if any bit strictly below position i is set */
+static int wide_any_below(const wide_t *a, int i)
+{
+    if (i <= 0)
+        return 0;
+    for (int l = 0; l < NLIMB; l++) {
+        int lo = l * 64;
+        if (lo >= i)
+            break;
+        int nb = i - lo >= 64 ? 64 : i - lo;
+        uint64_t mask = nb == 64 ? ~(uint64_t)0 : ((((uint64_t)1) << nb) - 1);
+        if (a->w[l] & mask)
+            return 1;
+    }
+    return 0;
+}
+
+/* Round the accumulator value acc * 2^base_exp to bf16: round-to-nearest,
+ * ties to even, subnormals below 2^-126 with last bit 2^-133, overflow to
+ * infinity.  An exact zero gives +0. */
+static uint16_t wide_to_bf16(const wide_t *acc, int base_exp)
+{
+    wide_t a = *acc;
+    int neg = (int)((a.w[NLIMB - 1] >> 63) & 1);
+    if (neg) { /* two's complement negation */
+        unsigned carry = 1;
+        for (int i = 0; i < NLIMB; i++) {
+            uint64_t v = ~a.w[i];
+            uint64_t s = v + carry;
+            carry = carry && s == 0;
+            a.w[i] = s;
+        }
+    }
+    int top = -1;
+    for (int i = NLIMB - 1; i >= 0 && top < 0; i--)
+        if (a.w[i])
+            top = i * 64 + 63 - __builtin_clzll(a.w[i]);
+    if (top < 0)
+        return 0;
+    int E = top + base_exp;                  /* |value| in [2^E, 2^(E+1)) */
+    int lsb_exp = E >= -126 ? E - 7 : -133;  /* weight of the last kept bit */
+    int L = lsb_exp - base_exp;              /* its bit index in a */
+    uint32_t q = 0;
+    for (int i = top; i >= L; i--)           /* at most 8 kept bits */
+        q = (q << 1) | (uint32_t)wide_bit(&a, i);
+    if (L > 0) {
+        int round = wide_bit(&a, L - 1);
+        int sticky = wide_any_below(&a, L - 1);
+        if (round && (sticky || (q & 1)))
+            q += 1;
+    }
+    uint32_t bits;
+    if (lsb_exp == -133)
+        bits = q;                            /* subnormal (0x80 = min normal) */
+    else
+        bits = ((uint32_t)(E + 127) << 7) + (q - 128); /* q in [128, 256] */
+    if (bits >= 0x7f80u)
+        bits = 0x7f80u;
+    return (uint16_t)((neg ? 0x8000u : 0u) | bits);
+}
+
+/* y = RNE_bf16(2^-5 * sum_k dec(qa[k]) 2^(sa[k/32]-127) dec(qw[k]) 2^(sw[k/32]-127)),
+ * the sum taken exactly.  Each E2M1 value is an integer multiple of 1/2, so
+ * each block of 32 contributes (sum of integer products) * 2^(sa+sw-256). */
+static uint16_t exact_dot(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw,
+                          const uint8_t *sw, int64_t K)
+{
+    wide_t acc;
+    memset(&acc, 0, sizeof acc);
+    for (int64_t b = 0; b < K / 32; b++) {
+        int64_t p = 0;
+        for (int i = 0; i < 32; i++) {
+            int64_t k = 32 * b + i;
+            int ca = (qa[k / 2] >> (4 * (k & 1))) & 15;
+            int cw = (qw[k / 2] >> (4 * (k & 1))) & 15;
+            int64_t ia = (int64_t)llround(2.0 * oracle_e2m1_decode(ca));
+            int64_t iw = (int64_t)llround(2.0 * oracle_e2m1_decode(cw));
+            p += ia * iw;
+        }
+        int E = (int)sa[b] + (int)sw[b] - 256;
+        wide_add_shifted(&acc, p, E + 256);
+    }
+    return wide_to_bf16(&acc, -256 - 5);
+}
+
+/* Full exact GEMM: qa [M, K/2], sa [M, K/32], qw [N, K/2], sw [N, K/32]
+ * -> y bf16 bits [M, N]. */
+int oracle_gemm(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const uint8_t *sw,
+                int64_t M, int64_t N, int64_t K, uint16_t *y, int nthreads)
+{
+    if (K <= 0 || K % 32 != 0)
+        return ORACLE_ERR_SHAPE;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel for schedule(static)
+#endif
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t n = 0; n < N; n++)
+            y[m * N + n] = exact_dot(qa + m * (K / 2), sa + m * (K / 32), qw + n * (K / 2),
+                                     sw + n * (K / 32), K);
+    (void)nthreads;
+    return ORACLE_OK;
+}
+
+/* Exact outputs at chosen (row, col) positions only. */
+int oracle_gemm_at(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const uint8_t *sw,
+                   int64_t K, const int64_t *rows, const int64_t *cols, int64_t count, uint16_t *out)
+{
+    if (K <= 0 || K % 32 != 0)
+        return ORACLE_ERR_SHAPE;
+    for (int64_t i = 0; i < count; i++)
+        out[i] = exact_dot(qa + rows[i] * (K / 2), sa + rows[i] * (K / 32), qw + cols[i] * (K / 2),
+                           sw + cols[i] * (K / 32), K);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Grouped form: rows [cum[g-1], cum[g]) use expert g                  */
+/* ------------------------------------------------------------------ */
+
+/* Validates group_list as the npu_grouped_matmul page states it (type 0:
+ * non-negative, non-decreasing cumulative sums; type 1: non-negative
+ * counts) and, for a single output tensor, that it covers all M rows.
+ * Writes the E+1 row offsets to off. */
+int oracle_group_offsets(const int64_t *group_list, int type, int64_t E, int64_t M, int64_t *off)
+{
+    if (E < 1 || E > 1024)
+        return ORACLE_ERR_TOO_MANY_GROUPS;
+    if (type != 0 && type != 1)
+        return ORACLE_ERR_GROUP_LIST_TYPE;
+    off[0] = 0;
+    for (int64_t g = 0; g < E; g++) {
+        int64_t v = group_list[g];
+        if (v < 0)
+            return ORACLE_ERR_GROUP_LIST_INVALID;
+        if (type == 0) {
+            if (v < off[g])
+                return ORACLE_ERR_GROUP_LIST_INVALID;
+            off[g + 1] = v;
+        } else {
+            off[g + 1] = off[g] + v;
+            if (off[g + 1] > M)
+                return ORACLE_ERR_GROUP_LIST_INVALID;
+        }
+    }
+    if (off[E] != M)
+        return ORACLE_ERR_GROUP_LIST_INVALID;
+    return ORACLE_OK;
+}
+
+/* Grouped MACAQ linear. x bf16 [M,K]; D [E,K]; W fp32 [E,N,K]. y [M,N]. */
+int oracle_grouped_mm(const uint16_t *x, const float *D, const float *W, const int64_t *group_list,
+                      int type, int64_t E, int64_t M, int64_t N, int64_t K, uint16_t *y,
+                      int nthreads)
+{
+    if (K <= 0 || K % 32 != 0 || N <= 0 || M < 0)
+        return ORACLE_ERR_SHAPE;
+    int64_t *off = (int64_t *)malloc(sizeof(int64_t) * (size_t)(E + 1 > 1 ? E + 1 : 2));
+    int st = oracle_group_offsets(group_list, type, E, M, off);
+    if (st != ORACLE_OK) {
+        free(off);
+        return st;
+    }
+    uint8_t *qw = (uint8_t *)malloc((size_t)(N * K / 2));
+    uint8_t *sw = (uint8_t *)malloc((size_t)(N * K / 32));
+    for (int64_t g = 0; g < E; g++) {
+        int64_t r0 = off[g], r1 = off[g + 1];
+        if (r1 == r0)
+            continue;
+        oracle_quantize_weights(W + g * N * K, D + g * K, N, K, qw, sw, nthreads);
+        uint8_t *qa = (uint8_t *)malloc((size_t)((r1 - r0) * K / 2));
+        uint8_t *sa = (uint8_t *)malloc((size_t)((r1 - r0) * K / 32));
+        oracle_quantize_act(x + r0 * K, D + g * K, r1 - r0, K, qa, sa, nthreads);
+        oracle_gemm(qa, sa, qw, sw, r1 - r0, N, K, y + r0 * N, nthreads);
+        free(qa);
+        free(sa);
+    }
+    free(qw);
+    free(sw);
+    free(off);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Diagnostics in binary64                                              */
+/* ------------------------------------------------------------------ */
+
+/* Plain x . W^T in binary64. */
+void oracle_linear_f64(const uint16_t *x, const float *W, int64_t M, int64_t N, int64_t K, double *out)
+{
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t n = 0; n < N; n++) {
+            double s = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                s += (double)bf16_bits_to_float(x[m * K + k]) * (double)W[n * K + k];
+            out[m * N + n] = s;
+        }
+}
+
+/* The MACAQ transform with every rounding and all quantisation removed:
+ * ((x/D) H) . ((W.D) H)^T / 32 in binary64.  Equal to x . W^T (up to
+ * binary64 rounding) exactly when readings R1 and R2 hold. */
+void oracle_transform_f64(const uint16_t *x, const float *D, const float *W, int64_t M, int64_t N,
+                          int64_t K, double *out)
+{
+    double *xa = (double *)malloc(sizeof(double) * (size_t)(M * K));
+    double *wa = (double *)malloc(sizeof(double) * (size_t)(N * K));
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t b = 0; b < K / 32; b++) {
+            double v[32];
+            for (int i = 0; i < 32; i++) {
+                int64_t k = 32 * b + i;
+                v[i] = (double)bf16_bits_to_float(x[m * K + k]) / (double)D[k];
+            }
+            fwht32_f64(v);
+            memcpy(xa + m * K + 32 * b, v, sizeof v);
+        }
+    for (int64_t n = 0; n < N; n++)
+        for (int64_t b = 0; b < K / 32; b++) {
+            double v[32];
+            for (int i = 0; i < 32; i++) {
+                int64_t k = 32 * b + i;
+                v[i] = (double)W[n * K + k] * (double)D[k];
+            }
+            fwht32_f64(v);
+            memcpy(wa + n * K + 32 * b, v, sizeof v);
+        }
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t n = 0; n < N; n++) {
+            double s = 0.0;
+            for (int64_t k = 0; k < K; k++)
+                s += xa[m * K + k] * wa[n * K + k];
+            out[m * N + n] = s / 32.0;
+        }
+    free(xa);
+    free(wa);
+}
+
+/* Decode codes and scales to binary64 values (for error reports). */
+void oracle_dequantize(const uint8_t *codes, const uint8_t *scales, int64_t R, int64_t K, double *out)
+{
+    for (int64_t r = 0; r < R; r++)
+        for (int64_t k = 0; k < K; k++) {
+            int c = (codes[r * (K / 2) + k / 2] >> (4 * (k & 1))) & 15;
+            int s = scales[r * (K / 32) + k / 32];
+            out[r * K + k] = ldexp(oracle_e2m1_decode(c), s - 127);
+        }
+}
+
+/* Plain MXFP4 W4A4 without D and H (the pages' native baseline): quantise
+ * x (bf16) and W (fp32) directly in blocks of 32 along K. */
+int oracle_quantize_plain(const float *v, int64_t R, int64_t K, uint8_t *codes, uint8_t *scales)
+{
+    if (K <= 0 || K % 32 != 0)
+        return ORACLE_ERR_SHAPE;
+    oracle_mx_quantize_blocks(v, R * K / 32, codes, scales);
+    return ORACLE_OK;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,456 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+None of these compares the oracle with itself: each check uses an independent
+route (a library routine, a closed form, brute force, exact rational
+arithmetic, or a hand derivation stored under tests/golden/).
+"""
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.linalg
+import torch
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def sylvester_by_popcount(n=32):
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    pc = np.vectorize(lambda v: bin(int(v)).count("1"))(i & j)
+    return np.where(pc % 2 == 0, 1.0, -1.0)
+
+
+# ----------------------------------------------------------------------------
+# Hadamard
+# ----------------------------------------------------------------------------
+
+def test_fwht_of_unit_vectors_gives_sylvester_columns():
+    eye = np.eye(32, dtype=np.float32)
+    cols = np.stack([oracle.fwht32(eye[j]) for j in range(32)], axis=1)
+    assert np.array_equal(cols, sylvester_by_popcount())
+    assert np.array_equal(cols, scipy.linalg.hadamard(32).astype(np.float32))
+
+
+def test_hadamard_is_orthogonal_times_32():
+    eye = np.eye(32, dtype=np.float32)
+    H = np.stack([oracle.fwht32(eye[j]) for j in range(32)], axis=1).astype(np.float64)
+    assert np.array_equal(H @ H.T, 32.0 * np.eye(32))
+
+
+def test_fwht_matches_library_matmul_when_sums_are_exact():
+    rng = np.random.default_rng(1)
+    v = rng.integers(-1000, 1000, size=(64, 32)).astype(np.float32)
+    got = oracle.fwht32(v.ravel()).reshape(64, 32)
+    want = v.astype(np.float64) @ scipy.linalg.hadamard(32).T.astype(np.float64)
+    assert np.array_equal(got.astype(np.float64), want)
+
+
+def test_fwht_all_equal_block():
+    for val in [1.0, -3.5, 0.15625, 1e-20, 6e30]:
+        got = oracle.fwht32(np.full(32, val, np.float32))
+        assert got[0] == np.float32(32 * np.float64(np.float32(val)))
+        assert np.all(got[1:] == 0)
+
+
+def test_fwht_twice_is_32_times_identity_on_exact_values():
+    rng = np.random.default_rng(2)
+    v = rng.integers(-64, 64, size=32).astype(np.float32)
+    assert np.array_equal(oracle.fwht32(oracle.fwht32(v)), 32 * v)
+
+
+def test_fwht_fp32_rounding_matches_stagewise_numpy_float32():
+    # each butterfly output is one binary32 rounding: numpy float32 adds in
+    # the same pairing order reproduce it; a different order generally not.
+    rng = np.random.default_rng(3)
+    v = (rng.standard_normal(32) * np.exp2(rng.integers(-20, 20, 32))).astype(np.float32)
+    w = v.copy()
+    h = 1
+    while h < 32:
+        out = w.copy()
+        for i in range(32):
+            if i & h:
+                continue
+            out[i] = np.float32(w[i] + w[i + h])
+            out[i + h] = np.float32(w[i] - w[i + h])
+        w = out
+        h <<= 1
+    assert np.array_equal(oracle.fwht32(v), w)
+
+
+# ----------------------------------------------------------------------------
+# BF16 rounding
+# ----------------------------------------------------------------------------
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(4)
+    bits = rng.integers(0, 2**32, size=20000, dtype=np.uint64).astype(np.uint32)
+    # force many exact ties and near-ties
+    bits[:4000] = (bits[:4000] & 0xFFFF0000) | 0x8000
+    bits[4000:6000] = (bits[4000:6000] & 0xFFFF0000) | 0x7FFF
+    f = bits.view(np.float32)
+    f = f[np.isfinite(f)]
+    got = oracle.f32_to_bf16(f)
+    want = torch.from_numpy(f.copy()).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, want)
+
+
+# ----------------------------------------------------------------------------
+# E2M1 and E8M0
+# ----------------------------------------------------------------------------
+
+def test_e2m1_table_matches_golden():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "e2m1_values.txt"))
+            if l.strip() and not l.startswith("#")]
+    for code, val in rows:
+        got = oracle.e2m1_decode(int(code))
+        assert got == float(val) and math.copysign(1, got) == math.copysign(1, float(val))
+
+
+def brute_force_e2m1(a: float) -> int:
+    """Nearest of the 8 magnitudes, ties to the even code, saturating."""
+    s = 8 if math.copysign(1.0, a) < 0 else 0
+    m = abs(a)
+    if m >= 6.0:  # saturation; below 6 the float64 distances are exact
+        return s | 7
+    d = np.abs(E2M1_GRID - m)
+    best = np.flatnonzero(d == d.min())
+    if best.size > 1:
+        best = best[best % 2 == 0]
+    return s | int(best[0])
+
+
+def test_e2m1_encode_exhaustive_over_bf16():
+    bits = np.arange(65536, dtype=np.uint32)
+    f32 = (bits << 16).view(np.float32)
+    ok = np.isfinite(f32)
+    vals = f32[ok].astype(np.float64)
+    ok = np.ones(vals.size, bool)
+    for v in vals[ok]:
+        assert oracle.e2m1_encode(v) == brute_force_e2m1(v), v
+
+
+def test_e2m1_tie_points():
+    for t, want in [(0.25, 0), (0.75, 2), (1.25, 2), (1.75, 4), (2.5, 4), (3.5, 6), (5.0, 6),
+                    (6.0, 7), (7.99, 7), (-0.25, 8), (-0.1, 8), (-5.0, 14)]:
+        assert oracle.e2m1_encode(t) == want, t
+
+
+def test_e8m0_defining_property():
+    # For every positive finite binary32 exponent and a few mantissas, the
+    # scale X = 2^(c-127) puts amax/X in [4, 8) unless clamped at c = 0.
+    for e in range(-149, 128):
+        for mant in [1.0, 1.3, 1.5, 1.999999]:
+            a = np.float32(mant * 2.0 ** e)
+            if not np.isfinite(a) or a == 0:
+                continue
+            c = oracle.e8m0_from_amax(a)
+            r = Fraction(float(a)) / Fraction(2) ** (c - 127)
+            assert r < 8
+            if c > 0:
+                assert r >= 4
+            else:
+                assert Fraction(float(a)) < Fraction(2) ** (-127 + 3)
+    assert oracle.e8m0_from_amax(0.0) == 0
+    assert oracle.e8m0_from_amax(float("inf")) == 255
+    assert oracle.e8m0_from_amax(float("nan")) == 255
+
+
+def test_round_trip_every_code_every_scale():
+    # A block holding every code once (and 6 to fix the scale) quantises back
+    # to itself for every scale code whose values are representable.
+    codes = np.array(list(range(16)) + [7] * 16)
+    for c in range(0, 253):
+        vals = np.array([np.ldexp(oracle.e2m1_decode(int(k)), c - 127) for k in codes])
+        f = vals.astype(np.float32)
+        assert np.array_equal(f.astype(np.float64), vals)
+        q, s = oracle.mx_quantize_blocks(f)
+        assert s[0] == c
+        got = oracle.unpack_codes(q)
+        assert np.array_equal(got, codes), c
+
+
+def test_idempotent_on_representable_random_blocks():
+    rng = np.random.default_rng(5)
+    for _ in range(300):
+        c = int(rng.integers(1, 250))
+        codes = rng.integers(0, 16, size=32)
+        codes[rng.integers(0, 32)] = 7  # amax code fixes the scale
+        vals = np.array([np.ldexp(oracle.e2m1_decode(int(k)), c - 127) for k in codes], np.float32)
+        q, s = oracle.mx_quantize_blocks(vals)
+        deq = oracle.dequantize(q.reshape(1, 16), s.reshape(1, 1))[0]
+        assert np.array_equal(deq, vals.astype(np.float64))
+
+
+def test_zero_and_negative_zero_blocks():
+    q, s = oracle.mx_quantize_blocks(np.zeros(32, np.float32))
+    assert s[0] == 0 and np.all(q == 0)
+    q, s = oracle.mx_quantize_blocks(-np.zeros(32, np.float32))
+    assert s[0] == 0 and np.all(q == 0x88)
+
+
+def test_random_blocks_against_brute_force():
+    rng = np.random.default_rng(6)
+    for _ in range(200):
+        v = (rng.standard_normal(32) * np.exp2(rng.integers(-30, 30))).astype(np.float32)
+        q, s = oracle.mx_quantize_blocks(v)
+        c = int(s[0])
+        amax = float(np.max(np.abs(v)))
+        r = Fraction(amax) / Fraction(2) ** (c - 127)
+        assert 4 <= r < 8
+        want = [brute_force_e2m1(float(np.ldexp(np.float64(x), 127 - c))) for x in v]
+        assert np.array_equal(oracle.unpack_codes(q), np.array(want))
+
+
+# ----------------------------------------------------------------------------
+# Activation and weight paths
+# ----------------------------------------------------------------------------
+
+def _pattern(name):
+    if name == "ones":
+        return np.ones(32, np.float32)
+    if name == "alt":
+        return np.array([(-1.0) ** i for i in range(32)], np.float32)
+    if name == "neg":
+        return -np.ones(32, np.float32)
+    if name == "zero":
+        return np.zeros(32, np.float32)
+    if name == "spike3":
+        v = np.zeros(32, np.float32)
+        v[0] = 3.0
+        return v
+    raise ValueError(name)
+
+
+def test_hand_derived_blocks():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "hand_blocks.txt"))
+            if l.strip() and not l.startswith("#")]
+    assert len(rows) == 6
+    for name, d, pat, scale, b0, brest in rows:
+        x = synth.to_bf16_bits(_pattern(pat)[None, :])
+        D = np.full(32, float(d), np.float32)
+        q, s = oracle.quantize_act(x, D)
+        assert int(s[0, 0]) == int(scale), name
+        assert int(q[0, 0]) == int(b0, 16), name
+        assert np.all(q[0, 1:] == int(brest, 16)), name
+
+
+def test_activation_steps_follow_definition():
+    # the rotated activations, re-derived with numpy float32 and torch bf16
+    rng = np.random.default_rng(7)
+    M, K = 3, 96
+    x = synth.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32) * 4)
+    D = (np.exp(rng.standard_normal(K)) * np.sign(rng.standard_normal(K))).astype(np.float32)
+    r = (np.float32(1.0) / D).astype(np.float32)
+    xs = synth.bf16_bits_to_f32(synth.to_bf16_bits(synth.bf16_bits_to_f32(x) * r))
+    H = scipy.linalg.hadamard(32).astype(np.float64)
+    u = oracle.act_rotate(x, D)
+    uf = synth.bf16_bits_to_f32(u).astype(np.float64)
+    ref = (xs.reshape(M, K // 32, 32).astype(np.float64) @ H.T).reshape(M, K)
+    # BF16 output of an FP32 butterfly: within one bf16 ulp of the exact rotation
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 7)
+    assert np.all(np.abs(uf - ref) <= ulp + 1e-30)
+
+
+def test_unquantised_transform_preserves_the_layer():
+    # pins R1 (x/D with W*D) and R2 (H H^T = 32 I, 1/32 afterwards)
+    rng = np.random.default_rng(8)
+    M, N, K = 5, 7, 128
+    x = synth.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    W = rng.standard_normal((N, K)).astype(np.float32)
+    D = (np.exp(rng.standard_normal(K)) * np.where(rng.random(K) < 0.3, -1, 1)).astype(np.float32)
+    got = oracle.transform_f64(x, D, W)
+    want = oracle.linear_f64(x, W)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+
+
+def test_weight_path_definition():
+    rng = np.random.default_rng(9)
+    N, K = 4, 64
+    W = rng.standard_normal((N, K)).astype(np.float32)
+    D = np.exp(rng.standard_normal(K)).astype(np.float32)
+    q, s = oracle.quantize_weights(W, D)
+    t = (W * D).astype(np.float32)
+    tt = np.stack([oracle.fwht32(row) for row in t])
+    q2, s2 = oracle.mx_quantize_blocks(tt)
+    assert np.array_equal(q.ravel(), q2) and np.array_equal(s.ravel(), s2)
+    # no bf16 rounding on the weight side: compare with an exact rotation
+    tb = t.reshape(N, K // 32, 32).astype(np.float64)
+    ref = (tb @ scipy.linalg.hadamard(32).T).reshape(N, K)
+    # five binary32 roundings per output: |err| <= 5 * 2^-24 * sum |t| of the block
+    bound = np.repeat(5 * 2.0 ** -24 * np.abs(tb).sum(axis=2), 32, axis=1)
+    assert np.all(np.abs(tt - ref) <= bound)
+
+
+# ----------------------------------------------------------------------------
+# Exact block-scaled GEMM
+# ----------------------------------------------------------------------------
+
+def fraction_to_bf16_bits(v: Fraction) -> int:
+    """Correct RNE rounding of an exact rational to bf16 (independent code)."""
+    if v == 0:
+        return 0
+    sign = 0x8000 if v < 0 else 0
+    a = abs(v)
+    e = math.floor(math.log2(a.numerator) - math.log2(a.denominator))
+    while Fraction(2) ** e > a:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= a:
+        e += 1
+    lsb = e - 7 if e >= -126 else -133
+    q = a / Fraction(2) ** lsb
+    fl = math.floor(q)
+    rem = q - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    if lsb == -133:
+        bits = fl
+    else:
+        bits = ((e + 127) << 7) + (fl - 128)
+    bits = min(bits, 0x7F80)
+    return sign | bits
+
+
+def exact_y(qa, sa, qw, sw):
+    M, K = qa.shape[0], qa.shape[1] * 2
+    N = qw.shape[0]
+    ca, cw = oracle.unpack_codes(qa), oracle.unpack_codes(qw)
+    out = np.zeros((M, N), np.uint16)
+    for m in range(M):
+        for n in range(N):
+            s = Fraction(0)
+            for k in range(K):
+                s += (Fraction(oracle.e2m1_decode(int(ca[m, k])))
+                      * Fraction(2) ** (int(sa[m, k // 32]) - 127)
+                      * Fraction(oracle.e2m1_decode(int(cw[n, k])))
+                      * Fraction(2) ** (int(sw[n, k // 32]) - 127))
+            out[m, n] = fraction_to_bf16_bits(s / 32)
+    return out
+
+
+@pytest.mark.parametrize("spread", ["narrow", "wide", "extreme"])
+def test_exact_gemm_against_rationals(spread):
+    rng = np.random.default_rng({"narrow": 10, "wide": 11, "extreme": 12}[spread])
+    M, N, K = 3, 4, 96
+    qa = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    qw = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    if spread == "narrow":
+        sa = rng.integers(120, 135, size=(M, K // 32), dtype=np.uint8)
+        sw = rng.integers(115, 125, size=(N, K // 32), dtype=np.uint8)
+    elif spread == "wide":
+        sa = rng.integers(60, 200, size=(M, K // 32), dtype=np.uint8)
+        sw = rng.integers(60, 200, size=(N, K // 32), dtype=np.uint8)
+    else:
+        sa = rng.choice(np.array([0, 1, 254, 127, 2], np.uint8), size=(M, K // 32))
+        sw = rng.choice(np.array([0, 254, 130, 3], np.uint8), size=(N, K // 32))
+    got = oracle.gemm(qa, sa, qw, sw)
+    assert np.array_equal(got, exact_y(qa, sa, qw, sw))
+    rows, cols = np.meshgrid(np.arange(M), np.arange(N), indexing="ij")
+    at = oracle.gemm_at(qa, sa, qw, sw, rows.ravel(), cols.ravel())
+    assert np.array_equal(at, got.ravel())
+
+
+def _pack(codes):
+    codes = np.asarray(codes, np.uint8)
+    return (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+
+
+def test_exact_gemm_cancellation_and_ties():
+    # +1 and -1 against +1, +1: the sum cancels to exactly +0
+    ca = np.zeros((1, 32), int); cw = np.zeros((1, 32), int)
+    ca[0, :2] = [0x2, 0xA]; cw[0, :2] = [0x2, 0x2]
+    s127 = np.full((1, 1), 127, np.uint8)
+    assert oracle.gemm(_pack(ca), s127, _pack(cw), s127)[0, 0] == 0
+    # 8 * (4 * 1) + 0.5 * 0.5 * 2^-1 = 32 + 1/8; / 32 = 1 + 2^-8: a tie between
+    # bf16 1.0 and 1 + 2^-7 -> even -> 1.0; one more tiny term breaks the tie upward
+    ca = np.zeros((1, 64), int); cw = np.zeros((1, 64), int)
+    ca[0, :8] = 6; cw[0, :8] = 2
+    ca[0, 32] = 1; cw[0, 32] = 1
+    sa = np.array([[127, 126]], np.uint8); sw = np.array([[127, 127]], np.uint8)
+    assert oracle.gemm(_pack(ca), sa, _pack(cw), sw)[0, 0] == 0x3F80
+    ca[0, 33] = 1; cw[0, 33] = 1
+    sa2 = np.array([[127, 100]], np.uint8)
+    ca2 = ca.copy(); ca2[0, 32] = 0; ca2[0, 33] = 0
+    # exact tie again but via block 1 at a much smaller scale plus the tie term
+    ca3 = np.zeros((1, 96), int); cw3 = np.zeros((1, 96), int)
+    ca3[0, :8] = 6; cw3[0, :8] = 2
+    ca3[0, 32] = 1; cw3[0, 32] = 1
+    ca3[0, 64] = 1; cw3[0, 64] = 1
+    sa3 = np.array([[127, 126, 60]], np.uint8); sw3 = np.array([[127, 127, 127]], np.uint8)
+    assert oracle.gemm(_pack(ca3), sa3, _pack(cw3), sw3)[0, 0] == 0x3F81
+    ca3[0, 64] = 9  # the tiny term negative: just below the tie -> 1.0
+    assert oracle.gemm(_pack(ca3), sa3, _pack(cw3), sw3)[0, 0] == 0x3F80
+
+
+# ----------------------------------------------------------------------------
+# Grouped form
+# ----------------------------------------------------------------------------
+
+def test_group_list_validation_rules():
+    M = 10
+    assert oracle.group_offsets([3, 7, 10], 0, M)[0] == oracle.OK
+    assert oracle.group_offsets([3, 4, 3], 1, M)[0] == oracle.OK
+    assert oracle.group_offsets([3, 2, 10], 0, M)[0] == oracle.ERR_GROUP_LIST_INVALID  # decreasing
+    assert oracle.group_offsets([-1, 2, 10], 0, M)[0] == oracle.ERR_GROUP_LIST_INVALID
+    assert oracle.group_offsets([3, -1, 8], 1, M)[0] == oracle.ERR_GROUP_LIST_INVALID
+    assert oracle.group_offsets([3, 7, 9], 0, M)[0] == oracle.ERR_GROUP_LIST_INVALID  # != M
+    assert oracle.group_offsets([3, 4, 4], 1, M)[0] == oracle.ERR_GROUP_LIST_INVALID
+    assert oracle.group_offsets([3, 7, 10], 2, M)[0] == oracle.ERR_GROUP_LIST_TYPE
+    assert oracle.group_offsets(np.zeros(1025, np.int64), 1, 0)[0] == oracle.ERR_TOO_MANY_GROUPS
+    st, off = oracle.group_offsets([0, 0, 4, 4, 10], 0, M)
+    assert st == oracle.OK and list(off) == [0, 0, 0, 4, 4, 10]
+
+
+def test_grouped_cumsum_equals_counts_and_replicated_banks_equal_dense():
+    p = synth.grouped(96, 4, 64, 48, seed=3, dist="uniform", group_list_type=1)
+    st1, y1 = oracle.grouped_mm(p.x, p.D, p.W, p.group_list, 1)
+    st0, y0 = oracle.grouped_mm(p.x, p.D, p.W, np.cumsum(p.group_list), 0)
+    assert st0 == st1 == oracle.OK and np.array_equal(y0, y1)
+    # replicated banks: every expert has expert 0's W and D
+    Wr = np.repeat(p.W[:1], 4, axis=0)
+    Dr = np.repeat(p.D[:1], 4, axis=0)
+    st, yr = oracle.grouped_mm(p.x, Dr, Wr, p.group_list, 1)
+    assert st == oracle.OK
+    assert np.array_equal(yr, oracle.dense_mm(p.x, p.D[0], p.W[0]))
+
+
+def test_grouped_rows_use_their_own_expert():
+    p = synth.grouped(64, 3, 64, 32, seed=4, dist="uniform", group_list_type=1)
+    st, y = oracle.grouped_mm(p.x, p.D, p.W, p.group_list, 1)
+    assert st == oracle.OK
+    off = np.concatenate([[0], np.cumsum(p.counts)])
+    for g in range(3):
+        rows = slice(off[g], off[g + 1])
+        assert np.array_equal(y[rows], oracle.dense_mm(p.x[rows], p.D[g], p.W[g]))
+
+
+def test_grouped_empty_groups():
+    p = synth.grouped(40, 4, 64, 32, seed=5, dist="uniform", group_list_type=1)
+    counts = np.array([0, 40, 0, 0], np.int64)
+    st, y = oracle.grouped_mm(p.x, p.D, p.W, counts, 1)
+    assert st == oracle.OK
+    assert np.array_equal(y, oracle.dense_mm(p.x, p.D[1], p.W[1]))
+
+
+# ----------------------------------------------------------------------------
+# Whole-layer sanity: the method's accuracy direction
+# ----------------------------------------------------------------------------
+
+def test_macaq_beats_plain_mxfp4_on_outlier_activations():
+    # Direction stated by the accuracy section (native error > MACAQ error);
+    # the size of the ratio on synthetic data is not pinned.
+    p = synth.dense(32, 256, 64, seed=0)
+    ref = oracle.linear_f64(p.x, p.W[0])
+    y = synth.bf16_bits_to_f32(oracle.dense_mm(p.x, p.D[0], p.W[0])).astype(np.float64)
+    qa, sa = oracle.quantize_plain(synth.bf16_bits_to_f32(p.x))
+    qw, sw = oracle.quantize_plain(p.W[0])
+    yp = synth.bf16_bits_to_f32(oracle.gemm(qa, sa, qw, sw)).astype(np.float64) * 32
+    nmse = lambda a: float(np.sum((a - ref) ** 2) / np.sum(ref ** 2))
+    assert nmse(y) < nmse(yp)
+    assert nmse(y) < 0.05
