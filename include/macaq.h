@@ -1,0 +1,165 @@
+/*
+ * macaq.h -- C ABI of the B200 (sm_100a) MACAQ W4A4 MXFP4 linear library.
+ *
+ * The operation (MACAQ page "MACAQ W4A4 fused dense and grouped matmul for
+ * Ascend 950", gitcode.com/cann/ops-nn/pull/12568, summary): for activations
+ * x (BF16) and a per-input-channel factor D, compute
+ *     y = RNE_bf16( 2^-5 * Q(H(x / D)) . Q(H(W * D))^T )
+ * where H is the block-32 unnormalised Sylvester Hadamard rotation along K
+ * (H.H^T = 32 I, hence the exact 2^-5), and Q is MXFP4 quantisation along K:
+ * blocks of 32 elements, one E8M0 scale per block chosen by OCP MX
+ * scale_alg = 0 (floor(log2 amax) - 2), E2M1 elements rounded to nearest even
+ * with saturation (same page, "Latency against existing native CANN
+ * operators": block32 E2M1, round-to-even, scale_alg=0).  The activation
+ * side keeps BF16 values between steps: xs = RNE_bf16(RN32(x * RN32(1/D))),
+ * u = RNE_bf16(FP32 butterfly of xs).  The weight side W * D -> H -> Q is
+ * done once, offline (same page: "weight transformation (W / D) @ H ... are
+ * offline"; read here as W * D so that the transform preserves x . W^T).
+ * The contraction accumulates in FP32 and writes BF16.
+ *
+ * The grouped form follows torch_npu.npu_grouped_matmul (function
+ * description: y_i = x_i @ weight_i; parameters group_list and
+ * group_list_type): rows [off_g, off_g + count_g) of x use expert g's D and
+ * weights; group_list holds E int64 values, cumulative sums (type 0) or
+ * counts (type 1), non-negative, cumulative sums non-decreasing, covering
+ * exactly M rows; at most 1024 groups.
+ *
+ * Conventions for every entry point:
+ *  - Pointers named *_dev are device pointers owned by the caller.  The
+ *    library never frees or keeps them; it allocates no memory on any call.
+ *  - BF16 tensors are passed as uint16_t bit patterns.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Calls are asynchronous on that stream; none synchronises
+ *    except macaq_prepare_weights, which reads D back to validate it.
+ *  - Return value: MACAQ_OK (0) or a negative status below.  A call that
+ *    returns an error launched nothing.  Errors found on the device (an
+ *    invalid group_list, a bounded wait that expired) are written to the
+ *    optional device word *status_dev, and the output is then left as it was
+ *    (group_list errors) or incomplete (timeouts).
+ *  - Shapes: 256 <= K <= 65536 with K % 256 == 0; 16 <= N <= 65536 with
+ *    N % 16 == 0 (the 65536 inner-axis limit is the npu_grouped_matmul
+ *    page's InnerLimit); 0 <= M <= 2^31 - 1 (M = 0 does nothing);
+ *    1 <= E <= 1024.
+ *  - Every pointer must be 16-byte aligned; y must not overlap any input.
+ */
+#ifndef MACAQ_H
+#define MACAQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MACAQ_ABI_VERSION 1
+
+#define MACAQ_OK 0
+#define MACAQ_ERR_NULL (-1)               /* a required pointer is NULL */
+#define MACAQ_ERR_ALIGN (-2)              /* a pointer is not 16-byte aligned */
+#define MACAQ_ERR_SHAPE (-3)              /* M, N, K or E outside the limits above */
+#define MACAQ_ERR_ARCH (-4)               /* current device is not sm_100 */
+#define MACAQ_ERR_ALIAS (-5)              /* the output overlaps an input */
+#define MACAQ_ERR_TOO_MANY_GROUPS (-6)    /* E < 1 or E > 1024 */
+#define MACAQ_ERR_GROUP_LIST_TYPE (-7)    /* group_list_type not 0 or 1 */
+#define MACAQ_ERR_CUDA (-8)               /* a CUDA runtime call failed */
+#define MACAQ_ERR_DEVICE_TIMEOUT (-9)     /* (device) a bounded wait expired */
+#define MACAQ_ERR_GROUP_LIST_INVALID (-10)/* (device) group_list breaks the rules */
+#define MACAQ_ERR_WORKSPACE (-11)         /* workspace missing or too small */
+#define MACAQ_ERR_BAD_D (-12)             /* D has a zero or non-finite entry */
+
+/* Name of a status code (static string). */
+const char *macaq_status_string(int status);
+/* MACAQ_ABI_VERSION of the loaded library. */
+int macaq_abi_version(void);
+
+/* ------------------------------------------------------------------ */
+/* Offline weight preparation                                          */
+/* ------------------------------------------------------------------ */
+
+/* Bytes of the prepared weight codes / scales for E experts of N x K.
+ * Prepared weights are stored as tensor-core-ready tiles of 128 rows x 256 K:
+ * codes 16384 bytes per tile (rows padded to a multiple of 128 with zero
+ * codes), scales 1024 bytes per tile.  Returns 0 for invalid shapes. */
+size_t macaq_weight_code_bytes(int64_t E, int64_t N, int64_t K);
+size_t macaq_weight_scale_bytes(int64_t E, int64_t N, int64_t K);
+
+/* Offline step of the MACAQ page's summary ("weight transformation ... are
+ * offline"): Wq/Ws <- MXFP4(H(W * D)) for each expert, FP32 throughout.
+ *   W_dev  fp32 [E, N, K] row-major; D_dev fp32 [E, K] (nonzero, finite);
+ *   Wq_dev macaq_weight_code_bytes(E,N,K) bytes; Ws_dev ..._scale_bytes.
+ * Synchronises `stream` once to check D (MACAQ_ERR_BAD_D). */
+int macaq_prepare_weights(const float *W_dev, const float *D_dev, int64_t E, int64_t N, int64_t K,
+                          uint8_t *Wq_dev, uint8_t *Ws_dev, void *stream);
+
+/* ------------------------------------------------------------------ */
+/* Hot path                                                            */
+/* ------------------------------------------------------------------ */
+
+/* Scratch bytes a dense (E = 1, group_list NULL) or grouped call of this shape
+ * needs.  The workspace holds split-K partial sums, tile counters and the
+ * quantised activations of the quantise-once path.  It must be zero-filled
+ * before its first use; every completed call leaves its counters at zero
+ * again, so one zero-fill at allocation is enough.  Calls that share a
+ * workspace must not run concurrently. */
+size_t macaq_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t E);
+
+/* Dense MACAQ linear (MACAQ page, summary: channel scaling, block-32 BF16
+ * Hadamard rotation, MXFP4 activation quantisation and matmul in one kernel,
+ * BF16 output).
+ *   x_dev  bf16 [M, K] row-major;  D_dev fp32 [K];
+ *   Wq_dev, Ws_dev from macaq_prepare_weights with E = 1;
+ *   y_dev  bf16 [M, N] row-major (written);
+ *   workspace_dev / workspace_bytes: see macaq_workspace_bytes (may be NULL
+ *   when that size is 0);
+ *   status_dev: optional int32 device word, written only on a device error. */
+int macaq_dense_mm(const uint16_t *x_dev, const float *D_dev, const uint8_t *Wq_dev, const uint8_t *Ws_dev,
+                   uint16_t *y_dev, int64_t M, int64_t N, int64_t K, void *workspace_dev,
+                   size_t workspace_bytes, int32_t *status_dev, void *stream);
+
+/* Grouped MACAQ linear (npu_grouped_matmul single-x / single-weight /
+ * single-y form, group_type 0).
+ *   D_dev fp32 [E, K]; Wq_dev/Ws_dev prepared with this E;
+ *   group_list_dev int64 [E] on the device (never read by the host);
+ *   group_list_type 0 = cumulative sums, 1 = counts.
+ * An invalid group_list writes MACAQ_ERR_GROUP_LIST_INVALID to *status_dev
+ * and leaves y untouched. */
+int macaq_grouped_mm(const uint16_t *x_dev, const float *D_dev, const uint8_t *Wq_dev, const uint8_t *Ws_dev,
+                     const int64_t *group_list_dev, int group_list_type, int64_t E, uint16_t *y_dev,
+                     int64_t M, int64_t N, int64_t K, void *workspace_dev, size_t workspace_bytes,
+                     int32_t *status_dev, void *stream);
+
+/* ------------------------------------------------------------------ */
+/* Test and ablation entry points (not the product's hot path)         */
+/* ------------------------------------------------------------------ */
+
+/* The activation prologue alone, writing canonical codes [M, K/2] (element
+ * 2j in the low nibble of byte j) and scales [M, K/32]. Same device code as
+ * the fused kernels. */
+int macaq_quantize_activations(const uint16_t *x_dev, const float *D_dev, uint8_t *codes_dev,
+                               uint8_t *scales_dev, int64_t M, int64_t K, void *stream);
+
+/* Prepared (tiled) weights -> canonical codes [E, N, K/2] and scales
+ * [E, N, K/32]. */
+int macaq_export_weights(const uint8_t *Wq_dev, const uint8_t *Ws_dev, uint8_t *codes_dev, uint8_t *scales_dev,
+                         int64_t E, int64_t N, int64_t K, void *stream);
+
+/* MX encoding of fp32 blocks of 32 (E8M0 from the block amax, E2M1
+ * round-to-nearest-even with saturation): n % 32 == 0; codes n/2 bytes,
+ * scales n/32 bytes.  Used to test the conversion instructions exhaustively. */
+int macaq_mx_encode_blocks(const float *v_dev, uint8_t *codes_dev, uint8_t *scales_dev, int64_t n,
+                           void *stream);
+
+/* Unfused ablation (the MACAQ page's "split MACAQ paths"): a separate
+ * quantisation kernel writes the activation codes to the workspace, then the
+ * block-scaled GEMM reads them.  Same arguments and result as
+ * macaq_dense_mm; needs macaq_unfused_workspace_bytes(M, K) bytes. */
+size_t macaq_unfused_workspace_bytes(int64_t M, int64_t K);
+int macaq_unfused_dense_mm(const uint16_t *x_dev, const float *D_dev, const uint8_t *Wq_dev,
+                           const uint8_t *Ws_dev, uint16_t *y_dev, int64_t M, int64_t N, int64_t K,
+                           void *workspace_dev, size_t workspace_bytes, int32_t *status_dev, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MACAQ_H */

@@ -1,0 +1,100 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/macaq.h declares, and refuses bad arguments by name
+before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import w4a4_mxfp4_quantize_b200 as mq
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "macaq.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    mq.build()
+    return mq.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(macaq_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for need in ["macaq_prepare_weights", "macaq_dense_mm", "macaq_grouped_mm", "macaq_workspace_bytes",
+                 "macaq_weight_code_bytes", "macaq_weight_scale_bytes", "macaq_quantize_activations",
+                 "macaq_export_weights", "macaq_unfused_dense_mm", "macaq_status_string"]:
+        assert need in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_functions():
+        assert hasattr(L, name), name
+    assert set(declared_functions()) <= set(mq.exported_symbols()) | {"macaq_abi_version"}
+
+
+def test_abi_version_and_status_strings(L):
+    assert L.macaq_abi_version() == 1
+    for code, name in mq.STATUS.items():
+        assert L.macaq_status_string(code).decode() == name
+    assert L.macaq_status_string(-99).decode() == "MACAQ_ERR_UNKNOWN"
+
+
+def test_weight_sizes(L):
+    assert L.macaq_weight_code_bytes(1, 1024, 1024) == 1024 * 512
+    assert L.macaq_weight_scale_bytes(1, 1024, 1024) == 1024 * 32
+    assert L.macaq_weight_code_bytes(2, 48, 256) == 2 * 128 * 128  # rows padded to 128
+    assert L.macaq_weight_code_bytes(1, 1000, 1024) == 0           # N % 16 != 0
+    assert L.macaq_weight_code_bytes(1, 1024, 1000) == 0           # K % 256 != 0
+    assert L.macaq_weight_code_bytes(1025, 1024, 1024) == 0        # E > 1024
+    assert L.macaq_unfused_workspace_bytes(16, 1024) == 128 * (512 + 32)
+
+
+P = ctypes.c_void_p
+A, B, C, Dp, Y = (P(i << 32) for i in range(1, 6))
+
+
+def dense(L, x=A, d=B, wq=C, ws=Dp, y=Y, M=16, N=1024, K=1024):
+    return L.macaq_dense_mm(x, d, wq, ws, y, M, N, K, None, 0, None, None)
+
+
+def test_dense_refusals_by_name(L):
+    assert dense(L, N=1000) == -3
+    assert dense(L, K=1000) == -3
+    assert dense(L, K=128) == -3
+    assert dense(L, K=65536 + 256) == -3
+    assert dense(L, N=65536 + 16) == -3
+    assert dense(L, M=-1) == -3
+    assert dense(L, x=None) == -1
+    assert dense(L, y=None) == -1
+    assert dense(L, x=P((1 << 32) + 8)) == -2
+    assert dense(L, y=P(1 << 32)) == -5           # y overlaps x
+    assert dense(L, M=0, x=None) == 0            # M = 0 is a no-op
+
+
+def test_grouped_refusals_by_name(L):
+    gl = P(9 << 32)
+
+    def g(E=4, t=1, glp=gl, N=1024, K=1024, M=64):
+        return L.macaq_grouped_mm(A, B, C, Dp, glp, t, E, Y, M, N, K, None, 0, None, None)
+
+    assert g(E=0) == -6
+    assert g(E=1025) == -6
+    assert g(t=2) == -7
+    assert g(t=-1) == -7
+    assert g(N=24) == -3
+    assert g(glp=None) == -1
+    assert g(glp=P((9 << 32) + 4)) == -2
+
+
+def test_no_gpu_means_a_named_cuda_error_not_a_fallback(L):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("GPU present")
+    assert dense(L) == -8

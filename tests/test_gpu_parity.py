@@ -1,0 +1,331 @@
+"""GPU parity of the CUDA path against the CPU oracle, through the C ABI.
+
+Bit-exact: activation codes and E8M0 scales, prepared weight codes and
+scales, and the MX conversion itself.  BF16 outputs: the tolerance described
+in tests/helpers.py.  Every input is seeded and synthetic (synth).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import w4a4_mxfp4_quantize_b200 as mq
+from helpers import compare, dequant_matmul_bf16, f32_dev, x_to_dev, y_to_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    mq.build()
+    mq.lib()
+    torch.cuda.init()
+
+
+# ----------------------------------------------------------------------------
+# MX conversion (E8M0 + E2M1 with the hardware cvt) -- bit exact
+# ----------------------------------------------------------------------------
+
+def _gpu_mx(blocks: np.ndarray):
+    q, s = mq.mx_encode_blocks(f32_dev(blocks.ravel()))
+    torch.cuda.synchronize()
+    return q.cpu().numpy(), s.cpu().numpy()
+
+
+def test_mx_encode_all_bf16_values_at_many_scales():
+    bits = np.arange(65536, dtype=np.uint32)
+    f = (bits << 16).view(np.float32)
+    f = f[np.isfinite(f)]
+    rng = np.random.default_rng(0)
+    f = f[rng.permutation(f.size)]
+    f = f[: f.size // 32 * 32]
+    q, s = _gpu_mx(f)
+    qo, so = oracle.mx_quantize_blocks(f)
+    assert np.array_equal(s, so)
+    assert np.array_equal(q, qo)
+
+
+def test_mx_encode_tie_points_and_saturation_edges():
+    rows = []
+    for c in [0, 1, 2, 3, 60, 120, 127, 130, 200, 250, 252]:
+        unit = np.ldexp(1.0, c - 127)
+        vals = [6.0, -6.0, 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -0.75, -1.25, -1.75, -2.5, -3.5,
+                -5.0, 0.2499, 0.7501, 5.0001, 4.9999, 7.99, -7.99, 0.0, -0.0, 1e-40, -1e-40, 2.9999, 3.0001,
+                1.2499, 1.7501, 0.5, 6.0]
+        blk = np.array([v * unit for v in vals], np.float64).astype(np.float32)
+        rows.append(blk)
+    blocks = np.stack(rows)
+    q, s = _gpu_mx(blocks)
+    qo, so = oracle.mx_quantize_blocks(blocks)
+    assert np.array_equal(s, so)
+    assert np.array_equal(q, qo)
+
+
+def test_mx_encode_random_wide_range_and_zero_blocks():
+    rng = np.random.default_rng(1)
+    v = (rng.standard_normal((4096, 32)) * np.exp2(rng.integers(-140, 120, (4096, 1)))).astype(np.float32)
+    v[::97] = 0.0
+    v[1::97] = -0.0
+    v[2::97, :31] = 0.0
+    q, s = _gpu_mx(v)
+    qo, so = oracle.mx_quantize_blocks(v)
+    assert np.array_equal(s, so)
+    assert np.array_equal(q, qo)
+
+
+# ----------------------------------------------------------------------------
+# Activation prologue -- bit exact on codes and scales
+# ----------------------------------------------------------------------------
+
+def _gpu_act(x_bits, D):
+    q, s = mq.quantize_activations(x_to_dev(x_bits), f32_dev(D))
+    torch.cuda.synchronize()
+    return q.cpu().numpy(), s.cpu().numpy()
+
+
+@pytest.mark.parametrize("cfg", [0, 1, 2])
+def test_activation_codes_bit_exact_on_dense_configs(cfg):
+    for p in synth.config(cfg):
+        q, s = _gpu_act(p.x, p.D[0])
+        qo, so = oracle.quantize_act(p.x, p.D[0])
+        assert np.array_equal(s, so), p.name
+        assert np.array_equal(q, qo), p.name
+
+
+def test_activation_codes_bit_exact_adversarial():
+    rng = np.random.default_rng(2)
+    M, K = 300, 512
+    x = rng.standard_normal((M, K)).astype(np.float32)
+    x[0] = 1.0                        # all-equal blocks
+    x[1] = 0.0                        # zero rows
+    x[2] = -0.0
+    x[3, ::2] = 1e-38                 # tiny values
+    x[4] *= 1e30                      # huge values
+    x[5] = np.where(np.arange(K) % 2, -1.0, 1.0)
+    x[6:40] *= np.exp2(rng.integers(-40, 40, (34, 1)))
+    xb = synth.to_bf16_bits(x)
+    xb[7] = rng.integers(0, 65536, K, dtype=np.uint32).astype(np.uint16) & 0x7F7F  # random finite patterns
+    D = np.exp(rng.standard_normal(K) * 2).astype(np.float32) * np.where(rng.random(K) < 0.3, -1, 1)
+    D = D.astype(np.float32)
+    q, s = _gpu_act(xb, D)
+    qo, so = oracle.quantize_act(xb, D)
+    assert np.array_equal(s, so)
+    assert np.array_equal(q, qo)
+
+
+# ----------------------------------------------------------------------------
+# Offline weight preparation -- bit exact
+# ----------------------------------------------------------------------------
+
+def _gpu_weights(W, D):
+    E, N, K = W.shape
+    Wq, Ws = mq.prepare_weights(f32_dev(W), f32_dev(D))
+    q, s = mq.export_weights(Wq, Ws, E, N, K)
+    torch.cuda.synchronize()
+    return Wq, Ws, q.cpu().numpy(), s.cpu().numpy()
+
+
+@pytest.mark.parametrize("shape", [(1, 1024, 1024), (1, 48, 256), (3, 144, 512), (2, 2048, 768)])
+def test_weight_prep_bit_exact(shape):
+    E, N, K = shape
+    rng = np.random.default_rng(3)
+    W = rng.normal(0, 0.02, shape).astype(np.float32)
+    W[0, 0] = 0.0
+    D = (np.exp(rng.standard_normal((E, K))) * np.where(rng.random((E, K)) < 0.2, -1, 1)).astype(np.float32)
+    _, _, q, s = _gpu_weights(W, D)
+    qo, so = oracle.quantize_weights(W, D)
+    assert np.array_equal(s, so)
+    assert np.array_equal(q, qo)
+
+
+def test_prepare_rejects_bad_d():
+    W = torch.zeros((1, 16, 256), device="cuda")
+    D = torch.ones((1, 256), device="cuda")
+    D[0, 7] = 0.0
+    with pytest.raises(mq.MacaqError) as e:
+        mq.prepare_weights(W, D)
+    assert e.value.status == -12
+
+
+# ----------------------------------------------------------------------------
+# Dense fused linear -- tolerance on BF16 output
+# ----------------------------------------------------------------------------
+
+def _run_dense(p: synth.Problem, fn=None):
+    fn = fn or mq.dense_mm
+    Wq, Ws = mq.prepare_weights(f32_dev(p.W), f32_dev(p.D))
+    y = fn(x_to_dev(p.x), f32_dev(p.D[0]), Wq, Ws, p.N)
+    torch.cuda.synchronize()
+    return y_to_bits(y)
+
+
+def _oracle_dense_full(p):
+    qa, sa = oracle.quantize_act(p.x, p.D[0])
+    qw, sw = oracle.quantize_weights(p.W[0], p.D[0])
+    return oracle.gemm(qa, sa, qw, sw)
+
+
+@pytest.mark.parametrize("M,K,N", [(1, 256, 16), (16, 256, 128), (5, 512, 48), (17, 1024, 144), (64, 768, 256),
+                                   (100, 512, 384), (128, 256, 128), (129, 512, 256), (300, 1024, 160)])
+def test_dense_small_shapes_exact_oracle(M, K, N):
+    p = synth.dense(M, K, N, seed=M + K + N)
+    compare(_run_dense(p), _oracle_dense_full(p), f"dense {M}x{K}x{N}")
+
+
+@pytest.mark.parametrize("cfg", [0, 1])
+def test_dense_configs_full_oracle(cfg):
+    for p in synth.config(cfg):
+        compare(_run_dense(p), _oracle_dense_full(p), p.name)
+
+
+def _check_large(p: synth.Problem, y_bits: np.ndarray, n_samples: int = 3000):
+    qa, sa = oracle.quantize_act(p.x, p.D[0])
+    qw, sw = oracle.quantize_weights(p.W[0], p.D[0])
+    rng = np.random.default_rng(7)
+    rows = rng.integers(0, p.M, n_samples)
+    cols = rng.integers(0, p.N, n_samples)
+    exact = oracle.gemm_at(qa, sa, qw, sw, rows, cols)
+    compare(y_bits[rows, cols], exact, p.name + " sampled exact")
+    compare(y_bits, dequant_matmul_bf16(qa, sa, qw, sw), p.name + " full f64")
+
+
+@pytest.mark.parametrize("i", [0, 3, 4])
+def test_dense_prefill_config(i):
+    p = synth.config(2)[i]
+    _check_large(p, _run_dense(p))
+
+
+def test_unfused_ablation_matches_oracle():
+    for p in [synth.dense(16, 1024, 1024, 0), synth.dense(200, 512, 384, 1), synth.config(2)[1]]:
+        y = _run_dense(p, mq.unfused_dense_mm)
+        if p.M <= 256:
+            compare(y, _oracle_dense_full(p), p.name + " unfused")
+        else:
+            _check_large(p, y)
+
+
+def test_dense_zero_rows_is_noop():
+    p = synth.dense(16, 256, 64, 0)
+    Wq, Ws = mq.prepare_weights(f32_dev(p.W), f32_dev(p.D))
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    y = mq.dense_mm(x, f32_dev(p.D[0]), Wq, Ws, 64)
+    assert y.shape == (0, 64)
+
+
+def test_dense_on_a_side_stream_and_repeatable():
+    p = synth.dense(96, 1024, 512, 5)
+    Wq, Ws = mq.prepare_weights(f32_dev(p.W), f32_dev(p.D))
+    x, D = x_to_dev(p.x), f32_dev(p.D[0])
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        ys = [mq.dense_mm(x, D, Wq, Ws, p.N, stream=s) for _ in range(3)]
+    s.synchronize()
+    a = [y_to_bits(y) for y in ys]
+    assert np.array_equal(a[0], a[1]) and np.array_equal(a[0], a[2])   # deterministic
+    compare(a[0], _oracle_dense_full(p), "side stream")
+
+
+def test_signed_d():
+    p = synth.dense(40, 512, 128, 9)
+    p.D = (p.D * np.where(np.arange(512) % 3 == 0, -1, 1)).astype(np.float32)
+    compare(_run_dense(p), _oracle_dense_full(p), "signed D")
+
+
+# ----------------------------------------------------------------------------
+# Grouped
+# ----------------------------------------------------------------------------
+
+def _run_grouped(p: synth.Problem, gl=None, gtype=None, status=None):
+    Wq, Ws = mq.prepare_weights(f32_dev(p.W), f32_dev(p.D))
+    gl = p.group_list if gl is None else gl
+    gtype = p.group_list_type if gtype is None else gtype
+    y = mq.grouped_mm(x_to_dev(p.x), f32_dev(p.D), Wq, Ws, torch.from_numpy(np.asarray(gl, np.int64)).cuda(),
+                      gtype, p.N, status=status)
+    torch.cuda.synchronize()
+    return y
+
+
+def _oracle_grouped(p):
+    st, y = oracle.grouped_mm(p.x, p.D, p.W, p.group_list, p.group_list_type)
+    assert st == 0
+    return y
+
+
+@pytest.mark.parametrize("T,E,K,N,dist,gtype", [(96, 4, 256, 128, "uniform", 1), (200, 5, 512, 144, "uniform", 0),
+                                                 (300, 16, 256, 64, "zipf", 0), (64, 3, 1024, 256, "uniform", 1)])
+def test_grouped_small_exact_oracle(T, E, K, N, dist, gtype):
+    p = synth.grouped(T, E, K, N, seed=T + E, dist=dist, group_list_type=gtype)
+    compare(y_to_bits(_run_grouped(p)), _oracle_grouped(p), p.name)
+
+
+def test_grouped_empty_groups_first_last_consecutive():
+    p = synth.grouped(120, 6, 256, 64, seed=11, dist="uniform", group_list_type=1)
+    for counts in ([0, 0, 60, 0, 60, 0], [120, 0, 0, 0, 0, 0], [0, 0, 0, 0, 0, 120], [1, 0, 0, 118, 0, 1]):
+        p.group_list = np.array(counts, np.int64)
+        p.group_list_type = 1
+        compare(y_to_bits(_run_grouped(p)), _oracle_grouped(p), f"grouped {counts}")
+
+
+def test_grouped_cumsum_equals_counts():
+    p = synth.grouped(150, 4, 512, 128, seed=12, dist="uniform", group_list_type=1)
+    y1 = y_to_bits(_run_grouped(p))
+    y0 = y_to_bits(_run_grouped(p, np.cumsum(p.group_list), 0))
+    assert np.array_equal(y0, y1)
+
+
+def test_grouped_replicated_banks_equal_dense():
+    p = synth.grouped(256, 4, 1024, 256, seed=13, dist="uniform", group_list_type=1)
+    p.W = np.repeat(p.W[:1], 4, axis=0)
+    p.D = np.repeat(p.D[:1], 4, axis=0)
+    yg = y_to_bits(_run_grouped(p))
+    pd = synth.Problem(x=p.x, W=p.W[:1], D=p.D[:1], M=p.M, N=p.N, K=p.K)
+    yd = _run_dense(pd)
+    compare(yg, yd, "replicated banks vs dense")
+    compare(yg, _oracle_dense_full(pd), "replicated banks vs oracle")
+
+
+@pytest.mark.parametrize("gl,gtype", [([10, 5, 30], 0), ([10, -1, 21], 1), ([10, 10, 10], 1), ([10, 20, 29], 0),
+                                      ([-3, 20, 30], 0)])
+def test_grouped_invalid_group_list_sets_status_and_leaves_y(gl, gtype):
+    p = synth.grouped(30, 3, 256, 64, seed=14, dist="uniform", group_list_type=1)
+    Wq, Ws = mq.prepare_weights(f32_dev(p.W), f32_dev(p.D))
+    y = torch.full((30, 64), 7.0, dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    mq.grouped_mm(x_to_dev(p.x), f32_dev(p.D), Wq, Ws, torch.tensor(gl, dtype=torch.int64, device="cuda"), gtype,
+                  64, out=y, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == -10
+    assert bool(torch.all(y == 7.0))
+
+
+@pytest.mark.parametrize("which", [0, 1])
+def test_grouped_config3(which):
+    p = synth.config(3)[which]
+    y = y_to_bits(_run_grouped(p))
+    _check_grouped_sampled(p, y)
+
+
+@pytest.mark.parametrize("which", [0, 1])
+def test_grouped_config4(which):
+    p = synth.config(4)[which]
+    assert (p.counts == 0).sum() > 0          # some groups empty
+    y = y_to_bits(_run_grouped(p))
+    _check_grouped_sampled(p, y)
+
+
+def _check_grouped_sampled(p, y, per_group=24):
+    off = np.concatenate([[0], np.cumsum(p.counts)])
+    rng = np.random.default_rng(5)
+    got, want = [], []
+    for g in range(p.E):
+        if p.counts[g] == 0:
+            continue
+        rows = rng.integers(off[g], off[g + 1], per_group)
+        cols = rng.integers(0, p.N, per_group)
+        qa, sa = oracle.quantize_act(p.x[rows], p.D[g])
+        qw, sw = oracle.quantize_weights(p.W[g][np.unique(cols)], p.D[g])
+        idx = np.searchsorted(np.unique(cols), cols)
+        want.append(oracle.gemm_at(qa, sa, qw, sw, np.arange(per_group), idx))
+        got.append(y[rows, cols])
+    compare(np.concatenate(got), np.concatenate(want), p.name + " sampled exact")

@@ -1,0 +1,255 @@
+"""B200-native MACAQ W4A4 MXFP4 linear (dense and grouped).
+
+A thin Python binding over the C ABI in ``include/macaq.h`` (library
+``libmacaq.so`` built in this directory).  This module only marshals
+arguments: every step of the computation runs in the library's sm_100a
+kernels.  PyTorch provides device memory and streams.  There is no CPU
+fallback: without the built library or a B200, every call raises.
+
+The operation (MACAQ page "MACAQ W4A4 fused dense and grouped matmul for
+Ascend 950", summary): y = BF16(2^-5 * MXFP4(H(x/D)) . MXFP4(H(W*D))^T) with H
+the block-32 Sylvester Hadamard rotation along K; grouped calls follow
+torch_npu.npu_grouped_matmul's group_list / group_list_type.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_ROOT = os.path.dirname(_HERE)
+_LIB_PATH = os.path.join(_HERE, "libmacaq.so")
+_SRC = os.path.join(_HERE, "csrc", "macaq.cu")
+_INCLUDE = os.path.join(_ROOT, "include")
+
+NVCC_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
+              "-Xcompiler", "-fPIC", "-shared"]
+
+STATUS = {
+    0: "MACAQ_OK", -1: "MACAQ_ERR_NULL", -2: "MACAQ_ERR_ALIGN", -3: "MACAQ_ERR_SHAPE",
+    -4: "MACAQ_ERR_ARCH", -5: "MACAQ_ERR_ALIAS", -6: "MACAQ_ERR_TOO_MANY_GROUPS",
+    -7: "MACAQ_ERR_GROUP_LIST_TYPE", -8: "MACAQ_ERR_CUDA", -9: "MACAQ_ERR_DEVICE_TIMEOUT",
+    -10: "MACAQ_ERR_GROUP_LIST_INVALID", -11: "MACAQ_ERR_WORKSPACE", -12: "MACAQ_ERR_BAD_D",
+}
+
+
+class MacaqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({status})")
+        self.status = status
+
+
+def _sources():
+    d = os.path.join(_HERE, "csrc")
+    return [os.path.join(d, f) for f in sorted(os.listdir(d))] + [os.path.join(_INCLUDE, "macaq.h")]
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile libmacaq.so for sm_100a in-tree (nvcc cross-compiles without a GPU)."""
+    newest = max(os.path.getmtime(f) for f in _sources())
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < newest:
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        cmd = ["nvcc", *NVCC_FLAGS, "-I" + _INCLUDE, "-o", tmp, _SRC]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+        subprocess.check_call(cmd)
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+_lib = None
+_lock = threading.Lock()
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SIG = {
+    "macaq_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "macaq_abi_version": (ctypes.c_int, []),
+    "macaq_weight_code_bytes": (ctypes.c_size_t, [_I64, _I64, _I64]),
+    "macaq_weight_scale_bytes": (ctypes.c_size_t, [_I64, _I64, _I64]),
+    "macaq_prepare_weights": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _P]),
+    "macaq_workspace_bytes": (ctypes.c_size_t, [_I64, _I64, _I64, _I64]),
+    "macaq_dense_mm": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, ctypes.c_size_t, _P, _P]),
+    "macaq_grouped_mm": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, _I64, _P, _I64, _I64, _I64, _P,
+                                        ctypes.c_size_t, _P, _P]),
+    "macaq_quantize_activations": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _P]),
+    "macaq_export_weights": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
+    "macaq_mx_encode_blocks": (ctypes.c_int, [_P, _P, _P, _I64, _P]),
+    "macaq_unfused_workspace_bytes": (ctypes.c_size_t, [_I64, _I64]),
+    "macaq_unfused_dense_mm": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, ctypes.c_size_t,
+                                              _P, _P]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        with _lock:
+            if _lib is None:
+                if not os.path.exists(_LIB_PATH):
+                    raise RuntimeError(f"libmacaq.so is not built ({_LIB_PATH}); run "
+                                       "w4a4_mxfp4_quantize_b200.build()")
+                L = ctypes.CDLL(_LIB_PATH)
+                for name, (res, args) in _SIG.items():
+                    f = getattr(L, name)
+                    f.restype = res
+                    f.argtypes = args
+                _lib = L
+    return _lib
+
+
+def exported_symbols() -> list[str]:
+    return list(_SIG)
+
+
+def _check(st: int, where: str):
+    if st != 0:
+        raise MacaqError(st, where)
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("expected contiguous CUDA tensors")
+
+
+# ---------------------------------------------------------------------------
+# workspace: one zero-filled buffer per (device, stream), grown on demand
+# ---------------------------------------------------------------------------
+_ws: dict = {}
+
+
+def workspace(nbytes: int, device: torch.device, stream=None) -> torch.Tensor | None:
+    if nbytes == 0:
+        return None
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    key = (device.index, s.cuda_stream)
+    buf = _ws.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _ws[key] = buf
+    return buf
+
+
+# ---------------------------------------------------------------------------
+# public API
+# ---------------------------------------------------------------------------
+
+def weight_bytes(E: int, N: int, K: int) -> tuple[int, int]:
+    L = lib()
+    return int(L.macaq_weight_code_bytes(E, N, K)), int(L.macaq_weight_scale_bytes(E, N, K))
+
+
+def prepare_weights(W: torch.Tensor, D: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Offline: W fp32 [N, K] or [E, N, K], D fp32 [K] or [E, K] -> (Wq, Ws) tile images."""
+    if W.dim() == 2:
+        W = W.unsqueeze(0)
+    if D.dim() == 1:
+        D = D.unsqueeze(0)
+    _require_cuda(W, D)
+    E, N, K = W.shape
+    qb, sb = weight_bytes(E, N, K)
+    if qb == 0:
+        raise MacaqError(-3, "prepare_weights")
+    Wq = torch.empty(qb, dtype=torch.uint8, device=W.device)
+    Ws = torch.empty(sb, dtype=torch.uint8, device=W.device)
+    _check(lib().macaq_prepare_weights(_ptr(W), _ptr(D), E, N, K, _ptr(Wq), _ptr(Ws), _stream_ptr(stream)),
+           "macaq_prepare_weights")
+    return Wq, Ws
+
+
+def dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: int,
+             out: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """y [M, N] bf16 = MACAQ linear of x bf16 [M, K] (fused kernel)."""
+    _require_cuda(x, D, Wq, Ws, out, status)
+    M, K = x.shape
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    L = lib()
+    need = int(L.macaq_workspace_bytes(M, N, K, 1))
+    ws = workspace(need, x.device, stream)
+    _check(L.macaq_dense_mm(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(y), M, N, K, _ptr(ws),
+                            0 if ws is None else ws.numel(), _ptr(status), _stream_ptr(stream)),
+           "macaq_dense_mm")
+    return y
+
+
+def grouped_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, group_list: torch.Tensor,
+               group_list_type: int, N: int, out: torch.Tensor | None = None,
+               status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Grouped MACAQ linear; group_list int64 [E] on the device (0 cumsum, 1 counts)."""
+    _require_cuda(x, D, Wq, Ws, group_list, out, status)
+    M, K = x.shape
+    E = group_list.numel()
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    L = lib()
+    need = int(L.macaq_workspace_bytes(M, N, K, E))
+    ws = workspace(need, x.device, stream)
+    _check(L.macaq_grouped_mm(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(group_list), int(group_list_type), E,
+                              _ptr(y), M, N, K, _ptr(ws), 0 if ws is None else ws.numel(), _ptr(status),
+                              _stream_ptr(stream)),
+           "macaq_grouped_mm")
+    return y
+
+
+def unfused_dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: int,
+                     out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Ablation: separate quantisation kernel, then the block-scaled GEMM."""
+    _require_cuda(x, D, Wq, Ws, out, status)
+    M, K = x.shape
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    L = lib()
+    need = int(L.macaq_unfused_workspace_bytes(M, K))
+    ws = workspace(need, x.device, stream)
+    _check(L.macaq_unfused_dense_mm(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(y), M, N, K, _ptr(ws),
+                                    0 if ws is None else ws.numel(), _ptr(status), _stream_ptr(stream)),
+           "macaq_unfused_dense_mm")
+    return y
+
+
+def quantize_activations(x: torch.Tensor, D: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Activation prologue alone: canonical codes [M, K/2] and E8M0 scales [M, K/32]."""
+    _require_cuda(x, D)
+    M, K = x.shape
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+    scales = torch.empty((M, K // 32), dtype=torch.uint8, device=x.device)
+    _check(lib().macaq_quantize_activations(_ptr(x), _ptr(D), _ptr(codes), _ptr(scales), M, K,
+                                            _stream_ptr(stream)), "macaq_quantize_activations")
+    return codes, scales
+
+
+def export_weights(Wq: torch.Tensor, Ws: torch.Tensor, E: int, N: int, K: int,
+                   stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Prepared tile images -> canonical codes [E, N, K/2] and scales [E, N, K/32]."""
+    _require_cuda(Wq, Ws)
+    codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=Wq.device)
+    scales = torch.empty((E, N, K // 32), dtype=torch.uint8, device=Wq.device)
+    _check(lib().macaq_export_weights(_ptr(Wq), _ptr(Ws), _ptr(codes), _ptr(scales), E, N, K,
+                                      _stream_ptr(stream)), "macaq_export_weights")
+    return codes, scales
+
+
+def mx_encode_blocks(v: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """MX encoding (E8M0 + E2M1) of fp32 blocks of 32."""
+    _require_cuda(v)
+    n = v.numel()
+    codes = torch.empty(n // 2, dtype=torch.uint8, device=v.device)
+    scales = torch.empty(n // 32, dtype=torch.uint8, device=v.device)
+    _check(lib().macaq_mx_encode_blocks(_ptr(v), _ptr(codes), _ptr(scales), n, _stream_ptr(stream)),
+           "macaq_mx_encode_blocks")
+    return codes, scales
