@@ -1,0 +1,409 @@
+"""Benchmark of the B200 MACAQ W4A4 MXFP4 linear.
+
+One step = one pass of the whole hot path over one batch of the headline
+workload: the dense M=128 MACAQ linear over the five Qwen3-0.6B-shaped
+projections (K, N) in {(1024,2048), (1024,1024), (2048,1024), (1024,3072),
+(3072,1024)}, bf16 activations with 1% outlier channels x20, MXFP4 weights
+prepared offline, BF16 output.  Inputs are seeded and synthetic (synth).
+
+Timing: W warm-up steps, then exactly K steps, each preceded (outside the
+timed interval) by a 256 MiB write that flushes the 126 MB L2; device time from
+CUDA events on the launching stream; barrier + synchronize around the timed
+region; max over ranks.  N > 1 GPUs run independent replicas (the layer needs
+no exchange), so scaling is weak.
+
+Also reported: e2e (the same calls with the activations copied from pinned
+host memory and the outputs copied back inside the timed interval), the
+roofline of the dominant kernel, the per-workload table of all five
+workloads (us/call, TFLOPS, fraction of roofline, unfused ablation), the
+clocks seen during the timed region, and the CPU oracle on a bounded sample.
+
+`--impl reference` times the CPU oracle (the reference arm) on the same
+workload and metric.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "fused W4A4 MXFP4 TFLOPS & µs/call vs FP4/HBM roofline, dense M=16/128/4096 + grouped"
+UNIT = "TFLOPS"
+WORKLOAD = "dense M=128 MACAQ W4A4 MXFP4 linear x 5 Qwen3-0.6B projections (K,N)=" \
+           "(1024,2048),(1024,1024),(2048,1024),(1024,3072),(3072,1024)"
+FP4_NOMINAL_TFLOPS = 9000.0   # NVIDIA's published dense FP4 figure for B200
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), float(pk["bf16_tflops"]), "measured"
+    except Exception:
+        return 6650.0, 1590.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out = ""
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        hi = [v for v in sm if v > 0.5 * max(sm)]
+        return {"sm_mhz": statistics.median(hi), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def x_dev(xbits, device):
+    return torch.from_numpy(np.ascontiguousarray(xbits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def f32(a, device):
+    return torch.from_numpy(np.ascontiguousarray(a, np.float32)).to(device)
+
+
+class Prepared:
+    """A problem with its weights prepared on the device (untimed, offline)."""
+
+    def __init__(self, p: synth.Problem, device, mq):
+        self.p = p
+        self.x = x_dev(p.x, device)
+        self.x_host = torch.from_numpy(np.ascontiguousarray(p.x).view(np.int16)).view(torch.bfloat16).pin_memory()
+        self.D = f32(p.D if p.E > 1 else p.D[0], device)
+        W = f32(p.W, device)
+        self.Wq, self.Ws = mq.prepare_weights(W, f32(p.D, device))
+        del W
+        self.y = torch.empty((p.M, p.N), dtype=torch.bfloat16, device=device)
+        self.y_host = torch.empty((p.M, p.N), dtype=torch.bfloat16).pin_memory()
+        self.gl = None if p.group_list is None else torch.from_numpy(p.group_list.astype(np.int64)).to(device)
+
+    def run(self, mq, stream, x=None, y=None):
+        x = self.x if x is None else x
+        y = self.y if y is None else y
+        if self.gl is None:
+            mq.dense_mm(x, self.D, self.Wq, self.Ws, self.p.N, out=y, stream=stream)
+        else:
+            mq.grouped_mm(x, self.D, self.Wq, self.Ws, self.gl, self.p.group_list_type, self.p.N, out=y,
+                          stream=stream)
+
+    def run_unfused(self, mq, stream):
+        mq.unfused_dense_mm(self.x, self.D, self.Wq, self.Ws, self.p.N, out=self.y, stream=stream)
+
+
+def time_calls(fn, flush, stream, reps: int, warm: int = 3, cold: bool = True):
+    """Median / IQR of per-call device time (us) with CUDA events on `stream`."""
+    for _ in range(warm):
+        fn()
+    evs = []
+    for _ in range(reps):
+        if cold:
+            flush()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        evs.append((a, b))
+    stream.synchronize()
+    t = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)
+    q = np.percentile(t, [25, 50, 75])
+    return float(q[1]), float(q[2] - q[0])
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle
+# ---------------------------------------------------------------------------
+def cpu_oracle_sample(problems, budget_s: float = 12.0, rows: int = 4, prepared=None):
+    """The oracle's hot path (activation quantisation + exact GEMM) on `rows`
+    rows of every problem, weights prepared beforehand (offline, untimed, as
+    on the GPU); returns (TFLOPS, seconds, threads, description, prepared)."""
+    import oracle
+    if prepared is None:
+        prepared = [oracle.quantize_weights(p.W[0], p.D[0]) for p in problems]
+    t0 = time.perf_counter()
+    flops = 0.0
+    n = 0
+    while True:
+        for p, (qw, sw) in zip(problems, prepared):
+            qa, sa = oracle.quantize_act(p.x[:rows], p.D[0])
+            oracle.gemm(qa, sa, qw, sw)
+            flops += 2.0 * rows * p.N * p.K
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 1000:
+            break
+    return flops / el / 1e12, el, oracle.num_threads(), (
+        f"{rows} of {problems[0].M} rows of each of the {len(problems)} projections, {n} passes "
+        "(activation quantisation + exact block-scaled GEMM; weights prepared beforehand)"), prepared
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    problems = synth.config(1)
+    steps = []
+    prepared = None
+    for _ in range(args.warmup):
+        *_, prepared = cpu_oracle_sample(problems, budget_s=0.0, rows=1, prepared=prepared)
+    for _ in range(args.steps):
+        v, el, cores, sample, _ = cpu_oracle_sample(problems, budget_s=min(10.0, 120.0 / max(1, args.steps)),
+                                                    rows=4, prepared=prepared)
+        steps.append((v, el))
+    value = statistics.median(v for v, _ in steps)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * statistics.median(el for _, el in steps), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4(e2m1,e8m0)->exact->bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": 128, "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=30)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-table", action="store_true", help="skip the per-workload table")
+    ap.add_argument("--table-reps", type=int, default=30)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        if dist is not None:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
+
+    import w4a4_mxfp4_quantize_b200 as mq
+    mq.lib()  # fails loudly when the CUDA library is missing
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    stream = torch.cuda.Stream(device)
+    hbm_gbs, bf16_tf, peak_kind = load_peaks()
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def flush():
+        flush_buf.fill_(1)
+
+    problems = [Prepared(p, device, mq) for p in synth.config(1)]
+    torch.cuda.synchronize()
+    flops_step = sum(pp.p.flops() for pp in problems)
+    bytes_step = sum(pp.p.algorithmic_bytes() for pp in problems)
+
+    def step(events=None):
+        for i, pp in enumerate(problems):
+            if events is not None:
+                events[i][0].record(stream)
+            pp.run(mq, stream)
+            if events is not None:
+                events[i][1].record(stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush()
+            step()
+    stream.synchronize()
+
+    # ---------------- timed region ----------------
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    step_ev, call_ev = [], []
+    with torch.cuda.stream(stream):
+        for _ in range(args.steps):
+            flush()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            ce = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in problems]
+            a.record(stream)
+            step(ce)
+            b.record(stream)
+            step_ev.append((a, b))
+            call_ev.append(ce)
+    stream.synchronize()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clocks = sampler.stop()
+
+    step_ms = [a.elapsed_time(b) for a, b in step_ev]
+    total_ms = sum(step_ms)
+    kernel_ms = [sum(s.elapsed_time(e) for s, e in ce) for ce in call_ev]
+    if dist is not None:
+        t = torch.tensor([total_ms], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+    ms_per_step = total_ms / args.steps
+
+    # roofline of the dominant kernel (the fused MMA kernel: one launch per call)
+    launch_s = statistics.mean(kernel_ms) * 1e-3
+    achieved_gbs = bytes_step / launch_s / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_gbs, "unit": "GB/s",
+                "frac": achieved_gbs / hbm_gbs, "traffic": None,
+                "peak_kind": f"{peak_kind} copy bandwidth (burst)",
+                "algorithmic_bytes_per_step": bytes_step, "launches_per_step": len(problems)}
+
+    # ---------------- e2e: host buffers through the public API ----------------
+    h2d = sum(pp.x_host.numel() * 2 for pp in problems)
+    d2h = sum(pp.y_host.numel() * 2 for pp in problems)
+    e2e_ms = []
+    with torch.cuda.stream(stream):
+        for it in range(args.warmup + args.steps):
+            flush()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for pp in problems:
+                pp.x.copy_(pp.x_host, non_blocking=True)
+                pp.run(mq, stream)
+                pp.y_host.copy_(pp.y, non_blocking=True)
+            b.record(stream)
+            if it >= args.warmup:
+                e2e_ms.append((a, b))
+    stream.synchronize()
+    e2e_total = sum(a.elapsed_time(b) for a, b in e2e_ms)
+    if dist is not None:
+        t = torch.tensor([e2e_total], device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    e2e = {"value": world * flops_step * args.steps / (e2e_total * 1e-3) / 1e12, "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "mxfp4(e2m1,e8m0)->f32->bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "global_batch": 128 * world, "per_gpu_batch": 128,
+                   "parallelism": f"replicas x{world}", "l2": "flushed (256 MiB write) before every timed step"},
+        "us_per_call": {pp.p.name: 1e3 * statistics.median(ce[i][0].elapsed_time(ce[i][1]) for ce in call_ev)
+                        for i, pp in enumerate(problems)},
+        "roofline": roofline,
+        "e2e": e2e,
+        "gpu_launches": len(problems) * args.steps,
+        "clocks": clocks,
+    }
+
+    if rank == 0:
+        # CPU oracle on the host cores (bounded sample)
+        v, el, cores, sample, _ = cpu_oracle_sample([pp.p for pp in problems], budget_s=12.0, rows=4)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                                "seconds": el}
+        if not args.no_table:
+            line["per_workload"] = workload_table(mq, device, stream, flush, hbm_gbs, args.table_reps)
+        print(json.dumps(line), flush=True)
+
+    for pp in problems:
+        del pp
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def workload_table(mq, device, stream, flush, hbm_gbs, reps):
+    """us/call (median, cold L2), TFLOPS and roofline fraction for every
+    problem of the five workloads, fused and unfused."""
+    rows = []
+    for cfg in range(5):
+        for p in synth.config(cfg):
+            pp = Prepared(p, device, mq)
+            torch.cuda.synchronize()
+            with torch.cuda.stream(stream):
+                us, iqr = time_calls(lambda: pp.run(mq, stream), flush, stream, reps)
+                us_warm, _ = time_calls(lambda: pp.run(mq, stream), flush, stream, reps, cold=False)
+                un = None
+                if p.E == 1:
+                    un, _ = time_calls(lambda: pp.run_unfused(mq, stream), flush, stream, reps)
+            t_roof = max(p.algorithmic_bytes() / (hbm_gbs * 1e9), p.flops() / (FP4_NOMINAL_TFLOPS * 1e12))
+            rows.append({
+                "config": cfg, "name": p.name, "us": us, "iqr_us": iqr, "us_warm_l2": us_warm,
+                "tflops": p.flops() / (us * 1e-6) / 1e12, "gbs": p.algorithmic_bytes() / (us * 1e-6) / 1e9,
+                "roofline_us": t_roof * 1e6, "frac_roofline": t_roof / (us * 1e-6), "unfused_us": un,
+            })
+            del pp
+            torch.cuda.empty_cache()
+    return rows
+
+
+if __name__ == "__main__":
+    main()

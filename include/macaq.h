@@ -96,12 +96,13 @@ int macaq_prepare_weights(const float *W_dev, const float *D_dev, int64_t E, int
 /* Hot path                                                            */
 /* ------------------------------------------------------------------ */
 
-/* Scratch bytes a dense (E = 1, group_list NULL) or grouped call of this shape
- * needs.  The workspace holds split-K partial sums, tile counters and the
- * quantised activations of the quantise-once path.  It must be zero-filled
- * before its first use; every completed call leaves its counters at zero
- * again, so one zero-fill at allocation is enough.  Calls that share a
- * workspace must not run concurrently. */
+/* Scratch bytes a dense (E = 1) or grouped call of this shape needs (0 when
+ * the chosen variant needs none).  The workspace holds split-K tile counters
+ * (its first 4096 bytes) and FP32 partial sums.  The counter region must be
+ * zero-filled before the workspace is first used; every completed call
+ * leaves it at zero again, so one zero-fill at allocation is enough, whatever
+ * shapes later calls have.  Calls that share a workspace must not run
+ * concurrently. */
 size_t macaq_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t E);
 
 /* Dense MACAQ linear (MACAQ page, summary: channel scaling, block-32 BF16

@@ -460,7 +460,7 @@ int oracle_gemm(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const u
 #ifdef _OPENMP
     if (nthreads > 0)
         omp_set_num_threads(nthreads);
-#pragma omp parallel for schedule(static)
+#pragma omp parallel for collapse(2) schedule(static)
 #endif
     for (int64_t m = 0; m < M; m++)
         for (int64_t n = 0; n < N; n++)

@@ -285,7 +285,7 @@ def test_grouped_replicated_banks_equal_dense():
     compare(yg, _oracle_dense_full(pd), "replicated banks vs oracle")
 
 
-@pytest.mark.parametrize("gl,gtype", [([10, 5, 30], 0), ([10, -1, 21], 1), ([10, 10, 10], 1), ([10, 20, 29], 0),
+@pytest.mark.parametrize("gl,gtype", [([10, 5, 30], 0), ([10, -1, 21], 1), ([10, 10, 11], 1), ([10, 20, 29], 0),
                                       ([-3, 20, 30], 0)])
 def test_grouped_invalid_group_list_sets_status_and_leaves_y(gl, gtype):
     p = synth.grouped(30, 3, 256, 64, seed=14, dist="uniform", group_list_type=1)

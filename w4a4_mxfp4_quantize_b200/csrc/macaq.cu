@@ -608,19 +608,24 @@ int pick_bt(int64_t rows_per_group) {
 int pick_splits(int64_t M, int64_t N, int64_t K, int bt, int sms) {
   const int64_t tiles = ((M + bt - 1) / bt) * ((N + 127) / 128);
   const int64_t KT = K / 256;
-  if (tiles >= sms) return 1;
+  if (tiles >= sms || tiles >= 1024) return 1;
   int64_t s = (sms + tiles - 1) / tiles;
   if (s > KT) s = KT;
   if (s > 32) s = 32;
   return static_cast<int>(s < 1 ? 1 : s);
 }
 
+// Split-K workspace: a fixed counter region first (so that its zeros survive
+// calls of other shapes that reuse the same buffer), then the FP32 partials.
+// Split-K is only chosen when the output tiles number fewer than the SMs.
+constexpr size_t kCounterBytes = 4096;  // 1024 counters; pick_splits never splits 1024+ tiles
+
 size_t dense_ws_bytes(int64_t M, int64_t N, int64_t K, int sms) {
   const int bt = pick_bt(M);
   const int s = pick_splits(M, N, K, bt, sms);
   if (s <= 1) return 0;
   const size_t tiles = static_cast<size_t>((M + bt - 1) / bt) * static_cast<size_t>((N + 127) / 128);
-  return tiles * s * 128 * bt * sizeof(float) + ((tiles * sizeof(uint32_t) + 255) / 256) * 256;
+  return kCounterBytes + tiles * s * 128 * bt * sizeof(float);
 }
 
 template <int BT, bool F>
@@ -757,9 +762,8 @@ int macaq_dense_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const u
   p.splits = splits;
   p.status = status;
   if (splits > 1) {
-    const size_t tiles = static_cast<size_t>((M + bt - 1) / bt) * p.NT;
-    p.partial = static_cast<float*>(workspace);
-    p.counters = reinterpret_cast<uint32_t*>(static_cast<uint8_t*>(workspace) + tiles * splits * 128 * bt * 4);
+    p.counters = static_cast<uint32_t*>(workspace);
+    p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
   }
   const int64_t tiles_total = static_cast<int64_t>((M + bt - 1) / bt) * p.NT * splits;
   const int grid = static_cast<int>(tiles_total < sms ? tiles_total : sms);
