@@ -120,7 +120,9 @@ def f32(a, device):
 
 
 class Prepared:
-    """A problem with its weights prepared on the device (untimed, offline)."""
+    """A problem with its weights prepared on the device (untimed, offline) and
+    its output and workspace allocated up front (so calls can be captured in a
+    CUDA graph)."""
 
     def __init__(self, p: synth.Problem, device, mq):
         self.p = p
@@ -133,34 +135,50 @@ class Prepared:
         self.y = torch.empty((p.M, p.N), dtype=torch.bfloat16, device=device)
         self.y_host = torch.empty((p.M, p.N), dtype=torch.bfloat16).pin_memory()
         self.gl = None if p.group_list is None else torch.from_numpy(p.group_list.astype(np.int64)).to(device)
+        nb = mq.workspace_bytes(p.M, p.N, p.K, p.E)
+        self.ws = torch.zeros(nb, dtype=torch.uint8, device=device) if nb else None
+        nu = mq.unfused_workspace_bytes(p.M, p.K) if p.E == 1 else 0
+        self.ws_unfused = torch.zeros(nu, dtype=torch.uint8, device=device) if nu else None
 
-    def run(self, mq, stream, x=None, y=None):
-        x = self.x if x is None else x
-        y = self.y if y is None else y
+    def run(self, mq, stream=None):
         if self.gl is None:
-            mq.dense_mm(x, self.D, self.Wq, self.Ws, self.p.N, out=y, stream=stream)
+            mq.dense_mm(self.x, self.D, self.Wq, self.Ws, self.p.N, out=self.y, stream=stream, ws=self.ws)
         else:
-            mq.grouped_mm(x, self.D, self.Wq, self.Ws, self.gl, self.p.group_list_type, self.p.N, out=y,
-                          stream=stream)
+            mq.grouped_mm(self.x, self.D, self.Wq, self.Ws, self.gl, self.p.group_list_type, self.p.N,
+                          out=self.y, stream=stream, ws=self.ws)
 
-    def run_unfused(self, mq, stream):
-        mq.unfused_dense_mm(self.x, self.D, self.Wq, self.Ws, self.p.N, out=self.y, stream=stream)
+    def run_unfused(self, mq, stream=None):
+        mq.unfused_dense_mm(self.x, self.D, self.Wq, self.Ws, self.p.N, out=self.y, stream=stream,
+                            ws=self.ws_unfused)
 
 
-def time_calls(fn, flush, stream, reps: int, warm: int = 3, cold: bool = True):
-    """Median / IQR of per-call device time (us) with CUDA events on `stream`."""
-    for _ in range(warm):
+def capture(fn, stream):
+    """Capture fn() (library calls on the current stream) into a CUDA graph."""
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        fn()  # warm-up outside capture
+    stream.synchronize()
+    with torch.cuda.graph(g, stream=stream):
         fn()
-    evs = []
-    for _ in range(reps):
-        if cold:
-            flush()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        fn()
-        b.record(stream)
-        evs.append((a, b))
+    return g
+
+
+def time_graph(g, flush, stream, reps: int, warm: int = 3, cold: bool = True):
+    """Median / IQR of the device time (us) of one graph replay, CUDA events on
+    `stream`; the L2 flush (when `cold`) runs before the start event."""
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            g.replay()
+        evs = []
+        for _ in range(reps):
+            if cold:
+                flush()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+            evs.append((a, b))
     stream.synchronize()
     t = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)
     q = np.percentile(t, [25, 50, 75])
@@ -267,18 +285,17 @@ def main():
     flops_step = sum(pp.p.flops() for pp in problems)
     bytes_step = sum(pp.p.algorithmic_bytes() for pp in problems)
 
-    def step(events=None):
-        for i, pp in enumerate(problems):
-            if events is not None:
-                events[i][0].record(stream)
-            pp.run(mq, stream)
-            if events is not None:
-                events[i][1].record(stream)
+    def step():
+        for pp in problems:
+            pp.run(mq)
+
+    step_graph = capture(step, stream)
+    call_graphs = [capture(lambda pp=pp: pp.run(mq), stream) for pp in problems]
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
             flush()
-            step()
+            step_graph.replay()
     stream.synchronize()
 
     # ---------------- timed region ----------------
@@ -288,18 +305,16 @@ def main():
     sampler = ClockSampler(local)
     sampler.start()
     time.sleep(0.3)
-    step_ev, call_ev = [], []
+    step_ev = []
     with torch.cuda.stream(stream):
         for _ in range(args.steps):
             flush()
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
-            ce = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in problems]
             a.record(stream)
-            step(ce)
+            step_graph.replay()
             b.record(stream)
             step_ev.append((a, b))
-            call_ev.append(ce)
     stream.synchronize()
     torch.cuda.synchronize()
     if dist is not None:
@@ -308,7 +323,6 @@ def main():
 
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
     total_ms = sum(step_ms)
-    kernel_ms = [sum(s.elapsed_time(e) for s, e in ce) for ce in call_ev]
     if dist is not None:
         t = torch.tensor([total_ms], device=device)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -316,15 +330,17 @@ def main():
     value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
     ms_per_step = total_ms / args.steps
 
-    # roofline of the dominant kernel (the fused MMA kernel: one launch per call)
-    launch_s = statistics.mean(kernel_ms) * 1e-3
+    # per-call device time (one graph per call, L2 flushed before each): the roofline figure
+    per_call_us = [time_graph(g, flush, stream, max(args.steps, 10))[0] for g in call_graphs]
+    launch_s = sum(per_call_us) * 1e-6
     achieved_gbs = bytes_step / launch_s / 1e9
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_gbs, "unit": "GB/s",
                 "frac": achieved_gbs / hbm_gbs, "traffic": None,
                 "peak_kind": f"{peak_kind} copy bandwidth (burst)",
+                "kernel": "fused_small_kernel (one launch per projection)",
                 "algorithmic_bytes_per_step": bytes_step, "launches_per_step": len(problems)}
 
-    # ---------------- e2e: host buffers through the public API ----------------
+    # ---------------- e2e: host buffers through the public API (eager calls) ----------------
     h2d = sum(pp.x_host.numel() * 2 for pp in problems)
     d2h = sum(pp.y_host.numel() * 2 for pp in problems)
     e2e_ms = []
@@ -348,7 +364,7 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_total = float(t.item())
     e2e = {"value": world * flops_step * args.steps / (e2e_total * 1e-3) / 1e12, "unit": UNIT,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "mode": "eager calls, no graph"}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -356,8 +372,8 @@ def main():
         "vs_baseline": None, "dtype": "mxfp4(e2m1,e8m0)->f32->bf16", "data": "synthetic",
         "config": {"workload": WORKLOAD, "global_batch": 128 * world, "per_gpu_batch": 128,
                    "parallelism": f"replicas x{world}", "l2": "flushed (256 MiB write) before every timed step"},
-        "us_per_call": {pp.p.name: 1e3 * statistics.median(ce[i][0].elapsed_time(ce[i][1]) for ce in call_ev)
-                        for i, pp in enumerate(problems)},
+        "us_per_call": {pp.p.name: us for pp, us in zip(problems, per_call_us)},
+        "timing": "CUDA graph of the step replayed; events on the launching stream",
         "roofline": roofline,
         "e2e": e2e,
         "gpu_launches": len(problems) * args.steps,
@@ -382,25 +398,27 @@ def main():
 
 def workload_table(mq, device, stream, flush, hbm_gbs, reps):
     """us/call (median, cold L2), TFLOPS and roofline fraction for every
-    problem of the five workloads, fused and unfused."""
+    problem of the five workloads, fused and unfused (CUDA graph per call)."""
     rows = []
     for cfg in range(5):
         for p in synth.config(cfg):
             pp = Prepared(p, device, mq)
             torch.cuda.synchronize()
-            with torch.cuda.stream(stream):
-                us, iqr = time_calls(lambda: pp.run(mq, stream), flush, stream, reps)
-                us_warm, _ = time_calls(lambda: pp.run(mq, stream), flush, stream, reps, cold=False)
-                un = None
-                if p.E == 1:
-                    un, _ = time_calls(lambda: pp.run_unfused(mq, stream), flush, stream, reps)
+            g = capture(lambda: pp.run(mq), stream)
+            us, iqr = time_graph(g, flush, stream, reps)
+            us_warm, _ = time_graph(g, flush, stream, reps, cold=False)
+            un = None
+            if p.E == 1:
+                gu = capture(lambda: pp.run_unfused(mq), stream)
+                un, _ = time_graph(gu, flush, stream, reps)
+                del gu
             t_roof = max(p.algorithmic_bytes() / (hbm_gbs * 1e9), p.flops() / (FP4_NOMINAL_TFLOPS * 1e12))
             rows.append({
                 "config": cfg, "name": p.name, "us": us, "iqr_us": iqr, "us_warm_l2": us_warm,
                 "tflops": p.flops() / (us * 1e-6) / 1e12, "gbs": p.algorithmic_bytes() / (us * 1e-6) / 1e9,
                 "roofline_us": t_roof * 1e6, "frac_roofline": t_roof / (us * 1e-6), "unfused_us": un,
             })
-            del pp
+            del g, pp
             torch.cuda.empty_cache()
     return rows
 

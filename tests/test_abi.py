@@ -53,7 +53,7 @@ def test_weight_sizes(L):
     assert L.macaq_weight_code_bytes(1, 1000, 1024) == 0           # N % 16 != 0
     assert L.macaq_weight_code_bytes(1, 1024, 1000) == 0           # K % 256 != 0
     assert L.macaq_weight_code_bytes(1025, 1024, 1024) == 0        # E > 1024
-    assert L.macaq_unfused_workspace_bytes(16, 1024) == 128 * (512 + 32)
+    assert L.macaq_unfused_workspace_bytes(16, 1024) == 4096 + 128 * (512 + 32)
 
 
 P = ctypes.c_void_p

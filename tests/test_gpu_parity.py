@@ -329,3 +329,50 @@ def _check_grouped_sampled(p, y, per_group=24):
         want.append(oracle.gemm_at(qa, sa, qw, sw, np.arange(per_group), idx))
         got.append(y[rows, cols])
     compare(np.concatenate(got), np.concatenate(want), p.name + " sampled exact")
+
+
+# ----------------------------------------------------------------------------
+# Launch-level properties
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,K,N", [(16, 1024, 1024), (128, 3072, 1024), (512, 1024, 384)])
+def test_graph_capture_replays_bit_identical(M, K, N):
+    # calls do no host synchronisation: capture once, replay many times
+    p = synth.dense(M, K, N, seed=21)
+    Wq, Ws = mq.prepare_weights(f32_dev(p.W), f32_dev(p.D))
+    x, D = x_to_dev(p.x), f32_dev(p.D[0])
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    nb = mq.workspace_bytes(M, N, K)
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda") if nb else None
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        mq.dense_mm(x, D, Wq, Ws, N, out=y, ws=ws)
+    s.synchronize()
+    first = y_to_bits(y)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        mq.dense_mm(x, D, Wq, Ws, N, out=y, ws=ws)
+    for _ in range(100):
+        y.fill_(0)
+        g.replay()
+    torch.cuda.synchronize()
+    assert np.array_equal(y_to_bits(y), first)
+    compare(first, _oracle_dense_full(p), "graph")
+
+
+@pytest.mark.parametrize("M", [129, 255, 256, 1000])
+def test_dense_quantise_once_path_ragged(M):
+    p = synth.dense(M, 512, 272, seed=M)
+    compare(_run_dense(p), _oracle_dense_full(p), f"two-kernel M={M}")
+
+
+def test_max_rows_sampled():
+    # the MACAQ page's maximum-row checks go to M = 65,536; one more row for a partial tile
+    for M in (65536, 65537):
+        rng = np.random.default_rng(M)
+        K, N = 256, 128
+        x = synth.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+        W = rng.normal(0, 0.02, (1, N, K)).astype(np.float32)
+        D = synth.make_d(x, W[0])[None, :]
+        p = synth.Problem(x=x, W=W, D=D, M=M, N=N, K=K)
+        _check_large(p, _run_dense(p), n_samples=2000)

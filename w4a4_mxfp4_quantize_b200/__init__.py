@@ -129,14 +129,28 @@ def _require_cuda(*ts):
 
 
 # ---------------------------------------------------------------------------
-# workspace: one zero-filled buffer per (device, stream), grown on demand
+# workspace: scratch for the quantise-once and grouped paths.  Callers may pass
+# their own (e.g. to capture calls in a CUDA graph); otherwise one buffer per
+# (device, stream) is kept and grown on demand.
 # ---------------------------------------------------------------------------
 _ws: dict = {}
 
 
-def workspace(nbytes: int, device: torch.device, stream=None) -> torch.Tensor | None:
+def workspace_bytes(M: int, N: int, K: int, E: int = 1) -> int:
+    return int(lib().macaq_workspace_bytes(M, N, K, E))
+
+
+def unfused_workspace_bytes(M: int, K: int) -> int:
+    return int(lib().macaq_unfused_workspace_bytes(M, K))
+
+
+def workspace(nbytes: int, device: torch.device, stream=None, given: torch.Tensor | None = None):
     if nbytes == 0:
         return None
+    if given is not None:
+        if given.numel() * given.element_size() < nbytes:
+            raise MacaqError(-11, "workspace")
+        return given
     s = stream if stream is not None else torch.cuda.current_stream(device)
     key = (device.index, s.cuda_stream)
     buf = _ws.get(key)
@@ -144,6 +158,10 @@ def workspace(nbytes: int, device: torch.device, stream=None) -> torch.Tensor | 
         buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
         _ws[key] = buf
     return buf
+
+
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
 
 
 # ---------------------------------------------------------------------------
@@ -174,23 +192,24 @@ def prepare_weights(W: torch.Tensor, D: torch.Tensor, stream=None) -> tuple[torc
 
 
 def dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: int,
-             out: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+             out: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None,
+             ws: torch.Tensor | None = None) -> torch.Tensor:
     """y [M, N] bf16 = MACAQ linear of x bf16 [M, K] (fused kernel)."""
     _require_cuda(x, D, Wq, Ws, out, status)
     M, K = x.shape
     y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     L = lib()
     need = int(L.macaq_workspace_bytes(M, N, K, 1))
-    ws = workspace(need, x.device, stream)
+    ws = workspace(need, x.device, stream, ws)
     _check(L.macaq_dense_mm(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(y), M, N, K, _ptr(ws),
-                            0 if ws is None else ws.numel(), _ptr(status), _stream_ptr(stream)),
+                            _nbytes(ws), _ptr(status), _stream_ptr(stream)),
            "macaq_dense_mm")
     return y
 
 
 def grouped_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, group_list: torch.Tensor,
                group_list_type: int, N: int, out: torch.Tensor | None = None,
-               status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+               status: torch.Tensor | None = None, stream=None, ws: torch.Tensor | None = None) -> torch.Tensor:
     """Grouped MACAQ linear; group_list int64 [E] on the device (0 cumsum, 1 counts)."""
     _require_cuda(x, D, Wq, Ws, group_list, out, status)
     M, K = x.shape
@@ -198,9 +217,9 @@ def grouped_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Ten
     y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     L = lib()
     need = int(L.macaq_workspace_bytes(M, N, K, E))
-    ws = workspace(need, x.device, stream)
+    ws = workspace(need, x.device, stream, ws)
     _check(L.macaq_grouped_mm(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(group_list), int(group_list_type), E,
-                              _ptr(y), M, N, K, _ptr(ws), 0 if ws is None else ws.numel(), _ptr(status),
+                              _ptr(y), M, N, K, _ptr(ws), _nbytes(ws), _ptr(status),
                               _stream_ptr(stream)),
            "macaq_grouped_mm")
     return y
@@ -208,16 +227,16 @@ def grouped_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Ten
 
 def unfused_dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: int,
                      out: torch.Tensor | None = None, status: torch.Tensor | None = None,
-                     stream=None) -> torch.Tensor:
+                     stream=None, ws: torch.Tensor | None = None) -> torch.Tensor:
     """Ablation: separate quantisation kernel, then the block-scaled GEMM."""
     _require_cuda(x, D, Wq, Ws, out, status)
     M, K = x.shape
     y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     L = lib()
     need = int(L.macaq_unfused_workspace_bytes(M, K))
-    ws = workspace(need, x.device, stream)
+    ws = workspace(need, x.device, stream, ws)
     _check(L.macaq_unfused_dense_mm(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(y), M, N, K, _ptr(ws),
-                                    0 if ws is None else ws.numel(), _ptr(status), _stream_ptr(stream)),
+                                    _nbytes(ws), _ptr(status), _stream_ptr(stream)),
            "macaq_unfused_dense_mm")
     return y
 

@@ -1,25 +1,38 @@
 // B200 (sm_100a) MACAQ W4A4 MXFP4 linear: kernels and the C ABI of macaq.h.
 //
+// Data layout.  Both MMA operands live in "tile images": 128 rows x 256 K
+// elements, E2M1 codes in 128-byte rows with the 128-byte XOR swizzle the
+// tensor core's K-major shared-memory descriptor expects (16384 bytes), plus a
+// 1024-byte E8M0 scale image in the order tcgen05.cp copies into tensor
+// memory.  Offline weights are stored as such images; activations are either
+// quantised straight into shared memory (fused path) or quantised once into
+// images in an L2-resident workspace (quantise-once path).
+//
+// The MMA is swapped: operand A = 128 output channels of weights (the MMA's M
+// side), operand B = a tile of BT tokens (its N side, 16..128), so the token
+// count maps to the narrow side of tcgen05.mma and D[n][t] sits in TMEM with
+// one output channel per lane.
+//
 // Kernels
-//   prep_weights_kernel   offline: W*D -> FWHT32 -> MX -> tensor-core tile images
-//   quant_act_kernel      activation prologue alone (canonical or tiled output)
-//   mma_kernel<BT,F>      the hot path: persistent, warp-specialised
-//       warp 0      bulk-copy producer (TMA engine) of weight code/scale tiles
-//                   (and of pre-quantised activation tiles when F = false)
-//       warp 1      TMEM owner and single-thread tcgen05.mma kind::mxf4 issuer
-//       warps 2-5   epilogue: tcgen05.ld -> x 2^-5 -> BF16 -> global
-//                   (or FP32 split-K partials + in-kernel ordered reduction)
-//       warps 6-13  (F = true) activation prologue: x/D, FWHT32, BF16, E8M0,
-//                   E2M1 written straight into the swizzled shared-memory
-//                   operand tile and its scale image
-//   The MMA is swapped: the weight tile (128 output channels) is operand A,
-//   the activation tile (BT tokens) is operand B, so small token counts map to
-//   the narrow N side of the instruction (N = BT in {16, 32, 64, 128}).
+//   prep_weights_kernel   offline: W*D -> FWHT32 -> MX -> weight tile images
+//   quant_tiles_kernel    activation prologue over all rows once -> tile images
+//                         (dense rows, or group-padded rows for the grouped form)
+//   group_tables_kernel   grouped: validate group_list, row offsets, tile prefix
+//   gemm_kernel           persistent, warp-specialised tcgen05 kind::mxf4 GEMM
+//                         over tile images; double-buffered TMEM accumulators;
+//                         epilogue staged in shared memory and written with
+//                         bulk stores; chained to the quantiser by
+//                         programmatic dependent launch
+//   fused_small_kernel    small M: one kernel, the activation prologue writes
+//                         the swizzled B tile straight into shared memory;
+//                         split-K across a thread-block cluster, partial sums
+//                         reduced through distributed shared memory
 #include <cuda_runtime.h>
 
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <utility>
 #include <vector>
 
 #include "macaq.h"
@@ -29,13 +42,23 @@
 namespace macaq {
 
 constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // bounded waits give up after 2 s
-constexpr int kStages = 4;
 constexpr int kMaxGroups = 1024;
+constexpr size_t kWsReserved = 4096;  // first bytes of every workspace, left untouched
+constexpr int kSmallM = 128;          // dense calls up to this many rows use the fused kernel
 
 __host__ __device__ constexpr int ceil_div(int64_t a, int64_t b) { return static_cast<int>((a + b - 1) / b); }
 
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ uint16_t bf16_bits(float v) {
+  __nv_bfloat16 h = __float2bfloat16_rn(v);
+  return *reinterpret_cast<uint16_t*>(&h);
+}
+
 // ============================================================================
-// Offline weight preparation
+// Offline weight preparation and test-only kernels
 // ============================================================================
 // CTA = 32 rows x one 256-wide K tile (256 threads, one 32-block each).
 __global__ void __launch_bounds__(256) prep_weights_kernel(const float* __restrict__ W, const float* __restrict__ D,
@@ -46,9 +69,8 @@ __global__ void __launch_bounds__(256) prep_weights_kernel(const float* __restri
   const int t = threadIdx.x >> 3, c = threadIdx.x & 7;
   const int row_global = blockIdx.x * 32 + t;  // over E * NT * 128 padded rows
   const int e = row_global / (NT * kRowsTile);
-  const int rpad = row_global % (NT * kRowsTile);
-  const int nt = rpad / kRowsTile, r = rpad % kRowsTile;
-  const int n = rpad;
+  const int n = row_global % (NT * kRowsTile);
+  const int nt = n / kRowsTile, r = n % kRowsTile;
   const int64_t k0 = static_cast<int64_t>(kt) * kKTile + c * kBlk;
   uint4 codes = make_uint4(0, 0, 0, 0);
   uint32_t scale = 0;
@@ -69,7 +91,7 @@ __global__ void __launch_bounds__(256) prep_weights_kernel(const float* __restri
   Ws[tile * kTileSfBytes + sf_offset(r, c)] = static_cast<uint8_t>(scale);
 }
 
-// Tiled images -> canonical row-major codes/scales (tests only).
+// Tile images -> canonical row-major codes/scales (tests only).
 __global__ void __launch_bounds__(256) export_tiles_kernel(const uint8_t* __restrict__ Tq,
                                                            const uint8_t* __restrict__ Ts,
                                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
@@ -89,15 +111,11 @@ __global__ void __launch_bounds__(256) export_tiles_kernel(const uint8_t* __rest
   scales[row * (K / kBlk) + kt * (kKTile / kBlk) + c] = s;
 }
 
-// ============================================================================
-// Standalone activation quantisation (test path and unfused ablation)
-// ============================================================================
-// CTA = 32 rows x one K tile, 256 threads.  kTiled: write 128-row tile images
-// (rows >= M of the last tile get zero codes); else canonical [M, K/2].
-template <bool kTiled>
-__global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restrict__ x, const float* __restrict__ D,
-                                                        uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                                                        int M, int K, int M_out) {
+// Activation prologue to canonical [M, K/2] codes and [M, K/32] scales (tests).
+__global__ void __launch_bounds__(256) quant_canonical_kernel(const uint16_t* __restrict__ x,
+                                                              const float* __restrict__ D,
+                                                              uint8_t* __restrict__ codes,
+                                                              uint8_t* __restrict__ scales, int M, int K) {
   __shared__ float r[kKTile];
   const int kt = blockIdx.y;
   const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
@@ -105,26 +123,16 @@ __global__ void __launch_bounds__(256) quant_act_kernel(const uint16_t* __restri
   __syncthreads();
   const int t = threadIdx.x >> 3, c = threadIdx.x & 7;
   const int m = blockIdx.x * 32 + t;
-  if (m >= M_out) return;
-  uint4 cv = make_uint4(0, 0, 0, 0);
-  uint32_t sc = 0;
-  if (m < M) {
-    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K + k0 + c * kBlk);
-    uint4 xv[4];
+  if (m >= M) return;
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K + k0 + c * kBlk);
+  uint4 xv[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
-    act_block(xv, r + c * kBlk, cv, sc);
-  }
-  if constexpr (kTiled) {
-    const int KT = K / kKTile;
-    const size_t tile = static_cast<size_t>(m / kRowsTile) * KT + kt;
-    const uint32_t rr = m % kRowsTile;
-    *reinterpret_cast<uint4*>(codes + tile * kTileCodeBytes + code_chunk_offset(rr, c)) = cv;
-    scales[tile * kTileSfBytes + sf_offset(rr, c)] = static_cast<uint8_t>(sc);
-  } else {
-    *reinterpret_cast<uint4*>(codes + static_cast<int64_t>(m) * (K / 2) + (k0 + c * kBlk) / 2) = cv;
-    scales[static_cast<int64_t>(m) * (K / kBlk) + k0 / kBlk + c] = static_cast<uint8_t>(sc);
-  }
+  for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
+  uint4 cv;
+  uint32_t sc;
+  act_block(xv, r + c * kBlk, cv, sc);
+  *reinterpret_cast<uint4*>(codes + static_cast<int64_t>(m) * (K / 2) + (k0 + c * kBlk) / 2) = cv;
+  scales[static_cast<int64_t>(m) * (K / kBlk) + k0 / kBlk + c] = static_cast<uint8_t>(sc);
 }
 
 // MX encoding of raw fp32 blocks (tests the conversion instructions).
@@ -147,57 +155,8 @@ __global__ void mx_encode_kernel(const float* __restrict__ v, uint8_t* __restric
 }
 
 // ============================================================================
-// Hot path: persistent warp-specialised block-scaled MMA kernel
+// Grouped form: device-side group_list validation and tables
 // ============================================================================
-struct MmaParams {
-  const uint8_t* Wq;  // weight tile images [E][NT][KT][16384]
-  const uint8_t* Ws;  // weight scale images [E][NT][KT][1024]
-  const uint16_t* x;  // bf16 [M, K] (fused prologue)
-  const float* D;     // fp32 [E, K]
-  const uint8_t* Aq;  // pre-quantised activation tile images [MT][KT][16384] (unfused)
-  const uint8_t* As;  // their scale images [MT][KT][1024]
-  uint16_t* y;        // bf16 [M, N]
-  const int64_t* group_list;  // device [E] or nullptr (dense)
-  int group_list_type;
-  int E, M, N, K, NT, KT;
-  int splits;          // split-K factor (1 = none)
-  float* partial;      // [tilesMN][splits][128 * BT] fp32 when splits > 1
-  uint32_t* counters;  // [tilesMN] arrival counters, zero between calls
-  int32_t* status;     // optional device status word
-};
-
-template <int BT>
-struct Cfg {
-  static constexpr int kAccStride = BT < 32 ? 32 : BT;            // TMEM columns per accumulator
-  static constexpr int kSfCol = 2 * kAccStride;                   // SFA at kSfCol, SFB at kSfCol + 8
-  static constexpr int kTmemNeed = 2 * kAccStride + 16;
-  static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128
-                                   : kTmemNeed <= 256 ? 256 : 512;
-  static constexpr int kBBytes = BT * 128;                       // activation codes per stage
-  static constexpr int kStageBytes = kTileCodeBytes + kBBytes + 2 * kTileSfBytes;
-  static constexpr int kOffB = kTileCodeBytes;
-  static constexpr int kOffSfa = kTileCodeBytes + kBBytes;
-  static constexpr int kOffSfb = kOffSfa + kTileSfBytes;
-  static constexpr int kBarOff = kStages * kStageBytes;           // barriers and small state
-  static constexpr int kRbufOff = kBarOff + 256;                  // 2 x 256 fp32 reciprocals + 2 flags
-  static constexpr int kScanOff = kRbufOff + 2 * kKTile * 4 + 64; // scan scratch (64 x int64)
-  static constexpr int kGroupOff = kScanOff + 64 * 8;             // group tables
-  static constexpr size_t smem_bytes(int E_grouped) {
-    return 1024 + kGroupOff + (E_grouped > 0 ? static_cast<size_t>(E_grouped + 1) * 12 + 16 : 0);
-  }
-  static_assert(BT % 16 == 0 && BT >= 16 && BT <= 128, "token tile");
-  static_assert(kStageBytes % 1024 == 0, "stage alignment");
-};
-
-constexpr int kProWarps = 8;  // prologue warps (fused)
-constexpr int kEpiWarp0 = 2;
-constexpr int kProWarp0 = 6;
-__host__ __device__ constexpr int mma_threads(bool fused) { return fused ? (kProWarp0 + kProWarps) * 32 : 192; }
-
-struct TileInfo {
-  int g, m0, rows, mg, nt, ks, kt0, kt1, mn;
-};
-
 // Block-wide exclusive scan of one int64 per thread (blockDim.x <= 1024).
 __device__ __forceinline__ int64_t block_excl_scan(int64_t v, int64_t* scratch, int64_t& total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
@@ -210,133 +169,234 @@ __device__ __forceinline__ int64_t block_excl_scan(int64_t v, int64_t* scratch, 
   if (lane == 31) scratch[warp] = inc;
   __syncthreads();
   if (warp == 0) {
-    int64_t w = lane < nw ? scratch[lane] : 0;
+    const int64_t w = lane < nw ? scratch[lane] : 0;
     int64_t wi = w;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int64_t u = __shfl_up_sync(0xffffffffu, wi, o);
       if (lane >= o) wi += u;
     }
-    if (lane < nw) scratch[32 + lane] = wi - w;  // exclusive warp prefix
-    if (lane == nw - 1) scratch[63] = wi;
+    if (lane < nw) scratch[32 + lane] = wi - w;
+    if (lane == nw - 1) scratch[64] = wi;
   }
   __syncthreads();
   const int64_t res = scratch[32 + warp] + inc - v;
-  total = scratch[63];
+  total = scratch[64];
   __syncthreads();
   return res;
 }
 
-// Validates group_list on the device (npu_grouped_matmul rules) and builds
-// row offsets goff[0..E] and m-tile prefix gtp[0..E].  Returns false if invalid.
-template <int BT>
-__device__ bool build_group_tables(const MmaParams& p, int64_t* goff, int* gtp, int64_t* scratch) {
-  const int E = p.E;
-  const int per = (E + blockDim.x - 1) / blockDim.x;
-  const int g0 = threadIdx.x * per, g1 = min(E, g0 + per);
-  int64_t cnt_sum = 0, tile_sum = 0;
+// One CTA of 1024 threads, thread g owns group g.  Rules (npu_grouped_matmul,
+// group_list / group_list_type): type 0 non-negative and non-decreasing
+// cumulative sums, type 1 non-negative counts; the rows must total M.
+// Writes goff[0..E] (row offsets), gtp[0..E] (prefix of 128-row tiles per
+// group) and *valid; on a violation also *status.
+__global__ void __launch_bounds__(1024) group_tables_kernel(const int64_t* __restrict__ gl, int type, int E, int M,
+                                                            int64_t* __restrict__ goff, int* __restrict__ gtp,
+                                                            int* __restrict__ valid, int32_t* status) {
+  __shared__ int64_t scratch[72];
+  const int g = threadIdx.x;
+  int64_t cnt = 0;
   bool bad = false;
-  for (int g = g0; g < g1; ++g) {
-    const int64_t v = p.group_list[g];
-    const int64_t prev = (p.group_list_type == 0 && g > 0) ? p.group_list[g - 1] : 0;
-    const int64_t cnt = p.group_list_type == 0 ? v - prev : v;
-    if (v < 0 || cnt < 0 || cnt > p.M) bad = true;
-    cnt_sum += cnt;
-    tile_sum += (cnt + BT - 1) / BT;
+  if (g < E) {
+    const int64_t v = gl[g];
+    const int64_t prev = (type == 0 && g > 0) ? gl[g - 1] : 0;
+    cnt = type == 0 ? v - prev : v;
+    bad = v < 0 || cnt < 0 || cnt > M;
   }
   bad = __syncthreads_or(bad);
-  if (bad) return false;
-  int64_t rows_total, tiles_total;
-  int64_t row_base = block_excl_scan(cnt_sum, scratch, rows_total);
-  int64_t tile_base = block_excl_scan(tile_sum, scratch, tiles_total);
-  if (rows_total != p.M) return false;  // uniform: every thread reads the same total
-  for (int g = g0; g < g1; ++g) {
-    const int64_t v = p.group_list[g];
-    const int64_t prev = (p.group_list_type == 0 && g > 0) ? p.group_list[g - 1] : 0;
-    const int64_t cnt = p.group_list_type == 0 ? v - prev : v;
-    goff[g] = row_base;
-    gtp[g] = static_cast<int>(tile_base);
-    row_base += cnt;
-    tile_base += (cnt + BT - 1) / BT;
-  }
-  if (threadIdx.x == 0) {
-    goff[E] = rows_total;
-    gtp[E] = static_cast<int>(tiles_total);
-  }
-  __syncthreads();
-  return true;
-}
-
-template <int BT>
-__device__ __forceinline__ TileInfo decode_tile(const MmaParams& p, int idx, const int64_t* goff, const int* gtp) {
-  TileInfo ti;
-  ti.ks = idx % p.splits;
-  const int rest = idx / p.splits;
-  ti.mn = rest;
-  ti.nt = rest % p.NT;
-  ti.mg = rest / p.NT;
-  if (p.group_list == nullptr) {
-    ti.g = 0;
-    ti.m0 = ti.mg * BT;
-    ti.rows = min(BT, p.M - ti.m0);
-  } else {
-    int lo = 0, hi = p.E;  // largest g with gtp[g] <= mg (skips empty groups)
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (gtp[mid] <= ti.mg) lo = mid; else hi = mid;
+  if (!bad) {
+    int64_t rows_total, tiles_total;
+    const int64_t rb = block_excl_scan(cnt, scratch, rows_total);
+    const int64_t tb = block_excl_scan((cnt + kRowsTile - 1) / kRowsTile, scratch, tiles_total);
+    bad = rows_total != M;
+    if (g < E) {
+      goff[g] = rb;
+      gtp[g] = static_cast<int>(tb);
     }
-    ti.g = lo;
-    ti.m0 = static_cast<int>(goff[lo]) + (ti.mg - gtp[lo]) * BT;
-    ti.rows = min(BT, static_cast<int>(goff[lo + 1]) - ti.m0);
+    if (g == 0) {
+      goff[E] = rows_total;
+      gtp[E] = static_cast<int>(tiles_total);
+    }
   }
-  ti.kt0 = static_cast<int>((static_cast<int64_t>(ti.ks) * p.KT) / p.splits);
-  ti.kt1 = static_cast<int>((static_cast<int64_t>(ti.ks + 1) * p.KT) / p.splits);
-  return ti;
+  if (g == 0) {
+    *valid = bad ? 0 : 1;
+    if (bad && status) *status = MACAQ_ERR_GROUP_LIST_INVALID;
+  }
+  pdl_trigger();
 }
 
-__device__ __forceinline__ uint16_t f32_to_bf16_bits(float v) {
-  __nv_bfloat16 h = __float2bfloat16_rn(v);
-  return *reinterpret_cast<uint16_t*>(&h);
+__device__ __forceinline__ int find_group(const int* gtp, int E, int pm) {
+  int lo = 0, hi = E;  // largest g with gtp[g] <= pm; empty groups are skipped
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (gtp[mid] <= pm) lo = mid; else hi = mid;
+  }
+  return lo;
 }
 
-template <int BT, bool kFused>
-__global__ void __launch_bounds__(mma_threads(kFused), 1) mma_kernel(const __grid_constant__ MmaParams p) {
-  using C = Cfg<BT>;
+// ============================================================================
+// Quantise-once: activation prologue over every row into tile images
+// ============================================================================
+// CTA = 32 rows of one 128-row tile x one K tile.  Dense: tile pm holds rows
+// [128 pm, 128 pm + 128).  Grouped: tile pm belongs to the group g with
+// gtp[g] <= pm < gtp[g+1] and holds that group's rows starting at
+// goff[g] + 128 (pm - gtp[g]); rows past the group's end are zero.
+struct QuantParams {
+  const uint16_t* x;
+  const float* D;        // [E, K]
+  uint8_t* Aq;           // [tiles][KT][16384]
+  uint8_t* As;           // [tiles][KT][1024]
+  int M, K, E;
+  const int64_t* goff;   // grouped tables (nullptr: dense)
+  const int* gtp;
+  const int* valid;
+};
+
+__global__ void __launch_bounds__(256) quant_tiles_kernel(const __grid_constant__ QuantParams p) {
+  __shared__ float r[kKTile];
+  pdl_trigger();  // the GEMM may start streaming weights; it waits for our results before reading them
+  const int pm = blockIdx.x >> 2, sub = blockIdx.x & 3;
+  const int kt = blockIdx.y;
+  const int KT = p.K / kKTile;
+  int g = 0, base, rows;
+  if (p.gtp != nullptr) {
+    pdl_wait();  // tables come from the preceding kernel
+    if (*p.valid == 0 || pm >= p.gtp[p.E]) return;
+    g = find_group(p.gtp, p.E, pm);
+    base = static_cast<int>(p.goff[g]) + (pm - p.gtp[g]) * kRowsTile;
+    rows = min(kRowsTile, static_cast<int>(p.goff[g + 1]) - base);
+  } else {
+    base = pm * kRowsTile;
+    rows = min(kRowsTile, p.M - base);
+  }
+  const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
+  r[threadIdx.x] = __frcp_rn(__ldg(p.D + static_cast<int64_t>(g) * p.K + k0 + threadIdx.x));
+  __syncthreads();
+  const int t = sub * 32 + (threadIdx.x >> 3), c = threadIdx.x & 7;
+  uint4 cv = make_uint4(0, 0, 0, 0);
+  uint32_t sc = 0;
+  if (t < rows) {
+    const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(base + t) * p.K + k0 + c * kBlk);
+    uint4 xv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
+    act_block(xv, r + c * kBlk, cv, sc);
+  }
+  const size_t tile = static_cast<size_t>(pm) * KT + kt;
+  *reinterpret_cast<uint4*>(p.Aq + tile * kTileCodeBytes + code_chunk_offset(t, c)) = cv;
+  p.As[tile * kTileSfBytes + sf_offset(t, c)] = static_cast<uint8_t>(sc);
+}
+
+// ============================================================================
+// Persistent GEMM over tile images
+// ============================================================================
+struct GemmParams {
+  const uint8_t* Wq;  // weight images [E][NT][KT]
+  const uint8_t* Ws;
+  const uint8_t* Aq;  // activation images [tiles][KT]
+  const uint8_t* As;
+  uint16_t* y;        // bf16 [M, N]
+  int M, N, K, NT, KT, E, MT;
+  const int64_t* goff;  // grouped tables (nullptr: dense with MT tiles)
+  const int* gtp;
+  const int* valid;
+  int32_t* status;
+  int wait_for_producer;  // dense: 1 when launched as a programmatic dependent of the quantiser
+};
+
+namespace gemm {
+constexpr int kStages = 4;
+constexpr int kThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
+constexpr int kStageBytes = 2 * kTileCodeBytes + 2 * kTileSfBytes;  // 34816
+constexpr int kOffB = kTileCodeBytes;
+constexpr int kOffSfa = 2 * kTileCodeBytes;
+constexpr int kOffSfb = kOffSfa + kTileSfBytes;
+constexpr int kStagingOff = kStages * kStageBytes;  // epilogue staging, 2 x 128 x 128 bf16
+constexpr int kStagingBytes = kRowsTile * kRowsTile * 2;
+constexpr int kBarOff = kStagingOff + 2 * kStagingBytes;
+constexpr int kGroupOff = kBarOff + 256;
+constexpr int kTmemCols = 512;  // accumulators at columns 0 and 128, scales at 256
+constexpr int kSfCol = 256;
+__host__ __device__ constexpr size_t smem_bytes(int E) {
+  return 1024 + kGroupOff + (E > 0 ? static_cast<size_t>(E + 1) * 12 + 16 : 0);
+}
+}  // namespace gemm
+
+struct GemmTile {
+  int g, m0, rows, pm, nt;
+};
+
+__device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int idx, int mtiles, const int64_t* goff,
+                                              const int* gtp) {
+  GemmTile t;
+  t.pm = idx % mtiles;
+  t.nt = idx / mtiles;
+  if (gtp == nullptr) {
+    t.g = 0;
+    t.m0 = t.pm * kRowsTile;
+    t.rows = min(kRowsTile, p.M - t.m0);
+  } else {
+    t.g = find_group(gtp, p.E, t.pm);
+    t.m0 = static_cast<int>(goff[t.g]) + (t.pm - gtp[t.g]) * kRowsTile;
+    t.rows = min(kRowsTile, static_cast<int>(goff[t.g + 1]) - t.m0);
+  }
+  return t;
+}
+
+// Issue the four MMAs of one 256-K stage: D (+)= W-tile x act-tile^T.
+__device__ __forceinline__ void mma_stage(uint32_t a_addr, uint32_t b_addr, uint32_t sfa_addr, uint32_t sfb_addr,
+                                          uint32_t sfa_col, uint32_t sfb_col, uint32_t d_tmem, uint32_t idesc_lo,
+                                          uint32_t idesc_hi, bool first) {
+  tc_cp_32x128b_warpx4(sfa_col, sdesc_sf_block(sfa_addr));
+  tc_cp_32x128b_warpx4(sfa_col + 4, sdesc_sf_block(sfa_addr + 512));
+  tc_cp_32x128b_warpx4(sfb_col, sdesc_sf_block(sfb_addr));
+  tc_cp_32x128b_warpx4(sfb_col + 4, sdesc_sf_block(sfb_addr + 512));
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    // scale bytes 0-1 of each 32-bit TMEM word for the first 64 K, bytes 2-3 for the next
+    const uint32_t sfid = static_cast<uint32_t>(k & 1) * 2u;
+    const uint32_t sfa = (sfa_col + (k >> 1) * 4) | (sfid << 30);
+    const uint32_t sfb = (sfb_col + (k >> 1) * 4) | (sfid << 30);
+    tc_mma_mxf4(d_tmem, sdesc_kmajor_sw128(a_addr + 32 * k), sdesc_kmajor_sw128(b_addr + 32 * k),
+                (k & 1) ? idesc_hi : idesc_lo, sfa, sfb, (!first || k > 0) ? 1u : 0u);
+  }
+}
+
+__global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
+  using namespace gemm;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff);
   uint64_t* empty = full + kStages;
   uint64_t* accf = empty + kStages;
   uint64_t* acce = accf + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acce + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  volatile int* epi_flag = abort_flag + 1;   // epilogue broadcast word
-  volatile int* pro_flag = abort_flag + 2;   // prologue broadcast words [2]
-  float* rbuf = reinterpret_cast<float*>(smem + C::kRbufOff);
-  int64_t* scan_scratch = reinterpret_cast<int64_t*>(smem + C::kScanOff);
-  int64_t* goff = reinterpret_cast<int64_t*>(smem + C::kGroupOff);
-  int* gtp = reinterpret_cast<int*>(goff + (p.E + 1));
-
+  volatile int* epi_flag = abort_flag + 1;
+  int64_t* goff = nullptr;
+  int* gtp = nullptr;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- tile space ----
-  int total_mtiles;
-  if (p.group_list != nullptr) {
-    if (!build_group_tables<BT>(p, goff, gtp, scan_scratch)) {
-      if (blockIdx.x == 0 && threadIdx.x == 0 && p.status) *p.status = MACAQ_ERR_GROUP_LIST_INVALID;
-      return;
+  int mtiles = p.MT;
+  if (p.gtp != nullptr) {
+    pdl_wait();  // tables and activation images come from the preceding kernels
+    if (*p.valid == 0) return;
+    goff = reinterpret_cast<int64_t*>(smem + kGroupOff);
+    gtp = reinterpret_cast<int*>(goff + p.E + 1);
+    for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
+      goff[i] = p.goff[i];
+      gtp[i] = p.gtp[i];
     }
-    total_mtiles = gtp[p.E];
-  } else {
-    total_mtiles = ceil_div(p.M, BT);
+    __syncthreads();
+    mtiles = gtp[p.E];
   }
-  const int total_tiles = total_mtiles * p.NT * p.splits;
-  if (static_cast<int>(blockIdx.x) >= total_tiles) return;
+  const int total = mtiles * p.NT;
+  if (static_cast<int>(blockIdx.x) >= total) return;
 
-  // ---- set-up ----
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], kFused ? 1 + kProWarps : 1);
+      mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -346,14 +406,203 @@ __global__ void __launch_bounds__(mma_threads(kFused), 1) mma_kernel(const __gri
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if constexpr (kFused) {
-    // scale rows >= BT of the activation scale image are never written: zero them once
-    for (int i = threadIdx.x; i < kStages * kTileSfBytes / 16; i += blockDim.x) {
-      const int s = i / (kTileSfBytes / 16), o = i % (kTileSfBytes / 16);
-      *reinterpret_cast<uint4*>(smem + s * C::kStageBytes + C::kOffSfb + o * 16) = make_uint4(0, 0, 0, 0);
-    }
-    fence_proxy_async_smem();
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kTmemCols);
+    tmem_relinquish();
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int my_tiles = (total - static_cast<int>(blockIdx.x) + static_cast<int>(gridDim.x) - 1) /
+                       static_cast<int>(gridDim.x);
+  const int KT = p.KT;
+
+  if (warp == 0) {
+    // ================= producer: bulk copies of weight and activation images =================
+    if (lane == 0) {
+      const int slots = my_tiles * KT;
+      const int pre = min(kStages, slots);
+      auto weights = [&](int j, int stage) {
+        const GemmTile t = gemm_tile(p, blockIdx.x + (j / KT) * gridDim.x, mtiles, goff, gtp);
+        const size_t wt = (static_cast<size_t>(t.g) * p.NT + t.nt) * KT + (j % KT);
+        uint8_t* sb = smem + stage * kStageBytes;
+        bulk_g2s(sb, p.Wq + wt * kTileCodeBytes, kTileCodeBytes, &full[stage]);
+        bulk_g2s(sb + kOffSfa, p.Ws + wt * kTileSfBytes, kTileSfBytes, &full[stage]);
+      };
+      auto acts = [&](int j, int stage) {
+        const GemmTile t = gemm_tile(p, blockIdx.x + (j / KT) * gridDim.x, mtiles, goff, gtp);
+        const size_t at = static_cast<size_t>(t.pm) * KT + (j % KT);
+        uint8_t* sb = smem + stage * kStageBytes;
+        bulk_g2s(sb + kOffB, p.Aq + at * kTileCodeBytes, kTileCodeBytes, &full[stage]);
+        bulk_g2s(sb + kOffSfb, p.As + at * kTileSfBytes, kTileSfBytes, &full[stage]);
+      };
+      // the weights of the first stages do not depend on the quantiser: issue them first
+      for (int j = 0; j < pre; ++j) {
+        mbar_arrive_expect_tx(&full[j], kStageBytes);
+        weights(j, j);
+      }
+      if (p.wait_for_producer) pdl_wait();
+      for (int j = 0; j < pre; ++j) acts(j, j);
+      for (int j = pre; j < slots; ++j) {
+        const int stage = j % kStages;
+        const uint32_t phase = (j / kStages) & 1;
+        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitTimeoutNs)) break;
+        mbar_arrive_expect_tx(&full[stage], kStageBytes);
+        weights(j, stage);
+        acts(j, stage);
+      }
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer =================
+    if (lane == 0) {
+      const uint32_t idesc_lo = idesc_mxf4(128, kRowsTile, 0, 0);
+      const uint32_t idesc_hi = idesc_mxf4(128, kRowsTile, 2, 2);
+      const uint32_t sfa_col = tmem + kSfCol, sfb_col = tmem + kSfCol + 8;
+      int j = 0;
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        const int acc = i & 1;
+        if (!mbar_wait(&acce[acc], ((i >> 1) & 1) ^ 1, abort_flag, kWaitTimeoutNs)) break;
+        tc_fence_after();
+        for (int kt = 0; kt < KT; ++kt, ++j) {
+          const int stage = j % kStages;
+          if (!mbar_wait(&full[stage], (j / kStages) & 1, abort_flag, kWaitTimeoutNs)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t a = smem_u32(smem + stage * kStageBytes);
+          mma_stage(a, a + kOffB, a + kOffSfa, a + kOffSfb, sfa_col, sfb_col, tmem + acc * kRowsTile, idesc_lo,
+                    idesc_hi, kt == 0);
+          tc_commit(&empty[stage]);
+        }
+        if (!ok) break;
+        tc_commit(&accf[acc]);
+      }
+    }
+  } else {
+    // ================= epilogue: TMEM -> BF16 -> staged rows -> bulk stores =================
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int et = threadIdx.x - 64;
+    const int n_local = q * 32 + lane;
+    for (int i = 0; i < my_tiles; ++i) {
+      const int acc = i & 1;
+      const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp);
+      uint8_t* staging = smem + kStagingOff + acc * kStagingBytes;
+      if (et == 0) {
+        bulk_wait_read<1>();  // the stores issued from this staging buffer two tiles ago have read it
+        *epi_flag = mbar_wait(&accf[acc], (i >> 1) & 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
+      }
+      named_bar_sync(1, 128);
+      if (!*epi_flag) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * kRowsTile;
+#pragma unroll 1
+      for (int c0 = 0; c0 < kRowsTile; c0 += 32) {
+        uint32_t r0[16], r1[16];
+        tmem_ld_32x32b_x16(taddr + c0, r0);
+        tmem_ld_32x32b_x16(taddr + c0 + 16, r1);
+        tmem_wait_ld();
+        uint16_t* row = reinterpret_cast<uint16_t*>(staging) + c0 * kRowsTile + n_local;
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj) {
+          row[jj * kRowsTile] = bf16_bits(__uint_as_float(r0[jj]) * 0.03125f);
+          row[(jj + 16) * kRowsTile] = bf16_bits(__uint_as_float(r1[jj]) * 0.03125f);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[acc]);  // accumulator free for the tile after next
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (et == 0) {
+        const int n0 = t.nt * kRowsTile;
+        const uint32_t bytes = static_cast<uint32_t>(min(kRowsTile, p.N - n0)) * 2u;
+        for (int tt = 0; tt < t.rows; ++tt)
+          bulk_s2g(p.y + static_cast<int64_t>(t.m0 + tt) * p.N + n0, staging + tt * kRowsTile * 2, bytes);
+        bulk_commit();
+      }
+    }
+    if (et == 0) bulk_wait_all<0>();
+  }
+
+  if (*abort_flag && threadIdx.x == 0 && p.status) *p.status = MACAQ_ERR_DEVICE_TIMEOUT;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ============================================================================
+// Small M: fused prologue + cluster split-K
+// ============================================================================
+struct FusedParams {
+  const uint8_t* Wq;
+  const uint8_t* Ws;
+  const uint16_t* x;  // bf16 [M, K]
+  const float* D;     // [K]
+  uint16_t* y;
+  int M, N, K, NT, KT, S;  // S = CTAs per cluster = K splits
+  int32_t* status;
+};
+
+namespace fused {
+constexpr int kStages = 4;
+constexpr int kProWarps = 8;
+constexpr int kThreads = (6 + kProWarps) * 32;  // warp 0 producer, 1 MMA, 2-5 epilogue, 6-13 prologue
+template <int BT>
+struct Cfg {
+  static constexpr int kBBytes = BT * 128;
+  static constexpr int kStageBytes = kTileCodeBytes + kBBytes + 2 * kTileSfBytes;
+  static constexpr int kOffB = kTileCodeBytes;
+  static constexpr int kOffSfa = kTileCodeBytes + kBBytes;
+  static constexpr int kOffSfb = kOffSfa + kTileSfBytes;
+  static constexpr int kBarOff = kStages * kStageBytes;
+  static constexpr int kRbufOff = kBarOff + 256;
+  static constexpr int kSmemBytes = 1024 + kRbufOff + 2 * kKTile * 4;
+  static constexpr int kSfCol = BT < 32 ? 32 : BT;
+  static constexpr int kTmemCols = kSfCol + 16 <= 64 ? 64 : kSfCol + 16 <= 128 ? 128 : 256;
+  static_assert(BT * kRowsTile * 4 <= kStages * kStageBytes, "FP32 partials fit in the stage buffers");
+  static_assert(kStageBytes % 1024 == 0, "stage alignment");
+};
+}  // namespace fused
+
+template <int BT>
+__global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const __grid_constant__ FusedParams p) {
+  using C = fused::Cfg<BT>;
+  using fused::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+  uint64_t* empty = full + kStages;
+  uint64_t* accf = empty + kStages;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accf + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* epi_flag = abort_flag + 1;
+  volatile int* pro_flag = abort_flag + 2;  // [2]
+  float* rbuf = reinterpret_cast<float*>(smem + C::kRbufOff);
+  float* part = reinterpret_cast<float*>(smem);  // FP32 partial tile [BT][128], after the mainloop
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int cid = blockIdx.x / p.S;
+  const int nt = cid % p.NT, mt = cid / p.NT;
+  const int m0 = mt * BT, rows = min(BT, p.M - m0);
+  const int kt0 = static_cast<int>(rank) * p.KT / p.S, kt1 = (static_cast<int>(rank) + 1) * p.KT / p.S;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1 + fused::kProWarps);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(&accf[0], 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // scale rows >= BT of the activation scale images are never written: zero them once
+  for (int i = threadIdx.x; i < kStages * kTileSfBytes / 16; i += blockDim.x) {
+    const int s = i / (kTileSfBytes / 16), o = i % (kTileSfBytes / 16);
+    *reinterpret_cast<uint4*>(smem + s * C::kStageBytes + C::kOffSfb + o * 16) = make_uint4(0, 0, 0, 0);
+  }
+  fence_proxy_async_smem();
   if (warp == 1) {
     tmem_alloc(tmem_holder, C::kTmemCols);
     tmem_relinquish();
@@ -364,183 +613,120 @@ __global__ void __launch_bounds__(mma_threads(kFused), 1) mma_kernel(const __gri
   const uint32_t tmem = *tmem_holder;
 
   if (warp == 0) {
-    // ================= bulk-copy producer =================
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int idx = blockIdx.x; idx < total_tiles && ok; idx += gridDim.x) {
-        const TileInfo ti = decode_tile<BT>(p, idx, goff, gtp);
-        for (int kt = ti.kt0; kt < ti.kt1; ++kt) {
-          if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitTimeoutNs)) { ok = false; break; }
-          uint8_t* sb = smem + stage * C::kStageBytes;
-          constexpr uint32_t bytes = kTileCodeBytes + kTileSfBytes + (kFused ? 0 : C::kBBytes + kTileSfBytes);
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          const size_t wt = (static_cast<size_t>(ti.g) * p.NT + ti.nt) * p.KT + kt;
-          bulk_g2s(sb, p.Wq + wt * kTileCodeBytes, kTileCodeBytes, &full[stage]);
-          bulk_g2s(sb + C::kOffSfa, p.Ws + wt * kTileSfBytes, kTileSfBytes, &full[stage]);
-          if constexpr (!kFused) {
-            const size_t at = static_cast<size_t>(ti.mg) * p.KT + kt;
-            bulk_g2s(sb + C::kOffB, p.Aq + at * kTileCodeBytes, C::kBBytes, &full[stage]);
-            bulk_g2s(sb + C::kOffSfb, p.As + at * kTileSfBytes, kTileSfBytes, &full[stage]);
-          }
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
-        }
+    if (lane == 0) {  // ---- producer: weight images ----
+      for (int kt = kt0, j = 0; kt < kt1; ++kt, ++j) {
+        const int stage = j % kStages;
+        if (!mbar_wait(&empty[stage], ((j / kStages) & 1) ^ 1, abort_flag, kWaitTimeoutNs)) break;
+        mbar_arrive_expect_tx(&full[stage], kTileCodeBytes + kTileSfBytes);
+        const size_t wt = static_cast<size_t>(nt) * p.KT + kt;
+        uint8_t* sb = smem + stage * C::kStageBytes;
+        bulk_g2s(sb, p.Wq + wt * kTileCodeBytes, kTileCodeBytes, &full[stage]);
+        bulk_g2s(sb + C::kOffSfa, p.Ws + wt * kTileSfBytes, kTileSfBytes, &full[stage]);
       }
     }
   } else if (warp == 1) {
-    // ================= MMA issuer =================
-    if (lane == 0) {
-      int stage = 0, acc = 0;
-      uint32_t phase = 0, acc_phase = 0;
-      const uint32_t idesc_lo = idesc_mxf4(128, BT, 0, 0);
-      const uint32_t idesc_hi = idesc_mxf4(128, BT, 2, 2);
+    if (lane == 0) {  // ---- MMA issuer ----
+      const uint32_t idesc_lo = idesc_mxf4(128, BT, 0, 0), idesc_hi = idesc_mxf4(128, BT, 2, 2);
       const uint32_t sfa_col = tmem + C::kSfCol, sfb_col = tmem + C::kSfCol + 8;
       bool ok = true;
-      for (int idx = blockIdx.x; idx < total_tiles && ok; idx += gridDim.x) {
-        const TileInfo ti = decode_tile<BT>(p, idx, goff, gtp);
-        if (!mbar_wait(&acce[acc], acc_phase ^ 1, abort_flag, kWaitTimeoutNs)) break;
+      for (int kt = kt0, j = 0; kt < kt1; ++kt, ++j) {
+        const int stage = j % kStages;
+        if (!mbar_wait(&full[stage], (j / kStages) & 1, abort_flag, kWaitTimeoutNs)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem + acc * C::kAccStride;
-        for (int kt = ti.kt0; kt < ti.kt1; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, kWaitTimeoutNs)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + stage * C::kStageBytes);
-          const uint32_t b_addr = a_addr + C::kOffB;
-          const uint32_t sfa_addr = a_addr + C::kOffSfa, sfb_addr = a_addr + C::kOffSfb;
-          tc_cp_32x128b_warpx4(sfa_col, sdesc_sf_block(sfa_addr));
-          tc_cp_32x128b_warpx4(sfa_col + 4, sdesc_sf_block(sfa_addr + 512));
-          tc_cp_32x128b_warpx4(sfb_col, sdesc_sf_block(sfb_addr));
-          tc_cp_32x128b_warpx4(sfb_col + 4, sdesc_sf_block(sfb_addr + 512));
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t sfid = static_cast<uint32_t>(k & 1) * 2u;
-            const uint32_t sfa = (sfa_col + (k >> 1) * 4) | (sfid << 30);
-            const uint32_t sfb = (sfb_col + (k >> 1) * 4) | (sfid << 30);
-            tc_mma_mxf4(d_tmem, sdesc_kmajor_sw128(a_addr + 32 * k), sdesc_kmajor_sw128(b_addr + 32 * k),
-                        (k & 1) ? idesc_hi : idesc_lo, sfa, sfb, (kt > ti.kt0 || k > 0) ? 1u : 0u);
-          }
-          tc_commit(&empty[stage]);
-          if (++stage == kStages) { stage = 0; phase ^= 1; }
-        }
-        if (!ok) break;
-        tc_commit(&accf[acc]);
-        acc ^= 1;
-        if (acc == 0) acc_phase ^= 1;
+        const uint32_t a = smem_u32(smem + stage * C::kStageBytes);
+        mma_stage(a, a + C::kOffB, a + C::kOffSfa, a + C::kOffSfb, sfa_col, sfb_col, tmem, idesc_lo, idesc_hi,
+                  kt == kt0);
+        tc_commit(&empty[stage]);
       }
+      if (ok) tc_commit(&accf[0]);
     }
-  } else if (warp < kEpiWarp0 + 4) {
-    // ================= epilogue =================
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int et = threadIdx.x - kEpiWarp0 * 32;
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int idx = blockIdx.x; idx < total_tiles; idx += gridDim.x) {
-      const TileInfo ti = decode_tile<BT>(p, idx, goff, gtp);
-      if (et == 0) *epi_flag = mbar_wait(&accf[acc], acc_phase, abort_flag, kWaitTimeoutNs) ? 1 : 0;
-      named_bar_sync(1, 128);
-      if (!*epi_flag) break;
+  } else if (warp < 6) {
+    // ---- epilogue: FP32 partial tile to shared memory ----
+    const int q = warp & 3;
+    const int et = threadIdx.x - 64;
+    if (et == 0) *epi_flag = mbar_wait(&accf[0], 0, abort_flag, kWaitTimeoutNs) ? 1 : 0;
+    named_bar_sync(1, 128);
+    if (*epi_flag) {
       tc_fence_after();
-      const int n = ti.nt * kRowsTile + q * 32 + lane;
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * C::kAccStride;
-      if (p.splits == 1) {
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      float* col = part + q * 32 + lane;
 #pragma unroll 1
-        for (int c0 = 0; c0 < BT; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld_32x32b_x16(taddr + c0, r);
-          tmem_wait_ld();
-          if (n < p.N) {
+      for (int c0 = 0; c0 < BT; c0 += 16) {
+        uint32_t r[16];
+        tmem_ld_32x32b_x16(taddr + c0, r);
+        tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int t = c0 + j;
-              if (t < ti.rows)
-                p.y[static_cast<int64_t>(ti.m0 + t) * p.N + n] = f32_to_bf16_bits(__uint_as_float(r[j]) * 0.03125f);
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acce[acc]);
-      } else {
-        float* part = p.partial + (static_cast<size_t>(ti.mn) * p.splits + ti.ks) * (kRowsTile * BT);
-#pragma unroll 1
-        for (int c0 = 0; c0 < BT; c0 += 16) {
-          uint32_t r[16];
-          tmem_ld_32x32b_x16(taddr + c0, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) __stcg(part + (c0 + j) * kRowsTile + q * 32 + lane, __uint_as_float(r[j]));
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&acce[acc]);
-        __threadfence();
-        named_bar_sync(1, 128);
-        if (et == 0) {
-          const uint32_t old = atomicAdd(p.counters + ti.mn, 1u);
-          *epi_flag = (old == static_cast<uint32_t>(p.splits - 1)) ? 2 : 1;
-        }
-        named_bar_sync(1, 128);
-        if (*epi_flag == 2) {
-          __threadfence();
-          const float* base = p.partial + static_cast<size_t>(ti.mn) * p.splits * (kRowsTile * BT);
-#pragma unroll 1
-          for (int t = 0; t < ti.rows; ++t) {
-            float s = 0.0f;
-            for (int kk = 0; kk < p.splits; ++kk)
-              s += __ldcg(base + static_cast<size_t>(kk) * (kRowsTile * BT) + t * kRowsTile + q * 32 + lane);
-            if (n < p.N) p.y[static_cast<int64_t>(ti.m0 + t) * p.N + n] = f32_to_bf16_bits(s * 0.03125f);
-          }
-          if (et == 0) p.counters[ti.mn] = 0u;  // ready for the next call
-        }
+        for (int jj = 0; jj < 16; ++jj) col[(c0 + jj) * kRowsTile] = __uint_as_float(r[jj]);
       }
-      acc ^= 1;
-      if (acc == 0) acc_phase ^= 1;
+    } else {
+      // no accumulator (timeout): contribute zeros; the status word reports the error
+      for (int tt = 0; tt < BT; ++tt) part[tt * kRowsTile + q * 32 + lane] = 0.0f;
     }
-  } else if constexpr (kFused) {
-    // ================= activation prologue =================
-    const int pt = threadIdx.x - kProWarp0 * 32;  // 0 .. 255
-    constexpr int kPT = kProWarps * 32;
-    int stage = 0, it = 0;
-    uint32_t phase = 0;
-    bool ok = true;
-    for (int idx = blockIdx.x; idx < total_tiles && ok; idx += gridDim.x) {
-      const TileInfo ti = decode_tile<BT>(p, idx, goff, gtp);
-      const float* Dg = p.D + static_cast<size_t>(ti.g) * p.K;
-      for (int kt = ti.kt0; kt < ti.kt1; ++kt, ++it) {
-        float* r = rbuf + (it & 1) * kKTile;
-        for (int j = pt; j < kKTile; j += kPT) r[j] = __frcp_rn(__ldg(Dg + kt * kKTile + j));
-        if (pt == 0) pro_flag[it & 1] = mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
-        named_bar_sync(2, kPT);
-        if (!pro_flag[it & 1]) { ok = false; break; }
-        uint8_t* sb = smem + stage * C::kStageBytes;
-        uint8_t* bcode = sb + C::kOffB;
-        uint8_t* bsf = sb + C::kOffSfb;
+  } else {
+    // ---- activation prologue: x/D, FWHT32, BF16, E8M0, E2M1 -> swizzled B tile ----
+    constexpr int kPT = fused::kProWarps * 32;
+    const int pt = threadIdx.x - 6 * 32;
+    for (int kt = kt0, j = 0; kt < kt1; ++kt, ++j) {
+      const int stage = j % kStages;
+      float* r = rbuf + (j & 1) * kKTile;
+      for (int i = pt; i < kKTile; i += kPT) r[i] = __frcp_rn(__ldg(p.D + static_cast<int64_t>(kt) * kKTile + i));
+      if (pt == 0)
+        pro_flag[j & 1] = mbar_wait(&empty[stage], ((j / kStages) & 1) ^ 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
+      named_bar_sync(2, kPT);
+      if (!pro_flag[j & 1]) break;
+      uint8_t* bcode = smem + stage * C::kStageBytes + C::kOffB;
+      uint8_t* bsf = smem + stage * C::kStageBytes + C::kOffSfb;
 #pragma unroll 1
-        for (int task = pt; task < BT * 8; task += kPT) {
-          const int t = task >> 3, c = task & 7;
-          uint4 cv = make_uint4(0, 0, 0, 0);
-          uint32_t sc = 0;
-          if (t < ti.rows) {
-            const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(ti.m0 + t) * p.K +
-                                                              static_cast<int64_t>(kt) * kKTile + c * kBlk);
-            uint4 xv[4];
+      for (int task = pt; task < BT * 8; task += kPT) {
+        const int t = task >> 3, c = task & 7;
+        uint4 cv = make_uint4(0, 0, 0, 0);
+        uint32_t sc = 0;
+        if (t < rows) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m0 + t) * p.K +
+                                                            static_cast<int64_t>(kt) * kKTile + c * kBlk);
+          uint4 xv[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
-            act_block(xv, r + c * kBlk, cv, sc);
-          }
-          *reinterpret_cast<uint4*>(bcode + code_chunk_offset(t, c)) = cv;
-          bsf[sf_offset(t, c)] = static_cast<uint8_t>(sc);
+          for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
+          act_block(xv, r + c * kBlk, cv, sc);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&full[stage]);
-        if (++stage == kStages) { stage = 0; phase ^= 1; }
+        *reinterpret_cast<uint4*>(bcode + code_chunk_offset(t, c)) = cv;
+        bsf[sf_offset(t, c)] = static_cast<uint8_t>(sc);
       }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&full[stage]);
     }
   }
 
-  // ---- tear-down ----
+  // ---- split-K reduction through distributed shared memory ----
+  __syncthreads();
+  cluster_sync_all();  // every CTA of the cluster has its partial tile in shared memory
+  {
+    const int t_lo = static_cast<int>(rank) * BT / p.S, t_hi = (static_cast<int>(rank) + 1) * BT / p.S;
+    const int n0 = nt * kRowsTile;
+    const uint32_t part_addr = smem_u32(part);
+    const int items = (t_hi - t_lo) * 16;
+    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+      const int t = t_lo + it / 16, n = (it % 16) * 8;
+      if (t >= rows || n0 + n >= p.N) continue;
+      float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      const uint32_t off = static_cast<uint32_t>((t * kRowsTile + n) * 4);
+      for (int src = 0; src < p.S; ++src) {  // fixed order: deterministic sums
+        const uint32_t ra = mapa_shared(part_addr + off, static_cast<uint32_t>(src));
+        const float4 a = ld_dsmem_f4(ra), b = ld_dsmem_f4(ra + 16);
+        s[0] += a.x; s[1] += a.y; s[2] += a.z; s[3] += a.w;
+        s[4] += b.x; s[5] += b.y; s[6] += b.z; s[7] += b.w;
+      }
+      uint4 o;
+      o.x = pack_bf16x2(s[0] * 0.03125f, s[1] * 0.03125f);
+      o.y = pack_bf16x2(s[2] * 0.03125f, s[3] * 0.03125f);
+      o.z = pack_bf16x2(s[4] * 0.03125f, s[5] * 0.03125f);
+      o.w = pack_bf16x2(s[6] * 0.03125f, s[7] * 0.03125f);
+      *reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(m0 + t) * p.N + n0 + n) = o;
+    }
+  }
+  cluster_sync_all();  // keep this CTA's shared memory alive until every reader is done
+
   if (*abort_flag && threadIdx.x == 0 && p.status) *p.status = MACAQ_ERR_DEVICE_TIMEOUT;
   tc_fence_before();
   __syncthreads();
@@ -563,6 +749,7 @@ struct DeviceState {
   bool probed = false;
   bool is_sm100 = false;
   int sms = 0;
+  bool attrs_set = false;
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -580,7 +767,22 @@ int current_device(int& dev, int& sms) {
     s.probed = true;
   }
   sms = s.sms;
-  return s.is_sm100 ? MACAQ_OK : MACAQ_ERR_ARCH;
+  if (!s.is_sm100) return MACAQ_ERR_ARCH;
+  if (!s.attrs_set) {  // once per device: opt in to the shared memory the kernels use
+    bool ok = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(gemm::smem_bytes(kMaxGroups))) == cudaSuccess;
+    ok = ok && cudaFuncSetAttribute(fused_small_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    fused::Cfg<16>::kSmemBytes) == cudaSuccess;
+    ok = ok && cudaFuncSetAttribute(fused_small_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    fused::Cfg<32>::kSmemBytes) == cudaSuccess;
+    ok = ok && cudaFuncSetAttribute(fused_small_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    fused::Cfg<64>::kSmemBytes) == cudaSuccess;
+    ok = ok && cudaFuncSetAttribute(fused_small_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    fused::Cfg<128>::kSmemBytes) == cudaSuccess;
+    if (!ok) return MACAQ_ERR_CUDA;
+    s.attrs_set = true;
+  }
+  return MACAQ_OK;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -595,81 +797,149 @@ bool valid_nk(int64_t N, int64_t K) {
 }
 
 int64_t pad128(int64_t n) { return (n + 127) / 128 * 128; }
+size_t align256(size_t n) { return (n + 255) / 256 * 256; }
 
-// Smallest token tile that covers M (the swapped MMA's N dimension).
-int pick_bt(int64_t rows_per_group) {
-  if (rows_per_group <= 16) return 16;
-  if (rows_per_group <= 32) return 32;
-  if (rows_per_group <= 64) return 64;
-  return 128;
-}
-
-// Split-K factor for a dense problem so that the grid covers the SMs.
-int pick_splits(int64_t M, int64_t N, int64_t K, int bt, int sms) {
-  const int64_t tiles = ((M + bt - 1) / bt) * ((N + 127) / 128);
-  const int64_t KT = K / 256;
-  if (tiles >= sms || tiles >= 1024) return 1;
-  int64_t s = (sms + tiles - 1) / tiles;
-  if (s > KT) s = KT;
-  if (s > 32) s = 32;
-  return static_cast<int>(s < 1 ? 1 : s);
-}
-
-// Split-K workspace: a fixed counter region first (so that its zeros survive
-// calls of other shapes that reuse the same buffer), then the FP32 partials.
-// Split-K is only chosen when the output tiles number fewer than the SMs.
-constexpr size_t kCounterBytes = 4096;  // 1024 counters; pick_splits never splits 1024+ tiles
-
-size_t dense_ws_bytes(int64_t M, int64_t N, int64_t K, int sms) {
-  const int bt = pick_bt(M);
-  const int s = pick_splits(M, N, K, bt, sms);
-  if (s <= 1) return 0;
-  const size_t tiles = static_cast<size_t>((M + bt - 1) / bt) * static_cast<size_t>((N + 127) / 128);
-  return kCounterBytes + tiles * s * 128 * bt * sizeof(float);
-}
-
-template <int BT, bool F>
-int launch_mma(const MmaParams& p, int grid, size_t smem, cudaStream_t st, int dev) {
-  static bool attr_set[kMaxDevices] = {};
-  static size_t attr_bytes[kMaxDevices] = {};
-  if (!attr_set[dev] || attr_bytes[dev] < smem) {
-    const size_t want = Cfg<BT>::smem_bytes(kMaxGroups);
-    if (cudaFuncSetAttribute(mma_kernel<BT, F>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(want > smem ? want : smem)) != cudaSuccess)
-      return MACAQ_ERR_CUDA;
-    attr_set[dev] = true;
-    attr_bytes[dev] = want > smem ? want : smem;
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, bool pdl,
+                      int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attrs[2];
+  int n = 0;
+  if (pdl) {
+    attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
   }
-  mma_kernel<BT, F><<<grid, mma_threads(F), smem, st>>>(p);
-  return cudaPeekAtLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
+  if (cluster_x > 1) {
+    attrs[n].id = cudaLaunchAttributeClusterDimension;
+    attrs[n].val.clusterDim.x = cluster_x;
+    attrs[n].val.clusterDim.y = 1;
+    attrs[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  cfg.attrs = attrs;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
-int dispatch_mma(int bt, bool fused, const MmaParams& p, int grid, int E_grouped, cudaStream_t st, int dev) {
-  switch (bt) {
+// ---- small-M fused plan: token tile BT and cluster size S ----
+struct FusedPlan {
+  int bt, S, ctas;
+};
+
+FusedPlan plan_fused(int64_t M, int64_t N, int64_t K, int sms) {
+  const int NT = static_cast<int>(pad128(N) / 128), KT = static_cast<int>(K / 256);
+  int S = 1;
+  for (int s = 8; s >= 1; --s)
+    if (KT % s == 0) {
+      S = s;
+      break;
+    }
+  FusedPlan best{128, S, 0};
+  for (int bt : {16, 32, 64, 128}) {
+    const int ctas = S * NT * ceil_div(M, bt);
+    best = {bt, S, ctas};
+    if (bt >= M || ctas <= sms) break;
+  }
+  return best;
+}
+
+int launch_fused(const FusedParams& p, const FusedPlan& plan, cudaStream_t st) {
+  const dim3 grid(plan.ctas), block(fused::kThreads);
+  cudaError_t e;
+  switch (plan.bt) {
     case 16:
-      return launch_mma<16, true>(p, grid, Cfg<16>::smem_bytes(E_grouped), st, dev);
+      e = launch_ex(fused_small_kernel<16>, grid, block, fused::Cfg<16>::kSmemBytes, st, false, plan.S, p);
+      break;
     case 32:
-      return launch_mma<32, true>(p, grid, Cfg<32>::smem_bytes(E_grouped), st, dev);
+      e = launch_ex(fused_small_kernel<32>, grid, block, fused::Cfg<32>::kSmemBytes, st, false, plan.S, p);
+      break;
     case 64:
-      return launch_mma<64, true>(p, grid, Cfg<64>::smem_bytes(E_grouped), st, dev);
+      e = launch_ex(fused_small_kernel<64>, grid, block, fused::Cfg<64>::kSmemBytes, st, false, plan.S, p);
+      break;
     default:
-      if (fused) return launch_mma<128, true>(p, grid, Cfg<128>::smem_bytes(E_grouped), st, dev);
-      return launch_mma<128, false>(p, grid, Cfg<128>::smem_bytes(E_grouped), st, dev);
+      e = launch_ex(fused_small_kernel<128>, grid, block, fused::Cfg<128>::kSmemBytes, st, false, plan.S, p);
   }
+  return e == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
-int check_dense_args(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y,
-                     int64_t M, int64_t N, int64_t K, int64_t E) {
+// ---- quantise-once workspace layouts ----
+struct DenseWs {
+  size_t act_codes, act_scales, total;
+};
+DenseWs dense_ws(int64_t M, int64_t K) {
+  const size_t tiles = static_cast<size_t>(pad128(M) / 128) * (K / 256);
+  DenseWs w;
+  w.act_codes = kWsReserved;
+  w.act_scales = w.act_codes + tiles * kTileCodeBytes;
+  w.total = w.act_scales + tiles * kTileSfBytes;
+  return w;
+}
+struct GroupedWs {
+  size_t goff, gtp, valid, act_codes, act_scales, total;
+  int tiles_upper;
+};
+GroupedWs grouped_ws(int64_t M, int64_t K, int64_t E) {
+  GroupedWs w;
+  w.tiles_upper = static_cast<int>(pad128(M) / 128 + E);
+  const size_t KT = K / 256;
+  w.goff = kWsReserved;
+  w.gtp = align256(w.goff + (E + 1) * 8);
+  w.valid = align256(w.gtp + (E + 1) * 4);
+  w.act_codes = align256(w.valid + 16);
+  w.act_scales = w.act_codes + static_cast<size_t>(w.tiles_upper) * KT * kTileCodeBytes;
+  w.total = w.act_scales + static_cast<size_t>(w.tiles_upper) * KT * kTileSfBytes;
+  return w;
+}
+
+int check_mm_args(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M,
+                  int64_t N, int64_t K, int64_t E) {
   if (M < 0 || M > INT32_MAX || !valid_nk(N, K)) return MACAQ_ERR_SHAPE;
   if (M == 0) return MACAQ_OK;
   if (!x || !D || !Wq || !Ws || !y) return MACAQ_ERR_NULL;
   if (!aligned16(x) || !aligned16(D) || !aligned16(Wq) || !aligned16(Ws) || !aligned16(y)) return MACAQ_ERR_ALIGN;
   const size_t ybytes = static_cast<size_t>(M) * N * 2;
-  if (overlaps(y, ybytes, x, static_cast<size_t>(M) * K * 2) || overlaps(y, ybytes, D, static_cast<size_t>(E) * K * 4) ||
+  if (overlaps(y, ybytes, x, static_cast<size_t>(M) * K * 2) ||
+      overlaps(y, ybytes, D, static_cast<size_t>(E) * K * 4) ||
       overlaps(y, ybytes, Wq, macaq_weight_code_bytes(E, N, K)) ||
       overlaps(y, ybytes, Ws, macaq_weight_scale_bytes(E, N, K)))
     return MACAQ_ERR_ALIAS;
   return MACAQ_OK;
+}
+
+int check_ws(void* ws, size_t ws_bytes, size_t need, const void* y, size_t ybytes, const void* x, size_t xbytes) {
+  if (!ws || ws_bytes < need || !aligned16(ws)) return MACAQ_ERR_WORKSPACE;
+  if (overlaps(ws, need, y, ybytes) || overlaps(ws, need, x, xbytes)) return MACAQ_ERR_ALIAS;
+  return MACAQ_OK;
+}
+
+// Dense quantise-once: the quantiser over all rows, then the GEMM (launched as
+// a programmatic dependent of the quantiser when `pdl`).
+int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y,
+                         int64_t M, int64_t N, int64_t K, uint8_t* ws, int32_t* status, cudaStream_t st, int sms,
+                         bool pdl) {
+  const DenseWs w = dense_ws(M, K);
+  const int MT = static_cast<int>(pad128(M) / 128), KT = static_cast<int>(K / 256);
+  QuantParams qp{};
+  qp.x = x; qp.D = D; qp.Aq = ws + w.act_codes; qp.As = ws + w.act_scales;
+  qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = 1;
+  quant_tiles_kernel<<<dim3(MT * 4, KT), 256, 0, st>>>(qp);
+  if (cudaPeekAtLastError() != cudaSuccess) return MACAQ_ERR_CUDA;
+  GemmParams gp{};
+  gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.As = qp.As; gp.y = y;
+  gp.M = static_cast<int>(M); gp.N = static_cast<int>(N); gp.K = static_cast<int>(K);
+  gp.NT = static_cast<int>(pad128(N) / 128); gp.KT = KT; gp.E = 1; gp.MT = MT;
+  gp.status = status;
+  gp.wait_for_producer = pdl ? 1 : 0;
+  const int tiles = MT * gp.NT;
+  const int grid = tiles < sms ? tiles : sms;
+  const cudaError_t e =
+      launch_ex(gemm_kernel, dim3(grid), dim3(gemm::kThreads), gemm::smem_bytes(0), st, pdl, 1, gp);
+  return e == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
 }  // namespace
@@ -714,8 +984,9 @@ int macaq_prepare_weights(const float* W, const float* D, int64_t E, int64_t N, 
   if (!W || !D || !Wq || !Ws) return MACAQ_ERR_NULL;
   if (!aligned16(W) || !aligned16(D) || !aligned16(Wq) || !aligned16(Ws)) return MACAQ_ERR_ALIGN;
   const size_t qb = macaq_weight_code_bytes(E, N, K), sb = macaq_weight_scale_bytes(E, N, K);
-  if (overlaps(Wq, qb, W, E * N * K * 4) || overlaps(Wq, qb, D, E * K * 4) || overlaps(Ws, sb, W, E * N * K * 4) ||
-      overlaps(Ws, sb, D, E * K * 4) || overlaps(Wq, qb, Ws, sb))
+  const size_t wb = static_cast<size_t>(E * N * K * 4), db = static_cast<size_t>(E * K * 4);
+  if (overlaps(Wq, qb, W, wb) || overlaps(Wq, qb, D, db) || overlaps(Ws, sb, W, wb) || overlaps(Ws, sb, D, db) ||
+      overlaps(Wq, qb, Ws, sb))
     return MACAQ_ERR_ALIAS;
   int dev, sms;
   int st = current_device(dev, sms);
@@ -736,65 +1007,79 @@ int macaq_prepare_weights(const float* W, const float* D, int64_t E, int64_t N, 
 
 size_t macaq_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t E) {
   if (M <= 0 || !valid_nk(N, K) || E < 1 || E > kMaxGroups) return 0;
-  if (E > 1) return 0;  // grouped calls run the fused kernel without split-K
-  int dev, sms;
-  if (current_device(dev, sms) != MACAQ_OK) sms = 148;
-  return dense_ws_bytes(M, N, K, sms);
+  if (E > 1) return grouped_ws(M, K, E).total;
+  if (M <= kSmallM) return 0;
+  return dense_ws(M, K).total;
 }
 
 int macaq_dense_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M,
                    int64_t N, int64_t K, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
-  int st = check_dense_args(x, D, Wq, Ws, y, M, N, K, 1);
+  int st = check_mm_args(x, D, Wq, Ws, y, M, N, K, 1);
   if (st != MACAQ_OK || M == 0) return st;
+  if (M > kSmallM) {
+    st = check_ws(workspace, workspace_bytes, dense_ws(M, K).total, y, static_cast<size_t>(M) * N * 2, x,
+                  static_cast<size_t>(M) * K * 2);
+    if (st != MACAQ_OK) return st;
+  }
   int dev, sms;
   st = current_device(dev, sms);
   if (st != MACAQ_OK) return st;
-  const int bt = pick_bt(M);
-  const int splits = pick_splits(M, N, K, bt, sms);
-  const size_t need = dense_ws_bytes(M, N, K, sms);
-  if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
-    return MACAQ_ERR_WORKSPACE;
-  MmaParams p{};
-  p.Wq = Wq; p.Ws = Ws; p.x = x; p.D = D; p.y = y;
-  p.group_list = nullptr; p.group_list_type = 0;
-  p.E = 1; p.M = static_cast<int>(M); p.N = static_cast<int>(N); p.K = static_cast<int>(K);
-  p.NT = static_cast<int>(pad128(N) / 128); p.KT = static_cast<int>(K / 256);
-  p.splits = splits;
-  p.status = status;
-  if (splits > 1) {
-    p.counters = static_cast<uint32_t*>(workspace);
-    p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kCounterBytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (M <= kSmallM) {
+    FusedParams p{};
+    p.Wq = Wq; p.Ws = Ws; p.x = x; p.D = D; p.y = y;
+    p.M = static_cast<int>(M); p.N = static_cast<int>(N); p.K = static_cast<int>(K);
+    p.NT = static_cast<int>(pad128(N) / 128); p.KT = static_cast<int>(K / 256);
+    const FusedPlan plan = plan_fused(M, N, K, sms);
+    p.S = plan.S;
+    p.status = status;
+    return launch_fused(p, plan, s);
   }
-  const int64_t tiles_total = static_cast<int64_t>((M + bt - 1) / bt) * p.NT * splits;
-  const int grid = static_cast<int>(tiles_total < sms ? tiles_total : sms);
-  return dispatch_mma(bt, true, p, grid, 0, static_cast<cudaStream_t>(stream), dev);
+  return run_dense_two_kernel(x, D, Wq, Ws, y, M, N, K, static_cast<uint8_t*>(workspace), status, s, sms, true);
 }
 
 int macaq_grouped_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws,
                      const int64_t* group_list, int group_list_type, int64_t E, uint16_t* y, int64_t M, int64_t N,
                      int64_t K, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
-  (void)workspace;
-  (void)workspace_bytes;
   if (E < 1 || E > kMaxGroups) return MACAQ_ERR_TOO_MANY_GROUPS;
   if (group_list_type != 0 && group_list_type != 1) return MACAQ_ERR_GROUP_LIST_TYPE;
-  int st = check_dense_args(x, D, Wq, Ws, y, M, N, K, E);
+  int st = check_mm_args(x, D, Wq, Ws, y, M, N, K, E);
   if (st != MACAQ_OK) return st;
   if (M == 0) return MACAQ_OK;
   if (!group_list) return MACAQ_ERR_NULL;
   if (!aligned16(group_list)) return MACAQ_ERR_ALIGN;
   if (overlaps(y, static_cast<size_t>(M) * N * 2, group_list, E * 8)) return MACAQ_ERR_ALIAS;
+  const GroupedWs w = grouped_ws(M, K, E);
+  st = check_ws(workspace, workspace_bytes, w.total, y, static_cast<size_t>(M) * N * 2, x,
+                static_cast<size_t>(M) * K * 2);
+  if (st != MACAQ_OK) return st;
   int dev, sms;
   st = current_device(dev, sms);
   if (st != MACAQ_OK) return st;
-  const int bt = pick_bt((M + E - 1) / E);
-  MmaParams p{};
-  p.Wq = Wq; p.Ws = Ws; p.x = x; p.D = D; p.y = y;
-  p.group_list = group_list; p.group_list_type = group_list_type;
-  p.E = static_cast<int>(E); p.M = static_cast<int>(M); p.N = static_cast<int>(N); p.K = static_cast<int>(K);
-  p.NT = static_cast<int>(pad128(N) / 128); p.KT = static_cast<int>(K / 256);
-  p.splits = 1;
-  p.status = status;
-  return dispatch_mma(bt, true, p, sms, static_cast<int>(E), static_cast<cudaStream_t>(stream), dev);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  int64_t* goff = reinterpret_cast<int64_t*>(ws + w.goff);
+  int* gtp = reinterpret_cast<int*>(ws + w.gtp);
+  int* valid = reinterpret_cast<int*>(ws + w.valid);
+  group_tables_kernel<<<1, 1024, 0, s>>>(group_list, group_list_type, static_cast<int>(E), static_cast<int>(M),
+                                         goff, gtp, valid, status);
+  if (cudaPeekAtLastError() != cudaSuccess) return MACAQ_ERR_CUDA;
+  const int KT = static_cast<int>(K / 256);
+  QuantParams qp{};
+  qp.x = x; qp.D = D; qp.Aq = ws + w.act_codes; qp.As = ws + w.act_scales;
+  qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = static_cast<int>(E);
+  qp.goff = goff; qp.gtp = gtp; qp.valid = valid;
+  if (launch_ex(quant_tiles_kernel, dim3(w.tiles_upper * 4, KT), dim3(256), 0, s, true, 1, qp) != cudaSuccess)
+    return MACAQ_ERR_CUDA;
+  GemmParams gp{};
+  gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.As = qp.As; gp.y = y;
+  gp.M = static_cast<int>(M); gp.N = static_cast<int>(N); gp.K = static_cast<int>(K);
+  gp.NT = static_cast<int>(pad128(N) / 128); gp.KT = KT; gp.E = static_cast<int>(E);
+  gp.goff = goff; gp.gtp = gtp; gp.valid = valid;
+  gp.status = status;
+  const cudaError_t e = launch_ex(gemm_kernel, dim3(sms), dim3(gemm::kThreads),
+                                  gemm::smem_bytes(static_cast<int>(E)), s, true, 1, gp);
+  return e == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
 int macaq_quantize_activations(const uint16_t* x, const float* D, uint8_t* codes, uint8_t* scales, int64_t M,
@@ -807,8 +1092,8 @@ int macaq_quantize_activations(const uint16_t* x, const float* D, uint8_t* codes
   int st = current_device(dev, sms);
   if (st != MACAQ_OK) return st;
   dim3 grid(static_cast<unsigned>((M + 31) / 32), static_cast<unsigned>(K / 256));
-  quant_act_kernel<false><<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      x, D, codes, scales, static_cast<int>(M), static_cast<int>(K), static_cast<int>(M));
+  quant_canonical_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      x, D, codes, scales, static_cast<int>(M), static_cast<int>(K));
   return cudaPeekAtLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
@@ -844,37 +1129,22 @@ int macaq_mx_encode_blocks(const float* v, uint8_t* codes, uint8_t* scales, int6
 
 size_t macaq_unfused_workspace_bytes(int64_t M, int64_t K) {
   if (M <= 0 || K < 256 || K > 65536 || K % 256) return 0;
-  return static_cast<size_t>(pad128(M)) * (K / 2 + K / 32);
+  return dense_ws(M, K).total;
 }
 
 int macaq_unfused_dense_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y,
                            int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes, int32_t* status,
                            void* stream) {
-  int st = check_dense_args(x, D, Wq, Ws, y, M, N, K, 1);
+  int st = check_mm_args(x, D, Wq, Ws, y, M, N, K, 1);
   if (st != MACAQ_OK || M == 0) return st;
+  st = check_ws(workspace, workspace_bytes, dense_ws(M, K).total, y, static_cast<size_t>(M) * N * 2, x,
+                static_cast<size_t>(M) * K * 2);
+  if (st != MACAQ_OK) return st;
   int dev, sms;
   st = current_device(dev, sms);
   if (st != MACAQ_OK) return st;
-  const size_t need = macaq_unfused_workspace_bytes(M, K);
-  if (!workspace || workspace_bytes < need || !aligned16(workspace)) return MACAQ_ERR_WORKSPACE;
-  if (overlaps(workspace, need, y, static_cast<size_t>(M) * N * 2)) return MACAQ_ERR_ALIAS;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int64_t Mp = pad128(M);
-  uint8_t* Aq = static_cast<uint8_t*>(workspace);
-  uint8_t* As = Aq + static_cast<size_t>(Mp) * (K / 2);
-  dim3 qgrid(static_cast<unsigned>(Mp / 32), static_cast<unsigned>(K / 256));
-  quant_act_kernel<true><<<qgrid, 256, 0, s>>>(x, D, Aq, As, static_cast<int>(M), static_cast<int>(K),
-                                                static_cast<int>(Mp));
-  if (cudaPeekAtLastError() != cudaSuccess) return MACAQ_ERR_CUDA;
-  MmaParams p{};
-  p.Wq = Wq; p.Ws = Ws; p.Aq = Aq; p.As = As; p.D = D; p.y = y;
-  p.E = 1; p.M = static_cast<int>(M); p.N = static_cast<int>(N); p.K = static_cast<int>(K);
-  p.NT = static_cast<int>(pad128(N) / 128); p.KT = static_cast<int>(K / 256);
-  p.splits = 1;
-  p.status = status;
-  const int64_t tiles = (Mp / 128) * p.NT;
-  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-  return dispatch_mma(128, false, p, grid, 0, s, dev);
+  return run_dense_two_kernel(x, D, Wq, Ws, y, M, N, K, static_cast<uint8_t*>(workspace), status,
+                              static_cast<cudaStream_t>(stream), sms, false);
 }
 
 }  // extern "C"
