@@ -116,18 +116,20 @@ __global__ void __launch_bounds__(256) quant_canonical_kernel(const uint16_t* __
                                                               const float* __restrict__ D,
                                                               uint8_t* __restrict__ codes,
                                                               uint8_t* __restrict__ scales, int M, int K) {
-  __shared__ float r[kKTile];
+  __shared__ __align__(16) float r[kKTile];
   const int kt = blockIdx.y;
   const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
-  r[threadIdx.x] = __frcp_rn(__ldg(D + k0 + threadIdx.x));
-  __syncthreads();
   const int t = threadIdx.x >> 3, c = threadIdx.x & 7;
   const int m = blockIdx.x * 32 + t;
-  if (m >= M) return;
-  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K + k0 + c * kBlk);
-  uint4 xv[4];
+  uint4 xv[4] = {};
+  if (m < M) {  // issue the activation loads before the reciprocals
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<int64_t>(m) * K + k0 + c * kBlk);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
+    for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
+  }
+  r[threadIdx.x] = __frcp_rn(__ldg(D + k0 + threadIdx.x));
+  __syncthreads();
+  if (m >= M) return;
   uint4 cv;
   uint32_t sc;
   act_block(xv, r + c * kBlk, cv, sc);
@@ -254,7 +256,7 @@ struct QuantParams {
 };
 
 __global__ void __launch_bounds__(256) quant_tiles_kernel(const __grid_constant__ QuantParams p) {
-  __shared__ float r[kKTile];
+  __shared__ __align__(16) float r[kKTile];
   pdl_trigger();  // the GEMM may start streaming weights; it waits for our results before reading them
   const int pm = blockIdx.x >> 2, sub = blockIdx.x & 3;
   const int kt = blockIdx.y;
@@ -271,18 +273,18 @@ __global__ void __launch_bounds__(256) quant_tiles_kernel(const __grid_constant_
     rows = min(kRowsTile, p.M - base);
   }
   const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
-  r[threadIdx.x] = __frcp_rn(__ldg(p.D + static_cast<int64_t>(g) * p.K + k0 + threadIdx.x));
-  __syncthreads();
   const int t = sub * 32 + (threadIdx.x >> 3), c = threadIdx.x & 7;
-  uint4 cv = make_uint4(0, 0, 0, 0);
-  uint32_t sc = 0;
-  if (t < rows) {
+  uint4 xv[4] = {};
+  if (t < rows) {  // issue the activation loads before the reciprocals
     const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(base + t) * p.K + k0 + c * kBlk);
-    uint4 xv[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
-    act_block(xv, r + c * kBlk, cv, sc);
   }
+  r[threadIdx.x] = __frcp_rn(__ldg(p.D + static_cast<int64_t>(g) * p.K + k0 + threadIdx.x));
+  __syncthreads();
+  uint4 cv = make_uint4(0, 0, 0, 0);
+  uint32_t sc = 0;
+  if (t < rows) act_block(xv, r + c * kBlk, cv, sc);
   const size_t tile = static_cast<size_t>(pm) * KT + kt;
   *reinterpret_cast<uint4*>(p.Aq + tile * kTileCodeBytes + code_chunk_offset(t, c)) = cv;
   p.As[tile * kTileSfBytes + sf_offset(t, c)] = static_cast<uint8_t>(sc);
@@ -487,10 +489,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
       const int acc = i & 1;
       const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp);
       uint8_t* staging = smem + kStagingOff + acc * kStagingBytes;
-      if (et == 0) {
-        bulk_wait_read<1>();  // the stores issued from this staging buffer two tiles ago have read it
-        *epi_flag = mbar_wait(&accf[acc], (i >> 1) & 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
-      }
+      bulk_wait_read<1>();  // my row store from this staging buffer (two tiles ago) has read it
+      if (et == 0) *epi_flag = mbar_wait(&accf[acc], (i >> 1) & 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
       named_bar_sync(1, 128);
       if (!*epi_flag) break;
       tc_fence_after();
@@ -513,15 +513,14 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
       if (lane == 0) mbar_arrive(&acce[acc]);  // accumulator free for the tile after next
       fence_proxy_async_smem();
       named_bar_sync(1, 128);
-      if (et == 0) {
+      if (et < t.rows) {  // thread et writes output row et of the tile (256 contiguous bytes)
         const int n0 = t.nt * kRowsTile;
         const uint32_t bytes = static_cast<uint32_t>(min(kRowsTile, p.N - n0)) * 2u;
-        for (int tt = 0; tt < t.rows; ++tt)
-          bulk_s2g(p.y + static_cast<int64_t>(t.m0 + tt) * p.N + n0, staging + tt * kRowsTile * 2, bytes);
-        bulk_commit();
+        bulk_s2g(p.y + static_cast<int64_t>(t.m0 + et) * p.N + n0, staging + et * kRowsTile * 2, bytes);
       }
+      bulk_commit();
     }
-    if (et == 0) bulk_wait_all<0>();
+    bulk_wait_all<0>();
   }
 
   if (*abort_flag && threadIdx.x == 0 && p.status) *p.status = MACAQ_ERR_DEVICE_TIMEOUT;
@@ -555,13 +554,18 @@ struct Cfg {
   static constexpr int kOffB = kTileCodeBytes;
   static constexpr int kOffSfa = kTileCodeBytes + kBBytes;
   static constexpr int kOffSfb = kOffSfa + kTileSfBytes;
-  static constexpr int kBarOff = kStages * kStageBytes;
+  // receive buffer of the cluster reduction: slot [source rank][owned row][128] FP32;
+  // S ranks own ceil(BT/S) rows each, so at most BT + 7 rows of slots
+  static constexpr int kRecvOff = kStages * kStageBytes;
+  static constexpr int kRecvBytes = (BT + 8) * kRowsTile * 4;
+  static constexpr int kBarOff = kRecvOff + kRecvBytes;
   static constexpr int kRbufOff = kBarOff + 256;
   static constexpr int kSmemBytes = 1024 + kRbufOff + 2 * kKTile * 4;
   static constexpr int kSfCol = BT < 32 ? 32 : BT;
   static constexpr int kTmemCols = kSfCol + 16 <= 64 ? 64 : kSfCol + 16 <= 128 ? 128 : 256;
-  static_assert(BT * kRowsTile * 4 <= kStages * kStageBytes, "FP32 partials fit in the stage buffers");
+  static constexpr int kTasks = (BT * 8 + kProWarps * 32 - 1) / (kProWarps * 32);  // blocks per prologue thread
   static_assert(kStageBytes % 1024 == 0, "stage alignment");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
 }  // namespace fused
 
@@ -579,7 +583,6 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   volatile int* epi_flag = abort_flag + 1;
   volatile int* pro_flag = abort_flag + 2;  // [2]
   float* rbuf = reinterpret_cast<float*>(smem + C::kRbufOff);
-  float* part = reinterpret_cast<float*>(smem);  // FP32 partial tile [BT][128], after the mainloop
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -611,6 +614,10 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // Remote shared memory may only be touched once every CTA of the cluster runs:
+  // arrive now, wait just before the first remote access.
+  cluster_arrive_relaxed();
+  bool cluster_waited = false;
 
   if (warp == 0) {
     if (lane == 0) {  // ---- producer: weight images ----
@@ -641,26 +648,33 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
       if (ok) tc_commit(&accf[0]);
     }
   } else if (warp < 6) {
-    // ---- epilogue: FP32 partial tile to shared memory ----
+    // ---- epilogue: push the FP32 partial tile into the owners' receive slots ----
     const int q = warp & 3;
     const int et = threadIdx.x - 64;
     if (et == 0) *epi_flag = mbar_wait(&accf[0], 0, abort_flag, kWaitTimeoutNs) ? 1 : 0;
     named_bar_sync(1, 128);
+    cluster_wait();
+    cluster_waited = true;
     if (*epi_flag) {
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      float* col = part + q * 32 + lane;
+      const int rpr = (BT + p.S - 1) / p.S;  // rows owned by each rank
+      const int n = q * 32 + lane;
+      const uint32_t recv = smem_u32(smem + C::kRecvOff);
 #pragma unroll 1
       for (int c0 = 0; c0 < BT; c0 += 16) {
         uint32_t r[16];
         tmem_ld_32x32b_x16(taddr + c0, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) col[(c0 + jj) * kRowsTile] = __uint_as_float(r[jj]);
+        for (int jj = 0; jj < 16; ++jj) {
+          const int t = c0 + jj;
+          if (t >= rows) break;
+          const int owner = t / rpr, lr = t - owner * rpr;
+          const uint32_t off = static_cast<uint32_t>(((static_cast<int>(rank) * rpr + lr) * kRowsTile + n) * 4);
+          st_dsmem_f32(mapa_shared(recv + off, static_cast<uint32_t>(owner)), __uint_as_float(r[jj]));
+        }
       }
-    } else {
-      // no accumulator (timeout): contribute zeros; the status word reports the error
-      for (int tt = 0; tt < BT; ++tt) part[tt * kRowsTile + q * 32 + lane] = 0.0f;
     }
   } else {
     // ---- activation prologue: x/D, FWHT32, BF16, E8M0, E2M1 -> swizzled B tile ----
@@ -669,6 +683,20 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
     for (int kt = kt0, j = 0; kt < kt1; ++kt, ++j) {
       const int stage = j % kStages;
       float* r = rbuf + (j & 1) * kKTile;
+      // the activation loads go out first; the reciprocals and the slot wait overlap them
+      uint4 xv[C::kTasks][4];
+#pragma unroll
+      for (int u = 0; u < C::kTasks; ++u) {
+        const int task = pt + u * kPT, t = task >> 3, c = task & 7;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xv[u][i] = make_uint4(0, 0, 0, 0);
+        if (task < BT * 8 && t < rows) {
+          const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m0 + t) * p.K +
+                                                            static_cast<int64_t>(kt) * kKTile + c * kBlk);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) xv[u][i] = __ldg(src + i);
+        }
+      }
       for (int i = pt; i < kKTile; i += kPT) r[i] = __frcp_rn(__ldg(p.D + static_cast<int64_t>(kt) * kKTile + i));
       if (pt == 0)
         pro_flag[j & 1] = mbar_wait(&empty[stage], ((j / kStages) & 1) ^ 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
@@ -676,19 +704,13 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
       if (!pro_flag[j & 1]) break;
       uint8_t* bcode = smem + stage * C::kStageBytes + C::kOffB;
       uint8_t* bsf = smem + stage * C::kStageBytes + C::kOffSfb;
-#pragma unroll 1
-      for (int task = pt; task < BT * 8; task += kPT) {
-        const int t = task >> 3, c = task & 7;
+#pragma unroll
+      for (int u = 0; u < C::kTasks; ++u) {
+        const int task = pt + u * kPT, t = task >> 3, c = task & 7;
+        if (task >= BT * 8) break;
         uint4 cv = make_uint4(0, 0, 0, 0);
         uint32_t sc = 0;
-        if (t < rows) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m0 + t) * p.K +
-                                                            static_cast<int64_t>(kt) * kKTile + c * kBlk);
-          uint4 xv[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
-          act_block(xv, r + c * kBlk, cv, sc);
-        }
+        if (t < rows) act_block(xv[u], r + c * kBlk, cv, sc);
         *reinterpret_cast<uint4*>(bcode + code_chunk_offset(t, c)) = cv;
         bsf[sf_offset(t, c)] = static_cast<uint8_t>(sc);
       }
@@ -698,22 +720,24 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
     }
   }
 
-  // ---- split-K reduction through distributed shared memory ----
+  // ---- split-K reduction: every rank has pushed its partials; sum the owned rows ----
+  __syncwarp();                         // reconverge (warps 0 and 1 ran single-lane roles)
+  if (!cluster_waited) cluster_wait();  // warp-uniform: the epilogue warps waited above
   __syncthreads();
-  cluster_sync_all();  // every CTA of the cluster has its partial tile in shared memory
+  cluster_sync_all();
   {
-    const int t_lo = static_cast<int>(rank) * BT / p.S, t_hi = (static_cast<int>(rank) + 1) * BT / p.S;
+    const int rpr = (BT + p.S - 1) / p.S;
+    const int t_lo = static_cast<int>(rank) * rpr, t_hi = min(BT, t_lo + rpr);
     const int n0 = nt * kRowsTile;
-    const uint32_t part_addr = smem_u32(part);
-    const int items = (t_hi - t_lo) * 16;
+    const float* recv = reinterpret_cast<const float*>(smem + C::kRecvOff);
+    const int items = max(0, t_hi - t_lo) * 16;
     for (int it = threadIdx.x; it < items; it += blockDim.x) {
-      const int t = t_lo + it / 16, n = (it % 16) * 8;
+      const int lr = it / 16, t = t_lo + lr, n = (it % 16) * 8;
       if (t >= rows || n0 + n >= p.N) continue;
       float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      const uint32_t off = static_cast<uint32_t>((t * kRowsTile + n) * 4);
       for (int src = 0; src < p.S; ++src) {  // fixed order: deterministic sums
-        const uint32_t ra = mapa_shared(part_addr + off, static_cast<uint32_t>(src));
-        const float4 a = ld_dsmem_f4(ra), b = ld_dsmem_f4(ra + 16);
+        const float4* v = reinterpret_cast<const float4*>(recv + ((src * rpr + lr) * kRowsTile + n));
+        const float4 a = v[0], b = v[1];
         s[0] += a.x; s[1] += a.y; s[2] += a.z; s[3] += a.w;
         s[4] += b.x; s[5] += b.y; s[6] += b.z; s[7] += b.w;
       }
@@ -725,7 +749,6 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
       *reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(m0 + t) * p.N + n0 + n) = o;
     }
   }
-  cluster_sync_all();  // keep this CTA's shared memory alive until every reader is done
 
   if (*abort_flag && threadIdx.x == 0 && p.status) *p.status = MACAQ_ERR_DEVICE_TIMEOUT;
   tc_fence_before();

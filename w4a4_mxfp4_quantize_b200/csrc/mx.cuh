@@ -38,14 +38,6 @@ __host__ __device__ __forceinline__ uint32_t sf_offset(uint32_t r, uint32_t c) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Round two floats to bf16 (nearest-even) and return them widened back.
-__device__ __forceinline__ void round_pair_bf16(float& a, float& b) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);  // .x = a (low half), .y = b
-  uint32_t w = *reinterpret_cast<uint32_t*>(&h);
-  a = bf16lo(w);
-  b = bf16hi(w);
-}
-
 // Unnormalised Walsh-Hadamard transform of 32 floats; each output of each
 // stage is one IEEE binary32 rounding (no contraction possible: no products).
 __device__ __forceinline__ void fwht32(float (&v)[32]) {
@@ -106,24 +98,100 @@ __device__ __forceinline__ void mx_encode_block(const float (&u)[32], uint4& cod
   scale = c;
 }
 
+// ---- packed two-lane FP32 arithmetic (sm_100 f32x2): each lane one IEEE rounding ----
+__device__ __forceinline__ uint64_t f2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// Round both lanes to bf16 (nearest-even); low lane in the low half.
+__device__ __forceinline__ uint32_t f2_to_bf16x2(uint64_t v) {
+  float lo, hi;
+  f2_split(v, lo, hi);
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) { return f2(bf16lo(w), bf16hi(w)); }
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+// Four lane pairs -> eight E2M1 codes in one word, element 0 in the lowest nibble.
+__device__ __forceinline__ uint32_t e2m1x8_f2(uint64_t a, uint64_t b, uint64_t c, uint64_t d) {
+  float a0, a1, b0, b1, c0, c1, d0, d1;
+  f2_split(a, a0, a1);
+  f2_split(b, b0, b1);
+  f2_split(c, c0, c1);
+  f2_split(d, d0, d1);
+  return e2m1x8(a0, a1, b0, b1, c0, c1, d0, d1);
+}
+
 // Activation block: 32 bf16 values (four 16-byte words) and the 32
-// reciprocals r = RN32(1/D) of their channels.
+// reciprocals r = RN32(1/D) of their channels (r must be 8-byte aligned).
+// Same arithmetic as the scalar definition, two lanes per instruction:
+//   xs = RNE_bf16(RN32(x * r)); FP32 butterfly h = 1, 2, 4, 8, 16;
+//   u = RNE_bf16(.); E8M0 from the block amax of |u|; E2M1 of u * 2^(127-c).
 __device__ __forceinline__ void act_block(const uint4 (&xv)[4], const float* __restrict__ r, uint4& codes,
                                           uint32_t& scale) {
-  float v[32];
   const uint32_t* w = reinterpret_cast<const uint32_t*>(xv);
+  const uint64_t* r2 = reinterpret_cast<const uint64_t*>(r);
+  uint64_t P[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    float a = __fmul_rn(bf16lo(w[j]), r[2 * j]);
-    float b = __fmul_rn(bf16hi(w[j]), r[2 * j + 1]);
-    round_pair_bf16(a, b);
-    v[2 * j] = a;
-    v[2 * j + 1] = b;
+    const uint32_t xs = f2_to_bf16x2(f2_mul(bf16x2_to_f2(w[j]), r2[j]));  // channel scaling, BF16
+    // butterfly stage h = 1 inside the pair: (v0 + v1, v0 - v1)
+    const float v0 = bf16lo(xs), v1 = bf16hi(xs);
+    P[j] = f2(__fadd_rn(v0, v1), __fsub_rn(v0, v1));
   }
-  fwht32(v);
+  // stages h = 2, 4, 8, 16: pairs of pairs (P[i], P[i + h/2])
 #pragma unroll
-  for (int j = 0; j < 16; ++j) round_pair_bf16(v[2 * j], v[2 * j + 1]);
-  mx_encode_block(v, codes, scale);
+  for (int hp = 1; hp < 16; hp <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (i & hp) continue;
+      const uint64_t a = P[i], b = P[i + hp];
+      P[i] = f2_add(a, b);
+      P[i + hp] = f2_sub(a, b);
+    }
+  }
+  uint32_t u[16];
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    u[j] = f2_to_bf16x2(P[j]);
+    m = max_u16x2(m, u[j] & 0x7FFF7FFFu);
+  }
+  const uint32_t amax16 = max(m & 0xFFFFu, m >> 16);
+  const uint32_t c = e8m0_from_amax_bits(amax16 << 16);
+  const float s = __uint_as_float((254u - min(c, 253u)) << 23);
+  const uint64_t s2 = f2(s, s);
+  uint32_t out[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    out[q] = e2m1x8_f2(f2_mul(bf16x2_to_f2(u[4 * q]), s2), f2_mul(bf16x2_to_f2(u[4 * q + 1]), s2),
+                       f2_mul(bf16x2_to_f2(u[4 * q + 2]), s2), f2_mul(bf16x2_to_f2(u[4 * q + 3]), s2));
+  codes = make_uint4(out[0], out[1], out[2], out[3]);
+  scale = c;
 }
 
 // Weight block: 32 fp32 weights and their 32 channel factors D (offline).
