@@ -307,16 +307,18 @@ struct GemmParams {
   int wait_for_producer;  // dense: 1 when launched as a programmatic dependent of the quantiser
 };
 
+// Large M: the MMA is not swapped.  Operand A = a 128-token activation tile,
+// operand B = 128 output channels of weights, D[t][n] in TMEM with one token
+// per lane, so each epilogue thread owns a contiguous run of an output row.
 namespace gemm {
-constexpr int kStages = 4;
+constexpr int kStages = 6;
 constexpr int kThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
 constexpr int kStageBytes = 2 * kTileCodeBytes + 2 * kTileSfBytes;  // 34816
-constexpr int kOffB = kTileCodeBytes;
-constexpr int kOffSfa = 2 * kTileCodeBytes;
-constexpr int kOffSfb = kOffSfa + kTileSfBytes;
-constexpr int kStagingOff = kStages * kStageBytes;  // epilogue staging, 2 x 128 x 128 bf16
-constexpr int kStagingBytes = kRowsTile * kRowsTile * 2;
-constexpr int kBarOff = kStagingOff + 2 * kStagingBytes;
+constexpr int kOffA = 0;                        // activation codes
+constexpr int kOffB = kTileCodeBytes;           // weight codes
+constexpr int kOffSfa = 2 * kTileCodeBytes;     // activation scales
+constexpr int kOffSfb = kOffSfa + kTileSfBytes; // weight scales
+constexpr int kBarOff = kStages * kStageBytes;
 constexpr int kGroupOff = kBarOff + 256;
 constexpr int kTmemCols = 512;  // accumulators at columns 0 and 128, scales at 256
 constexpr int kSfCol = 256;
@@ -429,15 +431,15 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
         const GemmTile t = gemm_tile(p, blockIdx.x + (j / KT) * gridDim.x, mtiles, goff, gtp);
         const size_t wt = (static_cast<size_t>(t.g) * p.NT + t.nt) * KT + (j % KT);
         uint8_t* sb = smem + stage * kStageBytes;
-        bulk_g2s(sb, p.Wq + wt * kTileCodeBytes, kTileCodeBytes, &full[stage]);
-        bulk_g2s(sb + kOffSfa, p.Ws + wt * kTileSfBytes, kTileSfBytes, &full[stage]);
+        bulk_g2s(sb + kOffB, p.Wq + wt * kTileCodeBytes, kTileCodeBytes, &full[stage]);
+        bulk_g2s(sb + kOffSfb, p.Ws + wt * kTileSfBytes, kTileSfBytes, &full[stage]);
       };
       auto acts = [&](int j, int stage) {
         const GemmTile t = gemm_tile(p, blockIdx.x + (j / KT) * gridDim.x, mtiles, goff, gtp);
         const size_t at = static_cast<size_t>(t.pm) * KT + (j % KT);
         uint8_t* sb = smem + stage * kStageBytes;
-        bulk_g2s(sb + kOffB, p.Aq + at * kTileCodeBytes, kTileCodeBytes, &full[stage]);
-        bulk_g2s(sb + kOffSfb, p.As + at * kTileSfBytes, kTileSfBytes, &full[stage]);
+        bulk_g2s(sb + kOffA, p.Aq + at * kTileCodeBytes, kTileCodeBytes, &full[stage]);
+        bulk_g2s(sb + kOffSfa, p.As + at * kTileSfBytes, kTileSfBytes, &full[stage]);
       };
       // the weights of the first stages do not depend on the quantiser: issue them first
       for (int j = 0; j < pre; ++j) {
@@ -472,8 +474,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
           if (!mbar_wait(&full[stage], (j / kStages) & 1, abort_flag, kWaitTimeoutNs)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a = smem_u32(smem + stage * kStageBytes);
-          mma_stage(a, a + kOffB, a + kOffSfa, a + kOffSfb, sfa_col, sfb_col, tmem + acc * kRowsTile, idesc_lo,
-                    idesc_hi, kt == 0);
+          mma_stage(a + kOffA, a + kOffB, a + kOffSfa, a + kOffSfb, sfa_col, sfb_col, tmem + acc * kRowsTile,
+                    idesc_lo, idesc_hi, kt == 0);
           tc_commit(&empty[stage]);
         }
         if (!ok) break;
@@ -481,46 +483,55 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
       }
     }
   } else {
-    // ================= epilogue: TMEM -> BF16 -> staged rows -> bulk stores =================
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // ================= epilogue: TMEM -> x 2^-5 -> BF16 -> 16-byte row stores =================
+    const int q = warp & 3;  // TMEM lane quarter this warp may access: tokens 32q .. 32q+31
     const int et = threadIdx.x - 64;
-    const int n_local = q * 32 + lane;
+    const int tl = q * 32 + lane;  // this thread's token within the tile
     for (int i = 0; i < my_tiles; ++i) {
       const int acc = i & 1;
       const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp);
-      uint8_t* staging = smem + kStagingOff + acc * kStagingBytes;
-      bulk_wait_read<1>();  // my row store from this staging buffer (two tiles ago) has read it
       if (et == 0) *epi_flag = mbar_wait(&accf[acc], (i >> 1) & 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
       named_bar_sync(1, 128);
       if (!*epi_flag) break;
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * kRowsTile;
+      const int n0 = t.nt * kRowsTile;
+      uint16_t* yrow = p.y + static_cast<int64_t>(t.m0 + tl) * p.N + n0;
+      const bool row_ok = tl < t.rows;
 #pragma unroll 1
-      for (int c0 = 0; c0 < kRowsTile; c0 += 32) {
-        uint32_t r0[16], r1[16];
-        tmem_ld_32x32b_x16(taddr + c0, r0);
-        tmem_ld_32x32b_x16(taddr + c0 + 16, r1);
+      for (int c0 = 0; c0 < kRowsTile; c0 += 64) {
+        uint32_t r0[32], r1[32];
+        tmem_ld_32x32b_x32(taddr + c0, r0);
+        tmem_ld_32x32b_x32(taddr + c0 + 32, r1);
         tmem_wait_ld();
-        uint16_t* row = reinterpret_cast<uint16_t*>(staging) + c0 * kRowsTile + n_local;
+        if (c0 + 64 >= kRowsTile) {  // last columns read: the accumulator is free for the tile after next
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acce[acc]);
+        }
+        if (row_ok) {
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          row[jj * kRowsTile] = bf16_bits(__uint_as_float(r0[jj]) * 0.03125f);
-          row[(jj + 16) * kRowsTile] = bf16_bits(__uint_as_float(r1[jj]) * 0.03125f);
+          for (int g = 0; g < 4; ++g) {  // four 8-column groups per 32 columns
+            if (n0 + c0 + 8 * g < p.N) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(r0[8 * g + 0]) * 0.03125f, __uint_as_float(r0[8 * g + 1]) * 0.03125f);
+              o.y = pack_bf16x2(__uint_as_float(r0[8 * g + 2]) * 0.03125f, __uint_as_float(r0[8 * g + 3]) * 0.03125f);
+              o.z = pack_bf16x2(__uint_as_float(r0[8 * g + 4]) * 0.03125f, __uint_as_float(r0[8 * g + 5]) * 0.03125f);
+              o.w = pack_bf16x2(__uint_as_float(r0[8 * g + 6]) * 0.03125f, __uint_as_float(r0[8 * g + 7]) * 0.03125f);
+              *reinterpret_cast<uint4*>(yrow + c0 + 8 * g) = o;
+            }
+            if (n0 + c0 + 32 + 8 * g < p.N) {
+              uint4 o;
+              o.x = pack_bf16x2(__uint_as_float(r1[8 * g + 0]) * 0.03125f, __uint_as_float(r1[8 * g + 1]) * 0.03125f);
+              o.y = pack_bf16x2(__uint_as_float(r1[8 * g + 2]) * 0.03125f, __uint_as_float(r1[8 * g + 3]) * 0.03125f);
+              o.z = pack_bf16x2(__uint_as_float(r1[8 * g + 4]) * 0.03125f, __uint_as_float(r1[8 * g + 5]) * 0.03125f);
+              o.w = pack_bf16x2(__uint_as_float(r1[8 * g + 6]) * 0.03125f, __uint_as_float(r1[8 * g + 7]) * 0.03125f);
+              *reinterpret_cast<uint4*>(yrow + c0 + 32 + 8 * g) = o;
+            }
+          }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acce[acc]);  // accumulator free for the tile after next
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (et < t.rows) {  // thread et writes output row et of the tile (256 contiguous bytes)
-        const int n0 = t.nt * kRowsTile;
-        const uint32_t bytes = static_cast<uint32_t>(min(kRowsTile, p.N - n0)) * 2u;
-        bulk_s2g(p.y + static_cast<int64_t>(t.m0 + et) * p.N + n0, staging + et * kRowsTile * 2, bytes);
-      }
-      bulk_commit();
     }
-    bulk_wait_all<0>();
   }
 
   if (*abort_flag && threadIdx.x == 0 && p.status) *p.status = MACAQ_ERR_DEVICE_TIMEOUT;
@@ -578,11 +589,13 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* empty = full + kStages;
   uint64_t* accf = empty + kStages;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* recv_bar = accf + 1;  // completes when every rank's partial rows for this CTA have landed
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(recv_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* epi_flag = abort_flag + 1;
   volatile int* pro_flag = abort_flag + 2;  // [2]
   float* rbuf = reinterpret_cast<float*>(smem + C::kRbufOff);
+  float* part = reinterpret_cast<float*>(smem);  // local FP32 partial tile [BT][128], after the mainloop
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -590,6 +603,10 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   const int nt = cid % p.NT, mt = cid / p.NT;
   const int m0 = mt * BT, rows = min(BT, p.M - m0);
   const int kt0 = static_cast<int>(rank) * p.KT / p.S, kt1 = (static_cast<int>(rank) + 1) * p.KT / p.S;
+  // split-K ownership: rank o reduces and writes rows [o * rpr, o * rpr + rows_of(o)) of the tile
+  const int rpr = (BT + p.S - 1) / p.S;
+  auto rows_of = [&](int o) { return max(0, min(rpr, BT - o * rpr)); };
+  const bool split = p.S > 1;  // launched as a cluster of S CTAs; S == 1 touches no cluster state
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -597,15 +614,15 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
       mbar_init(&empty[s], 1);
     }
     mbar_init(&accf[0], 1);
+    if (split) {
+      mbar_init(recv_bar, 1);
+      mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(p.S * rows_of(static_cast<int>(rank)) * kRowsTile * 4));
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  // scale rows >= BT of the activation scale images are never written: zero them once
-  for (int i = threadIdx.x; i < kStages * kTileSfBytes / 16; i += blockDim.x) {
-    const int s = i / (kTileSfBytes / 16), o = i % (kTileSfBytes / 16);
-    *reinterpret_cast<uint4*>(smem + s * C::kStageBytes + C::kOffSfb + o * 16) = make_uint4(0, 0, 0, 0);
-  }
-  fence_proxy_async_smem();
+  // (scale rows >= BT of the activation scale image are copied to TMEM but never
+  // read: the MMA's N extent is BT)
   if (warp == 1) {
     tmem_alloc(tmem_holder, C::kTmemCols);
     tmem_relinquish();
@@ -614,9 +631,10 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  // Remote shared memory may only be touched once every CTA of the cluster runs:
-  // arrive now, wait just before the first remote access.
-  cluster_arrive_relaxed();
+  // Remote shared memory may only be touched once every CTA of the cluster runs
+  // (and has initialised its receive barrier): arrive now, wait before the
+  // first remote access.
+  if (split) cluster_arrive_release();
   bool cluster_waited = false;
 
   if (warp == 0) {
@@ -648,43 +666,54 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
       if (ok) tc_commit(&accf[0]);
     }
   } else if (warp < 6) {
-    // ---- epilogue: push the FP32 partial tile into the owners' receive slots ----
+    // ---- epilogue: FP32 partial tile to local shared memory, then one bulk copy per owner ----
     const int q = warp & 3;
     const int et = threadIdx.x - 64;
     if (et == 0) *epi_flag = mbar_wait(&accf[0], 0, abort_flag, kWaitTimeoutNs) ? 1 : 0;
     named_bar_sync(1, 128);
-    cluster_wait();
-    cluster_waited = true;
     if (*epi_flag) {
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      const int rpr = (BT + p.S - 1) / p.S;  // rows owned by each rank
-      const int n = q * 32 + lane;
-      const uint32_t recv = smem_u32(smem + C::kRecvOff);
+      float* col = part + q * 32 + lane;
 #pragma unroll 1
-      for (int c0 = 0; c0 < BT; c0 += 16) {
-        uint32_t r[16];
-        tmem_ld_32x32b_x16(taddr + c0, r);
+      for (int c0 = 0; c0 < BT; c0 += 32) {
+        uint32_t r0[16], r1[16];
+        tmem_ld_32x32b_x16(taddr + c0, r0);
+        if (c0 + 16 < BT) tmem_ld_32x32b_x16(taddr + c0 + 16, r1);
         tmem_wait_ld();
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) {
-          const int t = c0 + jj;
-          if (t >= rows) break;
-          const int owner = t / rpr, lr = t - owner * rpr;
-          const uint32_t off = static_cast<uint32_t>(((static_cast<int>(rank) * rpr + lr) * kRowsTile + n) * 4);
-          st_dsmem_f32(mapa_shared(recv + off, static_cast<uint32_t>(owner)), __uint_as_float(r[jj]));
+        for (int jj = 0; jj < 16; ++jj) col[(c0 + jj) * kRowsTile] = __uint_as_float(r0[jj]);
+        if (c0 + 16 < BT) {
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) col[(c0 + 16 + jj) * kRowsTile] = __uint_as_float(r1[jj]);
         }
+      }
+      fence_proxy_async_smem();
+    }
+    if (split) cluster_wait_acquire();  // every CTA runs and has its receive barrier armed
+    cluster_waited = true;
+    named_bar_sync(1, 128);
+    if (split && *epi_flag && et == 0) {
+      const uint32_t recv = smem_u32(smem + C::kRecvOff);
+      const uint32_t slot = static_cast<uint32_t>(static_cast<int>(rank) * rpr * kRowsTile * 4);
+      for (int o = 0; o < p.S; ++o) {
+        const int n_rows = rows_of(o);
+        if (n_rows == 0) continue;
+        bulk_s2s_cluster(mapa_shared(recv + slot, static_cast<uint32_t>(o)), part + o * rpr * kRowsTile,
+                         static_cast<uint32_t>(n_rows * kRowsTile * 4),
+                         mapa_shared(smem_u32(recv_bar), static_cast<uint32_t>(o)));
       }
     }
   } else {
     // ---- activation prologue: x/D, FWHT32, BF16, E8M0, E2M1 -> swizzled B tile ----
+    // The next K tile's activations and D are loaded while this one is computed
+    // (two register buffers when a thread has at most two blocks per tile).
     constexpr int kPT = fused::kProWarps * 32;
+    constexpr bool kPipe = C::kTasks <= 2;
     const int pt = threadIdx.x - 6 * 32;
-    for (int kt = kt0, j = 0; kt < kt1; ++kt, ++j) {
-      const int stage = j % kStages;
-      float* r = rbuf + (j & 1) * kKTile;
-      // the activation loads go out first; the reciprocals and the slot wait overlap them
-      uint4 xv[C::kTasks][4];
+    uint4 xa[C::kTasks][4], xb[kPipe ? C::kTasks : 1][4];
+    float da = 0.f, db = 0.f;
+    auto load = [&](int kt, uint4 (&xv)[C::kTasks][4], float& d) {
 #pragma unroll
       for (int u = 0; u < C::kTasks; ++u) {
         const int task = pt + u * kPT, t = task >> 3, c = task & 7;
@@ -697,11 +726,17 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
           for (int i = 0; i < 4; ++i) xv[u][i] = __ldg(src + i);
         }
       }
-      for (int i = pt; i < kKTile; i += kPT) r[i] = __frcp_rn(__ldg(p.D + static_cast<int64_t>(kt) * kKTile + i));
+      d = __ldg(p.D + static_cast<int64_t>(kt) * kKTile + pt);  // kPT == kKTile: one channel each
+    };
+    static_assert(kPT == kKTile, "one reciprocal per prologue thread");
+    auto stage_body = [&](int kt, int j, uint4 (&xv)[C::kTasks][4], float d) -> bool {
+      const int stage = j % kStages;
+      float* r = rbuf + (j & 1) * kKTile;
+      r[pt] = __frcp_rn(d);
       if (pt == 0)
         pro_flag[j & 1] = mbar_wait(&empty[stage], ((j / kStages) & 1) ^ 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
       named_bar_sync(2, kPT);
-      if (!pro_flag[j & 1]) break;
+      if (!pro_flag[j & 1]) return false;
       uint8_t* bcode = smem + stage * C::kStageBytes + C::kOffB;
       uint8_t* bsf = smem + stage * C::kStageBytes + C::kOffSfb;
 #pragma unroll
@@ -717,21 +752,36 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[stage]);
+      return true;
+    };
+    if constexpr (kPipe) {
+      if (kt0 < kt1) load(kt0, xa, da);
+      for (int kt = kt0, j = 0; kt < kt1; kt += 2, j += 2) {
+        if (kt + 1 < kt1) load(kt + 1, xb, db);
+        if (!stage_body(kt, j, xa, da)) break;
+        if (kt + 1 >= kt1) break;
+        if (kt + 2 < kt1) load(kt + 2, xa, da);
+        if (!stage_body(kt + 1, j + 1, xb, db)) break;
+      }
+    } else {
+      for (int kt = kt0, j = 0; kt < kt1; ++kt, ++j) {
+        load(kt, xa, da);
+        if (!stage_body(kt, j, xa, da)) break;
+      }
     }
   }
 
-  // ---- split-K reduction: every rank has pushed its partials; sum the owned rows ----
-  __syncwarp();                         // reconverge (warps 0 and 1 ran single-lane roles)
-  if (!cluster_waited) cluster_wait();  // warp-uniform: the epilogue warps waited above
+  // ---- split-K reduction: wait for every rank's rows of this CTA, sum in rank order ----
+  __syncwarp();                                          // reconverge (warps 0 and 1 ran single-lane roles)
+  if (split && !cluster_waited) cluster_wait_acquire();  // warp-uniform: the epilogue warps waited above
+  if (split && threadIdx.x == 0) *epi_flag = mbar_wait(recv_bar, 0, abort_flag, kWaitTimeoutNs) ? 1 : 0;
   __syncthreads();
-  cluster_sync_all();
-  {
-    const int rpr = (BT + p.S - 1) / p.S;
-    const int t_lo = static_cast<int>(rank) * rpr, t_hi = min(BT, t_lo + rpr);
+  if (*epi_flag) {
+    const int t_lo = static_cast<int>(rank) * rpr, n_rows = rows_of(static_cast<int>(rank));
     const int n0 = nt * kRowsTile;
-    const float* recv = reinterpret_cast<const float*>(smem + C::kRecvOff);
-    const int items = max(0, t_hi - t_lo) * 16;
-    for (int it = threadIdx.x; it < items; it += blockDim.x) {
+    // without a split the local partial tile is the whole sum
+    const float* recv = split ? reinterpret_cast<const float*>(smem + C::kRecvOff) : part;
+    for (int it = threadIdx.x; it < n_rows * 16; it += blockDim.x) {
       const int lr = it / 16, t = t_lo + lr, n = (it % 16) * 8;
       if (t >= rows || n0 + n >= p.N) continue;
       float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -748,6 +798,13 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
       o.w = pack_bf16x2(s[6] * 0.03125f, s[7] * 0.03125f);
       *reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(m0 + t) * p.N + n0 + n) = o;
     }
+  }
+  // no CTA may leave while a copy it sent can still be reading its shared memory:
+  // every rank arrives only after its own receive barrier completed
+  if (split) {
+    __syncwarp();
+    cluster_arrive_release();
+    cluster_wait_acquire();
   }
 
   if (*abort_flag && threadIdx.x == 0 && p.status) *p.status = MACAQ_ERR_DEVICE_TIMEOUT;
@@ -854,19 +911,67 @@ struct FusedPlan {
   int bt, S, ctas;
 };
 
-FusedPlan plan_fused(int64_t M, int64_t N, int64_t K, int sms) {
-  const int NT = static_cast<int>(pad128(N) / 128), KT = static_cast<int>(K / 256);
-  int S = 1;
-  for (int s = 8; s >= 1; --s)
-    if (KT % s == 0) {
-      S = s;
-      break;
+template <int BT>
+int max_active_clusters(int S) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(S);
+  cfg.blockDim = dim3(fused::kThreads);
+  cfg.dynamicSmemBytes = fused::Cfg<BT>::kSmemBytes;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = S;
+  attr.val.clusterDim.y = 1;
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, fused_small_kernel<BT>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+// Co-resident clusters per (BT, S), measured once per device.
+int active_clusters(int dev, int bt_index, int S) {
+  static int cache[kMaxDevices][4][9] = {};
+  int& v = cache[dev][bt_index][S];
+  if (v == 0) {
+    switch (bt_index) {
+      case 0: v = max_active_clusters<16>(S); break;
+      case 1: v = max_active_clusters<32>(S); break;
+      case 2: v = max_active_clusters<64>(S); break;
+      default: v = max_active_clusters<128>(S);
     }
-  FusedPlan best{128, S, 0};
-  for (int bt : {16, 32, 64, 128}) {
-    const int ctas = S * NT * ceil_div(M, bt);
-    best = {bt, S, ctas};
-    if (bt >= M || ctas <= sms) break;
+    if (v <= 0) v = -1;  // query failed: treat as one cluster per wave
+  }
+  return v > 0 ? v : 1;
+}
+
+// Choose the token tile BT and the K split S (a divisor of K/256, at most 8
+// CTAs per cluster) that minimise (fixed latency of a wave + prologue work of
+// one CTA) x the number of waves the clusters need.  Units: one row x one
+// 256-wide K tile of prologue work; a wave's fixed latency (launch, set-up,
+// first loads, reduction) is worth about 300 of them.
+FusedPlan plan_fused(int dev, int64_t M, int64_t N, int64_t K) {
+  const int NT = static_cast<int>(pad128(N) / 128), KT = static_cast<int>(K / 256);
+  const int bts[4] = {16, 32, 64, 128};
+  FusedPlan best{128, 1, 0};
+  double best_cost = 1e30;
+  for (int bi = 0; bi < 4; ++bi) {
+    const int bt = bts[bi];
+    if (bi > 0 && bts[bi - 1] >= M) break;  // a larger tile than M only adds empty rows
+    const int clusters = NT * ceil_div(M, bt);
+    for (int S = 1; S <= 8 && S <= KT; ++S) {
+      if (KT % S) continue;
+      const int waves = ceil_div(clusters, active_clusters(dev, bi, S));
+      const double cost = static_cast<double>(waves) * (300.0 + static_cast<double>(M < bt ? M : bt) * (KT / S)) +
+                          0.25 * S;  // small bias against needless splitting
+      if (cost < best_cost) {
+        best_cost = cost;
+        best = {bt, S, clusters * S};
+      }
+    }
   }
   return best;
 }
@@ -1053,7 +1158,7 @@ int macaq_dense_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const u
     p.Wq = Wq; p.Ws = Ws; p.x = x; p.D = D; p.y = y;
     p.M = static_cast<int>(M); p.N = static_cast<int>(N); p.K = static_cast<int>(K);
     p.NT = static_cast<int>(pad128(N) / 128); p.KT = static_cast<int>(K / 256);
-    const FusedPlan plan = plan_fused(M, N, K, sms);
+    const FusedPlan plan = plan_fused(dev, M, N, K);
     p.S = plan.S;
     p.status = status;
     return launch_fused(p, plan, s);
