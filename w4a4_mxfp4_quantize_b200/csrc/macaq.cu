@@ -311,14 +311,16 @@ struct GemmParams {
 // operand B = 128 output channels of weights, D[t][n] in TMEM with one token
 // per lane, so each epilogue thread owns a contiguous run of an output row.
 namespace gemm {
-constexpr int kStages = 6;
+constexpr int kStages = 5;
 constexpr int kThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
 constexpr int kStageBytes = 2 * kTileCodeBytes + 2 * kTileSfBytes;  // 34816
 constexpr int kOffA = 0;                        // activation codes
 constexpr int kOffB = kTileCodeBytes;           // weight codes
 constexpr int kOffSfa = 2 * kTileCodeBytes;     // activation scales
 constexpr int kOffSfb = kOffSfa + kTileSfBytes; // weight scales
-constexpr int kBarOff = kStages * kStageBytes;
+constexpr int kStagingOff = kStages * kStageBytes;  // BF16 output tile, 128 rows x 256 bytes, swizzled
+constexpr int kStagingBytes = kRowsTile * kRowsTile * 2;
+constexpr int kBarOff = kStagingOff + kStagingBytes;
 constexpr int kGroupOff = kBarOff + 256;
 constexpr int kTmemCols = 512;  // accumulators at columns 0 and 128, scales at 256
 constexpr int kSfCol = 256;
@@ -483,52 +485,55 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
       }
     }
   } else {
-    // ================= epilogue: TMEM -> x 2^-5 -> BF16 -> 16-byte row stores =================
-    const int q = warp & 3;  // TMEM lane quarter this warp may access: tokens 32q .. 32q+31
+    // ================= epilogue: TMEM -> x 2^-5 -> BF16 -> staged tile -> coalesced rows =================
+    // Thread (q, lane) owns token row 32q + lane of the accumulator.  Rows are
+    // staged in shared memory with their 16-byte chunks XOR-swizzled by the row
+    // index (conflict-free row writes and row-run reads), then written out two
+    // full 256-byte rows per warp instruction.
+    const int q = warp & 3;
     const int et = threadIdx.x - 64;
-    const int tl = q * 32 + lane;  // this thread's token within the tile
+    const int tl = q * 32 + lane;
+    uint8_t* staging = smem + kStagingOff;
     for (int i = 0; i < my_tiles; ++i) {
       const int acc = i & 1;
       const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp);
       if (et == 0) *epi_flag = mbar_wait(&accf[acc], (i >> 1) & 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
-      named_bar_sync(1, 128);
+      named_bar_sync(1, 128);  // also: every thread has finished reading the previous tile's staging
       if (!*epi_flag) break;
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * kRowsTile;
-      const int n0 = t.nt * kRowsTile;
-      uint16_t* yrow = p.y + static_cast<int64_t>(t.m0 + tl) * p.N + n0;
-      const bool row_ok = tl < t.rows;
+      uint8_t* srow = staging + tl * (kRowsTile * 2);
 #pragma unroll 1
       for (int c0 = 0; c0 < kRowsTile; c0 += 64) {
         uint32_t r0[32], r1[32];
         tmem_ld_32x32b_x32(taddr + c0, r0);
         tmem_ld_32x32b_x32(taddr + c0 + 32, r1);
         tmem_wait_ld();
-        if (c0 + 64 >= kRowsTile) {  // last columns read: the accumulator is free for the tile after next
+        if (c0 + 64 >= kRowsTile) {  // all columns read: the accumulator is free for the tile after next
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acce[acc]);
         }
-        if (row_ok) {
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {  // four 8-column groups per 32 columns
-            if (n0 + c0 + 8 * g < p.N) {
-              uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(r0[8 * g + 0]) * 0.03125f, __uint_as_float(r0[8 * g + 1]) * 0.03125f);
-              o.y = pack_bf16x2(__uint_as_float(r0[8 * g + 2]) * 0.03125f, __uint_as_float(r0[8 * g + 3]) * 0.03125f);
-              o.z = pack_bf16x2(__uint_as_float(r0[8 * g + 4]) * 0.03125f, __uint_as_float(r0[8 * g + 5]) * 0.03125f);
-              o.w = pack_bf16x2(__uint_as_float(r0[8 * g + 6]) * 0.03125f, __uint_as_float(r0[8 * g + 7]) * 0.03125f);
-              *reinterpret_cast<uint4*>(yrow + c0 + 8 * g) = o;
-            }
-            if (n0 + c0 + 32 + 8 * g < p.N) {
-              uint4 o;
-              o.x = pack_bf16x2(__uint_as_float(r1[8 * g + 0]) * 0.03125f, __uint_as_float(r1[8 * g + 1]) * 0.03125f);
-              o.y = pack_bf16x2(__uint_as_float(r1[8 * g + 2]) * 0.03125f, __uint_as_float(r1[8 * g + 3]) * 0.03125f);
-              o.z = pack_bf16x2(__uint_as_float(r1[8 * g + 4]) * 0.03125f, __uint_as_float(r1[8 * g + 5]) * 0.03125f);
-              o.w = pack_bf16x2(__uint_as_float(r1[8 * g + 6]) * 0.03125f, __uint_as_float(r1[8 * g + 7]) * 0.03125f);
-              *reinterpret_cast<uint4*>(yrow + c0 + 32 + 8 * g) = o;
-            }
-          }
+        for (int g = 0; g < 8; ++g) {  // 8 chunks of 8 columns
+          const uint32_t* v = g < 4 ? r0 + 8 * g : r1 + 8 * (g - 4);
+          uint4 o;
+          o.x = pack_bf16x2(__uint_as_float(v[0]) * 0.03125f, __uint_as_float(v[1]) * 0.03125f);
+          o.y = pack_bf16x2(__uint_as_float(v[2]) * 0.03125f, __uint_as_float(v[3]) * 0.03125f);
+          o.z = pack_bf16x2(__uint_as_float(v[4]) * 0.03125f, __uint_as_float(v[5]) * 0.03125f);
+          o.w = pack_bf16x2(__uint_as_float(v[6]) * 0.03125f, __uint_as_float(v[7]) * 0.03125f);
+          const int chunk = c0 / 8 + g;
+          *reinterpret_cast<uint4*>(srow + ((chunk ^ (tl & 15)) << 4)) = o;
+        }
+      }
+      named_bar_sync(1, 128);
+      const int n0 = t.nt * kRowsTile;
+      const int c = et & 15;  // 16-byte chunk of the row this thread copies out
+#pragma unroll 4
+      for (int rr = et >> 4; rr < t.rows; rr += 8) {
+        if (n0 + 8 * c < p.N) {
+          const uint4 o = *reinterpret_cast<const uint4*>(staging + rr * (kRowsTile * 2) + ((c ^ (rr & 15)) << 4));
+          *reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(t.m0 + rr) * p.N + n0 + 8 * c) = o;
         }
       }
     }
@@ -754,7 +759,20 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
       if (lane == 0) mbar_arrive(&full[stage]);
       return true;
     };
-    if constexpr (kPipe) {
+    constexpr int kAhead = C::kTasks == 1 ? 4 : (C::kTasks == 2 ? 2 : 1);
+    if (kt1 - kt0 <= kAhead) {
+      // every stage's activations in flight at once
+      uint4 xs[kAhead][C::kTasks][4];
+      float ds[kAhead];
+#pragma unroll
+      for (int j = 0; j < kAhead; ++j)
+        if (j < kt1 - kt0) load(kt0 + j, xs[j], ds[j]);
+#pragma unroll
+      for (int j = 0; j < kAhead; ++j) {
+        if (j >= kt1 - kt0) break;
+        if (!stage_body(kt0 + j, j, xs[j], ds[j])) break;
+      }
+    } else if constexpr (kPipe) {
       if (kt0 < kt1) load(kt0, xa, da);
       for (int kt = kt0, j = 0; kt < kt1; kt += 2, j += 2) {
         if (kt + 1 < kt1) load(kt + 1, xb, db);
