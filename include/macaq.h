@@ -160,6 +160,35 @@ int macaq_unfused_dense_mm(const uint16_t *x_dev, const float *D_dev, const uint
                            const uint8_t *Ws_dev, uint16_t *y_dev, int64_t M, int64_t N, int64_t K,
                            void *workspace_dev, size_t workspace_bytes, int32_t *status_dev, void *stream);
 
+/* ------------------------------------------------------------------ */
+/* Dense call without any device allocation                            */
+/* ------------------------------------------------------------------ */
+
+/* Size of the library's own fixed scratch buffer (8 MiB per device). */
+#define MACAQ_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* Dense MACAQ linear for callers that cannot allocate device memory -- for
+ * example code running where cudaMalloc is not allowed, or hosts whose memory
+ * is planned ahead and may not grow.  The pages have no counterpart to it.
+ * It runs the quantise-once path of macaq_dense_mm for any M (one activation
+ * quantisation kernel, then the block-scaled GEMM) with its workspace taken
+ * from a fixed buffer that the library itself holds on every device it is
+ * loaded on, until the process exits: nothing is allocated or freed, here or
+ * inside any library routine it calls.
+ *   Same arguments and result as macaq_dense_mm, without the workspace.
+ *   Limit: the call needs 4096 + ceil(M/128)*128 * K * 17/32 bytes of
+ *   scratch; larger calls return MACAQ_ERR_WORKSPACE without launching.
+ *   The first call on a device looks up the buffer's device address (a
+ *   runtime query, no allocation); make that first call before any stream
+ *   capture on that device.
+ *   Every call shares the one buffer and fully rewrites the part it uses
+ *   (nothing in it has to start at zero).  Calls whose kernels overlap on the
+ *   GPU -- on different streams, or from different host threads -- race on
+ *   it and must be ordered by the caller. */
+int macaq_dense_mm_noalloc(const uint16_t *x_dev, const float *D_dev, const uint8_t *Wq_dev,
+                           const uint8_t *Ws_dev, uint16_t *y_dev, int64_t M, int64_t N, int64_t K,
+                           int32_t *status_dev, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

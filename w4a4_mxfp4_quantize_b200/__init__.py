@@ -80,6 +80,7 @@ _SIG = {
     "macaq_export_weights": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "macaq_mx_encode_blocks": (ctypes.c_int, [_P, _P, _P, _I64, _P]),
     "macaq_unfused_workspace_bytes": (ctypes.c_size_t, [_I64, _I64]),
+    "macaq_dense_mm_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "macaq_unfused_dense_mm": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, ctypes.c_size_t,
                                               _P, _P]),
 }
@@ -238,6 +239,19 @@ def unfused_dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: tor
     _check(L.macaq_unfused_dense_mm(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(y), M, N, K, _ptr(ws),
                                     _nbytes(ws), _ptr(status), _stream_ptr(stream)),
            "macaq_unfused_dense_mm")
+    return y
+
+
+def dense_mm_noalloc(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: int,
+                     out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                     stream=None) -> torch.Tensor:
+    """Dense MACAQ linear using the library's fixed device scratch buffer
+    instead of a caller workspace (for callers that cannot allocate)."""
+    _require_cuda(x, D, Wq, Ws, out, status)
+    M, K = x.shape
+    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _check(lib().macaq_dense_mm_noalloc(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(y), M, N, K, _ptr(status),
+                                        _stream_ptr(stream)), "macaq_dense_mm_noalloc")
     return y
 
 

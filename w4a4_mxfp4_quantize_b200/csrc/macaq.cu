@@ -1088,6 +1088,24 @@ int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, c
   return e == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
+// ---- scratch for callers that cannot allocate device memory ----
+// One fixed buffer per device that loads this library, held until exit.  Host
+// code must not hand the symbol itself to a kernel (in host code it names a
+// host-side shadow); the device address is looked up once per device with
+// that device current.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MACAQ_STATIC_SCRATCH_BYTES];
+
+int noalloc_scratch(int dev, uint8_t** out) {
+  static uint8_t* addr[kMaxDevices] = {};
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return MACAQ_ERR_CUDA;
+    addr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = addr[dev];
+  return MACAQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1276,6 +1294,21 @@ int macaq_mx_encode_blocks(const float* v, uint8_t* codes, uint8_t* scales, int6
 size_t macaq_unfused_workspace_bytes(int64_t M, int64_t K) {
   if (M <= 0 || K < 256 || K > 65536 || K % 256) return 0;
   return dense_ws(M, K).total;
+}
+
+int macaq_dense_mm_noalloc(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y,
+                           int64_t M, int64_t N, int64_t K, int32_t* status, void* stream) {
+  int st = check_mm_args(x, D, Wq, Ws, y, M, N, K, 1);
+  if (st != MACAQ_OK || M == 0) return st;
+  if (dense_ws(M, K).total > MACAQ_STATIC_SCRATCH_BYTES) return MACAQ_ERR_WORKSPACE;
+  int dev, sms;
+  st = current_device(dev, sms);
+  if (st != MACAQ_OK) return st;
+  uint8_t* scratch = nullptr;
+  st = noalloc_scratch(dev, &scratch);
+  if (st != MACAQ_OK) return st;
+  return run_dense_two_kernel(x, D, Wq, Ws, y, M, N, K, scratch, status, static_cast<cudaStream_t>(stream), sms,
+                              true);
 }
 
 int macaq_unfused_dense_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y,
