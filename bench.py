@@ -248,7 +248,14 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-table", action="store_true", help="skip the per-workload table")
     ap.add_argument("--table-reps", type=int, default=30)
+    ap.add_argument("--only", default=None,
+                    help="CFG or CFG:IDX: only run these problems' calls --iters times (for profilers; no JSON)")
+    ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--unfused", action="store_true", help="with --only: the unfused ablation instead")
     args = ap.parse_args()
+    if args.only is not None:
+        run_only(args)
+        return
     args.warmup = max(args.warmup, 3)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -394,6 +401,27 @@ def main():
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_only(args):
+    """Run the calls of one workload (or one problem of it) a few times, with
+    the L2 flushed before each, so that a profiler can capture them."""
+    import w4a4_mxfp4_quantize_b200 as mq
+    mq.lib()
+    device = torch.device("cuda", 0)
+    cfg, _, idx = args.only.partition(":")
+    probs = synth.config(int(cfg))
+    if idx:
+        probs = [probs[int(idx)]]
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    for p in probs:
+        pp = Prepared(p, device, mq)
+        for _ in range(args.iters):
+            flush_buf.fill_(1)
+            pp.run_unfused(mq) if args.unfused else pp.run(mq)
+        torch.cuda.synchronize()
+        print("ran", p.name, flush=True)
+        del pp
 
 
 def workload_table(mq, device, stream, flush, hbm_gbs, reps):
