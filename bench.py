@@ -47,6 +47,29 @@ FP4_NOMINAL_TFLOPS = 9000.0   # NVIDIA's published dense FP4 figure for B200
 L2_FLUSH_BYTES = 256 << 20
 
 
+def kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "w4a4_mxfp4_quantize_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(summary: str):
+    """DRAM bytes per launch recorded by an ncu summary under profiles/, or None
+    when the kernels have changed since those counters were taken."""
+    path = os.path.join(ROOT, "profiles", summary)
+    try:
+        fields = dict(line.split(":", 1) for line in open(path) if ":" in line and not line.startswith(("#", "|", " ")))
+        if fields.get("kernel_source_sha256_16", "").strip() != kernel_source_hash():
+            return None
+        return float(fields["dram_bytes_per_launch"].strip())
+    except Exception:
+        return None
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -342,7 +365,9 @@ def main():
     launch_s = sum(per_call_us) * 1e-6
     achieved_gbs = bytes_step / launch_s / 1e9
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_gbs, "unit": "GB/s",
-                "frac": achieved_gbs / hbm_gbs, "traffic": None,
+                "frac": achieved_gbs / hbm_gbs,
+                "traffic": profiled_traffic("fused_small_kernel_dense_M128.md"),
+                "traffic_unit": "DRAM bytes per launch (ncu, profiles/fused_small_kernel_dense_M128.md)",
                 "peak_kind": f"{peak_kind} copy bandwidth (burst)",
                 "kernel": "fused_small_kernel (one launch per projection)",
                 "algorithmic_bytes_per_step": bytes_step, "launches_per_step": len(problems)}
