@@ -579,7 +579,9 @@ struct Cfg {
   static constexpr int kSmemBytes = 1024 + kRbufOff + 2 * kKTile * 4;
   static constexpr int kSfCol = BT < 32 ? 32 : BT;
   static constexpr int kTmemCols = kSfCol + 16 <= 64 ? 64 : kSfCol + 16 <= 128 ? 128 : 256;
-  static constexpr int kTasks = (BT * 8 + kProWarps * 32 - 1) / (kProWarps * 32);  // blocks per prologue thread
+  // half-blocks (16 elements, one lane of a pair) per prologue thread and per K tile
+  static constexpr int kTasks = BT * 16 / (kProWarps * 32);
+  static_assert(BT * 16 % (kProWarps * 32) == 0, "whole pairs of lanes per thread");
   static_assert(kStageBytes % 1024 == 0, "stage alignment");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -711,30 +713,31 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
     }
   } else {
     // ---- activation prologue: x/D, FWHT32, BF16, E8M0, E2M1 -> swizzled B tile ----
-    // The next K tile's activations and D are loaded while this one is computed
-    // (two register buffers when a thread has at most two blocks per tile).
+    // Each 32-element block is computed by a pair of adjacent lanes (16 elements
+    // each), so every prologue warp is busy even for the smallest token tile.
+    // Rows past the tile's end are computed on zeros, which encode to zero
+    // codes and a zero scale (the lane pairs must stay converged).  The
+    // activation loads of up to kAhead K tiles are in flight before any compute.
     constexpr int kPT = fused::kProWarps * 32;
-    constexpr bool kPipe = C::kTasks <= 2;
+    static_assert(kPT == kKTile, "one reciprocal per prologue thread");
+    constexpr int kAhead = C::kTasks == 1 ? 4 : (C::kTasks == 2 ? 4 : (C::kTasks == 4 ? 2 : 1));
     const int pt = threadIdx.x - 6 * 32;
-    uint4 xa[C::kTasks][4], xb[kPipe ? C::kTasks : 1][4];
-    float da = 0.f, db = 0.f;
-    auto load = [&](int kt, uint4 (&xv)[C::kTasks][4], float& d) {
+    auto load = [&](int kt, uint4 (&xv)[C::kTasks][2], float& d) {
 #pragma unroll
       for (int u = 0; u < C::kTasks; ++u) {
-        const int task = pt + u * kPT, t = task >> 3, c = task & 7;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) xv[u][i] = make_uint4(0, 0, 0, 0);
-        if (task < BT * 8 && t < rows) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m0 + t) * p.K +
-                                                            static_cast<int64_t>(kt) * kKTile + c * kBlk);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) xv[u][i] = __ldg(src + i);
+        const int task = pt + u * kPT, t = task >> 4, c = (task >> 1) & 7, half = task & 1;
+        xv[u][0] = make_uint4(0, 0, 0, 0);
+        xv[u][1] = make_uint4(0, 0, 0, 0);
+        if (t < rows) {
+          const uint4* src = reinterpret_cast<const uint4*>(
+              p.x + static_cast<int64_t>(m0 + t) * p.K + static_cast<int64_t>(kt) * kKTile + c * kBlk + half * 16);
+          xv[u][0] = __ldg(src);
+          xv[u][1] = __ldg(src + 1);
         }
       }
-      d = __ldg(p.D + static_cast<int64_t>(kt) * kKTile + pt);  // kPT == kKTile: one channel each
+      d = __ldg(p.D + static_cast<int64_t>(kt) * kKTile + pt);
     };
-    static_assert(kPT == kKTile, "one reciprocal per prologue thread");
-    auto stage_body = [&](int kt, int j, uint4 (&xv)[C::kTasks][4], float d) -> bool {
+    auto stage_body = [&](int j, uint4 (&xv)[C::kTasks][2], float d) -> bool {
       const int stage = j % kStages;
       float* r = rbuf + (j & 1) * kKTile;
       r[pt] = __frcp_rn(d);
@@ -746,45 +749,49 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
       uint8_t* bsf = smem + stage * C::kStageBytes + C::kOffSfb;
 #pragma unroll
       for (int u = 0; u < C::kTasks; ++u) {
-        const int task = pt + u * kPT, t = task >> 3, c = task & 7;
-        if (task >= BT * 8) break;
-        uint4 cv = make_uint4(0, 0, 0, 0);
-        uint32_t sc = 0;
-        if (t < rows) act_block(xv[u], r + c * kBlk, cv, sc);
-        *reinterpret_cast<uint4*>(bcode + code_chunk_offset(t, c)) = cv;
-        bsf[sf_offset(t, c)] = static_cast<uint8_t>(sc);
+        const int task = pt + u * kPT, t = task >> 4, c = (task >> 1) & 7, half = task & 1;
+        uint2 cv;
+        uint32_t sc;
+        act_half_block(xv[u], r + c * kBlk + half * 16, cv, sc);
+        *reinterpret_cast<uint2*>(bcode + code_chunk_offset(t, c) + half * 8) = cv;
+        if (half == 0) bsf[sf_offset(t, c)] = static_cast<uint8_t>(sc);
       }
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&full[stage]);
       return true;
     };
-    constexpr int kAhead = C::kTasks == 1 ? 4 : (C::kTasks == 2 ? 2 : 1);
-    if (kt1 - kt0 <= kAhead) {
-      // every stage's activations in flight at once
-      uint4 xs[kAhead][C::kTasks][4];
+    const int nst = kt1 - kt0;
+    if (nst <= kAhead) {
+      uint4 xs[kAhead][C::kTasks][2];
       float ds[kAhead];
 #pragma unroll
       for (int j = 0; j < kAhead; ++j)
-        if (j < kt1 - kt0) load(kt0 + j, xs[j], ds[j]);
+        if (j < nst) load(kt0 + j, xs[j], ds[j]);
 #pragma unroll
       for (int j = 0; j < kAhead; ++j) {
-        if (j >= kt1 - kt0) break;
-        if (!stage_body(kt0 + j, j, xs[j], ds[j])) break;
+        if (j >= nst) break;
+        if (!stage_body(j, xs[j], ds[j])) break;
       }
-    } else if constexpr (kPipe) {
-      if (kt0 < kt1) load(kt0, xa, da);
-      for (int kt = kt0, j = 0; kt < kt1; kt += 2, j += 2) {
-        if (kt + 1 < kt1) load(kt + 1, xb, db);
-        if (!stage_body(kt, j, xa, da)) break;
-        if (kt + 1 >= kt1) break;
-        if (kt + 2 < kt1) load(kt + 2, xa, da);
-        if (!stage_body(kt + 1, j + 1, xb, db)) break;
+    } else if constexpr (C::kTasks >= 8) {
+      // the largest token tile: registers hold one K tile of loads
+      uint4 xa[C::kTasks][2];
+      float da = 0.f;
+      for (int j = 0; j < nst; ++j) {
+        load(kt0 + j, xa, da);
+        if (!stage_body(j, xa, da)) break;
       }
     } else {
-      for (int kt = kt0, j = 0; kt < kt1; ++kt, ++j) {
-        load(kt, xa, da);
-        if (!stage_body(kt, j, xa, da)) break;
+      // deeper K ranges: one tile of loads ahead
+      uint4 xa[C::kTasks][2], xb[C::kTasks][2];
+      float da = 0.f, db = 0.f;
+      load(kt0, xa, da);
+      for (int j = 0; j < nst; j += 2) {
+        if (j + 1 < nst) load(kt0 + j + 1, xb, db);
+        if (!stage_body(j, xa, da)) break;
+        if (j + 1 >= nst) break;
+        if (j + 2 < nst) load(kt0 + j + 2, xa, da);
+        if (!stage_body(j + 1, xb, db)) break;
       }
     }
   }

@@ -194,6 +194,61 @@ __device__ __forceinline__ void act_block(const uint4 (&xv)[4], const float* __r
   scale = c;
 }
 
+// The same block computed by two adjacent lanes (lane parity = half): each lane
+// holds 16 of the 32 values (half 0: elements 0-15, half 1: 16-31), does the
+// butterfly stages h = 1..8 in registers and stage h = 16 with one exchange
+// of its partner's values.  Both lanes of a pair must call it together (the
+// whole warp converged).  Output: this lane's 8 code bytes (element 2j of its
+// half in the low nibble of byte j) and the block scale (same in both lanes).
+__device__ __forceinline__ void act_half_block(const uint4 (&xv)[2], const float* __restrict__ r, uint2& codes,
+                                               uint32_t& scale) {
+  const uint32_t half = threadIdx.x & 1u;
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(xv);
+  const uint64_t* r2 = reinterpret_cast<const uint64_t*>(r);
+  uint64_t P[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint32_t xs = f2_to_bf16x2(f2_mul(bf16x2_to_f2(w[j]), r2[j]));
+    const float v0 = bf16lo(xs), v1 = bf16hi(xs);
+    P[j] = f2(__fadd_rn(v0, v1), __fsub_rn(v0, v1));  // stage h = 1
+  }
+#pragma unroll
+  for (int hp = 1; hp < 8; hp <<= 1) {  // stages h = 2, 4, 8
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i & hp) continue;
+      const uint64_t a = P[i], b = P[i + hp];
+      P[i] = f2_add(a, b);
+      P[i + hp] = f2_sub(a, b);
+    }
+  }
+  // stage h = 16 across the pair: half 0 keeps v[i] + v[i+16], half 1 keeps
+  // v[i] - v[i+16] = partner + (-mine); IEEE a - b == a + (-b) exactly.
+  const uint64_t neg = half ? 0x8000000080000000ull : 0ull;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const uint64_t q = __shfl_xor_sync(0xffffffffu, P[j], 1);
+    P[j] = f2_add(q, P[j] ^ neg);
+  }
+  uint32_t u[8];
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    u[j] = f2_to_bf16x2(P[j]);
+    m = max_u16x2(m, u[j] & 0x7FFF7FFFu);
+  }
+  m = max_u16x2(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  const uint32_t amax16 = max(m & 0xFFFFu, m >> 16);
+  const uint32_t c = e8m0_from_amax_bits(amax16 << 16);
+  const float s = __uint_as_float((254u - min(c, 253u)) << 23);
+  const uint64_t s2 = f2(s, s);
+  codes.x = e2m1x8_f2(f2_mul(bf16x2_to_f2(u[0]), s2), f2_mul(bf16x2_to_f2(u[1]), s2),
+                      f2_mul(bf16x2_to_f2(u[2]), s2), f2_mul(bf16x2_to_f2(u[3]), s2));
+  codes.y = e2m1x8_f2(f2_mul(bf16x2_to_f2(u[4]), s2), f2_mul(bf16x2_to_f2(u[5]), s2),
+                      f2_mul(bf16x2_to_f2(u[6]), s2), f2_mul(bf16x2_to_f2(u[7]), s2));
+  scale = c;
+}
+
 // Weight block: 32 fp32 weights and their 32 channel factors D (offline).
 __device__ __forceinline__ void weight_block(const float (&wv)[32], const float (&dv)[32], uint4& codes,
                                              uint32_t& scale) {
