@@ -205,6 +205,16 @@ def test_unfused_ablation_matches_oracle():
             _check_large(p, y)
 
 
+def test_binding_rejects_wrong_output_tensor():
+    p = synth.dense(16, 256, 64, 0)
+    Wq, Ws = mq.prepare_weights(f32_dev(p.W), f32_dev(p.D))
+    x, D = x_to_dev(p.x), f32_dev(p.D[0])
+    with pytest.raises(ValueError):
+        mq.dense_mm(x, D, Wq, Ws, 64, out=torch.empty((16, 32), dtype=torch.bfloat16, device="cuda"))
+    with pytest.raises(ValueError):
+        mq.dense_mm(x, D, Wq, Ws, 64, out=torch.empty((16, 64), dtype=torch.float32, device="cuda"))
+
+
 def test_dense_zero_rows_is_noop():
     p = synth.dense(16, 256, 64, 0)
     Wq, Ws = mq.prepare_weights(f32_dev(p.W), f32_dev(p.D))
@@ -376,3 +386,41 @@ def test_max_rows_sampled():
         D = synth.make_d(x, W[0])[None, :]
         p = synth.Problem(x=x, W=W, D=D, M=M, N=N, K=K)
         _check_large(p, _run_dense(p), n_samples=2000)
+
+
+@pytest.mark.parametrize("M", [64, 128, 512])
+def test_dependent_calls_on_one_stream(M):
+    # Calls overlap their set-up with the previous kernel (programmatic
+    # dependent launch); inputs written by the previous call and outputs read
+    # by it must still be ordered.  Chain: a -> y1 -> y2, then a write-after-read
+    # (the third call overwrites `a`, which the first call read).
+    K1, N1, N2 = 1024, 1024, 256  # square first layer: its output may overwrite its input buffer
+    p1 = synth.dense(M, K1, N1, seed=31)
+    p2 = synth.dense(M, N1, N2, seed=32)
+    Wq1, Ws1 = mq.prepare_weights(f32_dev(p1.W), f32_dev(p1.D))
+    Wq2, Ws2 = mq.prepare_weights(f32_dev(p2.W), f32_dev(p2.D))
+    D1, D2 = f32_dev(p1.D[0]), f32_dev(p2.D[0])
+    a = x_to_dev(p1.x)
+    a_copy = a.clone()
+    c = x_to_dev(synth.to_bf16_bits(np.random.default_rng(33).standard_normal((M, K1)).astype(np.float32)))
+    torch.cuda.synchronize()
+    # reference: one call at a time
+    r1 = mq.dense_mm(a_copy, D1, Wq1, Ws1, N1); torch.cuda.synchronize()
+    r2 = mq.dense_mm(r1, D2, Wq2, Ws2, N2); torch.cuda.synchronize()
+    r3 = mq.dense_mm(c, D1, Wq1, Ws1, N1); torch.cuda.synchronize()
+    # back to back on one stream, no host synchronisation
+    y1 = torch.empty((M, N1), dtype=torch.bfloat16, device="cuda")
+    y2 = torch.empty((M, N2), dtype=torch.bfloat16, device="cuda")
+    for _ in range(3):
+        mq.dense_mm(a, D1, Wq1, Ws1, N1, out=y1)
+        mq.dense_mm(y1, D2, Wq2, Ws2, N2, out=y2)
+        mq.dense_mm(c, D1, Wq1, Ws1, N1, out=a)    # overwrites the first call's input
+        mq.dense_mm(a_copy, D1, Wq1, Ws1, N1, out=y1)  # restore the chain for the next round
+        a.copy_(a_copy)
+    torch.cuda.synchronize()
+    assert np.array_equal(y_to_bits(y2), y_to_bits(r2))
+    mq.dense_mm(a, D1, Wq1, Ws1, N1, out=y1)
+    mq.dense_mm(c, D1, Wq1, Ws1, N1, out=a)
+    torch.cuda.synchronize()
+    assert np.array_equal(y_to_bits(y1), y_to_bits(r1))
+    assert np.array_equal(y_to_bits(a), y_to_bits(r3))

@@ -129,6 +129,15 @@ def _require_cuda(*ts):
             raise ValueError("expected contiguous CUDA tensors")
 
 
+def _output(out, M: int, N: int, device):
+    """The output tensor: the caller's (checked: bf16 [M, N]) or a new one."""
+    if out is None:
+        return torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    if out.dtype != torch.bfloat16 or tuple(out.shape) != (M, N):
+        raise ValueError(f"out must be bfloat16 of shape {(M, N)}, got {out.dtype} {tuple(out.shape)}")
+    return out
+
+
 # ---------------------------------------------------------------------------
 # workspace: scratch for the quantise-once and grouped paths.  Callers may pass
 # their own (e.g. to capture calls in a CUDA graph); otherwise one buffer per
@@ -198,7 +207,7 @@ def dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tenso
     """y [M, N] bf16 = MACAQ linear of x bf16 [M, K] (fused kernel)."""
     _require_cuda(x, D, Wq, Ws, out, status)
     M, K = x.shape
-    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    y = _output(out, M, N, x.device)
     L = lib()
     need = int(L.macaq_workspace_bytes(M, N, K, 1))
     ws = workspace(need, x.device, stream, ws)
@@ -215,7 +224,7 @@ def grouped_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Ten
     _require_cuda(x, D, Wq, Ws, group_list, out, status)
     M, K = x.shape
     E = group_list.numel()
-    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    y = _output(out, M, N, x.device)
     L = lib()
     need = int(L.macaq_workspace_bytes(M, N, K, E))
     ws = workspace(need, x.device, stream, ws)
@@ -232,7 +241,7 @@ def unfused_dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: tor
     """Ablation: separate quantisation kernel, then the block-scaled GEMM."""
     _require_cuda(x, D, Wq, Ws, out, status)
     M, K = x.shape
-    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    y = _output(out, M, N, x.device)
     L = lib()
     need = int(L.macaq_unfused_workspace_bytes(M, K))
     ws = workspace(need, x.device, stream, ws)
@@ -249,7 +258,7 @@ def dense_mm_noalloc(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: tor
     instead of a caller workspace (for callers that cannot allocate)."""
     _require_cuda(x, D, Wq, Ws, out, status)
     M, K = x.shape
-    y = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    y = _output(out, M, N, x.device)
     _check(lib().macaq_dense_mm_noalloc(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(y), M, N, K, _ptr(status),
                                         _stream_ptr(stream)), "macaq_dense_mm_noalloc")
     return y

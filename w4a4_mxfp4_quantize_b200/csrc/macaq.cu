@@ -269,6 +269,7 @@ __global__ void __launch_bounds__(256) quant_tiles_kernel(const __grid_constant_
     base = static_cast<int>(p.goff[g]) + (pm - p.gtp[g]) * kRowsTile;
     rows = min(kRowsTile, static_cast<int>(p.goff[g + 1]) - base);
   } else {
+    pdl_wait();  // x may come from the previous kernel on the stream
     base = pm * kRowsTile;
     rows = min(kRowsTile, p.M - base);
   }
@@ -638,6 +639,11 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // The next kernel on the stream may start its own set-up now; everything this
+  // kernel reads that an earlier kernel may have written (x, D) or writes (y)
+  // is touched only after griddepcontrol.wait below.  The offline-prepared
+  // weights are read before it.
+  pdl_trigger();
   // Remote shared memory may only be touched once every CTA of the cluster runs
   // (and has initialised its receive barrier): arrive now, wait before the
   // first remote access.
@@ -761,6 +767,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
       if (lane == 0) mbar_arrive(&full[stage]);
       return true;
     };
+    pdl_wait();  // x and D may come from the previous kernel on the stream
     const int nst = kt1 - kt0;
     if (nst <= kAhead) {
       uint4 xs[kAhead][C::kTasks][2];
@@ -797,6 +804,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   }
 
   // ---- split-K reduction: wait for every rank's rows of this CTA, sum in rank order ----
+  pdl_wait();  // y may still be read by the previous kernel on the stream
   __syncwarp();                                          // reconverge (warps 0 and 1 ran single-lane roles)
   if (split && !cluster_waited) cluster_wait_acquire();  // warp-uniform: the epilogue warps waited above
   if (split && threadIdx.x == 0) *epi_flag = mbar_wait(recv_bar, 0, abort_flag, kWaitTimeoutNs) ? 1 : 0;
@@ -1006,16 +1014,16 @@ int launch_fused(const FusedParams& p, const FusedPlan& plan, cudaStream_t st) {
   cudaError_t e;
   switch (plan.bt) {
     case 16:
-      e = launch_ex(fused_small_kernel<16>, grid, block, fused::Cfg<16>::kSmemBytes, st, false, plan.S, p);
+      e = launch_ex(fused_small_kernel<16>, grid, block, fused::Cfg<16>::kSmemBytes, st, true, plan.S, p);
       break;
     case 32:
-      e = launch_ex(fused_small_kernel<32>, grid, block, fused::Cfg<32>::kSmemBytes, st, false, plan.S, p);
+      e = launch_ex(fused_small_kernel<32>, grid, block, fused::Cfg<32>::kSmemBytes, st, true, plan.S, p);
       break;
     case 64:
-      e = launch_ex(fused_small_kernel<64>, grid, block, fused::Cfg<64>::kSmemBytes, st, false, plan.S, p);
+      e = launch_ex(fused_small_kernel<64>, grid, block, fused::Cfg<64>::kSmemBytes, st, true, plan.S, p);
       break;
     default:
-      e = launch_ex(fused_small_kernel<128>, grid, block, fused::Cfg<128>::kSmemBytes, st, false, plan.S, p);
+      e = launch_ex(fused_small_kernel<128>, grid, block, fused::Cfg<128>::kSmemBytes, st, true, plan.S, p);
   }
   return e == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
@@ -1080,8 +1088,8 @@ int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, c
   QuantParams qp{};
   qp.x = x; qp.D = D; qp.Aq = ws + w.act_codes; qp.As = ws + w.act_scales;
   qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = 1;
-  quant_tiles_kernel<<<dim3(MT * 4, KT), 256, 0, st>>>(qp);
-  if (cudaPeekAtLastError() != cudaSuccess) return MACAQ_ERR_CUDA;
+  if (launch_ex(quant_tiles_kernel, dim3(MT * 4, KT), dim3(256), 0, st, pdl, 1, qp) != cudaSuccess)
+    return MACAQ_ERR_CUDA;
   GemmParams gp{};
   gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.As = qp.As; gp.y = y;
   gp.M = static_cast<int>(M); gp.N = static_cast<int>(N); gp.K = static_cast<int>(K);
