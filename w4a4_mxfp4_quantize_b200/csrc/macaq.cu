@@ -323,8 +323,11 @@ constexpr int kStagingOff = kStages * kStageBytes;  // BF16 output tile, 128 row
 constexpr int kStagingBytes = kRowsTile * kRowsTile * 2;
 constexpr int kBarOff = kStagingOff + kStagingBytes;
 constexpr int kGroupOff = kBarOff + 256;
-constexpr int kTmemCols = 512;  // accumulators at columns 0 and 128, scales at 256
+// accumulators at columns 0 and 128; scale factors from column 256, 16 columns per
+// stage, so the copy of a stage's scales need not wait for the previous stage's MMAs
+constexpr int kTmemCols = 512;
 constexpr int kSfCol = 256;
+static_assert(kSfCol + 16 * kStages <= kTmemCols, "scale slots fit the allocation");
 __host__ __device__ constexpr size_t smem_bytes(int E) {
   return 1024 + kGroupOff + (E > 0 ? static_cast<size_t>(E + 1) * 12 + 16 : 0);
 }
@@ -351,22 +354,26 @@ __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int idx, int 
   return t;
 }
 
-// Issue the four MMAs of one 256-K stage: D (+)= W-tile x act-tile^T.
-__device__ __forceinline__ void mma_stage(uint32_t a_addr, uint32_t b_addr, uint32_t sfa_addr, uint32_t sfb_addr,
+// Issue the scale copies and the four MMAs of one 256-K stage: D (+)= A-tile x B-tile^T.
+// adesc / bdesc describe the stage's code images, sfadesc / sfbdesc its scale images
+// (two 512-byte blocks each).  A descriptor's start address field counts 16-byte
+// units, so the descriptor of a later address is the first one plus the distance / 16.
+__device__ __forceinline__ void mma_stage(uint64_t adesc, uint64_t bdesc, uint64_t sfadesc, uint64_t sfbdesc,
                                           uint32_t sfa_col, uint32_t sfb_col, uint32_t d_tmem, uint32_t idesc_lo,
                                           uint32_t idesc_hi, bool first) {
-  tc_cp_32x128b_warpx4(sfa_col, sdesc_sf_block(sfa_addr));
-  tc_cp_32x128b_warpx4(sfa_col + 4, sdesc_sf_block(sfa_addr + 512));
-  tc_cp_32x128b_warpx4(sfb_col, sdesc_sf_block(sfb_addr));
-  tc_cp_32x128b_warpx4(sfb_col + 4, sdesc_sf_block(sfb_addr + 512));
+  tc_cp_32x128b_warpx4(sfa_col, sfadesc);
+  tc_cp_32x128b_warpx4(sfa_col + 4, sfadesc + (512 >> 4));
+  tc_cp_32x128b_warpx4(sfb_col, sfbdesc);
+  tc_cp_32x128b_warpx4(sfb_col + 4, sfbdesc + (512 >> 4));
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    // scale bytes 0-1 of each 32-bit TMEM word for the first 64 K, bytes 2-3 for the next
+    // scale bytes 0-1 of each 32-bit TMEM word for the first 64 K, bytes 2-3 for the next;
+    // each 64-K step is 32 bytes further along the code rows
     const uint32_t sfid = static_cast<uint32_t>(k & 1) * 2u;
     const uint32_t sfa = (sfa_col + (k >> 1) * 4) | (sfid << 30);
     const uint32_t sfb = (sfb_col + (k >> 1) * 4) | (sfid << 30);
-    tc_mma_mxf4(d_tmem, sdesc_kmajor_sw128(a_addr + 32 * k), sdesc_kmajor_sw128(b_addr + 32 * k),
-                (k & 1) ? idesc_hi : idesc_lo, sfa, sfb, (!first || k > 0) ? 1u : 0u);
+    tc_mma_mxf4(d_tmem, adesc + 2 * k, bdesc + 2 * k, (k & 1) ? idesc_hi : idesc_lo, sfa, sfb,
+                (!first || k > 0) ? 1u : 0u);
   }
 }
 
@@ -427,37 +434,60 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
 
   if (warp == 0) {
     // ================= producer: bulk copies of weight and activation images =================
-    if (lane == 0) {
+    // A bulk-copy instruction holds up the path that issued it until the engine has
+    // taken its copy in, so the copies of a stage are not issued one after another:
+    // the warp stays converged and one predicated instruction starts them together.
+    // A single warp has no other work to hide its own latency behind, so the source
+    // of each copy is stepped along, not recomputed, and worked out before the wait.
+    {
       const int slots = my_tiles * KT;
       const int pre = min(kStages, slots);
-      auto weights = [&](int j, int stage) {
-        const GemmTile t = gemm_tile(p, blockIdx.x + (j / KT) * gridDim.x, mtiles, goff, gtp);
-        const size_t wt = (static_cast<size_t>(t.g) * p.NT + t.nt) * KT + (j % KT);
-        uint8_t* sb = smem + stage * kStageBytes;
-        bulk_g2s(sb + kOffB, p.Wq + wt * kTileCodeBytes, kTileCodeBytes, &full[stage]);
-        bulk_g2s(sb + kOffSfb, p.Ws + wt * kTileSfBytes, kTileSfBytes, &full[stage]);
+      // Copy c of a stage: 0 activation codes, 1 activation scales, 2 weight codes,
+      // 3 weight scales.  Image (t, kt) of kind c sits at base_c + (t * KT + kt) * bytes_c.
+      auto image = [&](int i, int c) -> const uint8_t* {  // k tile 0 of this CTA's i-th output tile
+        const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp);
+        const size_t tile = c < 2 ? static_cast<size_t>(t.pm) : static_cast<size_t>(t.g) * p.NT + t.nt;
+        const uint8_t* base = c == 0 ? p.Aq : c == 1 ? p.As : c == 2 ? p.Wq : p.Ws;
+        return base + tile * KT * ((c & 1) ? kTileSfBytes : kTileCodeBytes);
       };
-      auto acts = [&](int j, int stage) {
-        const GemmTile t = gemm_tile(p, blockIdx.x + (j / KT) * gridDim.x, mtiles, goff, gtp);
-        const size_t at = static_cast<size_t>(t.pm) * KT + (j % KT);
-        uint8_t* sb = smem + stage * kStageBytes;
-        bulk_g2s(sb + kOffA, p.Aq + at * kTileCodeBytes, kTileCodeBytes, &full[stage]);
-        bulk_g2s(sb + kOffSfa, p.As + at * kTileSfBytes, kTileSfBytes, &full[stage]);
-      };
-      // the weights of the first stages do not depend on the quantiser: issue them first
-      for (int j = 0; j < pre; ++j) {
-        mbar_arrive_expect_tx(&full[j], kStageBytes);
-        weights(j, j);
+      auto dst_off = [](int c) { return c == 0 ? kOffA : c == 1 ? kOffSfa : c == 2 ? kOffB : kOffSfb; };
+      if (lane == 0)
+        for (int j = 0; j < pre; ++j) mbar_arrive_expect_tx(&full[j], kStageBytes);
+      __syncwarp();
+      // first stages: lane 2s + h carries copy 2 + h, then copy h, of stage s; the
+      // weights do not depend on the quantiser and go out before its wait
+      {
+        const int j = min(lane >> 1, pre - 1), h = lane & 1;
+        const uint32_t bytes = h ? kTileSfBytes : kTileCodeBytes;
+        uint8_t* sb = smem + j * kStageBytes;
+        bulk_g2s_if(lane < 2 * pre, sb + dst_off(2 + h), image(j / KT, 2 + h) + (j % KT) * bytes, bytes, &full[j]);
+        if (p.wait_for_producer) pdl_wait();
+        bulk_g2s_if(lane < 2 * pre, sb + dst_off(h), image(j / KT, h) + (j % KT) * bytes, bytes, &full[j]);
       }
-      if (p.wait_for_producer) pdl_wait();
-      for (int j = 0; j < pre; ++j) acts(j, j);
+      // then lane c < 4 streams copy c of every stage
+      const int c = lane & 3;
+      const uint32_t bytes = (c & 1) ? kTileSfBytes : kTileCodeBytes, doff = dst_off(c);
+      int kt = pre % KT, i = pre / KT, stage = 0;
+      uint32_t phase = 1;  // slots from `pre` on reuse stages released once before
+      const uint8_t* img = pre < slots ? image(i, c) : nullptr;
       for (int j = pre; j < slots; ++j) {
-        const int stage = j % kStages;
-        const uint32_t phase = (j / kStages) & 1;
-        if (!mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitTimeoutNs)) break;
-        mbar_arrive_expect_tx(&full[stage], kStageBytes);
-        weights(j, stage);
-        acts(j, stage);
+        int ok = 1;
+        if (lane == 0) {
+          ok = mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
+          if (ok) mbar_arrive_expect_tx(&full[stage], kStageBytes);
+        }
+        __syncwarp();  // the stage is free for every lane, not only the one that waited
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        bulk_g2s_if(lane < 4, smem + stage * kStageBytes + doff, img + kt * bytes, bytes, &full[stage]);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+        if (++kt == KT) {
+          kt = 0;
+          if (j + 1 < slots) img = image(++i, c);
+        }
       }
     }
   } else if (warp == 1) {
@@ -465,21 +495,27 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
     if (lane == 0) {
       const uint32_t idesc_lo = idesc_mxf4(128, kRowsTile, 0, 0);
       const uint32_t idesc_hi = idesc_mxf4(128, kRowsTile, 2, 2);
-      const uint32_t sfa_col = tmem + kSfCol, sfb_col = tmem + kSfCol + 8;
-      int j = 0;
+      const uint64_t code0 = sdesc_kmajor_sw128(smem_u32(smem)), sf0 = sdesc_sf_block(smem_u32(smem));
+      int stage = 0;
+      uint32_t phase = 0;
       bool ok = true;
       for (int i = 0; i < my_tiles && ok; ++i) {
         const int acc = i & 1;
         if (!mbar_wait(&acce[acc], ((i >> 1) & 1) ^ 1, abort_flag, kWaitTimeoutNs)) break;
         tc_fence_after();
-        for (int kt = 0; kt < KT; ++kt, ++j) {
-          const int stage = j % kStages;
-          if (!mbar_wait(&full[stage], (j / kStages) & 1, abort_flag, kWaitTimeoutNs)) { ok = false; break; }
+        for (int kt = 0; kt < KT; ++kt) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, kWaitTimeoutNs)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a = smem_u32(smem + stage * kStageBytes);
-          mma_stage(a + kOffA, a + kOffB, a + kOffSfa, a + kOffSfb, sfa_col, sfb_col, tmem + acc * kRowsTile,
-                    idesc_lo, idesc_hi, kt == 0);
+          const uint32_t so = static_cast<uint32_t>(stage * kStageBytes) >> 4;
+          const uint32_t sfa_col = tmem + kSfCol + 16 * stage;
+          mma_stage(code0 + so + (kOffA >> 4), code0 + so + (kOffB >> 4), sf0 + so + (kOffSfa >> 4),
+                    sf0 + so + (kOffSfb >> 4), sfa_col, sfa_col + 8, tmem + acc * kRowsTile, idesc_lo, idesc_hi,
+                    kt == 0);
           tc_commit(&empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
         }
         if (!ok) break;
         tc_commit(&accf[acc]);
@@ -578,8 +614,9 @@ struct Cfg {
   static constexpr int kBarOff = kRecvOff + kRecvBytes;
   static constexpr int kRbufOff = kBarOff + 256;
   static constexpr int kSmemBytes = 1024 + kRbufOff + 2 * kKTile * 4;
+  // scale factors from kSfCol, 16 columns per stage
   static constexpr int kSfCol = BT < 32 ? 32 : BT;
-  static constexpr int kTmemCols = kSfCol + 16 <= 64 ? 64 : kSfCol + 16 <= 128 ? 128 : 256;
+  static constexpr int kTmemCols = kSfCol + 16 * kStages <= 64 ? 64 : kSfCol + 16 * kStages <= 128 ? 128 : 256;
   // half-blocks (16 elements, one lane of a pair) per prologue thread and per K tile
   static constexpr int kTasks = BT * 16 / (kProWarps * 32);
   static_assert(BT * 16 % (kProWarps * 32) == 0, "whole pairs of lanes per thread");
@@ -651,30 +688,43 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   bool cluster_waited = false;
 
   if (warp == 0) {
-    if (lane == 0) {  // ---- producer: weight images ----
-      for (int kt = kt0, j = 0; kt < kt1; ++kt, ++j) {
-        const int stage = j % kStages;
-        if (!mbar_wait(&empty[stage], ((j / kStages) & 1) ^ 1, abort_flag, kWaitTimeoutNs)) break;
-        mbar_arrive_expect_tx(&full[stage], kTileCodeBytes + kTileSfBytes);
-        const size_t wt = static_cast<size_t>(nt) * p.KT + kt;
-        uint8_t* sb = smem + stage * C::kStageBytes;
-        bulk_g2s(sb, p.Wq + wt * kTileCodeBytes, kTileCodeBytes, &full[stage]);
-        bulk_g2s(sb + C::kOffSfa, p.Ws + wt * kTileSfBytes, kTileSfBytes, &full[stage]);
+    // ---- producer: weight images; lanes 0 and 1 start a stage's two copies with one
+    // instruction of the converged warp ----
+    for (int kt = kt0, j = 0; kt < kt1; ++kt, ++j) {
+      const int stage = j % kStages;
+      int ok = 1;
+      if (lane == 0) {
+        ok = mbar_wait(&empty[stage], ((j / kStages) & 1) ^ 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
+        if (ok) mbar_arrive_expect_tx(&full[stage], kTileCodeBytes + kTileSfBytes);
       }
+      __syncwarp();  // the stage is free for every lane, not only the one that waited
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      const size_t wt = static_cast<size_t>(nt) * p.KT + kt;
+      uint8_t* sb = smem + stage * C::kStageBytes;
+      const bool sf = lane & 1;
+      bulk_g2s_if(lane < 2, sf ? sb + C::kOffSfa : sb, sf ? p.Ws + wt * kTileSfBytes : p.Wq + wt * kTileCodeBytes,
+                  sf ? kTileSfBytes : kTileCodeBytes, &full[stage]);
     }
   } else if (warp == 1) {
     if (lane == 0) {  // ---- MMA issuer ----
       const uint32_t idesc_lo = idesc_mxf4(128, BT, 0, 0), idesc_hi = idesc_mxf4(128, BT, 2, 2);
-      const uint32_t sfa_col = tmem + C::kSfCol, sfb_col = tmem + C::kSfCol + 8;
+      const uint64_t code0 = sdesc_kmajor_sw128(smem_u32(smem)), sf0 = sdesc_sf_block(smem_u32(smem));
       bool ok = true;
-      for (int kt = kt0, j = 0; kt < kt1; ++kt, ++j) {
-        const int stage = j % kStages;
-        if (!mbar_wait(&full[stage], (j / kStages) & 1, abort_flag, kWaitTimeoutNs)) { ok = false; break; }
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kt = kt0; kt < kt1; ++kt) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, kWaitTimeoutNs)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t a = smem_u32(smem + stage * C::kStageBytes);
-        mma_stage(a, a + C::kOffB, a + C::kOffSfa, a + C::kOffSfb, sfa_col, sfb_col, tmem, idesc_lo, idesc_hi,
-                  kt == kt0);
+        const uint32_t so = static_cast<uint32_t>(stage * C::kStageBytes) >> 4;
+        const uint32_t sfa_col = tmem + C::kSfCol + 16 * stage;
+        mma_stage(code0 + so, code0 + so + (C::kOffB >> 4), sf0 + so + (C::kOffSfa >> 4), sf0 + so + (C::kOffSfb >> 4),
+                  sfa_col, sfa_col + 8, tmem, idesc_lo, idesc_hi, kt == kt0);
         tc_commit(&empty[stage]);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
       }
       if (ok) tc_commit(&accf[0]);
     }
