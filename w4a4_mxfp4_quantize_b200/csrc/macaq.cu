@@ -30,6 +30,7 @@
 #include <cuda_runtime.h>
 
 #include <cmath>
+#include <algorithm>
 #include <cstdint>
 #include <cstring>
 #include <utility>
@@ -306,42 +307,62 @@ struct GemmParams {
   const int* valid;
   int32_t* status;
   int wait_for_producer;  // dense: 1 when launched as a programmatic dependent of the quantiser
+  int NT2;                // 256-wide output tiles: ceil(NT / 2)
+  int stages;             // pipeline depth (gemm::stages_for(E))
 };
 
 // Large M: the MMA is not swapped.  Operand A = a 128-token activation tile,
-// operand B = 128 output channels of weights, D[t][n] in TMEM with one token
-// per lane, so each epilogue thread owns a contiguous run of an output row.
+// operand B = 256 output channels of weights (two 128-row weight images side by
+// side in shared memory), D[t][n] in TMEM with one token per lane, so each
+// epilogue thread owns a contiguous run of an output row.  An M = 128 MMA takes
+// about as long to issue at N = 128 as at N = 256, so the wider tile doubles the
+// work per instruction.
 namespace gemm {
-constexpr int kStages = 5;
-constexpr int kThreads = 192;  // warp 0 producer, warp 1 MMA, warps 2-5 epilogue
-constexpr int kStageBytes = 2 * kTileCodeBytes + 2 * kTileSfBytes;  // 34816
-constexpr int kOffA = 0;                        // activation codes
-constexpr int kOffB = kTileCodeBytes;           // weight codes
-constexpr int kOffSfa = 2 * kTileCodeBytes;     // activation scales
-constexpr int kOffSfb = kOffSfa + kTileSfBytes; // weight scales
-constexpr int kStagingOff = kStages * kStageBytes;  // BF16 output tile, 128 rows x 256 bytes, swizzled
-constexpr int kStagingBytes = kRowsTile * kRowsTile * 2;
-constexpr int kBarOff = kStagingOff + kStagingBytes;
-constexpr int kGroupOff = kBarOff + 256;
-// accumulators at columns 0 and 128; scale factors from column 256, 16 columns per
-// stage, so the copy of a stage's scales need not wait for the previous stage's MMAs
+constexpr int kMaxStages = 4;
+constexpr int kThreads = 320;  // warp 0 producer, warp 1 MMA, warps 2-9 epilogue
+constexpr int kTileN = 256;
+constexpr int kOffA = 0;                                    // activation codes, 128 rows
+constexpr int kOffB = kTileCodeBytes;                       // weight codes, 256 rows (two images)
+constexpr int kOffSfa = 3 * kTileCodeBytes;                 // activation scales
+constexpr int kOffSfb = kOffSfa + kTileSfBytes;             // weight scales of the two images
+constexpr int kStageBytes = kOffSfb + 2 * kTileSfBytes;     // 52224
+constexpr int kHalfBBytes = kTileCodeBytes + kTileSfBytes;  // the second weight image of a stage
+constexpr int kStagingBytes = kRowsTile * 64 * 2;           // 128 rows x 64 columns of BF16, swizzled
+constexpr int kFixedBytes = kStagingBytes + 256;            // staging, barriers and flags
+// TMEM: the accumulator in columns 0-255; from column 256, 24 columns of scales per
+// stage (activation scales 8, weight scales 16)
 constexpr int kTmemCols = 512;
 constexpr int kSfCol = 256;
-static_assert(kSfCol + 16 * kStages <= kTmemCols, "scale slots fit the allocation");
-__host__ __device__ constexpr size_t smem_bytes(int E) {
-  return 1024 + kGroupOff + (E > 0 ? static_cast<size_t>(E + 1) * 12 + 16 : 0);
+constexpr int kSfCols = 24;
+static_assert(kSfCol + kSfCols * kMaxStages <= kTmemCols, "scale slots fit the allocation");
+static_assert(kStageBytes % 1024 == 0, "stage alignment");
+constexpr size_t kSmemLimit = 227 * 1024;
+__host__ __device__ constexpr size_t group_bytes(int E) {
+  return E > 0 ? static_cast<size_t>(E + 1) * 12 + 16 : 0;
 }
+// four stages when the group tables leave room for them, else three
+__host__ __device__ constexpr int stages_for(int E) {
+  return 1024 + static_cast<size_t>(kMaxStages) * kStageBytes + kFixedBytes + group_bytes(E) <= kSmemLimit
+             ? kMaxStages
+             : kMaxStages - 1;
+}
+__host__ __device__ constexpr size_t smem_bytes(int E) {
+  return 1024 + static_cast<size_t>(stages_for(E)) * kStageBytes + kFixedBytes + group_bytes(E);
+}
+static_assert(smem_bytes(0) <= kSmemLimit && smem_bytes(1024) <= kSmemLimit, "shared memory");
 }  // namespace gemm
 
 struct GemmTile {
-  int g, m0, rows, pm, nt;
+  int g, m0, rows, pm, nt;  // nt: the first of the tile's two weight images
+  bool two;                 // the second image exists (N may end half-way through a tile)
 };
 
 __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int idx, int mtiles, const int64_t* goff,
                                               const int* gtp) {
   GemmTile t;
   t.pm = idx % mtiles;
-  t.nt = idx / mtiles;
+  t.nt = 2 * (idx / mtiles);
+  t.two = t.nt + 1 < p.NT;
   if (gtp == nullptr) {
     t.g = 0;
     t.m0 = t.pm * kRowsTile;
@@ -352,6 +373,29 @@ __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int idx, int 
     t.rows = min(kRowsTile, static_cast<int>(goff[t.g + 1]) - t.m0);
   }
   return t;
+}
+
+// Scale copies and the four MMAs of one 256-K stage of the wide tile: D (+)= A x B^T
+// with N = 256.  Weight scales in TMEM: for each group of four scale blocks, eight
+// columns (rows 0-127 of B, then rows 128-255); activation scales four columns.
+__device__ __forceinline__ void mma_stage_wide(uint64_t adesc, uint64_t bdesc, uint64_t sfadesc, uint64_t sfbdesc,
+                                               uint32_t sf_col, uint32_t d_tmem, uint32_t idesc_lo,
+                                               uint32_t idesc_hi, bool first) {
+  constexpr uint64_t kBlk512 = 512 >> 4, kImg = kTileSfBytes >> 4;
+  tc_cp_32x128b_warpx4(sf_col, sfadesc);
+  tc_cp_32x128b_warpx4(sf_col + 4, sfadesc + kBlk512);
+  tc_cp_32x128b_warpx4(sf_col + 8, sfbdesc);
+  tc_cp_32x128b_warpx4(sf_col + 12, sfbdesc + kImg);
+  tc_cp_32x128b_warpx4(sf_col + 16, sfbdesc + kBlk512);
+  tc_cp_32x128b_warpx4(sf_col + 20, sfbdesc + kImg + kBlk512);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t sfid = static_cast<uint32_t>(k & 1) * 2u;
+    const uint32_t sfa = (sf_col + (k >> 1) * 4) | (sfid << 30);
+    const uint32_t sfb = (sf_col + 8 + (k >> 1) * 8) | (sfid << 30);
+    tc_mma_mxf4(d_tmem, adesc + 2 * k, bdesc + 2 * k, (k & 1) ? idesc_hi : idesc_lo, sfa, sfb,
+                (!first || k > 0) ? 1u : 0u);
+  }
 }
 
 // Issue the scale copies and the four MMAs of one 256-K stage: D (+)= A-tile x B-tile^T.
@@ -381,11 +425,13 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
   using namespace gemm;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kBarOff);
-  uint64_t* empty = full + kStages;
-  uint64_t* accf = empty + kStages;
-  uint64_t* acce = accf + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acce + 2);
+  const int S = p.stages;
+  uint8_t* staging = smem + S * kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(staging + kStagingBytes);
+  uint64_t* empty = full + kMaxStages;
+  uint64_t* accf = empty + kMaxStages;  // accumulator complete
+  uint64_t* acce = accf + 1;            // accumulator drained by the epilogue
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acce + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* epi_flag = abort_flag + 1;
   int64_t* goff = nullptr;
@@ -396,7 +442,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
   if (p.gtp != nullptr) {
     pdl_wait();  // tables and activation images come from the preceding kernels
     if (*p.valid == 0) return;
-    goff = reinterpret_cast<int64_t*>(smem + kGroupOff);
+    goff = reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(full) + 256);
     gtp = reinterpret_cast<int*>(goff + p.E + 1);
     for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
       goff[i] = p.goff[i];
@@ -405,18 +451,16 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
     __syncthreads();
     mtiles = gtp[p.E];
   }
-  const int total = mtiles * p.NT;
+  const int total = mtiles * p.NT2;
   if (static_cast<int>(blockIdx.x) >= total) return;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&accf[a], 1);
-      mbar_init(&acce[a], 4);
-    }
+    mbar_init(accf, 1);
+    mbar_init(acce, 8);  // one arrival per epilogue warp
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -435,143 +479,156 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
   if (warp == 0) {
     // ================= producer: bulk copies of weight and activation images =================
     // A bulk-copy instruction holds up the path that issued it until the engine has
-    // taken its copy in, so the copies of a stage are not issued one after another:
-    // the warp stays converged and one predicated instruction starts them together.
-    // A single warp has no other work to hide its own latency behind, so the source
-    // of each copy is stepped along, not recomputed, and worked out before the wait.
-    {
-      const int slots = my_tiles * KT;
-      const int pre = min(kStages, slots);
-      // Copy c of a stage: 0 activation codes, 1 activation scales, 2 weight codes,
-      // 3 weight scales.  Image (t, kt) of kind c sits at base_c + (t * KT + kt) * bytes_c.
-      auto image = [&](int i, int c) -> const uint8_t* {  // k tile 0 of this CTA's i-th output tile
-        const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp);
-        const size_t tile = c < 2 ? static_cast<size_t>(t.pm) : static_cast<size_t>(t.g) * p.NT + t.nt;
-        const uint8_t* base = c == 0 ? p.Aq : c == 1 ? p.As : c == 2 ? p.Wq : p.Ws;
-        return base + tile * KT * ((c & 1) ? kTileSfBytes : kTileCodeBytes);
-      };
-      auto dst_off = [](int c) { return c == 0 ? kOffA : c == 1 ? kOffSfa : c == 2 ? kOffB : kOffSfb; };
-      if (lane == 0)
-        for (int j = 0; j < pre; ++j) mbar_arrive_expect_tx(&full[j], kStageBytes);
-      __syncwarp();
-      // first stages: lane 2s + h carries copy 2 + h, then copy h, of stage s; the
-      // weights do not depend on the quantiser and go out before its wait
-      {
-        const int j = min(lane >> 1, pre - 1), h = lane & 1;
-        const uint32_t bytes = h ? kTileSfBytes : kTileCodeBytes;
-        uint8_t* sb = smem + j * kStageBytes;
-        bulk_g2s_if(lane < 2 * pre, sb + dst_off(2 + h), image(j / KT, 2 + h) + (j % KT) * bytes, bytes, &full[j]);
-        if (p.wait_for_producer) pdl_wait();
-        bulk_g2s_if(lane < 2 * pre, sb + dst_off(h), image(j / KT, h) + (j % KT) * bytes, bytes, &full[j]);
+    // taken its copy in, so the six copies of a stage are not issued one after
+    // another: the warp stays converged and one predicated instruction starts them
+    // together.  A single warp has no other work to hide its own latency behind, so
+    // the source of each copy is stepped along, not recomputed, and worked out
+    // before the wait.
+    const int slots = my_tiles * KT;
+    const int pre = min(S, slots);
+    // Copy c of a stage: 0 activation codes, 1 activation scales, 2 / 3 codes of the
+    // first / second weight image, 4 / 5 their scales.  Image (t, kt) of a kind sits at
+    // base + (t * KT + kt) * bytes.  Gives k tile 0 of this CTA's i-th output tile.
+    auto source = [&](int i, int c, const uint8_t*& src, uint32_t& bytes, uint32_t& doff, bool& on, bool& two) {
+      const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp);
+      const bool sf = c == 1 || c >= 4, second = c == 3 || c == 5;
+      two = t.two;
+      on = !second || t.two;
+      bytes = sf ? kTileSfBytes : kTileCodeBytes;
+      const size_t img = c < 2 ? static_cast<size_t>(t.pm)
+                               : static_cast<size_t>(t.g) * p.NT + t.nt + ((second && t.two) ? 1 : 0);
+      src = (c == 0 ? p.Aq : c == 1 ? p.As : sf ? p.Ws : p.Wq) + img * KT * bytes;
+      doff = c == 0   ? kOffA
+             : c == 1 ? kOffSfa
+             : c == 2 ? kOffB
+             : c == 3 ? kOffB + kTileCodeBytes
+             : c == 4 ? kOffSfb
+                      : kOffSfb + kTileSfBytes;
+    };
+    const uint8_t* src;
+    uint32_t bytes, doff;
+    bool on, two;
+    if (lane == 0)
+      for (int j = 0; j < pre; ++j) {
+        source(j / KT, 0, src, bytes, doff, on, two);
+        mbar_arrive_expect_tx(&full[j], two ? kStageBytes : kStageBytes - kHalfBBytes);
       }
-      // then lane c < 4 streams copy c of every stage
-      const int c = lane & 3;
-      const uint32_t bytes = (c & 1) ? kTileSfBytes : kTileCodeBytes, doff = dst_off(c);
-      int kt = pre % KT, i = pre / KT, stage = 0;
-      uint32_t phase = 1;  // slots from `pre` on reuse stages released once before
-      const uint8_t* img = pre < slots ? image(i, c) : nullptr;
-      for (int j = pre; j < slots; ++j) {
-        int ok = 1;
-        if (lane == 0) {
-          ok = mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
-          if (ok) mbar_arrive_expect_tx(&full[stage], kStageBytes);
-        }
-        __syncwarp();  // the stage is free for every lane, not only the one that waited
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) break;
-        bulk_g2s_if(lane < 4, smem + stage * kStageBytes + doff, img + kt * bytes, bytes, &full[stage]);
-        if (++stage == kStages) {
-          stage = 0;
-          phase ^= 1;
-        }
-        if (++kt == KT) {
-          kt = 0;
-          if (j + 1 < slots) img = image(++i, c);
-        }
+    __syncwarp();
+    {  // first stages: weights (lane 4s + w: copy 2 + w of stage s) before the quantiser's wait
+      const int j = min(lane >> 2, pre - 1);
+      source(j / KT, 2 + (lane & 3), src, bytes, doff, on, two);
+      bulk_g2s_if(on && lane < 4 * pre, smem + j * kStageBytes + doff, src + (j % KT) * bytes, bytes, &full[j]);
+    }
+    if (p.wait_for_producer) pdl_wait();
+    {  // then their activations (lane 2s + a: copy a of stage s)
+      const int j = min(lane >> 1, pre - 1);
+      source(j / KT, lane & 1, src, bytes, doff, on, two);
+      bulk_g2s_if(lane < 2 * pre, smem + j * kStageBytes + doff, src + (j % KT) * bytes, bytes, &full[j]);
+    }
+    // from then on lane c < 6 streams copy c of every stage
+    const int c = lane < 6 ? lane : 0;
+    int kt = pre % KT, i = pre / KT, stage = 0;
+    uint32_t phase = 1;  // slots from `pre` on reuse stages released once before
+    if (pre < slots) source(i, c, src, bytes, doff, on, two);
+    for (int j = pre; j < slots; ++j) {
+      int ok = 1;
+      if (lane == 0) {
+        ok = mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
+        if (ok) mbar_arrive_expect_tx(&full[stage], two ? kStageBytes : kStageBytes - kHalfBBytes);
+      }
+      __syncwarp();  // the stage is free for every lane, not only the one that waited
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      bulk_g2s_if(on && lane < 6, smem + stage * kStageBytes + doff, src + kt * bytes, bytes, &full[stage]);
+      if (++stage == S) {
+        stage = 0;
+        phase ^= 1;
+      }
+      if (++kt == KT) {
+        kt = 0;
+        if (j + 1 < slots) source(++i, c, src, bytes, doff, on, two);
       }
     }
   } else if (warp == 1) {
     // ================= MMA issuer =================
     if (lane == 0) {
-      const uint32_t idesc_lo = idesc_mxf4(128, kRowsTile, 0, 0);
-      const uint32_t idesc_hi = idesc_mxf4(128, kRowsTile, 2, 2);
+      const uint32_t idesc_lo = idesc_mxf4(128, kTileN, 0, 0);
+      const uint32_t idesc_hi = idesc_mxf4(128, kTileN, 2, 2);
       const uint64_t code0 = sdesc_kmajor_sw128(smem_u32(smem)), sf0 = sdesc_sf_block(smem_u32(smem));
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int i = 0; i < my_tiles && ok; ++i) {
-        const int acc = i & 1;
-        if (!mbar_wait(&acce[acc], ((i >> 1) & 1) ^ 1, abort_flag, kWaitTimeoutNs)) break;
+        if (!mbar_wait(acce, (i & 1) ^ 1, abort_flag, kWaitTimeoutNs)) break;
         tc_fence_after();
         for (int kt = 0; kt < KT; ++kt) {
           if (!mbar_wait(&full[stage], phase, abort_flag, kWaitTimeoutNs)) { ok = false; break; }
           tc_fence_after();
           const uint32_t so = static_cast<uint32_t>(stage * kStageBytes) >> 4;
-          const uint32_t sfa_col = tmem + kSfCol + 16 * stage;
-          mma_stage(code0 + so + (kOffA >> 4), code0 + so + (kOffB >> 4), sf0 + so + (kOffSfa >> 4),
-                    sf0 + so + (kOffSfb >> 4), sfa_col, sfa_col + 8, tmem + acc * kRowsTile, idesc_lo, idesc_hi,
-                    kt == 0);
+          mma_stage_wide(code0 + so + (kOffA >> 4), code0 + so + (kOffB >> 4), sf0 + so + (kOffSfa >> 4),
+                         sf0 + so + (kOffSfb >> 4), tmem + kSfCol + kSfCols * stage, tmem, idesc_lo, idesc_hi,
+                         kt == 0);
           tc_commit(&empty[stage]);
-          if (++stage == kStages) {
+          if (++stage == S) {
             stage = 0;
             phase ^= 1;
           }
         }
         if (!ok) break;
-        tc_commit(&accf[acc]);
+        tc_commit(accf);
       }
     }
   } else {
-    // ================= epilogue: TMEM -> x 2^-5 -> BF16 -> staged tile -> coalesced rows =================
-    // Thread (q, lane) owns token row 32q + lane of the accumulator.  Rows are
-    // staged in shared memory with their 16-byte chunks XOR-swizzled by the row
-    // index (conflict-free row writes and row-run reads), then written out two
-    // full 256-byte rows per warp instruction.
-    const int q = warp & 3;
+    // ================= epilogue: TMEM -> x 2^-5 -> BF16 -> staged chunks -> coalesced rows =================
+    // Warp w reads TMEM lanes 32 (w % 4) .. + 31 (accumulator rows) and columns
+    // 128 h .. + 127 with h = (w - 2) / 4.  The accumulator is drained into packed
+    // BF16 registers first and handed back, so the next tile's MMAs overlap the
+    // write-out.  Rows go out in 64-column chunks staged in shared memory with their
+    // 16-byte pieces XOR-swizzled by the row (conflict-free writes and reads).
+    const int q = warp & 3, h = (warp - 2) >> 2;
     const int et = threadIdx.x - 64;
     const int tl = q * 32 + lane;
-    uint8_t* staging = smem + kStagingOff;
     for (int i = 0; i < my_tiles; ++i) {
-      const int acc = i & 1;
       const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp);
-      if (et == 0) *epi_flag = mbar_wait(&accf[acc], (i >> 1) & 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
-      named_bar_sync(1, 128);  // also: every thread has finished reading the previous tile's staging
+      if (et == 0) *epi_flag = mbar_wait(accf, i & 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
+      named_bar_sync(1, 256);  // also: every thread has finished reading the previous tile's staging
       if (!*epi_flag) break;
       tc_fence_after();
-      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + acc * kRowsTile;
-      uint8_t* srow = staging + tl * (kRowsTile * 2);
-#pragma unroll 1
-      for (int c0 = 0; c0 < kRowsTile; c0 += 64) {
-        uint32_t r0[32], r1[32];
-        tmem_ld_32x32b_x32(taddr + c0, r0);
-        tmem_ld_32x32b_x32(taddr + c0 + 32, r1);
-        tmem_wait_ld();
-        if (c0 + 64 >= kRowsTile) {  // all columns read: the accumulator is free for the tile after next
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&acce[acc]);
-        }
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 128;
+      uint32_t pk[64];
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {  // 8 chunks of 8 columns
-          const uint32_t* v = g < 4 ? r0 + 8 * g : r1 + 8 * (g - 4);
-          uint4 o;
-          o.x = pack_bf16x2(__uint_as_float(v[0]) * 0.03125f, __uint_as_float(v[1]) * 0.03125f);
-          o.y = pack_bf16x2(__uint_as_float(v[2]) * 0.03125f, __uint_as_float(v[3]) * 0.03125f);
-          o.z = pack_bf16x2(__uint_as_float(v[4]) * 0.03125f, __uint_as_float(v[5]) * 0.03125f);
-          o.w = pack_bf16x2(__uint_as_float(v[6]) * 0.03125f, __uint_as_float(v[7]) * 0.03125f);
-          const int chunk = c0 / 8 + g;
-          *reinterpret_cast<uint4*>(srow + ((chunk ^ (tl & 15)) << 4)) = o;
-        }
+      for (int c0 = 0; c0 < 128; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(taddr + c0, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          pk[c0 / 2 + e] = pack_bf16x2(__uint_as_float(r[2 * e]) * 0.03125f, __uint_as_float(r[2 * e + 1]) * 0.03125f);
       }
-      named_bar_sync(1, 128);
-      const int n0 = t.nt * kRowsTile;
-      const int c = et & 15;  // 16-byte chunk of the row this thread copies out
-#pragma unroll 4
-      for (int rr = et >> 4; rr < t.rows; rr += 8) {
-        if (n0 + 8 * c < p.N) {
-          const uint4 o = *reinterpret_cast<const uint4*>(staging + rr * (kRowsTile * 2) + ((c ^ (rr & 15)) << 4));
-          *reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(t.m0 + rr) * p.N + n0 + 8 * c) = o;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce);
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        if ((ch >> 1) == h) {  // chunk ch = columns 64 ch .. + 63, held by half ch / 2
+          uint8_t* srow = staging + tl * 128;
+#pragma unroll
+          for (int g = 0; g < 8; ++g) {
+            const int b = (ch & 1) * 32 + 4 * g;
+            *reinterpret_cast<uint4*>(srow + ((g ^ (tl & 7)) << 4)) = make_uint4(pk[b], pk[b + 1], pk[b + 2], pk[b + 3]);
+          }
         }
+        named_bar_sync(1, 256);
+        const int n0 = t.nt * kRowsTile + ch * 64;
+        const int c = et & 7;  // 16-byte piece of a 128-byte row run
+        if (n0 + 8 * c < p.N) {
+#pragma unroll 4
+          for (int rr = et >> 3; rr < t.rows; rr += 32) {
+            const uint4 o = *reinterpret_cast<const uint4*>(staging + rr * 128 + ((c ^ (rr & 7)) << 4));
+            *reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(t.m0 + rr) * p.N + n0 + 8 * c) = o;
+          }
+        }
+        if (ch < 3) named_bar_sync(1, 256);  // read out before the next chunk overwrites it
       }
     }
   }
@@ -932,8 +989,9 @@ int current_device(int& dev, int& sms) {
   sms = s.sms;
   if (!s.is_sm100) return MACAQ_ERR_ARCH;
   if (!s.attrs_set) {  // once per device: opt in to the shared memory the kernels use
+    const size_t gemm_smem = gemm::kSmemLimit;  // smem_bytes(E) stays within it for every E
     bool ok = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   static_cast<int>(gemm::smem_bytes(kMaxGroups))) == cudaSuccess;
+                                   static_cast<int>(gemm_smem)) == cudaSuccess;
     ok = ok && cudaFuncSetAttribute(fused_small_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     fused::Cfg<16>::kSmemBytes) == cudaSuccess;
     ok = ok && cudaFuncSetAttribute(fused_small_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1144,9 +1202,10 @@ int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, c
   gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.As = qp.As; gp.y = y;
   gp.M = static_cast<int>(M); gp.N = static_cast<int>(N); gp.K = static_cast<int>(K);
   gp.NT = static_cast<int>(pad128(N) / 128); gp.KT = KT; gp.E = 1; gp.MT = MT;
+  gp.NT2 = (gp.NT + 1) / 2; gp.stages = gemm::stages_for(0);
   gp.status = status;
   gp.wait_for_producer = pdl ? 1 : 0;
-  const int tiles = MT * gp.NT;
+  const int tiles = MT * gp.NT2;
   const int grid = tiles < sms ? tiles : sms;
   const cudaError_t e =
       launch_ex(gemm_kernel, dim3(grid), dim3(gemm::kThreads), gemm::smem_bytes(0), st, pdl, 1, gp);
@@ -1304,6 +1363,7 @@ int macaq_grouped_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const
   gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.As = qp.As; gp.y = y;
   gp.M = static_cast<int>(M); gp.N = static_cast<int>(N); gp.K = static_cast<int>(K);
   gp.NT = static_cast<int>(pad128(N) / 128); gp.KT = KT; gp.E = static_cast<int>(E);
+  gp.NT2 = (gp.NT + 1) / 2; gp.stages = gemm::stages_for(static_cast<int>(E));
   gp.goff = goff; gp.gtp = gtp; gp.valid = valid;
   gp.status = status;
   const cudaError_t e = launch_ex(gemm_kernel, dim3(sms), dim3(gemm::kThreads),
