@@ -669,14 +669,21 @@ struct Cfg {
   static constexpr int kRecvOff = kStages * kStageBytes;
   static constexpr int kRecvBytes = (BT + 8) * kRowsTile * 4;
   static constexpr int kBarOff = kRecvOff + kRecvBytes;
-  static constexpr int kRbufOff = kBarOff + 256;
-  static constexpr int kSmemBytes = 1024 + kRbufOff + 2 * kKTile * 4;
+  // The prologue warps work as kGroups groups, group g on the CTA's K tiles g,
+  // g + kGroups, ...: a small token tile then has several K tiles in flight.
+  static constexpr int kGroups = BT <= 16 ? 2 : 1;
+  static constexpr int kGroupThreads = kProWarps * 32 / kGroups;
+  static constexpr int kRbufOff = kBarOff + 256;  // per group, two K tiles of reciprocals
+  static constexpr int kSmemBytes = 1024 + kRbufOff + kGroups * 2 * kKTile * 4;
   // scale factors from kSfCol, 16 columns per stage
   static constexpr int kSfCol = BT < 32 ? 32 : BT;
   static constexpr int kTmemCols = kSfCol + 16 * kStages <= 64 ? 64 : kSfCol + 16 * kStages <= 128 ? 128 : 256;
   // half-blocks (16 elements, one lane of a pair) per prologue thread and per K tile
-  static constexpr int kTasks = BT * 16 / (kProWarps * 32);
-  static_assert(BT * 16 % (kProWarps * 32) == 0, "whole pairs of lanes per thread");
+  static constexpr int kTasks = BT * 16 / kGroupThreads;
+  static_assert(BT * 16 % kGroupThreads == 0, "whole pairs of lanes per thread");
+  // reciprocals 1/D of a K tile per prologue thread
+  static constexpr int kRcp = kKTile / kGroupThreads;
+  static_assert(kKTile % kGroupThreads == 0, "whole reciprocals per thread");
   static_assert(kStageBytes % 1024 == 0, "stage alignment");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 };
@@ -695,7 +702,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(recv_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* epi_flag = abort_flag + 1;
-  volatile int* pro_flag = abort_flag + 2;  // [2]
+  volatile int* pro_flag = abort_flag + 2;  // [group][2]
   float* rbuf = reinterpret_cast<float*>(smem + C::kRbufOff);
   float* part = reinterpret_cast<float*>(smem);  // local FP32 partial tile [BT][128], after the mainloop
 
@@ -712,7 +719,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1 + fused::kProWarps);
+      mbar_init(&full[s], 1 + fused::kProWarps / C::kGroups);
       mbar_init(&empty[s], 1);
     }
     mbar_init(&accf[0], 1);
@@ -829,16 +836,17 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
     // Each 32-element block is computed by a pair of adjacent lanes (16 elements
     // each), so every prologue warp is busy even for the smallest token tile.
     // Rows past the tile's end are computed on zeros, which encode to zero
-    // codes and a zero scale (the lane pairs must stay converged).  The
-    // activation loads of up to kAhead K tiles are in flight before any compute.
-    constexpr int kPT = fused::kProWarps * 32;
-    static_assert(kPT == kKTile, "one reciprocal per prologue thread");
-    constexpr int kAhead = C::kTasks == 1 ? 4 : (C::kTasks == 2 ? 4 : (C::kTasks == 4 ? 2 : 1));
+    // codes and a zero scale (the lane pairs must stay converged).  Group g of
+    // the prologue warps takes the CTA's K tiles g, g + kGroups, ...; the
+    // activation loads of up to kAhead of its K tiles are in flight before any compute.
+    constexpr int kGT = C::kGroupThreads, kG = C::kGroups;
+    constexpr int kAhead = C::kTasks <= 2 ? 2 : 1;
     const int pt = threadIdx.x - 6 * 32;
-    auto load = [&](int kt, uint4 (&xv)[C::kTasks][2], float& d) {
+    const int grp = pt / kGT, gt = pt % kGT;
+    auto load = [&](int kt, uint4 (&xv)[C::kTasks][2], float (&d)[C::kRcp]) {
 #pragma unroll
       for (int u = 0; u < C::kTasks; ++u) {
-        const int task = pt + u * kPT, t = task >> 4, c = (task >> 1) & 7, half = task & 1;
+        const int task = gt + u * kGT, t = task >> 4, c = (task >> 1) & 7, half = task & 1;
         xv[u][0] = make_uint4(0, 0, 0, 0);
         xv[u][1] = make_uint4(0, 0, 0, 0);
         if (t < rows) {
@@ -848,26 +856,41 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
           xv[u][1] = __ldg(src + 1);
         }
       }
-      d = __ldg(p.D + static_cast<int64_t>(kt) * kKTile + pt);
+#pragma unroll
+      for (int e = 0; e < C::kRcp; ++e) d[e] = __ldg(p.D + static_cast<int64_t>(kt) * kKTile + gt + e * kGT);
     };
-    auto stage_body = [&](int j, uint4 (&xv)[C::kTasks][2], float d) -> bool {
-      const int stage = j % kStages;
-      float* r = rbuf + (j & 1) * kKTile;
-      r[pt] = __frcp_rn(d);
-      if (pt == 0)
-        pro_flag[j & 1] = mbar_wait(&empty[stage], ((j / kStages) & 1) ^ 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
-      named_bar_sync(2, kPT);
-      if (!pro_flag[j & 1]) return false;
+    // the group's jj-th K tile: CTA-local index j = grp + kG * jj
+    auto stage_body = [&](int jj, uint4 (&xv)[C::kTasks][2], const float (&d)[C::kRcp]) -> bool {
+      const int j = grp + kG * jj, stage = j % kStages;
+      const int slot = grp * 2 + (jj & 1);
+      float* r = rbuf + slot * kKTile;
+#pragma unroll
+      for (int e = 0; e < C::kRcp; ++e) r[gt + e * kGT] = __frcp_rn(d[e]);
+      if (gt == 0) pro_flag[slot] = mbar_wait(&empty[stage], ((j / kStages) & 1) ^ 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
+      named_bar_sync(2 + grp, kGT);
+      if (!pro_flag[slot]) return false;
       uint8_t* bcode = smem + stage * C::kStageBytes + C::kOffB;
       uint8_t* bsf = smem + stage * C::kStageBytes + C::kOffSfb;
+      // two tasks at a time, interleaved (two dependency chains per thread), where
+      // the registers allow
+      constexpr int kIlp = C::kTasks == 2 ? 2 : 1;
 #pragma unroll
-      for (int u = 0; u < C::kTasks; ++u) {
-        const int task = pt + u * kPT, t = task >> 4, c = (task >> 1) & 7, half = task & 1;
-        uint2 cv;
-        uint32_t sc;
-        act_half_block(xv[u], r + c * kBlk + half * 16, cv, sc);
-        *reinterpret_cast<uint2*>(bcode + code_chunk_offset(t, c) + half * 8) = cv;
-        if (half == 0) bsf[sf_offset(t, c)] = static_cast<uint8_t>(sc);
+      for (int u0 = 0; u0 < C::kTasks; u0 += kIlp) {
+        const float* rr[kIlp];
+        uint2 cv[kIlp];
+        uint32_t sc[kIlp];
+#pragma unroll
+        for (int v = 0; v < kIlp; ++v) {
+          const int task = gt + (u0 + v) * kGT, c = (task >> 1) & 7, half = task & 1;
+          rr[v] = r + c * kBlk + half * 16;
+        }
+        act_half_blocks<kIlp>(*reinterpret_cast<const uint4(*)[kIlp][2]>(&xv[u0]), rr, cv, sc);
+#pragma unroll
+        for (int v = 0; v < kIlp; ++v) {
+          const int task = gt + (u0 + v) * kGT, t = task >> 4, c = (task >> 1) & 7, half = task & 1;
+          *reinterpret_cast<uint2*>(bcode + code_chunk_offset(t, c) + half * 8) = cv[v];
+          if (half == 0) bsf[sf_offset(t, c)] = static_cast<uint8_t>(sc[v]);
+        }
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -876,36 +899,38 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
     };
     pdl_wait();  // x and D may come from the previous kernel on the stream
     const int nst = kt1 - kt0;
-    if (nst <= kAhead) {
+    const int gst = nst > grp ? (nst - grp + kG - 1) / kG : 0;  // this group's K tiles
+    auto kt_of = [&](int jj) { return kt0 + grp + kG * jj; };
+    if (gst <= kAhead) {
       uint4 xs[kAhead][C::kTasks][2];
-      float ds[kAhead];
+      float ds[kAhead][C::kRcp];
 #pragma unroll
-      for (int j = 0; j < kAhead; ++j)
-        if (j < nst) load(kt0 + j, xs[j], ds[j]);
+      for (int jj = 0; jj < kAhead; ++jj)
+        if (jj < gst) load(kt_of(jj), xs[jj], ds[jj]);
 #pragma unroll
-      for (int j = 0; j < kAhead; ++j) {
-        if (j >= nst) break;
-        if (!stage_body(j, xs[j], ds[j])) break;
+      for (int jj = 0; jj < kAhead; ++jj) {
+        if (jj >= gst) break;
+        if (!stage_body(jj, xs[jj], ds[jj])) break;
       }
     } else if constexpr (C::kTasks >= 8) {
       // the largest token tile: registers hold one K tile of loads
       uint4 xa[C::kTasks][2];
-      float da = 0.f;
-      for (int j = 0; j < nst; ++j) {
-        load(kt0 + j, xa, da);
-        if (!stage_body(j, xa, da)) break;
+      float da[C::kRcp];
+      for (int jj = 0; jj < gst; ++jj) {
+        load(kt_of(jj), xa, da);
+        if (!stage_body(jj, xa, da)) break;
       }
     } else {
-      // deeper K ranges: one tile of loads ahead
+      // deeper K ranges: one K tile of loads ahead
       uint4 xa[C::kTasks][2], xb[C::kTasks][2];
-      float da = 0.f, db = 0.f;
-      load(kt0, xa, da);
-      for (int j = 0; j < nst; j += 2) {
-        if (j + 1 < nst) load(kt0 + j + 1, xb, db);
-        if (!stage_body(j, xa, da)) break;
-        if (j + 1 >= nst) break;
-        if (j + 2 < nst) load(kt0 + j + 2, xa, da);
-        if (!stage_body(j + 1, xb, db)) break;
+      float da[C::kRcp], db[C::kRcp];
+      load(kt_of(0), xa, da);
+      for (int jj = 0; jj < gst; jj += 2) {
+        if (jj + 1 < gst) load(kt_of(jj + 1), xb, db);
+        if (!stage_body(jj, xa, da)) break;
+        if (jj + 1 >= gst) break;
+        if (jj + 2 < gst) load(kt_of(jj + 2), xa, da);
+        if (!stage_body(jj + 1, xb, db)) break;
       }
     }
   }

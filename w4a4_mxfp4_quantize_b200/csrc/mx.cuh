@@ -249,6 +249,73 @@ __device__ __forceinline__ void act_half_block(const uint4 (&xv)[2], const float
   scale = c;
 }
 
+// T independent half-blocks, each step done for all T before the next step, so
+// that one thread keeps T dependency chains in flight.  Same arithmetic as
+// act_half_block; lane pairs as there.
+template <int T>
+__device__ __forceinline__ void act_half_blocks(const uint4 (&xv)[T][2], const float* const (&r)[T],
+                                                uint2 (&codes)[T], uint32_t (&scale)[T]) {
+  const uint64_t neg = (threadIdx.x & 1u) ? 0x8000000080000000ull : 0ull;
+  uint64_t P[T][8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+      const uint32_t w = reinterpret_cast<const uint32_t*>(xv[t])[j];
+      const uint64_t r2 = reinterpret_cast<const uint64_t*>(r[t])[j];
+      const uint32_t xs = f2_to_bf16x2(f2_mul(bf16x2_to_f2(w), r2));
+      const float v0 = bf16lo(xs), v1 = bf16hi(xs);
+      P[t][j] = f2(__fadd_rn(v0, v1), __fsub_rn(v0, v1));  // stage h = 1
+    }
+  }
+#pragma unroll
+  for (int hp = 1; hp < 8; hp <<= 1) {  // stages h = 2, 4, 8
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i & hp) continue;
+#pragma unroll
+      for (int t = 0; t < T; ++t) {
+        const uint64_t a = P[t][i], b = P[t][i + hp];
+        P[t][i] = f2_add(a, b);
+        P[t][i + hp] = f2_sub(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {  // stage h = 16 across the pair
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+      const uint64_t q = __shfl_xor_sync(0xffffffffu, P[t][j], 1);
+      P[t][j] = f2_add(q, P[t][j] ^ neg);
+    }
+  }
+  uint32_t u[T][8], m[T];
+#pragma unroll
+  for (int t = 0; t < T; ++t) m[t] = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+      u[t][j] = f2_to_bf16x2(P[t][j]);
+      m[t] = max_u16x2(m[t], u[t][j] & 0x7FFF7FFFu);
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < T; ++t) m[t] = max_u16x2(m[t], __shfl_xor_sync(0xffffffffu, m[t], 1));
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+    const uint32_t amax16 = max(m[t] & 0xFFFFu, m[t] >> 16);
+    const uint32_t c = e8m0_from_amax_bits(amax16 << 16);
+    const float s = __uint_as_float((254u - min(c, 253u)) << 23);
+    const uint64_t s2 = f2(s, s);
+    codes[t].x = e2m1x8_f2(f2_mul(bf16x2_to_f2(u[t][0]), s2), f2_mul(bf16x2_to_f2(u[t][1]), s2),
+                           f2_mul(bf16x2_to_f2(u[t][2]), s2), f2_mul(bf16x2_to_f2(u[t][3]), s2));
+    codes[t].y = e2m1x8_f2(f2_mul(bf16x2_to_f2(u[t][4]), s2), f2_mul(bf16x2_to_f2(u[t][5]), s2),
+                           f2_mul(bf16x2_to_f2(u[t][6]), s2), f2_mul(bf16x2_to_f2(u[t][7]), s2));
+    scale[t] = c;
+  }
+}
+
 // Weight block: 32 fp32 weights and their 32 channel factors D (offline).
 __device__ __forceinline__ void weight_block(const float (&wv)[32], const float (&dv)[32], uint4& codes,
                                              uint32_t& scale) {
