@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(256) quant_canonical_kernel(const uint16_t* __
                                                               const float* __restrict__ D,
                                                               uint8_t* __restrict__ codes,
                                                               uint8_t* __restrict__ scales, int M, int K) {
-  __shared__ __align__(16) float r[kKTile];
+  __shared__ __align__(16) float r[kRcpTile];
   const int kt = blockIdx.y;
   const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
   const int t = threadIdx.x >> 3, c = threadIdx.x & 7;
@@ -128,12 +128,12 @@ __global__ void __launch_bounds__(256) quant_canonical_kernel(const uint16_t* __
 #pragma unroll
     for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
   }
-  r[threadIdx.x] = __frcp_rn(__ldg(D + k0 + threadIdx.x));
+  r[rcp_index(threadIdx.x)] = __frcp_rn(__ldg(D + k0 + threadIdx.x));
   __syncthreads();
   if (m >= M) return;
   uint4 cv;
   uint32_t sc;
-  act_block(xv, r + c * kBlk, cv, sc);
+  act_block(xv, r + c * kRcpStride, cv, sc);
   *reinterpret_cast<uint4*>(codes + static_cast<int64_t>(m) * (K / 2) + (k0 + c * kBlk) / 2) = cv;
   scales[static_cast<int64_t>(m) * (K / kBlk) + k0 / kBlk + c] = static_cast<uint8_t>(sc);
 }
@@ -257,7 +257,7 @@ struct QuantParams {
 };
 
 __global__ void __launch_bounds__(256) quant_tiles_kernel(const __grid_constant__ QuantParams p) {
-  __shared__ __align__(16) float r[kKTile];
+  __shared__ __align__(16) float r[kRcpTile];
   pdl_trigger();  // the GEMM may start streaming weights; it waits for our results before reading them
   const int pm = blockIdx.x >> 2, sub = blockIdx.x & 3;
   const int kt = blockIdx.y;
@@ -282,11 +282,11 @@ __global__ void __launch_bounds__(256) quant_tiles_kernel(const __grid_constant_
 #pragma unroll
     for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
   }
-  r[threadIdx.x] = __frcp_rn(__ldg(p.D + static_cast<int64_t>(g) * p.K + k0 + threadIdx.x));
+  r[rcp_index(threadIdx.x)] = __frcp_rn(__ldg(p.D + static_cast<int64_t>(g) * p.K + k0 + threadIdx.x));
   __syncthreads();
   uint4 cv = make_uint4(0, 0, 0, 0);
   uint32_t sc = 0;
-  if (t < rows) act_block(xv, r + c * kBlk, cv, sc);
+  if (t < rows) act_block(xv, r + c * kRcpStride, cv, sc);
   const size_t tile = static_cast<size_t>(pm) * KT + kt;
   *reinterpret_cast<uint4*>(p.Aq + tile * kTileCodeBytes + code_chunk_offset(t, c)) = cv;
   p.As[tile * kTileSfBytes + sf_offset(t, c)] = static_cast<uint8_t>(sc);
@@ -674,7 +674,7 @@ struct Cfg {
   static constexpr int kGroups = BT <= 16 ? 2 : 1;
   static constexpr int kGroupThreads = kProWarps * 32 / kGroups;
   static constexpr int kRbufOff = kBarOff + 256;  // per group, two K tiles of reciprocals
-  static constexpr int kSmemBytes = 1024 + kRbufOff + kGroups * 2 * kKTile * 4;
+  static constexpr int kSmemBytes = 1024 + kRbufOff + kGroups * 2 * kRcpTile * 4;
   // scale factors from kSfCol, 16 columns per stage
   static constexpr int kSfCol = BT < 32 ? 32 : BT;
   static constexpr int kTmemCols = kSfCol + 16 * kStages <= 64 ? 64 : kSfCol + 16 * kStages <= 128 ? 128 : 256;
@@ -863,9 +863,9 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
     auto stage_body = [&](int jj, uint4 (&xv)[C::kTasks][2], const float (&d)[C::kRcp]) -> bool {
       const int j = grp + kG * jj, stage = j % kStages;
       const int slot = grp * 2 + (jj & 1);
-      float* r = rbuf + slot * kKTile;
+      float* r = rbuf + slot * kRcpTile;
 #pragma unroll
-      for (int e = 0; e < C::kRcp; ++e) r[gt + e * kGT] = __frcp_rn(d[e]);
+      for (int e = 0; e < C::kRcp; ++e) r[rcp_index(gt + e * kGT)] = __frcp_rn(d[e]);
       if (gt == 0) pro_flag[slot] = mbar_wait(&empty[stage], ((j / kStages) & 1) ^ 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
       named_bar_sync(2 + grp, kGT);
       if (!pro_flag[slot]) return false;
@@ -882,7 +882,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
 #pragma unroll
         for (int v = 0; v < kIlp; ++v) {
           const int task = gt + (u0 + v) * kGT, c = (task >> 1) & 7, half = task & 1;
-          rr[v] = r + c * kBlk + half * 16;
+          rr[v] = r + c * kRcpStride + half * 16;
         }
         act_half_blocks<kIlp>(*reinterpret_cast<const uint4(*)[kIlp][2]>(&xv[u0]), rr, cv, sc);
 #pragma unroll
