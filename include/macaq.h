@@ -78,9 +78,10 @@ int macaq_abi_version(void);
 /* ------------------------------------------------------------------ */
 
 /* Bytes of the prepared weight codes / scales for E experts of N x K.
- * Prepared weights are stored as tensor-core-ready tiles of 128 rows x 256 K:
- * codes 16384 bytes per tile (rows padded to a multiple of 128 with zero
- * codes), scales 1024 bytes per tile.  Returns 0 for invalid shapes. */
+ * Prepared weights are stored as tensor-core-ready tiles of 128 rows x 256 K
+ * (codes 16384 bytes per tile, scales 1024 bytes per tile), kept in pairs of
+ * row tiles per K tile so that 256 rows are contiguous; rows are padded to a
+ * multiple of 256 with zero codes and scales.  Returns 0 for invalid shapes. */
 size_t macaq_weight_code_bytes(int64_t E, int64_t N, int64_t K);
 size_t macaq_weight_scale_bytes(int64_t E, int64_t N, int64_t K);
 

@@ -49,7 +49,8 @@ def test_abi_version_and_status_strings(L):
 def test_weight_sizes(L):
     assert L.macaq_weight_code_bytes(1, 1024, 1024) == 1024 * 512
     assert L.macaq_weight_scale_bytes(1, 1024, 1024) == 1024 * 32
-    assert L.macaq_weight_code_bytes(2, 48, 256) == 2 * 128 * 128  # rows padded to 128
+    assert L.macaq_weight_code_bytes(2, 48, 256) == 2 * 256 * 128  # rows padded to 256 (image pairs)
+    assert L.macaq_weight_scale_bytes(1, 384, 512) == 512 * 16     # three images and a zero fourth
     assert L.macaq_weight_code_bytes(1, 1000, 1024) == 0           # N % 16 != 0
     assert L.macaq_weight_code_bytes(1, 1024, 1000) == 0           # K % 256 != 0
     assert L.macaq_weight_code_bytes(1025, 1024, 1024) == 0        # E > 1024

@@ -59,12 +59,27 @@ __device__ __forceinline__ uint16_t bf16_bits(float v) {
 }
 
 // ============================================================================
+// Image layouts
+// ============================================================================
+// Weights: 128-row x 256-K images (codes 16384 bytes, scales 1024) in pairs, so
+// the 256 rows of a wide GEMM tile are one contiguous run per K tile: image
+// (e, nt, kt) is number ((e * NT2 + nt / 2) * KT + kt) * 2 + nt % 2, with
+// NT2 = ceil(NT / 2) pairs per expert (an odd NT leaves a zero image).
+__host__ __device__ __forceinline__ size_t weight_image(int e, int nt, int kt, int NT2, int KT) {
+  return ((static_cast<size_t>(e) * NT2 + (nt >> 1)) * KT + kt) * 2 + (nt & 1);
+}
+// Activations (workspace): per (row tile, K tile) one image of codes followed by
+// its scales, so a stage's activation operand is a single copy.
+constexpr int kActImageBytes = kTileCodeBytes + kTileSfBytes;  // 17408
+
+// ============================================================================
 // Offline weight preparation and test-only kernels
 // ============================================================================
 // CTA = 32 rows x one 256-wide K tile (256 threads, one 32-block each).
 __global__ void __launch_bounds__(256) prep_weights_kernel(const float* __restrict__ W, const float* __restrict__ D,
                                                            uint8_t* __restrict__ Wq, uint8_t* __restrict__ Ws,
                                                            int N, int K, int NT) {
+  // NT: 128-row images per expert including an odd NT's zero image (2 * NT2)
   const int KT = K / kKTile;
   const int kt = blockIdx.y;
   const int t = threadIdx.x >> 3, c = threadIdx.x & 7;
@@ -87,12 +102,12 @@ __global__ void __launch_bounds__(256) prep_weights_kernel(const float* __restri
     }
     weight_block(wv, dv, codes, scale);
   }
-  const size_t tile = (static_cast<size_t>(e) * NT + nt) * KT + kt;
+  const size_t tile = weight_image(e, nt, kt, NT / 2, KT);
   *reinterpret_cast<uint4*>(Wq + tile * kTileCodeBytes + code_chunk_offset(r, c)) = codes;
   Ws[tile * kTileSfBytes + sf_offset(r, c)] = static_cast<uint8_t>(scale);
 }
 
-// Tile images -> canonical row-major codes/scales (tests only).
+// Weight images -> canonical row-major codes/scales (tests only); RT = NT2.
 __global__ void __launch_bounds__(256) export_tiles_kernel(const uint8_t* __restrict__ Tq,
                                                            const uint8_t* __restrict__ Ts,
                                                            uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
@@ -104,7 +119,7 @@ __global__ void __launch_bounds__(256) export_tiles_kernel(const uint8_t* __rest
   if (row_global >= rows_total) return;
   const int e = row_global / R, n = row_global % R;
   const int nt = n / kRowsTile, r = n % kRowsTile;
-  const size_t tile = (static_cast<size_t>(e) * RT + nt) * KT + kt;
+  const size_t tile = weight_image(e, nt, kt, RT, KT);
   const uint4 v = *reinterpret_cast<const uint4*>(Tq + tile * kTileCodeBytes + code_chunk_offset(r, c));
   const uint8_t s = Ts[tile * kTileSfBytes + sf_offset(r, c)];
   const int64_t row = static_cast<int64_t>(e) * R + n;
@@ -248,8 +263,7 @@ __device__ __forceinline__ int find_group(const int* gtp, int E, int pm) {
 struct QuantParams {
   const uint16_t* x;
   const float* D;        // [E, K]
-  uint8_t* Aq;           // [tiles][KT][16384]
-  uint8_t* As;           // [tiles][KT][1024]
+  uint8_t* Aq;           // [tiles][KT] activation images of kActImageBytes
   int M, K, E;
   const int64_t* goff;   // grouped tables (nullptr: dense)
   const int* gtp;
@@ -288,18 +302,18 @@ __global__ void __launch_bounds__(256) quant_tiles_kernel(const __grid_constant_
   uint32_t sc = 0;
   if (t < rows) act_block(xv, r + c * kRcpStride, cv, sc);
   const size_t tile = static_cast<size_t>(pm) * KT + kt;
-  *reinterpret_cast<uint4*>(p.Aq + tile * kTileCodeBytes + code_chunk_offset(t, c)) = cv;
-  p.As[tile * kTileSfBytes + sf_offset(t, c)] = static_cast<uint8_t>(sc);
+  uint8_t* img = p.Aq + tile * kActImageBytes;
+  *reinterpret_cast<uint4*>(img + code_chunk_offset(t, c)) = cv;
+  img[kTileCodeBytes + sf_offset(t, c)] = static_cast<uint8_t>(sc);
 }
 
 // ============================================================================
 // Persistent GEMM over tile images
 // ============================================================================
 struct GemmParams {
-  const uint8_t* Wq;  // weight images [E][NT][KT]
+  const uint8_t* Wq;  // weight images, pairs per K tile (weight_image)
   const uint8_t* Ws;
-  const uint8_t* Aq;  // activation images [tiles][KT]
-  const uint8_t* As;
+  const uint8_t* Aq;  // activation images [tiles][KT], kActImageBytes each
   uint16_t* y;        // bf16 [M, N]
   int M, N, K, NT, KT, E, MT;
   const int64_t* goff;  // grouped tables (nullptr: dense with MT tiles)
@@ -321,12 +335,13 @@ namespace gemm {
 constexpr int kMaxStages = 4;
 constexpr int kThreads = 320;  // warp 0 producer, warp 1 MMA, warps 2-9 epilogue
 constexpr int kTileN = 256;
-constexpr int kOffA = 0;                                    // activation codes, 128 rows
-constexpr int kOffB = kTileCodeBytes;                       // weight codes, 256 rows (two images)
-constexpr int kOffSfa = 3 * kTileCodeBytes;                 // activation scales
+// A stage takes three copies: the weight codes of an image pair (32 KB), the
+// activation image (codes then scales, 17 KB) and the pair's scales (2 KB).
+constexpr int kOffB = 0;                                    // weight codes, 256 rows (two images)
+constexpr int kOffA = 2 * kTileCodeBytes;                   // activation codes, 128 rows
+constexpr int kOffSfa = kOffA + kTileCodeBytes;             // activation scales (same copy)
 constexpr int kOffSfb = kOffSfa + kTileSfBytes;             // weight scales of the two images
 constexpr int kStageBytes = kOffSfb + 2 * kTileSfBytes;     // 52224
-constexpr int kHalfBBytes = kTileCodeBytes + kTileSfBytes;  // the second weight image of a stage
 constexpr int kStagingBytes = kRowsTile * 64 * 2;           // 128 rows x 64 columns of BF16, swizzled
 constexpr int kFixedBytes = kStagingBytes + 256;            // staging, barriers and flags
 // TMEM: the accumulator in columns 0-255; from column 256, 24 columns of scales per
@@ -354,7 +369,6 @@ static_assert(smem_bytes(0) <= kSmemLimit && smem_bytes(1024) <= kSmemLimit, "sh
 
 struct GemmTile {
   int g, m0, rows, pm, nt;  // nt: the first of the tile's two weight images
-  bool two;                 // the second image exists (N may end half-way through a tile)
 };
 
 __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int idx, int mtiles, const int64_t* goff,
@@ -362,7 +376,6 @@ __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int idx, int 
   GemmTile t;
   t.pm = idx % mtiles;
   t.nt = 2 * (idx / mtiles);
-  t.two = t.nt + 1 < p.NT;
   if (gtp == nullptr) {
     t.g = 0;
     t.m0 = t.pm * kRowsTile;
@@ -479,74 +492,63 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
   if (warp == 0) {
     // ================= producer: bulk copies of weight and activation images =================
     // A bulk-copy instruction holds up the path that issued it until the engine has
-    // taken its copy in, so the six copies of a stage are not issued one after
+    // taken its copy in, so the three copies of a stage are not issued one after
     // another: the warp stays converged and one predicated instruction starts them
     // together.  A single warp has no other work to hide its own latency behind, so
     // the source of each copy is stepped along, not recomputed, and worked out
     // before the wait.
     const int slots = my_tiles * KT;
     const int pre = min(S, slots);
-    // Copy c of a stage: 0 activation codes, 1 activation scales, 2 / 3 codes of the
-    // first / second weight image, 4 / 5 their scales.  Image (t, kt) of a kind sits at
-    // base + (t * KT + kt) * bytes.  Gives k tile 0 of this CTA's i-th output tile.
-    auto source = [&](int i, int c, const uint8_t*& src, uint32_t& bytes, uint32_t& doff, bool& on, bool& two) {
+    // Copy c of a stage: 0 activation image, 1 codes of the weight pair, 2 its
+    // scales.  Gives k tile 0 of this CTA's i-th output tile; k tile kt is
+    // kt * step further on.
+    auto source = [&](int i, int c, const uint8_t*& src, uint32_t& bytes, uint32_t& doff, uint32_t& step) {
       const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp);
-      const bool sf = c == 1 || c >= 4, second = c == 3 || c == 5;
-      two = t.two;
-      on = !second || t.two;
-      bytes = sf ? kTileSfBytes : kTileCodeBytes;
-      const size_t img = c < 2 ? static_cast<size_t>(t.pm)
-                               : static_cast<size_t>(t.g) * p.NT + t.nt + ((second && t.two) ? 1 : 0);
-      src = (c == 0 ? p.Aq : c == 1 ? p.As : sf ? p.Ws : p.Wq) + img * KT * bytes;
-      doff = c == 0   ? kOffA
-             : c == 1 ? kOffSfa
-             : c == 2 ? kOffB
-             : c == 3 ? kOffB + kTileCodeBytes
-             : c == 4 ? kOffSfb
-                      : kOffSfb + kTileSfBytes;
+      const size_t img = weight_image(t.g, t.nt, 0, p.NT2, KT);
+      bytes = c == 0 ? kActImageBytes : c == 1 ? 2 * kTileCodeBytes : 2 * kTileSfBytes;
+      step = c == 0 ? kActImageBytes : bytes;
+      src = c == 0 ? p.Aq + static_cast<size_t>(t.pm) * KT * kActImageBytes
+                   : (c == 1 ? p.Wq + img * kTileCodeBytes : p.Ws + img * kTileSfBytes);
+      doff = c == 0 ? kOffA : c == 1 ? kOffB : kOffSfb;
     };
     const uint8_t* src;
-    uint32_t bytes, doff;
-    bool on, two;
+    uint32_t bytes, doff, step;
     if (lane == 0)
-      for (int j = 0; j < pre; ++j) {
-        source(j / KT, 0, src, bytes, doff, on, two);
-        mbar_arrive_expect_tx(&full[j], two ? kStageBytes : kStageBytes - kHalfBBytes);
-      }
+      for (int j = 0; j < pre; ++j) mbar_arrive_expect_tx(&full[j], kStageBytes);
     __syncwarp();
-    {  // first stages: weights (lane 4s + w: copy 2 + w of stage s) before the quantiser's wait
-      const int j = min(lane >> 2, pre - 1);
-      source(j / KT, 2 + (lane & 3), src, bytes, doff, on, two);
-      bulk_g2s_if(on && lane < 4 * pre, smem + j * kStageBytes + doff, src + (j % KT) * bytes, bytes, &full[j]);
+    {  // first stages: weights (lane 2s + w: copy 1 + w of stage s) before the quantiser's wait
+      const int j = min(lane >> 1, pre - 1);
+      source(j / KT, 1 + (lane & 1), src, bytes, doff, step);
+      bulk_g2s_if(lane < 2 * pre, smem + j * kStageBytes + doff, src + (j % KT) * step, bytes, &full[j]);
     }
     if (p.wait_for_producer) pdl_wait();
-    {  // then their activations (lane 2s + a: copy a of stage s)
-      const int j = min(lane >> 1, pre - 1);
-      source(j / KT, lane & 1, src, bytes, doff, on, two);
-      bulk_g2s_if(lane < 2 * pre, smem + j * kStageBytes + doff, src + (j % KT) * bytes, bytes, &full[j]);
+    {  // then their activations (lane s: copy 0 of stage s)
+      const int j = min(lane, pre - 1);
+      source(j / KT, 0, src, bytes, doff, step);
+      bulk_g2s_if(lane < pre, smem + j * kStageBytes + doff, src + (j % KT) * step, bytes, &full[j]);
     }
-    // from then on lane c < 6 streams copy c of every stage
-    const int c = lane < 6 ? lane : 0;
+    // from then on lane c < 3 streams copy c of every stage
+    const int c = lane < 3 ? lane : 0;
     int kt = pre % KT, i = pre / KT, stage = 0;
     uint32_t phase = 1;  // slots from `pre` on reuse stages released once before
-    if (pre < slots) source(i, c, src, bytes, doff, on, two);
+    if (pre < slots) source(i, c, src, bytes, doff, step);
     for (int j = pre; j < slots; ++j) {
       int ok = 1;
       if (lane == 0) {
         ok = mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
-        if (ok) mbar_arrive_expect_tx(&full[stage], two ? kStageBytes : kStageBytes - kHalfBBytes);
+        if (ok) mbar_arrive_expect_tx(&full[stage], kStageBytes);
       }
       __syncwarp();  // the stage is free for every lane, not only the one that waited
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      bulk_g2s_if(on && lane < 6, smem + stage * kStageBytes + doff, src + kt * bytes, bytes, &full[stage]);
+      bulk_g2s_if(lane < 3, smem + stage * kStageBytes + doff, src + kt * step, bytes, &full[stage]);
       if (++stage == S) {
         stage = 0;
         phase ^= 1;
       }
       if (++kt == KT) {
         kt = 0;
-        if (j + 1 < slots) source(++i, c, src, bytes, doff, on, two);
+        if (j + 1 < slots) source(++i, c, src, bytes, doff, step);
       }
     }
   } else if (warp == 1) {
@@ -764,7 +766,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
       __syncwarp();  // the stage is free for every lane, not only the one that waited
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
-      const size_t wt = static_cast<size_t>(nt) * p.KT + kt;
+      const size_t wt = weight_image(0, nt, kt, (p.NT + 1) / 2, p.KT);
       uint8_t* sb = smem + stage * C::kStageBytes;
       const bool sf = lane & 1;
       bulk_g2s_if(lane < 2, sf ? sb + C::kOffSfa : sb, sf ? p.Ws + wt * kTileSfBytes : p.Wq + wt * kTileCodeBytes,
@@ -1043,6 +1045,7 @@ bool valid_nk(int64_t N, int64_t K) {
 }
 
 int64_t pad128(int64_t n) { return (n + 127) / 128 * 128; }
+int64_t pad256(int64_t n) { return (n + 255) / 256 * 256; }
 size_t align256(size_t n) { return (n + 255) / 256 * 256; }
 
 template <typename... KArgs, typename... Args>
@@ -1163,18 +1166,17 @@ int launch_fused(const FusedParams& p, const FusedPlan& plan, cudaStream_t st) {
 
 // ---- quantise-once workspace layouts ----
 struct DenseWs {
-  size_t act_codes, act_scales, total;
+  size_t act, total;
 };
 DenseWs dense_ws(int64_t M, int64_t K) {
   const size_t tiles = static_cast<size_t>(pad128(M) / 128) * (K / 256);
   DenseWs w;
-  w.act_codes = kWsReserved;
-  w.act_scales = w.act_codes + tiles * kTileCodeBytes;
-  w.total = w.act_scales + tiles * kTileSfBytes;
+  w.act = kWsReserved;
+  w.total = w.act + tiles * kActImageBytes;
   return w;
 }
 struct GroupedWs {
-  size_t goff, gtp, valid, act_codes, act_scales, total;
+  size_t goff, gtp, valid, act, total;
   int tiles_upper;
 };
 GroupedWs grouped_ws(int64_t M, int64_t K, int64_t E) {
@@ -1184,9 +1186,8 @@ GroupedWs grouped_ws(int64_t M, int64_t K, int64_t E) {
   w.goff = kWsReserved;
   w.gtp = align256(w.goff + (E + 1) * 8);
   w.valid = align256(w.gtp + (E + 1) * 4);
-  w.act_codes = align256(w.valid + 16);
-  w.act_scales = w.act_codes + static_cast<size_t>(w.tiles_upper) * KT * kTileCodeBytes;
-  w.total = w.act_scales + static_cast<size_t>(w.tiles_upper) * KT * kTileSfBytes;
+  w.act = align256(w.valid + 16);
+  w.total = w.act + static_cast<size_t>(w.tiles_upper) * KT * kActImageBytes;
   return w;
 }
 
@@ -1219,12 +1220,12 @@ int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, c
   const DenseWs w = dense_ws(M, K);
   const int MT = static_cast<int>(pad128(M) / 128), KT = static_cast<int>(K / 256);
   QuantParams qp{};
-  qp.x = x; qp.D = D; qp.Aq = ws + w.act_codes; qp.As = ws + w.act_scales;
+  qp.x = x; qp.D = D; qp.Aq = ws + w.act;
   qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = 1;
   if (launch_ex(quant_tiles_kernel, dim3(MT * 4, KT), dim3(256), 0, st, pdl, 1, qp) != cudaSuccess)
     return MACAQ_ERR_CUDA;
   GemmParams gp{};
-  gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.As = qp.As; gp.y = y;
+  gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.y = y;
   gp.M = static_cast<int>(M); gp.N = static_cast<int>(N); gp.K = static_cast<int>(K);
   gp.NT = static_cast<int>(pad128(N) / 128); gp.KT = KT; gp.E = 1; gp.MT = MT;
   gp.NT2 = (gp.NT + 1) / 2; gp.stages = gemm::stages_for(0);
@@ -1282,12 +1283,12 @@ int macaq_abi_version(void) { return MACAQ_ABI_VERSION; }
 
 size_t macaq_weight_code_bytes(int64_t E, int64_t N, int64_t K) {
   if (E < 1 || E > kMaxGroups || !valid_nk(N, K)) return 0;
-  return static_cast<size_t>(E) * pad128(N) * (K / 2);
+  return static_cast<size_t>(E) * pad256(N) * (K / 2);
 }
 
 size_t macaq_weight_scale_bytes(int64_t E, int64_t N, int64_t K) {
   if (E < 1 || E > kMaxGroups || !valid_nk(N, K)) return 0;
-  return static_cast<size_t>(E) * pad128(N) * (K / 32);
+  return static_cast<size_t>(E) * pad256(N) * (K / 32);
 }
 
 int macaq_prepare_weights(const float* W, const float* D, int64_t E, int64_t N, int64_t K, uint8_t* Wq, uint8_t* Ws,
@@ -1312,9 +1313,9 @@ int macaq_prepare_weights(const float* W, const float* D, int64_t E, int64_t N, 
     return MACAQ_ERR_CUDA;
   for (float d : hD)
     if (!(d != 0.0f) || !std::isfinite(d)) return MACAQ_ERR_BAD_D;
-  const int NT = static_cast<int>(pad128(N) / 128);
-  dim3 grid(static_cast<unsigned>(E * NT * 4), static_cast<unsigned>(K / 256));
-  prep_weights_kernel<<<grid, 256, 0, s>>>(W, D, Wq, Ws, static_cast<int>(N), static_cast<int>(K), NT);
+  const int NTP = static_cast<int>(pad256(N) / 128);  // images per expert, pairs complete
+  dim3 grid(static_cast<unsigned>(E * NTP * 4), static_cast<unsigned>(K / 256));
+  prep_weights_kernel<<<grid, 256, 0, s>>>(W, D, Wq, Ws, static_cast<int>(N), static_cast<int>(K), NTP);
   return cudaPeekAtLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
@@ -1379,13 +1380,13 @@ int macaq_grouped_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const
   if (cudaPeekAtLastError() != cudaSuccess) return MACAQ_ERR_CUDA;
   const int KT = static_cast<int>(K / 256);
   QuantParams qp{};
-  qp.x = x; qp.D = D; qp.Aq = ws + w.act_codes; qp.As = ws + w.act_scales;
+  qp.x = x; qp.D = D; qp.Aq = ws + w.act;
   qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = static_cast<int>(E);
   qp.goff = goff; qp.gtp = gtp; qp.valid = valid;
   if (launch_ex(quant_tiles_kernel, dim3(w.tiles_upper * 4, KT), dim3(256), 0, s, true, 1, qp) != cudaSuccess)
     return MACAQ_ERR_CUDA;
   GemmParams gp{};
-  gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.As = qp.As; gp.y = y;
+  gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.y = y;
   gp.M = static_cast<int>(M); gp.N = static_cast<int>(N); gp.K = static_cast<int>(K);
   gp.NT = static_cast<int>(pad128(N) / 128); gp.KT = KT; gp.E = static_cast<int>(E);
   gp.NT2 = (gp.NT + 1) / 2; gp.stages = gemm::stages_for(static_cast<int>(E));
@@ -1422,7 +1423,7 @@ int macaq_export_weights(const uint8_t* Wq, const uint8_t* Ws, uint8_t* codes, u
   if (st != MACAQ_OK) return st;
   dim3 grid(static_cast<unsigned>((E * N + 31) / 32), static_cast<unsigned>(K / 256));
   export_tiles_kernel<<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      Wq, Ws, codes, scales, static_cast<int>(N), static_cast<int>(K), static_cast<int>(pad128(N) / 128),
+      Wq, Ws, codes, scales, static_cast<int>(N), static_cast<int>(K), static_cast<int>(pad256(N) / 256),
       static_cast<int>(E * N));
   return cudaPeekAtLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
