@@ -211,7 +211,8 @@ __device__ __forceinline__ int64_t block_excl_scan(int64_t v, int64_t* scratch, 
 // group) and *valid; on a violation also *status.
 __global__ void __launch_bounds__(1024) group_tables_kernel(const int64_t* __restrict__ gl, int type, int E, int M,
                                                             int64_t* __restrict__ goff, int* __restrict__ gtp,
-                                                            int* __restrict__ valid, int32_t* status) {
+                                                            int4* __restrict__ tinfo, int* __restrict__ valid,
+                                                            int32_t* status) {
   __shared__ int64_t scratch[72];
   const int g = threadIdx.x;
   int64_t cnt = 0;
@@ -236,6 +237,11 @@ __global__ void __launch_bounds__(1024) group_tables_kernel(const int64_t* __res
       goff[E] = rows_total;
       gtp[E] = static_cast<int>(tiles_total);
     }
+    // per row tile: {group, first row, rows}, one load for the quantiser
+    if (g < E && !bad)
+      for (int64_t j = 0; j * kRowsTile < cnt; ++j)
+        tinfo[tb + j] = make_int4(g, static_cast<int>(rb + j * kRowsTile),
+                                  static_cast<int>(cnt - j * kRowsTile < kRowsTile ? cnt - j * kRowsTile : kRowsTile), 0);
   }
   if (g == 0) {
     *valid = bad ? 0 : 1;
@@ -256,55 +262,93 @@ __device__ __forceinline__ int find_group(const int* gtp, int E, int pm) {
 // ============================================================================
 // Quantise-once: activation prologue over every row into tile images
 // ============================================================================
-// CTA = 32 rows of one 128-row tile x one K tile.  Dense: tile pm holds rows
-// [128 pm, 128 pm + 128).  Grouped: tile pm belongs to the group g with
-// gtp[g] <= pm < gtp[g+1] and holds that group's rows starting at
-// goff[g] + 128 (pm - gtp[g]); rows past the group's end are zero.
+// Work unit = 32 rows of one 128-row tile x one K tile (one 32-element block per
+// thread).  Dense: tile pm holds rows [128 pm, 128 pm + 128).  Grouped: tile pm
+// belongs to the group g with gtp[g] <= pm < gtp[g+1] and holds that group's
+// rows starting at goff[g] + 128 (pm - gtp[g]); rows past the group's end are zero.
+// The grid is persistent: each CTA walks units blockIdx.x, + gridDim.x, ..., with
+// the next unit's activations and D loaded while the current unit is computed.
 struct QuantParams {
   const uint16_t* x;
   const float* D;        // [E, K]
   uint8_t* Aq;           // [tiles][KT] activation images of kActImageBytes
-  int M, K, E;
+  int M, K, E, MT;       // MT: dense row tiles
   const int64_t* goff;   // grouped tables (nullptr: dense)
   const int* gtp;
+  const int4* tinfo;     // grouped: per row tile {group, first row, rows}
   const int* valid;
 };
 
-__global__ void __launch_bounds__(256) quant_tiles_kernel(const __grid_constant__ QuantParams p) {
-  __shared__ __align__(16) float r[kRcpTile];
+__global__ void __launch_bounds__(256, 3) quant_tiles_kernel(const __grid_constant__ QuantParams p) {
+  __shared__ __align__(16) float r[2][kRcpTile];
   pdl_trigger();  // the GEMM may start streaming weights; it waits for our results before reading them
-  const int pm = blockIdx.x >> 2, sub = blockIdx.x & 3;
-  const int kt = blockIdx.y;
+  pdl_wait();     // x (and the grouped tables) may come from the preceding kernels
   const int KT = p.K / kKTile;
-  int g = 0, base, rows;
+  int tiles = p.MT;
   if (p.gtp != nullptr) {
-    pdl_wait();  // tables come from the preceding kernel
-    if (*p.valid == 0 || pm >= p.gtp[p.E]) return;
-    g = find_group(p.gtp, p.E, pm);
-    base = static_cast<int>(p.goff[g]) + (pm - p.gtp[g]) * kRowsTile;
-    rows = min(kRowsTile, static_cast<int>(p.goff[g + 1]) - base);
-  } else {
-    pdl_wait();  // x may come from the previous kernel on the stream
-    base = pm * kRowsTile;
-    rows = min(kRowsTile, p.M - base);
+    if (*p.valid == 0) return;
+    tiles = p.gtp[p.E];
   }
-  const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
-  const int t = sub * 32 + (threadIdx.x >> 3), c = threadIdx.x & 7;
-  uint4 xv[4] = {};
-  if (t < rows) {  // issue the activation loads before the reciprocals
-    const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(base + t) * p.K + k0 + c * kBlk);
+  const int units = tiles * 4 * KT;
+  const int tr = threadIdx.x >> 3, c = threadIdx.x & 7;
+  // unit u: kt = u % KT, sub = (u / KT) % 4, pm = u / (4 KT); t = row within the tile
+  struct Unit {
+    uint8_t* img;  // the unit's activation image
+    int t;         // this thread's row in the tile
+    bool live;     // the row exists
+  };
+  // works out unit u and issues its loads (x block, D value)
+  auto fetch = [&](int u, Unit& w, uint4 (&xv)[4], float& d) {
+    const int kt = u % KT, q = u / KT, pm = q >> 2;
+    w.t = (q & 3) * 32 + tr;
+    int base, rows, g = 0;
+    if (p.gtp != nullptr) {
+      const int4 ti = p.tinfo[pm];
+      g = ti.x;
+      base = ti.y;
+      rows = ti.z;
+    } else {
+      base = pm * kRowsTile;
+      rows = min(kRowsTile, p.M - base);
+    }
+    w.live = w.t < rows;
+    w.img = p.Aq + (static_cast<size_t>(pm) * KT + kt) * kActImageBytes;
+    const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
+    xv[0] = xv[1] = xv[2] = xv[3] = make_uint4(0, 0, 0, 0);
+    if (w.live) {
+      const uint4* src =
+          reinterpret_cast<const uint4*>(p.x + (static_cast<int64_t>(base) + w.t) * p.K + k0 + c * kBlk);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
+      for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
+    }
+    d = __ldg(p.D + static_cast<int64_t>(g) * p.K + k0 + threadIdx.x);
+  };
+  int u = blockIdx.x;
+  if (u >= units) return;
+  Unit wa;
+  uint4 xa[4];
+  float da;
+  fetch(u, wa, xa, da);
+  for (int buf = 0; u < units; u += gridDim.x, buf ^= 1) {
+    const int un = u + gridDim.x;
+    Unit wb{};
+    uint4 xb[4];
+    float db = 0.f;
+    if (un < units) fetch(un, wb, xb, db);
+    r[buf][rcp_index(threadIdx.x)] = __frcp_rn(da);
+    __syncthreads();  // also: no thread still reads r[buf] from two units back
+    uint4 cv = make_uint4(0, 0, 0, 0);
+    uint32_t sc = 0;
+    if (wa.live) act_block(xa, r[buf] + c * kRcpStride, cv, sc);
+    *reinterpret_cast<uint4*>(wa.img + code_chunk_offset(wa.t, c)) = cv;
+    wa.img[kTileCodeBytes + sf_offset(wa.t, c)] = static_cast<uint8_t>(sc);
+    if (un < units) {
+      wa = wb;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xa[i] = xb[i];
+      da = db;
+    }
   }
-  r[rcp_index(threadIdx.x)] = __frcp_rn(__ldg(p.D + static_cast<int64_t>(g) * p.K + k0 + threadIdx.x));
-  __syncthreads();
-  uint4 cv = make_uint4(0, 0, 0, 0);
-  uint32_t sc = 0;
-  if (t < rows) act_block(xv, r + c * kRcpStride, cv, sc);
-  const size_t tile = static_cast<size_t>(pm) * KT + kt;
-  uint8_t* img = p.Aq + tile * kActImageBytes;
-  *reinterpret_cast<uint4*>(img + code_chunk_offset(t, c)) = cv;
-  img[kTileCodeBytes + sf_offset(t, c)] = static_cast<uint8_t>(sc);
 }
 
 // ============================================================================
@@ -1176,7 +1220,7 @@ DenseWs dense_ws(int64_t M, int64_t K) {
   return w;
 }
 struct GroupedWs {
-  size_t goff, gtp, valid, act, total;
+  size_t goff, gtp, valid, tinfo, act, total;
   int tiles_upper;
 };
 GroupedWs grouped_ws(int64_t M, int64_t K, int64_t E) {
@@ -1186,7 +1230,8 @@ GroupedWs grouped_ws(int64_t M, int64_t K, int64_t E) {
   w.goff = kWsReserved;
   w.gtp = align256(w.goff + (E + 1) * 8);
   w.valid = align256(w.gtp + (E + 1) * 4);
-  w.act = align256(w.valid + 16);
+  w.tinfo = align256(w.valid + 16);
+  w.act = align256(w.tinfo + static_cast<size_t>(w.tiles_upper) * 16);
   w.total = w.act + static_cast<size_t>(w.tiles_upper) * KT * kActImageBytes;
   return w;
 }
@@ -1212,6 +1257,12 @@ int check_ws(void* ws, size_t ws_bytes, size_t need, const void* y, size_t ybyte
   return MACAQ_OK;
 }
 
+// Persistent quantiser grid: three CTAs per SM at most, no more than the units.
+int quant_grid(int tiles, int KT, int sms) {
+  const int64_t units = static_cast<int64_t>(tiles) * 4 * KT;
+  return static_cast<int>(std::min<int64_t>(units, static_cast<int64_t>(sms) * 3));
+}
+
 // Dense quantise-once: the quantiser over all rows, then the GEMM (launched as
 // a programmatic dependent of the quantiser when `pdl`).
 int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y,
@@ -1221,8 +1272,8 @@ int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, c
   const int MT = static_cast<int>(pad128(M) / 128), KT = static_cast<int>(K / 256);
   QuantParams qp{};
   qp.x = x; qp.D = D; qp.Aq = ws + w.act;
-  qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = 1;
-  if (launch_ex(quant_tiles_kernel, dim3(MT * 4, KT), dim3(256), 0, st, pdl, 1, qp) != cudaSuccess)
+  qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = 1; qp.MT = MT;
+  if (launch_ex(quant_tiles_kernel, dim3(quant_grid(MT, KT, sms)), dim3(256), 0, st, pdl, 1, qp) != cudaSuccess)
     return MACAQ_ERR_CUDA;
   GemmParams gp{};
   gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.y = y;
@@ -1375,15 +1426,17 @@ int macaq_grouped_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const
   int64_t* goff = reinterpret_cast<int64_t*>(ws + w.goff);
   int* gtp = reinterpret_cast<int*>(ws + w.gtp);
   int* valid = reinterpret_cast<int*>(ws + w.valid);
+  int4* tinfo = reinterpret_cast<int4*>(ws + w.tinfo);
   group_tables_kernel<<<1, 1024, 0, s>>>(group_list, group_list_type, static_cast<int>(E), static_cast<int>(M),
-                                         goff, gtp, valid, status);
+                                         goff, gtp, tinfo, valid, status);
   if (cudaPeekAtLastError() != cudaSuccess) return MACAQ_ERR_CUDA;
   const int KT = static_cast<int>(K / 256);
   QuantParams qp{};
   qp.x = x; qp.D = D; qp.Aq = ws + w.act;
   qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = static_cast<int>(E);
-  qp.goff = goff; qp.gtp = gtp; qp.valid = valid;
-  if (launch_ex(quant_tiles_kernel, dim3(w.tiles_upper * 4, KT), dim3(256), 0, s, true, 1, qp) != cudaSuccess)
+  qp.goff = goff; qp.gtp = gtp; qp.tinfo = tinfo; qp.valid = valid;
+  if (launch_ex(quant_tiles_kernel, dim3(quant_grid(w.tiles_upper, KT, sms)), dim3(256), 0, s, true, 1, qp) !=
+      cudaSuccess)
     return MACAQ_ERR_CUDA;
   GemmParams gp{};
   gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.y = y;
