@@ -264,10 +264,12 @@ __device__ __forceinline__ int find_group(const int* gtp, int E, int pm) {
 // ============================================================================
 // Work unit = 32 rows of one 128-row tile x one K tile (one 32-element block per
 // thread).  Dense: tile pm holds rows [128 pm, 128 pm + 128).  Grouped: tile pm
-// belongs to the group g with gtp[g] <= pm < gtp[g+1] and holds that group's
-// rows starting at goff[g] + 128 (pm - gtp[g]); rows past the group's end are zero.
-// The grid is persistent: each CTA walks units blockIdx.x, + gridDim.x, ..., with
-// the next unit's activations and D loaded while the current unit is computed.
+// belongs to group g and holds that group's rows from a first row given by the
+// per-tile table; rows past the group's end are zero.  The grid is persistent:
+// each CTA walks units blockIdx.x, + gridDim.x, ...; every thread keeps the
+// activations of its next kQuantAhead units in flight with cp.async into its own
+// slots of a shared-memory ring (no registers held), so HBM streams while the
+// ALUs work.
 struct QuantParams {
   const uint16_t* x;
   const float* D;        // [E, K]
@@ -279,7 +281,13 @@ struct QuantParams {
   const int* valid;
 };
 
+constexpr int kQuantStages = 4;                 // ring slots: the current unit and three ahead
+constexpr int kQuantAhead = kQuantStages - 1;
+constexpr int kQuantSlotBytes = 256 * 64;       // one unit: 256 threads x one 32-element block
+constexpr int kQuantSmem = kQuantStages * kQuantSlotBytes;
+
 __global__ void __launch_bounds__(256, 3) quant_tiles_kernel(const __grid_constant__ QuantParams p) {
+  extern __shared__ __align__(16) uint8_t qsmem[];  // ring [kQuantStages][256][64]
   __shared__ __align__(16) float r[2][kRcpTile];
   pdl_trigger();  // the GEMM may start streaming weights; it waits for our results before reading them
   pdl_wait();     // x (and the grouped tables) may come from the preceding kernels
@@ -291,14 +299,15 @@ __global__ void __launch_bounds__(256, 3) quant_tiles_kernel(const __grid_consta
   }
   const int units = tiles * 4 * KT;
   const int tr = threadIdx.x >> 3, c = threadIdx.x & 7;
-  // unit u: kt = u % KT, sub = (u / KT) % 4, pm = u / (4 KT); t = row within the tile
   struct Unit {
-    uint8_t* img;  // the unit's activation image
-    int t;         // this thread's row in the tile
-    bool live;     // the row exists
+    uint8_t* img;     // the unit's activation image
+    const float* dp;  // D of this thread's channel
+    int t;            // this thread's row in the tile
+    bool live;        // the row exists
   };
-  // works out unit u and issues its loads (x block, D value)
-  auto fetch = [&](int u, Unit& w, uint4 (&xv)[4], float& d) {
+  // unit u: kt = u % KT, sub = (u / KT) % 4, pm = u / (4 KT); issues its activation copy into `slot`
+  auto fetch = [&](int u, int slot) {
+    Unit w;
     const int kt = u % KT, q = u / KT, pm = q >> 2;
     w.t = (q & 3) * 32 + tr;
     int base, rows, g = 0;
@@ -314,41 +323,57 @@ __global__ void __launch_bounds__(256, 3) quant_tiles_kernel(const __grid_consta
     w.live = w.t < rows;
     w.img = p.Aq + (static_cast<size_t>(pm) * KT + kt) * kActImageBytes;
     const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
-    xv[0] = xv[1] = xv[2] = xv[3] = make_uint4(0, 0, 0, 0);
+    w.dp = p.D + static_cast<int64_t>(g) * p.K + k0 + threadIdx.x;
     if (w.live) {
-      const uint4* src =
-          reinterpret_cast<const uint4*>(p.x + (static_cast<int64_t>(base) + w.t) * p.K + k0 + c * kBlk);
+      const uint16_t* src = p.x + (static_cast<int64_t>(base) + w.t) * p.K + k0 + c * kBlk;
+      uint8_t* dst = qsmem + (slot * 256 + threadIdx.x) * 64;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
+      for (int i = 0; i < 4; ++i) cp_async16(dst + 16 * i, src + 8 * i);
     }
-    d = __ldg(p.D + static_cast<int64_t>(g) * p.K + k0 + threadIdx.x);
+    cp_async_commit();  // one group per unit, empty when the row does not exist
+    return w;
   };
   int u = blockIdx.x;
   if (u >= units) return;
-  Unit wa;
-  uint4 xa[4];
-  float da;
-  fetch(u, wa, xa, da);
-  for (int buf = 0; u < units; u += gridDim.x, buf ^= 1) {
-    const int un = u + gridDim.x;
-    Unit wb{};
-    uint4 xb[4];
-    float db = 0.f;
-    if (un < units) fetch(un, wb, xb, db);
-    r[buf][rcp_index(threadIdx.x)] = __frcp_rn(da);
-    __syncthreads();  // also: no thread still reads r[buf] from two units back
-    uint4 cv = make_uint4(0, 0, 0, 0);
-    uint32_t sc = 0;
-    if (wa.live) act_block(xa, r[buf] + c * kRcpStride, cv, sc);
-    *reinterpret_cast<uint4*>(wa.img + code_chunk_offset(wa.t, c)) = cv;
-    wa.img[kTileCodeBytes + sf_offset(wa.t, c)] = static_cast<uint8_t>(sc);
-    if (un < units) {
-      wa = wb;
+  Unit ring[kQuantStages];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) xa[i] = xb[i];
-      da = db;
+  for (int s = 0; s < kQuantAhead; ++s) {
+    const int us = u + s * static_cast<int>(gridDim.x);
+    if (us < units) ring[s] = fetch(us, s);
+    else cp_async_commit();
+  }
+  float d = __ldg(ring[0].dp);
+  // unit i of this CTA uses ring slot i % kQuantStages; unrolled so slots are static
+  while (u < units) {
+#pragma unroll
+    for (int k = 0; k < kQuantStages; ++k) {
+      if (u >= units) break;
+      {  // the unit kQuantAhead ahead goes into the slot freed last iteration
+        const int ua = u + kQuantAhead * static_cast<int>(gridDim.x);
+        const int sa = (k + kQuantAhead) % kQuantStages;
+        if (ua < units) ring[sa] = fetch(ua, sa);
+        else cp_async_commit();
+      }
+      const Unit w = ring[k];
+      const int un = u + static_cast<int>(gridDim.x);
+      const float dn = un < units ? __ldg(ring[(k + 1) % kQuantStages].dp) : 0.f;
+      r[k & 1][rcp_index(threadIdx.x)] = __frcp_rn(d);
+      cp_async_wait<kQuantAhead>();  // this thread's copy of this unit has landed
+      __syncthreads();               // every reciprocal written; r[k & 1] of two units back no longer read
+      uint4 cv = make_uint4(0, 0, 0, 0);
+      uint32_t sc = 0;
+      if (w.live) {
+        const uint4* xs = reinterpret_cast<const uint4*>(qsmem + (k * 256 + threadIdx.x) * 64);
+        const uint4 xv[4] = {xs[0], xs[1], xs[2], xs[3]};
+        act_block(xv, r[k & 1] + c * kRcpStride, cv, sc);
+      }
+      *reinterpret_cast<uint4*>(w.img + code_chunk_offset(w.t, c)) = cv;
+      w.img[kTileCodeBytes + sf_offset(w.t, c)] = static_cast<uint8_t>(sc);
+      d = dn;
+      u = un;
     }
   }
+  cp_async_wait<0>();  // no copy may still be writing this CTA's shared memory at exit
 }
 
 // ============================================================================
@@ -1071,6 +1096,8 @@ int current_device(int& dev, int& sms) {
                                     fused::Cfg<64>::kSmemBytes) == cudaSuccess;
     ok = ok && cudaFuncSetAttribute(fused_small_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     fused::Cfg<128>::kSmemBytes) == cudaSuccess;
+    ok = ok && cudaFuncSetAttribute(quant_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmem) ==
+                   cudaSuccess;
     if (!ok) return MACAQ_ERR_CUDA;
     s.attrs_set = true;
   }
@@ -1273,7 +1300,8 @@ int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, c
   QuantParams qp{};
   qp.x = x; qp.D = D; qp.Aq = ws + w.act;
   qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = 1; qp.MT = MT;
-  if (launch_ex(quant_tiles_kernel, dim3(quant_grid(MT, KT, sms)), dim3(256), 0, st, pdl, 1, qp) != cudaSuccess)
+  if (launch_ex(quant_tiles_kernel, dim3(quant_grid(MT, KT, sms)), dim3(256), kQuantSmem, st, pdl, 1, qp) !=
+      cudaSuccess)
     return MACAQ_ERR_CUDA;
   GemmParams gp{};
   gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.y = y;
@@ -1435,8 +1463,8 @@ int macaq_grouped_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const
   qp.x = x; qp.D = D; qp.Aq = ws + w.act;
   qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = static_cast<int>(E);
   qp.goff = goff; qp.gtp = gtp; qp.tinfo = tinfo; qp.valid = valid;
-  if (launch_ex(quant_tiles_kernel, dim3(quant_grid(w.tiles_upper, KT, sms)), dim3(256), 0, s, true, 1, qp) !=
-      cudaSuccess)
+  if (launch_ex(quant_tiles_kernel, dim3(quant_grid(w.tiles_upper, KT, sms)), dim3(256), kQuantSmem, s, true, 1,
+                qp) != cudaSuccess)
     return MACAQ_ERR_CUDA;
   GemmParams gp{};
   gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.y = y;
