@@ -281,12 +281,12 @@ struct QuantParams {
   const int* valid;
 };
 
-constexpr int kQuantStages = 4;                 // ring slots: the current unit and three ahead
+constexpr int kQuantStages = 3;                 // ring slots: the current unit and two ahead
 constexpr int kQuantAhead = kQuantStages - 1;
 constexpr int kQuantSlotBytes = 256 * 64;       // one unit: 256 threads x one 32-element block
 constexpr int kQuantSmem = kQuantStages * kQuantSlotBytes;
 
-__global__ void __launch_bounds__(256, 3) quant_tiles_kernel(const __grid_constant__ QuantParams p) {
+__global__ void __launch_bounds__(256, 4) quant_tiles_kernel(const __grid_constant__ QuantParams p) {
   extern __shared__ __align__(16) uint8_t qsmem[];  // ring [kQuantStages][256][64]
   __shared__ __align__(16) float r[2][kRcpTile];
   pdl_trigger();  // the GEMM may start streaming weights; it waits for our results before reading them
@@ -343,6 +343,7 @@ __global__ void __launch_bounds__(256, 3) quant_tiles_kernel(const __grid_consta
     else cp_async_commit();
   }
   float d = __ldg(ring[0].dp);
+  int buf = 0;  // reciprocal buffer of this unit: alternates unit by unit
   // unit i of this CTA uses ring slot i % kQuantStages; unrolled so slots are static
   while (u < units) {
 #pragma unroll
@@ -357,20 +358,21 @@ __global__ void __launch_bounds__(256, 3) quant_tiles_kernel(const __grid_consta
       const Unit w = ring[k];
       const int un = u + static_cast<int>(gridDim.x);
       const float dn = un < units ? __ldg(ring[(k + 1) % kQuantStages].dp) : 0.f;
-      r[k & 1][rcp_index(threadIdx.x)] = __frcp_rn(d);
+      r[buf][rcp_index(threadIdx.x)] = __frcp_rn(d);
       cp_async_wait<kQuantAhead>();  // this thread's copy of this unit has landed
-      __syncthreads();               // every reciprocal written; r[k & 1] of two units back no longer read
+      __syncthreads();               // every reciprocal written; r[buf] of two units back no longer read
       uint4 cv = make_uint4(0, 0, 0, 0);
       uint32_t sc = 0;
       if (w.live) {
         const uint4* xs = reinterpret_cast<const uint4*>(qsmem + (k * 256 + threadIdx.x) * 64);
         const uint4 xv[4] = {xs[0], xs[1], xs[2], xs[3]};
-        act_block(xv, r[k & 1] + c * kRcpStride, cv, sc);
+        act_block(xv, r[buf] + c * kRcpStride, cv, sc);
       }
       *reinterpret_cast<uint4*>(w.img + code_chunk_offset(w.t, c)) = cv;
       w.img[kTileCodeBytes + sf_offset(w.t, c)] = static_cast<uint8_t>(sc);
       d = dn;
       u = un;
+      buf ^= 1;
     }
   }
   cp_async_wait<0>();  // no copy may still be writing this CTA's shared memory at exit
@@ -1284,10 +1286,10 @@ int check_ws(void* ws, size_t ws_bytes, size_t need, const void* y, size_t ybyte
   return MACAQ_OK;
 }
 
-// Persistent quantiser grid: three CTAs per SM at most, no more than the units.
+// Persistent quantiser grid: four CTAs per SM at most, no more than the units.
 int quant_grid(int tiles, int KT, int sms) {
   const int64_t units = static_cast<int64_t>(tiles) * 4 * KT;
-  return static_cast<int>(std::min<int64_t>(units, static_cast<int64_t>(sms) * 3));
+  return static_cast<int>(std::min<int64_t>(units, static_cast<int64_t>(sms) * 4));
 }
 
 // Dense quantise-once: the quantiser over all rows, then the GEMM (launched as
