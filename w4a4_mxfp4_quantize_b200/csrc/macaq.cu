@@ -1191,10 +1191,13 @@ int active_clusters(int dev, int bt_index, int S) {
 }
 
 // Choose the token tile BT and the K split S (a divisor of K/256, at most 8
-// CTAs per cluster) that minimise (fixed latency of a wave + prologue work of
-// one CTA) x the number of waves the clusters need.  Units: one row x one
-// 256-wide K tile of prologue work; a wave's fixed latency (launch, set-up,
-// first loads, reduction) is worth about 300 of them.
+// CTAs per cluster) that minimise the time of a call, modelled per wave of
+// clusters (µs, fitted to measured B200 timings of every feasible plan of the
+// M = 16 and M = 128 workloads):
+//   fixed 4.5 (launch, set-up, first loads, epilogue)
+//   + max(prologue 0.55 per 16 rows per K tile, MMA issue 0.65 per K tile)
+//     (the two overlap stage by stage; the slower sets the pace)
+//   + split-K reduction 1.1 + 0.2 S when S > 1.
 FusedPlan plan_fused(int dev, int64_t M, int64_t N, int64_t K) {
   const int NT = static_cast<int>(pad128(N) / 128), KT = static_cast<int>(K / 256);
   const int bts[4] = {16, 32, 64, 128};
@@ -1207,9 +1210,10 @@ FusedPlan plan_fused(int dev, int64_t M, int64_t N, int64_t K) {
     for (int S = 1; S <= 8 && S <= KT; ++S) {
       if (KT % S) continue;
       const int waves = ceil_div(clusters, active_clusters(dev, bi, S));
-      const double cost = static_cast<double>(waves) * (300.0 + static_cast<double>(M < bt ? M : bt) * (KT / S)) +
-                          0.25 * S;  // small bias against needless splitting
-      if (cost < best_cost) {
+      const double stages = static_cast<double>(KT / S), rows16 = static_cast<double>(M < bt ? M : bt) / 16.0;
+      const double per_wave = 4.5 + std::max(0.55 * rows16 * stages, 0.65 * stages) + (S > 1 ? 1.1 + 0.2 * S : 0.0);
+      const double cost = static_cast<double>(waves) * per_wave;
+      if (cost < best_cost - 1e-9) {
         best_cost = cost;
         best = {bt, S, clusters * S};
       }
