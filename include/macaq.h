@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define MACAQ_ABI_VERSION 1
+#define MACAQ_ABI_VERSION 2
 
 #define MACAQ_OK 0
 #define MACAQ_ERR_NULL (-1)               /* a required pointer is NULL */
@@ -98,12 +98,10 @@ int macaq_prepare_weights(const float *W_dev, const float *D_dev, int64_t E, int
 /* ------------------------------------------------------------------ */
 
 /* Scratch bytes a dense (E = 1) or grouped call of this shape needs (0 when
- * the chosen variant needs none).  The workspace holds split-K tile counters
- * (its first 4096 bytes) and FP32 partial sums.  The counter region must be
- * zero-filled before the workspace is first used; every completed call
- * leaves it at zero again, so one zero-fill at allocation is enough, whatever
- * shapes later calls have.  Calls that share a workspace must not run
- * concurrently. */
+ * the chosen variant needs none: dense M <= 128 runs in one kernel).  The
+ * workspace holds the quantised activation tiles and, for grouped calls, the
+ * group tables; its first 4096 bytes are left untouched.  Nothing in it has to
+ * start at zero.  Calls that share a workspace must not run concurrently. */
 size_t macaq_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t E);
 
 /* Dense MACAQ linear (MACAQ page, summary: channel scaling, block-32 BF16
@@ -130,6 +128,28 @@ int macaq_grouped_mm(const uint16_t *x_dev, const float *D_dev, const uint8_t *W
                      const int64_t *group_list_dev, int group_list_type, int64_t E, uint16_t *y_dev,
                      int64_t M, int64_t N, int64_t K, void *workspace_dev, size_t workspace_bytes,
                      int32_t *status_dev, void *stream);
+
+/* ------------------------------------------------------------------ */
+/* Plain MXFP4 W4A4 baseline                                           */
+/* ------------------------------------------------------------------ */
+
+/* The MACAQ page's native comparison (its "native" W4A4 path quantises x and W
+ * with dynamic MX quantisation only): no channel scaling and no Hadamard
+ * rotation.  Activations: the BF16 values themselves, MXFP4 per 32 along K
+ * (E8M0 from the block amax, E2M1 round-to-nearest-even with saturation);
+ * weights: the FP32 values, same rules; y = RNE_bf16(block-scaled sum) with
+ * FP32 accumulation and no 2^-5.  Same tile formats, workspace sizes
+ * (macaq_workspace_bytes), status codes and error behaviour as the MACAQ
+ * calls above; there is no D argument. */
+int macaq_prepare_weights_plain(const float *W_dev, int64_t E, int64_t N, int64_t K, uint8_t *Wq_dev,
+                                uint8_t *Ws_dev, void *stream);
+int macaq_dense_mm_plain(const uint16_t *x_dev, const uint8_t *Wq_dev, const uint8_t *Ws_dev, uint16_t *y_dev,
+                         int64_t M, int64_t N, int64_t K, void *workspace_dev, size_t workspace_bytes,
+                         int32_t *status_dev, void *stream);
+int macaq_grouped_mm_plain(const uint16_t *x_dev, const uint8_t *Wq_dev, const uint8_t *Ws_dev,
+                           const int64_t *group_list_dev, int group_list_type, int64_t E, uint16_t *y_dev,
+                           int64_t M, int64_t N, int64_t K, void *workspace_dev, size_t workspace_bytes,
+                           int32_t *status_dev, void *stream);
 
 /* ------------------------------------------------------------------ */
 /* Test and ablation entry points (not the product's hot path)         */

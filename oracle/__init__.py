@@ -70,6 +70,8 @@ def _L():
             "oracle_quantize_weights": (I, [P, P, I64, I64, P, P, I]),
             "oracle_gemm": (I, [P, P, P, P, I64, I64, I64, P, I]),
             "oracle_gemm_at": (I, [P, P, P, P, I64, P, P, I64, P]),
+            "oracle_gemm_plain": (I, [P, P, P, P, I64, I64, I64, P, I]),
+            "oracle_gemm_at_plain": (I, [P, P, P, P, I64, P, P, I64, P]),
             "oracle_group_offsets": (I, [P, I, I64, I64, P]),
             "oracle_grouped_mm": (I, [P, P, P, P, I, I64, I64, I64, I64, P, I]),
             "oracle_linear_f64": (None, [P, P, I64, I64, I64, P]),
@@ -297,6 +299,61 @@ def quantize_plain(v) -> tuple[np.ndarray, np.ndarray]:
     st = _L().oracle_quantize_plain(_p(v), R, K, _p(codes), _p(scales))
     assert st == OK, st
     return codes, scales
+
+
+def gemm_plain(qa, sa, qw, sw, nthreads: int = 0) -> np.ndarray:
+    """Plain MXFP4 product: y = RNE_bf16(exact block-scaled sum), no 2^-5."""
+    qa, sa, qw, sw = (_c(a, np.uint8) for a in (qa, sa, qw, sw))
+    M, K = qa.shape[0], qa.shape[1] * 2
+    N = qw.shape[0]
+    y = np.empty((M, N), np.uint16)
+    st = _L().oracle_gemm_plain(_p(qa), _p(sa), _p(qw), _p(sw), M, N, K, _p(y), nthreads)
+    assert st == OK, st
+    return y
+
+
+def gemm_at_plain(qa, sa, qw, sw, rows, cols) -> np.ndarray:
+    """Plain MXFP4 outputs at the given (row, col) pairs only."""
+    qa, sa, qw, sw = (_c(a, np.uint8) for a in (qa, sa, qw, sw))
+    K = qa.shape[1] * 2
+    rows = _c(rows, np.int64)
+    cols = _c(cols, np.int64)
+    out = np.empty(rows.size, np.uint16)
+    st = _L().oracle_gemm_at_plain(_p(qa), _p(sa), _p(qw), _p(sw), K, _p(rows), _p(cols), rows.size,
+                                   _p(out))
+    assert st == OK, st
+    return out
+
+
+def quantize_act_plain(x_bf16) -> tuple[np.ndarray, np.ndarray]:
+    """Plain MXFP4 of BF16 activations (their exact FP32 values), no D and no H."""
+    x = _c(x_bf16, np.uint16)
+    return quantize_plain(bf16_to_f64(x).astype(np.float32))
+
+
+def dense_mm_plain(x_bf16, W, nthreads: int = 0) -> np.ndarray:
+    """Whole dense plain MXFP4 W4A4 linear (the native baseline): bf16 bits [M, N]."""
+    qa, sa = quantize_act_plain(x_bf16)
+    qw, sw = quantize_plain(W)
+    return gemm_plain(qa, sa, qw, sw, nthreads)
+
+
+def grouped_mm_plain(x_bf16, W, group_list, group_list_type: int, nthreads: int = 0):
+    """Grouped plain MXFP4 linear: rows of group g against W[g].  Returns
+    (status, y bf16 bits [M, N])."""
+    x = _c(x_bf16, np.uint16)
+    W = _c(W, np.float32)
+    M = x.shape[0]
+    E, N, _ = W.shape
+    st, off = group_offsets(group_list, group_list_type, M)
+    y = np.zeros((M, N), np.uint16)
+    if st != OK:
+        return st, y
+    for g in range(E):
+        a, b = int(off[g]), int(off[g + 1])
+        if b > a:
+            y[a:b] = dense_mm_plain(x[a:b], W[g], nthreads)
+    return OK, y
 
 
 def num_threads() -> int:

@@ -33,6 +33,12 @@
  *       no BF16 rounding (offline preparation);
  *   R7  y = RNE_bf16(2^-5 * exact sum of the decoded block-scaled products).
  *
+ * The plain MXFP4 baseline (the MACAQ page's native W4A4 comparison, which
+ * quantises x and W directly with the dynamic MX quantiser) skips D and H:
+ * activations are the BF16 values themselves, weights the FP32 values, both
+ * quantised by R4/R5, and y = RNE_bf16(exact sum) with no 2^-5 (there is no
+ * Hadamard product to undo).
+ *
  * Build:  gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fopenmp -shared -fPIC
  * (no FMA contraction: every float operation is one IEEE binary32 rounding).
  */
@@ -426,11 +432,12 @@ static uint16_t wide_to_bf16(const wide_t *acc, int base_exp)
     return (uint16_t)((neg ? 0x8000u : 0u) | bits);
 }
 
-/* y = RNE_bf16(2^-5 * sum_k dec(qa[k]) 2^(sa[k/32]-127) dec(qw[k]) 2^(sw[k/32]-127)),
- * the sum taken exactly.  Each E2M1 value is an integer multiple of 1/2, so
- * each block of 32 contributes (sum of integer products) * 2^(sa+sw-256). */
+/* y = RNE_bf16(2^out_exp * sum_k dec(qa[k]) 2^(sa[k/32]-127) dec(qw[k]) 2^(sw[k/32]-127)),
+ * the sum taken exactly; out_exp = -5 for MACAQ (R7), 0 for plain MXFP4.
+ * Each E2M1 value is an integer multiple of 1/2, so each block of 32
+ * contributes (sum of integer products) * 2^(sa+sw-256). */
 static uint16_t exact_dot(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw,
-                          const uint8_t *sw, int64_t K)
+                          const uint8_t *sw, int64_t K, int out_exp)
 {
     wide_t acc;
     memset(&acc, 0, sizeof acc);
@@ -447,13 +454,13 @@ static uint16_t exact_dot(const uint8_t *qa, const uint8_t *sa, const uint8_t *q
         int E = (int)sa[b] + (int)sw[b] - 256;
         wide_add_shifted(&acc, p, E + 256);
     }
-    return wide_to_bf16(&acc, -256 - 5);
+    return wide_to_bf16(&acc, -256 + out_exp);
 }
 
 /* Full exact GEMM: qa [M, K/2], sa [M, K/32], qw [N, K/2], sw [N, K/32]
  * -> y bf16 bits [M, N]. */
-int oracle_gemm(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const uint8_t *sw,
-                int64_t M, int64_t N, int64_t K, uint16_t *y, int nthreads)
+static int gemm_exp(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const uint8_t *sw,
+                    int64_t M, int64_t N, int64_t K, uint16_t *y, int nthreads, int out_exp)
 {
     if (K <= 0 || K % 32 != 0)
         return ORACLE_ERR_SHAPE;
@@ -465,21 +472,47 @@ int oracle_gemm(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const u
     for (int64_t m = 0; m < M; m++)
         for (int64_t n = 0; n < N; n++)
             y[m * N + n] = exact_dot(qa + m * (K / 2), sa + m * (K / 32), qw + n * (K / 2),
-                                     sw + n * (K / 32), K);
+                                     sw + n * (K / 32), K, out_exp);
     (void)nthreads;
     return ORACLE_OK;
 }
 
+int oracle_gemm(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const uint8_t *sw,
+                int64_t M, int64_t N, int64_t K, uint16_t *y, int nthreads)
+{
+    return gemm_exp(qa, sa, qw, sw, M, N, K, y, nthreads, -5);
+}
+
+/* Plain MXFP4 product: the same exact sum without the 2^-5. */
+int oracle_gemm_plain(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const uint8_t *sw,
+                      int64_t M, int64_t N, int64_t K, uint16_t *y, int nthreads)
+{
+    return gemm_exp(qa, sa, qw, sw, M, N, K, y, nthreads, 0);
+}
+
 /* Exact outputs at chosen (row, col) positions only. */
-int oracle_gemm_at(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const uint8_t *sw,
-                   int64_t K, const int64_t *rows, const int64_t *cols, int64_t count, uint16_t *out)
+static int gemm_at_exp(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const uint8_t *sw,
+                       int64_t K, const int64_t *rows, const int64_t *cols, int64_t count, uint16_t *out,
+                       int out_exp)
 {
     if (K <= 0 || K % 32 != 0)
         return ORACLE_ERR_SHAPE;
     for (int64_t i = 0; i < count; i++)
         out[i] = exact_dot(qa + rows[i] * (K / 2), sa + rows[i] * (K / 32), qw + cols[i] * (K / 2),
-                           sw + cols[i] * (K / 32), K);
+                           sw + cols[i] * (K / 32), K, out_exp);
     return ORACLE_OK;
+}
+
+int oracle_gemm_at(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const uint8_t *sw,
+                   int64_t K, const int64_t *rows, const int64_t *cols, int64_t count, uint16_t *out)
+{
+    return gemm_at_exp(qa, sa, qw, sw, K, rows, cols, count, out, -5);
+}
+
+int oracle_gemm_at_plain(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const uint8_t *sw,
+                         int64_t K, const int64_t *rows, const int64_t *cols, int64_t count, uint16_t *out)
+{
+    return gemm_at_exp(qa, sa, qw, sw, K, rows, cols, count, out, 0);
 }
 
 /* ------------------------------------------------------------------ */

@@ -317,7 +317,7 @@ def fraction_to_bf16_bits(v: Fraction) -> int:
     return sign | bits
 
 
-def exact_y(qa, sa, qw, sw):
+def exact_y(qa, sa, qw, sw, div=32):
     M, K = qa.shape[0], qa.shape[1] * 2
     N = qw.shape[0]
     ca, cw = oracle.unpack_codes(qa), oracle.unpack_codes(qw)
@@ -330,7 +330,7 @@ def exact_y(qa, sa, qw, sw):
                       * Fraction(2) ** (int(sa[m, k // 32]) - 127)
                       * Fraction(oracle.e2m1_decode(int(cw[n, k])))
                       * Fraction(2) ** (int(sw[n, k // 32]) - 127))
-            out[m, n] = fraction_to_bf16_bits(s / 32)
+            out[m, n] = fraction_to_bf16_bits(s / div)
     return out
 
 
@@ -354,6 +354,59 @@ def test_exact_gemm_against_rationals(spread):
     rows, cols = np.meshgrid(np.arange(M), np.arange(N), indexing="ij")
     at = oracle.gemm_at(qa, sa, qw, sw, rows.ravel(), cols.ravel())
     assert np.array_equal(at, got.ravel())
+
+
+@pytest.mark.parametrize("spread", ["narrow", "wide", "extreme"])
+def test_plain_exact_gemm_against_rationals(spread):
+    # plain MXFP4 product: the same exact sum, rounded once to bf16, no 2^-5
+    rng = np.random.default_rng({"narrow": 20, "wide": 21, "extreme": 22}[spread])
+    M, N, K = 3, 4, 96
+    qa = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+    qw = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+    if spread == "narrow":
+        sa = rng.integers(120, 135, size=(M, K // 32), dtype=np.uint8)
+        sw = rng.integers(115, 125, size=(N, K // 32), dtype=np.uint8)
+    elif spread == "wide":
+        sa = rng.integers(60, 200, size=(M, K // 32), dtype=np.uint8)
+        sw = rng.integers(60, 200, size=(N, K // 32), dtype=np.uint8)
+    else:
+        sa = rng.choice(np.array([0, 1, 254, 127, 2], np.uint8), size=(M, K // 32))
+        sw = rng.choice(np.array([0, 254, 130, 3], np.uint8), size=(N, K // 32))
+    got = oracle.gemm_plain(qa, sa, qw, sw)
+    assert np.array_equal(got, exact_y(qa, sa, qw, sw, div=1))
+    rows, cols = np.meshgrid(np.arange(M), np.arange(N), indexing="ij")
+    assert np.array_equal(oracle.gemm_at_plain(qa, sa, qw, sw, rows.ravel(), cols.ravel()), got.ravel())
+
+
+def test_plain_linear_is_exact_on_representable_operands():
+    # Values that are E2M1 codes times a power of two with the block amax in
+    # [4, 8) x 2^k quantise losslessly, so the plain layer reduces to the
+    # correctly rounded exact product x . W^T.
+    rng = np.random.default_rng(23)
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+    M, N, K = 3, 5, 64
+    def representable(rows):
+        v = rng.choice(grid, size=(rows, K)) * rng.choice([-1, 1], size=(rows, K))
+        v[:, ::32] = 6.0 * rng.choice([-1, 1], size=(rows, K // 32))  # fixes each block's amax
+        scale = 2.0 ** rng.integers(-6, 4, size=(rows, K // 32))
+        return v * np.repeat(scale, 32, axis=1)
+    x = representable(M)
+    W = representable(N)
+    xb = synth.to_bf16_bits(x.astype(np.float32))
+    assert np.array_equal(synth.bf16_bits_to_f32(xb).astype(np.float64), x)  # exact in bf16 too
+    y = oracle.dense_mm_plain(xb, W.astype(np.float32))
+    for m in range(M):
+        for n in range(N):
+            s = sum((Fraction(x[m, k]) * Fraction(W[n, k]) for k in range(K)), Fraction(0))
+            assert y[m, n] == fraction_to_bf16_bits(s), (m, n)
+
+
+def test_plain_grouped_replicated_banks_equal_dense():
+    p = synth.dense(40, 256, 48, seed=3)
+    W = np.stack([p.W[0]] * 3)
+    st, yg = oracle.grouped_mm_plain(p.x, W, np.array([10, 0, 30], np.int64), 1)
+    assert st == 0
+    assert np.array_equal(yg, oracle.dense_mm_plain(p.x, p.W[0]))
 
 
 def _pack(codes):
@@ -448,9 +501,7 @@ def test_macaq_beats_plain_mxfp4_on_outlier_activations():
     p = synth.dense(32, 256, 64, seed=0)
     ref = oracle.linear_f64(p.x, p.W[0])
     y = synth.bf16_bits_to_f32(oracle.dense_mm(p.x, p.D[0], p.W[0])).astype(np.float64)
-    qa, sa = oracle.quantize_plain(synth.bf16_bits_to_f32(p.x))
-    qw, sw = oracle.quantize_plain(p.W[0])
-    yp = synth.bf16_bits_to_f32(oracle.gemm(qa, sa, qw, sw)).astype(np.float64) * 32
+    yp = synth.bf16_bits_to_f32(oracle.dense_mm_plain(p.x, p.W[0])).astype(np.float64)
     nmse = lambda a: float(np.sum((a - ref) ** 2) / np.sum(ref ** 2))
     assert nmse(y) < nmse(yp)
     assert nmse(y) < 0.05

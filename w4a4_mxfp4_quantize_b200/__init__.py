@@ -83,6 +83,10 @@ _SIG = {
     "macaq_dense_mm_noalloc": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, _P]),
     "macaq_unfused_dense_mm": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, ctypes.c_size_t,
                                               _P, _P]),
+    "macaq_prepare_weights_plain": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
+    "macaq_dense_mm_plain": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, ctypes.c_size_t, _P, _P]),
+    "macaq_grouped_mm_plain": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _I64, _P, _I64, _I64, _I64, _P,
+                                              ctypes.c_size_t, _P, _P]),
 }
 
 
@@ -232,6 +236,52 @@ def grouped_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Ten
                               _ptr(y), M, N, K, _ptr(ws), _nbytes(ws), _ptr(status),
                               _stream_ptr(stream)),
            "macaq_grouped_mm")
+    return y
+
+
+def prepare_weights_plain(W: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Offline, plain MXFP4 baseline: W fp32 [N, K] or [E, N, K] -> (Wq, Ws) tile images of W itself."""
+    if W.dim() == 2:
+        W = W.unsqueeze(0)
+    _require_cuda(W)
+    E, N, K = W.shape
+    qb, sb = weight_bytes(E, N, K)
+    if qb == 0:
+        raise MacaqError(-3, "prepare_weights_plain")
+    Wq = torch.empty(qb, dtype=torch.uint8, device=W.device)
+    Ws = torch.empty(sb, dtype=torch.uint8, device=W.device)
+    _check(lib().macaq_prepare_weights_plain(_ptr(W), E, N, K, _ptr(Wq), _ptr(Ws), _stream_ptr(stream)),
+           "macaq_prepare_weights_plain")
+    return Wq, Ws
+
+
+def dense_mm_plain(x: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: int, out: torch.Tensor | None = None,
+                   status: torch.Tensor | None = None, stream=None, ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Plain MXFP4 W4A4 baseline (no D, no Hadamard): y [M, N] bf16."""
+    _require_cuda(x, Wq, Ws, out, status)
+    M, K = x.shape
+    y = _output(out, M, N, x.device)
+    L = lib()
+    ws = workspace(int(L.macaq_workspace_bytes(M, N, K, 1)), x.device, stream, ws)
+    _check(L.macaq_dense_mm_plain(_ptr(x), _ptr(Wq), _ptr(Ws), _ptr(y), M, N, K, _ptr(ws), _nbytes(ws),
+                                  _ptr(status), _stream_ptr(stream)),
+           "macaq_dense_mm_plain")
+    return y
+
+
+def grouped_mm_plain(x: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, group_list: torch.Tensor,
+                     group_list_type: int, N: int, out: torch.Tensor | None = None,
+                     status: torch.Tensor | None = None, stream=None, ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Grouped plain MXFP4 W4A4 baseline; group_list as in grouped_mm."""
+    _require_cuda(x, Wq, Ws, group_list, out, status)
+    M, K = x.shape
+    E = group_list.numel()
+    y = _output(out, M, N, x.device)
+    L = lib()
+    ws = workspace(int(L.macaq_workspace_bytes(M, N, K, E)), x.device, stream, ws)
+    _check(L.macaq_grouped_mm_plain(_ptr(x), _ptr(Wq), _ptr(Ws), _ptr(group_list), int(group_list_type), E,
+                                    _ptr(y), M, N, K, _ptr(ws), _nbytes(ws), _ptr(status), _stream_ptr(stream)),
+           "macaq_grouped_mm_plain")
     return y
 
 

@@ -76,6 +76,8 @@ constexpr int kActImageBytes = kTileCodeBytes + kTileSfBytes;  // 17408
 // Offline weight preparation and test-only kernels
 // ============================================================================
 // CTA = 32 rows x one 256-wide K tile (256 threads, one 32-block each).
+// kPlain: plain MXFP4 of W itself (no D, no Hadamard; D is not read).
+template <bool kPlain>
 __global__ void __launch_bounds__(256) prep_weights_kernel(const float* __restrict__ W, const float* __restrict__ D,
                                                            uint8_t* __restrict__ Wq, uint8_t* __restrict__ Ws,
                                                            int N, int K, int NT) {
@@ -91,16 +93,25 @@ __global__ void __launch_bounds__(256) prep_weights_kernel(const float* __restri
   uint4 codes = make_uint4(0, 0, 0, 0);
   uint32_t scale = 0;
   if (n < N) {
-    float wv[32], dv[32];
+    float wv[32];
     const float4* wp = reinterpret_cast<const float4*>(W + (static_cast<int64_t>(e) * N + n) * K + k0);
-    const float4* dp = reinterpret_cast<const float4*>(D + static_cast<int64_t>(e) * K + k0);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float4 a = __ldg(wp + i), b = __ldg(dp + i);
+      const float4 a = __ldg(wp + i);
       wv[4 * i] = a.x; wv[4 * i + 1] = a.y; wv[4 * i + 2] = a.z; wv[4 * i + 3] = a.w;
-      dv[4 * i] = b.x; dv[4 * i + 1] = b.y; dv[4 * i + 2] = b.z; dv[4 * i + 3] = b.w;
     }
-    weight_block(wv, dv, codes, scale);
+    if constexpr (kPlain) {
+      mx_encode_block(wv, codes, scale);
+    } else {
+      float dv[32];
+      const float4* dp = reinterpret_cast<const float4*>(D + static_cast<int64_t>(e) * K + k0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 b = __ldg(dp + i);
+        dv[4 * i] = b.x; dv[4 * i + 1] = b.y; dv[4 * i + 2] = b.z; dv[4 * i + 3] = b.w;
+      }
+      weight_block(wv, dv, codes, scale);
+    }
   }
   const size_t tile = weight_image(e, nt, kt, NT / 2, KT);
   *reinterpret_cast<uint4*>(Wq + tile * kTileCodeBytes + code_chunk_offset(r, c)) = codes;
@@ -279,6 +290,7 @@ struct QuantParams {
   const int* gtp;
   const int4* tinfo;     // grouped: per row tile {group, first row, rows}
   const int* valid;
+  int plain;             // plain MXFP4 (no D, no Hadamard; D not read)
 };
 
 constexpr int kQuantStages = 3;                 // ring slots: the current unit and two ahead
@@ -323,7 +335,7 @@ __global__ void __launch_bounds__(256, 4) quant_tiles_kernel(const __grid_consta
     w.live = w.t < rows;
     w.img = p.Aq + (static_cast<size_t>(pm) * KT + kt) * kActImageBytes;
     const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
-    w.dp = p.D + static_cast<int64_t>(g) * p.K + k0 + threadIdx.x;
+    w.dp = p.plain ? nullptr : p.D + static_cast<int64_t>(g) * p.K + k0 + threadIdx.x;
     if (w.live) {
       const uint16_t* src = p.x + (static_cast<int64_t>(base) + w.t) * p.K + k0 + c * kBlk;
       uint8_t* dst = qsmem + (slot * 256 + threadIdx.x) * 64;
@@ -342,7 +354,7 @@ __global__ void __launch_bounds__(256, 4) quant_tiles_kernel(const __grid_consta
     if (us < units) ring[s] = fetch(us, s);
     else cp_async_commit();
   }
-  float d = __ldg(ring[0].dp);
+  float d = p.plain ? 1.f : __ldg(ring[0].dp);
   int buf = 0;  // reciprocal buffer of this unit: alternates unit by unit
   // unit i of this CTA uses ring slot i % kQuantStages; unrolled so slots are static
   while (u < units) {
@@ -357,7 +369,7 @@ __global__ void __launch_bounds__(256, 4) quant_tiles_kernel(const __grid_consta
       }
       const Unit w = ring[k];
       const int un = u + static_cast<int>(gridDim.x);
-      const float dn = un < units ? __ldg(ring[(k + 1) % kQuantStages].dp) : 0.f;
+      const float dn = (un < units && !p.plain) ? __ldg(ring[(k + 1) % kQuantStages].dp) : 1.f;
       r[buf][rcp_index(threadIdx.x)] = __frcp_rn(d);
       cp_async_wait<kQuantAhead>();  // this thread's copy of this unit has landed
       __syncthreads();               // every reciprocal written; r[buf] of two units back no longer read
@@ -366,7 +378,8 @@ __global__ void __launch_bounds__(256, 4) quant_tiles_kernel(const __grid_consta
       if (w.live) {
         const uint4* xs = reinterpret_cast<const uint4*>(qsmem + (k * 256 + threadIdx.x) * 64);
         const uint4 xv[4] = {xs[0], xs[1], xs[2], xs[3]};
-        act_block(xv, r[buf] + c * kRcpStride, cv, sc);
+        if (p.plain) act_block_plain(xv, cv, sc);
+        else act_block(xv, r[buf] + c * kRcpStride, cv, sc);
       }
       *reinterpret_cast<uint4*>(w.img + code_chunk_offset(w.t, c)) = cv;
       w.img[kTileCodeBytes + sf_offset(w.t, c)] = static_cast<uint8_t>(sc);
@@ -394,6 +407,7 @@ struct GemmParams {
   int wait_for_producer;  // dense: 1 when launched as a programmatic dependent of the quantiser
   int NT2;                // 256-wide output tiles: ceil(NT / 2)
   int stages;             // pipeline depth (gemm::stages_for(E))
+  float out_scale;        // 2^-5 (MACAQ: undoes the two unnormalised Hadamards), 1 (plain MXFP4)
 };
 
 // Large M: the MMA is not swapped.  Operand A = a 128-token activation tile,
@@ -660,6 +674,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
     // 16-byte pieces XOR-swizzled by the row (conflict-free writes and reads).
     const int q = warp & 3, h = (warp - 2) >> 2;
     const int et = threadIdx.x - 64;
+    const float os = p.out_scale;
     const int tl = q * 32 + lane;
     for (int i = 0; i < my_tiles; ++i) {
       const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp);
@@ -676,7 +691,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e)
-          pk[c0 / 2 + e] = pack_bf16x2(__uint_as_float(r[2 * e]) * 0.03125f, __uint_as_float(r[2 * e + 1]) * 0.03125f);
+          pk[c0 / 2 + e] = pack_bf16x2(__uint_as_float(r[2 * e]) * os, __uint_as_float(r[2 * e + 1]) * os);
       }
       tc_fence_before();
       __syncwarp();
@@ -724,6 +739,8 @@ struct FusedParams {
   uint16_t* y;
   int M, N, K, NT, KT, S;  // S = CTAs per cluster = K splits
   int32_t* status;
+  int plain;               // plain MXFP4 (no D, no Hadamard; D not read)
+  float out_scale;         // 2^-5 (MACAQ) or 1 (plain)
 };
 
 namespace fused {
@@ -930,7 +947,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
         }
       }
 #pragma unroll
-      for (int e = 0; e < C::kRcp; ++e) d[e] = __ldg(p.D + static_cast<int64_t>(kt) * kKTile + gt + e * kGT);
+      for (int e = 0; e < C::kRcp; ++e) d[e] = p.plain ? 1.f : __ldg(p.D + static_cast<int64_t>(kt) * kKTile + gt + e * kGT);
     };
     // the group's jj-th K tile: CTA-local index j = grp + kG * jj
     auto stage_body = [&](int jj, uint4 (&xv)[C::kTasks][2], const float (&d)[C::kRcp]) -> bool {
@@ -957,7 +974,8 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
           const int task = gt + (u0 + v) * kGT, c = (task >> 1) & 7, half = task & 1;
           rr[v] = r + c * kRcpStride + half * 16;
         }
-        act_half_blocks<kIlp>(*reinterpret_cast<const uint4(*)[kIlp][2]>(&xv[u0]), rr, cv, sc);
+        if (p.plain) act_half_blocks_plain<kIlp>(*reinterpret_cast<const uint4(*)[kIlp][2]>(&xv[u0]), cv, sc);
+        else act_half_blocks<kIlp>(*reinterpret_cast<const uint4(*)[kIlp][2]>(&xv[u0]), rr, cv, sc);
 #pragma unroll
         for (int v = 0; v < kIlp; ++v) {
           const int task = gt + (u0 + v) * kGT, t = task >> 4, c = (task >> 1) & 7, half = task & 1;
@@ -1030,10 +1048,11 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
         s[4] += b.x; s[5] += b.y; s[6] += b.z; s[7] += b.w;
       }
       uint4 o;
-      o.x = pack_bf16x2(s[0] * 0.03125f, s[1] * 0.03125f);
-      o.y = pack_bf16x2(s[2] * 0.03125f, s[3] * 0.03125f);
-      o.z = pack_bf16x2(s[4] * 0.03125f, s[5] * 0.03125f);
-      o.w = pack_bf16x2(s[6] * 0.03125f, s[7] * 0.03125f);
+      const float os = p.out_scale;
+      o.x = pack_bf16x2(s[0] * os, s[1] * os);
+      o.y = pack_bf16x2(s[2] * os, s[3] * os);
+      o.z = pack_bf16x2(s[4] * os, s[5] * os);
+      o.w = pack_bf16x2(s[6] * os, s[7] * os);
       *reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(m0 + t) * p.N + n0 + n) = o;
     }
   }
@@ -1269,15 +1288,17 @@ GroupedWs grouped_ws(int64_t M, int64_t K, int64_t E) {
   return w;
 }
 
+// plain: plain MXFP4 call, D is not used (and may be null).
 int check_mm_args(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M,
-                  int64_t N, int64_t K, int64_t E) {
+                  int64_t N, int64_t K, int64_t E, bool plain = false) {
   if (M < 0 || M > INT32_MAX || !valid_nk(N, K)) return MACAQ_ERR_SHAPE;
   if (M == 0) return MACAQ_OK;
-  if (!x || !D || !Wq || !Ws || !y) return MACAQ_ERR_NULL;
-  if (!aligned16(x) || !aligned16(D) || !aligned16(Wq) || !aligned16(Ws) || !aligned16(y)) return MACAQ_ERR_ALIGN;
+  if (!x || (!D && !plain) || !Wq || !Ws || !y) return MACAQ_ERR_NULL;
+  if (!aligned16(x) || (!plain && !aligned16(D)) || !aligned16(Wq) || !aligned16(Ws) || !aligned16(y))
+    return MACAQ_ERR_ALIGN;
   const size_t ybytes = static_cast<size_t>(M) * N * 2;
   if (overlaps(y, ybytes, x, static_cast<size_t>(M) * K * 2) ||
-      overlaps(y, ybytes, D, static_cast<size_t>(E) * K * 4) ||
+      (!plain && overlaps(y, ybytes, D, static_cast<size_t>(E) * K * 4)) ||
       overlaps(y, ybytes, Wq, macaq_weight_code_bytes(E, N, K)) ||
       overlaps(y, ybytes, Ws, macaq_weight_scale_bytes(E, N, K)))
     return MACAQ_ERR_ALIAS;
@@ -1300,12 +1321,12 @@ int quant_grid(int tiles, int KT, int sms) {
 // a programmatic dependent of the quantiser when `pdl`).
 int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y,
                          int64_t M, int64_t N, int64_t K, uint8_t* ws, int32_t* status, cudaStream_t st, int sms,
-                         bool pdl) {
+                         bool pdl, bool plain = false) {
   const DenseWs w = dense_ws(M, K);
   const int MT = static_cast<int>(pad128(M) / 128), KT = static_cast<int>(K / 256);
   QuantParams qp{};
   qp.x = x; qp.D = D; qp.Aq = ws + w.act;
-  qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = 1; qp.MT = MT;
+  qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = 1; qp.MT = MT; qp.plain = plain ? 1 : 0;
   if (launch_ex(quant_tiles_kernel, dim3(quant_grid(MT, KT, sms)), dim3(256), kQuantSmem, st, pdl, 1, qp) !=
       cudaSuccess)
     return MACAQ_ERR_CUDA;
@@ -1314,6 +1335,7 @@ int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, c
   gp.M = static_cast<int>(M); gp.N = static_cast<int>(N); gp.K = static_cast<int>(K);
   gp.NT = static_cast<int>(pad128(N) / 128); gp.KT = KT; gp.E = 1; gp.MT = MT;
   gp.NT2 = (gp.NT + 1) / 2; gp.stages = gemm::stages_for(0);
+  gp.out_scale = plain ? 1.0f : 0.03125f;
   gp.status = status;
   gp.wait_for_producer = pdl ? 1 : 0;
   const int tiles = MT * gp.NT2;
@@ -1400,7 +1422,26 @@ int macaq_prepare_weights(const float* W, const float* D, int64_t E, int64_t N, 
     if (!(d != 0.0f) || !std::isfinite(d)) return MACAQ_ERR_BAD_D;
   const int NTP = static_cast<int>(pad256(N) / 128);  // images per expert, pairs complete
   dim3 grid(static_cast<unsigned>(E * NTP * 4), static_cast<unsigned>(K / 256));
-  prep_weights_kernel<<<grid, 256, 0, s>>>(W, D, Wq, Ws, static_cast<int>(N), static_cast<int>(K), NTP);
+  prep_weights_kernel<false><<<grid, 256, 0, s>>>(W, D, Wq, Ws, static_cast<int>(N), static_cast<int>(K), NTP);
+  return cudaPeekAtLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
+}
+
+int macaq_prepare_weights_plain(const float* W, int64_t E, int64_t N, int64_t K, uint8_t* Wq, uint8_t* Ws,
+                                void* stream) {
+  if (E < 1 || E > kMaxGroups) return MACAQ_ERR_TOO_MANY_GROUPS;
+  if (!valid_nk(N, K)) return MACAQ_ERR_SHAPE;
+  if (!W || !Wq || !Ws) return MACAQ_ERR_NULL;
+  if (!aligned16(W) || !aligned16(Wq) || !aligned16(Ws)) return MACAQ_ERR_ALIGN;
+  const size_t qb = macaq_weight_code_bytes(E, N, K), sb = macaq_weight_scale_bytes(E, N, K);
+  const size_t wb = static_cast<size_t>(E * N * K * 4);
+  if (overlaps(Wq, qb, W, wb) || overlaps(Ws, sb, W, wb) || overlaps(Wq, qb, Ws, sb)) return MACAQ_ERR_ALIAS;
+  int dev, sms;
+  int st = current_device(dev, sms);
+  if (st != MACAQ_OK) return st;
+  const int NTP = static_cast<int>(pad256(N) / 128);
+  dim3 grid(static_cast<unsigned>(E * NTP * 4), static_cast<unsigned>(K / 256));
+  prep_weights_kernel<true><<<grid, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      W, nullptr, Wq, Ws, static_cast<int>(N), static_cast<int>(K), NTP);
   return cudaPeekAtLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
@@ -1411,9 +1452,9 @@ size_t macaq_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t E) {
   return dense_ws(M, K).total;
 }
 
-int macaq_dense_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M,
-                   int64_t N, int64_t K, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
-  int st = check_mm_args(x, D, Wq, Ws, y, M, N, K, 1);
+static int dense_impl(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M,
+               int64_t N, int64_t K, void* workspace, size_t workspace_bytes, int32_t* status, void* stream, bool plain) {
+  int st = check_mm_args(x, D, Wq, Ws, y, M, N, K, 1, plain);
   if (st != MACAQ_OK || M == 0) return st;
   if (M > kSmallM) {
     st = check_ws(workspace, workspace_bytes, dense_ws(M, K).total, y, static_cast<size_t>(M) * N * 2, x,
@@ -1432,17 +1473,20 @@ int macaq_dense_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const u
     const FusedPlan plan = plan_fused(dev, M, N, K);
     p.S = plan.S;
     p.status = status;
+    p.plain = plain ? 1 : 0;
+    p.out_scale = plain ? 1.0f : 0.03125f;
     return launch_fused(p, plan, s);
   }
-  return run_dense_two_kernel(x, D, Wq, Ws, y, M, N, K, static_cast<uint8_t*>(workspace), status, s, sms, true);
+  return run_dense_two_kernel(x, D, Wq, Ws, y, M, N, K, static_cast<uint8_t*>(workspace), status, s, sms, true,
+                              plain);
 }
 
-int macaq_grouped_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws,
-                     const int64_t* group_list, int group_list_type, int64_t E, uint16_t* y, int64_t M, int64_t N,
-                     int64_t K, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, const int64_t* group_list,
+                 int group_list_type, int64_t E, uint16_t* y, int64_t M, int64_t N, int64_t K, void* workspace,
+                 size_t workspace_bytes, int32_t* status, void* stream, bool plain) {
   if (E < 1 || E > kMaxGroups) return MACAQ_ERR_TOO_MANY_GROUPS;
   if (group_list_type != 0 && group_list_type != 1) return MACAQ_ERR_GROUP_LIST_TYPE;
-  int st = check_mm_args(x, D, Wq, Ws, y, M, N, K, E);
+  int st = check_mm_args(x, D, Wq, Ws, y, M, N, K, E, plain);
   if (st != MACAQ_OK) return st;
   if (M == 0) return MACAQ_OK;
   if (!group_list) return MACAQ_ERR_NULL;
@@ -1468,7 +1512,7 @@ int macaq_grouped_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const
   QuantParams qp{};
   qp.x = x; qp.D = D; qp.Aq = ws + w.act;
   qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = static_cast<int>(E);
-  qp.goff = goff; qp.gtp = gtp; qp.tinfo = tinfo; qp.valid = valid;
+  qp.goff = goff; qp.gtp = gtp; qp.tinfo = tinfo; qp.valid = valid; qp.plain = plain ? 1 : 0;
   if (launch_ex(quant_tiles_kernel, dim3(quant_grid(w.tiles_upper, KT, sms)), dim3(256), kQuantSmem, s, true, 1,
                 qp) != cudaSuccess)
     return MACAQ_ERR_CUDA;
@@ -1478,10 +1522,35 @@ int macaq_grouped_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const
   gp.NT = static_cast<int>(pad128(N) / 128); gp.KT = KT; gp.E = static_cast<int>(E);
   gp.NT2 = (gp.NT + 1) / 2; gp.stages = gemm::stages_for(static_cast<int>(E));
   gp.goff = goff; gp.gtp = gtp; gp.valid = valid;
+  gp.out_scale = plain ? 1.0f : 0.03125f;
   gp.status = status;
   const cudaError_t e = launch_ex(gemm_kernel, dim3(sms), dim3(gemm::kThreads),
                                   gemm::smem_bytes(static_cast<int>(E)), s, true, 1, gp);
   return e == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
+}
+
+int macaq_dense_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M,
+                   int64_t N, int64_t K, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  return dense_impl(x, D, Wq, Ws, y, M, N, K, workspace, workspace_bytes, status, stream, false);
+}
+
+int macaq_dense_mm_plain(const uint16_t* x, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M, int64_t N,
+                         int64_t K, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  return dense_impl(x, nullptr, Wq, Ws, y, M, N, K, workspace, workspace_bytes, status, stream, true);
+}
+
+int macaq_grouped_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws,
+                     const int64_t* group_list, int group_list_type, int64_t E, uint16_t* y, int64_t M, int64_t N,
+                     int64_t K, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  return grouped_impl(x, D, Wq, Ws, group_list, group_list_type, E, y, M, N, K, workspace, workspace_bytes, status,
+                      stream, false);
+}
+
+int macaq_grouped_mm_plain(const uint16_t* x, const uint8_t* Wq, const uint8_t* Ws, const int64_t* group_list,
+                           int group_list_type, int64_t E, uint16_t* y, int64_t M, int64_t N, int64_t K,
+                           void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  return grouped_impl(x, nullptr, Wq, Ws, group_list, group_list_type, E, y, M, N, K, workspace, workspace_bytes,
+                      status, stream, true);
 }
 
 int macaq_quantize_activations(const uint16_t* x, const float* D, uint8_t* codes, uint8_t* scales, int64_t M,

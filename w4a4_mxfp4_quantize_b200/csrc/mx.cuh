@@ -256,6 +256,56 @@ __device__ __forceinline__ void act_half_block(const uint4 (&xv)[2], const float
   scale = c;
 }
 
+// Plain MXFP4 (no D, no Hadamard): the block's BF16 values are encoded as they
+// are.  amax over |x| in BF16 (exact), E8M0 and E2M1 as in act_block.
+__device__ __forceinline__ void act_block_plain(const uint4 (&xv)[4], uint4& codes, uint32_t& scale) {
+  const uint32_t* w = reinterpret_cast<const uint32_t*>(xv);
+  uint32_t m = 0;
+#pragma unroll
+  for (int j = 0; j < 16; ++j) m = max_u16x2(m, w[j] & 0x7FFF7FFFu);
+  const uint32_t amax16 = max(m & 0xFFFFu, m >> 16);
+  const uint32_t c = e8m0_from_amax_bits(amax16 << 16);
+  const float s = __uint_as_float((254u - min(c, 253u)) << 23);
+  const uint64_t s2 = f2(s, s);
+  uint32_t out[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    out[q] = e2m1x8_f2(f2_mul(bf16x2_to_f2(w[4 * q]), s2), f2_mul(bf16x2_to_f2(w[4 * q + 1]), s2),
+                       f2_mul(bf16x2_to_f2(w[4 * q + 2]), s2), f2_mul(bf16x2_to_f2(w[4 * q + 3]), s2));
+  codes = make_uint4(out[0], out[1], out[2], out[3]);
+  scale = c;
+}
+
+// Plain MXFP4 of T half-blocks held by lane pairs (the partner holds the other
+// 16 values of each block; the block amax is combined across the pair).
+template <int T>
+__device__ __forceinline__ void act_half_blocks_plain(const uint4 (&xv)[T][2], uint2 (&codes)[T],
+                                                      uint32_t (&scale)[T]) {
+  uint32_t m[T];
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(xv[t]);
+    m[t] = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) m[t] = max_u16x2(m[t], w[j] & 0x7FFF7FFFu);
+  }
+#pragma unroll
+  for (int t = 0; t < T; ++t) m[t] = max_u16x2(m[t], __shfl_xor_sync(0xffffffffu, m[t], 1));
+#pragma unroll
+  for (int t = 0; t < T; ++t) {
+    const uint32_t* w = reinterpret_cast<const uint32_t*>(xv[t]);
+    const uint32_t amax16 = max(m[t] & 0xFFFFu, m[t] >> 16);
+    const uint32_t c = e8m0_from_amax_bits(amax16 << 16);
+    const float s = __uint_as_float((254u - min(c, 253u)) << 23);
+    const uint64_t s2 = f2(s, s);
+    codes[t].x = e2m1x8_f2(f2_mul(bf16x2_to_f2(w[0]), s2), f2_mul(bf16x2_to_f2(w[1]), s2),
+                           f2_mul(bf16x2_to_f2(w[2]), s2), f2_mul(bf16x2_to_f2(w[3]), s2));
+    codes[t].y = e2m1x8_f2(f2_mul(bf16x2_to_f2(w[4]), s2), f2_mul(bf16x2_to_f2(w[5]), s2),
+                           f2_mul(bf16x2_to_f2(w[6]), s2), f2_mul(bf16x2_to_f2(w[7]), s2));
+    scale[t] = c;
+  }
+}
+
 // T independent half-blocks, each step done for all T before the next step, so
 // that one thread keeps T dependency chains in flight.  Same arithmetic as
 // act_half_block; lane pairs as there.
