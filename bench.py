@@ -174,6 +174,33 @@ class Prepared:
         mq.unfused_dense_mm(self.x, self.D, self.Wq, self.Ws, self.p.N, out=self.y, stream=stream,
                             ws=self.ws_unfused)
 
+    def prepare_plain(self, mq, device):
+        """Plain MXFP4 weights of the same W (the native baseline)."""
+        W = f32(self.p.W, device)
+        self.Wq_plain, self.Ws_plain = mq.prepare_weights_plain(W)
+        del W
+
+    def run_plain(self, mq, stream=None):
+        if self.gl is None:
+            mq.dense_mm_plain(self.x, self.Wq_plain, self.Ws_plain, self.p.N, out=self.y, stream=stream,
+                              ws=self.ws)
+        else:
+            mq.grouped_mm_plain(self.x, self.Wq_plain, self.Ws_plain, self.gl, self.p.group_list_type, self.p.N,
+                                out=self.y, stream=stream, ws=self.ws)
+
+
+def layer_nmse(p: synth.Problem, y: torch.Tensor, rows: np.ndarray) -> float:
+    """Normalised squared error of output rows against the unquantised layer
+    x . W^T in float64 (numpy; the rows' own experts for grouped problems)."""
+    yb = y[torch.from_numpy(rows).to(y.device)].float().cpu().numpy().astype(np.float64)
+    x = synth.bf16_bits_to_f32(p.x[rows]).astype(np.float64)
+    if p.E == 1:
+        ref = x @ p.W[0].astype(np.float64).T
+    else:
+        g = np.searchsorted(np.cumsum(p.counts), rows, side="right")
+        ref = np.stack([x[i] @ p.W[g[i]].astype(np.float64).T for i in range(rows.size)])
+    return float(np.sum((yb - ref) ** 2) / np.sum(ref ** 2))
+
 
 def capture(fn, stream):
     """Capture fn() (library calls on the current stream) into a CUDA graph."""
@@ -451,7 +478,9 @@ def run_only(args):
 
 def workload_table(mq, device, stream, flush, hbm_gbs, reps):
     """us/call (median, cold L2), TFLOPS and roofline fraction for every
-    problem of the five workloads, fused and unfused (CUDA graph per call)."""
+    problem of the five workloads, fused and unfused (CUDA graph per call), the
+    plain MXFP4 baseline's time, and both paths' error against the unquantised
+    layer on sampled rows."""
     rows = []
     for cfg in range(5):
         for p in synth.config(cfg):
@@ -465,11 +494,25 @@ def workload_table(mq, device, stream, flush, hbm_gbs, reps):
                 gu = capture(lambda: pp.run_unfused(mq), stream)
                 un, _ = time_graph(gu, flush, stream, reps)
                 del gu
+            # accuracy against the unquantised layer on sampled rows, then the plain MXFP4 baseline
+            rows_s = np.unique(np.random.default_rng(cfg).integers(0, p.M, min(p.M, 16)))
+            pp.run(mq, stream)
+            stream.synchronize()
+            nmse = layer_nmse(p, pp.y, rows_s)
+            pp.prepare_plain(mq, device)
+            gp = capture(lambda: pp.run_plain(mq), stream)
+            plain_us, _ = time_graph(gp, flush, stream, reps)
+            del gp
+            pp.run_plain(mq, stream)
+            stream.synchronize()
+            nmse_plain = layer_nmse(p, pp.y, rows_s)
             t_roof = max(p.algorithmic_bytes() / (hbm_gbs * 1e9), p.flops() / (FP4_NOMINAL_TFLOPS * 1e12))
             rows.append({
                 "config": cfg, "name": p.name, "us": us, "iqr_us": iqr, "us_warm_l2": us_warm,
                 "tflops": p.flops() / (us * 1e-6) / 1e12, "gbs": p.algorithmic_bytes() / (us * 1e-6) / 1e9,
                 "roofline_us": t_roof * 1e6, "frac_roofline": t_roof / (us * 1e-6), "unfused_us": un,
+                "plain_us": plain_us, "plain_over_macaq_time": plain_us / us,
+                "nmse": nmse, "nmse_plain": nmse_plain, "nmse_plain_over_macaq": nmse_plain / nmse if nmse else None,
             })
             del g, pp
             torch.cuda.empty_cache()
