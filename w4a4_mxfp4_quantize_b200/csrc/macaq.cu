@@ -1232,7 +1232,7 @@ FusedPlan plan_fused(int dev, int64_t M, int64_t N, int64_t K) {
       const double stages = static_cast<double>(KT / S), rows16 = static_cast<double>(M < bt ? M : bt) / 16.0;
       const double per_wave = 4.5 + std::max(0.55 * rows16 * stages, 0.65 * stages) + (S > 1 ? 1.1 + 0.2 * S : 0.0);
       const double cost = static_cast<double>(waves) * per_wave;
-      if (cost < best_cost - 1e-9) {
+      if (cost <= best_cost + 1e-9) {  // on a tie the larger tile / split (measured faster)
         best_cost = cost;
         best = {bt, S, clusters * S};
       }
