@@ -61,7 +61,7 @@ extern "C" {
 #define MACAQ_ERR_ARCH (-4)               /* current device is not sm_100 */
 #define MACAQ_ERR_ALIAS (-5)              /* the output overlaps an input */
 #define MACAQ_ERR_TOO_MANY_GROUPS (-6)    /* E < 1 or E > 1024 */
-#define MACAQ_ERR_GROUP_LIST_TYPE (-7)    /* group_list_type not 0 or 1 */
+#define MACAQ_ERR_GROUP_LIST_TYPE (-7)    /* group_list_type not 0, 1 or 2 */
 #define MACAQ_ERR_CUDA (-8)               /* a CUDA runtime call failed */
 #define MACAQ_ERR_DEVICE_TIMEOUT (-9)     /* (device) a bounded wait expired */
 #define MACAQ_ERR_GROUP_LIST_INVALID (-10)/* (device) group_list breaks the rules */
@@ -120,8 +120,11 @@ int macaq_dense_mm(const uint16_t *x_dev, const float *D_dev, const uint8_t *Wq_
 /* Grouped MACAQ linear (npu_grouped_matmul single-x / single-weight /
  * single-y form, group_type 0).
  *   D_dev fp32 [E, K]; Wq_dev/Ws_dev prepared with this E;
- *   group_list_dev int64 [E] on the device (never read by the host);
- *   group_list_type 0 = cumulative sums, 1 = counts.
+ *   group_list_dev int64 on the device (never read by the host): [E] for
+ *   group_list_type 0 (cumulative sums) and 1 (counts); [E, 2] rows of
+ *   (group index, group size) for type 2, the row ranges following one
+ *   another along M in list order, each using the named expert's W and D
+ *   (npu_grouped_matmul, group_list_type 2);
  * An invalid group_list writes MACAQ_ERR_GROUP_LIST_INVALID to *status_dev
  * and leaves y untouched. */
 int macaq_grouped_mm(const uint16_t *x_dev, const float *D_dev, const uint8_t *Wq_dev, const uint8_t *Ws_dev,

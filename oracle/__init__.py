@@ -237,7 +237,7 @@ def group_offsets(group_list, group_list_type: int, M: int):
     """Row offsets [E+1] from group_list (npu_grouped_matmul, group_list and
     group_list_type).  Returns (status, offsets)."""
     gl = _c(group_list, np.int64)
-    E = gl.size
+    E = gl.shape[0] if group_list_type == 2 else gl.size  # type 2: [E, 2] rows of (expert, rows)
     off = np.zeros(max(E + 1, 2), np.int64)
     st = _L().oracle_group_offsets(_p(gl), int(group_list_type), E, M, _p(off))
     return int(st), off[:E + 1]
@@ -349,10 +349,12 @@ def grouped_mm_plain(x_bf16, W, group_list, group_list_type: int, nthreads: int 
     y = np.zeros((M, N), np.uint16)
     if st != OK:
         return st, y
+    gl = _c(group_list, np.int64)
     for g in range(E):
         a, b = int(off[g]), int(off[g + 1])
+        e = int(gl[g, 0]) if group_list_type == 2 else g
         if b > a:
-            y[a:b] = dense_mm_plain(x[a:b], W[g], nthreads)
+            y[a:b] = dense_mm_plain(x[a:b], W[e], nthreads)
     return OK, y
 
 

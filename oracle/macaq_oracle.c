@@ -13,7 +13,8 @@
  * matrix multiplication with BF16 output; the weight transform (W, D, H) is
  * offline.  The grouped form follows the torch_npu npu_grouped_matmul page
  * (function description: y_i = x_i @ weight_i; parameters: group_list,
- * group_list_type 0 = cumulative sum, 1 = per-group counts).
+ * group_list_type 0 = cumulative sum, 1 = per-group counts, 2 = [E, 2] rows of
+ * (group index, group size) whose sizes follow one another along M).
  *
  * Readings taken where the pages are silent (each one is listed, with the
  * reason, in the design notes of the repository):
@@ -527,12 +528,15 @@ int oracle_group_offsets(const int64_t *group_list, int type, int64_t E, int64_t
 {
     if (E < 1 || E > 1024)
         return ORACLE_ERR_TOO_MANY_GROUPS;
-    if (type != 0 && type != 1)
+    if (type != 0 && type != 1 && type != 2)
         return ORACLE_ERR_GROUP_LIST_TYPE;
     off[0] = 0;
     for (int64_t g = 0; g < E; g++) {
-        int64_t v = group_list[g];
+        /* type 2: row g is [expert index, rows of the grouped axis] */
+        int64_t v = type == 2 ? group_list[2 * g + 1] : group_list[g];
         if (v < 0)
+            return ORACLE_ERR_GROUP_LIST_INVALID;
+        if (type == 2 && (group_list[2 * g] < 0 || group_list[2 * g] >= E))
             return ORACLE_ERR_GROUP_LIST_INVALID;
         if (type == 0) {
             if (v < off[g])
@@ -568,10 +572,12 @@ int oracle_grouped_mm(const uint16_t *x, const float *D, const float *W, const i
         int64_t r0 = off[g], r1 = off[g + 1];
         if (r1 == r0)
             continue;
-        oracle_quantize_weights(W + g * N * K, D + g * K, N, K, qw, sw, nthreads);
+        /* the rows of list entry g use expert e (type 2 names it; otherwise e = g) */
+        int64_t e = type == 2 ? group_list[2 * g] : g;
+        oracle_quantize_weights(W + e * N * K, D + e * K, N, K, qw, sw, nthreads);
         uint8_t *qa = (uint8_t *)malloc((size_t)((r1 - r0) * K / 2));
         uint8_t *sa = (uint8_t *)malloc((size_t)((r1 - r0) * K / 32));
-        oracle_quantize_act(x + r0 * K, D + g * K, r1 - r0, K, qa, sa, nthreads);
+        oracle_quantize_act(x + r0 * K, D + e * K, r1 - r0, K, qa, sa, nthreads);
         oracle_gemm(qa, sa, qw, sw, r1 - r0, N, K, y + r0 * N, nthreads);
         free(qa);
         free(sa);

@@ -87,8 +87,9 @@ def test_grouped_refusals_by_name(L):
 
     assert g(E=0) == -6
     assert g(E=1025) == -6
-    assert g(t=2) == -7
+    assert g(t=3) == -7
     assert g(t=-1) == -7
+    assert g(t=2) == -11  # type 2 is accepted; the missing workspace is the next refusal
     assert g(N=24) == -3
     assert g(glp=None) == -1
     assert g(glp=P((9 << 32) + 4)) == -2

@@ -296,7 +296,9 @@ def test_grouped_replicated_banks_equal_dense():
 
 
 @pytest.mark.parametrize("gl,gtype", [([10, 5, 30], 0), ([10, -1, 21], 1), ([10, 10, 11], 1), ([10, 20, 29], 0),
-                                      ([-3, 20, 30], 0)])
+                                      ([-3, 20, 30], 0), ([[0, 10], [3, 10], [1, 10]], 2),
+                                      ([[0, 10], [2, 10], [1, 9]], 2), ([[0, 10], [-1, 10], [1, 10]], 2),
+                                      ([[0, 40], [2, -10], [1, 0]], 2)])
 def test_grouped_invalid_group_list_sets_status_and_leaves_y(gl, gtype):
     p = synth.grouped(30, 3, 256, 64, seed=14, dist="uniform", group_list_type=1)
     Wq, Ws = mq.prepare_weights(f32_dev(p.W), f32_dev(p.D))
@@ -307,6 +309,21 @@ def test_grouped_invalid_group_list_sets_status_and_leaves_y(gl, gtype):
     torch.cuda.synchronize()
     assert int(status.item()) == -10
     assert bool(torch.all(y == 7.0))
+
+
+@pytest.mark.parametrize("T,E,K,N", [(200, 5, 512, 144), (300, 16, 256, 256)])
+def test_grouped_type2_named_experts(T, E, K, N):
+    # type 2: [E, 2] rows of (group index, group size); the row ranges follow the
+    # list order and use the named expert, which may repeat or never appear
+    p = synth.grouped(T, E, K, N, seed=T + E + 1, dist="zipf", group_list_type=1)
+    rng = np.random.default_rng(E)
+    idx = rng.integers(0, E, E)
+    idx[0] = idx[-1]                      # one expert named twice
+    gl2 = np.ascontiguousarray(np.stack([idx, p.counts]).T.astype(np.int64))
+    st, want = oracle.grouped_mm(p.x, p.D, p.W, gl2, 2)
+    assert st == 0
+    got = y_to_bits(_run_grouped(p, gl=gl2, gtype=2))
+    compare(got, want, p.name + " type 2")
 
 
 @pytest.mark.parametrize("which", [0, 1])

@@ -454,7 +454,13 @@ def test_group_list_validation_rules():
     assert oracle.group_offsets([3, -1, 8], 1, M)[0] == oracle.ERR_GROUP_LIST_INVALID
     assert oracle.group_offsets([3, 7, 9], 0, M)[0] == oracle.ERR_GROUP_LIST_INVALID  # != M
     assert oracle.group_offsets([3, 4, 4], 1, M)[0] == oracle.ERR_GROUP_LIST_INVALID
-    assert oracle.group_offsets([3, 7, 10], 2, M)[0] == oracle.ERR_GROUP_LIST_TYPE
+    assert oracle.group_offsets([3, 7, 10], 3, M)[0] == oracle.ERR_GROUP_LIST_TYPE
+    # type 2: [E, 2] rows of (group index, group size); sizes add up along M
+    assert oracle.group_offsets([[2, 3], [0, 7], [1, 0]], 2, M)[0] == oracle.OK
+    assert oracle.group_offsets([[2, 3], [0, 6], [1, 0]], 2, M)[0] == oracle.ERR_GROUP_LIST_INVALID  # sum != M
+    assert oracle.group_offsets([[3, 3], [0, 7], [1, 0]], 2, M)[0] == oracle.ERR_GROUP_LIST_INVALID  # index >= E
+    assert oracle.group_offsets([[2, 3], [-1, 7], [1, 0]], 2, M)[0] == oracle.ERR_GROUP_LIST_INVALID
+    assert oracle.group_offsets([[2, -3], [0, 13], [1, 0]], 2, M)[0] == oracle.ERR_GROUP_LIST_INVALID
     assert oracle.group_offsets(np.zeros(1025, np.int64), 1, 0)[0] == oracle.ERR_TOO_MANY_GROUPS
     st, off = oracle.group_offsets([0, 0, 4, 4, 10], 0, M)
     assert st == oracle.OK and list(off) == [0, 0, 0, 4, 4, 10]
@@ -471,6 +477,25 @@ def test_grouped_cumsum_equals_counts_and_replicated_banks_equal_dense():
     st, yr = oracle.grouped_mm(p.x, Dr, Wr, p.group_list, 1)
     assert st == oracle.OK
     assert np.array_equal(yr, oracle.dense_mm(p.x, p.D[0], p.W[0]))
+
+
+def test_grouped_type2_rows_use_the_named_expert():
+    # type 2 names each range's expert: permuting the experts and naming them in the
+    # list gives the same output as the counts form on the original order
+    p = synth.grouped(80, 4, 64, 32, seed=6, dist="uniform", group_list_type=1)
+    perm = np.array([2, 0, 3, 1])
+    Wp, Dp = np.empty_like(p.W), np.empty_like(p.D)
+    Wp[perm], Dp[perm] = p.W, p.D  # expert g now lives at index perm[g]
+    gl2 = np.stack([perm, p.counts]).T.astype(np.int64)
+    st2, y2 = oracle.grouped_mm(p.x, Dp, Wp, gl2, 2)
+    st1, y1 = oracle.grouped_mm(p.x, p.D, p.W, p.counts.astype(np.int64), 1)
+    assert st1 == st2 == oracle.OK and np.array_equal(y1, y2)
+    # an expert named twice and one never named
+    gl3 = np.array([[1, 30], [1, 20], [3, 30], [0, 0]], np.int64)
+    st3, y3 = oracle.grouped_mm(p.x, p.D, p.W, gl3, 2)
+    assert st3 == oracle.OK
+    assert np.array_equal(y3[:50], oracle.dense_mm(p.x[:50], p.D[1], p.W[1]))
+    assert np.array_equal(y3[50:], oracle.dense_mm(p.x[50:], p.D[3], p.W[3]))
 
 
 def test_grouped_rows_use_their_own_expert():

@@ -221,13 +221,23 @@ def dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tenso
     return y
 
 
+def _groups(group_list: torch.Tensor, group_list_type: int) -> int:
+    """Number of group_list entries: rows of the [E, 2] form for type 2."""
+    if group_list_type == 2:
+        if group_list.dim() != 2 or group_list.shape[1] != 2:
+            raise MacaqError(-3, "group_list of type 2 must be [E, 2]")
+        return int(group_list.shape[0])
+    return group_list.numel()
+
+
 def grouped_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, group_list: torch.Tensor,
                group_list_type: int, N: int, out: torch.Tensor | None = None,
                status: torch.Tensor | None = None, stream=None, ws: torch.Tensor | None = None) -> torch.Tensor:
-    """Grouped MACAQ linear; group_list int64 [E] on the device (0 cumsum, 1 counts)."""
+    """Grouped MACAQ linear; group_list int64 on the device: [E] for type 0 (cumsum) and 1
+    (counts), [E, 2] rows of (group index, group size) for type 2."""
     _require_cuda(x, D, Wq, Ws, group_list, out, status)
     M, K = x.shape
-    E = group_list.numel()
+    E = _groups(group_list, group_list_type)
     y = _output(out, M, N, x.device)
     L = lib()
     need = int(L.macaq_workspace_bytes(M, N, K, E))
@@ -275,7 +285,7 @@ def grouped_mm_plain(x: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, group_
     """Grouped plain MXFP4 W4A4 baseline; group_list as in grouped_mm."""
     _require_cuda(x, Wq, Ws, group_list, out, status)
     M, K = x.shape
-    E = group_list.numel()
+    E = _groups(group_list, group_list_type)
     y = _output(out, M, N, x.device)
     L = lib()
     ws = workspace(int(L.macaq_workspace_bytes(M, N, K, E)), x.device, stream, ws)

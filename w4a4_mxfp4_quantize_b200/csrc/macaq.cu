@@ -219,20 +219,29 @@ __device__ __forceinline__ int64_t block_excl_scan(int64_t v, int64_t* scratch, 
 // group_list / group_list_type): type 0 non-negative and non-decreasing
 // cumulative sums, type 1 non-negative counts; the rows must total M.
 // Writes goff[0..E] (row offsets), gtp[0..E] (prefix of 128-row tiles per
-// group) and *valid; on a violation also *status.
+// list entry), gexp[0..E) (the expert of each entry: the entry itself for types
+// 0 and 1, the named group index for type 2) and *valid; on a violation also
+// *status.
 __global__ void __launch_bounds__(1024) group_tables_kernel(const int64_t* __restrict__ gl, int type, int E, int M,
                                                             int64_t* __restrict__ goff, int* __restrict__ gtp,
-                                                            int4* __restrict__ tinfo, int* __restrict__ valid,
-                                                            int32_t* status) {
+                                                            int* __restrict__ gexp, int4* __restrict__ tinfo,
+                                                            int* __restrict__ valid, int32_t* status) {
   __shared__ int64_t scratch[72];
   const int g = threadIdx.x;
   int64_t cnt = 0;
   bool bad = false;
+  int ex = g;  // the expert whose weights this list entry's rows use
   if (g < E) {
-    const int64_t v = gl[g];
-    const int64_t prev = (type == 0 && g > 0) ? gl[g - 1] : 0;
-    cnt = type == 0 ? v - prev : v;
-    bad = v < 0 || cnt < 0 || cnt > M;
+    if (type == 2) {  // [E, 2] rows of (group index, group size)
+      ex = static_cast<int>(gl[2 * g] < 0 || gl[2 * g] >= E ? -1 : gl[2 * g]);
+      cnt = gl[2 * g + 1];
+      bad = ex < 0 || cnt < 0 || cnt > M;
+    } else {
+      const int64_t v = gl[g];
+      const int64_t prev = (type == 0 && g > 0) ? gl[g - 1] : 0;
+      cnt = type == 0 ? v - prev : v;
+      bad = v < 0 || cnt < 0 || cnt > M;
+    }
   }
   bad = __syncthreads_or(bad);
   if (!bad) {
@@ -243,6 +252,7 @@ __global__ void __launch_bounds__(1024) group_tables_kernel(const int64_t* __res
     if (g < E) {
       goff[g] = rb;
       gtp[g] = static_cast<int>(tb);
+      gexp[g] = ex;
     }
     if (g == 0) {
       goff[E] = rows_total;
@@ -251,7 +261,7 @@ __global__ void __launch_bounds__(1024) group_tables_kernel(const int64_t* __res
     // per row tile: {group, first row, rows}, one load for the quantiser
     if (g < E && !bad)
       for (int64_t j = 0; j * kRowsTile < cnt; ++j)
-        tinfo[tb + j] = make_int4(g, static_cast<int>(rb + j * kRowsTile),
+        tinfo[tb + j] = make_int4(ex, static_cast<int>(rb + j * kRowsTile),
                                   static_cast<int>(cnt - j * kRowsTile < kRowsTile ? cnt - j * kRowsTile : kRowsTile), 0);
   }
   if (g == 0) {
@@ -402,6 +412,7 @@ struct GemmParams {
   int M, N, K, NT, KT, E, MT;
   const int64_t* goff;  // grouped tables (nullptr: dense with MT tiles)
   const int* gtp;
+  const int* gexp;      // expert of each group_list entry
   const int* valid;
   int32_t* status;
   int wait_for_producer;  // dense: 1 when launched as a programmatic dependent of the quantiser
@@ -438,7 +449,7 @@ static_assert(kSfCol + kSfCols * kMaxStages <= kTmemCols, "scale slots fit the a
 static_assert(kStageBytes % 1024 == 0, "stage alignment");
 constexpr size_t kSmemLimit = 227 * 1024;
 __host__ __device__ constexpr size_t group_bytes(int E) {
-  return E > 0 ? static_cast<size_t>(E + 1) * 12 + 16 : 0;
+  return E > 0 ? static_cast<size_t>(E + 1) * 16 + 16 : 0;  // goff (8), gtp (4), gexp (4) per entry
 }
 // four stages when the group tables leave room for them, else three
 __host__ __device__ constexpr int stages_for(int E) {
@@ -457,7 +468,7 @@ struct GemmTile {
 };
 
 __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int idx, int mtiles, const int64_t* goff,
-                                              const int* gtp) {
+                                              const int* gtp, const int* gexp) {
   GemmTile t;
   t.pm = idx % mtiles;
   t.nt = 2 * (idx / mtiles);
@@ -466,9 +477,10 @@ __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int idx, int 
     t.m0 = t.pm * kRowsTile;
     t.rows = min(kRowsTile, p.M - t.m0);
   } else {
-    t.g = find_group(gtp, p.E, t.pm);
-    t.m0 = static_cast<int>(goff[t.g]) + (t.pm - gtp[t.g]) * kRowsTile;
-    t.rows = min(kRowsTile, static_cast<int>(goff[t.g + 1]) - t.m0);
+    const int e = find_group(gtp, p.E, t.pm);  // list entry; its rows use expert gexp[e]
+    t.g = gexp[e];
+    t.m0 = static_cast<int>(goff[e]) + (t.pm - gtp[e]) * kRowsTile;
+    t.rows = min(kRowsTile, static_cast<int>(goff[e + 1]) - t.m0);
   }
   return t;
 }
@@ -534,6 +546,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
   volatile int* epi_flag = abort_flag + 1;
   int64_t* goff = nullptr;
   int* gtp = nullptr;
+  int* gexp = nullptr;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   int mtiles = p.MT;
@@ -542,9 +555,11 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
     if (*p.valid == 0) return;
     goff = reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(full) + 256);
     gtp = reinterpret_cast<int*>(goff + p.E + 1);
+    gexp = gtp + p.E + 1;
     for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
       goff[i] = p.goff[i];
       gtp[i] = p.gtp[i];
+      if (i < p.E) gexp[i] = p.gexp[i];
     }
     __syncthreads();
     mtiles = gtp[p.E];
@@ -588,7 +603,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
     // scales.  Gives k tile 0 of this CTA's i-th output tile; k tile kt is
     // kt * step further on.
     auto source = [&](int i, int c, const uint8_t*& src, uint32_t& bytes, uint32_t& doff, uint32_t& step) {
-      const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp);
+      const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp, gexp);
       const size_t img = weight_image(t.g, t.nt, 0, p.NT2, KT);
       bytes = c == 0 ? kActImageBytes : c == 1 ? 2 * kTileCodeBytes : 2 * kTileSfBytes;
       step = c == 0 ? kActImageBytes : bytes;
@@ -677,7 +692,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
     const float os = p.out_scale;
     const int tl = q * 32 + lane;
     for (int i = 0; i < my_tiles; ++i) {
-      const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp);
+      const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp, gexp);
       if (et == 0) *epi_flag = mbar_wait(accf, i & 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
       named_bar_sync(1, 256);  // also: every thread has finished reading the previous tile's staging
       if (!*epi_flag) break;
@@ -820,6 +835,59 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
     *abort_flag = 0;
     fence_mbar_init();
   }
+  const int nst = kt1 - kt0;                   // K tiles of this CTA
+  const int pre = nst < kStages ? nst : kStages;  // first-use stages: no wait for a free slot
+  if (warp == 0) {
+    // The weights do not depend on any earlier kernel: their first stages go out as
+    // soon as the barriers exist (lane 0 initialised them), before the set-up below.
+    __syncwarp();
+    if (lane == 0)
+      for (int j = 0; j < pre; ++j) mbar_arrive_expect_tx(&full[j], kTileCodeBytes + kTileSfBytes);
+    __syncwarp();
+    const int j = min(lane >> 1, pre - 1);
+    const bool sf = lane & 1;
+    const size_t wt = weight_image(0, nt, kt0 + j, (p.NT + 1) / 2, p.KT);
+    uint8_t* sb = smem + j * C::kStageBytes;
+    bulk_g2s_if(lane < 2 * pre, sf ? sb + C::kOffSfa : sb, sf ? p.Ws + wt * kTileSfBytes : p.Wq + wt * kTileCodeBytes,
+                sf ? kTileSfBytes : kTileCodeBytes, &full[j]);
+  }
+  // Activation prologue set-up.  Each 32-element block is computed by a pair of
+  // adjacent lanes (16 elements each), so every prologue warp is busy even for the
+  // smallest token tile.  Rows past the tile's end are computed on zeros, which
+  // encode to zero codes and a zero scale (the lane pairs must stay converged).
+  // Group g of the prologue warps takes the CTA's K tiles g, g + kGroups, ...; the
+  // activation loads of its first kAhead K tiles are issued as soon as x may be
+  // read, so they land while the rest of the CTA sets up.
+  constexpr int kGT = C::kGroupThreads, kG = C::kGroups;
+  constexpr int kAhead = C::kTasks <= 2 ? 2 : 1;
+  const int pt = static_cast<int>(threadIdx.x) - 6 * 32;
+  const int grp = pt / kGT, gt = pt % kGT;
+  auto load = [&](int kt, uint4 (&xv)[C::kTasks][2], float (&d)[C::kRcp]) {
+#pragma unroll
+    for (int u = 0; u < C::kTasks; ++u) {
+      const int task = gt + u * kGT, t = task >> 4, c = (task >> 1) & 7, half = task & 1;
+      xv[u][0] = make_uint4(0, 0, 0, 0);
+      xv[u][1] = make_uint4(0, 0, 0, 0);
+      if (t < rows) {
+        const uint4* src = reinterpret_cast<const uint4*>(
+            p.x + static_cast<int64_t>(m0 + t) * p.K + static_cast<int64_t>(kt) * kKTile + c * kBlk + half * 16);
+        xv[u][0] = __ldg(src);
+        xv[u][1] = __ldg(src + 1);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < C::kRcp; ++e) d[e] = p.plain ? 1.f : __ldg(p.D + static_cast<int64_t>(kt) * kKTile + gt + e * kGT);
+  };
+  const int gst = nst > grp ? (nst - grp + kG - 1) / kG : 0;  // this group's K tiles
+  auto kt_of = [&](int jj) { return kt0 + grp + kG * jj; };
+  uint4 xpre[kAhead][C::kTasks][2];
+  float dpre[kAhead][C::kRcp];
+  if (warp >= 6) {
+    pdl_wait();  // x and D may come from the previous kernel on the stream
+#pragma unroll
+    for (int jj = 0; jj < kAhead; ++jj)
+      if (jj < gst) load(kt_of(jj), xpre[jj], dpre[jj]);
+  }
   // (scale rows >= BT of the activation scale image are copied to TMEM but never
   // read: the MMA's N extent is BT)
   if (warp == 1) {
@@ -844,8 +912,8 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   if (warp == 0) {
     // ---- producer: weight images; lanes 0 and 1 start a stage's two copies with one
     // instruction of the converged warp ----
-    for (int kt = kt0, j = 0; kt < kt1; ++kt, ++j) {
-      const int stage = j % kStages;
+    for (int j = pre; j < nst; ++j) {
+      const int kt = kt0 + j, stage = j % kStages;
       int ok = 1;
       if (lane == 0) {
         ok = mbar_wait(&empty[stage], ((j / kStages) & 1) ^ 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
@@ -923,32 +991,6 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
     }
   } else {
     // ---- activation prologue: x/D, FWHT32, BF16, E8M0, E2M1 -> swizzled B tile ----
-    // Each 32-element block is computed by a pair of adjacent lanes (16 elements
-    // each), so every prologue warp is busy even for the smallest token tile.
-    // Rows past the tile's end are computed on zeros, which encode to zero
-    // codes and a zero scale (the lane pairs must stay converged).  Group g of
-    // the prologue warps takes the CTA's K tiles g, g + kGroups, ...; the
-    // activation loads of up to kAhead of its K tiles are in flight before any compute.
-    constexpr int kGT = C::kGroupThreads, kG = C::kGroups;
-    constexpr int kAhead = C::kTasks <= 2 ? 2 : 1;
-    const int pt = threadIdx.x - 6 * 32;
-    const int grp = pt / kGT, gt = pt % kGT;
-    auto load = [&](int kt, uint4 (&xv)[C::kTasks][2], float (&d)[C::kRcp]) {
-#pragma unroll
-      for (int u = 0; u < C::kTasks; ++u) {
-        const int task = gt + u * kGT, t = task >> 4, c = (task >> 1) & 7, half = task & 1;
-        xv[u][0] = make_uint4(0, 0, 0, 0);
-        xv[u][1] = make_uint4(0, 0, 0, 0);
-        if (t < rows) {
-          const uint4* src = reinterpret_cast<const uint4*>(
-              p.x + static_cast<int64_t>(m0 + t) * p.K + static_cast<int64_t>(kt) * kKTile + c * kBlk + half * 16);
-          xv[u][0] = __ldg(src);
-          xv[u][1] = __ldg(src + 1);
-        }
-      }
-#pragma unroll
-      for (int e = 0; e < C::kRcp; ++e) d[e] = p.plain ? 1.f : __ldg(p.D + static_cast<int64_t>(kt) * kKTile + gt + e * kGT);
-    };
     // the group's jj-th K tile: CTA-local index j = grp + kG * jj
     auto stage_body = [&](int jj, uint4 (&xv)[C::kTasks][2], const float (&d)[C::kRcp]) -> bool {
       const int j = grp + kG * jj, stage = j % kStages;
@@ -988,36 +1030,38 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
       if (lane == 0) mbar_arrive(&full[stage]);
       return true;
     };
-    pdl_wait();  // x and D may come from the previous kernel on the stream
-    const int nst = kt1 - kt0;
-    const int gst = nst > grp ? (nst - grp + kG - 1) / kG : 0;  // this group's K tiles
-    auto kt_of = [&](int jj) { return kt0 + grp + kG * jj; };
     if (gst <= kAhead) {
-      uint4 xs[kAhead][C::kTasks][2];
-      float ds[kAhead][C::kRcp];
-#pragma unroll
-      for (int jj = 0; jj < kAhead; ++jj)
-        if (jj < gst) load(kt_of(jj), xs[jj], ds[jj]);
 #pragma unroll
       for (int jj = 0; jj < kAhead; ++jj) {
         if (jj >= gst) break;
-        if (!stage_body(jj, xs[jj], ds[jj])) break;
+        if (!stage_body(jj, xpre[jj], dpre[jj])) break;
       }
     } else if constexpr (C::kTasks >= 8) {
       // the largest token tile: registers hold one K tile of loads
-      uint4 xa[C::kTasks][2];
-      float da[C::kRcp];
-      for (int jj = 0; jj < gst; ++jj) {
-        load(kt_of(jj), xa, da);
-        if (!stage_body(jj, xa, da)) break;
+      if (stage_body(0, xpre[0], dpre[0])) {
+        uint4 xa[C::kTasks][2];
+        float da[C::kRcp];
+        for (int jj = 1; jj < gst; ++jj) {
+          load(kt_of(jj), xa, da);
+          if (!stage_body(jj, xa, da)) break;
+        }
       }
     } else {
       // deeper K ranges: one K tile of loads ahead
       uint4 xa[C::kTasks][2], xb[C::kTasks][2];
       float da[C::kRcp], db[C::kRcp];
-      load(kt_of(0), xa, da);
+#pragma unroll
+      for (int u = 0; u < C::kTasks; ++u) xa[u][0] = xpre[0][u][0], xa[u][1] = xpre[0][u][1];
+#pragma unroll
+      for (int e = 0; e < C::kRcp; ++e) da[e] = dpre[0][e];
+      if constexpr (kAhead >= 2) {
+#pragma unroll
+        for (int u = 0; u < C::kTasks; ++u) xb[u][0] = xpre[1][u][0], xb[u][1] = xpre[1][u][1];
+#pragma unroll
+        for (int e = 0; e < C::kRcp; ++e) db[e] = dpre[1][e];
+      }
       for (int jj = 0; jj < gst; jj += 2) {
-        if (jj + 1 < gst) load(kt_of(jj + 1), xb, db);
+        if (jj + 1 < gst && !(kAhead >= 2 && jj == 0)) load(kt_of(jj + 1), xb, db);
         if (!stage_body(jj, xa, da)) break;
         if (jj + 1 >= gst) break;
         if (jj + 2 < gst) load(kt_of(jj + 2), xa, da);
@@ -1272,7 +1316,7 @@ DenseWs dense_ws(int64_t M, int64_t K) {
   return w;
 }
 struct GroupedWs {
-  size_t goff, gtp, valid, tinfo, act, total;
+  size_t goff, gtp, gexp, valid, tinfo, act, total;
   int tiles_upper;
 };
 GroupedWs grouped_ws(int64_t M, int64_t K, int64_t E) {
@@ -1281,7 +1325,8 @@ GroupedWs grouped_ws(int64_t M, int64_t K, int64_t E) {
   const size_t KT = K / 256;
   w.goff = kWsReserved;
   w.gtp = align256(w.goff + (E + 1) * 8);
-  w.valid = align256(w.gtp + (E + 1) * 4);
+  w.gexp = align256(w.gtp + (E + 1) * 4);
+  w.valid = align256(w.gexp + E * 4);
   w.tinfo = align256(w.valid + 16);
   w.act = align256(w.tinfo + static_cast<size_t>(w.tiles_upper) * 16);
   w.total = w.act + static_cast<size_t>(w.tiles_upper) * KT * kActImageBytes;
@@ -1485,13 +1530,14 @@ static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, co
                  int group_list_type, int64_t E, uint16_t* y, int64_t M, int64_t N, int64_t K, void* workspace,
                  size_t workspace_bytes, int32_t* status, void* stream, bool plain) {
   if (E < 1 || E > kMaxGroups) return MACAQ_ERR_TOO_MANY_GROUPS;
-  if (group_list_type != 0 && group_list_type != 1) return MACAQ_ERR_GROUP_LIST_TYPE;
+  if (group_list_type < 0 || group_list_type > 2) return MACAQ_ERR_GROUP_LIST_TYPE;
   int st = check_mm_args(x, D, Wq, Ws, y, M, N, K, E, plain);
   if (st != MACAQ_OK) return st;
   if (M == 0) return MACAQ_OK;
   if (!group_list) return MACAQ_ERR_NULL;
   if (!aligned16(group_list)) return MACAQ_ERR_ALIGN;
-  if (overlaps(y, static_cast<size_t>(M) * N * 2, group_list, E * 8)) return MACAQ_ERR_ALIAS;
+  const size_t gl_bytes = static_cast<size_t>(E) * (group_list_type == 2 ? 16 : 8);
+  if (overlaps(y, static_cast<size_t>(M) * N * 2, group_list, gl_bytes)) return MACAQ_ERR_ALIAS;
   const GroupedWs w = grouped_ws(M, K, E);
   st = check_ws(workspace, workspace_bytes, w.total, y, static_cast<size_t>(M) * N * 2, x,
                 static_cast<size_t>(M) * K * 2);
@@ -1505,8 +1551,9 @@ static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, co
   int* gtp = reinterpret_cast<int*>(ws + w.gtp);
   int* valid = reinterpret_cast<int*>(ws + w.valid);
   int4* tinfo = reinterpret_cast<int4*>(ws + w.tinfo);
+  int* gexp = reinterpret_cast<int*>(ws + w.gexp);
   group_tables_kernel<<<1, 1024, 0, s>>>(group_list, group_list_type, static_cast<int>(E), static_cast<int>(M),
-                                         goff, gtp, tinfo, valid, status);
+                                         goff, gtp, gexp, tinfo, valid, status);
   if (cudaPeekAtLastError() != cudaSuccess) return MACAQ_ERR_CUDA;
   const int KT = static_cast<int>(K / 256);
   QuantParams qp{};
@@ -1521,7 +1568,7 @@ static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, co
   gp.M = static_cast<int>(M); gp.N = static_cast<int>(N); gp.K = static_cast<int>(K);
   gp.NT = static_cast<int>(pad128(N) / 128); gp.KT = KT; gp.E = static_cast<int>(E);
   gp.NT2 = (gp.NT + 1) / 2; gp.stages = gemm::stages_for(static_cast<int>(E));
-  gp.goff = goff; gp.gtp = gtp; gp.valid = valid;
+  gp.goff = goff; gp.gtp = gtp; gp.gexp = gexp; gp.valid = valid;
   gp.out_scale = plain ? 1.0f : 0.03125f;
   gp.status = status;
   const cudaError_t e = launch_ex(gemm_kernel, dim3(sms), dim3(gemm::kThreads),
