@@ -429,7 +429,7 @@ struct GemmParams {
 // work per instruction.
 namespace gemm {
 constexpr int kMaxStages = 4;
-constexpr int kThreads = 320;  // warp 0 producer, warp 1 MMA, warps 2-9 epilogue
+constexpr int kThreads = 352;  // warp 0 producer, warp 1 MMA, warps 2-9 epilogue, warp 10 scale copies
 constexpr int kTileN = 256;
 // A stage takes three copies: the weight codes of an image pair (32 KB), the
 // activation image (codes then scales, 17 KB) and the pair's scales (2 KB).
@@ -485,12 +485,15 @@ __device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int idx, int 
   return t;
 }
 
-// Scale copies and the four MMAs of one 256-K stage of the wide tile: D (+)= A x B^T
-// with N = 256.  Weight scales in TMEM: for each group of four scale blocks, eight
-// columns (rows 0-127 of B, then rows 128-255); activation scales four columns.
-__device__ __forceinline__ void mma_stage_wide(uint64_t adesc, uint64_t bdesc, uint64_t sfadesc, uint64_t sfbdesc,
-                                               uint32_t sf_col, uint32_t d_tmem, uint32_t idesc_lo,
-                                               uint32_t idesc_hi, bool first) {
+// Scale copies of one 256-K stage of the wide tile into its TMEM slot.  Weight
+// scales: for each group of four scale blocks, eight columns (rows 0-127 of B, then
+// rows 128-255); activation scales four columns.
+//
+// The copies are issued by a warp of their own, not by the MMA issuer: measured on
+// B200, a thread whose instruction stream mixes tcgen05.cp with an mbarrier wait
+// between stages issues block-scaled MMAs at ~190-200 cycles each instead of ~140,
+// while an issuer that only waits and issues MMAs keeps ~148.
+__device__ __forceinline__ void scale_copies_wide(uint64_t sfadesc, uint64_t sfbdesc, uint32_t sf_col) {
   constexpr uint64_t kBlk512 = 512 >> 4, kImg = kTileSfBytes >> 4;
   tc_cp_32x128b_warpx4(sf_col, sfadesc);
   tc_cp_32x128b_warpx4(sf_col + 4, sfadesc + kBlk512);
@@ -498,6 +501,12 @@ __device__ __forceinline__ void mma_stage_wide(uint64_t adesc, uint64_t bdesc, u
   tc_cp_32x128b_warpx4(sf_col + 12, sfbdesc + kImg);
   tc_cp_32x128b_warpx4(sf_col + 16, sfbdesc + kBlk512);
   tc_cp_32x128b_warpx4(sf_col + 20, sfbdesc + kImg + kBlk512);
+}
+
+// The four MMAs of one 256-K stage of the wide tile: D (+)= A x B^T with N = 256,
+// scales from the stage's TMEM slot (scale_copies_wide).
+__device__ __forceinline__ void mma_stage_wide(uint64_t adesc, uint64_t bdesc, uint32_t sf_col, uint32_t d_tmem,
+                                               uint32_t idesc_lo, uint32_t idesc_hi, bool first) {
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const uint32_t sfid = static_cast<uint32_t>(k & 1) * 2u;
@@ -508,17 +517,21 @@ __device__ __forceinline__ void mma_stage_wide(uint64_t adesc, uint64_t bdesc, u
   }
 }
 
-// Issue the scale copies and the four MMAs of one 256-K stage: D (+)= A-tile x B-tile^T.
-// adesc / bdesc describe the stage's code images, sfadesc / sfbdesc its scale images
-// (two 512-byte blocks each).  A descriptor's start address field counts 16-byte
-// units, so the descriptor of a later address is the first one plus the distance / 16.
-__device__ __forceinline__ void mma_stage(uint64_t adesc, uint64_t bdesc, uint64_t sfadesc, uint64_t sfbdesc,
-                                          uint32_t sfa_col, uint32_t sfb_col, uint32_t d_tmem, uint32_t idesc_lo,
-                                          uint32_t idesc_hi, bool first) {
+// Scale copies of one 256-K stage: sfadesc / sfbdesc describe the stage's scale
+// images (two 512-byte blocks each).  A descriptor's start address field counts
+// 16-byte units, so the descriptor of a later address is the first one plus the
+// distance / 16.
+__device__ __forceinline__ void scale_copies(uint64_t sfadesc, uint64_t sfbdesc, uint32_t sfa_col, uint32_t sfb_col) {
   tc_cp_32x128b_warpx4(sfa_col, sfadesc);
   tc_cp_32x128b_warpx4(sfa_col + 4, sfadesc + (512 >> 4));
   tc_cp_32x128b_warpx4(sfb_col, sfbdesc);
   tc_cp_32x128b_warpx4(sfb_col + 4, sfbdesc + (512 >> 4));
+}
+
+// The four MMAs of one 256-K stage: D (+)= A-tile x B-tile^T; adesc / bdesc describe
+// the stage's code images, the scales sit in TMEM from sfa_col / sfb_col.
+__device__ __forceinline__ void mma_stage(uint64_t adesc, uint64_t bdesc, uint32_t sfa_col, uint32_t sfb_col,
+                                          uint32_t d_tmem, uint32_t idesc_lo, uint32_t idesc_hi, bool first) {
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     // scale bytes 0-1 of each 32-bit TMEM word for the first 64 K, bytes 2-3 for the next;
@@ -539,8 +552,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
   uint8_t* staging = smem + S * kStageBytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(staging + kStagingBytes);
   uint64_t* empty = full + kMaxStages;
-  uint64_t* accf = empty + kMaxStages;  // accumulator complete
-  uint64_t* acce = accf + 1;            // accumulator drained by the epilogue
+  uint64_t* sfull = empty + kMaxStages;  // the stage's scales are in TMEM
+  uint64_t* accf = sfull + kMaxStages;   // accumulator complete
+  uint64_t* acce = accf + 1;             // accumulator drained by the epilogue
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(acce + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* epi_flag = abort_flag + 1;
@@ -571,6 +585,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sfull[s], 1);
     }
     mbar_init(accf, 1);
     mbar_init(acce, 8);  // one arrival per epilogue warp
@@ -656,7 +671,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
     if (lane == 0) {
       const uint32_t idesc_lo = idesc_mxf4(128, kTileN, 0, 0);
       const uint32_t idesc_hi = idesc_mxf4(128, kTileN, 2, 2);
-      const uint64_t code0 = sdesc_kmajor_sw128(smem_u32(smem)), sf0 = sdesc_sf_block(smem_u32(smem));
+      const uint64_t code0 = sdesc_kmajor_sw128(smem_u32(smem));
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
@@ -664,12 +679,16 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
         if (!mbar_wait(acce, (i & 1) ^ 1, abort_flag, kWaitTimeoutNs)) break;
         tc_fence_after();
         for (int kt = 0; kt < KT; ++kt) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, kWaitTimeoutNs)) { ok = false; break; }
+          // operands in shared memory, then their scales in TMEM (warp 10)
+          if (!mbar_wait(&full[stage], phase, abort_flag, kWaitTimeoutNs) ||
+              !mbar_wait(&sfull[stage], phase, abort_flag, kWaitTimeoutNs)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint32_t so = static_cast<uint32_t>(stage * kStageBytes) >> 4;
-          mma_stage_wide(code0 + so + (kOffA >> 4), code0 + so + (kOffB >> 4), sf0 + so + (kOffSfa >> 4),
-                         sf0 + so + (kOffSfb >> 4), tmem + kSfCol + kSfCols * stage, tmem, idesc_lo, idesc_hi,
-                         kt == 0);
+          mma_stage_wide(code0 + so + (kOffA >> 4), code0 + so + (kOffB >> 4), tmem + kSfCol + kSfCols * stage, tmem,
+                         idesc_lo, idesc_hi, kt == 0);
           tc_commit(&empty[stage]);
           if (++stage == S) {
             stage = 0;
@@ -678,6 +697,26 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
         }
         if (!ok) break;
         tc_commit(accf);
+      }
+    }
+  } else if (warp == 10) {
+    // ================= scale copies: each stage's scales into its TMEM slot =================
+    // A slot is rewritten only after its stage was refilled, which the producer does
+    // only after the MMAs that read the slot's previous contents completed.
+    if (lane == 0) {
+      const uint64_t sf0 = sdesc_sf_block(smem_u32(smem));
+      const int slots = my_tiles * KT;
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int j = 0; j < slots; ++j) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, kWaitTimeoutNs)) break;
+        const uint32_t so = static_cast<uint32_t>(stage * kStageBytes) >> 4;
+        scale_copies_wide(sf0 + so + (kOffSfa >> 4), sf0 + so + (kOffSfb >> 4), tmem + kSfCol + kSfCols * stage);
+        tc_commit(&sfull[stage]);
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
       }
     }
   } else {
@@ -930,6 +969,8 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
     }
   } else if (warp == 1) {
     if (lane == 0) {  // ---- MMA issuer ----
+      // This kernel is latency-bound: the scale copies go into the MMA issuer's own
+      // stream (no hand-off to another warp on the critical path).
       const uint32_t idesc_lo = idesc_mxf4(128, BT, 0, 0), idesc_hi = idesc_mxf4(128, BT, 2, 2);
       const uint64_t code0 = sdesc_kmajor_sw128(smem_u32(smem)), sf0 = sdesc_sf_block(smem_u32(smem));
       bool ok = true;
@@ -940,8 +981,9 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
         tc_fence_after();
         const uint32_t so = static_cast<uint32_t>(stage * C::kStageBytes) >> 4;
         const uint32_t sfa_col = tmem + C::kSfCol + 16 * stage;
-        mma_stage(code0 + so, code0 + so + (C::kOffB >> 4), sf0 + so + (C::kOffSfa >> 4), sf0 + so + (C::kOffSfb >> 4),
-                  sfa_col, sfa_col + 8, tmem, idesc_lo, idesc_hi, kt == kt0);
+        scale_copies(sf0 + so + (C::kOffSfa >> 4), sf0 + so + (C::kOffSfb >> 4), sfa_col, sfa_col + 8);
+        mma_stage(code0 + so, code0 + so + (C::kOffB >> 4), sfa_col, sfa_col + 8, tmem, idesc_lo, idesc_hi,
+                  kt == kt0);
         tc_commit(&empty[stage]);
         if (++stage == kStages) {
           stage = 0;
