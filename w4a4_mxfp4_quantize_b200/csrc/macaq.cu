@@ -520,7 +520,7 @@ __device__ __forceinline__ void mma_stage_wide(uint64_t adesc, uint64_t bdesc, u
 // Scale copies of one 256-K stage: sfadesc / sfbdesc describe the stage's scale
 // images (two 512-byte blocks each).  A descriptor's start address field counts
 // 16-byte units, so the descriptor of a later address is the first one plus the
-// distance / 16.
+// distance / 16.  Issued by a warp other than the MMA issuer (see scale_copies_wide).
 __device__ __forceinline__ void scale_copies(uint64_t sfadesc, uint64_t sfbdesc, uint32_t sfa_col, uint32_t sfb_col) {
   tc_cp_32x128b_warpx4(sfa_col, sfadesc);
   tc_cp_32x128b_warpx4(sfa_col + 4, sfadesc + (512 >> 4));
@@ -843,7 +843,8 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   uint64_t* empty = full + kStages;
   uint64_t* accf = empty + kStages;
   uint64_t* recv_bar = accf + 1;  // completes when every rank's partial rows for this CTA have landed
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(recv_bar + 1);
+  uint64_t* sfull = recv_bar + 1;  // [kStages] the stage's scales are in TMEM
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sfull + kStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   volatile int* epi_flag = abort_flag + 1;
   volatile int* pro_flag = abort_flag + 2;  // [group][2]
@@ -865,6 +866,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1 + fused::kProWarps / C::kGroups);
       mbar_init(&empty[s], 1);
+      mbar_init(&sfull[s], 1);
     }
     mbar_init(&accf[0], 1);
     if (split) {
@@ -969,19 +971,22 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
     }
   } else if (warp == 1) {
     if (lane == 0) {  // ---- MMA issuer ----
-      // This kernel is latency-bound: the scale copies go into the MMA issuer's own
-      // stream (no hand-off to another warp on the critical path).
+      // The scale copies come from warp 2: measured on this kernel, the hand-off costs
+      // less than the slower MMA issue of a thread that mixes tcgen05.cp and waits.
       const uint32_t idesc_lo = idesc_mxf4(128, BT, 0, 0), idesc_hi = idesc_mxf4(128, BT, 2, 2);
-      const uint64_t code0 = sdesc_kmajor_sw128(smem_u32(smem)), sf0 = sdesc_sf_block(smem_u32(smem));
+      const uint64_t code0 = sdesc_kmajor_sw128(smem_u32(smem));
       bool ok = true;
       int stage = 0;
       uint32_t phase = 0;
       for (int kt = kt0; kt < kt1; ++kt) {
-        if (!mbar_wait(&full[stage], phase, abort_flag, kWaitTimeoutNs)) { ok = false; break; }
+        if (!mbar_wait(&full[stage], phase, abort_flag, kWaitTimeoutNs) ||
+            !mbar_wait(&sfull[stage], phase, abort_flag, kWaitTimeoutNs)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         const uint32_t so = static_cast<uint32_t>(stage * C::kStageBytes) >> 4;
         const uint32_t sfa_col = tmem + C::kSfCol + 16 * stage;
-        scale_copies(sf0 + so + (C::kOffSfa >> 4), sf0 + so + (C::kOffSfb >> 4), sfa_col, sfa_col + 8);
         mma_stage(code0 + so, code0 + so + (C::kOffB >> 4), sfa_col, sfa_col + 8, tmem, idesc_lo, idesc_hi,
                   kt == kt0);
         tc_commit(&empty[stage]);
@@ -993,9 +998,29 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
       if (ok) tc_commit(&accf[0]);
     }
   } else if (warp < 6) {
-    // ---- epilogue: FP32 partial tile to local shared memory, then one bulk copy per owner ----
+    // ---- during the mainloop, warp 2 copies each stage's scales into its TMEM slot (a
+    // slot is rewritten only after its stage was refilled, which happens only after
+    // the MMAs that read the slot completed); then the epilogue: FP32 partial tile to
+    // local shared memory, then one bulk copy per owner ----
     const int q = warp & 3;
     const int et = threadIdx.x - 64;
+    if (et == 0) {
+      const uint64_t sf0 = sdesc_sf_block(smem_u32(smem));
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int kt = kt0; kt < kt1; ++kt) {
+        if (!mbar_wait(&full[stage], phase, abort_flag, kWaitTimeoutNs)) break;
+        const uint32_t so = static_cast<uint32_t>(stage * C::kStageBytes) >> 4;
+        const uint32_t sfa_col = tmem + C::kSfCol + 16 * stage;
+        scale_copies(sf0 + so + (C::kOffSfa >> 4), sf0 + so + (C::kOffSfb >> 4), sfa_col, sfa_col + 8);
+        tc_commit(&sfull[stage]);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    __syncwarp();
     if (et == 0) *epi_flag = mbar_wait(&accf[0], 0, abort_flag, kWaitTimeoutNs) ? 1 : 0;
     named_bar_sync(1, 128);
     if (*epi_flag) {
