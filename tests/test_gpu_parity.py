@@ -393,6 +393,50 @@ def test_dense_quantise_once_path_ragged(M):
     compare(_run_dense(p), _oracle_dense_full(p), f"two-kernel M={M}")
 
 
+def _decode_activation_images(ws: np.ndarray, M: int, K: int):
+    """Canonical codes [M, K/2] and scales [M, K/32] read back from the dense
+    quantise-once workspace: 4096 reserved bytes, then one image per (128-row
+    tile, 256-K tile) of 17408 bytes -- 16384 code bytes (row r at 128 r, its
+    16-byte chunk for block c at (c ^ (r mod 8)) * 16) then 1024 scale bytes
+    (block c of row r at 512 (c // 4) + 16 (r mod 32) + 4 (r // 32) + c mod 4)."""
+    KT = K // 256
+    tiles = (M + 127) // 128
+    imgs = ws[4096:4096 + tiles * KT * 17408].reshape(tiles, KT, 17408)
+    r = np.arange(128)[:, None]
+    c = np.arange(8)[None, :]
+    phys = (c ^ (r & 7))                                     # [128, 8] physical chunk of logical block c
+    codes = imgs[:, :, :16384].reshape(tiles, KT, 128, 8, 16)
+    codes = np.take_along_axis(codes, phys[None, None, :, :, None], axis=3)     # logical block order
+    codes = codes.transpose(0, 2, 1, 3, 4).reshape(tiles * 128, K // 2)[:M]
+    sf_idx = 512 * (c // 4) + 16 * (r % 32) + 4 * (r // 32) + (c % 4)           # [128, 8]
+    scales = imgs[:, :, 16384:][:, :, sf_idx]                                  # [tiles, KT, 128, 8]
+    scales = scales.transpose(0, 2, 1, 3).reshape(tiles * 128, K // 32)[:M]
+    return codes, scales
+
+
+@pytest.mark.parametrize("M,K,plain", [(300, 768, False), (4096, 1024, False), (1000, 512, True)])
+def test_quantise_once_activation_images_bit_exact(M, K, plain):
+    # the quantiser of the two-kernel path writes each row's codes and scales
+    # into the GEMM's tile images; rows past M are never written (their output
+    # rows are never stored), so only rows < M are compared
+    p = synth.dense(M, K, 256, seed=7 + M)
+    x = x_to_dev(p.x)
+    ws = torch.zeros(mq.workspace_bytes(M, 256, K), dtype=torch.uint8, device="cuda")
+    if plain:
+        Wq, Ws = mq.prepare_weights_plain(f32_dev(p.W))
+        mq.dense_mm_plain(x, Wq, Ws, 256, ws=ws)
+        qa, sa = oracle.quantize_act_plain(p.x)
+    else:
+        D = f32_dev(p.D[0])
+        Wq, Ws = mq.prepare_weights(f32_dev(p.W), f32_dev(p.D))
+        mq.dense_mm(x, D, Wq, Ws, 256, ws=ws)
+        qa, sa = oracle.quantize_act(p.x, p.D[0])
+    torch.cuda.synchronize()
+    codes, scales = _decode_activation_images(ws.cpu().numpy(), M, K)
+    assert np.array_equal(codes, qa), "activation codes differ from the oracle"
+    assert np.array_equal(scales, sa), "activation scales differ from the oracle"
+
+
 def test_max_rows_sampled():
     # the MACAQ page's maximum-row checks go to M = 65,536; one more row for a partial tile
     for M in (65536, 65537):

@@ -186,47 +186,59 @@ __global__ void mx_encode_kernel(const float* __restrict__ v, uint8_t* __restric
 // ============================================================================
 // Grouped form: device-side group_list validation and tables
 // ============================================================================
-// Block-wide exclusive scan of one int64 per thread (blockDim.x <= 1024).
-__device__ __forceinline__ int64_t block_excl_scan(int64_t v, int64_t* scratch, int64_t& total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
-  int64_t inc = v;
+// Block-wide exclusive scans of three int64 per thread at once (blockDim.x a
+// multiple of 32, at most 1024): one pass of warp shuffles, one exchange of the
+// warp totals through shared memory.  tot receives the three block totals.
+__device__ __forceinline__ void block_excl_scan3(const int64_t (&v)[3], int64_t (&res)[3], int64_t (&tot)[3],
+                                                 int64_t* scratch /* [32][3] + [32][3] */) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int64_t inc[3] = {v[0], v[1], v[2]};
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int64_t u = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += u;
-  }
-  if (lane == 31) scratch[warp] = inc;
-  __syncthreads();
-  if (warp == 0) {
-    const int64_t w = lane < nw ? scratch[lane] : 0;
-    int64_t wi = w;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int64_t u = __shfl_up_sync(0xffffffffu, wi, o);
-      if (lane >= o) wi += u;
+    for (int i = 0; i < 3; ++i) {
+      const int64_t u = __shfl_up_sync(0xffffffffu, inc[i], o);
+      if (lane >= o) inc[i] += u;
     }
-    if (lane < nw) scratch[32 + lane] = wi - w;
-    if (lane == nw - 1) scratch[64] = wi;
   }
+  if (lane == 31)
+    for (int i = 0; i < 3; ++i) scratch[warp * 3 + i] = inc[i];
   __syncthreads();
-  const int64_t res = scratch[32 + warp] + inc - v;
-  total = scratch[64];
-  __syncthreads();
-  return res;
+  // every warp scans the warp totals itself (no second barrier round)
+  int64_t wi[3];
+#pragma unroll
+  for (int i = 0; i < 3; ++i) wi[i] = lane < nw ? scratch[lane * 3 + i] : 0;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+#pragma unroll
+    for (int i = 0; i < 3; ++i) {
+      const int64_t u = __shfl_up_sync(0xffffffffu, wi[i], o);
+      if (lane >= o) wi[i] += u;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 3; ++i) {
+    const int64_t before = warp > 0 ? __shfl_sync(0xffffffffu, wi[i], warp - 1) : 0;  // totals of earlier warps
+    res[i] = before + inc[i] - v[i];
+    tot[i] = __shfl_sync(0xffffffffu, wi[i], nw - 1);
+  }
 }
 
-// One CTA of 1024 threads, thread g owns group g.  Rules (npu_grouped_matmul,
+// One CTA of 32 * ceil(E / 32) threads, thread g owns group g.  Rules (npu_grouped_matmul,
 // group_list / group_list_type): type 0 non-negative and non-decreasing
 // cumulative sums, type 1 non-negative counts; the rows must total M.
 // Writes goff[0..E] (row offsets), gtp[0..E] (prefix of 128-row tiles per
 // list entry), gexp[0..E) (the expert of each entry: the entry itself for types
-// 0 and 1, the named group index for type 2) and *valid; on a violation also
+// 0 and 1, the named group index for type 2), the slab table for the quantiser
+// (per 32-row slab holding rows: {expert, first row of x, rows, 4 * tile +
+// quarter of the tile}), its length *nslabs and *valid; on a violation also
 // *status.
 __global__ void __launch_bounds__(1024) group_tables_kernel(const int64_t* __restrict__ gl, int type, int E, int M,
                                                             int64_t* __restrict__ goff, int* __restrict__ gtp,
-                                                            int* __restrict__ gexp, int4* __restrict__ tinfo,
-                                                            int* __restrict__ valid, int32_t* status) {
-  __shared__ int64_t scratch[72];
+                                                            int* __restrict__ gexp, int4* __restrict__ slabs,
+                                                            int* __restrict__ nslabs, int* __restrict__ valid,
+                                                            int32_t* status) {
+  __shared__ int64_t scratch[96];
   const int g = threadIdx.x;
   int64_t cnt = 0;
   bool bad = false;
@@ -245,9 +257,11 @@ __global__ void __launch_bounds__(1024) group_tables_kernel(const int64_t* __res
   }
   bad = __syncthreads_or(bad);
   if (!bad) {
-    int64_t rows_total, tiles_total;
-    const int64_t rb = block_excl_scan(cnt, scratch, rows_total);
-    const int64_t tb = block_excl_scan((cnt + kRowsTile - 1) / kRowsTile, scratch, tiles_total);
+    const int64_t v[3] = {cnt, (cnt + kRowsTile - 1) / kRowsTile, (cnt + 31) / 32};
+    int64_t pre[3], tot[3];
+    block_excl_scan3(v, pre, tot, scratch);
+    const int64_t rb = pre[0], tb = pre[1], sb = pre[2];
+    const int64_t rows_total = tot[0], tiles_total = tot[1], slabs_total = tot[2];
     bad = rows_total != M;
     if (g < E) {
       goff[g] = rb;
@@ -257,12 +271,13 @@ __global__ void __launch_bounds__(1024) group_tables_kernel(const int64_t* __res
     if (g == 0) {
       goff[E] = rows_total;
       gtp[E] = static_cast<int>(tiles_total);
+      *nslabs = static_cast<int>(slabs_total);
     }
-    // per row tile: {group, first row, rows}, one load for the quantiser
+    // slab j of this entry: rows [rb + 32 j, ...) of x, quarter j % 4 of tile tb + j / 4
     if (g < E && !bad)
-      for (int64_t j = 0; j * kRowsTile < cnt; ++j)
-        tinfo[tb + j] = make_int4(ex, static_cast<int>(rb + j * kRowsTile),
-                                  static_cast<int>(cnt - j * kRowsTile < kRowsTile ? cnt - j * kRowsTile : kRowsTile), 0);
+      for (int64_t j = 0; j * 32 < cnt; ++j)
+        slabs[sb + j] = make_int4(ex, static_cast<int>(rb + 32 * j),
+                                  static_cast<int>(cnt - 32 * j < 32 ? cnt - 32 * j : 32), static_cast<int>(4 * tb + j));
   }
   if (g == 0) {
     *valid = bad ? 0 : 1;
@@ -283,118 +298,132 @@ __device__ __forceinline__ int find_group(const int* gtp, int E, int pm) {
 // ============================================================================
 // Quantise-once: activation prologue over every row into tile images
 // ============================================================================
-// Work unit = 32 rows of one 128-row tile x one K tile (one 32-element block per
-// thread).  Dense: tile pm holds rows [128 pm, 128 pm + 128).  Grouped: tile pm
-// belongs to group g and holds that group's rows from a first row given by the
-// per-tile table; rows past the group's end are zero.  The grid is persistent:
-// each CTA walks units blockIdx.x, + gridDim.x, ...; every thread keeps the
-// activations of its next kQuantAhead units in flight with cp.async into its own
-// slots of a shared-memory ring (no registers held), so HBM streams while the
-// ALUs work.
+// Work unit = one 32-row slab of a 128-row tile x one K tile: thread (tr, c) =
+// (threadIdx.x / 8, threadIdx.x % 8) takes row tr of the slab and its 32-element
+// block c.  Only slabs that hold rows are enumerated: dense, slab s is rows
+// [32 s, 32 s + 32) of x (quarter s % 4 of tile s / 4); grouped, the slab table
+// written by group_tables_kernel gives each slab's expert, first row of x, row
+// count and quarter.  Rows past a slab's end are neither read nor written: the
+// GEMM never stores the output rows they feed (a row of the product depends on
+// its own activation row only).  Unit u is slab u % L of K tile u / L; the grid
+// is persistent, each CTA stepping through units blockIdx.x, + gridDim.x, ...
+// with the slab and K tile advanced incrementally (no division per unit).
+// Every thread keeps the activations of its next kQuantAhead units in flight
+// with cp.async into its own slots of a shared-memory ring (no registers held),
+// so HBM streams while the ALUs work.
 struct QuantParams {
   const uint16_t* x;
-  const float* D;        // [E, K]
-  uint8_t* Aq;           // [tiles][KT] activation images of kActImageBytes
-  int M, K, E, MT;       // MT: dense row tiles
-  const int64_t* goff;   // grouped tables (nullptr: dense)
-  const int* gtp;
-  const int4* tinfo;     // grouped: per row tile {group, first row, rows}
+  const float* D;       // [E, K]
+  uint8_t* Aq;          // [tiles][KT] activation images of kActImageBytes
+  int M, K;
+  const int4* slabs;    // grouped: slab table (nullptr: dense)
+  const int* nslabs;    // grouped: its length
   const int* valid;
-  int plain;             // plain MXFP4 (no D, no Hadamard; D not read)
+  int plain;            // plain MXFP4 (no D, no Hadamard; D not read)
 };
 
 constexpr int kQuantStages = 3;                 // ring slots: the current unit and two ahead
 constexpr int kQuantAhead = kQuantStages - 1;
 constexpr int kQuantSlotBytes = 256 * 64;       // one unit: 256 threads x one 32-element block
+// Within a slot, 16-byte chunk j of thread i sits at (j * 256 + i) * 16: a warp's
+// loads of chunk j are 512 consecutive bytes (no bank conflict).
 constexpr int kQuantSmem = kQuantStages * kQuantSlotBytes;
 
 __global__ void __launch_bounds__(256, 4) quant_tiles_kernel(const __grid_constant__ QuantParams p) {
-  extern __shared__ __align__(16) uint8_t qsmem[];  // ring [kQuantStages][256][64]
+  extern __shared__ __align__(16) uint8_t qsmem[];  // ring [kQuantStages][4 chunks][256 threads][16]
   __shared__ __align__(16) float r[2][kRcpTile];
   pdl_trigger();  // the GEMM may start streaming weights; it waits for our results before reading them
   pdl_wait();     // x (and the grouped tables) may come from the preceding kernels
   const int KT = p.K / kKTile;
-  int tiles = p.MT;
-  if (p.gtp != nullptr) {
+  int L = (p.M + 31) / 32;
+  if (p.slabs != nullptr) {
     if (*p.valid == 0) return;
-    tiles = p.gtp[p.E];
+    L = *p.nslabs;
   }
-  const int units = tiles * 4 * KT;
+  const int units = L * KT;
+  const int G = static_cast<int>(gridDim.x);
+  if (L <= 0 || static_cast<int>(blockIdx.x) >= units) return;
   const int tr = threadIdx.x >> 3, c = threadIdx.x & 7;
+  const int gq = G / L, gr = G % L;  // one stride of G units: gq K tiles and gr slabs further
   struct Unit {
-    uint8_t* img;     // the unit's activation image
-    const float* dp;  // D of this thread's channel
-    int t;            // this thread's row in the tile
-    bool live;        // the row exists
+    uint8_t* img;  // the unit's activation image
+    float d;       // D of this thread's channel (loaded with the activations)
+    int t;         // this thread's row in the tile; negative: the row does not exist
   };
-  // unit u: kt = u % KT, sub = (u / KT) % 4, pm = u / (4 KT); issues its activation copy into `slot`
-  auto fetch = [&](int u, int slot) {
+  // Issues the activation copy of the unit at (slab s, K tile kt) into ring `slot`.
+  auto fetch = [&](int sl, int kt, int slot) {
     Unit w;
-    const int kt = u % KT, q = u / KT, pm = q >> 2;
-    w.t = (q & 3) * 32 + tr;
-    int base, rows, g = 0;
-    if (p.gtp != nullptr) {
-      const int4 ti = p.tinfo[pm];
-      g = ti.x;
-      base = ti.y;
-      rows = ti.z;
+    int ex = 0, row0, nrows, quarter;
+    if (p.slabs != nullptr) {
+      const int4 e = p.slabs[sl];
+      ex = e.x;
+      row0 = e.y;
+      nrows = e.z;
+      quarter = e.w;
     } else {
-      base = pm * kRowsTile;
-      rows = min(kRowsTile, p.M - base);
+      row0 = sl * 32;
+      nrows = min(32, p.M - row0);
+      quarter = sl;
     }
-    w.live = w.t < rows;
-    w.img = p.Aq + (static_cast<size_t>(pm) * KT + kt) * kActImageBytes;
+    const bool live = tr < nrows;
+    w.t = live ? (quarter & 3) * 32 + tr : -1;
+    w.img = p.Aq + (static_cast<size_t>(quarter >> 2) * KT + kt) * kActImageBytes;
     const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
-    w.dp = p.plain ? nullptr : p.D + static_cast<int64_t>(g) * p.K + k0 + threadIdx.x;
-    if (w.live) {
-      const uint16_t* src = p.x + (static_cast<int64_t>(base) + w.t) * p.K + k0 + c * kBlk;
-      uint8_t* dst = qsmem + (slot * 256 + threadIdx.x) * 64;
+    w.d = p.plain ? 1.f : __ldg(p.D + static_cast<int64_t>(ex) * p.K + k0 + threadIdx.x);
+    if (live) {
+      const uint16_t* src = p.x + (static_cast<int64_t>(row0) + tr) * p.K + k0 + c * kBlk;
+      uint8_t* dst = qsmem + slot * kQuantSlotBytes + threadIdx.x * 16;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) cp_async16(dst + 16 * i, src + 8 * i);
+      for (int i = 0; i < 4; ++i) cp_async16(dst + 4096 * i, src + 8 * i);
     }
     cp_async_commit();  // one group per unit, empty when the row does not exist
     return w;
   };
-  int u = blockIdx.x;
-  if (u >= units) return;
+  // (fs, fk): slab and K tile of the next unit to fetch; fk == KT past the end
+  int fs = static_cast<int>(blockIdx.x) % L, fk = static_cast<int>(blockIdx.x) / L;
+  auto step = [&]() {
+    fs += gr;
+    fk += gq;
+    if (fs >= L) {
+      fs -= L;
+      ++fk;
+    }
+  };
   Unit ring[kQuantStages];
 #pragma unroll
   for (int s = 0; s < kQuantAhead; ++s) {
-    const int us = u + s * static_cast<int>(gridDim.x);
-    if (us < units) ring[s] = fetch(us, s);
+    if (fk < KT) ring[s] = fetch(fs, fk, s);
     else cp_async_commit();
+    step();
   }
-  float d = p.plain ? 1.f : __ldg(ring[0].dp);
   int buf = 0;  // reciprocal buffer of this unit: alternates unit by unit
+  int u = static_cast<int>(blockIdx.x);
   // unit i of this CTA uses ring slot i % kQuantStages; unrolled so slots are static
   while (u < units) {
 #pragma unroll
     for (int k = 0; k < kQuantStages; ++k) {
       if (u >= units) break;
       {  // the unit kQuantAhead ahead goes into the slot freed last iteration
-        const int ua = u + kQuantAhead * static_cast<int>(gridDim.x);
         const int sa = (k + kQuantAhead) % kQuantStages;
-        if (ua < units) ring[sa] = fetch(ua, sa);
+        if (fk < KT) ring[sa] = fetch(fs, fk, sa);
         else cp_async_commit();
+        step();
       }
       const Unit w = ring[k];
-      const int un = u + static_cast<int>(gridDim.x);
-      const float dn = (un < units && !p.plain) ? __ldg(ring[(k + 1) % kQuantStages].dp) : 1.f;
-      r[buf][rcp_index(threadIdx.x)] = __frcp_rn(d);
+      r[buf][rcp_index(threadIdx.x)] = __frcp_rn(w.d);
       cp_async_wait<kQuantAhead>();  // this thread's copy of this unit has landed
       __syncthreads();               // every reciprocal written; r[buf] of two units back no longer read
-      uint4 cv = make_uint4(0, 0, 0, 0);
-      uint32_t sc = 0;
-      if (w.live) {
-        const uint4* xs = reinterpret_cast<const uint4*>(qsmem + (k * 256 + threadIdx.x) * 64);
-        const uint4 xv[4] = {xs[0], xs[1], xs[2], xs[3]};
+      if (w.t >= 0) {
+        uint4 cv;
+        uint32_t sc;
+        const uint4* xs = reinterpret_cast<const uint4*>(qsmem + k * kQuantSlotBytes) + threadIdx.x;
+        const uint4 xv[4] = {xs[0], xs[256], xs[512], xs[768]};
         if (p.plain) act_block_plain(xv, cv, sc);
         else act_block(xv, r[buf] + c * kRcpStride, cv, sc);
+        *reinterpret_cast<uint4*>(w.img + code_chunk_offset(w.t, c)) = cv;
+        w.img[kTileCodeBytes + sf_offset(w.t, c)] = static_cast<uint8_t>(sc);
       }
-      *reinterpret_cast<uint4*>(w.img + code_chunk_offset(w.t, c)) = cv;
-      w.img[kTileCodeBytes + sf_offset(w.t, c)] = static_cast<uint8_t>(sc);
-      d = dn;
-      u = un;
+      u += G;
       buf ^= 1;
     }
   }
@@ -1383,7 +1412,7 @@ DenseWs dense_ws(int64_t M, int64_t K) {
   return w;
 }
 struct GroupedWs {
-  size_t goff, gtp, gexp, valid, tinfo, act, total;
+  size_t goff, gtp, gexp, valid, slabs, act, total;
   int tiles_upper;
 };
 GroupedWs grouped_ws(int64_t M, int64_t K, int64_t E) {
@@ -1394,8 +1423,8 @@ GroupedWs grouped_ws(int64_t M, int64_t K, int64_t E) {
   w.gtp = align256(w.goff + (E + 1) * 8);
   w.gexp = align256(w.gtp + (E + 1) * 4);
   w.valid = align256(w.gexp + E * 4);
-  w.tinfo = align256(w.valid + 16);
-  w.act = align256(w.tinfo + static_cast<size_t>(w.tiles_upper) * 16);
+  w.slabs = align256(w.valid + 16);  // valid flag, then the slab count
+  w.act = align256(w.slabs + static_cast<size_t>((M + 31) / 32 + E) * 16);
   w.total = w.act + static_cast<size_t>(w.tiles_upper) * KT * kActImageBytes;
   return w;
 }
@@ -1423,10 +1452,11 @@ int check_ws(void* ws, size_t ws_bytes, size_t need, const void* y, size_t ybyte
   return MACAQ_OK;
 }
 
-// Persistent quantiser grid: four CTAs per SM at most, no more than the units.
-int quant_grid(int tiles, int KT, int sms) {
-  const int64_t units = static_cast<int64_t>(tiles) * 4 * KT;
-  return static_cast<int>(std::min<int64_t>(units, static_cast<int64_t>(sms) * 4));
+// Persistent quantiser grid: four CTAs per SM at most, no more than the units
+// (32-row slabs x K tiles; for grouped calls an upper bound).
+int quant_grid(int64_t slabs, int KT, int sms) {
+  const int64_t units = slabs * KT;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, static_cast<int64_t>(sms) * 4)));
 }
 
 // Dense quantise-once: the quantiser over all rows, then the GEMM (launched as
@@ -1438,8 +1468,9 @@ int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, c
   const int MT = static_cast<int>(pad128(M) / 128), KT = static_cast<int>(K / 256);
   QuantParams qp{};
   qp.x = x; qp.D = D; qp.Aq = ws + w.act;
-  qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = 1; qp.MT = MT; qp.plain = plain ? 1 : 0;
-  if (launch_ex(quant_tiles_kernel, dim3(quant_grid(MT, KT, sms)), dim3(256), kQuantSmem, st, pdl, 1, qp) !=
+  qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.plain = plain ? 1 : 0;
+  if (launch_ex(quant_tiles_kernel, dim3(quant_grid((M + 31) / 32, KT, sms)), dim3(256), kQuantSmem, st, pdl, 1,
+                qp) !=
       cudaSuccess)
     return MACAQ_ERR_CUDA;
   GemmParams gp{};
@@ -1617,18 +1648,18 @@ static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, co
   int64_t* goff = reinterpret_cast<int64_t*>(ws + w.goff);
   int* gtp = reinterpret_cast<int*>(ws + w.gtp);
   int* valid = reinterpret_cast<int*>(ws + w.valid);
-  int4* tinfo = reinterpret_cast<int4*>(ws + w.tinfo);
+  int4* slabs = reinterpret_cast<int4*>(ws + w.slabs);
   int* gexp = reinterpret_cast<int*>(ws + w.gexp);
-  group_tables_kernel<<<1, 1024, 0, s>>>(group_list, group_list_type, static_cast<int>(E), static_cast<int>(M),
-                                         goff, gtp, gexp, tinfo, valid, status);
+  group_tables_kernel<<<1, static_cast<unsigned>((E + 31) / 32 * 32), 0, s>>>(group_list, group_list_type, static_cast<int>(E), static_cast<int>(M),
+                                         goff, gtp, gexp, slabs, valid + 1, valid, status);
   if (cudaPeekAtLastError() != cudaSuccess) return MACAQ_ERR_CUDA;
   const int KT = static_cast<int>(K / 256);
   QuantParams qp{};
   qp.x = x; qp.D = D; qp.Aq = ws + w.act;
-  qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.E = static_cast<int>(E);
-  qp.goff = goff; qp.gtp = gtp; qp.tinfo = tinfo; qp.valid = valid; qp.plain = plain ? 1 : 0;
-  if (launch_ex(quant_tiles_kernel, dim3(quant_grid(w.tiles_upper, KT, sms)), dim3(256), kQuantSmem, s, true, 1,
-                qp) != cudaSuccess)
+  qp.M = static_cast<int>(M); qp.K = static_cast<int>(K);
+  qp.slabs = slabs; qp.nslabs = valid + 1; qp.valid = valid; qp.plain = plain ? 1 : 0;
+  if (launch_ex(quant_tiles_kernel, dim3(quant_grid((M + 31) / 32 + E, KT, sms)), dim3(256), kQuantSmem, s, true,
+                1, qp) != cudaSuccess)
     return MACAQ_ERR_CUDA;
   GemmParams gp{};
   gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.y = y;
