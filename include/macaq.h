@@ -52,7 +52,7 @@
 extern "C" {
 #endif
 
-#define MACAQ_ABI_VERSION 2
+#define MACAQ_ABI_VERSION 3
 
 #define MACAQ_OK 0
 #define MACAQ_ERR_NULL (-1)               /* a required pointer is NULL */
@@ -67,6 +67,7 @@ extern "C" {
 #define MACAQ_ERR_GROUP_LIST_INVALID (-10)/* (device) group_list breaks the rules */
 #define MACAQ_ERR_WORKSPACE (-11)         /* workspace missing or too small */
 #define MACAQ_ERR_BAD_D (-12)             /* D has a zero or non-finite entry */
+#define MACAQ_ERR_ACT_TYPE (-13)          /* act_type not 0, 1, 2, 4 or 5 */
 
 /* Name of a status code (static string). */
 const char *macaq_status_string(int status);
@@ -131,6 +132,34 @@ int macaq_grouped_mm(const uint16_t *x_dev, const float *D_dev, const uint8_t *W
                      const int64_t *group_list_dev, int group_list_type, int64_t E, uint16_t *y_dev,
                      int64_t M, int64_t N, int64_t K, void *workspace_dev, size_t workspace_bytes,
                      int32_t *status_dev, void *stream);
+
+/* ------------------------------------------------------------------ */
+/* Output bias and activation                                          */
+/* ------------------------------------------------------------------ */
+
+/* The dense and grouped calls above with npu_grouped_matmul's bias and
+ * act_type (that page, parameters bias and act_type; function description
+ * y_i = x_i @ weight_i + bias_i):
+ *     y = RNE_bf16( act( 2^-5 * (block-scaled FP32 sum) + bias[n] ) )
+ * evaluated in FP32 before the single rounding to BF16.
+ *   bias_dev: fp32, [N] for the dense call, [E, N] for the grouped call (the
+ *     rows of a group_list entry take the row of the expert they use), or
+ *     NULL for no bias; 16-byte aligned; must not overlap y.
+ *   act_type: 0 none, 1 RELU, 2 GELU_TANH (0.5 v (1 + tanh(sqrt(2/pi)
+ *     (v + 0.044715 v^3)))), 4 FAST_GELU (read as v * sigmoid(1.702 v); the
+ *     page names it without a formula), 5 SILU (v * sigmoid(v)).  3 is not
+ *     supported on the page and, like any other value, returns
+ *     MACAQ_ERR_ACT_TYPE without launching.
+ * All other arguments, the workspace and the error behaviour are those of
+ * macaq_dense_mm / macaq_grouped_mm; with bias NULL and act_type 0 the result
+ * is theirs. */
+int macaq_dense_mm_ex(const uint16_t *x_dev, const float *D_dev, const uint8_t *Wq_dev, const uint8_t *Ws_dev,
+                      const float *bias_dev, int act_type, uint16_t *y_dev, int64_t M, int64_t N, int64_t K,
+                      void *workspace_dev, size_t workspace_bytes, int32_t *status_dev, void *stream);
+int macaq_grouped_mm_ex(const uint16_t *x_dev, const float *D_dev, const uint8_t *Wq_dev, const uint8_t *Ws_dev,
+                        const int64_t *group_list_dev, int group_list_type, int64_t E, const float *bias_dev,
+                        int act_type, uint16_t *y_dev, int64_t M, int64_t N, int64_t K, void *workspace_dev,
+                        size_t workspace_bytes, int32_t *status_dev, void *stream);
 
 /* ------------------------------------------------------------------ */
 /* Plain MXFP4 W4A4 baseline                                           */
@@ -205,8 +234,8 @@ int macaq_unfused_dense_mm(const uint16_t *x_dev, const float *D_dev, const uint
  *   The first call on a device looks up the buffer's device address (a
  *   runtime query, no allocation); make that first call before any stream
  *   capture on that device.
- *   Every call shares the one buffer and fully rewrites the part it uses
- *   (nothing in it has to start at zero).  Calls whose kernels overlap on the
+ *   Every call shares the one buffer and rewrites every byte of it whose
+ *   value reaches the output (nothing in it has to start at zero).  Calls whose kernels overlap on the
  *   GPU -- on different streams, or from different host threads -- race on
  *   it and must be ordered by the caller. */
 int macaq_dense_mm_noalloc(const uint16_t *x_dev, const float *D_dev, const uint8_t *Wq_dev,

@@ -34,6 +34,9 @@ ERR_SHAPE = -3
 ERR_TOO_MANY_GROUPS = -6
 ERR_GROUP_LIST_TYPE = -7
 ERR_GROUP_LIST_INVALID = -10
+ERR_ACT_TYPE = -13
+# npu_grouped_matmul act_type values (3 is not supported on that page)
+ACT_NONE, ACT_RELU, ACT_GELU_TANH, ACT_FAST_GELU, ACT_SILU = 0, 1, 2, 4, 5
 
 
 def build(force: bool = False) -> str:
@@ -74,6 +77,11 @@ def _L():
             "oracle_gemm_at_plain": (I, [P, P, P, P, I64, P, P, I64, P]),
             "oracle_group_offsets": (I, [P, I, I64, I64, P]),
             "oracle_grouped_mm": (I, [P, P, P, P, I, I64, I64, I64, I64, P, I]),
+            "oracle_grouped_mm_ex": (I, [P, P, P, P, I, I64, I64, I64, I64, P, I, P, I]),
+            "oracle_gemm_ex": (I, [P, P, P, P, I64, I64, I64, P, I, P, I]),
+            "oracle_gemm_at_ex": (I, [P, P, P, P, I64, P, P, I64, P, I, P]),
+            "oracle_act_array": (None, [P, I64, I, P]),
+            "oracle_f64_to_bf16_array": (None, [P, I64, P]),
             "oracle_linear_f64": (None, [P, P, I64, I64, I64, P]),
             "oracle_transform_f64": (None, [P, P, P, I64, I64, I64, P]),
             "oracle_dequantize": (None, [P, P, I64, I64, P]),
@@ -233,6 +241,64 @@ def dense_mm(x_bf16, D, W, nthreads: int = 0) -> np.ndarray:
     return gemm(qa, sa, qw, sw, nthreads)
 
 
+def _bias_ptr(bias):
+    if bias is None:
+        return None, None
+    b = _c(bias, np.float32)
+    return b, _p(b)
+
+
+def act(v, act_type: int) -> np.ndarray:
+    """npu_grouped_matmul's activation act_type (1 RELU, 2 GELU_TANH, 4 FAST_GELU,
+    5 SILU, 0 none) applied in binary64."""
+    v = _c(v, np.float64)
+    out = np.empty_like(v)
+    _L().oracle_act_array(_p(v), v.size, int(act_type), _p(out))
+    return out
+
+
+def f64_to_bf16(v) -> np.ndarray:
+    """binary64 -> bf16 bits, round to nearest even (one rounding)."""
+    v = _c(v, np.float64)
+    out = np.empty(v.shape, np.uint16)
+    _L().oracle_f64_to_bf16_array(_p(v), v.size, _p(out))
+    return out
+
+
+def gemm_ex(qa, sa, qw, sw, bias=None, act_type: int = 0, nthreads: int = 0) -> np.ndarray:
+    """y = RNE_bf16(act(2^-5 * exact sum + bias[n])) as bf16 bits [M, N]
+    (npu_grouped_matmul: y_i = x_i @ weight_i + bias_i, then act_type)."""
+    qa, sa, qw, sw = (_c(a, np.uint8) for a in (qa, sa, qw, sw))
+    M, K = qa.shape[0], qa.shape[1] * 2
+    N = qw.shape[0]
+    b, bp = _bias_ptr(bias)
+    y = np.empty((M, N), np.uint16)
+    st = _L().oracle_gemm_ex(_p(qa), _p(sa), _p(qw), _p(sw), M, N, K, bp, int(act_type), _p(y), nthreads)
+    assert st == OK, st
+    return y
+
+
+def gemm_at_ex(qa, sa, qw, sw, rows, cols, bias=None, act_type: int = 0) -> np.ndarray:
+    """gemm_ex at the given (row, col) pairs only."""
+    qa, sa, qw, sw = (_c(a, np.uint8) for a in (qa, sa, qw, sw))
+    K = qa.shape[1] * 2
+    rows = _c(rows, np.int64)
+    cols = _c(cols, np.int64)
+    b, bp = _bias_ptr(bias)
+    out = np.empty(rows.size, np.uint16)
+    st = _L().oracle_gemm_at_ex(_p(qa), _p(sa), _p(qw), _p(sw), K, _p(rows), _p(cols), rows.size, bp,
+                                int(act_type), _p(out))
+    assert st == OK, st
+    return out
+
+
+def dense_mm_ex(x_bf16, D, W, bias=None, act_type: int = 0, nthreads: int = 0) -> np.ndarray:
+    """Dense MACAQ linear with bias and activation: bf16 bits [M, N]."""
+    qa, sa = quantize_act(x_bf16, D, nthreads)
+    qw, sw = quantize_weights(W, D, nthreads)
+    return gemm_ex(qa, sa, qw, sw, bias, act_type, nthreads)
+
+
 def group_offsets(group_list, group_list_type: int, M: int):
     """Row offsets [E+1] from group_list (npu_grouped_matmul, group_list and
     group_list_type).  Returns (status, offsets)."""
@@ -255,6 +321,23 @@ def grouped_mm(x_bf16, D, W, group_list, group_list_type: int, nthreads: int = 0
     y = np.zeros((M, N), np.uint16)
     st = _L().oracle_grouped_mm(_p(x), _p(D), _p(W), _p(gl), int(group_list_type), E, M, N, K,
                                 _p(y), nthreads)
+    return int(st), y
+
+
+def grouped_mm_ex(x_bf16, D, W, group_list, group_list_type: int, bias=None, act_type: int = 0,
+                  nthreads: int = 0):
+    """Grouped MACAQ linear with per-expert bias [E, N] and activation.
+    Returns (status, y bf16 bits [M, N])."""
+    x = _c(x_bf16, np.uint16)
+    D = _c(D, np.float32)
+    W = _c(W, np.float32)
+    gl = _c(group_list, np.int64)
+    M, K = x.shape
+    E, N, _ = W.shape
+    b, bp = _bias_ptr(bias)
+    y = np.zeros((M, N), np.uint16)
+    st = _L().oracle_grouped_mm_ex(_p(x), _p(D), _p(W), _p(gl), int(group_list_type), E, M, N, K, bp,
+                                   int(act_type), _p(y), nthreads)
     return int(st), y
 
 

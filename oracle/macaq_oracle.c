@@ -33,6 +33,13 @@
  *   R6  weights take the same steps on t = FWHT32(RN32(W*D)) in FP32 with
  *       no BF16 rounding (offline preparation);
  *   R7  y = RNE_bf16(2^-5 * exact sum of the decoded block-scaled products).
+ *   R15 with the npu_grouped_matmul page's bias and act_type (parameters
+ *       bias, act_type: 1 RELU, 2 GELU_TANH, 4 FAST_GELU, 5 SILU; 3 is not
+ *       supported there), the epilogue is y = RNE_bf16(act(s + bias[n])) with
+ *       s = 2^-5 * exact sum (the bias in output units, the page's
+ *       y_i = x_i @ weight_i + bias_i), evaluated here in binary64;
+ *       FAST_GELU, which the page does not define, is read as
+ *       v / (1 + exp(-1.702 v)).
  *
  * The plain MXFP4 baseline (the MACAQ page's native W4A4 comparison, which
  * quantises x and W directly with the dynamic MX quantiser) skips D and H:
@@ -58,6 +65,7 @@
 #define ORACLE_ERR_TOO_MANY_GROUPS (-6)
 #define ORACLE_ERR_GROUP_LIST_TYPE (-7)
 #define ORACLE_ERR_GROUP_LIST_INVALID (-10)
+#define ORACLE_ERR_ACT_TYPE (-13)
 
 /* ------------------------------------------------------------------ */
 /* binary16-brain (bf16) <-> binary32                                  */
@@ -517,6 +525,171 @@ int oracle_gemm_at_plain(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw
 }
 
 /* ------------------------------------------------------------------ */
+/* Epilogue: bias and activation (R15)                                 */
+/* ------------------------------------------------------------------ */
+
+/* The accumulator value acc * 2^base_exp correctly rounded to binary64 (round
+ * to nearest, ties to even).  Every sum here lies far inside the normal
+ * binary64 range. */
+static double wide_to_f64(const wide_t *acc, int base_exp)
+{
+    wide_t a = *acc;
+    int neg = (int)((a.w[NLIMB - 1] >> 63) & 1);
+    if (neg) {
+        unsigned carry = 1;
+        for (int i = 0; i < NLIMB; i++) {
+            uint64_t v = ~a.w[i];
+            uint64_t s = v + carry;
+            carry = carry && s == 0;
+            a.w[i] = s;
+        }
+    }
+    int top = -1;
+    for (int i = NLIMB - 1; i >= 0 && top < 0; i--)
+        if (a.w[i])
+            top = i * 64 + 63 - __builtin_clzll(a.w[i]);
+    if (top < 0)
+        return 0.0;
+    int L = top - 52; /* bit index of the last kept bit (53 significant bits) */
+    uint64_t q = 0;
+    for (int i = top; i >= (L > 0 ? L : 0); i--)
+        q = (q << 1) | (uint64_t)wide_bit(&a, i);
+    if (L > 0) {
+        int round = wide_bit(&a, L - 1);
+        int sticky = wide_any_below(&a, L - 1);
+        if (round && (sticky || (q & 1)))
+            q += 1; /* a carry to 2^53 is still exact in binary64 */
+    } else {
+        L = 0;
+    }
+    double v = ldexp((double)q, L + base_exp);
+    return neg ? -v : v;
+}
+
+/* 2^out_exp * exact sum, rounded once to binary64. */
+static double exact_dot_f64(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const uint8_t *sw,
+                            int64_t K, int out_exp)
+{
+    wide_t acc;
+    memset(&acc, 0, sizeof acc);
+    for (int64_t b = 0; b < K / 32; b++) {
+        int64_t p = 0;
+        for (int i = 0; i < 32; i++) {
+            int64_t k = 32 * b + i;
+            int ca = (qa[k / 2] >> (4 * (k & 1))) & 15;
+            int cw = (qw[k / 2] >> (4 * (k & 1))) & 15;
+            p += (int64_t)llround(2.0 * oracle_e2m1_decode(ca)) * (int64_t)llround(2.0 * oracle_e2m1_decode(cw));
+        }
+        wide_add_shifted(&acc, p, (int)sa[b] + (int)sw[b]);
+    }
+    return wide_to_f64(&acc, -256 + out_exp);
+}
+
+/* The activation functions of npu_grouped_matmul's act_type, in binary64.
+ * Returns NAN for an unsupported type (the callers check it first). */
+double oracle_act(double v, int act)
+{
+    switch (act) {
+    case 0:
+        return v;
+    case 1: /* RELU */
+        return v > 0.0 ? v : 0.0;
+    case 2: /* GELU_TANH: 0.5 v (1 + tanh(sqrt(2/pi) (v + 0.044715 v^3))) */
+        return 0.5 * v * (1.0 + tanh(sqrt(2.0 / M_PI) * (v + 0.044715 * v * v * v)));
+    case 4: /* FAST_GELU (R15): v * sigmoid(1.702 v) */
+        return v / (1.0 + exp(-1.702 * v));
+    case 5: /* SILU: v * sigmoid(v) */
+        return v / (1.0 + exp(-v));
+    default:
+        return NAN;
+    }
+}
+
+void oracle_act_array(const double *v, int64_t n, int act, double *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = oracle_act(v[i], act);
+}
+
+/* binary64 -> bf16 bits, round to nearest, ties to even; subnormals keep
+ * their last bit at 2^-133; overflow gives infinity. */
+uint16_t oracle_f64_to_bf16(double v)
+{
+    if (isnan(v))
+        return 0x7fc0u;
+    uint16_t sign = signbit(v) ? 0x8000u : 0u;
+    double a = fabs(v);
+    if (a == 0.0)
+        return sign;
+    if (isinf(a))
+        return (uint16_t)(sign | 0x7f80u);
+    int e = ilogb(a);                      /* a in [2^e, 2^(e+1)) */
+    int lsb = e >= -126 ? e - 7 : -133;    /* weight of the last kept bit */
+    double q = nearbyint(ldexp(a, -lsb));  /* exact scaling, then round half to even */
+    double r = ldexp(q, lsb);
+    if (r >= 0x1p128)
+        return (uint16_t)(sign | 0x7f80u);
+    float f = (float)r; /* exactly representable: at most 8 significant bits */
+    uint32_t bits;
+    memcpy(&bits, &f, 4);
+    return (uint16_t)(sign | ((bits >> 16) & 0x7fffu));
+}
+
+void oracle_f64_to_bf16_array(const double *v, int64_t n, uint16_t *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = oracle_f64_to_bf16(v[i]);
+}
+
+static int act_supported(int act) { return act == 0 || act == 1 || act == 2 || act == 4 || act == 5; }
+
+/* y[m, n] = RNE_bf16(act(2^-5 * exact sum + bias[n])); bias may be NULL.
+ * With no bias and no activation this is oracle_gemm (one rounding). */
+int oracle_gemm_ex(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const uint8_t *sw, int64_t M,
+                   int64_t N, int64_t K, const float *bias, int act, uint16_t *y, int nthreads)
+{
+    if (!act_supported(act))
+        return ORACLE_ERR_ACT_TYPE;
+    if (!bias && act == 0)
+        return oracle_gemm(qa, sa, qw, sw, M, N, K, y, nthreads);
+    if (K <= 0 || K % 32 != 0)
+        return ORACLE_ERR_SHAPE;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel for collapse(2) schedule(static)
+#endif
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t n = 0; n < N; n++) {
+            double s = exact_dot_f64(qa + m * (K / 2), sa + m * (K / 32), qw + n * (K / 2), sw + n * (K / 32), K, -5);
+            if (bias)
+                s += (double)bias[n];
+            y[m * N + n] = oracle_f64_to_bf16(oracle_act(s, act));
+        }
+    (void)nthreads;
+    return ORACLE_OK;
+}
+
+/* The same at chosen (row, col) positions; bias indexed by col. */
+int oracle_gemm_at_ex(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const uint8_t *sw, int64_t K,
+                      const int64_t *rows, const int64_t *cols, int64_t count, const float *bias, int act,
+                      uint16_t *out)
+{
+    if (!act_supported(act))
+        return ORACLE_ERR_ACT_TYPE;
+    if (K <= 0 || K % 32 != 0)
+        return ORACLE_ERR_SHAPE;
+    for (int64_t i = 0; i < count; i++) {
+        double s = exact_dot_f64(qa + rows[i] * (K / 2), sa + rows[i] * (K / 32), qw + cols[i] * (K / 2),
+                                 sw + cols[i] * (K / 32), K, -5);
+        if (bias)
+            s += (double)bias[cols[i]];
+        out[i] = oracle_f64_to_bf16(oracle_act(s, act));
+    }
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
 /* Grouped form: rows [cum[g-1], cum[g]) use expert g                  */
 /* ------------------------------------------------------------------ */
 
@@ -553,13 +726,16 @@ int oracle_group_offsets(const int64_t *group_list, int type, int64_t E, int64_t
     return ORACLE_OK;
 }
 
-/* Grouped MACAQ linear. x bf16 [M,K]; D [E,K]; W fp32 [E,N,K]. y [M,N]. */
-int oracle_grouped_mm(const uint16_t *x, const float *D, const float *W, const int64_t *group_list,
-                      int type, int64_t E, int64_t M, int64_t N, int64_t K, uint16_t *y,
-                      int nthreads)
+/* Grouped MACAQ linear. x bf16 [M,K]; D [E,K]; W fp32 [E,N,K]; bias fp32
+ * [E,N] or NULL (each entry's rows take its expert's bias); y [M,N]. */
+int oracle_grouped_mm_ex(const uint16_t *x, const float *D, const float *W, const int64_t *group_list,
+                         int type, int64_t E, int64_t M, int64_t N, int64_t K, const float *bias, int act,
+                         uint16_t *y, int nthreads)
 {
     if (K <= 0 || K % 32 != 0 || N <= 0 || M < 0)
         return ORACLE_ERR_SHAPE;
+    if (!act_supported(act))
+        return ORACLE_ERR_ACT_TYPE;
     int64_t *off = (int64_t *)malloc(sizeof(int64_t) * (size_t)(E + 1 > 1 ? E + 1 : 2));
     int st = oracle_group_offsets(group_list, type, E, M, off);
     if (st != ORACLE_OK) {
@@ -578,7 +754,7 @@ int oracle_grouped_mm(const uint16_t *x, const float *D, const float *W, const i
         uint8_t *qa = (uint8_t *)malloc((size_t)((r1 - r0) * K / 2));
         uint8_t *sa = (uint8_t *)malloc((size_t)((r1 - r0) * K / 32));
         oracle_quantize_act(x + r0 * K, D + e * K, r1 - r0, K, qa, sa, nthreads);
-        oracle_gemm(qa, sa, qw, sw, r1 - r0, N, K, y + r0 * N, nthreads);
+        oracle_gemm_ex(qa, sa, qw, sw, r1 - r0, N, K, bias ? bias + e * N : NULL, act, y + r0 * N, nthreads);
         free(qa);
         free(sa);
     }
@@ -586,6 +762,13 @@ int oracle_grouped_mm(const uint16_t *x, const float *D, const float *W, const i
     free(sw);
     free(off);
     return ORACLE_OK;
+}
+
+int oracle_grouped_mm(const uint16_t *x, const float *D, const float *W, const int64_t *group_list,
+                      int type, int64_t E, int64_t M, int64_t N, int64_t K, uint16_t *y,
+                      int nthreads)
+{
+    return oracle_grouped_mm_ex(x, D, W, group_list, type, E, M, N, K, NULL, 0, y, nthreads);
 }
 
 /* ------------------------------------------------------------------ */

@@ -40,7 +40,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.macaq_abi_version() == 2
+    assert L.macaq_abi_version() == 3
     for code, name in mq.STATUS.items():
         assert L.macaq_status_string(code).decode() == name
     assert L.macaq_status_string(-99).decode() == "MACAQ_ERR_UNKNOWN"
@@ -95,8 +95,28 @@ def test_grouped_refusals_by_name(L):
     assert g(glp=P((9 << 32) + 4)) == -2
 
 
+def test_epilogue_refusals_by_name(L):
+    bias = P(11 << 32)
+
+    def d(act=0, b=bias, M=16, N=1024):
+        return L.macaq_dense_mm_ex(A, B, C, Dp, b, act, Y, M, N, 1024, None, 0, None, None)
+
+    def g(act=0, b=bias, E=4):
+        return L.macaq_grouped_mm_ex(A, B, C, Dp, P(9 << 32), 1, E, b, act, Y, 64, 1024, 1024, None, 0, None, None)
+
+    for act in (3, 6, -1, 100):      # act_type 3 is "not supported" on the npu_grouped_matmul page
+        assert d(act=act) == -13
+        assert g(act=act) == -13
+    assert d(b=P((11 << 32) + 4)) == -2           # bias not 16-byte aligned
+    assert d(b=P((5 << 32) + 64)) == -5           # bias inside y ([16, 1024] bf16 at 5 << 32)
+    assert g(b=P((5 << 32) + 4096), E=4) == -5
+    assert d(act=3, M=0) == -13                   # refused even when there is nothing to compute
+    assert g(act=2, b=None) == -11                # accepted; the missing workspace is the next refusal
+
+
 def test_no_gpu_means_a_named_cuda_error_not_a_fallback(L):
     import torch
     if torch.cuda.is_available():
         pytest.skip("GPU present")
     assert dense(L) == -8
+    assert L.macaq_dense_mm_ex(A, B, C, Dp, None, 5, Y, 16, 1024, 1024, None, 0, None, None) == -8

@@ -530,3 +530,118 @@ def test_macaq_beats_plain_mxfp4_on_outlier_activations():
     nmse = lambda a: float(np.sum((a - ref) ** 2) / np.sum(ref ** 2))
     assert nmse(y) < nmse(yp)
     assert nmse(y) < 0.05
+
+
+# ----------------------------------------------------------------------------
+# Epilogue: bias and act_type (npu_grouped_matmul, parameters bias and act_type)
+# ----------------------------------------------------------------------------
+
+ACTS = [oracle.ACT_RELU, oracle.ACT_GELU_TANH, oracle.ACT_FAST_GELU, oracle.ACT_SILU]
+
+
+def test_activations_match_library_routines():
+    v = np.linspace(-12.0, 12.0, 4001)
+    t = torch.from_numpy(v)
+    assert np.array_equal(oracle.act(v, oracle.ACT_RELU), np.maximum(v, 0.0))
+    np.testing.assert_allclose(oracle.act(v, oracle.ACT_GELU_TANH),
+                               torch.nn.functional.gelu(t, approximate="tanh").numpy(), rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(oracle.act(v, oracle.ACT_SILU), torch.nn.functional.silu(t).numpy(),
+                               rtol=1e-13, atol=1e-15)
+    assert np.array_equal(oracle.act(v, oracle.ACT_NONE), v)
+
+
+def test_activations_odd_part_is_the_identity():
+    # f(v) - f(-v) == v for every sigmoid- or tanh-gated form v * g(v) with
+    # g(v) + g(-v) == 1: a dropped factor, a wrong sign or a missing 0.5 breaks it
+    v = np.linspace(-30.0, 30.0, 6001)
+    for a in (oracle.ACT_RELU, oracle.ACT_GELU_TANH, oracle.ACT_FAST_GELU, oracle.ACT_SILU):
+        np.testing.assert_allclose(oracle.act(v, a) - oracle.act(-v, a), v, rtol=1e-12, atol=1e-12)
+
+
+def test_gelu_forms_approximate_the_exact_gelu():
+    # exact GELU v * Phi(v) from the error function; the tanh form is within
+    # 1e-3 of it, the 1.702-sigmoid form (FAST_GELU reading) within 2.5e-2
+    v = np.linspace(-8.0, 8.0, 3201)
+    exact = np.array([x * 0.5 * (1.0 + math.erf(x / math.sqrt(2.0))) for x in v])
+    assert np.max(np.abs(oracle.act(v, oracle.ACT_GELU_TANH) - exact)) < 1e-3
+    assert np.max(np.abs(oracle.act(v, oracle.ACT_FAST_GELU) - exact)) < 2.5e-2
+    # and the sigmoid slope: FAST_GELU'(0) = 1/2 like GELU, second derivative 1.702/2
+    h = 1e-4
+    d2 = (oracle.act(np.array([h]), 4)[0] - 2 * 0.0 + oracle.act(np.array([-h]), 4)[0]) / h ** 2
+    assert abs(d2 - 1.702 / 2) < 1e-6
+
+
+def test_f64_to_bf16_rounds_once_to_nearest_even():
+    # every positive finite bf16 value and the midpoints between neighbours
+    bits = np.arange(1, 0x7f80, dtype=np.uint32)
+    vals = (bits << 16).view(np.float32).astype(np.float64)
+    assert np.array_equal(oracle.f64_to_bf16(vals), bits.astype(np.uint16))
+    assert np.array_equal(oracle.f64_to_bf16(-vals), (bits | 0x8000).astype(np.uint16))
+    lo, hi = vals[:-1], vals[1:]
+    mid = (lo + hi) / 2                          # exact in binary64
+    even = np.where(bits[:-1] % 2 == 0, bits[:-1], bits[1:]).astype(np.uint16)
+    assert np.array_equal(oracle.f64_to_bf16(mid), even)
+    up = np.nextafter(mid, np.inf)
+    dn = np.nextafter(mid, -np.inf)
+    assert np.array_equal(oracle.f64_to_bf16(up), bits[1:].astype(np.uint16))
+    assert np.array_equal(oracle.f64_to_bf16(dn), bits[:-1].astype(np.uint16))
+    assert oracle.f64_to_bf16(np.array([2.0 ** 128]))[0] == 0x7f80
+    assert oracle.f64_to_bf16(np.array([-0.0]))[0] == 0x8000
+
+
+def test_epilogue_on_zero_activations_is_act_of_bias():
+    # x = 0 makes every code and the exact sum zero, so y = RNE_bf16(act(bias)):
+    # the bias is added in output units (after the 2^-5), then the activation
+    rng = np.random.default_rng(11)
+    K, N = 256, 64
+    x = np.zeros((4, K), np.uint16)
+    D = np.ones(K, np.float32)
+    W = rng.standard_normal((N, K)).astype(np.float32)
+    bias = (rng.standard_normal(N) * 3).astype(np.float32)
+    for a in [oracle.ACT_NONE] + ACTS:
+        y = oracle.dense_mm_ex(x, D, W, bias, a)
+        ref = np.array([oracle.act(np.array([float(b)]), a)[0] for b in bias])
+        assert np.array_equal(y, np.broadcast_to(oracle.f64_to_bf16(ref), y.shape)), a
+
+
+def test_epilogue_without_bias_agrees_with_the_plain_product():
+    # relu commutes with rounding to bf16, and a zero bias changes nothing
+    p = synth.dense(24, 512, 48, seed=3)
+    qa, sa = oracle.quantize_act(p.x, p.D[0])
+    qw, sw = oracle.quantize_weights(p.W[0], p.D[0])
+    y = oracle.gemm(qa, sa, qw, sw)
+    yv = synth.bf16_bits_to_f32(y).astype(np.float64)
+    assert np.array_equal(oracle.gemm_ex(qa, sa, qw, sw, np.zeros(48, np.float32), 0), y)
+    relu = oracle.gemm_ex(qa, sa, qw, sw, None, oracle.ACT_RELU)
+    assert np.array_equal(synth.bf16_bits_to_f32(relu).astype(np.float64), np.maximum(yv, 0.0))
+    rows, cols = np.array([0, 5, 23]), np.array([47, 0, 13])
+    b = np.linspace(-1, 1, 48).astype(np.float32)
+    full = oracle.gemm_ex(qa, sa, qw, sw, b, oracle.ACT_SILU)
+    assert np.array_equal(oracle.gemm_at_ex(qa, sa, qw, sw, rows, cols, b, oracle.ACT_SILU), full[rows, cols])
+
+
+def test_epilogue_refuses_act_type_3_and_unknown_values():
+    qa = np.zeros((1, 16), np.uint8)
+    sa = np.zeros((1, 1), np.uint8)
+    for a in (3, 6, -1):
+        with pytest.raises(AssertionError):
+            oracle.gemm_ex(qa, sa, qa, sa, None, a)
+
+
+def test_grouped_epilogue_uses_each_experts_bias():
+    # replicated weight banks with per-expert biases: entry g's rows equal the
+    # dense product with bias g
+    rng = np.random.default_rng(5)
+    M, K, N, E = 40, 256, 32, 3
+    p = synth.dense(M, K, N, seed=9)
+    W = np.repeat(p.W, E, axis=0)
+    D = np.repeat(p.D, E, axis=0)
+    bias = rng.standard_normal((E, N)).astype(np.float32)
+    counts = np.array([10, 0, 30], np.int64)
+    st, y = oracle.grouped_mm_ex(p.x, D, W, counts, 1, bias, oracle.ACT_GELU_TANH)
+    assert st == oracle.OK
+    off = np.concatenate([[0], np.cumsum(counts)])
+    for g in range(E):
+        if counts[g]:
+            ref = oracle.dense_mm_ex(p.x[off[g]:off[g + 1]], p.D[0], p.W[0], bias[g], oracle.ACT_GELU_TANH)
+            assert np.array_equal(y[off[g]:off[g + 1]], ref)

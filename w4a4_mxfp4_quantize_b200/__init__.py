@@ -34,7 +34,11 @@ STATUS = {
     -4: "MACAQ_ERR_ARCH", -5: "MACAQ_ERR_ALIAS", -6: "MACAQ_ERR_TOO_MANY_GROUPS",
     -7: "MACAQ_ERR_GROUP_LIST_TYPE", -8: "MACAQ_ERR_CUDA", -9: "MACAQ_ERR_DEVICE_TIMEOUT",
     -10: "MACAQ_ERR_GROUP_LIST_INVALID", -11: "MACAQ_ERR_WORKSPACE", -12: "MACAQ_ERR_BAD_D",
+    -13: "MACAQ_ERR_ACT_TYPE",
 }
+
+# npu_grouped_matmul act_type values accepted by the _ex calls (3 is not supported)
+ACT_NONE, ACT_RELU, ACT_GELU_TANH, ACT_FAST_GELU, ACT_SILU = 0, 1, 2, 4, 5
 
 
 class MacaqError(RuntimeError):
@@ -76,6 +80,10 @@ _SIG = {
     "macaq_dense_mm": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, ctypes.c_size_t, _P, _P]),
     "macaq_grouped_mm": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, _I64, _P, _I64, _I64, _I64, _P,
                                         ctypes.c_size_t, _P, _P]),
+    "macaq_dense_mm_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, _P, _I64, _I64, _I64, _P,
+                                         ctypes.c_size_t, _P, _P]),
+    "macaq_grouped_mm_ex": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P, _I64,
+                                           _I64, _I64, _P, ctypes.c_size_t, _P, _P]),
     "macaq_quantize_activations": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _P]),
     "macaq_export_weights": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P]),
     "macaq_mx_encode_blocks": (ctypes.c_int, [_P, _P, _P, _I64, _P]),
@@ -205,19 +213,35 @@ def prepare_weights(W: torch.Tensor, D: torch.Tensor, stream=None) -> tuple[torc
     return Wq, Ws
 
 
+def _check_bias(bias, shape):
+    if bias is None:
+        return
+    _require_cuda(bias)
+    if bias.dtype != torch.float32 or tuple(bias.shape) != shape:
+        raise ValueError(f"bias must be float32 of shape {shape}, got {bias.dtype} {tuple(bias.shape)}")
+
+
 def dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: int,
              out: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None,
-             ws: torch.Tensor | None = None) -> torch.Tensor:
-    """y [M, N] bf16 = MACAQ linear of x bf16 [M, K] (fused kernel)."""
+             ws: torch.Tensor | None = None, bias: torch.Tensor | None = None,
+             act_type: int = ACT_NONE) -> torch.Tensor:
+    """y [M, N] bf16 = MACAQ linear of x bf16 [M, K]; optional fp32 bias [N] and
+    output activation act_type (npu_grouped_matmul's bias and act_type)."""
     _require_cuda(x, D, Wq, Ws, out, status)
     M, K = x.shape
+    _check_bias(bias, (N,))
     y = _output(out, M, N, x.device)
     L = lib()
     need = int(L.macaq_workspace_bytes(M, N, K, 1))
     ws = workspace(need, x.device, stream, ws)
-    _check(L.macaq_dense_mm(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(y), M, N, K, _ptr(ws),
-                            _nbytes(ws), _ptr(status), _stream_ptr(stream)),
-           "macaq_dense_mm")
+    if bias is None and act_type == ACT_NONE:
+        _check(L.macaq_dense_mm(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(y), M, N, K, _ptr(ws),
+                                _nbytes(ws), _ptr(status), _stream_ptr(stream)),
+               "macaq_dense_mm")
+    else:
+        _check(L.macaq_dense_mm_ex(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(bias), int(act_type), _ptr(y),
+                                   M, N, K, _ptr(ws), _nbytes(ws), _ptr(status), _stream_ptr(stream)),
+               "macaq_dense_mm_ex")
     return y
 
 
@@ -232,20 +256,29 @@ def _groups(group_list: torch.Tensor, group_list_type: int) -> int:
 
 def grouped_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, group_list: torch.Tensor,
                group_list_type: int, N: int, out: torch.Tensor | None = None,
-               status: torch.Tensor | None = None, stream=None, ws: torch.Tensor | None = None) -> torch.Tensor:
+               status: torch.Tensor | None = None, stream=None, ws: torch.Tensor | None = None,
+               bias: torch.Tensor | None = None, act_type: int = ACT_NONE) -> torch.Tensor:
     """Grouped MACAQ linear; group_list int64 on the device: [E] for type 0 (cumsum) and 1
-    (counts), [E, 2] rows of (group index, group size) for type 2."""
+    (counts), [E, 2] rows of (group index, group size) for type 2.  Optional fp32 bias
+    [E, N] (per expert) and output activation act_type."""
     _require_cuda(x, D, Wq, Ws, group_list, out, status)
     M, K = x.shape
     E = _groups(group_list, group_list_type)
+    _check_bias(bias, (E, N))
     y = _output(out, M, N, x.device)
     L = lib()
     need = int(L.macaq_workspace_bytes(M, N, K, E))
     ws = workspace(need, x.device, stream, ws)
-    _check(L.macaq_grouped_mm(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(group_list), int(group_list_type), E,
-                              _ptr(y), M, N, K, _ptr(ws), _nbytes(ws), _ptr(status),
-                              _stream_ptr(stream)),
-           "macaq_grouped_mm")
+    if bias is None and act_type == ACT_NONE:
+        _check(L.macaq_grouped_mm(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(group_list), int(group_list_type), E,
+                                  _ptr(y), M, N, K, _ptr(ws), _nbytes(ws), _ptr(status),
+                                  _stream_ptr(stream)),
+               "macaq_grouped_mm")
+    else:
+        _check(L.macaq_grouped_mm_ex(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(group_list), int(group_list_type),
+                                     E, _ptr(bias), int(act_type), _ptr(y), M, N, K, _ptr(ws), _nbytes(ws),
+                                     _ptr(status), _stream_ptr(stream)),
+               "macaq_grouped_mm_ex")
     return y
 
 

@@ -58,6 +58,34 @@ __device__ __forceinline__ uint16_t bf16_bits(float v) {
   return *reinterpret_cast<uint16_t*>(&h);
 }
 
+// Output activation of npu_grouped_matmul's act_type (parameter act_type: 0 none,
+// 1 RELU, 2 GELU_TANH, 4 FAST_GELU, 5 SILU), in FP32 with CUDA's expf / tanhf.
+// FAST_GELU, which the page names without defining, is v * sigmoid(1.702 v).
+template <int ACT>
+__device__ __forceinline__ float act_value(float v) {
+  if constexpr (ACT == 1) {
+    return fmaxf(v, 0.f);
+  } else if constexpr (ACT == 2) {
+    const float u = 0.7978845608028654f * (v + 0.044715f * v * v * v);  // sqrt(2/pi) (v + 0.044715 v^3)
+    return 0.5f * v * (1.f + tanhf(u));
+  } else if constexpr (ACT == 4) {
+    return v / (1.f + expf(-1.702f * v));
+  } else if constexpr (ACT == 5) {
+    return v / (1.f + expf(-v));
+  } else {
+    return v;
+  }
+}
+__device__ __forceinline__ float act_value_rt(float v, int act) {
+  switch (act) {
+    case 1: return act_value<1>(v);
+    case 2: return act_value<2>(v);
+    case 4: return act_value<4>(v);
+    case 5: return act_value<5>(v);
+    default: return v;
+  }
+}
+
 // ============================================================================
 // Image layouts
 // ============================================================================
@@ -143,7 +171,7 @@ __global__ void __launch_bounds__(256) quant_canonical_kernel(const uint16_t* __
                                                               const float* __restrict__ D,
                                                               uint8_t* __restrict__ codes,
                                                               uint8_t* __restrict__ scales, int M, int K) {
-  __shared__ __align__(16) float r[kRcpTile];
+  __shared__ __align__(16) float r[kQRcpTile];
   const int kt = blockIdx.y;
   const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
   const int t = threadIdx.x >> 3, c = threadIdx.x & 7;
@@ -154,12 +182,12 @@ __global__ void __launch_bounds__(256) quant_canonical_kernel(const uint16_t* __
 #pragma unroll
     for (int i = 0; i < 4; ++i) xv[i] = __ldg(src + i);
   }
-  r[rcp_index(threadIdx.x)] = __frcp_rn(__ldg(D + k0 + threadIdx.x));
+  r[qrcp_index(threadIdx.x)] = __frcp_rn(__ldg(D + k0 + threadIdx.x));
   __syncthreads();
   if (m >= M) return;
   uint4 cv;
   uint32_t sc;
-  act_block(xv, r + c * kRcpStride, cv, sc);
+  act_block(xv, r + c * kQRcpStride, cv, sc);
   *reinterpret_cast<uint4*>(codes + static_cast<int64_t>(m) * (K / 2) + (k0 + c * kBlk) / 2) = cv;
   scales[static_cast<int64_t>(m) * (K / kBlk) + k0 / kBlk + c] = static_cast<uint8_t>(sc);
 }
@@ -331,7 +359,7 @@ constexpr int kQuantSmem = kQuantStages * kQuantSlotBytes;
 
 __global__ void __launch_bounds__(256, 4) quant_tiles_kernel(const __grid_constant__ QuantParams p) {
   extern __shared__ __align__(16) uint8_t qsmem[];  // ring [kQuantStages][4 chunks][256 threads][16]
-  __shared__ __align__(16) float r[2][kRcpTile];
+  __shared__ __align__(16) float r[2][kQRcpTile];
   pdl_trigger();  // the GEMM may start streaming weights; it waits for our results before reading them
   pdl_wait();     // x (and the grouped tables) may come from the preceding kernels
   const int KT = p.K / kKTile;
@@ -410,7 +438,7 @@ __global__ void __launch_bounds__(256, 4) quant_tiles_kernel(const __grid_consta
         step();
       }
       const Unit w = ring[k];
-      r[buf][rcp_index(threadIdx.x)] = __frcp_rn(w.d);
+      r[buf][qrcp_index(threadIdx.x)] = __frcp_rn(w.d);
       cp_async_wait<kQuantAhead>();  // this thread's copy of this unit has landed
       __syncthreads();               // every reciprocal written; r[buf] of two units back no longer read
       if (w.t >= 0) {
@@ -419,7 +447,7 @@ __global__ void __launch_bounds__(256, 4) quant_tiles_kernel(const __grid_consta
         const uint4* xs = reinterpret_cast<const uint4*>(qsmem + k * kQuantSlotBytes) + threadIdx.x;
         const uint4 xv[4] = {xs[0], xs[256], xs[512], xs[768]};
         if (p.plain) act_block_plain(xv, cv, sc);
-        else act_block(xv, r[buf] + c * kRcpStride, cv, sc);
+        else act_block(xv, r[buf] + c * kQRcpStride, cv, sc);
         *reinterpret_cast<uint4*>(w.img + code_chunk_offset(w.t, c)) = cv;
         w.img[kTileCodeBytes + sf_offset(w.t, c)] = static_cast<uint8_t>(sc);
       }
@@ -448,7 +476,34 @@ struct GemmParams {
   int NT2;                // 256-wide output tiles: ceil(NT / 2)
   int stages;             // pipeline depth (gemm::stages_for(E))
   float out_scale;        // 2^-5 (MACAQ: undoes the two unnormalised Hadamards), 1 (plain MXFP4)
+  const float* bias;      // fp32 [E][N] (expert g's row for its tiles) or nullptr
+  int act;                // act_type: 0 none, 1 RELU, 2 GELU_TANH, 4 FAST_GELU, 5 SILU
 };
+
+// Epilogue drain of 64 accumulator columns of one thread's row of the tile:
+// v = acc * out_scale (+ bias[n]), then the activation, packed to BF16 pairs.
+// Columns n >= N (the zero rows of a ragged weight tile) take no bias.
+template <int ACT>
+__device__ __forceinline__ void drain64(uint32_t taddr, float os, const float* brow, int ncol0, int N,
+                                        uint32_t (&pk)[32]) {
+#pragma unroll
+  for (int c0 = 0; c0 < 64; c0 += 16) {
+    uint32_t r[16];
+    tmem_ld_32x32b_x16(taddr + c0, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      float v0 = __uint_as_float(r[2 * e]) * os, v1 = __uint_as_float(r[2 * e + 1]) * os;
+      const int n = ncol0 + c0 + 2 * e;
+      if (brow != nullptr && n < N) {
+        const float2 b = __ldg(reinterpret_cast<const float2*>(brow + n));  // warp-uniform: a broadcast
+        v0 += b.x;
+        v1 += b.y;
+      }
+      pk[c0 / 2 + e] = pack_bf16x2(act_value<ACT>(v0), act_value<ACT>(v1));
+    }
+  }
+}
 
 // Large M: the MMA is not swapped.  Operand A = a 128-token activation tile,
 // operand B = 256 output channels of weights (two 128-row weight images side by
@@ -573,6 +628,9 @@ __device__ __forceinline__ void mma_stage(uint64_t adesc, uint64_t bdesc, uint32
   }
 }
 
+// kEpilogue: the bias / activation epilogue (p.bias, p.act) is compiled in; the
+// plain kernel keeps its registers for the plain drain.
+template <bool kEpilogue>
 __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
   using namespace gemm;
   extern __shared__ uint8_t smem_raw[];
@@ -766,32 +824,19 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
       if (!*epi_flag) break;
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 128;
-      uint32_t pk[64];
+      // Chunk ch of the tile = columns 64 ch .. + 63, held by half ch / 2.  A chunk is
+      // staged with its 16-byte pieces XOR-swizzled by the row, then all 256
+      // threads store it as coalesced 128-byte row runs.
+      const int c = et & 7;  // 16-byte piece of a 128-byte row run
+      auto stage_chunk = [&](const uint32_t* src) {
+        uint8_t* srow = staging + tl * 128;
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(taddr + c0, r);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          pk[c0 / 2 + e] = pack_bf16x2(__uint_as_float(r[2 * e]) * os, __uint_as_float(r[2 * e + 1]) * os);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(acce);
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        if ((ch >> 1) == h) {  // chunk ch = columns 64 ch .. + 63, held by half ch / 2
-          uint8_t* srow = staging + tl * 128;
-#pragma unroll
-          for (int g = 0; g < 8; ++g) {
-            const int b = (ch & 1) * 32 + 4 * g;
-            *reinterpret_cast<uint4*>(srow + ((g ^ (tl & 7)) << 4)) = make_uint4(pk[b], pk[b + 1], pk[b + 2], pk[b + 3]);
-          }
-        }
-        named_bar_sync(1, 256);
+        for (int g = 0; g < 8; ++g)
+          *reinterpret_cast<uint4*>(srow + ((g ^ (tl & 7)) << 4)) =
+              make_uint4(src[4 * g], src[4 * g + 1], src[4 * g + 2], src[4 * g + 3]);
+      };
+      auto store_chunk = [&](int ch) {
         const int n0 = t.nt * kRowsTile + ch * 64;
-        const int c = et & 7;  // 16-byte piece of a 128-byte row run
         if (n0 + 8 * c < p.N) {
 #pragma unroll 4
           for (int rr = et >> 3; rr < t.rows; rr += 32) {
@@ -799,7 +844,59 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
             *reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(t.m0 + rr) * p.N + n0 + 8 * c) = o;
           }
         }
-        if (ch < 3) named_bar_sync(1, 256);  // read out before the next chunk overwrites it
+      };
+      if constexpr (!kEpilogue) {
+        // the whole row into packed registers first, then the accumulator is free
+        // for the next tile's MMAs while the chunks go out
+        uint32_t pk[64];
+#pragma unroll
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(taddr + c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pk[c0 / 2 + e] = pack_bf16x2(__uint_as_float(r[2 * e]) * os, __uint_as_float(r[2 * e + 1]) * os);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acce);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          if ((ch >> 1) == h) stage_chunk(pk + (ch & 1) * 32);
+          named_bar_sync(1, 256);
+          store_chunk(ch);
+          if (ch < 3) named_bar_sync(1, 256);  // read out before the next chunk overwrites it
+        }
+      } else {
+        // bias and/or activation: 64 columns at a time (fewer live registers); the
+        // accumulator is released after the second half has been read
+        const float* brow = p.bias != nullptr ? p.bias + static_cast<int64_t>(t.g) * p.N : nullptr;
+#pragma unroll 1
+        for (int part = 0; part < 2; ++part) {
+          uint32_t pk[32];
+          const uint32_t ta = taddr + part * 64;
+          const int nc = t.nt * kRowsTile + h * 128 + part * 64;
+          switch (p.act) {
+            case 1: drain64<1>(ta, os, brow, nc, p.N, pk); break;
+            case 2: drain64<2>(ta, os, brow, nc, p.N, pk); break;
+            case 4: drain64<4>(ta, os, brow, nc, p.N, pk); break;
+            case 5: drain64<5>(ta, os, brow, nc, p.N, pk); break;
+            default: drain64<0>(ta, os, brow, nc, p.N, pk);
+          }
+          if (part == 1) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(acce);
+          }
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {  // chunk 2 hh + part comes from half hh
+            if (hh == h) stage_chunk(pk);
+            named_bar_sync(1, 256);
+            store_chunk(2 * hh + part);
+            if (part == 0 || hh == 0) named_bar_sync(1, 256);
+          }
+        }
       }
     }
   }
@@ -824,6 +921,8 @@ struct FusedParams {
   int32_t* status;
   int plain;               // plain MXFP4 (no D, no Hadamard; D not read)
   float out_scale;         // 2^-5 (MACAQ) or 1 (plain)
+  const float* bias;       // fp32 [N] or nullptr
+  int act;                 // act_type (act_value)
 };
 
 namespace fused {
@@ -862,7 +961,8 @@ struct Cfg {
 };
 }  // namespace fused
 
-template <int BT>
+// kEpilogue: the bias / activation epilogue (p.bias, p.act) is compiled in.
+template <int BT, bool kEpilogue = false>
 __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const __grid_constant__ FusedParams p) {
   using C = fused::Cfg<BT>;
   using fused::kStages;
@@ -1187,12 +1287,26 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
         s[0] += a.x; s[1] += a.y; s[2] += a.z; s[3] += a.w;
         s[4] += b.x; s[5] += b.y; s[6] += b.z; s[7] += b.w;
       }
-      uint4 o;
       const float os = p.out_scale;
-      o.x = pack_bf16x2(s[0] * os, s[1] * os);
-      o.y = pack_bf16x2(s[2] * os, s[3] * os);
-      o.z = pack_bf16x2(s[4] * os, s[5] * os);
-      o.w = pack_bf16x2(s[6] * os, s[7] * os);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s[i] *= os;
+      if constexpr (kEpilogue) {
+        if (p.bias != nullptr) {
+          const float4* b = reinterpret_cast<const float4*>(p.bias + n0 + n);
+          const float4 b0 = __ldg(b), b1 = __ldg(b + 1);
+          s[0] += b0.x; s[1] += b0.y; s[2] += b0.z; s[3] += b0.w;
+          s[4] += b1.x; s[5] += b1.y; s[6] += b1.z; s[7] += b1.w;
+        }
+        if (p.act != 0) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) s[i] = act_value_rt(s[i], p.act);
+        }
+      }
+      uint4 o;
+      o.x = pack_bf16x2(s[0], s[1]);
+      o.y = pack_bf16x2(s[2], s[3]);
+      o.z = pack_bf16x2(s[4], s[5]);
+      o.w = pack_bf16x2(s[6], s[7]);
       *reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(m0 + t) * p.N + n0 + n) = o;
     }
   }
@@ -1247,15 +1361,25 @@ int current_device(int& dev, int& sms) {
   if (!s.is_sm100) return MACAQ_ERR_ARCH;
   if (!s.attrs_set) {  // once per device: opt in to the shared memory the kernels use
     const size_t gemm_smem = gemm::kSmemLimit;  // smem_bytes(E) stays within it for every E
-    bool ok = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    bool ok = cudaFuncSetAttribute(gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    static_cast<int>(gemm_smem)) == cudaSuccess;
+    ok = ok && cudaFuncSetAttribute(gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    static_cast<int>(gemm_smem)) == cudaSuccess;
     ok = ok && cudaFuncSetAttribute(fused_small_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    fused::Cfg<16>::kSmemBytes) == cudaSuccess;
+    ok = ok && cudaFuncSetAttribute(fused_small_kernel<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     fused::Cfg<16>::kSmemBytes) == cudaSuccess;
     ok = ok && cudaFuncSetAttribute(fused_small_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     fused::Cfg<32>::kSmemBytes) == cudaSuccess;
+    ok = ok && cudaFuncSetAttribute(fused_small_kernel<32, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    fused::Cfg<32>::kSmemBytes) == cudaSuccess;
     ok = ok && cudaFuncSetAttribute(fused_small_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     fused::Cfg<64>::kSmemBytes) == cudaSuccess;
+    ok = ok && cudaFuncSetAttribute(fused_small_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    fused::Cfg<64>::kSmemBytes) == cudaSuccess;
     ok = ok && cudaFuncSetAttribute(fused_small_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    fused::Cfg<128>::kSmemBytes) == cudaSuccess;
+    ok = ok && cudaFuncSetAttribute(fused_small_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     fused::Cfg<128>::kSmemBytes) == cudaSuccess;
     ok = ok && cudaFuncSetAttribute(quant_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmem) ==
                    cudaSuccess;
@@ -1381,22 +1505,28 @@ FusedPlan plan_fused(int dev, int64_t M, int64_t N, int64_t K) {
   return best;
 }
 
-int launch_fused(const FusedParams& p, const FusedPlan& plan, cudaStream_t st) {
+template <bool kEpilogue>
+cudaError_t launch_fused_kind(const FusedParams& p, const FusedPlan& plan, cudaStream_t st) {
   const dim3 grid(plan.ctas), block(fused::kThreads);
-  cudaError_t e;
   switch (plan.bt) {
     case 16:
-      e = launch_ex(fused_small_kernel<16>, grid, block, fused::Cfg<16>::kSmemBytes, st, true, plan.S, p);
-      break;
+      return launch_ex(fused_small_kernel<16, kEpilogue>, grid, block, fused::Cfg<16>::kSmemBytes, st, true, plan.S,
+                       p);
     case 32:
-      e = launch_ex(fused_small_kernel<32>, grid, block, fused::Cfg<32>::kSmemBytes, st, true, plan.S, p);
-      break;
+      return launch_ex(fused_small_kernel<32, kEpilogue>, grid, block, fused::Cfg<32>::kSmemBytes, st, true, plan.S,
+                       p);
     case 64:
-      e = launch_ex(fused_small_kernel<64>, grid, block, fused::Cfg<64>::kSmemBytes, st, true, plan.S, p);
-      break;
+      return launch_ex(fused_small_kernel<64, kEpilogue>, grid, block, fused::Cfg<64>::kSmemBytes, st, true, plan.S,
+                       p);
     default:
-      e = launch_ex(fused_small_kernel<128>, grid, block, fused::Cfg<128>::kSmemBytes, st, true, plan.S, p);
+      return launch_ex(fused_small_kernel<128, kEpilogue>, grid, block, fused::Cfg<128>::kSmemBytes, st, true,
+                       plan.S, p);
   }
+}
+
+int launch_fused(const FusedParams& p, const FusedPlan& plan, cudaStream_t st) {
+  const cudaError_t e = (p.bias != nullptr || p.act != 0) ? launch_fused_kind<true>(p, plan, st)
+                                                          : launch_fused_kind<false>(p, plan, st);
   return e == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
@@ -1461,9 +1591,24 @@ int quant_grid(int64_t slabs, int KT, int sms) {
 
 // Dense quantise-once: the quantiser over all rows, then the GEMM (launched as
 // a programmatic dependent of the quantiser when `pdl`).
+// Output epilogue of the _ex calls: fp32 bias (nullptr: none) and act_type.
+struct Epilogue {
+  const float* bias = nullptr;
+  int act = 0;
+};
+bool act_supported(int act) { return act == 0 || act == 1 || act == 2 || act == 4 || act == 5; }
+// bias: 16-byte aligned, rows * N floats, not overlapping y.
+int check_epilogue(const Epilogue& ep, int64_t rows, int64_t N, const void* y, size_t ybytes) {
+  if (!act_supported(ep.act)) return MACAQ_ERR_ACT_TYPE;
+  if (ep.bias == nullptr) return MACAQ_OK;
+  if (!aligned16(ep.bias)) return MACAQ_ERR_ALIGN;
+  if (overlaps(y, ybytes, ep.bias, static_cast<size_t>(rows) * N * 4)) return MACAQ_ERR_ALIAS;
+  return MACAQ_OK;
+}
+
 int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y,
                          int64_t M, int64_t N, int64_t K, uint8_t* ws, int32_t* status, cudaStream_t st, int sms,
-                         bool pdl, bool plain = false) {
+                         bool pdl, bool plain = false, Epilogue ep = Epilogue()) {
   const DenseWs w = dense_ws(M, K);
   const int MT = static_cast<int>(pad128(M) / 128), KT = static_cast<int>(K / 256);
   QuantParams qp{};
@@ -1479,12 +1624,15 @@ int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, c
   gp.NT = static_cast<int>(pad128(N) / 128); gp.KT = KT; gp.E = 1; gp.MT = MT;
   gp.NT2 = (gp.NT + 1) / 2; gp.stages = gemm::stages_for(0);
   gp.out_scale = plain ? 1.0f : 0.03125f;
+  gp.bias = ep.bias;
+  gp.act = ep.act;
   gp.status = status;
   gp.wait_for_producer = pdl ? 1 : 0;
   const int tiles = MT * gp.NT2;
   const int grid = tiles < sms ? tiles : sms;
   const cudaError_t e =
-      launch_ex(gemm_kernel, dim3(grid), dim3(gemm::kThreads), gemm::smem_bytes(0), st, pdl, 1, gp);
+      launch_ex(gp.bias != nullptr || gp.act != 0 ? gemm_kernel<true> : gemm_kernel<false>, dim3(grid),
+                dim3(gemm::kThreads), gemm::smem_bytes(0), st, pdl, 1, gp);
   return e == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
@@ -1525,6 +1673,7 @@ const char* macaq_status_string(int s) {
     case MACAQ_ERR_GROUP_LIST_INVALID: return "MACAQ_ERR_GROUP_LIST_INVALID";
     case MACAQ_ERR_WORKSPACE: return "MACAQ_ERR_WORKSPACE";
     case MACAQ_ERR_BAD_D: return "MACAQ_ERR_BAD_D";
+    case MACAQ_ERR_ACT_TYPE: return "MACAQ_ERR_ACT_TYPE";
     default: return "MACAQ_ERR_UNKNOWN";
   }
 }
@@ -1596,8 +1745,10 @@ size_t macaq_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t E) {
 }
 
 static int dense_impl(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M,
-               int64_t N, int64_t K, void* workspace, size_t workspace_bytes, int32_t* status, void* stream, bool plain) {
+               int64_t N, int64_t K, void* workspace, size_t workspace_bytes, int32_t* status, void* stream, bool plain,
+               Epilogue ep = Epilogue()) {
   int st = check_mm_args(x, D, Wq, Ws, y, M, N, K, 1, plain);
+  if (st == MACAQ_OK) st = check_epilogue(ep, 1, N, y, static_cast<size_t>(M) * N * 2);
   if (st != MACAQ_OK || M == 0) return st;
   if (M > kSmallM) {
     st = check_ws(workspace, workspace_bytes, dense_ws(M, K).total, y, static_cast<size_t>(M) * N * 2, x,
@@ -1618,18 +1769,21 @@ static int dense_impl(const uint16_t* x, const float* D, const uint8_t* Wq, cons
     p.status = status;
     p.plain = plain ? 1 : 0;
     p.out_scale = plain ? 1.0f : 0.03125f;
+    p.bias = ep.bias;
+    p.act = ep.act;
     return launch_fused(p, plan, s);
   }
   return run_dense_two_kernel(x, D, Wq, Ws, y, M, N, K, static_cast<uint8_t*>(workspace), status, s, sms, true,
-                              plain);
+                              plain, ep);
 }
 
 static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, const int64_t* group_list,
                  int group_list_type, int64_t E, uint16_t* y, int64_t M, int64_t N, int64_t K, void* workspace,
-                 size_t workspace_bytes, int32_t* status, void* stream, bool plain) {
+                 size_t workspace_bytes, int32_t* status, void* stream, bool plain, Epilogue ep = Epilogue()) {
   if (E < 1 || E > kMaxGroups) return MACAQ_ERR_TOO_MANY_GROUPS;
   if (group_list_type < 0 || group_list_type > 2) return MACAQ_ERR_GROUP_LIST_TYPE;
   int st = check_mm_args(x, D, Wq, Ws, y, M, N, K, E, plain);
+  if (st == MACAQ_OK) st = check_epilogue(ep, E, N, y, static_cast<size_t>(M) * N * 2);
   if (st != MACAQ_OK) return st;
   if (M == 0) return MACAQ_OK;
   if (!group_list) return MACAQ_ERR_NULL;
@@ -1668,8 +1822,11 @@ static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, co
   gp.NT2 = (gp.NT + 1) / 2; gp.stages = gemm::stages_for(static_cast<int>(E));
   gp.goff = goff; gp.gtp = gtp; gp.gexp = gexp; gp.valid = valid;
   gp.out_scale = plain ? 1.0f : 0.03125f;
+  gp.bias = ep.bias;
+  gp.act = ep.act;
   gp.status = status;
-  const cudaError_t e = launch_ex(gemm_kernel, dim3(sms), dim3(gemm::kThreads),
+  const cudaError_t e = launch_ex(gp.bias != nullptr || gp.act != 0 ? gemm_kernel<true> : gemm_kernel<false>,
+                                  dim3(sms), dim3(gemm::kThreads),
                                   gemm::smem_bytes(static_cast<int>(E)), s, true, 1, gp);
   return e == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
@@ -1677,6 +1834,26 @@ static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, co
 int macaq_dense_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M,
                    int64_t N, int64_t K, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
   return dense_impl(x, D, Wq, Ws, y, M, N, K, workspace, workspace_bytes, status, stream, false);
+}
+
+int macaq_dense_mm_ex(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, const float* bias,
+                      int act_type, uint16_t* y, int64_t M, int64_t N, int64_t K, void* workspace,
+                      size_t workspace_bytes, int32_t* status, void* stream) {
+  Epilogue ep;
+  ep.bias = bias;
+  ep.act = act_type;
+  return dense_impl(x, D, Wq, Ws, y, M, N, K, workspace, workspace_bytes, status, stream, false, ep);
+}
+
+int macaq_grouped_mm_ex(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws,
+                        const int64_t* group_list, int group_list_type, int64_t E, const float* bias, int act_type,
+                        uint16_t* y, int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                        int32_t* status, void* stream) {
+  Epilogue ep;
+  ep.bias = bias;
+  ep.act = act_type;
+  return grouped_impl(x, D, Wq, Ws, group_list, group_list_type, E, y, M, N, K, workspace, workspace_bytes, status,
+                      stream, false, ep);
 }
 
 int macaq_dense_mm_plain(const uint16_t* x, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M, int64_t N,

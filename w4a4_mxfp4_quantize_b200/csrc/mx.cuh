@@ -78,6 +78,12 @@ __device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v
 constexpr int kRcpStride = kBlk + 2;
 constexpr int kRcpTile = 8 * kRcpStride;  // floats per K tile
 __host__ __device__ constexpr int rcp_index(int k) { return (k >> 5) * kRcpStride + (k & 31); }
+// The quantisers' layout: blocks 36 floats apart, so each block starts on a 16-byte
+// boundary and a warp's 16-byte loads of the same element of the eight blocks
+// cover all 32 banks once.
+constexpr int kQRcpStride = kBlk + 4;
+constexpr int kQRcpTile = 8 * kQRcpStride;
+__host__ __device__ constexpr int qrcp_index(int k) { return (k >> 5) * kQRcpStride + (k & 31); }
 
 __device__ __forceinline__ uint32_t e8m0_from_amax_bits(uint32_t amax_bits) {
   const uint32_t e = amax_bits >> 23;  // sign is clear
@@ -154,18 +160,21 @@ __device__ __forceinline__ uint32_t e2m1x8_f2(uint64_t a, uint64_t b, uint64_t c
 }
 
 // Activation block: 32 bf16 values (four 16-byte words) and the 32
-// reciprocals r = RN32(1/D) of their channels (r must be 8-byte aligned).
+// reciprocals r = RN32(1/D) of their channels (r must be 16-byte aligned).
 // Same arithmetic as the scalar definition, two lanes per instruction:
 //   xs = RNE_bf16(RN32(x * r)); FP32 butterfly h = 1, 2, 4, 8, 16;
 //   u = RNE_bf16(.); E8M0 from the block amax of |u|; E2M1 of u * 2^(127-c).
 __device__ __forceinline__ void act_block(const uint4 (&xv)[4], const float* __restrict__ r, uint4& codes,
                                           uint32_t& scale) {
   const uint32_t* w = reinterpret_cast<const uint32_t*>(xv);
-  const uint64_t* r2 = reinterpret_cast<const uint64_t*>(r);
+  const uint4* r4 = reinterpret_cast<const uint4*>(r);
   uint64_t P[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    const uint32_t xs = f2_to_bf16x2(f2_mul(bf16x2_to_f2(w[j]), r2[j]));  // channel scaling, BF16
+    const uint4 rq = r4[j >> 1];  // four reciprocals per 16-byte load
+    const uint64_t r2 = (j & 1) ? f2(__uint_as_float(rq.z), __uint_as_float(rq.w))
+                                : f2(__uint_as_float(rq.x), __uint_as_float(rq.y));
+    const uint32_t xs = f2_to_bf16x2(f2_mul(bf16x2_to_f2(w[j]), r2));  // channel scaling, BF16
     // butterfly stage h = 1 inside the pair: (v0 + v1, v0 - v1)
     const float v0 = bf16lo(xs), v1 = bf16hi(xs);
     P[j] = f2(__fadd_rn(v0, v1), __fsub_rn(v0, v1));
