@@ -94,6 +94,28 @@ size_t macaq_weight_scale_bytes(int64_t E, int64_t N, int64_t K);
 int macaq_prepare_weights(const float *W_dev, const float *D_dev, int64_t E, int64_t N, int64_t K,
                           uint8_t *Wq_dev, uint8_t *Ws_dev, void *stream);
 
+/* Offline calibration of the channel factors D.  The MACAQ page lists
+ * calibration among the offline steps ("Calibration, weight transformation
+ * ... are offline"; the accuracy pilot calibrates on 1,024 tokens) without
+ * stating the rule; the rule here is the square-root range balance that makes
+ * max|x[:,k]| / D[k] equal max|W[:,k]| * D[k]:
+ *     D[e, k] = clamp(sqrt(a / w), 1e-2, 1e2)   (binary64, rounded to fp32)
+ *     a = max |x[t, k]| over expert e's calibration rows t,
+ *     w = max |W[e, n, k]| over n;
+ * w = 0 < a gives 1e2, a = w = 0 gives 1, an expert with no rows gives 1.
+ *   x_dev   bf16 [T, K] calibration activations (may be NULL when T = 0);
+ *   W_dev   fp32 [E, N, K], the same weights later passed to
+ *           macaq_prepare_weights;
+ *   group_list_dev: NULL (E must be 1: every row is expert 0's) or a group
+ *           list over the T rows in the form of macaq_grouped_mm (types 0, 1,
+ *           2); it is read back to the host and checked (offline), an invalid
+ *           list returns MACAQ_ERR_GROUP_LIST_INVALID without launching;
+ *   D_dev   fp32 [E, K] (written); must not overlap the inputs.
+ * Shapes: 0 <= T <= 2^31 - 1; 1 <= N <= 65536; K as above; 1 <= E <= 1024.
+ * Synchronises `stream` once when a group list is given. */
+int macaq_calibrate_d(const uint16_t *x_dev, int64_t T, const float *W_dev, int64_t E, int64_t N, int64_t K,
+                      const int64_t *group_list_dev, int group_list_type, float *D_dev, void *stream);
+
 /* ------------------------------------------------------------------ */
 /* Hot path                                                            */
 /* ------------------------------------------------------------------ */

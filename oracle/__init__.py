@@ -81,6 +81,7 @@ def _L():
             "oracle_gemm_ex": (I, [P, P, P, P, I64, I64, I64, P, I, P, I]),
             "oracle_gemm_at_ex": (I, [P, P, P, P, I64, P, P, I64, P, I, P]),
             "oracle_act_array": (None, [P, I64, I, P]),
+            "oracle_calibrate_d": (I, [P, I64, P, I64, I64, I64, P, I, P]),
             "oracle_f64_to_bf16_array": (None, [P, I64, P]),
             "oracle_linear_f64": (None, [P, P, I64, I64, I64, P]),
             "oracle_transform_f64": (None, [P, P, P, I64, I64, I64, P]),
@@ -339,6 +340,22 @@ def grouped_mm_ex(x_bf16, D, W, group_list, group_list_type: int, bias=None, act
     st = _L().oracle_grouped_mm_ex(_p(x), _p(D), _p(W), _p(gl), int(group_list_type), E, M, N, K, bp,
                                    int(act_type), _p(y), nthreads)
     return int(st), y
+
+
+def calibrate_d(x_bf16, W, group_list=None, group_list_type: int = 1):
+    """Offline channel factors D [E, K] from calibration activations x bf16 [T, K]
+    and weights W fp32 [E, N, K] (reading R16).  Returns (status, D)."""
+    x = _c(x_bf16, np.uint16)
+    W = _c(W, np.float32)
+    if W.ndim == 2:
+        W = W[None]
+    T, K = x.shape
+    E, N, _ = W.shape
+    gl = None if group_list is None else _c(group_list, np.int64)
+    D = np.empty((E, K), np.float32)
+    st = _L().oracle_calibrate_d(_p(x), T, _p(W), E, N, K, None if gl is None else _p(gl), int(group_list_type),
+                                 _p(D))
+    return int(st), D
 
 
 def linear_f64(x_bf16, W) -> np.ndarray:

@@ -39,7 +39,13 @@
  *       s = 2^-5 * exact sum (the bias in output units, the page's
  *       y_i = x_i @ weight_i + bias_i), evaluated here in binary64;
  *       FAST_GELU, which the page does not define, is read as
- *       v / (1 + exp(-1.702 v)).
+ *       v / (1 + exp(-1.702 v));
+ *   R16 offline calibration of D (the MACAQ page lists calibration among the
+ *       offline steps without stating the rule): per expert and input
+ *       channel k, D[k] = clamp(sqrt(a / w), 1e-2, 1e2) in binary64, rounded
+ *       to fp32, with a = max |x[:, k]| over that expert's calibration rows
+ *       and w = max |W[:, k]| over its N weight rows; w = 0 < a gives 1e2,
+ *       a = w = 0 gives 1, an expert with no rows gives D = 1 everywhere.
  *
  * The plain MXFP4 baseline (the MACAQ page's native W4A4 comparison, which
  * quantises x and W directly with the dynamic MX quantiser) skips D and H:
@@ -769,6 +775,81 @@ int oracle_grouped_mm(const uint16_t *x, const float *D, const float *W, const i
                       int nthreads)
 {
     return oracle_grouped_mm_ex(x, D, W, group_list, type, E, M, N, K, NULL, 0, y, nthreads);
+}
+
+/* ------------------------------------------------------------------ */
+/* Offline calibration of D (R16)                                      */
+/* ------------------------------------------------------------------ */
+
+static float calib_value(double a, double w)
+{
+    double d;
+    if (a == 0.0 && w == 0.0)
+        d = 1.0;
+    else if (w == 0.0)
+        d = 1e2;
+    else
+        d = sqrt(a / w);
+    if (d < 1e-2)
+        d = 1e-2;
+    if (d > 1e2)
+        d = 1e2;
+    return (float)d;
+}
+
+/* x bf16 [T, K] calibration activations; W fp32 [E, N, K]; group_list as in
+ * oracle_group_offsets (NULL: all T rows belong to expert 0, E must be 1).
+ * Writes D fp32 [E, K]. */
+int oracle_calibrate_d(const uint16_t *x, int64_t T, const float *W, int64_t E, int64_t N, int64_t K,
+                       const int64_t *group_list, int type, float *D)
+{
+    if (E < 1 || N < 1 || K < 1 || T < 0)
+        return ORACLE_ERR_SHAPE;
+    int64_t *off = (int64_t *)malloc(sizeof(int64_t) * (size_t)(E + 1));
+    if (group_list) {
+        int st = oracle_group_offsets(group_list, type, E, T, off);
+        if (st != ORACLE_OK) {
+            free(off);
+            return st;
+        }
+    } else {
+        if (E != 1) {
+            free(off);
+            return ORACLE_ERR_SHAPE;
+        }
+        off[0] = 0;
+        off[1] = T;
+    }
+    double *a = (double *)calloc((size_t)(E * K), sizeof(double));
+    int64_t *rows = (int64_t *)calloc((size_t)E, sizeof(int64_t));
+    for (int64_t g = 0; g < E; g++) {
+        int64_t e = (group_list && type == 2) ? group_list[2 * g] : g; /* the expert of list entry g */
+        rows[e] += off[g + 1] - off[g];
+        for (int64_t r = off[g]; r < off[g + 1]; r++)
+            for (int64_t k = 0; k < K; k++) {
+                double v = fabs(oracle_bf16_to_f64(x[r * K + k]));
+                if (v > a[e * K + k])
+                    a[e * K + k] = v;
+            }
+    }
+    for (int64_t e = 0; e < E; e++)
+        for (int64_t k = 0; k < K; k++) {
+            if (rows[e] == 0) {
+                D[e * K + k] = 1.0f;
+                continue;
+            }
+            double w = 0.0;
+            for (int64_t n = 0; n < N; n++) {
+                double v = fabs((double)W[(e * N + n) * K + k]);
+                if (v > w)
+                    w = v;
+            }
+            D[e * K + k] = calib_value(a[e * K + k], w);
+        }
+    free(a);
+    free(rows);
+    free(off);
+    return ORACLE_OK;
 }
 
 /* ------------------------------------------------------------------ */

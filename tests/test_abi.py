@@ -114,6 +114,24 @@ def test_epilogue_refusals_by_name(L):
     assert g(act=2, b=None) == -11                # accepted; the missing workspace is the next refusal
 
 
+def test_calibration_refusals_by_name(L):
+    x, W, D, gl = P(1 << 32), P(2 << 32), P(3 << 32), P(4 << 32)
+
+    def c(x=x, T=1024, W=W, E=1, N=512, K=1024, gl=None, t=1, D=D):
+        return L.macaq_calibrate_d(x, T, W, E, N, K, gl, t, D, None)
+
+    assert c(E=0) == -6
+    assert c(E=1025, gl=gl) == -6
+    assert c(K=1000) == -3
+    assert c(N=0) == -3
+    assert c(T=-1) == -3
+    assert c(E=4) == -1                 # a group list is needed for E > 1
+    assert c(D=None) == -1
+    assert c(E=4, gl=gl, t=3) == -7
+    assert c(D=P((3 << 32) + 4)) == -2
+    assert c(D=P((1 << 32) + 1024)) == -5   # D inside x
+
+
 def test_no_gpu_means_a_named_cuda_error_not_a_fallback(L):
     import torch
     if torch.cuda.is_available():

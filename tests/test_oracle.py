@@ -645,3 +645,83 @@ def test_grouped_epilogue_uses_each_experts_bias():
         if counts[g]:
             ref = oracle.dense_mm_ex(p.x[off[g]:off[g + 1]], p.D[0], p.W[0], bias[g], oracle.ACT_GELU_TANH)
             assert np.array_equal(y[off[g]:off[g + 1]], ref)
+
+
+# ----------------------------------------------------------------------------
+# Offline calibration of D (reading R16: D = clamp(sqrt(max|x| / max|W|), 1e-2, 1e2))
+# ----------------------------------------------------------------------------
+
+def test_calibration_equalises_the_channel_ranges():
+    # the defining property of the square-root rule: after x / D and W * D both
+    # sides of every channel have the same range, sqrt(max|x| max|W|)
+    p = synth.dense(200, 512, 96, seed=13)
+    st, D = oracle.calibrate_d(p.x, p.W)
+    assert st == oracle.OK
+    a = np.abs(synth.bf16_bits_to_f32(p.x).astype(np.float64)).max(axis=0)
+    w = np.abs(p.W[0].astype(np.float64)).max(axis=0)
+    d = D[0].astype(np.float64)
+    free = (d > 1e-2) & (d < 1e2)
+    assert free.mean() > 0.9
+    np.testing.assert_allclose((a / d)[free], (w * d)[free], rtol=2.5e-7)
+    np.testing.assert_allclose((a / d)[free], np.sqrt(a * w)[free], rtol=1.5e-7)
+
+
+def test_calibration_special_cases():
+    K, N, T = 256, 8, 4
+    x = np.zeros((T, K), np.float32)
+    W = np.zeros((N, K), np.float32)
+    x[:, 1] = 1.0                  # w = 0 < a             -> 1e2
+    W[:, 2] = 1.0                  # a = 0 < w             -> clamp(0) = 1e-2
+    x[:, 3], W[:, 3] = 2.0 ** 20, 2.0 ** -20   # a / w = 2^40 -> clamp 1e2
+    x[:, 4], W[:, 4] = 2.0 ** -20, 2.0 ** 20   # a / w = 2^-40 -> clamp 1e-2
+    x[:, 5], W[:, 5] = 9.0, 1.0                # sqrt(9) = 3 exactly
+    x[2, 6], W[5, 6] = -16.0, -4.0             # magnitudes: sqrt(4) = 2
+    st, D = oracle.calibrate_d(synth.to_bf16_bits(x), W)
+    assert st == oracle.OK
+    expect = np.ones(K, np.float32)            # column 0 and the rest: a = w = 0 -> 1
+    expect[[1, 2, 3, 4, 5, 6]] = [1e2, 1e-2, 1e2, 1e-2, 3.0, 2.0]
+    assert np.array_equal(D[0], expect.astype(np.float32))
+
+
+def test_calibration_scales_with_the_square_root_of_the_activation_range():
+    p = synth.dense(64, 256, 32, seed=17)
+    xf = synth.bf16_bits_to_f32(p.x)
+    _, D1 = oracle.calibrate_d(p.x, p.W)
+    _, D4 = oracle.calibrate_d(synth.to_bf16_bits(xf * 4.0), p.W)   # exact in bf16
+    free = (D1 > 2e-2) & (D1 < 50)
+    assert np.array_equal(D4[free], (D1 * 2)[free])
+
+
+def test_calibration_takes_each_experts_rows():
+    # type 2 names the expert of each row range; an expert named twice is
+    # calibrated on both of its ranges, an expert never named gets D = 1
+    rng = np.random.default_rng(19)
+    E, K, N = 4, 256, 16
+    xf = rng.standard_normal((60, K)).astype(np.float32)
+    xf[:, 7] *= 50
+    xb = synth.to_bf16_bits(xf)
+    W = rng.standard_normal((E, N, K)).astype(np.float32)
+    gl = np.array([[2, 20], [0, 15], [2, 25], [3, 0]], np.int64)
+    st, D = oracle.calibrate_d(xb, W, gl, 2)
+    assert st == oracle.OK
+    _, D2 = oracle.calibrate_d(np.concatenate([xb[:20], xb[35:60]]), W[2])
+    _, D0 = oracle.calibrate_d(xb[20:35], W[0])
+    assert np.array_equal(D[2], D2[0]) and np.array_equal(D[0], D0[0])
+    assert np.array_equal(D[1], np.ones(K, np.float32)) and np.array_equal(D[3], np.ones(K, np.float32))
+    # counts and cumulative sums give the same factors
+    counts = np.array([10, 0, 30, 20], np.int64)
+    _, Dc = oracle.calibrate_d(xb, W, counts, 1)
+    _, Ds = oracle.calibrate_d(xb, W, np.cumsum(counts), 0)
+    assert np.array_equal(Dc, Ds)
+    assert oracle.calibrate_d(xb, W, np.array([10, 0, 30, 19], np.int64), 1)[0] == oracle.ERR_GROUP_LIST_INVALID
+
+
+def test_calibration_reproduces_the_generator_factors():
+    # the workload generator states the same rule independently (dense, and
+    # grouped with Zipf-skewed counts including empty experts)
+    p = synth.dense(128, 1024, 256, seed=0)
+    st, D = oracle.calibrate_d(p.x, p.W)
+    assert st == oracle.OK and np.array_equal(D, p.D)
+    g = synth.grouped(2048, 32, 512, 64, seed=1, dist="zipf", group_list_type=0)
+    st, D = oracle.calibrate_d(g.x, g.W, g.group_list, g.group_list_type)
+    assert st == oracle.OK and np.array_equal(D, g.D)

@@ -92,6 +92,7 @@ _SIG = {
     "macaq_unfused_dense_mm": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, _P, ctypes.c_size_t,
                                               _P, _P]),
     "macaq_prepare_weights_plain": (ctypes.c_int, [_P, _I64, _I64, _I64, _P, _P, _P]),
+    "macaq_calibrate_d": (ctypes.c_int, [_P, _I64, _P, _I64, _I64, _I64, _P, ctypes.c_int, _P, _P]),
     "macaq_dense_mm_plain": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, ctypes.c_size_t, _P, _P]),
     "macaq_grouped_mm_plain": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _I64, _P, _I64, _I64, _I64, _P,
                                               ctypes.c_size_t, _P, _P]),
@@ -219,6 +220,21 @@ def _check_bias(bias, shape):
     _require_cuda(bias)
     if bias.dtype != torch.float32 or tuple(bias.shape) != shape:
         raise ValueError(f"bias must be float32 of shape {shape}, got {bias.dtype} {tuple(bias.shape)}")
+
+
+def calibrate_d(x_cal: torch.Tensor, W: torch.Tensor, group_list: torch.Tensor | None = None,
+                group_list_type: int = 1, stream=None) -> torch.Tensor:
+    """Offline: channel factors D fp32 [E, K] from calibration activations x_cal bf16
+    [T, K] and weights W fp32 [N, K] or [E, N, K] (rows split by group_list when E > 1)."""
+    if W.dim() == 2:
+        W = W.unsqueeze(0)
+    _require_cuda(x_cal, W, group_list)
+    T, K = x_cal.shape
+    E, N, _ = W.shape
+    D = torch.empty((E, K), dtype=torch.float32, device=W.device)
+    _check(lib().macaq_calibrate_d(_ptr(x_cal), T, _ptr(W), E, N, K, _ptr(group_list), int(group_list_type),
+                                   _ptr(D), _stream_ptr(stream)), "macaq_calibrate_d")
+    return D
 
 
 def dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: int,

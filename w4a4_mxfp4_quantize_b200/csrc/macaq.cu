@@ -324,6 +324,73 @@ __device__ __forceinline__ int find_group(const int* gtp, int E, int pm) {
 }
 
 // ============================================================================
+// Offline calibration of D
+// ============================================================================
+// The MACAQ page lists calibration among the offline steps without a rule; the
+// rule here is the square-root range balance D[k] = clamp(sqrt(a / w), 1e-2,
+// 1e2) per expert and input channel, a = max |x[:, k]| over the expert's
+// calibration rows, w = max |W[:, k]| over its weight rows, in binary64 and
+// rounded once to fp32 (w = 0 < a gives 1e2, a = w = 0 gives 1, an expert with
+// no rows gives 1).  One CTA per (256 channels, expert): 1024 threads = 256
+// channels x 4 row lanes, the lanes' maxima combined in shared memory.
+struct CalibParams {
+  const uint16_t* x;  // bf16 [T, K]
+  const float* W;     // [E, N, K]
+  const int64_t* gl;  // group_list (validated by the host) or nullptr: every row is expert 0's
+  int type;
+  int E, N, K;
+  int64_t T;
+  float* D;           // [E, K]
+};
+
+__global__ void __launch_bounds__(1024) calibrate_kernel(const __grid_constant__ CalibParams p) {
+  __shared__ float sa[4][256], sw[4][256];
+  const int c = threadIdx.x & 255, lanes = threadIdx.x >> 8;
+  const int e = blockIdx.y;
+  const int64_t k = static_cast<int64_t>(blockIdx.x) * 256 + c;
+  float w = 0.f, a = 0.f;  // maxima of magnitudes: exact in any order
+  for (int n = lanes; n < p.N; n += 4) w = fmaxf(w, fabsf(__ldg(p.W + (static_cast<int64_t>(e) * p.N + n) * p.K + k)));
+  int64_t rows = 0;
+  auto scan = [&](int64_t r0, int64_t r1) {
+    for (int64_t r = r0 + lanes; r < r1; r += 4) a = fmaxf(a, fabsf(bf16lo(__ldg(p.x + r * p.K + k))));
+  };
+  if (p.gl == nullptr) {
+    scan(0, p.T);
+    rows = p.T;
+  } else {
+    int64_t r0 = 0;
+    for (int j = 0; j < p.E; ++j) {  // list entry j: its rows and the expert they use
+      int64_t cnt;
+      int ex = j;
+      if (p.type == 2) {
+        ex = static_cast<int>(p.gl[2 * j]);
+        cnt = p.gl[2 * j + 1];
+      } else {
+        cnt = p.type == 1 ? p.gl[j] : p.gl[j] - (j > 0 ? p.gl[j - 1] : 0);
+      }
+      if (ex == e) {
+        scan(r0, r0 + cnt);
+        rows += cnt;
+      }
+      r0 += cnt;
+    }
+  }
+  sa[lanes][c] = a;
+  sw[lanes][c] = w;
+  __syncthreads();
+  if (lanes == 0) {
+    a = fmaxf(fmaxf(sa[0][c], sa[1][c]), fmaxf(sa[2][c], sa[3][c]));
+    w = fmaxf(fmaxf(sw[0][c], sw[1][c]), fmaxf(sw[2][c], sw[3][c]));
+    double d;
+    if (rows == 0 || (a == 0.f && w == 0.f)) d = 1.0;
+    else if (w == 0.f) d = 1e2;
+    else d = sqrt(static_cast<double>(a) / static_cast<double>(w));  // IEEE divide and square root
+    d = fmin(fmax(d, 1e-2), 1e2);
+    p.D[static_cast<int64_t>(e) * p.K + k] = static_cast<float>(d);
+  }
+}
+
+// ============================================================================
 // Quantise-once: activation prologue over every row into tile images
 // ============================================================================
 // Work unit = one 32-row slab of a 128-row tile x one K tile: thread (tr, c) =
@@ -1854,6 +1921,54 @@ int macaq_grouped_mm_ex(const uint16_t* x, const float* D, const uint8_t* Wq, co
   ep.act = act_type;
   return grouped_impl(x, D, Wq, Ws, group_list, group_list_type, E, y, M, N, K, workspace, workspace_bytes, status,
                       stream, false, ep);
+}
+
+int macaq_calibrate_d(const uint16_t* x, int64_t T, const float* W, int64_t E, int64_t N, int64_t K,
+                      const int64_t* group_list, int group_list_type, float* D, void* stream) {
+  if (E < 1 || E > kMaxGroups) return MACAQ_ERR_TOO_MANY_GROUPS;
+  if (T < 0 || T > INT32_MAX || N < 1 || N > 65536 || K < 256 || K > 65536 || K % 256) return MACAQ_ERR_SHAPE;
+  if (!W || !D || (T > 0 && !x) || (!group_list && E != 1)) return MACAQ_ERR_NULL;
+  if (group_list && (group_list_type < 0 || group_list_type > 2)) return MACAQ_ERR_GROUP_LIST_TYPE;
+  if ((x && !aligned16(x)) || !aligned16(W) || !aligned16(D) || (group_list && !aligned16(group_list)))
+    return MACAQ_ERR_ALIGN;
+  const size_t dbytes = static_cast<size_t>(E) * K * 4;
+  const size_t gl_len = group_list ? static_cast<size_t>(E) * (group_list_type == 2 ? 2 : 1) : 0;
+  if (overlaps(D, dbytes, x, static_cast<size_t>(T) * K * 2) || overlaps(D, dbytes, W, static_cast<size_t>(E) * N * K * 4) ||
+      overlaps(D, dbytes, group_list, gl_len * 8))
+    return MACAQ_ERR_ALIAS;
+  int dev, sms;
+  int st = current_device(dev, sms);
+  if (st != MACAQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (group_list) {  // offline: read the list back and check it (npu_grouped_matmul's group_list rules)
+    std::vector<int64_t> h(gl_len);
+    if (cudaMemcpyAsync(h.data(), group_list, gl_len * 8, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return MACAQ_ERR_CUDA;
+    int64_t total = 0, prev = 0;
+    for (int64_t j = 0; j < E; ++j) {
+      int64_t cnt;
+      if (group_list_type == 2) {
+        if (h[2 * j] < 0 || h[2 * j] >= E) return MACAQ_ERR_GROUP_LIST_INVALID;
+        cnt = h[2 * j + 1];
+      } else if (group_list_type == 1) {
+        cnt = h[j];
+      } else {
+        if (h[j] < prev) return MACAQ_ERR_GROUP_LIST_INVALID;
+        cnt = h[j] - prev;
+        prev = h[j];
+      }
+      if (cnt < 0 || cnt > T) return MACAQ_ERR_GROUP_LIST_INVALID;
+      total += cnt;
+      if (total > T) return MACAQ_ERR_GROUP_LIST_INVALID;
+    }
+    if (total != T) return MACAQ_ERR_GROUP_LIST_INVALID;
+  }
+  CalibParams p{};
+  p.x = x; p.W = W; p.gl = group_list; p.type = group_list_type;
+  p.E = static_cast<int>(E); p.N = static_cast<int>(N); p.K = static_cast<int>(K); p.T = T; p.D = D;
+  calibrate_kernel<<<dim3(static_cast<unsigned>(K / 256), static_cast<unsigned>(E)), 1024, 0, s>>>(p);
+  return cudaPeekAtLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
 int macaq_dense_mm_plain(const uint16_t* x, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M, int64_t N,
