@@ -214,8 +214,11 @@ def capture(fn, stream):
 
 
 def time_graph(g, flush, stream, reps: int, warm: int = 3, cold: bool = True):
-    """Median / IQR of the device time (us) of one graph replay, CUDA events on
-    `stream`; the L2 flush (when `cold`) runs before the start event."""
+    """Mean (10% trimmed at each end) and IQR of the device time (us) of one graph
+    replay, CUDA events on `stream`; the L2 flush (when `cold`) runs before the
+    start event.  Event timestamps on this GPU advance in 2.048 us ticks; each
+    replay starts at an independent phase of the tick, so the mean of the ticked
+    durations is unbiased where a median would snap to the tick grid."""
     with torch.cuda.stream(stream):
         for _ in range(warm):
             g.replay()
@@ -230,9 +233,10 @@ def time_graph(g, flush, stream, reps: int, warm: int = 3, cold: bool = True):
             b.record(stream)
             evs.append((a, b))
     stream.synchronize()
-    t = sorted(a.elapsed_time(b) * 1e3 for a, b in evs)
-    q = np.percentile(t, [25, 50, 75])
-    return float(q[1]), float(q[2] - q[0])
+    t = np.sort([a.elapsed_time(b) * 1e3 for a, b in evs])
+    cut = len(t) // 10
+    q = np.percentile(t, [25, 75])
+    return float(np.mean(t[cut:len(t) - cut])), float(q[1] - q[0])
 
 
 # ---------------------------------------------------------------------------
@@ -388,7 +392,7 @@ def main():
     ms_per_step = total_ms / args.steps
 
     # per-call device time (one graph per call, L2 flushed before each): the roofline figure
-    per_call_us = [time_graph(g, flush, stream, max(args.steps, 10))[0] for g in call_graphs]
+    per_call_us = [time_graph(g, flush, stream, max(args.steps, 30))[0] for g in call_graphs]
     launch_s = sum(per_call_us) * 1e-6
     achieved_gbs = bytes_step / launch_s / 1e9
     roofline = {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm_gbs, "unit": "GB/s",
@@ -477,7 +481,7 @@ def run_only(args):
 
 
 def workload_table(mq, device, stream, flush, hbm_gbs, reps):
-    """us/call (median, cold L2), TFLOPS and roofline fraction for every
+    """us/call (trimmed mean, cold L2), TFLOPS and roofline fraction for every
     problem of the five workloads, fused and unfused (CUDA graph per call), the
     plain MXFP4 baseline's time, and both paths' error against the unquantised
     layer on sampled rows."""
