@@ -1048,6 +1048,21 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   float* part = reinterpret_cast<float*>(smem);  // local FP32 partial tile [BT][128], after the mainloop
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Work that needs no kernel parameter goes first: the first read of the
+  // parameters stalls each SM for hundreds of cycles (measured ~900).
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1 + fused::kProWarps / C::kGroups);
+      mbar_init(&empty[s], 1);
+      mbar_init(&sfull[s], 1);
+    }
+    mbar_init(&accf[0], 1);
+    *abort_flag = 0;
+  }
   const uint32_t rank = cluster_ctarank();
   const int cid = blockIdx.x / p.S;
   const int nt = cid % p.NT, mt = cid / p.NT;
@@ -1059,34 +1074,33 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   const bool split = p.S > 1;  // launched as a cluster of S CTAs; S == 1 touches no cluster state
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full[s], 1 + fused::kProWarps / C::kGroups);
-      mbar_init(&empty[s], 1);
-      mbar_init(&sfull[s], 1);
-    }
-    mbar_init(&accf[0], 1);
     if (split) {
       mbar_init(recv_bar, 1);
       mbar_arrive_expect_tx(recv_bar, static_cast<uint32_t>(p.S * rows_of(static_cast<int>(rank)) * kRowsTile * 4));
     }
-    *abort_flag = 0;
     fence_mbar_init();
   }
   const int nst = kt1 - kt0;                   // K tiles of this CTA
   const int pre = nst < kStages ? nst : kStages;  // first-use stages: no wait for a free slot
-  if (warp == 0) {
-    // The weights do not depend on any earlier kernel: their first stages go out as
-    // soon as the barriers exist (lane 0 initialised them), before the set-up below.
-    __syncwarp();
+  // The weights do not depend on any earlier kernel.  A bulk copy holds its
+  // issuing warp ~150 cycles, so only stage 0's two copies go out before the
+  // set-up barrier (which every warp waits for); the other first-use stages
+  // follow right after it.  Lanes 2j and 2j + 1 copy stage j's codes and scales.
+  auto first_copies = [&](int j0, int j1) {
     if (lane == 0)
-      for (int j = 0; j < pre; ++j) mbar_arrive_expect_tx(&full[j], kTileCodeBytes + kTileSfBytes);
+      for (int j = j0; j < j1; ++j) mbar_arrive_expect_tx(&full[j], kTileCodeBytes + kTileSfBytes);
     __syncwarp();
-    const int j = min(lane >> 1, pre - 1);
+    const int j = min(j0 + (lane >> 1), j1 - 1);
     const bool sf = lane & 1;
     const size_t wt = weight_image(0, nt, kt0 + j, (p.NT + 1) / 2, p.KT);
     uint8_t* sb = smem + j * C::kStageBytes;
-    bulk_g2s_if(lane < 2 * pre, sf ? sb + C::kOffSfa : sb, sf ? p.Ws + wt * kTileSfBytes : p.Wq + wt * kTileCodeBytes,
-                sf ? kTileSfBytes : kTileCodeBytes, &full[j]);
+    bulk_g2s_if(lane < 2 * (j1 - j0), sf ? sb + C::kOffSfa : sb,
+                sf ? p.Ws + wt * kTileSfBytes : p.Wq + wt * kTileCodeBytes, sf ? kTileSfBytes : kTileCodeBytes,
+                &full[j]);
+  };
+  if (warp == 0) {
+    __syncwarp();  // lane 0 initialised the barriers
+    first_copies(0, 1);
   }
   // Activation prologue set-up.  Each 32-element block is computed by a pair of
   // adjacent lanes (16 elements each), so every prologue warp is busy even for the
@@ -1127,10 +1141,6 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   }
   // (scale rows >= BT of the activation scale image are copied to TMEM but never
   // read: the MMA's N extent is BT)
-  if (warp == 1) {
-    tmem_alloc(tmem_holder, C::kTmemCols);
-    tmem_relinquish();
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1149,6 +1159,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   if (warp == 0) {
     // ---- producer: weight images; lanes 0 and 1 start a stage's two copies with one
     // instruction of the converged warp ----
+    if (pre > 1) first_copies(1, pre);
     for (int j = pre; j < nst; ++j) {
       const int kt = kt0 + j, stage = j % kStages;
       int ok = 1;
