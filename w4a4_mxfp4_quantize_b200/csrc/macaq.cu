@@ -1230,7 +1230,35 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
     __syncwarp();
     if (et == 0) *epi_flag = mbar_wait(&accf[0], 0, abort_flag, kWaitTimeoutNs) ? 1 : 0;
     named_bar_sync(1, 128);
-    if (*epi_flag) {
+    if (*epi_flag && !split) {
+      // Without a K split the accumulator is the whole sum: each thread holds output
+      // channel n0 + 32 q + lane for every token of the tile and stores it directly
+      // (a warp writes 64 contiguous bytes of a y row per token).
+      tc_fence_after();
+      const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      const int n = nt * kRowsTile + q * 32 + lane;
+      const float os = p.out_scale;
+      float b = 0.f;
+      if constexpr (kEpilogue) {
+        if (p.bias != nullptr && n < p.N) b = __ldg(p.bias + n);
+      }
+      pdl_wait();  // y may still be read by the previous kernel on the stream
+#pragma unroll 1
+      for (int c0 = 0; c0 < BT; c0 += 16) {
+        uint32_t r0[16];
+        tmem_ld_32x32b_x16(taddr + c0, r0);
+        tmem_wait_ld();
+        if (n < p.N) {
+#pragma unroll
+          for (int jj = 0; jj < 16; ++jj) {
+            if (c0 + jj >= rows) break;
+            float v = __uint_as_float(r0[jj]) * os;
+            if constexpr (kEpilogue) v = act_value_rt(v + b, p.act);
+            p.y[static_cast<int64_t>(m0 + c0 + jj) * p.N + n] = bf16_bits(v);
+          }
+        }
+      }
+    } else if (*epi_flag) {
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16);
       float* col = part + q * 32 + lane;
@@ -1350,7 +1378,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   if (split && !cluster_waited) cluster_wait_acquire();  // warp-uniform: the epilogue warps waited above
   if (split && threadIdx.x == 0) *epi_flag = mbar_wait(recv_bar, 0, abort_flag, kWaitTimeoutNs) ? 1 : 0;
   __syncthreads();
-  if (*epi_flag) {
+  if (*epi_flag && split) {  // (without a split the epilogue warps stored y already)
     const int t_lo = static_cast<int>(rank) * rpr, n_rows = rows_of(static_cast<int>(rank));
     const int n0 = nt * kRowsTile;
     // without a split the local partial tile is the whole sum
