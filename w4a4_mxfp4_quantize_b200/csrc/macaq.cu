@@ -8,25 +8,32 @@
 // quantised straight into shared memory (fused path) or quantised once into
 // images in an L2-resident workspace (quantise-once path).
 //
-// The MMA is swapped: operand A = 128 output channels of weights (the MMA's M
-// side), operand B = a tile of BT tokens (its N side, 16..128), so the token
-// count maps to the narrow side of tcgen05.mma and D[n][t] sits in TMEM with
-// one output channel per lane.
+// Small M (fused kernel): the MMA is swapped, operand A = 128 output channels of
+// weights (the MMA's M side), operand B = a tile of BT tokens (its N side,
+// 16..128), so the token count maps to the narrow side of tcgen05.mma and
+// D[n][t] sits in TMEM with one output channel per lane.  Large M (GEMM): A = a
+// 128-token activation tile, B = 256 output channels (two weight images), one
+// token per TMEM lane.
 //
 // Kernels
+//   calibrate_kernel      offline: channel factors D from calibration rows and W
 //   prep_weights_kernel   offline: W*D -> FWHT32 -> MX -> weight tile images
 //   quant_tiles_kernel    activation prologue over all rows once -> tile images
-//                         (dense rows, or group-padded rows for the grouped form)
-//   group_tables_kernel   grouped: validate group_list, row offsets, tile prefix
+//                         (dense rows, or group-padded rows for the grouped form;
+//                         only 32-row slabs that hold rows)
+//   group_tables_kernel   grouped: validate group_list; row offsets, tile prefix,
+//                         experts and the quantiser's slab table
 //   gemm_kernel           persistent, warp-specialised tcgen05 kind::mxf4 GEMM
-//                         over tile images; double-buffered TMEM accumulators;
-//                         epilogue staged in shared memory and written with
-//                         bulk stores; chained to the quantiser by
-//                         programmatic dependent launch
+//                         over tile images, 128 x 256 output tiles, one TMEM
+//                         accumulator drained to registers, epilogue staged in
+//                         shared memory and stored as coalesced row runs;
+//                         chained to the quantiser by programmatic dependent
+//                         launch
 //   fused_small_kernel    small M: one kernel, the activation prologue writes
 //                         the swizzled B tile straight into shared memory;
-//                         split-K across a thread-block cluster, partial sums
-//                         reduced through distributed shared memory
+//                         optional split-K across a thread-block cluster, partial
+//                         sums reduced through distributed shared memory
+//   quant_canonical_kernel, export_tiles_kernel, mx_encode_kernel: tests only
 #include <cuda_runtime.h>
 
 #include <cmath>
