@@ -48,12 +48,20 @@ L2_FLUSH_BYTES = 256 << 20
 
 
 def kernel_source_hash() -> str:
+    """Hash of the kernel sources with comments and blank lines removed, so that a
+    profile stays matched to its kernels across edits of prose only."""
     import hashlib
+    import re
     h = hashlib.sha256()
     d = os.path.join(ROOT, "w4a4_mxfp4_quantize_b200", "csrc")
     for f in sorted(os.listdir(d)):
-        with open(os.path.join(d, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(d, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"(?m)^\s*//.*$", "", text)        # whole-line comments
+        text = re.sub(r"(?m)\s+//[^\"\n]*$", "", text)   # trailing comments (not inside strings)
+        text = "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+        h.update(f.encode() + b"\0" + text.encode())
     return h.hexdigest()[:16]
 
 
