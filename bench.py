@@ -274,6 +274,21 @@ def cpu_oracle_sample(problems, budget_s: float = 12.0, rows: int = 4, prepared=
         "(activation quantisation + exact block-scaled GEMM; weights prepared beforehand)"), prepared
 
 
+def max_over_ranks(total_ms: float, dist, device) -> float:
+    """The job's time: the largest of the ranks' timed totals (every rank takes part)."""
+    if dist is None:
+        return total_ms
+    t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_step: float, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: every rank runs the same step on its own data
+    (replicas), so the job does world x the step's FLOPs in the slowest rank's time."""
+    return world * flops_step * steps / (total_ms * 1e-3) / 1e12
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return
@@ -391,12 +406,8 @@ def main():
     clocks = sampler.stop()
 
     step_ms = [a.elapsed_time(b) for a, b in step_ev]
-    total_ms = sum(step_ms)
-    if dist is not None:
-        t = torch.tensor([total_ms], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+    total_ms = max_over_ranks(sum(step_ms), dist, device)
+    value = job_tflops(world, flops_step, args.steps, total_ms)
     ms_per_step = total_ms / args.steps
 
     # The dominant kernel is the only one launched in the timed region (one fused
@@ -435,12 +446,8 @@ def main():
             if it >= args.warmup:
                 e2e_ms.append((a, b))
     stream.synchronize()
-    e2e_total = sum(a.elapsed_time(b) for a, b in e2e_ms)
-    if dist is not None:
-        t = torch.tensor([e2e_total], device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
-    e2e = {"value": world * flops_step * args.steps / (e2e_total * 1e-3) / 1e12, "unit": UNIT,
+    e2e_total = max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ms), dist, device)
+    e2e = {"value": job_tflops(world, flops_step, args.steps, e2e_total), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "mode": "eager calls, no graph"}
 
     line = {
