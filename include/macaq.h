@@ -129,7 +129,9 @@ size_t macaq_workspace_bytes(int64_t M, int64_t N, int64_t K, int64_t E);
 
 /* Dense MACAQ linear (MACAQ page, summary: channel scaling, block-32 BF16
  * Hadamard rotation, MXFP4 activation quantisation and matmul in one kernel,
- * BF16 output).
+ * BF16 output).  M <= 128 runs as that one kernel; larger M quantises every
+ * activation row once into the workspace and then runs the block-scaled GEMM
+ * (two kernels, the second launched as a programmatic dependent of the first).
  *   x_dev  bf16 [M, K] row-major;  D_dev fp32 [K];
  *   Wq_dev, Ws_dev from macaq_prepare_weights with E = 1;
  *   y_dev  bf16 [M, N] row-major (written);
