@@ -885,8 +885,10 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
     // Warp w reads TMEM lanes 32 (w % 4) .. + 31 (accumulator rows) and columns
     // 128 h .. + 127 with h = (w - 2) / 4.  The accumulator is drained into packed
     // BF16 registers first and handed back, so the next tile's MMAs overlap the
-    // write-out.  Rows go out in 64-column chunks staged in shared memory with their
-    // 16-byte pieces XOR-swizzled by the row (conflict-free writes and reads).
+    // write-out (the bias / activation instantiation drains 64 columns at a time and
+    // hands the accumulator back after the second half).  Rows go out in 64-column
+    // chunks staged in shared memory with their 16-byte pieces XOR-swizzled by the
+    // row (conflict-free writes and reads).
     const int q = warp & 3, h = (warp - 2) >> 2;
     const int et = threadIdx.x - 64;
     const float os = p.out_scale;
@@ -1002,7 +1004,9 @@ struct FusedParams {
 namespace fused {
 constexpr int kStages = 4;
 constexpr int kProWarps = 8;
-constexpr int kThreads = (6 + kProWarps) * 32;  // warp 0 producer, 1 MMA, 2-5 epilogue, 6-13 prologue
+// warp 0 producer, 1 MMA, 2-5 epilogue (warp 2 also issues the scale copies during
+// the mainloop), 6-13 prologue
+constexpr int kThreads = (6 + kProWarps) * 32;
 template <int BT>
 struct Cfg {
   static constexpr int kBBytes = BT * 128;

@@ -8,8 +8,11 @@
 //   both:        E8M0 scale = floor(log2 amax) - 2 + 127 clamped at 0
 //                (OCP MX scale_alg = 0); E2M1 code = RNE with saturation of
 //                value * 2^(127 - scale); sign bit copied from the value.
-// One thread owns one 32-element block, so the whole rotation and the block
-// amax stay in registers (no shuffles, no shared memory).
+// The quantisers give each thread one whole 32-element block (act_block: the
+// rotation and the block amax stay in its registers); the fused kernel splits a
+// block across a lane pair (act_half_block(s): 16 elements per lane, the last
+// butterfly stage and the amax through one exchange each).  Both compute the
+// same values in the same order.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
