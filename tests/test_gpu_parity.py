@@ -485,3 +485,32 @@ def test_dependent_calls_on_one_stream(M):
     torch.cuda.synchronize()
     assert np.array_equal(y_to_bits(y1), y_to_bits(r1))
     assert np.array_equal(y_to_bits(a), y_to_bits(r3))
+
+
+@pytest.mark.parametrize("kind", ["dense", "grouped"])
+def test_padding_rows_never_reach_the_output(kind):
+    # The quantiser writes only real rows of the activation images; padding rows
+    # keep whatever the workspace held.  Fill it with 0xFF (E8M0 255 = NaN scales,
+    # E2M1 -6 codes) first: every output must stay finite and match the oracle.
+    if kind == "dense":
+        p = synth.dense(300, 512, 144, seed=41)       # ragged last row tile (44 rows)
+        need = mq.workspace_bytes(p.M, p.N, p.K)
+    else:
+        p = synth.grouped(300, 6, 512, 144, seed=42, dist="zipf")
+        need = mq.workspace_bytes(p.M, p.N, p.K, p.E)
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device="cuda")
+    x = x_to_dev(p.x)
+    Wq, Ws = mq.prepare_weights(f32_dev(p.W), f32_dev(p.D))
+    if kind == "dense":
+        y = mq.dense_mm(x, f32_dev(p.D[0]), Wq, Ws, p.N, ws=ws)
+        qa, sa = oracle.quantize_act(p.x, p.D[0])
+        qw, sw = oracle.quantize_weights(p.W[0], p.D[0])
+        ref = oracle.gemm(qa, sa, qw, sw)
+    else:
+        gl = torch.from_numpy(p.group_list).cuda()
+        y = mq.grouped_mm(x, f32_dev(p.D), Wq, Ws, gl, p.group_list_type, p.N, ws=ws)
+        st, ref = oracle.grouped_mm(p.x, p.D, p.W, p.group_list, p.group_list_type)
+        assert st == oracle.OK
+    torch.cuda.synchronize()
+    assert bool(torch.isfinite(y.float()).all())
+    compare(y_to_bits(y), ref, f"{kind} with a poisoned workspace")
