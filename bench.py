@@ -178,6 +178,19 @@ class Prepared:
             mq.grouped_mm(self.x, self.D, self.Wq, self.Ws, self.gl, self.p.group_list_type, self.p.N,
                           out=self.y, stream=stream, ws=self.ws)
 
+    def run_epilogue(self, mq, stream=None):
+        """The same call with an fp32 bias and GELU_TANH (npu_grouped_matmul's bias and act_type)."""
+        if getattr(self, "bias", None) is None:
+            rows = 1 if self.gl is None else self.p.E
+            b = np.random.default_rng(3).standard_normal((rows, self.p.N)).astype(np.float32) * 0.5
+            self.bias = f32(b[0] if self.gl is None else b, self.y.device)
+        if self.gl is None:
+            mq.dense_mm(self.x, self.D, self.Wq, self.Ws, self.p.N, out=self.y, stream=stream, ws=self.ws,
+                        bias=self.bias, act_type=mq.ACT_GELU_TANH)
+        else:
+            mq.grouped_mm(self.x, self.D, self.Wq, self.Ws, self.gl, self.p.group_list_type, self.p.N,
+                          out=self.y, stream=stream, ws=self.ws, bias=self.bias, act_type=mq.ACT_GELU_TANH)
+
     def run_unfused(self, mq, stream=None):
         mq.unfused_dense_mm(self.x, self.D, self.Wq, self.Ws, self.p.N, out=self.y, stream=stream,
                             ws=self.ws_unfused)
@@ -471,6 +484,7 @@ def main():
                                 "seconds": el}
         if not args.no_table:
             line["per_workload"] = workload_table(mq, device, stream, flush, hbm_gbs, args.table_reps)
+            line["calibration"] = calibration_table(mq, device, stream, flush, hbm_gbs, args.table_reps)
         print(json.dumps(line), flush=True)
 
     for pp in problems:
@@ -519,6 +533,9 @@ def workload_table(mq, device, stream, flush, hbm_gbs, reps):
                 gu = capture(lambda: pp.run_unfused(mq), stream)
                 un, _ = time_graph(gu, flush, stream, reps)
                 del gu
+            ge = capture(lambda: pp.run_epilogue(mq), stream)
+            epi_us, _ = time_graph(ge, flush, stream, reps)
+            del ge
             # accuracy against the unquantised layer on sampled rows, then the plain MXFP4 baseline
             rows_s = np.unique(np.random.default_rng(cfg).integers(0, p.M, min(p.M, 16)))
             pp.run(mq, stream)
@@ -537,11 +554,29 @@ def workload_table(mq, device, stream, flush, hbm_gbs, reps):
                 "tflops": p.flops() / (us * 1e-6) / 1e12, "gbs": p.algorithmic_bytes() / (us * 1e-6) / 1e9,
                 "roofline_us": t_roof * 1e6, "frac_roofline": t_roof / (us * 1e-6), "unfused_us": un,
                 "plain_us": plain_us, "plain_over_macaq_time": plain_us / us,
+                "bias_gelu_tanh_us": epi_us,
                 "nmse": nmse, "nmse_plain": nmse_plain, "nmse_plain_over_macaq": nmse_plain / nmse if nmse else None,
             })
             del g, pp
             torch.cuda.empty_cache()
     return rows
+
+
+def calibration_table(mq, device, stream, flush, hbm_gbs, reps):
+    """Offline D calibration (macaq_calibrate_d) on 1,024 calibration tokens (the
+    MACAQ page's pilot size) for each Qwen3-0.6B-shaped projection: us per call
+    (trimmed mean, cold L2) and its bytes (x, W, D) against the HBM bandwidth."""
+    out = []
+    for (K, N) in synth.QWEN_PAIRS:
+        p = synth.dense(1024, K, N, seed=11)
+        x, W = x_dev(p.x, device), f32(p.W, device)
+        g = capture(lambda: mq.calibrate_d(x, W, stream=stream), stream)
+        us, _ = time_graph(g, flush, stream, reps)
+        nbytes = 1024 * K * 2 + N * K * 4 + K * 4
+        out.append({"name": f"calibrate T=1024 K={K} N={N}", "us": us, "gbs": nbytes / (us * 1e-6) / 1e9,
+                    "frac_hbm": nbytes / (us * 1e-6) / 1e9 / hbm_gbs})
+        del g, x, W
+    return out
 
 
 if __name__ == "__main__":

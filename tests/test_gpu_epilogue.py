@@ -3,7 +3,9 @@ act_type) against the CPU oracle, through the C ABI's _ex entry points.
 
 The oracle adds the bias to 2^-5 times the exact block-scaled sum and applies
 the activation in binary64, then rounds once to BF16; the kernels do the same
-in FP32.  Outputs are judged by the tolerance in tests/helpers.py.
+in FP32, the gated activations through a hardware half-precision tanh.  Outputs
+are judged by the tolerance in tests/helpers.py, and the gated activations also
+by their own error bound.
 """
 import numpy as np
 import pytest
@@ -12,7 +14,7 @@ import torch
 import oracle
 import synth
 import w4a4_mxfp4_quantize_b200 as mq
-from helpers import compare, f32_dev, x_to_dev, y_to_bits
+from helpers import bf16_ulp, compare, f32_dev, x_to_dev, y_to_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -111,3 +113,31 @@ def test_act_type_3_is_refused_without_launching():
     assert e.value.status == -13
     torch.cuda.synchronize()
     assert bool((y == 7.0).all())
+
+
+@pytest.mark.parametrize("M", [64, 1000])
+@pytest.mark.parametrize("act", [mq.ACT_GELU_TANH, mq.ACT_FAST_GELU, mq.ACT_SILU])
+def test_gated_activation_error_bound(M, act):
+    # The gated forms are v sigmoid(a) = h + h tanh(a / 2), h = v / 2, with a hardware
+    # half-precision tanh: the argument rounded to FP16 (relative 2^-11, times
+    # tanh' <= 1 and |u| tanh'(u) <= 0.45), the approximation (~2^-11) and the FP16
+    # result (2^-12 near 1) keep |tanh error| below ~1e-3, so |y - y_exact| <= 5e-4 |v|
+    # before the BF16 rounding of each side (one ulp between them).  v is the
+    # oracle's pre-activation value (bias included).
+    K, N = 512, 400
+    p = synth.dense(M, K, N, seed=40 + act)
+    bias = _bias(N, seed=41)
+    x, D = x_to_dev(p.x), f32_dev(p.D[0])
+    Wq, Ws = mq.prepare_weights(f32_dev(p.W), f32_dev(p.D))
+    y = y_to_bits(mq.dense_mm(x, D, Wq, Ws, N, bias=f32_dev(bias), act_type=act))
+    qa, sa = oracle.quantize_act(p.x, p.D[0])
+    qw, sw = oracle.quantize_weights(p.W[0], p.D[0])
+    v = synth.bf16_bits_to_f32(oracle.gemm_ex(qa, sa, qw, sw, bias, mq.ACT_NONE)).astype(np.float64)
+    ref = synth.bf16_bits_to_f32(oracle.gemm_ex(qa, sa, qw, sw, bias, act)).astype(np.float64)
+    got = synth.bf16_bits_to_f32(y).astype(np.float64)
+    err = np.abs(got - ref)
+    bound = 6e-4 * np.abs(v) + bf16_ulp(np.maximum(np.abs(got), np.abs(ref)))
+    bad = np.flatnonzero(err > bound)
+    assert bad.size == 0, (act, bad[:5], v.ravel()[bad[:5]], got.ravel()[bad[:5]], ref.ravel()[bad[:5]])
+    # a large share agrees bit for bit: the error is a fraction of one BF16 ulp
+    assert np.mean(got == ref) > 0.3

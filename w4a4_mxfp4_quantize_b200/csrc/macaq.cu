@@ -66,19 +66,56 @@ __device__ __forceinline__ uint16_t bf16_bits(float v) {
 }
 
 // Output activation of npu_grouped_matmul's act_type (parameter act_type: 0 none,
-// 1 RELU, 2 GELU_TANH, 4 FAST_GELU, 5 SILU), in FP32 with CUDA's expf / tanhf.
-// FAST_GELU, which the page names without defining, is v * sigmoid(1.702 v).
+// 1 RELU, 2 GELU_TANH, 4 FAST_GELU, 5 SILU), in FP32.  The three gated forms are
+// v * sigmoid(a) with a = 2u, u = sqrt(2/pi) (v + 0.044715 v^3) for GELU_TANH
+// (0.5 (1 + tanh u) = sigmoid(2u)), a = 1.702 v for FAST_GELU (named on the page
+// without a formula), a = v for SILU, and are evaluated as
+//   v sigmoid(a) = h + h tanh(a / 2),  h = v / 2,
+// with tanh taken in half precision by the hardware (tanh_h: the argument rounded
+// to FP16, relative error of the approximation about 2^-11) and no division.
+// The error in y is at most about 5e-4 |v|, far below the MXFP4 quantisation
+// noise of v.  One special-function operation per two outputs keeps the epilogue
+// under the tile's MMA time: an exponential plus a reciprocal per output (two
+// such operations at 16 per clock per SM) took twice as long as the tensor core
+// needs for a 128 x 256 tile at K = 1024.  act_value (one output) and act_pair
+// (two, in packed FP32 pair instructions) take the same steps and give the same
+// bits.
+constexpr float kGeluC0 = 0.7978845608028654f;    // sqrt(2/pi)
+constexpr float kGeluC1 = 0.035677408136300125f;  // sqrt(2/pi) x 0.044715
+constexpr float kFastGeluHalf = 0.851f;           // 1.702 / 2
 template <int ACT>
 __device__ __forceinline__ float act_value(float v) {
   if constexpr (ACT == 1) {
     return fmaxf(v, 0.f);
   } else if constexpr (ACT == 2) {
-    const float u = 0.7978845608028654f * (v + 0.044715f * v * v * v);  // sqrt(2/pi) (v + 0.044715 v^3)
-    return 0.5f * v * (1.f + tanhf(u));
+    const float u = v * fmaf(v * v, kGeluC1, kGeluC0);
+    const float h = 0.5f * v;
+    return fmaf(h, tanh_h(u), h);
   } else if constexpr (ACT == 4) {
-    return v / (1.f + expf(-1.702f * v));
+    const float h = 0.5f * v;
+    return fmaf(h, tanh_h(kFastGeluHalf * v), h);
   } else if constexpr (ACT == 5) {
-    return v / (1.f + expf(-v));
+    const float h = 0.5f * v;
+    return fmaf(h, tanh_h(h), h);
+  } else {
+    return v;
+  }
+}
+template <int ACT>
+__device__ __forceinline__ float2 act_pair(float2 v) {
+  const float2 half = make_float2(0.5f, 0.5f);
+  if constexpr (ACT == 1) {
+    return make_float2(fmaxf(v.x, 0.f), fmaxf(v.y, 0.f));
+  } else if constexpr (ACT == 2) {
+    const float2 u = fmul2(v, ffma2(fmul2(v, v), make_float2(kGeluC1, kGeluC1), make_float2(kGeluC0, kGeluC0)));
+    const float2 h = fmul2(v, half);
+    return ffma2(h, tanh_h2(u), h);
+  } else if constexpr (ACT == 4) {
+    const float2 h = fmul2(v, half);
+    return ffma2(h, tanh_h2(fmul2(v, make_float2(kFastGeluHalf, kFastGeluHalf))), h);
+  } else if constexpr (ACT == 5) {
+    const float2 h = fmul2(v, half);
+    return ffma2(h, tanh_h2(h), h);
   } else {
     return v;
   }
@@ -338,8 +375,15 @@ __device__ __forceinline__ int find_group(const int* gtp, int E, int pm) {
 // 1e2) per expert and input channel, a = max |x[:, k]| over the expert's
 // calibration rows, w = max |W[:, k]| over its weight rows, in binary64 and
 // rounded once to fp32 (w = 0 < a gives 1e2, a = w = 0 gives 1, an expert with
-// no rows gives 1).  One CTA per (256 channels, expert): 1024 threads = 256
-// channels x 4 row lanes, the lanes' maxima combined in shared memory.
+// no rows gives 1).  A cluster of kCalibCluster CTAs per (64 channels, expert)
+// splits the weight rows and the calibration rows; in each CTA 1024 threads =
+// 64 channels x 16 row lanes, whose maxima are combined in shared memory; rank 0
+// then combines the CTAs' maxima through distributed shared memory.  64 channels
+// keep each warp's loads on whole 128-byte (W) and 64-byte (x) row segments
+// while giving K / 8 CTAs per expert (128 for K = 1024), enough to cover the SMs.
+constexpr int kCalibCluster = 8;
+constexpr int kCalibCols = 64;
+constexpr int kCalibLanes = 1024 / kCalibCols;
 struct CalibParams {
   const uint16_t* x;  // bf16 [T, K]
   const float* W;     // [E, N, K]
@@ -351,15 +395,39 @@ struct CalibParams {
 };
 
 __global__ void __launch_bounds__(1024) calibrate_kernel(const __grid_constant__ CalibParams p) {
-  __shared__ float sa[4][256], sw[4][256];
-  const int c = threadIdx.x & 255, lanes = threadIdx.x >> 8;
+  __shared__ float sa[kCalibLanes][kCalibCols], sw[kCalibLanes][kCalibCols];
+  const int c = threadIdx.x % kCalibCols, lanes = threadIdx.x / kCalibCols;
+  const int rank = static_cast<int>(cluster_ctarank());
   const int e = blockIdx.y;
-  const int64_t k = static_cast<int64_t>(blockIdx.x) * 256 + c;
+  const int64_t k = static_cast<int64_t>(blockIdx.x / kCalibCluster) * kCalibCols + c;
+  // this thread's rows: lane + kCalibLanes rank, then every kCalibLanes x kCalibCluster
+  const int first = lanes + kCalibLanes * rank, stride = kCalibLanes * kCalibCluster;
   float w = 0.f, a = 0.f;  // maxima of magnitudes: exact in any order
-  for (int n = lanes; n < p.N; n += 4) w = fmaxf(w, fabsf(__ldg(p.W + (static_cast<int64_t>(e) * p.N + n) * p.K + k)));
+  {
+    // eight independent loads in flight per thread (one at a time would wait a
+    // full memory latency per row)
+    float wm[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const float* wp = p.W + static_cast<int64_t>(e) * p.N * p.K + k;
+    int n = first;
+    for (; n + 7 * stride < p.N; n += 8 * stride) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) wm[u] = fmaxf(wm[u], fabsf(__ldg(wp + static_cast<int64_t>(n + u * stride) * p.K)));
+    }
+    for (; n < p.N; n += stride) wm[0] = fmaxf(wm[0], fabsf(__ldg(wp + static_cast<int64_t>(n) * p.K)));
+#pragma unroll
+    for (int u = 0; u < 8; ++u) w = fmaxf(w, wm[u]);
+  }
   int64_t rows = 0;
   auto scan = [&](int64_t r0, int64_t r1) {
-    for (int64_t r = r0 + lanes; r < r1; r += 4) a = fmaxf(a, fabsf(bf16lo(__ldg(p.x + r * p.K + k))));
+    float am[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int64_t r = r0 + first;
+    for (; r + 7 * stride < r1; r += 8 * stride) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) am[u] = fmaxf(am[u], fabsf(bf16lo(__ldg(p.x + (r + u * stride) * p.K + k))));
+    }
+    for (; r < r1; r += stride) am[0] = fmaxf(am[0], fabsf(bf16lo(__ldg(p.x + r * p.K + k))));
+#pragma unroll
+    for (int u = 0; u < 8; ++u) a = fmaxf(a, am[u]);
   };
   if (p.gl == nullptr) {
     scan(0, p.T);
@@ -385,9 +453,20 @@ __global__ void __launch_bounds__(1024) calibrate_kernel(const __grid_constant__
   sa[lanes][c] = a;
   sw[lanes][c] = w;
   __syncthreads();
-  if (lanes == 0) {
-    a = fmaxf(fmaxf(sa[0][c], sa[1][c]), fmaxf(sa[2][c], sa[3][c]));
-    w = fmaxf(fmaxf(sw[0][c], sw[1][c]), fmaxf(sw[2][c], sw[3][c]));
+  if (lanes == 0) {  // this CTA's maxima into row 0
+    for (int l = 1; l < kCalibLanes; ++l) {
+      sa[0][c] = fmaxf(sa[0][c], sa[l][c]);
+      sw[0][c] = fmaxf(sw[0][c], sw[l][c]);
+    }
+  }
+  cluster_sync_all();  // every CTA's maxima are in its shared memory
+  if (rank == 0 && lanes == 0) {
+    a = 0.f;
+    w = 0.f;
+    for (int o = 0; o < kCalibCluster; ++o) {
+      a = fmaxf(a, ld_dsmem_f32(mapa_shared(smem_u32(&sa[0][c]), static_cast<uint32_t>(o))));
+      w = fmaxf(w, ld_dsmem_f32(mapa_shared(smem_u32(&sw[0][c]), static_cast<uint32_t>(o))));
+    }
     double d;
     if (rows == 0 || (a == 0.f && w == 0.f)) d = 1.0;
     else if (w == 0.f) d = 1e2;
@@ -395,6 +474,7 @@ __global__ void __launch_bounds__(1024) calibrate_kernel(const __grid_constant__
     d = fmin(fmax(d, 1e-2), 1e2);
     p.D[static_cast<int64_t>(e) * p.K + k] = static_cast<float>(d);
   }
+  cluster_sync_all();  // no CTA leaves while rank 0 may still read its shared memory
 }
 
 // ============================================================================
@@ -554,27 +634,27 @@ struct GemmParams {
   int act;                // act_type: 0 none, 1 RELU, 2 GELU_TANH, 4 FAST_GELU, 5 SILU
 };
 
-// Epilogue drain of 64 accumulator columns of one thread's row of the tile:
-// v = acc * out_scale (+ bias[n]), then the activation, packed to BF16 pairs.
-// Columns n >= N (the zero rows of a ragged weight tile) take no bias.
+// Epilogue drain of the 128 accumulator columns of one thread's row of its half
+// tile: v = acc * out_scale (+ bias[n]), then the activation, packed to BF16
+// pairs.  Columns n >= N (the zero rows of a ragged weight tile) take no bias.
 template <int ACT>
-__device__ __forceinline__ void drain64(uint32_t taddr, float os, const float* brow, int ncol0, int N,
-                                        uint32_t (&pk)[32]) {
+__device__ __forceinline__ void drain128(uint32_t taddr, float os, const float* brow, int ncol0, int N,
+                                         uint32_t (&pk)[64]) {
+  const int nb = brow != nullptr ? N - ncol0 : 0;  // leading columns that take a bias (a multiple of 16)
+  const float2 os2 = make_float2(os, os);
 #pragma unroll
-  for (int c0 = 0; c0 < 64; c0 += 16) {
+  for (int c0 = 0; c0 < 128; c0 += 16) {
     uint32_t r[16];
     tmem_ld_32x32b_x16(taddr + c0, r);
     tmem_wait_ld();
+    const bool inb = c0 + 16 <= nb;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      float v0 = __uint_as_float(r[2 * e]) * os, v1 = __uint_as_float(r[2 * e + 1]) * os;
-      const int n = ncol0 + c0 + 2 * e;
-      if (brow != nullptr && n < N) {
-        const float2 b = __ldg(reinterpret_cast<const float2*>(brow + n));  // warp-uniform: a broadcast
-        v0 += b.x;
-        v1 += b.y;
-      }
-      pk[c0 / 2 + e] = pack_bf16x2(act_value<ACT>(v0), act_value<ACT>(v1));
+      float2 b = make_float2(0.f, 0.f);
+      if (inb) b = __ldg(reinterpret_cast<const float2*>(brow + ncol0 + c0 + 2 * e));  // warp-uniform: a broadcast
+      const float2 v = ffma2(make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), os2, b);
+      const float2 y = act_pair<ACT>(v);
+      pk[c0 / 2 + e] = pack_bf16x2(y.x, y.y);
     }
   }
 }
@@ -885,8 +965,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
     // Warp w reads TMEM lanes 32 (w % 4) .. + 31 (accumulator rows) and columns
     // 128 h .. + 127 with h = (w - 2) / 4.  The accumulator is drained into packed
     // BF16 registers first and handed back, so the next tile's MMAs overlap the
-    // write-out (the bias / activation instantiation drains 64 columns at a time and
-    // hands the accumulator back after the second half).  Rows go out in 64-column
+    // write-out (the bias / activation instantiation applies them during the drain).  Rows go out in 64-column
     // chunks staged in shared memory with their 16-byte pieces XOR-swizzled by the
     // row (conflict-free writes and reads).
     const int q = warp & 3, h = (warp - 2) >> 2;
@@ -945,33 +1024,27 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
           if (ch < 3) named_bar_sync(1, 256);  // read out before the next chunk overwrites it
         }
       } else {
-        // bias and/or activation: 64 columns at a time (fewer live registers); the
-        // accumulator is released after the second half has been read
+        // bias and/or activation applied while the row is drained; as above, the
+        // accumulator is handed back before the chunks go out
         const float* brow = p.bias != nullptr ? p.bias + static_cast<int64_t>(t.g) * p.N : nullptr;
-#pragma unroll 1
-        for (int part = 0; part < 2; ++part) {
-          uint32_t pk[32];
-          const uint32_t ta = taddr + part * 64;
-          const int nc = t.nt * kRowsTile + h * 128 + part * 64;
-          switch (p.act) {
-            case 1: drain64<1>(ta, os, brow, nc, p.N, pk); break;
-            case 2: drain64<2>(ta, os, brow, nc, p.N, pk); break;
-            case 4: drain64<4>(ta, os, brow, nc, p.N, pk); break;
-            case 5: drain64<5>(ta, os, brow, nc, p.N, pk); break;
-            default: drain64<0>(ta, os, brow, nc, p.N, pk);
-          }
-          if (part == 1) {
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acce);
-          }
+        const int nc = t.nt * kRowsTile + h * 128;
+        uint32_t pk[64];
+        switch (p.act) {
+          case 1: drain128<1>(taddr, os, brow, nc, p.N, pk); break;
+          case 2: drain128<2>(taddr, os, brow, nc, p.N, pk); break;
+          case 4: drain128<4>(taddr, os, brow, nc, p.N, pk); break;
+          case 5: drain128<5>(taddr, os, brow, nc, p.N, pk); break;
+          default: drain128<0>(taddr, os, brow, nc, p.N, pk);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acce);
 #pragma unroll
-          for (int hh = 0; hh < 2; ++hh) {  // chunk 2 hh + part comes from half hh
-            if (hh == h) stage_chunk(pk);
-            named_bar_sync(1, 256);
-            store_chunk(2 * hh + part);
-            if (part == 0 || hh == 0) named_bar_sync(1, 256);
-          }
+        for (int ch = 0; ch < 4; ++ch) {
+          if ((ch >> 1) == h) stage_chunk(pk + (ch & 1) * 32);
+          named_bar_sync(1, 256);
+          store_chunk(ch);
+          if (ch < 3) named_bar_sync(1, 256);
         }
       }
     }
@@ -2017,8 +2090,10 @@ int macaq_calibrate_d(const uint16_t* x, int64_t T, const float* W, int64_t E, i
   CalibParams p{};
   p.x = x; p.W = W; p.gl = group_list; p.type = group_list_type;
   p.E = static_cast<int>(E); p.N = static_cast<int>(N); p.K = static_cast<int>(K); p.T = T; p.D = D;
-  calibrate_kernel<<<dim3(static_cast<unsigned>(K / 256), static_cast<unsigned>(E)), 1024, 0, s>>>(p);
-  return cudaPeekAtLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
+  const cudaError_t e = launch_ex(calibrate_kernel,
+                                  dim3(static_cast<unsigned>(K / kCalibCols * kCalibCluster), static_cast<unsigned>(E)),
+                                  dim3(1024), 0, s, false, kCalibCluster, p);
+  return e == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
 int macaq_dense_mm_plain(const uint16_t* x, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M, int64_t N,

@@ -259,6 +259,65 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
 }  // namespace macaq
 
 namespace macaq {
+// Packed FP32 pair arithmetic (sm_100 .f32x2 forms): one instruction for two
+// lanes, each lane rounded exactly as the scalar fma / mul.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{.reg .b64 a, b, c, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %5};\n\t"
+      "mov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\t"
+      "mov.b64 {%0, %1}, d;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{.reg .b64 a, b, d;\n\t"
+      "mov.b64 a, {%2, %3};\n\t"
+      "mov.b64 b, {%4, %5};\n\t"
+      "mul.rn.f32x2 d, a, b;\n\t"
+      "mov.b64 {%0, %1}, d;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// Hardware tanh in half precision: the FP32 argument rounded to FP16 (RN), one
+// special-function-unit operation (tanh.approx.f16), the result widened exactly
+// to FP32.  The pair form does two lanes in one operation (tanh.approx.f16x2)
+// and gives the same bits lane by lane.
+__device__ __forceinline__ float tanh_h(float x) {
+  float y;
+  asm("{.reg .b16 h;\n\t"
+      "cvt.rn.f16.f32 h, %1;\n\t"
+      "tanh.approx.f16 h, h;\n\t"
+      "cvt.f32.f16 %0, h;}"
+      : "=f"(y)
+      : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float2 tanh_h2(float2 x) {
+  float2 y;
+  asm("{.reg .b32 p;\n\t"
+      ".reg .b16 lo, hi;\n\t"
+      "cvt.rn.f16x2.f32 p, %3, %2;\n\t"  // upper half from the first source
+      "tanh.approx.f16x2 p, p;\n\t"
+      "mov.b32 {lo, hi}, p;\n\t"
+      "cvt.f32.f16 %0, lo;\n\t"
+      "cvt.f32.f16 %1, hi;}"
+      : "=f"(y.x), "=f"(y.y)
+      : "f"(x.x), "f"(x.y));
+  return y;
+}
+
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
 __device__ __forceinline__ void st_dsmem_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
