@@ -174,6 +174,11 @@ int macaq_grouped_mm(const uint16_t *x_dev, const float *D_dev, const uint8_t *W
  *     page names it without a formula), 5 SILU (v * sigmoid(v)).  3 is not
  *     supported on the page and, like any other value, returns
  *     MACAQ_ERR_ACT_TYPE without launching.
+ *   The gated forms (2, 4, 5) are evaluated as h + h tanh(a / 2), h = v / 2,
+ *   a = 2 sqrt(2/pi) (v + 0.044715 v^3), 1.702 v or v (the same functions),
+ *   with a hardware half-precision tanh: before the rounding to BF16 the
+ *   result is within about 5e-4 |v| of the exact activation of v.  RELU and
+ *   act_type 0 add no error.
  * All other arguments, the workspace and the error behaviour are those of
  * macaq_dense_mm / macaq_grouped_mm; with bias NULL and act_type 0 the result
  * is theirs. */
