@@ -14,9 +14,12 @@ no exchange), so scaling is weak.
 
 Also reported: e2e (the same calls with the activations copied from pinned
 host memory and the outputs copied back inside the timed interval), the
-roofline of the dominant kernel, the per-workload table of all five
-workloads (us/call, TFLOPS, fraction of roofline, unfused ablation), the
-clocks seen during the timed region, and the CPU oracle on a bounded sample.
+roofline of the dominant kernel, the clocks seen during the timed region, and,
+on one GPU, the per-workload table of all five workloads (us/call, TFLOPS,
+fraction of roofline, ALU bound of the activation prologue, unfused ablation,
+plain MXFP4, bias + GELU_TANH, eager calls allocating y), the D calibration
+times, and the CPU oracle on a bounded sample (all cores, one thread, and a
+decoded binary64 GEMM).
 
 `--impl reference` times the CPU oracle (the reference arm) on the same
 workload and metric.
@@ -178,6 +181,14 @@ class Prepared:
             mq.grouped_mm(self.x, self.D, self.Wq, self.Ws, self.gl, self.p.group_list_type, self.p.N,
                           out=self.y, stream=stream, ws=self.ws)
 
+    def run_alloc(self, mq, stream=None):
+        """The call as made without a preallocated output: the binding allocates y
+        (torch.empty through the caching allocator) on every call."""
+        if self.gl is None:
+            return mq.dense_mm(self.x, self.D, self.Wq, self.Ws, self.p.N, stream=stream)
+        return mq.grouped_mm(self.x, self.D, self.Wq, self.Ws, self.gl, self.p.group_list_type, self.p.N,
+                             stream=stream)
+
     def run_epilogue(self, mq, stream=None):
         """The same call with an fp32 bias and GELU_TANH (npu_grouped_matmul's bias and act_type)."""
         if getattr(self, "bias", None) is None:
@@ -263,28 +274,62 @@ def time_graph(g, flush, stream, reps: int, warm: int = 3, cold: bool = True):
 # ---------------------------------------------------------------------------
 # reference arm: the CPU oracle
 # ---------------------------------------------------------------------------
-def cpu_oracle_sample(problems, budget_s: float = 12.0, rows: int = 4, prepared=None):
+def cpu_oracle_sample(problems, budget_s: float = 12.0, rows: int = 4, prepared=None, nthreads: int = 0):
     """The oracle's hot path (activation quantisation + exact GEMM) on `rows`
     rows of every problem, weights prepared beforehand (offline, untimed, as
-    on the GPU); returns (TFLOPS, seconds, threads, description, prepared)."""
+    on the GPU), on `nthreads` threads (0: all host cores); returns (TFLOPS,
+    seconds, threads, description, prepared)."""
     import oracle
     if prepared is None:
         prepared = [oracle.quantize_weights(p.W[0], p.D[0]) for p in problems]
+    threads = nthreads if nthreads > 0 else oracle.num_threads()
     t0 = time.perf_counter()
     flops = 0.0
     n = 0
     while True:
         for p, (qw, sw) in zip(problems, prepared):
-            qa, sa = oracle.quantize_act(p.x[:rows], p.D[0])
-            oracle.gemm(qa, sa, qw, sw)
+            qa, sa = oracle.quantize_act(p.x[:rows], p.D[0], threads)
+            oracle.gemm(qa, sa, qw, sw, threads)
             flops += 2.0 * rows * p.N * p.K
         n += 1
         el = time.perf_counter() - t0
         if el >= budget_s or n >= 1000:
             break
-    return flops / el / 1e12, el, oracle.num_threads(), (
+    return flops / el / 1e12, el, threads, (
         f"{rows} of {problems[0].M} rows of each of the {len(problems)} projections, {n} passes "
         "(activation quantisation + exact block-scaled GEMM; weights prepared beforehand)"), prepared
+
+
+def cpu_oracle_detail(problems, prepared, cores: int, budget_s: float = 4.0) -> dict:
+    """Two more host-side figures beside the all-core oracle: the same hot path
+    on one thread, and a dequantised binary64 GEMM (activation quantisation,
+    both operands decoded to their values, one BLAS matmul, the 2^-5 scale;
+    weights decoded beforehand) on 4 rows of every problem: the exact GEMM is a
+    correctness tool, the decoded one the speed a plain CPU implementation of
+    the same arithmetic reaches."""
+    import oracle
+    v1, el1, _, _, _ = cpu_oracle_sample(problems, budget_s=budget_s, rows=1, prepared=prepared, nthreads=1)
+    p0 = problems[0]
+    oracle.quantize_act(p0.x[:1], p0.D[0], cores)  # back to every core for later oracle calls
+    wdec = [oracle.dequantize(qw, sw) for (qw, sw) in prepared]
+    rows = 4
+    t0 = time.perf_counter()
+    flops, n = 0.0, 0
+    while True:
+        for p, w in zip(problems, wdec):
+            qa, sa = oracle.quantize_act(p.x[:rows], p.D[0], cores)
+            _ = (oracle.dequantize(qa, sa) @ w.T) * 2.0 ** -5
+            flops += 2.0 * rows * p.N * p.K
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or n >= 1000:
+            break
+    return {
+        "single_thread": {"value": v1, "unit": UNIT, "cores": 1, "seconds": el1,
+                          "sample": "1 row of each projection, exact GEMM"},
+        "dequant_f64_gemm": {"value": flops / el / 1e12, "unit": UNIT, "cores": cores, "seconds": el,
+                             "sample": f"{rows} rows of each projection, {n} passes, decoded operands, BLAS matmul"},
+    }
 
 
 def max_over_ranks(total_ms: float, dist, device) -> float:
@@ -478,13 +523,19 @@ def main():
     }
 
     if rank == 0:
-        # CPU oracle on the host cores (bounded sample)
-        v, el, cores, sample, _ = cpu_oracle_sample([pp.p for pp in problems], budget_s=12.0, rows=4)
-        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
-                                "seconds": el}
-        if not args.no_table:
-            line["per_workload"] = workload_table(mq, device, stream, flush, hbm_gbs, args.table_reps)
-            line["calibration"] = calibration_table(mq, device, stream, flush, hbm_gbs, args.table_reps)
+        if world == 1:
+            # CPU oracle on the host cores (bounded sample), and the per-workload tables:
+            # one GPU only (at N > 1 the other ranks would wait for them at the barrier)
+            v, el, cores, sample, prepared = cpu_oracle_sample([pp.p for pp in problems], budget_s=12.0, rows=4)
+            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample,
+                                    "seconds": el}
+            try:  # supplementary host figures: their failure must not cost the line
+                line["cpu_baseline"].update(cpu_oracle_detail([pp.p for pp in problems], prepared, cores))
+            except Exception as e:  # noqa: BLE001
+                line["cpu_baseline"]["detail_error"] = f"{type(e).__name__}: {e}"[:200]
+            if not args.no_table:
+                line["per_workload"] = workload_table(mq, device, stream, flush, hbm_gbs, args.table_reps)
+                line["calibration"] = calibration_table(mq, device, stream, flush, hbm_gbs, args.table_reps)
         print(json.dumps(line), flush=True)
 
     for pp in problems:
@@ -515,12 +566,47 @@ def run_only(args):
         del pp
 
 
+# Lane operations per activation element of the quantise-once prologue (scale by
+# 1/D, Hadamard butterfly, block maximum, E8M0 and E2M1 encoding, packing, loads
+# and stores): ncu counted 2,224,128 warp instructions for quant_tiles_kernel at
+# M = 4096, K = 1024, i.e. x 32 lanes / (4096 x 1024) elements.
+QUANT_LANE_OPS_PER_ELEMENT = 2224128 * 32 / (4096 * 1024)
+SM_MAX_MHZ = 1965.0  # B200 clocks.max.sm
+
+
+def alu_bound_us(rows: int, K: int, sms: int, mhz: float = SM_MAX_MHZ) -> float:
+    """Time the activation prologue needs at full issue rate: rows x K elements x
+    lane operations each / (SMs x 128 lanes x clock)."""
+    return rows * K * QUANT_LANE_OPS_PER_ELEMENT / (sms * 128 * mhz * 1e6) * 1e6
+
+
+def time_eager(fn, stream, calls: int = 20, trials: int = 15, warm: int = 20) -> float:
+    """Median us per call over `trials` blocks of `calls` eager calls (host launch
+    included, L2 not flushed), CUDA events on `stream`."""
+    out = []
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            fn()
+        for _ in range(trials):
+            t0 = torch.cuda.Event(enable_timing=True)
+            t1 = torch.cuda.Event(enable_timing=True)
+            t0.record(stream)
+            for _ in range(calls):
+                fn()
+            t1.record(stream)
+            t1.synchronize()
+            out.append(t0.elapsed_time(t1) * 1e3 / calls)
+    return statistics.median(out)
+
+
 def workload_table(mq, device, stream, flush, hbm_gbs, reps):
     """us/call (trimmed mean, cold L2), TFLOPS and roofline fraction for every
     problem of the five workloads, fused and unfused (CUDA graph per call), the
     plain MXFP4 baseline's time, and both paths' error against the unquantised
-    layer on sampled rows."""
+    layer on sampled rows; also eager calls that allocate y on every call, and
+    the ALU bound of the activation prologue."""
     rows = []
+    sms = torch.cuda.get_device_properties(device).multi_processor_count
     for cfg in range(5):
         for p in synth.config(cfg):
             pp = Prepared(p, device, mq)
@@ -533,6 +619,11 @@ def workload_table(mq, device, stream, flush, hbm_gbs, reps):
                 gu = capture(lambda: pp.run_unfused(mq), stream)
                 un, _ = time_graph(gu, flush, stream, reps)
                 del gu
+            try:  # a supplementary series: its failure must not cost the table
+                eager_alloc_us, eager_err = time_eager(lambda: pp.run_alloc(mq, stream), stream), None
+            except Exception as e:  # noqa: BLE001
+                eager_alloc_us, eager_err = None, f"{type(e).__name__}: {e}"[:200]
+                torch.cuda.synchronize()
             ge = capture(lambda: pp.run_epilogue(mq), stream)
             epi_us, _ = time_graph(ge, flush, stream, reps)
             del ge
@@ -554,7 +645,9 @@ def workload_table(mq, device, stream, flush, hbm_gbs, reps):
                 "tflops": p.flops() / (us * 1e-6) / 1e12, "gbs": p.algorithmic_bytes() / (us * 1e-6) / 1e9,
                 "roofline_us": t_roof * 1e6, "frac_roofline": t_roof / (us * 1e-6), "unfused_us": un,
                 "plain_us": plain_us, "plain_over_macaq_time": plain_us / us,
-                "bias_gelu_tanh_us": epi_us,
+                "bias_gelu_tanh_us": epi_us, "eager_alloc_us": eager_alloc_us,
+                **({"eager_alloc_error": eager_err} if eager_err else {}),
+                "alu_bound_us": alu_bound_us(p.M, p.K, sms),
                 "nmse": nmse, "nmse_plain": nmse_plain, "nmse_plain_over_macaq": nmse_plain / nmse if nmse else None,
             })
             del g, pp
