@@ -87,6 +87,7 @@ def _L():
             "oracle_transform_f64": (None, [P, P, P, I64, I64, I64, P]),
             "oracle_dequantize": (None, [P, P, I64, I64, P]),
             "oracle_quantize_plain": (I, [P, I64, I64, P, P]),
+            "oracle_act_rotate_reading": (I, [P, P, I64, I64, I, P]),
             "oracle_num_threads": (I, []),
         }
         for name, (res, args) in sig.items():
@@ -179,6 +180,32 @@ def act_rotate(x_bf16: np.ndarray, D: np.ndarray) -> np.ndarray:
     u = np.empty_like(x)
     _L().oracle_act_rotate(_p(x), _p(D), M, K, _p(u))
     return u
+
+
+READING_R3, READING_TRUE_DIVISION, READING_BF16_STAGES, READING_EXACT_ROTATION = 0, 1, 2, 3
+
+
+def act_rotate_reading(x_bf16: np.ndarray, D: np.ndarray, reading: int) -> np.ndarray:
+    """Rotated BF16 activations under reading 0 (R3, the parity reference) or
+    one of the other plain readings of the summary's scaling and BF16 rotation:
+    1 true division by D, 2 BF16 rounding at every butterfly stage, 3 exact
+    rotation rounded once.  Used only to measure how often the reading matters."""
+    x = _c(x_bf16, np.uint16)
+    D = _c(D, np.float32)
+    M, K = x.shape
+    u = np.empty_like(x)
+    st = _L().oracle_act_rotate_reading(_p(x), _p(D), M, K, int(reading), _p(u))
+    assert st == OK, st
+    return u
+
+
+def quantize_act_reading(x_bf16: np.ndarray, D: np.ndarray, reading: int):
+    """Activation codes [M, K/2] and scales [M, K/32] under `reading`: the
+    rotation of act_rotate_reading, then the same E8M0 / E2M1 steps (R4, R5)."""
+    u = act_rotate_reading(x_bf16, D, reading)
+    M, K = u.shape
+    codes, scales = mx_quantize_blocks(bf16_to_f64(u).astype(np.float32))
+    return codes.reshape(M, K // 2), scales.reshape(M, K // 32)
 
 
 def quantize_act(x_bf16: np.ndarray, D: np.ndarray, nthreads: int = 0):

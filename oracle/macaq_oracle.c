@@ -47,6 +47,11 @@
  *       and w = max |W[:, k]| over its N weight rows; w = 0 < a gives 1e2,
  *       a = w = 0 gives 1, an expert with no rows gives D = 1 everywhere.
  *
+ * Other plain readings of R3 (true division by D, BF16 rounding at every
+ * butterfly stage, exact rotation rounded once) are implemented beside it by
+ * oracle_act_rotate_reading, only to measure how often the choice changes the
+ * codes; R3 alone is the parity reference.
+ *
  * The plain MXFP4 baseline (the MACAQ page's native W4A4 comparison, which
  * quantises x and W directly with the dynamic MX quantiser) skips D and H:
  * activations are the BF16 values themselves, weights the FP32 values, both
@@ -925,6 +930,68 @@ int oracle_quantize_plain(const float *v, int64_t R, int64_t K, uint8_t *codes, 
     if (K <= 0 || K % 32 != 0)
         return ORACLE_ERR_SHAPE;
     oracle_mx_quantize_blocks(v, R * K / 32, codes, scales);
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
+/* Other readings of the activation arithmetic (alternatives to R3)    */
+/* ------------------------------------------------------------------ */
+
+/* The summary names a channel scaling by raw D and a BF16 Hadamard rotation
+ * without fixing the working precision of either.  R3 (reading 0) is the
+ * parity reference; the others are equally plain readings, kept here only to
+ * measure how often the choice changes the MXFP4 codes:
+ *   1  true division: xs = RNE_bf16(RN32(x / D)), then R3's FP32 butterfly;
+ *   2  BF16 at every butterfly stage: each sum and difference of two BF16
+ *      values rounded once to BF16 (the arithmetic of packed BF16 adds);
+ *   3  exact rotation: the butterfly in binary64, exact for BF16 inputs
+ *      whose exponents span fewer than 45 binades within a block, then one
+ *      rounding to BF16.
+ * u receives M x K BF16 bit patterns. */
+int oracle_act_rotate_reading(const uint16_t *x, const float *D, int64_t M, int64_t K, int reading,
+                              uint16_t *u)
+{
+    if (K <= 0 || K % 32 != 0 || M < 0 || reading < 0 || reading > 3)
+        return ORACLE_ERR_SHAPE;
+    if (reading == 0) {
+        oracle_act_rotate(x, D, M, K, u);
+        return ORACLE_OK;
+    }
+    for (int64_t m = 0; m < M; m++) {
+        for (int64_t b = 0; b < K / 32; b++) {
+            const int64_t base = m * K + 32 * b;
+            float xs[32];
+            for (int i = 0; i < 32; i++) {
+                int64_t k = 32 * b + i;
+                float xf = bf16_bits_to_float(x[base + i]);
+                float s = reading == 1 ? xf / D[k] : xf * (1.0f / D[k]); /* one RN32 each */
+                xs[i] = bf16_bits_to_float(float_to_bf16_rne(s));
+            }
+            if (reading == 1) {
+                fwht32_f32(xs);
+                for (int i = 0; i < 32; i++)
+                    u[base + i] = float_to_bf16_rne(xs[i]);
+                continue;
+            }
+            double v[32];
+            for (int i = 0; i < 32; i++)
+                v[i] = (double)xs[i];
+            if (reading == 3) {
+                fwht32_f64(v);
+            } else {
+                for (int h = 1; h < 32; h <<= 1)
+                    for (int i = 0; i < 32; i++) {
+                        if (i & h)
+                            continue;
+                        double a = v[i], c = v[i + h]; /* BF16 values: a + c and a - c exact here */
+                        v[i] = oracle_bf16_to_f64(oracle_f64_to_bf16(a + c));
+                        v[i + h] = oracle_bf16_to_f64(oracle_f64_to_bf16(a - c));
+                    }
+            }
+            for (int i = 0; i < 32; i++)
+                u[base + i] = oracle_f64_to_bf16(v[i]);
+        }
+    }
     return ORACLE_OK;
 }
 
