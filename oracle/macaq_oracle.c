@@ -58,7 +58,7 @@
  * quantised by R4/R5, and y = RNE_bf16(exact sum) with no 2^-5 (there is no
  * Hadamard product to undo).
  *
- * Build:  gcc -O2 -std=c11 -ffp-contract=off -fno-fast-math -fopenmp -shared -fPIC
+ * Build:  gcc -O2 -std=gnu11 -ffp-contract=off -fno-fast-math -fopenmp -shared -fPIC
  * (no FMA contraction: every float operation is one IEEE binary32 rounding).
  */
 #include <stdint.h>
