@@ -136,6 +136,28 @@ def _stream_ptr(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
+def _arg(t, name: str, dtype, ndim: int | None = None, min_numel: int = 0):
+    """Element type, rank and size of an argument, checked before the call (the
+    library reads min_numel elements of it; a wrong element type would make it
+    read another tensor's bytes, or past the end)."""
+    if t is None:
+        return
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got shape {tuple(t.shape)}")
+    if t.numel() < min_numel:
+        raise ValueError(f"{name} holds {t.numel()} elements; the call reads {min_numel}")
+
+
+def _weights_args(Wq, Ws, E: int, N: int, K: int):
+    """Weight tile images: uint8, at least the bytes macaq_weight_*_bytes give
+    (0 for a shape the library refuses, which it then reports itself)."""
+    qb, sb = weight_bytes(E, N, K)
+    _arg(Wq, "Wq", torch.uint8, min_numel=qb)
+    _arg(Ws, "Ws", torch.uint8, min_numel=sb)
+
+
 def _require_cuda(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
@@ -202,8 +224,10 @@ def prepare_weights(W: torch.Tensor, D: torch.Tensor, stream=None) -> tuple[torc
         W = W.unsqueeze(0)
     if D.dim() == 1:
         D = D.unsqueeze(0)
-    _require_cuda(W, D)
+    _arg(W, "W", torch.float32, ndim=3)
     E, N, K = W.shape
+    _arg(D, "D", torch.float32, min_numel=E * K)
+    _require_cuda(W, D)
     qb, sb = weight_bytes(E, N, K)
     if qb == 0:
         raise MacaqError(-3, "prepare_weights")
@@ -228,9 +252,14 @@ def calibrate_d(x_cal: torch.Tensor, W: torch.Tensor, group_list: torch.Tensor |
     [T, K] and weights W fp32 [N, K] or [E, N, K] (rows split by group_list when E > 1)."""
     if W.dim() == 2:
         W = W.unsqueeze(0)
-    _require_cuda(x_cal, W, group_list)
+    _arg(x_cal, "x_cal", torch.bfloat16, ndim=2)
+    _arg(W, "W", torch.float32, ndim=3)
+    _arg(group_list, "group_list", torch.int64)
     T, K = x_cal.shape
-    E, N, _ = W.shape
+    E, N, KW = W.shape
+    if KW != K:
+        raise ValueError(f"W has {KW} input channels, x_cal {K}")
+    _require_cuda(x_cal, W, group_list)
     D = torch.empty((E, K), dtype=torch.float32, device=W.device)
     _check(lib().macaq_calibrate_d(_ptr(x_cal), T, _ptr(W), E, N, K, _ptr(group_list), int(group_list_type),
                                    _ptr(D), _stream_ptr(stream)), "macaq_calibrate_d")
@@ -243,6 +272,7 @@ def dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tenso
              act_type: int = ACT_NONE) -> torch.Tensor:
     """y [M, N] bf16 = MACAQ linear of x bf16 [M, K]; optional fp32 bias [N] and
     output activation act_type (npu_grouped_matmul's bias and act_type)."""
+    _dense_args(x, D, Wq, Ws, N, status)
     _require_cuda(x, D, Wq, Ws, out, status)
     M, K = x.shape
     _check_bias(bias, (N,))
@@ -261,6 +291,26 @@ def dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tenso
     return y
 
 
+def _dense_args(x, D, Wq, Ws, N: int, status):
+    _arg(x, "x", torch.bfloat16, ndim=2)
+    K = x.shape[1]
+    _arg(D, "D", torch.float32, min_numel=K)
+    if Wq is not None:
+        _weights_args(Wq, Ws, 1, N, K)
+    _arg(status, "status", torch.int32, min_numel=1)
+
+
+def _grouped_args(x, D, Wq, Ws, group_list, group_list_type: int, N: int, status) -> int:
+    _arg(x, "x", torch.bfloat16, ndim=2)
+    _arg(group_list, "group_list", torch.int64)
+    E = _groups(group_list, group_list_type)
+    K = x.shape[1]
+    _arg(D, "D", torch.float32, min_numel=E * K)
+    _weights_args(Wq, Ws, E, N, K)
+    _arg(status, "status", torch.int32, min_numel=1)
+    return E
+
+
 def _groups(group_list: torch.Tensor, group_list_type: int) -> int:
     """Number of group_list entries: rows of the [E, 2] form for type 2."""
     if group_list_type == 2:
@@ -277,9 +327,9 @@ def grouped_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Ten
     """Grouped MACAQ linear; group_list int64 on the device: [E] for type 0 (cumsum) and 1
     (counts), [E, 2] rows of (group index, group size) for type 2.  Optional fp32 bias
     [E, N] (per expert) and output activation act_type."""
+    E = _grouped_args(x, D, Wq, Ws, group_list, group_list_type, N, status)
     _require_cuda(x, D, Wq, Ws, group_list, out, status)
     M, K = x.shape
-    E = _groups(group_list, group_list_type)
     _check_bias(bias, (E, N))
     y = _output(out, M, N, x.device)
     L = lib()
@@ -302,6 +352,7 @@ def prepare_weights_plain(W: torch.Tensor, stream=None) -> tuple[torch.Tensor, t
     """Offline, plain MXFP4 baseline: W fp32 [N, K] or [E, N, K] -> (Wq, Ws) tile images of W itself."""
     if W.dim() == 2:
         W = W.unsqueeze(0)
+    _arg(W, "W", torch.float32, ndim=3)
     _require_cuda(W)
     E, N, K = W.shape
     qb, sb = weight_bytes(E, N, K)
@@ -317,6 +368,7 @@ def prepare_weights_plain(W: torch.Tensor, stream=None) -> tuple[torch.Tensor, t
 def dense_mm_plain(x: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: int, out: torch.Tensor | None = None,
                    status: torch.Tensor | None = None, stream=None, ws: torch.Tensor | None = None) -> torch.Tensor:
     """Plain MXFP4 W4A4 baseline (no D, no Hadamard): y [M, N] bf16."""
+    _dense_args(x, None, Wq, Ws, N, status)
     _require_cuda(x, Wq, Ws, out, status)
     M, K = x.shape
     y = _output(out, M, N, x.device)
@@ -332,9 +384,9 @@ def grouped_mm_plain(x: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, group_
                      group_list_type: int, N: int, out: torch.Tensor | None = None,
                      status: torch.Tensor | None = None, stream=None, ws: torch.Tensor | None = None) -> torch.Tensor:
     """Grouped plain MXFP4 W4A4 baseline; group_list as in grouped_mm."""
+    E = _grouped_args(x, None, Wq, Ws, group_list, group_list_type, N, status)
     _require_cuda(x, Wq, Ws, group_list, out, status)
     M, K = x.shape
-    E = _groups(group_list, group_list_type)
     y = _output(out, M, N, x.device)
     L = lib()
     ws = workspace(int(L.macaq_workspace_bytes(M, N, K, E)), x.device, stream, ws)
@@ -348,6 +400,7 @@ def unfused_dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: tor
                      out: torch.Tensor | None = None, status: torch.Tensor | None = None,
                      stream=None, ws: torch.Tensor | None = None) -> torch.Tensor:
     """Ablation: separate quantisation kernel, then the block-scaled GEMM."""
+    _dense_args(x, D, Wq, Ws, N, status)
     _require_cuda(x, D, Wq, Ws, out, status)
     M, K = x.shape
     y = _output(out, M, N, x.device)
@@ -365,6 +418,7 @@ def dense_mm_noalloc(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: tor
                      stream=None) -> torch.Tensor:
     """Dense MACAQ linear using the library's fixed device scratch buffer
     instead of a caller workspace (for callers that cannot allocate)."""
+    _dense_args(x, D, Wq, Ws, N, status)
     _require_cuda(x, D, Wq, Ws, out, status)
     M, K = x.shape
     y = _output(out, M, N, x.device)
@@ -375,6 +429,7 @@ def dense_mm_noalloc(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: tor
 
 def quantize_activations(x: torch.Tensor, D: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
     """Activation prologue alone: canonical codes [M, K/2] and E8M0 scales [M, K/32]."""
+    _dense_args(x, D, None, None, 0, None)
     _require_cuda(x, D)
     M, K = x.shape
     codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
@@ -387,6 +442,7 @@ def quantize_activations(x: torch.Tensor, D: torch.Tensor, stream=None) -> tuple
 def export_weights(Wq: torch.Tensor, Ws: torch.Tensor, E: int, N: int, K: int,
                    stream=None) -> tuple[torch.Tensor, torch.Tensor]:
     """Prepared tile images -> canonical codes [E, N, K/2] and scales [E, N, K/32]."""
+    _weights_args(Wq, Ws, E, N, K)
     _require_cuda(Wq, Ws)
     codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=Wq.device)
     scales = torch.empty((E, N, K // 32), dtype=torch.uint8, device=Wq.device)
@@ -397,6 +453,7 @@ def export_weights(Wq: torch.Tensor, Ws: torch.Tensor, E: int, N: int, K: int,
 
 def mx_encode_blocks(v: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
     """MX encoding (E8M0 + E2M1) of fp32 blocks of 32."""
+    _arg(v, "v", torch.float32)
     _require_cuda(v)
     n = v.numel()
     codes = torch.empty(n // 2, dtype=torch.uint8, device=v.device)
