@@ -181,12 +181,16 @@ class Prepared:
             mq.grouped_mm(self.x, self.D, self.Wq, self.Ws, self.gl, self.p.group_list_type, self.p.N,
                           out=self.y, stream=stream, ws=self.ws)
 
-    def run_alloc(self, mq, stream=None):
+    def run_alloc(self, mq, stream=None, alt: bool = False):
         """The call as made without a preallocated output: the binding allocates y
-        (torch.empty through the caching allocator) on every call."""
+        (torch.empty through the caching allocator) on every call.  alt takes a
+        second, distinct activation buffer holding the same values."""
+        if alt and getattr(self, "x_alt", None) is None:
+            self.x_alt = self.x.clone()
+        x = self.x_alt if alt else self.x
         if self.gl is None:
-            return mq.dense_mm(self.x, self.D, self.Wq, self.Ws, self.p.N, stream=stream)
-        return mq.grouped_mm(self.x, self.D, self.Wq, self.Ws, self.gl, self.p.group_list_type, self.p.N,
+            return mq.dense_mm(x, self.D, self.Wq, self.Ws, self.p.N, stream=stream)
+        return mq.grouped_mm(x, self.D, self.Wq, self.Ws, self.gl, self.p.group_list_type, self.p.N,
                              stream=stream)
 
     def run_epilogue(self, mq, stream=None):
@@ -582,17 +586,18 @@ def alu_bound_us(rows: int, K: int, sms: int, mhz: float = SM_MAX_MHZ) -> float:
 
 def time_eager(fn, stream, calls: int = 20, trials: int = 15, warm: int = 20) -> float:
     """Median us per call over `trials` blocks of `calls` eager calls (host launch
-    included, L2 not flushed), CUDA events on `stream`."""
+    included, L2 not flushed), CUDA events on `stream`; fn(i) is told the call's
+    index, so that callers can alternate inputs."""
     out = []
     with torch.cuda.stream(stream):
-        for _ in range(warm):
-            fn()
+        for i in range(warm):
+            fn(i)
         for _ in range(trials):
             t0 = torch.cuda.Event(enable_timing=True)
             t1 = torch.cuda.Event(enable_timing=True)
             t0.record(stream)
-            for _ in range(calls):
-                fn()
+            for i in range(calls):
+                fn(i)
             t1.record(stream)
             t1.synchronize()
             out.append(t0.elapsed_time(t1) * 1e3 / calls)
@@ -620,7 +625,8 @@ def workload_table(mq, device, stream, flush, hbm_gbs, reps):
                 un, _ = time_graph(gu, flush, stream, reps)
                 del gu
             try:  # a supplementary series: its failure must not cost the table
-                eager_alloc_us, eager_err = time_eager(lambda: pp.run_alloc(mq, stream), stream), None
+                eager_alloc_us = time_eager(lambda i: pp.run_alloc(mq, stream, alt=bool(i & 1)), stream)
+                eager_err = None
             except Exception as e:  # noqa: BLE001
                 eager_alloc_us, eager_err = None, f"{type(e).__name__}: {e}"[:200]
                 torch.cuda.synchronize()

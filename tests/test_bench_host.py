@@ -44,3 +44,20 @@ def test_decoded_gemm_equals_the_exact_oracle_gemm_on_these_operands():
     qa, sa = oracle.quantize_act(p.x, p.D[0])
     dec = (oracle.dequantize(qa, sa) @ oracle.dequantize(qw, sw).T) * 2.0 ** -5
     assert np.array_equal(oracle.f64_to_bf16(dec), oracle.gemm(qa, sa, qw, sw))
+
+
+def test_eager_series_alternates_two_distinct_activation_buffers():
+    import types
+    import torch
+    seen = []
+    fake = types.SimpleNamespace(dense_mm=lambda x, *a, **k: seen.append((x.data_ptr(), x.clone())))
+    pp = object.__new__(bench.Prepared)
+    pp.x = torch.arange(64, dtype=torch.float32).reshape(4, 16)
+    pp.D = pp.Wq = pp.Ws = None
+    pp.gl = None
+    pp.p = types.SimpleNamespace(N=16)
+    for i in range(4):
+        pp.run_alloc(fake, None, alt=bool(i & 1))
+    ptrs = [s[0] for s in seen]
+    assert ptrs[0] == ptrs[2] and ptrs[1] == ptrs[3] and ptrs[0] != ptrs[1]
+    assert all(torch.equal(s[1], pp.x) for s in seen)
