@@ -22,15 +22,17 @@
  * group_list_type): rows [off_g, off_g + count_g) of x use expert g's D and
  * weights; group_list holds E int64 values, cumulative sums (type 0) or
  * counts (type 1), non-negative, cumulative sums non-decreasing, covering
- * exactly M rows; at most 1024 groups.
+ * exactly M rows, or E rows of (group index, group size) (type 2, see
+ * macaq_grouped_mm); at most 1024 groups.
  *
  * Conventions for every entry point:
  *  - Pointers named *_dev are device pointers owned by the caller.  The
  *    library never frees or keeps them; it allocates no memory on any call.
  *  - BF16 tensors are passed as uint16_t bit patterns.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
- *    stream).  Calls are asynchronous on that stream; none synchronises
- *    except macaq_prepare_weights, which reads D back to validate it.
+ *    stream).  Calls are asynchronous on that stream; none of the hot-path
+ *    calls synchronises.  Two offline calls do: macaq_prepare_weights reads D
+ *    back to validate it, and macaq_calibrate_d reads its group list back.
  *  - Return value: MACAQ_OK (0) or a negative status below.  A call that
  *    returns an error launched nothing.  Errors found on the device (an
  *    invalid group_list, a bounded wait that expired) are written to the
@@ -264,9 +266,9 @@ int macaq_unfused_dense_mm(const uint16_t *x_dev, const float *D_dev, const uint
  *   runtime query, no allocation); make that first call before any stream
  *   capture on that device.
  *   Every call shares the one buffer and rewrites every byte of it whose
- *   value reaches the output (nothing in it has to start at zero).  Calls whose kernels overlap on the
- *   GPU -- on different streams, or from different host threads -- race on
- *   it and must be ordered by the caller. */
+ *   value reaches the output (nothing in it has to start at zero).  Calls
+ *   whose kernels overlap on the GPU -- on different streams, or from
+ *   different host threads -- race on it and must be ordered by the caller. */
 int macaq_dense_mm_noalloc(const uint16_t *x_dev, const float *D_dev, const uint8_t *Wq_dev,
                            const uint8_t *Ws_dev, uint16_t *y_dev, int64_t M, int64_t N, int64_t K,
                            int32_t *status_dev, void *stream);
