@@ -190,7 +190,7 @@ def _check_large(p: synth.Problem, y_bits: np.ndarray, n_samples: int = 3000):
     compare(y_bits, dequant_matmul_bf16(qa, sa, qw, sw), p.name + " full f64")
 
 
-@pytest.mark.parametrize("i", [0, 3, 4])
+@pytest.mark.parametrize("i", [0, 1, 2, 3, 4])
 def test_dense_prefill_config(i):
     p = synth.config(2)[i]
     _check_large(p, _run_dense(p))
