@@ -47,6 +47,12 @@
  *       and w = max |W[:, k]| over its N weight rows; w = 0 < a gives 1e2,
  *       a = w = 0 gives 1, an expert with no rows gives D = 1 everywhere.
  *
+ * Parity unpinned by the pages (readings both sides implement identically,
+ * with no printed value to check them against): the last-bit rounding order
+ * of R3's butterfly, the sign of zero codes in R5, the FAST_GELU formula in
+ * R15 and the calibration rule in R16 (against MACAQ's own, unpublished one).
+ * Each is still pinned to its own definition by the host tests.
+ *
  * Other plain readings of R3 (true division by D, BF16 rounding at every
  * butterfly stage, exact rotation rounded once) are implemented beside it by
  * oracle_act_rotate_reading, only to measure how often the choice changes the
