@@ -537,6 +537,10 @@ def main():
                 line["cpu_baseline"].update(cpu_oracle_detail([pp.p for pp in problems], prepared, cores))
             except Exception as e:  # noqa: BLE001
                 line["cpu_baseline"]["detail_error"] = f"{type(e).__name__}: {e}"[:200]
+            try:  # supplementary: its failure must not cost the line
+                line["launch_floor"] = launch_floor(device, stream, flush, args.table_reps)
+            except Exception as e:  # noqa: BLE001
+                line["launch_floor"] = {"error": f"{type(e).__name__}: {e}"[:200]}
             if not args.no_table:
                 line["per_workload"] = workload_table(mq, device, stream, flush, hbm_gbs, args.table_reps)
                 line["calibration"] = calibration_table(mq, device, stream, flush, hbm_gbs, args.table_reps)
@@ -659,6 +663,19 @@ def workload_table(mq, device, stream, flush, hbm_gbs, reps):
             del g, pp
             torch.cuda.empty_cache()
     return rows
+
+
+def launch_floor(device, stream, flush, reps: int, launches: int = 5) -> dict:
+    """The floor a chain of dependent launches sets, measured the way the step is:
+    a CUDA graph of `launches` dependent one-element adds (torch's kernels, no
+    work to speak of), L2 flushed before each replay, device time per launch.
+    The step's kernels cannot finish faster than this per launch."""
+    t = torch.zeros(1, device=device)
+    g = capture(lambda: [t.add_(1.0) for _ in range(launches)], stream)
+    us, _ = time_graph(g, flush, stream, reps)
+    del g
+    return {"us_per_launch": us / launches, "launches": launches,
+            "what": "CUDA graph of dependent one-element adds, L2 flushed before each replay"}
 
 
 def calibration_table(mq, device, stream, flush, hbm_gbs, reps):
