@@ -668,8 +668,10 @@ def workload_table(mq, device, stream, flush, hbm_gbs, reps):
 def launch_floor(device, stream, flush, reps: int, launches: int = 5) -> dict:
     """The floor a chain of dependent launches sets, measured the way the step is:
     a CUDA graph of `launches` dependent one-element adds (torch's kernels, no
-    work to speak of), L2 flushed before each replay, device time per launch.
-    The step's kernels cannot finish faster than this per launch."""
+    work to speak of), L2 flushed before each replay, device time per launch: the
+    share of the step's per-launch time that launching and chaining alone cost
+    (the step's kernels also use programmatic dependent launch, which can overlap
+    a launch with its predecessor's tail)."""
     t = torch.zeros(1, device=device)
     g = capture(lambda: [t.add_(1.0) for _ in range(launches)], stream)
     us, _ = time_graph(g, flush, stream, reps)
