@@ -270,6 +270,19 @@ def test_unquantised_transform_preserves_the_layer():
     assert np.allclose(got, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
 
 
+def test_unquantised_linear_is_the_library_matmul():
+    # the reference layer x . W^T against numpy's binary64 matmul (independent of
+    # the oracle's own loops); a transposed operand or a dropped row fails it
+    rng = np.random.default_rng(18)
+    M, N, K = 6, 9, 96
+    x = synth.to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    W = rng.standard_normal((N, K)).astype(np.float32)
+    want = oracle.bf16_to_f64(x) @ W.astype(np.float64).T
+    got = oracle.linear_f64(x, W)
+    assert got.shape == (M, N)
+    assert np.allclose(got, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+
+
 def test_weight_path_definition():
     rng = np.random.default_rng(9)
     N, K = 4, 64
