@@ -193,6 +193,15 @@ class Prepared:
         return mq.grouped_mm(x, self.D, self.Wq, self.Ws, self.gl, self.p.group_list_type, self.p.N,
                              stream=stream)
 
+    def run_type2(self, mq, stream=None):
+        """The grouped call with the same groups written as group_list_type 2:
+        [E, 2] rows of (group index, group size) in expert order."""
+        if getattr(self, "gl2", None) is None:
+            rows = np.stack([np.arange(self.p.E), self.p.counts], axis=1).astype(np.int64)
+            self.gl2 = torch.from_numpy(rows).to(self.y.device)
+        mq.grouped_mm(self.x, self.D, self.Wq, self.Ws, self.gl2, 2, self.p.N, out=self.y, stream=stream,
+                      ws=self.ws)
+
     def run_epilogue(self, mq, stream=None):
         """The same call with an fp32 bias and GELU_TANH (npu_grouped_matmul's bias and act_type)."""
         if getattr(self, "bias", None) is None:
@@ -634,6 +643,14 @@ def workload_table(mq, device, stream, flush, hbm_gbs, reps):
             except Exception as e:  # noqa: BLE001
                 eager_alloc_us, eager_err = None, f"{type(e).__name__}: {e}"[:200]
                 torch.cuda.synchronize()
+            type2_us = None
+            if p.E > 1:
+                try:  # supplementary: its failure must not cost the table
+                    g2 = capture(lambda: pp.run_type2(mq), stream)
+                    type2_us, _ = time_graph(g2, flush, stream, reps)
+                    del g2
+                except Exception:  # noqa: BLE001
+                    type2_us = None
             ge = capture(lambda: pp.run_epilogue(mq), stream)
             epi_us, _ = time_graph(ge, flush, stream, reps)
             del ge
@@ -655,7 +672,7 @@ def workload_table(mq, device, stream, flush, hbm_gbs, reps):
                 "tflops": p.flops() / (us * 1e-6) / 1e12, "gbs": p.algorithmic_bytes() / (us * 1e-6) / 1e9,
                 "roofline_us": t_roof * 1e6, "frac_roofline": t_roof / (us * 1e-6), "unfused_us": un,
                 "plain_us": plain_us, "plain_over_macaq_time": plain_us / us,
-                "bias_gelu_tanh_us": epi_us, "eager_alloc_us": eager_alloc_us,
+                "bias_gelu_tanh_us": epi_us, "eager_alloc_us": eager_alloc_us, "group_list_type2_us": type2_us,
                 **({"eager_alloc_error": eager_err} if eager_err else {}),
                 "alu_bound_us": alu_bound_us(p.M, p.K, sms),
                 "nmse": nmse, "nmse_plain": nmse_plain, "nmse_plain_over_macaq": nmse_plain / nmse if nmse else None,

@@ -61,3 +61,24 @@ def test_eager_series_alternates_two_distinct_activation_buffers():
     ptrs = [s[0] for s in seen]
     assert ptrs[0] == ptrs[2] and ptrs[1] == ptrs[3] and ptrs[0] != ptrs[1]
     assert all(torch.equal(s[1], pp.x) for s in seen)
+
+
+def test_type2_list_covers_the_same_groups():
+    import types
+    import numpy as np
+    import torch
+    import synth
+    p = synth.grouped(300, 16, 256, 64, seed=1, dist="zipf", group_list_type=0)
+    calls = []
+    fake = types.SimpleNamespace(grouped_mm=lambda x, D, Wq, Ws, gl, t, N, **k: calls.append((gl.clone(), t, N)))
+    pp = object.__new__(bench.Prepared)
+    pp.p, pp.x, pp.D, pp.Wq, pp.Ws, pp.ws = p, None, None, None, None, None
+    pp.y = torch.empty(0)
+    pp.run_type2(fake)
+    gl, t, N = calls[0]
+    assert t == 2 and N == p.N and tuple(gl.shape) == (p.E, 2) and gl.dtype == torch.int64
+    rows = gl.numpy()
+    assert np.array_equal(rows[:, 0], np.arange(p.E))
+    assert np.array_equal(rows[:, 1], p.counts) and rows[:, 1].sum() == p.M
+    # the type-0 list of the same problem gives the same row ranges
+    assert np.array_equal(np.cumsum(rows[:, 1]), p.group_list)
