@@ -56,7 +56,9 @@ _lib = None
 def _L():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
+        # MACAQ_ORACLE_LIB: a test may load a deliberately mutated build instead,
+        # to check that the pins catch each planted mistake
+        lib = ctypes.CDLL(os.environ.get("MACAQ_ORACLE_LIB") or build())
         P = ctypes.c_void_p
         I64 = ctypes.c_int64
         I = ctypes.c_int

@@ -1,0 +1,78 @@
+"""The oracle's pins catch plausible mistakes.
+
+Each case plants one mistake in a temporary copy of oracle/macaq_oracle.c (the
+oracle itself is never changed), builds it with the oracle's own flags, and runs
+the host pin suites against that build: every mutant must fail at least one
+pin.  An unmutated copy built the same way must pass, so a failure is the
+planted mistake's and not the harness's.
+"""
+import concurrent.futures
+import os
+import subprocess
+import sys
+import tempfile
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "macaq_oracle.c")
+PINS = ["tests/test_oracle.py", "tests/test_oracle_readings.py"]
+
+# (name, text in the oracle, replacement): each a mistake someone could make
+MUTANTS = [
+    ("butterfly difference sign", "float b = v[i + h];\n            v[i] = a + b;\n            v[i + h] = a - b;",
+     "float b = v[i + h];\n            v[i] = a + b;\n            v[i + h] = b - a;"),
+    ("E8M0 offset of the largest E2M1 exponent", "int c = floor_log2 - 2 + 127;", "int c = floor_log2 - 1 + 127;"),
+    ("E2M1 tie at 0.25 rounded up", "if (a <= 0.25)", "if (a < 0.25)"),
+    ("E2M1 tie at 2.5 rounded up", "else if (a <= 2.5)", "else if (a < 2.5)"),
+    ("activations multiplied by D", "float prod = bf16_bits_to_float(xrow[k]) * r;",
+     "float prod = bf16_bits_to_float(xrow[k]) / r;"),
+    ("no BF16 rounding of the scaled activations", "v[i] = bf16_bits_to_float(float_to_bf16_rne(prod));",
+     "v[i] = prod;"),
+    ("weights divided by D", "t[i] = W[n * K + k] * D[k];", "t[i] = W[n * K + k] / D[k];"),
+    ("output scale 2^-4", "return gemm_exp(qa, sa, qw, sw, M, N, K, y, nthreads, -5);",
+     "return gemm_exp(qa, sa, qw, sw, M, N, K, y, nthreads, -4);"),
+    ("plain path keeps 2^-5", "return gemm_exp(qa, sa, qw, sw, M, N, K, y, nthreads, 0);",
+     "return gemm_exp(qa, sa, qw, sw, M, N, K, y, nthreads, -5);"),
+    ("counts read as cumulative sums", "        if (type == 0) {\n            if (v < off[g])",
+     "        if (type == 1) {\n            if (v < off[g])"),
+    ("calibration ratio inverted", "d = sqrt(a / w);", "d = sqrt(w / a);"),
+    ("GELU cubic coefficient", "(v + 0.044715 * v * v * v)", "(v + 0.04715 * v * v * v)"),
+    ("FAST_GELU slope", "return v / (1.0 + exp(-1.702 * v));", "return v / (1.0 + exp(-1.72 * v));"),
+    ("BF16 ties rounded up", "if (dropped > 0x8000u || (dropped == 0x8000u && (keep & 1u)))",
+     "if (dropped >= 0x8000u)"),
+]
+
+
+def _build(text: str, out: str):
+    with tempfile.NamedTemporaryFile("w", suffix=".c", delete=False) as f:
+        f.write(text)
+        c = f.name
+    try:
+        subprocess.check_call(["gcc", "-O2", "-std=gnu11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
+                               "-shared", "-fPIC", "-o", out, c, "-lm"])
+    finally:
+        os.unlink(c)
+
+
+def _run_pins(lib: str) -> int:
+    env = dict(os.environ, MACAQ_ORACLE_LIB=lib, OMP_NUM_THREADS="2")
+    return subprocess.run([sys.executable, "-m", "pytest", *PINS, "-x", "-q", "-p", "no:cacheprovider",
+                           "-m", "not gpu"], cwd=ROOT, env=env, capture_output=True, timeout=600).returncode
+
+
+def test_every_planted_mistake_fails_a_pin(tmp_path):
+    src = open(SRC).read()
+    jobs = [("control", None, None)] + MUTANTS
+    libs = []
+    for i, (name, old, new) in enumerate(jobs):
+        if old is not None:
+            assert src.count(old) == 1, f"{name}: the text to mutate must occur once"
+        lib = str(tmp_path / f"m{i}.so")
+        _build(src if old is None else src.replace(old, new), lib)
+        libs.append((name, lib))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=4) as ex:
+        codes = list(ex.map(lambda nl: _run_pins(nl[1]), libs))
+    assert codes[0] == 0, "the unmutated build must pass every pin"
+    survivors = [name for (name, _), rc in zip(libs[1:], codes[1:]) if rc == 0]
+    assert not survivors, f"mistakes no pin caught: {survivors}"
