@@ -660,6 +660,26 @@ def test_grouped_epilogue_uses_each_experts_bias():
             assert np.array_equal(y[off[g]:off[g + 1]], ref)
 
 
+def test_grouped_type2_bias_follows_the_named_expert():
+    # type-2 rows name their expert; with replicated banks the bias is the only
+    # thing that differs between experts, so each range must carry the bias of
+    # the expert it names (not of its position in the list)
+    rng = np.random.default_rng(6)
+    M, K, N, E = 45, 256, 32, 4
+    p = synth.dense(M, K, N, seed=10)
+    W = np.repeat(p.W, E, axis=0)
+    D = np.repeat(p.D, E, axis=0)
+    bias = rng.standard_normal((E, N)).astype(np.float32)
+    gl = np.array([[3, 10], [3, 5], [0, 0], [1, 30]], np.int64)   # expert 3 twice, expert 2 never
+    st, y = oracle.grouped_mm_ex(p.x, D, W, gl, 2, bias, oracle.ACT_SILU)
+    assert st == oracle.OK
+    r0 = 0
+    for e, n in gl:
+        ref = oracle.dense_mm_ex(p.x[r0:r0 + n], p.D[0], p.W[0], bias[e], oracle.ACT_SILU)
+        assert np.array_equal(y[r0:r0 + n], ref)
+        r0 += n
+
+
 # ----------------------------------------------------------------------------
 # Offline calibration of D (reading R16: D = clamp(sqrt(max|x| / max|W|), 1e-2, 1e2))
 # ----------------------------------------------------------------------------

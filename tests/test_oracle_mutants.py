@@ -18,7 +18,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "macaq_oracle.c")
 PINS = ["tests/test_oracle.py", "tests/test_oracle_readings.py"]
 
-# (name, text in the oracle, replacement): each a mistake someone could make
+# (name, text in the oracle, replacement[, occurrences replaced, default 1]):
+# each a mistake someone could make
 MUTANTS = [
     ("butterfly difference sign", "float b = v[i + h];\n            v[i] = a + b;\n            v[i + h] = a - b;",
      "float b = v[i + h];\n            v[i] = a + b;\n            v[i + h] = b - a;"),
@@ -41,6 +42,16 @@ MUTANTS = [
     ("FAST_GELU slope", "return v / (1.0 + exp(-1.702 * v));", "return v / (1.0 + exp(-1.72 * v));"),
     ("BF16 ties rounded up", "if (dropped > 0x8000u || (dropped == 0x8000u && (keep & 1u)))",
      "if (dropped >= 0x8000u)"),
+    ("type-2 rows use the list position, not the named expert",
+     "int64_t e = type == 2 ? group_list[2 * g] : g;", "int64_t e = g;"),
+    ("grouped bias taken by list position", "bias ? bias + e * N : NULL", "bias ? bias + g * N : NULL"),
+    ("grouped activations scaled by expert 0's D", "oracle_quantize_act(x + r0 * K, D + e * K,",
+     "oracle_quantize_act(x + r0 * K, D,"),
+    ("weight scale dropped from the exact dot", "int E = (int)sa[b] + (int)sw[b] - 256;",
+     "int E = (int)sa[b] + 127 - 256;"),
+    ("code nibbles swapped in both exact dots", "int ca = (qa[k / 2] >> (4 * (k & 1))) & 15;",
+     "int ca = (qa[k / 2] >> (4 * (1 - (k & 1)))) & 15;", 2),
+    ("type-2 index bound off by one", "group_list[2 * g] >= E))", "group_list[2 * g] > E))"),
 ]
 
 
@@ -65,9 +76,10 @@ def test_every_planted_mistake_fails_a_pin(tmp_path):
     src = open(SRC).read()
     jobs = [("control", None, None)] + MUTANTS
     libs = []
-    for i, (name, old, new) in enumerate(jobs):
+    for i, (name, old, new, *count) in enumerate(jobs):
         if old is not None:
-            assert src.count(old) == 1, f"{name}: the text to mutate must occur once"
+            want = count[0] if count else 1
+            assert src.count(old) == want, f"{name}: the text to mutate must occur {want} time(s)"
         lib = str(tmp_path / f"m{i}.so")
         _build(src if old is None else src.replace(old, new), lib)
         libs.append((name, lib))
