@@ -151,6 +151,7 @@ def test_e8m0_defining_property():
             if not np.isfinite(a) or a == 0:
                 continue
             c = oracle.e8m0_from_amax(a)
+            assert 0 <= c <= 254          # an E8M0 code (255 is NaN); tiny amax clamps to 0
             r = Fraction(float(a)) / Fraction(2) ** (c - 127)
             assert r < 8
             if c > 0:

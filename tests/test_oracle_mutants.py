@@ -52,6 +52,19 @@ MUTANTS = [
     ("code nibbles swapped in both exact dots", "int ca = (qa[k / 2] >> (4 * (k & 1))) & 15;",
      "int ca = (qa[k / 2] >> (4 * (1 - (k & 1)))) & 15;", 2),
     ("type-2 index bound off by one", "group_list[2 * g] >= E))", "group_list[2 * g] > E))"),
+    ("calibration rows of a type-2 entry credited to its position",
+     "int64_t e = (group_list && type == 2) ? group_list[2 * g] : g;", "int64_t e = g;"),
+    ("calibration ignores an expert without rows", "            if (rows[e] == 0) {\n                D[e * K + k] = 1.0f;",
+     "            if (rows[e] < 0) {\n                D[e * K + k] = 1.0f;"),
+    ("calibration lower clamp 1e-3", "    if (d < 1e-2)\n        d = 1e-2;", "    if (d < 1e-3)\n        d = 1e-3;"),
+    ("E8M0 not clamped at 0", "    if (c < 0)\n        c = 0;", "    if (c < -1)\n        c = 0;"),
+    ("BF16 from binary64 ties away from zero", "double q = nearbyint(ldexp(a, -lsb));", "double q = round(ldexp(a, -lsb));"),
+    ("weights not rotated", "            fwht32_f32(t);\n            double d[32];", "            double d[32];"),
+    ("SILU as v sigmoid(2v)", "return v / (1.0 + exp(-v));", "return v / (1.0 + exp(-2.0 * v));"),
+    ("true-division reading multiplies by the reciprocal",
+     "float s = reading == 1 ? xf / D[k] : xf * (1.0f / D[k]);", "float s = xf * (1.0f / D[k]);"),
+    ("BF16-stage reading rounds only the sums",
+     "v[i + h] = oracle_bf16_to_f64(oracle_f64_to_bf16(a - c));", "v[i + h] = a - c;"),
 ]
 
 

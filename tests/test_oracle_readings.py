@@ -94,6 +94,21 @@ def test_bf16_stages_worked_example():
     assert to_f64(oracle.act_rotate_reading(x, D, R2))[0, 0] == 1.0
 
 
+def test_bf16_stages_round_the_differences_too():
+    # block [1, 2^-9, 2^-10, -2^-10, 0, ...], D = 1.  Row 3 of H is (+, -, -, +, ...),
+    # so the exact u[3] = 1 - 2^-9 - 2^-10 - 2^-10 = 1 - 2^-8 (a BF16 value), which
+    # R3's FP32 butterfly and reading 3 reach.  With BF16 stages the difference
+    # 1 - 2^-9 at h = 1 is a tie between 1 - 2^-8 and 1 and goes to the even 1; at
+    # h = 2, 1 - 2^-9 is again a tie and gives 1; later stages add zeros: u[3] = 1.
+    K = 32
+    x = np.zeros((1, K), np.uint16)
+    x[0, :4] = bf16(np.array([1.0, 2.0 ** -9, 2.0 ** -10, -(2.0 ** -10)]))
+    D = np.ones(K, np.float32)
+    assert to_f64(oracle.act_rotate_reading(x, D, R0))[0, 3] == 1 - 2.0 ** -8
+    assert to_f64(oracle.act_rotate_reading(x, D, R3))[0, 3] == 1 - 2.0 ** -8
+    assert to_f64(oracle.act_rotate_reading(x, D, R2))[0, 3] == 1.0
+
+
 @pytest.mark.parametrize("reading", [R1, R2, R3])
 def test_readings_agree_when_every_partial_sum_is_exact_in_bf16(reading):
     # entries in {-1, 0, 1} and D = 1: every partial sum is an integer of magnitude
