@@ -428,6 +428,27 @@ def _pack(codes):
     return (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
 
 
+def test_exact_gemm_subnormal_outputs():
+    # one product 1.5 x 1.0 per output, scales chosen so that 2^-5 times it lands
+    # in BF16's subnormal range (last bit 2^-133): 1.5 x 2^(64+65-259) = 12 x 2^-133
+    # exactly, and 1.5 x 2^(64+62-259) = 1.5 x 2^-133, a tie between 1 and 2 units
+    # that rounds to the even 2
+    qa = np.zeros((1, 16), np.uint8)
+    qa[0, 0] = 3                      # code 3 = 1.5 (element 0, low nibble)
+    qw = np.zeros((2, 16), np.uint8)
+    qw[:, 0] = 2                      # code 2 = 1.0
+    sa = np.array([[64]], np.uint8)
+    sw = np.array([[65], [62]], np.uint8)
+    y = oracle.gemm(qa, sa, qw, sw)
+    unit = Fraction(2) ** -133
+    for n, s_w in enumerate((65, 62)):
+        exact = Fraction(3, 2) * Fraction(2) ** (64 + s_w - 254 - 5)
+        q = exact / unit
+        units = int(q) + (1 if (q - int(q) > Fraction(1, 2) or (q - int(q) == Fraction(1, 2) and int(q) % 2)) else 0)
+        assert y[0, n] == units        # BF16 subnormal bits = number of 2^-133 units
+    assert list(y[0]) == [0x000C, 0x0002]
+
+
 def test_exact_gemm_cancellation_and_ties():
     # +1 and -1 against +1, +1: the sum cancels to exactly +0
     ca = np.zeros((1, 32), int); cw = np.zeros((1, 32), int)
@@ -528,6 +549,20 @@ def test_grouped_empty_groups():
     st, y = oracle.grouped_mm(p.x, p.D, p.W, counts, 1)
     assert st == oracle.OK
     assert np.array_equal(y, oracle.dense_mm(p.x, p.D[1], p.W[1]))
+
+
+def test_grouped_one_row_groups():
+    # groups of a single row at the start, middle and end, around empty ones:
+    # each row equals the dense product with its own expert
+    p = synth.grouped(40, 5, 64, 32, seed=7, dist="uniform", group_list_type=1)
+    counts = np.array([1, 0, 38, 0, 1], np.int64)
+    st, y = oracle.grouped_mm(p.x, p.D, p.W, counts, 1)
+    assert st == oracle.OK
+    off = np.concatenate([[0], np.cumsum(counts)])
+    for g in range(5):
+        if counts[g]:
+            want = oracle.dense_mm(p.x[off[g]:off[g + 1]], p.D[g], p.W[g])
+            assert np.array_equal(y[off[g]:off[g + 1]], want), g
 
 
 # ----------------------------------------------------------------------------

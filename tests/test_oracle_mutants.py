@@ -18,6 +18,9 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "macaq_oracle.c")
 PINS = ["tests/test_oracle.py", "tests/test_oracle_readings.py"]
 
+# the BF16 rounding step of the exact GEMM (the binary64 one beside it is alike)
+BF_ROUND = "        q = (q << 1) | (uint32_t)wide_bit(&a, i);\n    if (L > 0) {\n        int round = wide_bit(&a, L - 1);\n        int sticky = wide_any_below(&a, L - 1);\n        if (round && (sticky || (q & 1)))"
+
 # (name, text in the oracle, replacement[, occurrences replaced, default 1]):
 # each a mistake someone could make
 MUTANTS = [
@@ -65,6 +68,14 @@ MUTANTS = [
      "float s = reading == 1 ? xf / D[k] : xf * (1.0f / D[k]);", "float s = xf * (1.0f / D[k]);"),
     ("BF16-stage reading rounds only the sums",
      "v[i + h] = oracle_bf16_to_f64(oracle_f64_to_bf16(a - c));", "v[i + h] = a - c;"),
+    ("exact GEMM rounding without the sticky bit", BF_ROUND, BF_ROUND.replace("(sticky || (q & 1))", "(q & 1)")),
+    ("exact GEMM ties away from zero", BF_ROUND, BF_ROUND.replace("round && (sticky || (q & 1))", "round")),
+    ("exact GEMM without BF16 subnormals", "int lsb_exp = E >= -126 ? E - 7 : -133;", "int lsb_exp = E - 7;"),
+    ("bias added after the activation",
+     "            if (bias)\n                s += (double)bias[n];\n            y[m * N + n] = oracle_f64_to_bf16(oracle_act(s, act));",
+     "            y[m * N + n] = oracle_f64_to_bf16(oracle_act(s, act) + (bias ? (double)bias[n] : 0.0));"),
+    ("one-row groups skipped with the empty ones", "        if (r1 == r0)\n            continue;",
+     "        if (r1 <= r0 + 1)\n            continue;"),
 ]
 
 
