@@ -76,6 +76,16 @@ MUTANTS = [
      "            y[m * N + n] = oracle_f64_to_bf16(oracle_act(s, act) + (bias ? (double)bias[n] : 0.0));"),
     ("one-row groups skipped with the empty ones", "        if (r1 == r0)\n            continue;",
      "        if (r1 <= r0 + 1)\n            continue;"),
+    ("block amax without the absolute value", "        float a = (float)fabs(v[i]);\n        if (a > amax || isnan(a))",
+     "        float a = (float)v[i];\n        if (a > amax || isnan(a))"),
+    ("codes packed high nibble first", "codes[j] = (uint8_t)(lo | (hi << 4));", "codes[j] = (uint8_t)(hi | (lo << 4));"),
+    ("one D per block instead of per channel", "float r = 1.0f / D[k];                            /* RN32(1/D) */",
+     "float r = 1.0f / D[32 * b];                       /* RN32(1/D) */"),
+    ("RELU leaks negatives", "return v > 0.0 ? v : 0.0;", "return v > 0.0 ? v : 0.01 * v;"),
+    ("calibration skips the last weight row", "            for (int64_t n = 0; n < N; n++) {\n                double v = fabs((double)W[(e * N + n) * K + k]);",
+     "            for (int64_t n = 0; n + 1 < N; n++) {\n                double v = fabs((double)W[(e * N + n) * K + k]);"),
+    ("calibration skips the last row of each group", "        for (int64_t r = off[g]; r < off[g + 1]; r++)",
+     "        for (int64_t r = off[g]; r + 1 < off[g + 1]; r++)"),
 ]
 
 
