@@ -449,6 +449,20 @@ def test_exact_gemm_subnormal_outputs():
     assert list(y[0]) == [0x000C, 0x0002]
 
 
+def test_plain_grouped_rows_use_the_named_expert():
+    # type-2 list with one-row ranges, a repeated expert and an empty entry: each
+    # range equals the plain dense product with the expert it names
+    p = synth.grouped(40, 4, 64, 32, seed=8, dist="uniform", group_list_type=1)
+    gl = np.array([[2, 1], [0, 0], [3, 38], [2, 1]], np.int64)
+    st, y = oracle.grouped_mm_plain(p.x, p.W, gl, 2)
+    assert st == oracle.OK
+    r0 = 0
+    for e, n in gl:
+        if n:
+            assert np.array_equal(y[r0:r0 + n], oracle.dense_mm_plain(p.x[r0:r0 + n], p.W[e])), (e, n)
+        r0 += n
+
+
 def test_exact_gemm_cancellation_and_ties():
     # +1 and -1 against +1, +1: the sum cancels to exactly +0
     ca = np.zeros((1, 32), int); cw = np.zeros((1, 32), int)

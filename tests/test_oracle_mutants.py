@@ -122,3 +122,49 @@ def test_every_planted_mistake_fails_a_pin(tmp_path):
     assert codes[0] == 0, "the unmutated build must pass every pin"
     survivors = [name for (name, _), rc in zip(libs[1:], codes[1:]) if rc == 0]
     assert not survivors, f"mistakes no pin caught: {survivors}"
+
+
+# Mistakes in the oracle's Python layer, planted in a copy of the package
+PY_MUTANTS = [
+    ("plain type-2 rows use the list position", "e = int(gl[g, 0]) if group_list_type == 2 else g", "e = g"),
+    ("plain activations taken as their bit patterns", "return quantize_plain(bf16_to_f64(x).astype(np.float32))",
+     "return quantize_plain(x.astype(np.float32))"),
+    ("BF16 widening shifted by 15", "return (h.astype(np.uint32) << 16).view(np.float32).astype(np.float64)",
+     "return (h.astype(np.uint32) << 15).view(np.float32).astype(np.float64)"),
+    ("plain one-row groups skipped", "        if b > a:\n            y[a:b] = dense_mm_plain(", "        if b > a + 1:\n            y[a:b] = dense_mm_plain("),
+]
+
+
+def _tree_copy(dst: str, init_text: str):
+    import shutil
+    ignore = shutil.ignore_patterns("__pycache__", "*.so", "*.so.tmp*")
+    shutil.copytree(os.path.join(ROOT, "oracle"), os.path.join(dst, "oracle"), ignore=ignore)
+    shutil.copytree(os.path.join(ROOT, "synth"), os.path.join(dst, "synth"), ignore=ignore)
+    shutil.copytree(os.path.join(ROOT, "tests", "golden"), os.path.join(dst, "tests", "golden"))
+    for f in ["tests/conftest.py", *PINS, "pytest.ini"]:
+        shutil.copy(os.path.join(ROOT, f), os.path.join(dst, f))
+    with open(os.path.join(dst, "oracle", "__init__.py"), "w") as f:
+        f.write(init_text)
+
+
+def _run_pins_in(tree: str) -> int:
+    env = dict(os.environ, OMP_NUM_THREADS="2")
+    env.pop("MACAQ_ORACLE_LIB", None)
+    return subprocess.run([sys.executable, "-m", "pytest", *PINS, "-x", "-q", "-p", "no:cacheprovider",
+                           "-m", "not gpu"], cwd=tree, env=env, capture_output=True, timeout=600).returncode
+
+
+def test_every_planted_python_mistake_fails_a_pin(tmp_path):
+    init = open(os.path.join(ROOT, "oracle", "__init__.py")).read()
+    trees = []
+    for i, (name, old, new) in enumerate([("control", None, None)] + PY_MUTANTS):
+        if old is not None:
+            assert init.count(old) == 1, f"{name}: the text to mutate must occur once"
+        tree = str(tmp_path / f"t{i}")
+        _tree_copy(tree, init if old is None else init.replace(old, new))
+        trees.append((name, tree))
+    with concurrent.futures.ThreadPoolExecutor(max_workers=4) as ex:
+        codes = list(ex.map(lambda nt: _run_pins_in(nt[1]), trees))
+    assert codes[0] == 0, "the unmutated copy must pass every pin"
+    survivors = [name for (name, _), rc in zip(trees[1:], codes[1:]) if rc == 0]
+    assert not survivors, f"mistakes no pin caught: {survivors}"
