@@ -74,12 +74,11 @@ __device__ __forceinline__ uint16_t bf16_bits(float v) {
 // with tanh taken in half precision by the hardware (tanh_h: the argument rounded
 // to FP16, relative error of the approximation about 2^-11) and no division.
 // The error in y is at most about 5e-4 |v|, far below the MXFP4 quantisation
-// noise of v.  One special-function operation per two outputs keeps the epilogue
-// under the tile's MMA time: an exponential plus a reciprocal per output (two
-// such operations at 16 per clock per SM) took twice as long as the tensor core
-// needs for a 128 x 256 tile at K = 1024.  act_value (one output) and act_pair
-// (two, in packed FP32 pair instructions) take the same steps and give the same
-// bits.
+// noise of v.  The form needs one special-function operation per two outputs;
+// an exponential plus a reciprocal per output (two such operations, at 16 per
+// clock per SM) alone took about twice the tensor core's time for a 128 x 256
+// tile at K = 1024.  act_value (one output) and act_pair (two, in packed FP32
+// pair instructions) take the same steps and give the same bits.
 constexpr float kGeluC0 = 0.7978845608028654f;    // sqrt(2/pi)
 constexpr float kGeluC1 = 0.035677408136300125f;  // sqrt(2/pi) x 0.044715
 constexpr float kFastGeluHalf = 0.851f;           // 1.702 / 2
