@@ -69,6 +69,7 @@ def test_dense_refusals_by_name(L):
     assert dense(L, N=1000) == -3
     assert dense(L, K=1000) == -3
     assert dense(L, K=128) == -3
+    assert dense(L, K=288) == -3                   # a whole number of 32-blocks, but not of 256-wide tiles
     assert dense(L, K=65536 + 256) == -3
     assert dense(L, N=65536 + 16) == -3
     assert dense(L, M=-1) == -3

@@ -27,6 +27,7 @@ int main(void) {
     CHECK(macaq_weight_code_bytes(2, 48, 256) == (size_t)2 * 256 * 128);   /* rows padded to 256 */
     CHECK(macaq_weight_code_bytes(1, 130, 1024) == 0);                     /* N % 16 != 0 */
     CHECK(macaq_weight_code_bytes(1, 1024, 1000) == 0);                    /* K % 256 != 0 */
+    CHECK(macaq_weight_code_bytes(1, 1024, 288) == 0);                     /* K % 32 == 0, K % 256 != 0 */
     CHECK(macaq_weight_code_bytes(1025, 1024, 1024) == 0);                 /* E > 1024 */
     CHECK(macaq_workspace_bytes(128, 1024, 1024, 1) == 0);                 /* fused: no scratch */
     CHECK(macaq_workspace_bytes(4096, 1024, 1024, 1) > 0);

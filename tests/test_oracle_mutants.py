@@ -168,3 +168,56 @@ def test_every_planted_python_mistake_fails_a_pin(tmp_path):
     assert codes[0] == 0, "the unmutated copy must pass every pin"
     survivors = [name for (name, _), rc in zip(trees[1:], codes[1:]) if rc == 0]
     assert not survivors, f"mistakes no pin caught: {survivors}"
+
+
+# Mistakes in the C boundary's host-side checks, planted in copies of the
+# library source and caught by the device-free boundary tests.  Each mutant is a
+# full nvcc build (about a minute), so this case runs only on request
+# (MACAQ_ABI_MUTANTS=1).
+ABI_SRC = os.path.join(ROOT, "w4a4_mxfp4_quantize_b200", "csrc", "macaq.cu")
+ABI_TESTS = ["tests/test_abi.py", "tests/test_c_header.py"]
+ABI_MUTANTS = [
+    ("act_type 3 accepted", "bool act_supported(int act) { return act == 0 || act == 1 || act == 2 || act == 4 || act == 5; }",
+     "bool act_supported(int act) { return act >= 0 && act <= 5; }"),
+    ("K % 32 accepted", "return K >= 256 && K <= 65536 && K % 256 == 0 && N >= 16", "return K >= 256 && K <= 65536 && K % 32 == 0 && N >= 16"),
+    ("N % 8 accepted", "N <= 65536 && N % 16 == 0;", "N <= 65536 && N % 8 == 0;"),
+    ("alignment of x not checked", "if (!aligned16(x) || (!plain && !aligned16(D))", "if ((!plain && !aligned16(D))"),
+    ("y overlapping x not refused", "if (overlaps(y, ybytes, x, static_cast<size_t>(M) * K * 2) ||", "if (false ||"),
+    ("bias alignment not checked", "if (!aligned16(ep.bias)) return MACAQ_ERR_ALIGN;", ""),
+    ("group_list_type -1 accepted", "if (group_list_type < 0 || group_list_type > 2) return MACAQ_ERR_GROUP_LIST_TYPE;",
+     "if (group_list_type > 2) return MACAQ_ERR_GROUP_LIST_TYPE;"),
+    ("weight rows padded to 128", "return static_cast<size_t>(E) * pad256(N) * (K / 2);",
+     "return static_cast<size_t>(E) * ((N + 127) / 128 * 128) * (K / 2);"),
+    ("status name of act_type refusal", 'case MACAQ_ERR_ACT_TYPE: return "MACAQ_ERR_ACT_TYPE";',
+     'case MACAQ_ERR_ACT_TYPE: return "MACAQ_ERR_SHAPE";'),
+]
+
+
+def _abi_build_and_test(name: str, text: str, d: str) -> int:
+    os.makedirs(d, exist_ok=True)
+    src = os.path.join(d, "macaq.cu")
+    with open(src, "w") as f:
+        f.write(text)
+    lib = os.path.join(d, "libmacaq.so")
+    import w4a4_mxfp4_quantize_b200 as mq
+    subprocess.check_call(["nvcc", *mq.NVCC_FLAGS, "-I" + os.path.join(ROOT, "include"),
+                           "-I" + os.path.dirname(ABI_SRC), "-o", lib, src])
+    code = ("import sys, pytest, w4a4_mxfp4_quantize_b200 as mq; mq._LIB_PATH = sys.argv[1]; "
+            "sys.exit(pytest.main([*sys.argv[2:], '-x', '-q', '-p', 'no:cacheprovider', '-m', 'not gpu']))")
+    return subprocess.run([sys.executable, "-c", code, lib, *ABI_TESTS], cwd=ROOT, capture_output=True,
+                          timeout=600).returncode
+
+
+@pytest.mark.skipif(os.environ.get("MACAQ_ABI_MUTANTS") != "1", reason="nvcc builds; run with MACAQ_ABI_MUTANTS=1")
+def test_every_planted_boundary_mistake_fails_a_boundary_test(tmp_path):
+    src = open(ABI_SRC).read()
+    jobs = [("control", None, None)] + ABI_MUTANTS
+    for name, old, _ in ABI_MUTANTS:
+        assert src.count(old) == 1, f"{name}: the text to mutate must occur once"
+    with concurrent.futures.ThreadPoolExecutor(max_workers=5) as ex:
+        codes = list(ex.map(lambda ij: _abi_build_and_test(
+            ij[1][0], src if ij[1][1] is None else src.replace(ij[1][1], ij[1][2]), str(tmp_path / f"a{ij[0]}")),
+            enumerate(jobs)))
+    assert codes[0] == 0, "the unmutated build must pass the boundary tests"
+    survivors = [name for (name, _, _), rc in zip(jobs[1:], codes[1:]) if rc == 0]
+    assert not survivors, f"mistakes no boundary test caught: {survivors}"
