@@ -546,11 +546,11 @@ def main():
                 line["cpu_baseline"].update(cpu_oracle_detail([pp.p for pp in problems], prepared, cores))
             except Exception as e:  # noqa: BLE001
                 line["cpu_baseline"]["detail_error"] = f"{type(e).__name__}: {e}"[:200]
-            try:  # supplementary: its failure must not cost the line
-                line["launch_floor"] = launch_floor(device, stream, flush, args.table_reps)
-            except Exception as e:  # noqa: BLE001
-                line["launch_floor"] = {"error": f"{type(e).__name__}: {e}"[:200]}
             if not args.no_table:
+                try:  # supplementary: its failure must not cost the line
+                    line["launch_floor"] = launch_floor(device, stream, flush, args.table_reps)
+                except Exception as e:  # noqa: BLE001
+                    line["launch_floor"] = {"error": f"{type(e).__name__}: {e}"[:200]}
                 line["per_workload"] = workload_table(mq, device, stream, flush, hbm_gbs, args.table_reps)
                 line["calibration"] = calibration_table(mq, device, stream, flush, hbm_gbs, args.table_reps)
         print(json.dumps(line), flush=True)
