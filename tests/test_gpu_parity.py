@@ -476,7 +476,7 @@ def test_dependent_calls_on_one_stream(M):
         mq.dense_mm(a, D1, Wq1, Ws1, N1, out=y1)
         mq.dense_mm(y1, D2, Wq2, Ws2, N2, out=y2)
         mq.dense_mm(c, D1, Wq1, Ws1, N1, out=a)    # overwrites the first call's input
-        mq.dense_mm(a_copy, D1, Wq1, Ws1, N1, out=y1)  # restore the chain for the next round
+        mq.dense_mm(a_copy, D1, Wq1, Ws1, N1, out=y1)  # restore the chain for the next iteration
         a.copy_(a_copy)
     torch.cuda.synchronize()
     assert np.array_equal(y_to_bits(y2), y_to_bits(r2))
