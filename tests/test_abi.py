@@ -1,9 +1,17 @@
 """Host-side checks of the C ABI that need no GPU: the library loads, exports
 every symbol include/macaq.h declares, and refuses bad arguments by name
-before touching the device."""
+before touching the device.
+
+The refusal tests pass made-up device addresses.  They rely on the library
+refusing each call before any launch, so they run only in a process that sees
+no CUDA device: where a GPU is visible, one test re-runs them in a child
+process with CUDA_VISIBLE_DEVICES set empty.  A broken host check then ends in
+a named CUDA error there, never in a kernel reading unmapped memory."""
 import ctypes
 import os
 import re
+import subprocess
+import sys
 
 import pytest
 
@@ -40,7 +48,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.macaq_abi_version() == 3
+    assert L.macaq_abi_version() == 4
     for code, name in mq.STATUS.items():
         assert L.macaq_status_string(code).decode() == name
     assert L.macaq_status_string(-99).decode() == "MACAQ_ERR_UNKNOWN"
@@ -57,6 +65,26 @@ def test_weight_sizes(L):
     assert L.macaq_unfused_workspace_bytes(16, 1024) == 4096 + 128 * (512 + 32)
 
 
+def _device_visible() -> bool:
+    import torch
+    return torch.cuda.is_available()
+
+
+# every test below that passes made-up addresses carries this mark
+hidden_device = pytest.mark.skipif(_device_visible(), reason="made-up device addresses: run with the device hidden")
+
+
+def test_fake_address_refusals_run_with_the_device_hidden():
+    if not _device_visible():
+        pytest.skip("no device visible: the refusal tests run in this process")
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.abspath(__file__), "-x", "-q", "-p",
+                        "no:cacheprovider", "-m", "not gpu", "-k", "by_name or no_gpu"],
+                       cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+    assert " passed" in r.stdout and "skipped" not in r.stdout.splitlines()[-1], r.stdout[-2000:]
+
+
 P = ctypes.c_void_p
 A, B, C, Dp, Y = (P(i << 32) for i in range(1, 6))
 
@@ -65,6 +93,7 @@ def dense(L, x=A, d=B, wq=C, ws=Dp, y=Y, M=16, N=1024, K=1024):
     return L.macaq_dense_mm(x, d, wq, ws, y, M, N, K, None, 0, None, None)
 
 
+@hidden_device
 def test_dense_refusals_by_name(L):
     assert dense(L, N=1000) == -3
     assert dense(L, K=1000) == -3
@@ -80,6 +109,7 @@ def test_dense_refusals_by_name(L):
     assert dense(L, M=0, x=None) == 0            # M = 0 is a no-op
 
 
+@hidden_device
 def test_grouped_refusals_by_name(L):
     gl = P(9 << 32)
 
@@ -96,6 +126,7 @@ def test_grouped_refusals_by_name(L):
     assert g(glp=P((9 << 32) + 4)) == -2
 
 
+@hidden_device
 def test_epilogue_refusals_by_name(L):
     bias = P(11 << 32)
 
@@ -115,6 +146,7 @@ def test_epilogue_refusals_by_name(L):
     assert g(act=2, b=None) == -11                # accepted; the missing workspace is the next refusal
 
 
+@hidden_device
 def test_calibration_refusals_by_name(L):
     x, W, D, gl = P(1 << 32), P(2 << 32), P(3 << 32), P(4 << 32)
 
@@ -133,9 +165,67 @@ def test_calibration_refusals_by_name(L):
     assert c(D=P((1 << 32) + 1024)) == -5   # D inside x
 
 
+@hidden_device
 def test_no_gpu_means_a_named_cuda_error_not_a_fallback(L):
     import torch
     if torch.cuda.is_available():
         pytest.skip("GPU present")
     assert dense(L) == -8
     assert L.macaq_dense_mm_ex(A, B, C, Dp, None, 5, Y, 16, 1024, 1024, None, 0, None, None) == -8
+
+
+@hidden_device
+def test_noalloc_refusals_by_name(L):
+    # the size check of the fixed scratch buffer comes before any device access
+    M, K, N = 65536, 1024, 128  # needs ~34 MiB of scratch, above the 8 MiB buffer
+    assert L.macaq_dense_mm_noalloc(A, B, C, Dp, Y, M, N, K, None, None) == -11
+    assert L.macaq_dense_mm_noalloc(A, B, C, Dp, Y, 16, 1000, 1024, None, None) == -3
+    assert L.macaq_dense_mm_noalloc(None, B, C, Dp, Y, 16, 1024, 1024, None, None) == -1
+
+
+@hidden_device
+def test_probe_and_plan_refusals_by_name(L):
+    import ctypes as ct
+    bt, s, c = ct.c_int(0), ct.c_int(0), ct.c_int(0)
+    assert L.macaq_fused_plan(129, 1024, 1024, ct.byref(bt), ct.byref(s), ct.byref(c)) == -3  # fused: M <= 128
+    assert L.macaq_fused_plan(16, 1000, 1024, ct.byref(bt), ct.byref(s), ct.byref(c)) == -3
+    assert L.macaq_fused_plan(16, 1024, 1024, None, ct.byref(s), ct.byref(c)) == -1
+
+    def probe(M=16, bt=16, s=1, c=0, codes=P(12 << 32), scales=P(13 << 32), K=1024):
+        return L.macaq_fused_probe(A, B, C, Dp, Y, M, 1024, K, bt, s, c, 0, codes, scales, None, None)
+
+    assert probe(M=129) == -3
+    assert probe(bt=48) == -3
+    assert probe(s=3) == -3                    # 3 does not divide K/256 = 4
+    assert probe(s=9, K=4608) == -3            # at most 8 CTAs per cluster
+    assert probe(c=-1) == -3
+    assert probe(c=9) == -3
+    assert probe(scales=None) == -1            # codes and scales come together
+    assert probe(codes=P((12 << 32) + 8)) == -2
+    assert probe(codes=P((5 << 32) + 64)) == -5   # codes inside y
+    assert L.macaq_test_wait_expiry(10, P(12 << 32), None) == -3      # below 1 us
+    assert L.macaq_test_wait_expiry(2 * 10 ** 9, P(12 << 32), None) == -3
+    assert L.macaq_test_wait_expiry(10 ** 6, None, None) == -1
+
+
+@hidden_device
+def test_weight_list_and_transposed_refusals_by_name(L):
+    gl, wql, wsl = P(9 << 32), P(14 << 32), P(15 << 32)
+
+    def g(E=4, t=1, q=wql, w=wsl, act=0, N=1024):
+        return L.macaq_grouped_mm_list(A, B, q, w, gl, t, E, None, act, Y, 64, N, 1024, None, 0, None, None)
+
+    assert g(E=0) == -6
+    assert g(t=3) == -7
+    assert g(q=None) == -1
+    assert g(w=P((15 << 32) + 8)) == -2           # the table itself must be 16-byte aligned
+    assert g(q=P((5 << 32) + 64)) == -5           # a table inside y
+    assert g(act=3) == -13
+    assert g(N=24) == -3
+    assert g() == -11                              # accepted; the missing workspace is the next refusal
+    W, D, Wq, Ws = P(1 << 32), P(2 << 32), P(3 << 32), P(4 << 32)
+    assert L.macaq_prepare_weights_transposed(W, D, 1, 1000, 1024, Wq, Ws, None) == -3
+    assert L.macaq_prepare_weights_transposed(W, D, 0, 1024, 1024, Wq, Ws, None) == -6
+    assert L.macaq_prepare_weights_transposed(None, D, 1, 1024, 1024, Wq, Ws, None) == -1
+    assert L.macaq_prepare_weights_transposed(W, P((2 << 32) + 4), 1, 1024, 1024, Wq, Ws, None) == -2
+

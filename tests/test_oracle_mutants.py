@@ -132,6 +132,9 @@ PY_MUTANTS = [
     ("BF16 widening shifted by 15", "return (h.astype(np.uint32) << 16).view(np.float32).astype(np.float64)",
      "return (h.astype(np.uint32) << 15).view(np.float32).astype(np.float64)"),
     ("plain one-row groups skipped", "        if b > a:\n            y[a:b] = dense_mm_plain(", "        if b > a + 1:\n            y[a:b] = dense_mm_plain("),
+    ("weight-list type-2 rows use the list position", "e = int(gl[j, 0]) if group_list_type == 2 else j", "e = j"),
+    ("weight-list entries use expert 0's D", "y[a:b] = dense_mm(x[a:b], D[e], W_list[e], nthreads)",
+     "y[a:b] = dense_mm(x[a:b], D[0], W_list[e], nthreads)"),
 ]
 
 
@@ -148,7 +151,7 @@ def _tree_copy(dst: str, init_text: str):
 
 
 def _run_pins_in(tree: str) -> int:
-    env = dict(os.environ, OMP_NUM_THREADS="2")
+    env = dict(os.environ, OMP_NUM_THREADS="2", CUDA_VISIBLE_DEVICES="")
     env.pop("MACAQ_ORACLE_LIB", None)
     return subprocess.run([sys.executable, "-m", "pytest", *PINS, "-x", "-q", "-p", "no:cacheprovider",
                            "-m", "not gpu"], cwd=tree, env=env, capture_output=True, timeout=600).returncode
@@ -204,11 +207,20 @@ def _abi_build_and_test(name: str, text: str, d: str) -> int:
                            "-I" + os.path.dirname(ABI_SRC), "-o", lib, src])
     code = ("import sys, pytest, w4a4_mxfp4_quantize_b200 as mq; mq._LIB_PATH = sys.argv[1]; "
             "sys.exit(pytest.main([*sys.argv[2:], '-x', '-q', '-p', 'no:cacheprovider', '-m', 'not gpu']))")
-    return subprocess.run([sys.executable, "-c", code, lib, *ABI_TESTS], cwd=ROOT, capture_output=True,
+    # The boundary tests pass made-up device addresses; a mutant that lets one
+    # through must meet a process that sees no device, never launch a kernel.
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    return subprocess.run([sys.executable, "-c", code, lib, *ABI_TESTS], cwd=ROOT, env=env, capture_output=True,
                           timeout=600).returncode
 
 
+def _device_visible() -> bool:
+    import torch
+    return torch.cuda.is_available()
+
+
 @pytest.mark.skipif(os.environ.get("MACAQ_ABI_MUTANTS") != "1", reason="nvcc builds; run with MACAQ_ABI_MUTANTS=1")
+@pytest.mark.skipif(_device_visible(), reason="mutated host checks: run only where no device is visible")
 def test_every_planted_boundary_mistake_fails_a_boundary_test(tmp_path):
     src = open(ABI_SRC).read()
     jobs = [("control", None, None)] + ABI_MUTANTS
