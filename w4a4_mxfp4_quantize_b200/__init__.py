@@ -13,6 +13,7 @@ torch_npu.npu_grouped_matmul's group_list / group_list_type.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import subprocess
@@ -96,6 +97,13 @@ _SIG = {
     "macaq_dense_mm_plain": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, ctypes.c_size_t, _P, _P]),
     "macaq_grouped_mm_plain": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _I64, _P, _I64, _I64, _I64, _P,
                                               ctypes.c_size_t, _P, _P]),
+    "macaq_fused_plan": (ctypes.c_int, [_I64, _I64, _I64, _P, _P, _P]),
+    "macaq_fused_probe": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, ctypes.c_int, _P, _P, _P, _P]),
+    "macaq_test_wait_expiry": (ctypes.c_int, [_I64, _P, _P]),
+    "macaq_prepare_weights_transposed": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _P]),
+    "macaq_grouped_mm_list": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P, _I64,
+                                             _I64, _I64, _P, ctypes.c_size_t, _P, _P]),
 }
 
 
@@ -158,6 +166,14 @@ def _weights_args(Wq, Ws, E: int, N: int, K: int):
     _arg(Ws, "Ws", torch.uint8, min_numel=sb)
 
 
+def _on(stream):
+    """Allocations for a call (its output, workspace and result tensors) are made
+    on the stream its kernels run on: the caching allocator then hands their
+    memory to no other stream while those kernels may still use it, and the
+    workspace's zero fill is ordered before them."""
+    return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+
+
 def _require_cuda(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
@@ -200,7 +216,8 @@ def workspace(nbytes: int, device: torch.device, stream=None, given: torch.Tenso
     key = (device.index, s.cuda_stream)
     buf = _ws.get(key)
     if buf is None or buf.numel() < nbytes:
-        buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        with _on(stream):
+            buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
         _ws[key] = buf
     return buf
 
@@ -231,11 +248,64 @@ def prepare_weights(W: torch.Tensor, D: torch.Tensor, stream=None) -> tuple[torc
     qb, sb = weight_bytes(E, N, K)
     if qb == 0:
         raise MacaqError(-3, "prepare_weights")
-    Wq = torch.empty(qb, dtype=torch.uint8, device=W.device)
-    Ws = torch.empty(sb, dtype=torch.uint8, device=W.device)
+    with _on(stream):
+        Wq = torch.empty(qb, dtype=torch.uint8, device=W.device)
+        Ws = torch.empty(sb, dtype=torch.uint8, device=W.device)
     _check(lib().macaq_prepare_weights(_ptr(W), _ptr(D), E, N, K, _ptr(Wq), _ptr(Ws), _stream_ptr(stream)),
            "macaq_prepare_weights")
     return Wq, Ws
+
+
+def prepare_weights_transposed(W_kn: torch.Tensor, D: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Offline, from weights stored transposed: W_kn fp32 [K, N] or [E, K, N], D fp32
+    [K] or [E, K] -> the same (Wq, Ws) as prepare_weights on the [E, N, K] weights."""
+    if W_kn.dim() == 2:
+        W_kn = W_kn.unsqueeze(0)
+    if D.dim() == 1:
+        D = D.unsqueeze(0)
+    _arg(W_kn, "W_kn", torch.float32, ndim=3)
+    E, K, N = W_kn.shape
+    _arg(D, "D", torch.float32, min_numel=E * K)
+    _require_cuda(W_kn, D)
+    qb, sb = weight_bytes(E, N, K)
+    if qb == 0:
+        raise MacaqError(-3, "prepare_weights_transposed")
+    with _on(stream):
+        Wq = torch.empty(qb, dtype=torch.uint8, device=W_kn.device)
+        Ws = torch.empty(sb, dtype=torch.uint8, device=W_kn.device)
+    _check(lib().macaq_prepare_weights_transposed(_ptr(W_kn), _ptr(D), E, N, K, _ptr(Wq), _ptr(Ws),
+                                                  _stream_ptr(stream)), "macaq_prepare_weights_transposed")
+    return Wq, Ws
+
+
+def grouped_mm_list(x: torch.Tensor, D: torch.Tensor, Wq_list, Ws_list, group_list: torch.Tensor,
+                    group_list_type: int, N: int, out: torch.Tensor | None = None,
+                    status: torch.Tensor | None = None, stream=None, ws: torch.Tensor | None = None,
+                    bias: torch.Tensor | None = None, act_type: int = ACT_NONE) -> torch.Tensor:
+    """Grouped MACAQ linear with one prepared weight pair per expert (npu_grouped_matmul's
+    weight as a list): Wq_list[e], Ws_list[e] from prepare_weights on expert e's [N, K]."""
+    _arg(x, "x", torch.bfloat16, ndim=2)
+    _arg(group_list, "group_list", torch.int64)
+    E = _groups(group_list, group_list_type)
+    if len(Wq_list) != E or len(Ws_list) != E:
+        raise ValueError(f"Wq_list and Ws_list need {E} entries, one per group_list entry")
+    M, K = x.shape
+    _arg(D, "D", torch.float32, min_numel=E * K)
+    for e in range(E):
+        _weights_args(Wq_list[e], Ws_list[e], 1, N, K)
+    _arg(status, "status", torch.int32, min_numel=1)
+    _require_cuda(x, D, group_list, out, status, *Wq_list, *Ws_list)
+    _check_bias(bias, (E, N))
+    with _on(stream):
+        y = _output(out, M, N, x.device)
+        tables = torch.tensor([[w.data_ptr() for w in Wq_list], [w.data_ptr() for w in Ws_list]],
+                              dtype=torch.int64).to(x.device, non_blocking=False)
+    L = lib()
+    ws = workspace(int(L.macaq_workspace_bytes(M, N, K, E)), x.device, stream, ws)
+    _check(L.macaq_grouped_mm_list(_ptr(x), _ptr(D), _ptr(tables[0]), _ptr(tables[1]), _ptr(group_list),
+                                   int(group_list_type), E, _ptr(bias), int(act_type), _ptr(y), M, N, K, _ptr(ws),
+                                   _nbytes(ws), _ptr(status), _stream_ptr(stream)), "macaq_grouped_mm_list")
+    return y
 
 
 def _check_bias(bias, shape):
@@ -260,7 +330,8 @@ def calibrate_d(x_cal: torch.Tensor, W: torch.Tensor, group_list: torch.Tensor |
     if KW != K:
         raise ValueError(f"W has {KW} input channels, x_cal {K}")
     _require_cuda(x_cal, W, group_list)
-    D = torch.empty((E, K), dtype=torch.float32, device=W.device)
+    with _on(stream):
+        D = torch.empty((E, K), dtype=torch.float32, device=W.device)
     _check(lib().macaq_calibrate_d(_ptr(x_cal), T, _ptr(W), E, N, K, _ptr(group_list), int(group_list_type),
                                    _ptr(D), _stream_ptr(stream)), "macaq_calibrate_d")
     return D
@@ -276,7 +347,8 @@ def dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tenso
     _require_cuda(x, D, Wq, Ws, out, status)
     M, K = x.shape
     _check_bias(bias, (N,))
-    y = _output(out, M, N, x.device)
+    with _on(stream):
+        y = _output(out, M, N, x.device)
     L = lib()
     need = int(L.macaq_workspace_bytes(M, N, K, 1))
     ws = workspace(need, x.device, stream, ws)
@@ -331,7 +403,8 @@ def grouped_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Ten
     _require_cuda(x, D, Wq, Ws, group_list, out, status)
     M, K = x.shape
     _check_bias(bias, (E, N))
-    y = _output(out, M, N, x.device)
+    with _on(stream):
+        y = _output(out, M, N, x.device)
     L = lib()
     need = int(L.macaq_workspace_bytes(M, N, K, E))
     ws = workspace(need, x.device, stream, ws)
@@ -358,8 +431,9 @@ def prepare_weights_plain(W: torch.Tensor, stream=None) -> tuple[torch.Tensor, t
     qb, sb = weight_bytes(E, N, K)
     if qb == 0:
         raise MacaqError(-3, "prepare_weights_plain")
-    Wq = torch.empty(qb, dtype=torch.uint8, device=W.device)
-    Ws = torch.empty(sb, dtype=torch.uint8, device=W.device)
+    with _on(stream):
+        Wq = torch.empty(qb, dtype=torch.uint8, device=W.device)
+        Ws = torch.empty(sb, dtype=torch.uint8, device=W.device)
     _check(lib().macaq_prepare_weights_plain(_ptr(W), E, N, K, _ptr(Wq), _ptr(Ws), _stream_ptr(stream)),
            "macaq_prepare_weights_plain")
     return Wq, Ws
@@ -371,7 +445,8 @@ def dense_mm_plain(x: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: int, 
     _dense_args(x, None, Wq, Ws, N, status)
     _require_cuda(x, Wq, Ws, out, status)
     M, K = x.shape
-    y = _output(out, M, N, x.device)
+    with _on(stream):
+        y = _output(out, M, N, x.device)
     L = lib()
     ws = workspace(int(L.macaq_workspace_bytes(M, N, K, 1)), x.device, stream, ws)
     _check(L.macaq_dense_mm_plain(_ptr(x), _ptr(Wq), _ptr(Ws), _ptr(y), M, N, K, _ptr(ws), _nbytes(ws),
@@ -387,7 +462,8 @@ def grouped_mm_plain(x: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, group_
     E = _grouped_args(x, None, Wq, Ws, group_list, group_list_type, N, status)
     _require_cuda(x, Wq, Ws, group_list, out, status)
     M, K = x.shape
-    y = _output(out, M, N, x.device)
+    with _on(stream):
+        y = _output(out, M, N, x.device)
     L = lib()
     ws = workspace(int(L.macaq_workspace_bytes(M, N, K, E)), x.device, stream, ws)
     _check(L.macaq_grouped_mm_plain(_ptr(x), _ptr(Wq), _ptr(Ws), _ptr(group_list), int(group_list_type), E,
@@ -403,7 +479,8 @@ def unfused_dense_mm(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: tor
     _dense_args(x, D, Wq, Ws, N, status)
     _require_cuda(x, D, Wq, Ws, out, status)
     M, K = x.shape
-    y = _output(out, M, N, x.device)
+    with _on(stream):
+        y = _output(out, M, N, x.device)
     L = lib()
     need = int(L.macaq_unfused_workspace_bytes(M, K))
     ws = workspace(need, x.device, stream, ws)
@@ -421,7 +498,8 @@ def dense_mm_noalloc(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: tor
     _dense_args(x, D, Wq, Ws, N, status)
     _require_cuda(x, D, Wq, Ws, out, status)
     M, K = x.shape
-    y = _output(out, M, N, x.device)
+    with _on(stream):
+        y = _output(out, M, N, x.device)
     _check(lib().macaq_dense_mm_noalloc(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(y), M, N, K, _ptr(status),
                                         _stream_ptr(stream)), "macaq_dense_mm_noalloc")
     return y
@@ -432,11 +510,47 @@ def quantize_activations(x: torch.Tensor, D: torch.Tensor, stream=None) -> tuple
     _dense_args(x, D, None, None, 0, None)
     _require_cuda(x, D)
     M, K = x.shape
-    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
-    scales = torch.empty((M, K // 32), dtype=torch.uint8, device=x.device)
+    with _on(stream):
+        codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+        scales = torch.empty((M, K // 32), dtype=torch.uint8, device=x.device)
     _check(lib().macaq_quantize_activations(_ptr(x), _ptr(D), _ptr(codes), _ptr(scales), M, K,
                                             _stream_ptr(stream)), "macaq_quantize_activations")
     return codes, scales
+
+
+def fused_plan(M: int, N: int, K: int) -> tuple[int, int, int]:
+    """(token tile, K split, N share) that dense_mm's fused kernel uses for this shape (M <= 128)."""
+    bt, s, c = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().macaq_fused_plan(M, N, K, ctypes.byref(bt), ctypes.byref(s), ctypes.byref(c)), "macaq_fused_plan")
+    return bt.value, s.value, c.value
+
+
+def fused_probe(x: torch.Tensor, D: torch.Tensor | None, Wq: torch.Tensor, Ws: torch.Tensor, N: int,
+                token_tile: int, k_split: int, n_share: int = 0, plain: bool = False, dump: bool = True,
+                stream=None):
+    """Test only: the fused kernel with a given plan; returns (y, codes, scales), the
+    last two being its own activation operand tiles in canonical form (None
+    without dump)."""
+    _dense_args(x, None if plain else D, Wq, Ws, N, None)
+    _require_cuda(x, D, Wq, Ws)
+    M, K = x.shape
+    with _on(stream):
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+        codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device) if dump else None
+        scales = torch.empty((M, K // 32), dtype=torch.uint8, device=x.device) if dump else None
+    _check(lib().macaq_fused_probe(_ptr(x), None if plain else _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(y), M, N, K,
+                                   int(token_tile), int(k_split), int(n_share), int(bool(plain)), _ptr(codes),
+                                   _ptr(scales), None, _stream_ptr(stream)), "macaq_fused_probe")
+    return y, codes, scales
+
+
+def run_wait_expiry(timeout_ns: int, stream=None) -> torch.Tensor:
+    """Test only: run the kernels' bounded wait out on purpose; returns the device status word."""
+    with _on(stream):
+        status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    _check(lib().macaq_test_wait_expiry(int(timeout_ns), _ptr(status), _stream_ptr(stream)),
+           "macaq_test_wait_expiry")
+    return status
 
 
 def export_weights(Wq: torch.Tensor, Ws: torch.Tensor, E: int, N: int, K: int,
@@ -444,8 +558,9 @@ def export_weights(Wq: torch.Tensor, Ws: torch.Tensor, E: int, N: int, K: int,
     """Prepared tile images -> canonical codes [E, N, K/2] and scales [E, N, K/32]."""
     _weights_args(Wq, Ws, E, N, K)
     _require_cuda(Wq, Ws)
-    codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=Wq.device)
-    scales = torch.empty((E, N, K // 32), dtype=torch.uint8, device=Wq.device)
+    with _on(stream):
+        codes = torch.empty((E, N, K // 2), dtype=torch.uint8, device=Wq.device)
+        scales = torch.empty((E, N, K // 32), dtype=torch.uint8, device=Wq.device)
     _check(lib().macaq_export_weights(_ptr(Wq), _ptr(Ws), _ptr(codes), _ptr(scales), E, N, K,
                                       _stream_ptr(stream)), "macaq_export_weights")
     return codes, scales
@@ -456,8 +571,9 @@ def mx_encode_blocks(v: torch.Tensor, stream=None) -> tuple[torch.Tensor, torch.
     _arg(v, "v", torch.float32)
     _require_cuda(v)
     n = v.numel()
-    codes = torch.empty(n // 2, dtype=torch.uint8, device=v.device)
-    scales = torch.empty(n // 32, dtype=torch.uint8, device=v.device)
+    with _on(stream):
+        codes = torch.empty(n // 2, dtype=torch.uint8, device=v.device)
+        scales = torch.empty(n // 32, dtype=torch.uint8, device=v.device)
     _check(lib().macaq_mx_encode_blocks(_ptr(v), _ptr(codes), _ptr(scales), n, _stream_ptr(stream)),
            "macaq_mx_encode_blocks")
     return codes, scales
