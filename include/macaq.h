@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define MACAQ_ABI_VERSION 3
+#define MACAQ_ABI_VERSION 4
 
 #define MACAQ_OK 0
 #define MACAQ_ERR_NULL (-1)               /* a required pointer is NULL */
@@ -95,6 +95,14 @@ size_t macaq_weight_scale_bytes(int64_t E, int64_t N, int64_t K);
  * Synchronises `stream` once to check D (MACAQ_ERR_BAD_D). */
 int macaq_prepare_weights(const float *W_dev, const float *D_dev, int64_t E, int64_t N, int64_t K,
                           uint8_t *Wq_dev, uint8_t *Ws_dev, void *stream);
+
+/* The same preparation from weights stored transposed: W_kn_dev fp32
+ * [E, K, N] row-major (element (n, k) of expert e at (e K + k) N + n), the
+ * npu_grouped_matmul page's transposed weight layout (constraints: the weight
+ * may be given transposed).  Produces the same Wq/Ws as macaq_prepare_weights
+ * on the [E, N, K] weights, with the same checks and synchronisation. */
+int macaq_prepare_weights_transposed(const float *W_kn_dev, const float *D_dev, int64_t E, int64_t N, int64_t K,
+                                     uint8_t *Wq_dev, uint8_t *Ws_dev, void *stream);
 
 /* Offline calibration of the channel factors D.  The MACAQ page lists
  * calibration among the offline steps ("Calibration, weight transformation
@@ -192,6 +200,24 @@ int macaq_grouped_mm_ex(const uint16_t *x_dev, const float *D_dev, const uint8_t
                         int act_type, uint16_t *y_dev, int64_t M, int64_t N, int64_t K, void *workspace_dev,
                         size_t workspace_bytes, int32_t *status_dev, void *stream);
 
+/* Grouped MACAQ linear with one weight tensor per expert: npu_grouped_matmul's
+ * weight given as a list of tensors (parameter weight, List[Tensor]; the
+ * single-x / several-weight / single-y case of its constraints), with its
+ * bias and act_type as in macaq_grouped_mm_ex.
+ *   Wq_list_dev, Ws_list_dev: device arrays of E uint64 device addresses; entry
+ *     e is expert e's code / scale images, each prepared separately with
+ *     macaq_prepare_weights(E = 1) for this N and K, anywhere in memory.  The
+ *     tables are read on the device, never by the host: an address that is
+ *     NULL, not 16-byte aligned or overlapping y writes MACAQ_ERR_NULL,
+ *     MACAQ_ERR_ALIGN or MACAQ_ERR_ALIAS to *status_dev and leaves y as it was.
+ *   D_dev fp32 [E, K]; bias_dev [E, N] or NULL; group_list, workspace and all
+ *     other arguments as in macaq_grouped_mm_ex.
+ * The result is that of macaq_grouped_mm_ex on the same weights stacked. */
+int macaq_grouped_mm_list(const uint16_t *x_dev, const float *D_dev, const uint64_t *Wq_list_dev,
+                          const uint64_t *Ws_list_dev, const int64_t *group_list_dev, int group_list_type, int64_t E,
+                          const float *bias_dev, int act_type, uint16_t *y_dev, int64_t M, int64_t N, int64_t K,
+                          void *workspace_dev, size_t workspace_bytes, int32_t *status_dev, void *stream);
+
 /* ------------------------------------------------------------------ */
 /* Plain MXFP4 W4A4 baseline                                           */
 /* ------------------------------------------------------------------ */
@@ -219,10 +245,41 @@ int macaq_grouped_mm_plain(const uint16_t *x_dev, const uint8_t *Wq_dev, const u
 /* ------------------------------------------------------------------ */
 
 /* The activation prologue alone, writing canonical codes [M, K/2] (element
- * 2j in the low nibble of byte j) and scales [M, K/32]. Same device code as
- * the fused kernels. */
+ * 2j in the low nibble of byte j) and scales [M, K/32].  It runs the
+ * one-block-per-thread form of the prologue, the form of the quantise-once
+ * path (dense M > 128 and grouped calls); the fused small-M kernel computes the
+ * same values with each block split over a lane pair, and its own codes and
+ * scales are read out by macaq_fused_probe. */
 int macaq_quantize_activations(const uint16_t *x_dev, const float *D_dev, uint8_t *codes_dev,
                                uint8_t *scales_dev, int64_t M, int64_t K, void *stream);
+
+/* The plan macaq_dense_mm chooses on the current device for a call of this
+ * shape with 1 <= M <= 128 (the fused kernel): the token tile (rows of x per
+ * CTA: 16, 32, 64 or 128) and the K split (CTAs of a thread-block cluster that
+ * share one output tile's K range, reducing their partial sums in rank
+ * order). */
+int macaq_fused_plan(int64_t M, int64_t N, int64_t K, int *token_tile, int *k_split);
+
+/* The fused small-M kernel of macaq_dense_mm (1 <= M <= 128) with a given plan
+ * (token_tile and k_split as macaq_fused_plan reports them; k_split divides
+ * K/256 and is at most 8), writing y as macaq_dense_mm does.  plain != 0 runs
+ * the plain MXFP4 prologue of macaq_dense_mm_plain (D unused, may be NULL).
+ * With codes_dev and scales_dev given, the activation operand of every K tile
+ * is also copied out just before the tensor core reads it, exactly as the
+ * kernel's prologue placed it in shared memory: canonical codes [M, K/2] and
+ * E8M0 scales [M, K/32] of the fused path itself (both NULL: no copy).
+ * A plan the kernel or the device cannot run returns MACAQ_ERR_SHAPE. */
+int macaq_fused_probe(const uint16_t *x_dev, const float *D_dev, const uint8_t *Wq_dev, const uint8_t *Ws_dev,
+                      uint16_t *y_dev, int64_t M, int64_t N, int64_t K, int token_tile, int k_split, int plain,
+                      uint8_t *codes_dev, uint8_t *scales_dev, int32_t *status_dev, void *stream);
+
+/* The kernels' bounded wait run out on purpose: one CTA waits, with the wait
+ * every kernel uses on its mbarriers, on a barrier that nothing arrives on,
+ * for timeout_ns (1 us .. 1 s); a second warp's wait on it must then give up
+ * at the CTA's abort flag.  Nothing asynchronous is issued, so nothing is in
+ * flight when the waits end.  Writes MACAQ_ERR_DEVICE_TIMEOUT to *status_dev
+ * when both waits gave up as designed, MACAQ_OK otherwise. */
+int macaq_test_wait_expiry(int64_t timeout_ns, int32_t *status_dev, void *stream);
 
 /* Prepared (tiled) weights -> canonical codes [E, N, K/2] and scales
  * [E, N, K/32]. */

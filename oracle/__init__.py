@@ -354,6 +354,32 @@ def grouped_mm(x_bf16, D, W, group_list, group_list_type: int, nthreads: int = 0
     return int(st), y
 
 
+def grouped_mm_list(x_bf16, D, W_list, group_list, group_list_type: int, nthreads: int = 0):
+    """Grouped MACAQ linear with one weight tensor per expert (npu_grouped_matmul,
+    parameter weight given as a list of tensors, the single-x / several-weight /
+    single-y case of its constraints).  The rows of list entry j (group_list as in
+    grouped_mm) are the dense MACAQ linear of the expert e the entry uses (e = j
+    for types 0 and 1, the named index for type 2) with D[e] and W_list[e] [N, K].
+    Written as that definition (one dense call per entry), independently of the
+    C routine behind grouped_mm.  Returns (status, y bf16 bits [M, N])."""
+    x = _c(x_bf16, np.uint16)
+    D = _c(D, np.float32)
+    M = x.shape[0]
+    E = len(W_list)
+    N = W_list[0].shape[0]
+    st, off = group_offsets(group_list, group_list_type, M)
+    y = np.zeros((M, N), np.uint16)
+    if st != OK:
+        return st, y
+    gl = _c(group_list, np.int64)
+    for j in range(E):
+        a, b = int(off[j]), int(off[j + 1])
+        e = int(gl[j, 0]) if group_list_type == 2 else j
+        if b > a:
+            y[a:b] = dense_mm(x[a:b], D[e], W_list[e], nthreads)
+    return OK, y
+
+
 def grouped_mm_ex(x_bf16, D, W, group_list, group_list_type: int, bias=None, act_type: int = 0,
                   nthreads: int = 0):
     """Grouped MACAQ linear with per-expert bias [E, N] and activation.

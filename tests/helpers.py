@@ -70,3 +70,21 @@ def dequant_matmul_bf16(qa, sa, qw, sw) -> np.ndarray:
     B = oracle.dequantize(qw, sw)
     y = (A @ B.T) / 32.0
     return synth.to_bf16_bits(y.astype(np.float32))
+
+
+def assert_mx_equal(codes, scales, ref_codes, ref_scales, label: str = ""):
+    """Activation MX encodings compared bit-exactly: the E8M0 scales everywhere,
+    the E2M1 codes of every block whose scale is finite.  A block whose scale is
+    255 is NaN as a whole (OCP MX: a NaN scale makes every element of its block
+    NaN), so its element codes carry no value.  Such blocks arise only where x/D
+    leaves the binary32 range (inf - inf in the butterfly), and the signs of the
+    NaN elements then follow each machine's NaN propagation (IEEE 754 leaves the
+    sign of a NaN result unspecified): the GPU and the host differ there."""
+    scales, ref_scales = np.asarray(scales), np.asarray(ref_scales)
+    assert np.array_equal(scales, ref_scales), f"{label}: scales differ from the oracle"
+    finite = ref_scales != 255
+    c = np.asarray(codes).reshape(*finite.shape, 16)
+    r = np.asarray(ref_codes).reshape(*finite.shape, 16)
+    bad = np.argwhere((c != r).any(axis=-1) & finite)
+    assert bad.size == 0, f"{label}: codes differ from the oracle in {len(bad)} blocks, first {bad[:3].tolist()}"
+

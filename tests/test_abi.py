@@ -186,20 +186,18 @@ def test_noalloc_refusals_by_name(L):
 @hidden_device
 def test_probe_and_plan_refusals_by_name(L):
     import ctypes as ct
-    bt, s, c = ct.c_int(0), ct.c_int(0), ct.c_int(0)
-    assert L.macaq_fused_plan(129, 1024, 1024, ct.byref(bt), ct.byref(s), ct.byref(c)) == -3  # fused: M <= 128
-    assert L.macaq_fused_plan(16, 1000, 1024, ct.byref(bt), ct.byref(s), ct.byref(c)) == -3
-    assert L.macaq_fused_plan(16, 1024, 1024, None, ct.byref(s), ct.byref(c)) == -1
+    bt, s = ct.c_int(0), ct.c_int(0)
+    assert L.macaq_fused_plan(129, 1024, 1024, ct.byref(bt), ct.byref(s)) == -3   # fused kernel: M <= 128
+    assert L.macaq_fused_plan(16, 1000, 1024, ct.byref(bt), ct.byref(s)) == -3
+    assert L.macaq_fused_plan(16, 1024, 1024, None, ct.byref(s)) == -1
 
-    def probe(M=16, bt=16, s=1, c=0, codes=P(12 << 32), scales=P(13 << 32), K=1024):
-        return L.macaq_fused_probe(A, B, C, Dp, Y, M, 1024, K, bt, s, c, 0, codes, scales, None, None)
+    def probe(M=16, bt=16, s=1, codes=P(12 << 32), scales=P(13 << 32), K=1024):
+        return L.macaq_fused_probe(A, B, C, Dp, Y, M, 1024, K, bt, s, 0, codes, scales, None, None)
 
     assert probe(M=129) == -3
     assert probe(bt=48) == -3
     assert probe(s=3) == -3                    # 3 does not divide K/256 = 4
     assert probe(s=9, K=4608) == -3            # at most 8 CTAs per cluster
-    assert probe(c=-1) == -3
-    assert probe(c=9) == -3
     assert probe(scales=None) == -1            # codes and scales come together
     assert probe(codes=P((12 << 32) + 8)) == -2
     assert probe(codes=P((5 << 32) + 64)) == -5   # codes inside y

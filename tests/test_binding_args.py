@@ -99,3 +99,19 @@ def test_prepare_and_calibrate_refusals():
         mq.mx_encode_blocks(torch.zeros(64, dtype=torch.float64))
     with pytest.raises(ValueError, match="Wq holds"):
         mq.export_weights(torch.zeros(10, dtype=torch.uint8), torch.zeros(10, dtype=torch.uint8), 1, N, K)
+
+
+def test_weight_list_and_transposed_refusals():
+    qb, sb = mq.weight_bytes(1, N, K)
+    a = grouped_args()
+    wq = [torch.zeros(qb, dtype=torch.uint8) for _ in range(E)]
+    wsc = [torch.zeros(sb, dtype=torch.uint8) for _ in range(E)]
+    with pytest.raises(ValueError, match="need 3 entries"):
+        mq.grouped_mm_list(a["x"], a["D"], wq[:2], wsc[:2], a["group_list"], 1, N)
+    with pytest.raises(ValueError, match="Wq holds"):
+        mq.grouped_mm_list(a["x"], a["D"], [torch.zeros(10, dtype=torch.uint8)] * E, wsc, a["group_list"], 1, N)
+    with pytest.raises(ValueError, match="expected contiguous CUDA tensors"):
+        mq.grouped_mm_list(a["x"], a["D"], wq, wsc, a["group_list"], 1, N)
+    with pytest.raises(ValueError, match="W_kn must be torch.float32"):
+        mq.prepare_weights_transposed(torch.zeros((K, N), dtype=torch.float64), torch.ones(K))
+

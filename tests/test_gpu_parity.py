@@ -11,7 +11,7 @@ import torch
 import oracle
 import synth
 import w4a4_mxfp4_quantize_b200 as mq
-from helpers import compare, dequant_matmul_bf16, f32_dev, x_to_dev, y_to_bits
+from helpers import assert_mx_equal, compare, dequant_matmul_bf16, f32_dev, x_to_dev, y_to_bits
 
 pytestmark = pytest.mark.gpu
 
@@ -89,8 +89,7 @@ def test_activation_codes_bit_exact_on_dense_configs(cfg):
     for p in synth.config(cfg):
         q, s = _gpu_act(p.x, p.D[0])
         qo, so = oracle.quantize_act(p.x, p.D[0])
-        assert np.array_equal(s, so), p.name
-        assert np.array_equal(q, qo), p.name
+        assert_mx_equal(q, s, qo, so, p.name)
 
 
 def test_activation_codes_bit_exact_adversarial():
@@ -110,8 +109,7 @@ def test_activation_codes_bit_exact_adversarial():
     D = D.astype(np.float32)
     q, s = _gpu_act(xb, D)
     qo, so = oracle.quantize_act(xb, D)
-    assert np.array_equal(s, so)
-    assert np.array_equal(q, qo)
+    assert_mx_equal(q, s, qo, so, "adversarial")
 
 
 # ----------------------------------------------------------------------------
@@ -433,8 +431,7 @@ def test_quantise_once_activation_images_bit_exact(M, K, plain):
         qa, sa = oracle.quantize_act(p.x, p.D[0])
     torch.cuda.synchronize()
     codes, scales = _decode_activation_images(ws.cpu().numpy(), M, K)
-    assert np.array_equal(codes, qa), "activation codes differ from the oracle"
-    assert np.array_equal(scales, sa), "activation scales differ from the oracle"
+    assert_mx_equal(codes, scales, qa, sa, f"images M={M} K={K}")
 
 
 def test_max_rows_sampled():

@@ -547,6 +547,23 @@ def test_grouped_type2_rows_use_the_named_expert():
     assert np.array_equal(y3[50:], oracle.dense_mm(p.x[50:], p.D[3], p.W[3]))
 
 
+def test_grouped_weight_list_equals_the_stacked_weights():
+    # npu_grouped_matmul's weight given as a list (one tensor per expert) is the
+    # same layer as the stacked [E, N, K] weight: the list form is written as one
+    # dense call per entry, the stacked form is the C grouped routine
+    p = synth.grouped(120, 5, 64, 32, seed=8, dist="zipf", group_list_type=1)
+    W_list = [np.ascontiguousarray(p.W[e]) for e in range(p.E)]
+    gl2 = np.ascontiguousarray(np.stack([np.array([4, 0, 2, 2, 1]), p.counts]).T.astype(np.int64))
+    for gl, t in [(p.counts.astype(np.int64), 1), (np.cumsum(p.counts).astype(np.int64), 0), (gl2, 2)]:
+        st_l, y_l = oracle.grouped_mm_list(p.x, p.D, W_list, gl, t)
+        st_s, y_s = oracle.grouped_mm(p.x, p.D, p.W, gl, t)
+        assert st_l == st_s == oracle.OK
+        assert np.array_equal(y_l, y_s), t
+    bad = p.counts.astype(np.int64).copy()
+    bad[0] += 1
+    assert oracle.grouped_mm_list(p.x, p.D, W_list, bad, 1)[0] == oracle.ERR_GROUP_LIST_INVALID
+
+
 def test_grouped_rows_use_their_own_expert():
     p = synth.grouped(64, 3, 64, 32, seed=4, dist="uniform", group_list_type=1)
     st, y = oracle.grouped_mm(p.x, p.D, p.W, p.group_list, 1)

@@ -97,9 +97,9 @@ _SIG = {
     "macaq_dense_mm_plain": (ctypes.c_int, [_P, _P, _P, _P, _I64, _I64, _I64, _P, ctypes.c_size_t, _P, _P]),
     "macaq_grouped_mm_plain": (ctypes.c_int, [_P, _P, _P, _P, ctypes.c_int, _I64, _P, _I64, _I64, _I64, _P,
                                               ctypes.c_size_t, _P, _P]),
-    "macaq_fused_plan": (ctypes.c_int, [_I64, _I64, _I64, _P, _P, _P]),
+    "macaq_fused_plan": (ctypes.c_int, [_I64, _I64, _I64, _P, _P]),
     "macaq_fused_probe": (ctypes.c_int, [_P, _P, _P, _P, _P, _I64, _I64, _I64, ctypes.c_int, ctypes.c_int,
-                                         ctypes.c_int, ctypes.c_int, _P, _P, _P, _P]),
+                                         ctypes.c_int, _P, _P, _P, _P]),
     "macaq_test_wait_expiry": (ctypes.c_int, [_I64, _P, _P]),
     "macaq_prepare_weights_transposed": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _P]),
     "macaq_grouped_mm_list": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P, _I64,
@@ -298,11 +298,12 @@ def grouped_mm_list(x: torch.Tensor, D: torch.Tensor, Wq_list, Ws_list, group_li
     _check_bias(bias, (E, N))
     with _on(stream):
         y = _output(out, M, N, x.device)
-        tables = torch.tensor([[w.data_ptr() for w in Wq_list], [w.data_ptr() for w in Ws_list]],
-                              dtype=torch.int64).to(x.device, non_blocking=False)
+        # two separate device tables (each starts 16-byte aligned, as the C call requires)
+        wq_table = torch.tensor([w.data_ptr() for w in Wq_list], dtype=torch.int64).to(x.device)
+        ws_table = torch.tensor([w.data_ptr() for w in Ws_list], dtype=torch.int64).to(x.device)
     L = lib()
     ws = workspace(int(L.macaq_workspace_bytes(M, N, K, E)), x.device, stream, ws)
-    _check(L.macaq_grouped_mm_list(_ptr(x), _ptr(D), _ptr(tables[0]), _ptr(tables[1]), _ptr(group_list),
+    _check(L.macaq_grouped_mm_list(_ptr(x), _ptr(D), _ptr(wq_table), _ptr(ws_table), _ptr(group_list),
                                    int(group_list_type), E, _ptr(bias), int(act_type), _ptr(y), M, N, K, _ptr(ws),
                                    _nbytes(ws), _ptr(status), _stream_ptr(stream)), "macaq_grouped_mm_list")
     return y
@@ -518,16 +519,15 @@ def quantize_activations(x: torch.Tensor, D: torch.Tensor, stream=None) -> tuple
     return codes, scales
 
 
-def fused_plan(M: int, N: int, K: int) -> tuple[int, int, int]:
-    """(token tile, K split, N share) that dense_mm's fused kernel uses for this shape (M <= 128)."""
-    bt, s, c = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
-    _check(lib().macaq_fused_plan(M, N, K, ctypes.byref(bt), ctypes.byref(s), ctypes.byref(c)), "macaq_fused_plan")
-    return bt.value, s.value, c.value
+def fused_plan(M: int, N: int, K: int) -> tuple[int, int]:
+    """(token tile, K split) that dense_mm's fused kernel uses for this shape (M <= 128)."""
+    bt, s = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().macaq_fused_plan(M, N, K, ctypes.byref(bt), ctypes.byref(s)), "macaq_fused_plan")
+    return bt.value, s.value
 
 
 def fused_probe(x: torch.Tensor, D: torch.Tensor | None, Wq: torch.Tensor, Ws: torch.Tensor, N: int,
-                token_tile: int, k_split: int, n_share: int = 0, plain: bool = False, dump: bool = True,
-                stream=None):
+                token_tile: int, k_split: int, plain: bool = False, dump: bool = True, stream=None):
     """Test only: the fused kernel with a given plan; returns (y, codes, scales), the
     last two being its own activation operand tiles in canonical form (None
     without dump)."""
@@ -539,8 +539,8 @@ def fused_probe(x: torch.Tensor, D: torch.Tensor | None, Wq: torch.Tensor, Ws: t
         codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device) if dump else None
         scales = torch.empty((M, K // 32), dtype=torch.uint8, device=x.device) if dump else None
     _check(lib().macaq_fused_probe(_ptr(x), None if plain else _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(y), M, N, K,
-                                   int(token_tile), int(k_split), int(n_share), int(bool(plain)), _ptr(codes),
-                                   _ptr(scales), None, _stream_ptr(stream)), "macaq_fused_probe")
+                                   int(token_tile), int(k_split), int(bool(plain)), _ptr(codes), _ptr(scales),
+                                   None, _stream_ptr(stream)), "macaq_fused_probe")
     return y, codes, scales
 
 

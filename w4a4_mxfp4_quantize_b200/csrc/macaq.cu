@@ -148,7 +148,8 @@ constexpr int kActImageBytes = kTileCodeBytes + kTileSfBytes;  // 17408
 // ============================================================================
 // CTA = 32 rows x one 256-wide K tile (256 threads, one 32-block each).
 // kPlain: plain MXFP4 of W itself (no D, no Hadamard; D is not read).
-template <bool kPlain>
+// kTrans: W is stored transposed, [E, K, N] (element (n, k) at (e K + k) N + n).
+template <bool kPlain, bool kTrans = false>
 __global__ void __launch_bounds__(256) prep_weights_kernel(const float* __restrict__ W, const float* __restrict__ D,
                                                            uint8_t* __restrict__ Wq, uint8_t* __restrict__ Ws,
                                                            int N, int K, int NT) {
@@ -165,11 +166,17 @@ __global__ void __launch_bounds__(256) prep_weights_kernel(const float* __restri
   uint32_t scale = 0;
   if (n < N) {
     float wv[32];
-    const float4* wp = reinterpret_cast<const float4*>(W + (static_cast<int64_t>(e) * N + n) * K + k0);
+    if constexpr (kTrans) {
+      const float* wp = W + (static_cast<int64_t>(e) * K + k0) * N + n;  // offline: strided reads are fine
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 a = __ldg(wp + i);
-      wv[4 * i] = a.x; wv[4 * i + 1] = a.y; wv[4 * i + 2] = a.z; wv[4 * i + 3] = a.w;
+      for (int i = 0; i < 32; ++i) wv[i] = __ldg(wp + static_cast<int64_t>(i) * N);
+    } else {
+      const float4* wp = reinterpret_cast<const float4*>(W + (static_cast<int64_t>(e) * N + n) * K + k0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 a = __ldg(wp + i);
+        wv[4 * i] = a.x; wv[4 * i + 1] = a.y; wv[4 * i + 2] = a.z; wv[4 * i + 3] = a.w;
+      }
     }
     if constexpr (kPlain) {
       mx_encode_block(wv, codes, scale);
@@ -254,6 +261,32 @@ __global__ void mx_encode_kernel(const float* __restrict__ v, uint8_t* __restric
   scales[b] = static_cast<uint8_t>(sc);
 }
 
+// The bounded wait of the kernels run out on purpose (tests).  One CTA of two
+// warps: warp 0 waits on an mbarrier that nothing ever arrives on, with the
+// kernels' own bounded wait (mbar_wait) and a limit of timeout_ns; when it gives
+// up it raises the CTA's abort flag, and warp 1's wait on the same barrier then
+// gives up at the flag (its own limit is the same, as a bound only).  Nothing asynchronous (no
+// bulk copy, no tensor-core operation) is issued, so nothing is in flight when
+// the waits end.  Thread 0 then reports the expiry to *status the way the
+// kernels do.
+__global__ void __launch_bounds__(64) wait_expiry_kernel(uint64_t timeout_ns, int32_t* status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  __shared__ int gave_up[2];
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) gave_up[0] = mbar_wait(&bar, 0, &abort_flag, timeout_ns) ? 0 : 1;
+  __syncthreads();
+  if (threadIdx.x == 32) gave_up[1] = mbar_wait(&bar, 0, &abort_flag, timeout_ns) ? 0 : 1;
+  __syncthreads();
+  if (threadIdx.x == 0 && status)
+    *status = (abort_flag && gave_up[0] && gave_up[1]) ? MACAQ_ERR_DEVICE_TIMEOUT : MACAQ_OK;
+}
+
 // ============================================================================
 // Grouped form: device-side group_list validation and tables
 // ============================================================================
@@ -304,15 +337,41 @@ __device__ __forceinline__ void block_excl_scan3(const int64_t (&v)[3], int64_t 
 // (per 32-row slab holding rows: {expert, first row of x, rows, 4 * tile +
 // quarter of the tile}), its length *nslabs and *valid; on a violation also
 // *status.
+// Weight-list calls (one weight tensor per expert) also pass the device tables
+// of the experts' code and scale images; each pointer must be non-null,
+// 16-byte aligned (the bulk copies read from it) and must not overlap y, else
+// the call is refused on the device with *status set (MACAQ_ERR_NULL, _ALIGN,
+// _ALIAS) and y left as it was.
+struct WeightList {
+  const uint64_t* wq;  // [E] device addresses of the experts' code images (nullptr: stacked weights)
+  const uint64_t* ws;  // [E] and of their scale images
+  uint64_t wq_bytes, ws_bytes;  // bytes of one expert's images
+  uint64_t y_lo, y_hi;          // the output's byte range
+};
+
 __global__ void __launch_bounds__(1024) group_tables_kernel(const int64_t* __restrict__ gl, int type, int E, int M,
                                                             int64_t* __restrict__ goff, int* __restrict__ gtp,
                                                             int* __restrict__ gexp, int4* __restrict__ slabs,
                                                             int* __restrict__ nslabs, int* __restrict__ valid,
-                                                            int32_t* status) {
+                                                            int32_t* status, const WeightList wl) {
   __shared__ int64_t scratch[96];
+  __shared__ int list_err;
   const int g = threadIdx.x;
+  pdl_trigger();  // the quantiser may set up; it reads the tables only after this kernel completes
   int64_t cnt = 0;
   bool bad = false;
+  if (g == 0) list_err = 0;
+  __syncthreads();
+  if (wl.wq != nullptr && g < E) {
+    const uint64_t a = wl.wq[g], b = wl.ws[g];
+    int err = 0;
+    if (a == 0 || b == 0) err = MACAQ_ERR_NULL;
+    else if ((a | b) & 15u) err = MACAQ_ERR_ALIGN;
+    else if ((a < wl.y_hi && wl.y_lo < a + wl.wq_bytes) || (b < wl.y_hi && wl.y_lo < b + wl.ws_bytes))
+      err = MACAQ_ERR_ALIAS;
+    if (err != 0) atomicCAS(&list_err, 0, err);
+  }
+  __syncthreads();
   int ex = g;  // the expert whose weights this list entry's rows use
   if (g < E) {
     if (type == 2) {  // [E, 2] rows of (group index, group size)
@@ -351,10 +410,10 @@ __global__ void __launch_bounds__(1024) group_tables_kernel(const int64_t* __res
                                   static_cast<int>(cnt - 32 * j < 32 ? cnt - 32 * j : 32), static_cast<int>(4 * tb + j));
   }
   if (g == 0) {
-    *valid = bad ? 0 : 1;
-    if (bad && status) *status = MACAQ_ERR_GROUP_LIST_INVALID;
+    *valid = (bad || list_err != 0) ? 0 : 1;
+    if (status && list_err != 0) *status = list_err;
+    else if (bad && status) *status = MACAQ_ERR_GROUP_LIST_INVALID;
   }
-  pdl_trigger();
 }
 
 __device__ __forceinline__ int find_group(const int* gtp, int E, int pm) {
@@ -631,29 +690,39 @@ struct GemmParams {
   float out_scale;        // 2^-5 (MACAQ: undoes the two unnormalised Hadamards), 1 (plain MXFP4)
   const float* bias;      // fp32 [E][N] (expert g's row for its tiles) or nullptr
   int act;                // act_type: 0 none, 1 RELU, 2 GELU_TANH, 4 FAST_GELU, 5 SILU
+  const uint64_t* wq_list;  // weight-list form: [E] addresses of each expert's images (else nullptr)
+  const uint64_t* ws_list;
 };
 
-// Epilogue drain of the 128 accumulator columns of one thread's row of its half
-// tile: v = acc * out_scale (+ bias[n]), then the activation, packed to BF16
-// pairs.  Columns n >= N (the zero rows of a ragged weight tile) take no bias.
-template <int ACT>
-__device__ __forceinline__ void drain128(uint32_t taddr, float os, const float* brow, int ncol0, int N,
-                                         uint32_t (&pk)[64]) {
-  const int nb = brow != nullptr ? N - ncol0 : 0;  // leading columns that take a bias (a multiple of 16)
+// Epilogue of the 128 accumulator columns of one thread's row of its half
+// tile, already loaded into registers: v = acc * out_scale (+ bias[n]), then the
+// activation, packed to BF16 pairs.  kEpi < 0: scaling only (no bias, no
+// activation); otherwise act_type kEpi with an optional bias.  Columns n >= N
+// (the zero rows of a ragged weight tile) take no bias.
+template <int kEpi>
+__device__ __forceinline__ void finish128(const uint32_t (&r)[128], float os, const float* brow, int ncol0, int N,
+                                          uint32_t (&pk)[64]) {
   const float2 os2 = make_float2(os, os);
+  if constexpr (kEpi < 0) {
 #pragma unroll
-  for (int c0 = 0; c0 < 128; c0 += 16) {
-    uint32_t r[16];
-    tmem_ld_32x32b_x16(taddr + c0, r);
-    tmem_wait_ld();
-    const bool inb = c0 + 16 <= nb;
+    for (int e = 0; e < 64; ++e) {
+      const float2 v = fmul2(make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), os2);
+      pk[e] = pack_bf16x2(v.x, v.y);
+    }
+  } else {
+    const int nb = brow != nullptr ? N - ncol0 : 0;  // leading columns that take a bias (a multiple of 16)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      float2 b = make_float2(0.f, 0.f);
-      if (inb) b = __ldg(reinterpret_cast<const float2*>(brow + ncol0 + c0 + 2 * e));  // warp-uniform: a broadcast
-      const float2 v = ffma2(make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), os2, b);
-      const float2 y = act_pair<ACT>(v);
-      pk[c0 / 2 + e] = pack_bf16x2(y.x, y.y);
+    for (int c0 = 0; c0 < 128; c0 += 16) {
+      const bool inb = c0 + 16 <= nb;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        float2 b = make_float2(0.f, 0.f);
+        if (inb) b = __ldg(reinterpret_cast<const float2*>(brow + ncol0 + c0 + 2 * e));  // warp-uniform: a broadcast
+        const float2 v =
+            ffma2(make_float2(__uint_as_float(r[c0 + 2 * e]), __uint_as_float(r[c0 + 2 * e + 1])), os2, b);
+        const float2 y = act_pair<kEpi>(v);
+        pk[c0 / 2 + e] = pack_bf16x2(y.x, y.y);
+      }
     }
   }
 }
@@ -685,19 +754,21 @@ constexpr int kSfCols = 24;
 static_assert(kSfCol + kSfCols * kMaxStages <= kTmemCols, "scale slots fit the allocation");
 static_assert(kStageBytes % 1024 == 0, "stage alignment");
 constexpr size_t kSmemLimit = 227 * 1024;
-__host__ __device__ constexpr size_t group_bytes(int E) {
-  return E > 0 ? static_cast<size_t>(E + 1) * 16 + 16 : 0;  // goff (8), gtp (4), gexp (4) per entry
+// goff (8), gtp (4), gexp (4) per entry; the weight-list form adds the two image
+// address tables (8 + 8 per expert)
+__host__ __device__ constexpr size_t group_bytes(int E, bool list = false) {
+  return E > 0 ? static_cast<size_t>(E + 1) * 16 + 16 + (list ? static_cast<size_t>(E) * 16 : 0) : 0;
 }
 // four stages when the group tables leave room for them, else three
-__host__ __device__ constexpr int stages_for(int E) {
-  return 1024 + static_cast<size_t>(kMaxStages) * kStageBytes + kFixedBytes + group_bytes(E) <= kSmemLimit
+__host__ __device__ constexpr int stages_for(int E, bool list = false) {
+  return 1024 + static_cast<size_t>(kMaxStages) * kStageBytes + kFixedBytes + group_bytes(E, list) <= kSmemLimit
              ? kMaxStages
              : kMaxStages - 1;
 }
-__host__ __device__ constexpr size_t smem_bytes(int E) {
-  return 1024 + static_cast<size_t>(stages_for(E)) * kStageBytes + kFixedBytes + group_bytes(E);
+__host__ __device__ constexpr size_t smem_bytes(int E, bool list = false) {
+  return 1024 + static_cast<size_t>(stages_for(E, list)) * kStageBytes + kFixedBytes + group_bytes(E, list);
 }
-static_assert(smem_bytes(0) <= kSmemLimit && smem_bytes(1024) <= kSmemLimit, "shared memory");
+static_assert(smem_bytes(0) <= kSmemLimit && smem_bytes(1024, true) <= kSmemLimit, "shared memory");
 }  // namespace gemm
 
 struct GemmTile {
@@ -781,9 +852,9 @@ __device__ __forceinline__ void mma_stage(uint64_t adesc, uint64_t bdesc, uint32
   }
 }
 
-// kEpilogue: the bias / activation epilogue (p.bias, p.act) is compiled in; the
-// plain kernel keeps its registers for the plain drain.
-template <bool kEpilogue>
+// kEpi < 0: the output is the scaled sum; kEpi = act_type (0, 1, 2, 4, 5): an
+// optional bias (p.bias) and that activation are applied in the epilogue.
+template <int kEpi>
 __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_constant__ GemmParams p) {
   using namespace gemm;
   extern __shared__ uint8_t smem_raw[];
@@ -801,6 +872,8 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
   int64_t* goff = nullptr;
   int* gtp = nullptr;
   int* gexp = nullptr;
+  uint64_t* wql = nullptr;  // weight-list form: each expert's code / scale image addresses
+  uint64_t* wsl = nullptr;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   int mtiles = p.MT;
@@ -810,10 +883,18 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
     goff = reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(full) + 256);
     gtp = reinterpret_cast<int*>(goff + p.E + 1);
     gexp = gtp + p.E + 1;
+    if (p.wq_list != nullptr) {
+      wql = reinterpret_cast<uint64_t*>(goff + 2 * (p.E + 1));  // after goff, gtp, gexp (16 bytes per entry + 16)
+      wsl = wql + p.E;
+    }
     for (int i = threadIdx.x; i <= p.E; i += blockDim.x) {
       goff[i] = p.goff[i];
       gtp[i] = p.gtp[i];
       if (i < p.E) gexp[i] = p.gexp[i];
+      if (wql != nullptr && i < p.E) {
+        wql[i] = p.wq_list[i];
+        wsl[i] = p.ws_list[i];
+      }
     }
     __syncthreads();
     mtiles = gtp[p.E];
@@ -859,11 +940,14 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
     // kt * step further on.
     auto source = [&](int i, int c, const uint8_t*& src, uint32_t& bytes, uint32_t& doff, uint32_t& step) {
       const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp, gexp);
-      const size_t img = weight_image(t.g, t.nt, 0, p.NT2, KT);
+      // stacked weights: expert t.g's images follow the others'; weight list: its own base
+      const size_t img = weight_image(wql != nullptr ? 0 : t.g, t.nt, 0, p.NT2, KT);
+      const uint8_t* wq = wql != nullptr ? reinterpret_cast<const uint8_t*>(wql[t.g]) : p.Wq;
+      const uint8_t* ws = wql != nullptr ? reinterpret_cast<const uint8_t*>(wsl[t.g]) : p.Ws;
       bytes = c == 0 ? kActImageBytes : c == 1 ? 2 * kTileCodeBytes : 2 * kTileSfBytes;
       step = c == 0 ? kActImageBytes : bytes;
       src = c == 0 ? p.Aq + static_cast<size_t>(t.pm) * KT * kActImageBytes
-                   : (c == 1 ? p.Wq + img * kTileCodeBytes : p.Ws + img * kTileSfBytes);
+                   : (c == 1 ? wq + img * kTileCodeBytes : ws + img * kTileSfBytes);
       doff = c == 0 ? kOffA : c == 1 ? kOffB : kOffSfb;
     };
     const uint8_t* src;
@@ -962,11 +1046,9 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
   } else {
     // ================= epilogue: TMEM -> x 2^-5 -> BF16 -> staged chunks -> coalesced rows =================
     // Warp w reads TMEM lanes 32 (w % 4) .. + 31 (accumulator rows) and columns
-    // 128 h .. + 127 with h = (w - 2) / 4.  The accumulator is drained into packed
-    // BF16 registers first and handed back, so the next tile's MMAs overlap the
-    // write-out (the bias / activation instantiation applies them during the drain).  Rows go out in 64-column
-    // chunks staged in shared memory with their 16-byte pieces XOR-swizzled by the
-    // row (conflict-free writes and reads).
+    // 128 h .. + 127 with h = (w - 2) / 4.  Rows go out in 64-column chunks staged
+    // in shared memory with their 16-byte pieces XOR-swizzled by the row
+    // (conflict-free writes and reads).
     const int q = warp & 3, h = (warp - 2) >> 2;
     const int et = threadIdx.x - 64;
     const float os = p.out_scale;
@@ -999,52 +1081,30 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
           }
         }
       };
-      if constexpr (!kEpilogue) {
-        // the whole row into packed registers first, then the accumulator is free
-        // for the next tile's MMAs while the chunks go out
-        uint32_t pk[64];
+      // The whole 128-column run of the row is loaded with one wait and the
+      // accumulator handed back at once, so the next tile's MMAs overlap the
+      // scaling (bias, activation), packing and write-out of this one.
+      uint32_t r[128];
+      tmem_ld_32x32b_x32(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      tmem_ld_32x32b_x32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
+      tmem_ld_32x32b_x32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acce);
+      uint32_t pk[64];
+      {
+        const float* brow = nullptr;
+        if constexpr (kEpi >= 0) brow = p.bias != nullptr ? p.bias + static_cast<int64_t>(t.g) * p.N : nullptr;
+        finish128<kEpi>(r, os, brow, t.nt * kRowsTile + h * 128, p.N, pk);
+      }
 #pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(taddr + c0, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            pk[c0 / 2 + e] = pack_bf16x2(__uint_as_float(r[2 * e]) * os, __uint_as_float(r[2 * e + 1]) * os);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acce);
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          if ((ch >> 1) == h) stage_chunk(pk + (ch & 1) * 32);
-          named_bar_sync(1, 256);
-          store_chunk(ch);
-          if (ch < 3) named_bar_sync(1, 256);  // read out before the next chunk overwrites it
-        }
-      } else {
-        // bias and/or activation applied while the row is drained; as above, the
-        // accumulator is handed back before the chunks go out
-        const float* brow = p.bias != nullptr ? p.bias + static_cast<int64_t>(t.g) * p.N : nullptr;
-        const int nc = t.nt * kRowsTile + h * 128;
-        uint32_t pk[64];
-        switch (p.act) {
-          case 1: drain128<1>(taddr, os, brow, nc, p.N, pk); break;
-          case 2: drain128<2>(taddr, os, brow, nc, p.N, pk); break;
-          case 4: drain128<4>(taddr, os, brow, nc, p.N, pk); break;
-          case 5: drain128<5>(taddr, os, brow, nc, p.N, pk); break;
-          default: drain128<0>(taddr, os, brow, nc, p.N, pk);
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(acce);
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          if ((ch >> 1) == h) stage_chunk(pk + (ch & 1) * 32);
-          named_bar_sync(1, 256);
-          store_chunk(ch);
-          if (ch < 3) named_bar_sync(1, 256);
-        }
+      for (int ch = 0; ch < 4; ++ch) {
+        if ((ch >> 1) == h) stage_chunk(pk + (ch & 1) * 32);
+        named_bar_sync(1, 256);
+        store_chunk(ch);
+        if (ch < 3) named_bar_sync(1, 256);  // read out before the next chunk overwrites it
       }
     }
   }
@@ -1071,6 +1131,8 @@ struct FusedParams {
   float out_scale;         // 2^-5 (MACAQ) or 1 (plain)
   const float* bias;       // fp32 [N] or nullptr
   int act;                 // act_type (act_value)
+  uint8_t* dump_codes;     // test instantiation only: canonical [M, K/2] codes of the operand tiles
+  uint8_t* dump_scales;    // and [M, K/32] scales, copied out of shared memory before each MMA
 };
 
 namespace fused {
@@ -1111,8 +1173,27 @@ struct Cfg {
 };
 }  // namespace fused
 
+// Test instantiations: the activation operand tile of one K tile (BT rows of
+// swizzled codes and its scale image) as the tensor core will read it, copied to
+// canonical codes [M, K/2] and scales [M, K/32] by the MMA issuer between the
+// wait for the tile and the MMAs that read it.  Only the CTAs of the first
+// channel tile copy, so every (row, K tile) is written once.
+template <int BT>
+__device__ __forceinline__ void dump_act_tile(const uint8_t* bcode, const uint8_t* bsf, const FusedParams& p, int m0,
+                                              int rows, int kt) {
+  for (int t = 0; t < rows; ++t) {
+    const int64_t row = m0 + t;
+    for (int c = 0; c < 8; ++c) {
+      *reinterpret_cast<uint4*>(p.dump_codes + row * (p.K / 2) + kt * (kKTile / 2) + c * (kBlk / 2)) =
+          *reinterpret_cast<const uint4*>(bcode + code_chunk_offset(t, c));
+      p.dump_scales[row * (p.K / kBlk) + kt * (kKTile / kBlk) + c] = bsf[sf_offset(t, c)];
+    }
+  }
+}
+
 // kEpilogue: the bias / activation epilogue (p.bias, p.act) is compiled in.
-template <int BT, bool kEpilogue = false>
+// kDump: test instantiation copying the activation operand tiles out (dump_act_tile).
+template <int BT, bool kEpilogue = false, bool kDump = false>
 __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const __grid_constant__ FusedParams p) {
   using C = fused::Cfg<BT>;
   using fused::kStages;
@@ -1275,6 +1356,11 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
           break;
         }
         tc_fence_after();
+        if constexpr (kDump) {
+          if (nt == 0 && p.dump_codes != nullptr)
+            dump_act_tile<BT>(smem + stage * C::kStageBytes + C::kOffB, smem + stage * C::kStageBytes + C::kOffSfb,
+                              p, m0, rows, kt);
+        }
         const uint32_t so = static_cast<uint32_t>(stage * C::kStageBytes) >> 4;
         const uint32_t sfa_col = tmem + C::kSfCol + 16 * stage;
         mma_stage(code0 + so, code0 + so + (C::kOffB >> 4), sfa_col, sfa_col + 8, tmem, idesc_lo, idesc_hi,
@@ -1533,6 +1619,16 @@ struct DeviceState {
 };
 DeviceState g_dev[kMaxDevices];
 
+// Shared-memory opt-in of the fused kernel's instantiations for one token tile.
+template <int BT>
+bool fused_attrs() {
+  const int bytes = fused::Cfg<BT>::kSmemBytes;
+  const auto a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  return cudaFuncSetAttribute(fused_small_kernel<BT, false, false>, a, bytes) == cudaSuccess &&
+         cudaFuncSetAttribute(fused_small_kernel<BT, true, false>, a, bytes) == cudaSuccess &&
+         cudaFuncSetAttribute(fused_small_kernel<BT, false, true>, a, bytes) == cudaSuccess;
+}
+
 int current_device(int& dev, int& sms) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MACAQ_ERR_CUDA;
   DeviceState& s = g_dev[dev];
@@ -1550,26 +1646,15 @@ int current_device(int& dev, int& sms) {
   if (!s.is_sm100) return MACAQ_ERR_ARCH;
   if (!s.attrs_set) {  // once per device: opt in to the shared memory the kernels use
     const size_t gemm_smem = gemm::kSmemLimit;  // smem_bytes(E) stays within it for every E
-    bool ok = cudaFuncSetAttribute(gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   static_cast<int>(gemm_smem)) == cudaSuccess;
-    ok = ok && cudaFuncSetAttribute(gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    static_cast<int>(gemm_smem)) == cudaSuccess;
-    ok = ok && cudaFuncSetAttribute(fused_small_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    fused::Cfg<16>::kSmemBytes) == cudaSuccess;
-    ok = ok && cudaFuncSetAttribute(fused_small_kernel<16, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    fused::Cfg<16>::kSmemBytes) == cudaSuccess;
-    ok = ok && cudaFuncSetAttribute(fused_small_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    fused::Cfg<32>::kSmemBytes) == cudaSuccess;
-    ok = ok && cudaFuncSetAttribute(fused_small_kernel<32, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    fused::Cfg<32>::kSmemBytes) == cudaSuccess;
-    ok = ok && cudaFuncSetAttribute(fused_small_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    fused::Cfg<64>::kSmemBytes) == cudaSuccess;
-    ok = ok && cudaFuncSetAttribute(fused_small_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    fused::Cfg<64>::kSmemBytes) == cudaSuccess;
-    ok = ok && cudaFuncSetAttribute(fused_small_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    fused::Cfg<128>::kSmemBytes) == cudaSuccess;
-    ok = ok && cudaFuncSetAttribute(fused_small_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    fused::Cfg<128>::kSmemBytes) == cudaSuccess;
+    const auto a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+    const int gs = static_cast<int>(gemm_smem);
+    bool ok = cudaFuncSetAttribute(gemm_kernel<-1>, a, gs) == cudaSuccess &&
+              cudaFuncSetAttribute(gemm_kernel<0>, a, gs) == cudaSuccess &&
+              cudaFuncSetAttribute(gemm_kernel<1>, a, gs) == cudaSuccess &&
+              cudaFuncSetAttribute(gemm_kernel<2>, a, gs) == cudaSuccess &&
+              cudaFuncSetAttribute(gemm_kernel<4>, a, gs) == cudaSuccess &&
+              cudaFuncSetAttribute(gemm_kernel<5>, a, gs) == cudaSuccess;
+    ok = ok && fused_attrs<16>() && fused_attrs<32>() && fused_attrs<64>() && fused_attrs<128>();
     ok = ok && cudaFuncSetAttribute(quant_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmem) ==
                    cudaSuccess;
     if (!ok) return MACAQ_ERR_CUDA;
@@ -1646,6 +1731,15 @@ int max_active_clusters(int S) {
   return n;
 }
 
+int max_active_clusters_any(int bt_index, int S) {
+  switch (bt_index) {
+    case 0: return max_active_clusters<16>(S);
+    case 1: return max_active_clusters<32>(S);
+    case 2: return max_active_clusters<64>(S);
+    default: return max_active_clusters<128>(S);
+  }
+}
+
 // Co-resident clusters per (BT, S), measured once per device.
 int active_clusters(int dev, int bt_index, int S) {
   static int cache[kMaxDevices][4][9] = {};
@@ -1694,21 +1788,21 @@ FusedPlan plan_fused(int dev, int64_t M, int64_t N, int64_t K) {
   return best;
 }
 
-template <bool kEpilogue>
+template <bool kEpilogue, bool kDump = false>
 cudaError_t launch_fused_kind(const FusedParams& p, const FusedPlan& plan, cudaStream_t st) {
   const dim3 grid(plan.ctas), block(fused::kThreads);
   switch (plan.bt) {
     case 16:
-      return launch_ex(fused_small_kernel<16, kEpilogue>, grid, block, fused::Cfg<16>::kSmemBytes, st, true, plan.S,
-                       p);
+      return launch_ex(fused_small_kernel<16, kEpilogue, kDump>, grid, block, fused::Cfg<16>::kSmemBytes, st, true,
+                       plan.S, p);
     case 32:
-      return launch_ex(fused_small_kernel<32, kEpilogue>, grid, block, fused::Cfg<32>::kSmemBytes, st, true, plan.S,
-                       p);
+      return launch_ex(fused_small_kernel<32, kEpilogue, kDump>, grid, block, fused::Cfg<32>::kSmemBytes, st, true,
+                       plan.S, p);
     case 64:
-      return launch_ex(fused_small_kernel<64, kEpilogue>, grid, block, fused::Cfg<64>::kSmemBytes, st, true, plan.S,
-                       p);
+      return launch_ex(fused_small_kernel<64, kEpilogue, kDump>, grid, block, fused::Cfg<64>::kSmemBytes, st, true,
+                       plan.S, p);
     default:
-      return launch_ex(fused_small_kernel<128, kEpilogue>, grid, block, fused::Cfg<128>::kSmemBytes, st, true,
+      return launch_ex(fused_small_kernel<128, kEpilogue, kDump>, grid, block, fused::Cfg<128>::kSmemBytes, st, true,
                        plan.S, p);
   }
 }
@@ -1749,8 +1843,10 @@ GroupedWs grouped_ws(int64_t M, int64_t K, int64_t E) {
 }
 
 // plain: plain MXFP4 call, D is not used (and may be null).
+// weight_bytes: bytes of each of Wq and Ws when they are not prepared weights
+// (the weight-list form passes tables of addresses); 0: prepared images of E experts.
 int check_mm_args(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M,
-                  int64_t N, int64_t K, int64_t E, bool plain = false) {
+                  int64_t N, int64_t K, int64_t E, bool plain = false, size_t weight_bytes = 0) {
   if (M < 0 || M > INT32_MAX || !valid_nk(N, K)) return MACAQ_ERR_SHAPE;
   if (M == 0) return MACAQ_OK;
   if (!x || (!D && !plain) || !Wq || !Ws || !y) return MACAQ_ERR_NULL;
@@ -1759,8 +1855,8 @@ int check_mm_args(const uint16_t* x, const float* D, const uint8_t* Wq, const ui
   const size_t ybytes = static_cast<size_t>(M) * N * 2;
   if (overlaps(y, ybytes, x, static_cast<size_t>(M) * K * 2) ||
       (!plain && overlaps(y, ybytes, D, static_cast<size_t>(E) * K * 4)) ||
-      overlaps(y, ybytes, Wq, macaq_weight_code_bytes(E, N, K)) ||
-      overlaps(y, ybytes, Ws, macaq_weight_scale_bytes(E, N, K)))
+      overlaps(y, ybytes, Wq, weight_bytes ? weight_bytes : macaq_weight_code_bytes(E, N, K)) ||
+      overlaps(y, ybytes, Ws, weight_bytes ? weight_bytes : macaq_weight_scale_bytes(E, N, K)))
     return MACAQ_ERR_ALIAS;
   return MACAQ_OK;
 }
@@ -1795,6 +1891,19 @@ int check_epilogue(const Epilogue& ep, int64_t rows, int64_t N, const void* y, s
   return MACAQ_OK;
 }
 
+// The GEMM instantiation for an epilogue: scaling only, or bias and act_type.
+using GemmKernel = void (*)(GemmParams);
+GemmKernel gemm_for(const float* bias, int act) {
+  if (bias == nullptr && act == 0) return gemm_kernel<-1>;
+  switch (act) {
+    case 1: return gemm_kernel<1>;
+    case 2: return gemm_kernel<2>;
+    case 4: return gemm_kernel<4>;
+    case 5: return gemm_kernel<5>;
+    default: return gemm_kernel<0>;
+  }
+}
+
 int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y,
                          int64_t M, int64_t N, int64_t K, uint8_t* ws, int32_t* status, cudaStream_t st, int sms,
                          bool pdl, bool plain = false, Epilogue ep = Epilogue()) {
@@ -1820,7 +1929,7 @@ int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, c
   const int tiles = MT * gp.NT2;
   const int grid = tiles < sms ? tiles : sms;
   const cudaError_t e =
-      launch_ex(gp.bias != nullptr || gp.act != 0 ? gemm_kernel<true> : gemm_kernel<false>, dim3(grid),
+      launch_ex(gemm_for(gp.bias, gp.act), dim3(grid),
                 dim3(gemm::kThreads), gemm::smem_bytes(0), st, pdl, 1, gp);
   return e == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
@@ -1879,8 +1988,21 @@ size_t macaq_weight_scale_bytes(int64_t E, int64_t N, int64_t K) {
   return static_cast<size_t>(E) * pad256(N) * (K / 32);
 }
 
+static int prepare_impl(const float* W, const float* D, int64_t E, int64_t N, int64_t K, uint8_t* Wq, uint8_t* Ws,
+                        void* stream, bool trans);
+
 int macaq_prepare_weights(const float* W, const float* D, int64_t E, int64_t N, int64_t K, uint8_t* Wq, uint8_t* Ws,
                           void* stream) {
+  return prepare_impl(W, D, E, N, K, Wq, Ws, stream, false);
+}
+
+int macaq_prepare_weights_transposed(const float* W_kn, const float* D, int64_t E, int64_t N, int64_t K, uint8_t* Wq,
+                                     uint8_t* Ws, void* stream) {
+  return prepare_impl(W_kn, D, E, N, K, Wq, Ws, stream, true);
+}
+
+static int prepare_impl(const float* W, const float* D, int64_t E, int64_t N, int64_t K, uint8_t* Wq, uint8_t* Ws,
+                        void* stream, bool trans) {
   if (E < 1 || E > kMaxGroups) return MACAQ_ERR_TOO_MANY_GROUPS;
   if (!valid_nk(N, K)) return MACAQ_ERR_SHAPE;
   if (!W || !D || !Wq || !Ws) return MACAQ_ERR_NULL;
@@ -1903,7 +2025,10 @@ int macaq_prepare_weights(const float* W, const float* D, int64_t E, int64_t N, 
     if (!(d != 0.0f) || !std::isfinite(d)) return MACAQ_ERR_BAD_D;
   const int NTP = static_cast<int>(pad256(N) / 128);  // images per expert, pairs complete
   dim3 grid(static_cast<unsigned>(E * NTP * 4), static_cast<unsigned>(K / 256));
-  prep_weights_kernel<false><<<grid, 256, 0, s>>>(W, D, Wq, Ws, static_cast<int>(N), static_cast<int>(K), NTP);
+  if (trans)
+    prep_weights_kernel<false, true><<<grid, 256, 0, s>>>(W, D, Wq, Ws, static_cast<int>(N), static_cast<int>(K), NTP);
+  else
+    prep_weights_kernel<false, false><<<grid, 256, 0, s>>>(W, D, Wq, Ws, static_cast<int>(N), static_cast<int>(K), NTP);
   return cudaPeekAtLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
@@ -1966,12 +2091,26 @@ static int dense_impl(const uint16_t* x, const float* D, const uint8_t* Wq, cons
                               plain, ep);
 }
 
+// Weight-list form: device tables of E image addresses (see WeightList).
+struct ListArg {
+  const uint64_t* wq = nullptr;
+  const uint64_t* ws = nullptr;
+};
+
 static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, const int64_t* group_list,
                  int group_list_type, int64_t E, uint16_t* y, int64_t M, int64_t N, int64_t K, void* workspace,
-                 size_t workspace_bytes, int32_t* status, void* stream, bool plain, Epilogue ep = Epilogue()) {
+                 size_t workspace_bytes, int32_t* status, void* stream, bool plain, Epilogue ep = Epilogue(),
+                 ListArg list = ListArg()) {
   if (E < 1 || E > kMaxGroups) return MACAQ_ERR_TOO_MANY_GROUPS;
   if (group_list_type < 0 || group_list_type > 2) return MACAQ_ERR_GROUP_LIST_TYPE;
-  int st = check_mm_args(x, D, Wq, Ws, y, M, N, K, E, plain);
+  const bool listed = list.wq != nullptr || list.ws != nullptr;
+  int st;
+  if (!listed) {
+    st = check_mm_args(x, D, Wq, Ws, y, M, N, K, E, plain);
+  } else {  // the tables are checked here, the addresses in them on the device (group_tables_kernel)
+    st = check_mm_args(x, D, reinterpret_cast<const uint8_t*>(list.wq), reinterpret_cast<const uint8_t*>(list.ws), y,
+                       M, N, K, E, plain, /*weight_bytes=*/static_cast<size_t>(E) * 8);
+  }
   if (st == MACAQ_OK) st = check_epilogue(ep, E, N, y, static_cast<size_t>(M) * N * 2);
   if (st != MACAQ_OK) return st;
   if (M == 0) return MACAQ_OK;
@@ -1993,8 +2132,18 @@ static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, co
   int* valid = reinterpret_cast<int*>(ws + w.valid);
   int4* slabs = reinterpret_cast<int4*>(ws + w.slabs);
   int* gexp = reinterpret_cast<int*>(ws + w.gexp);
-  group_tables_kernel<<<1, static_cast<unsigned>((E + 31) / 32 * 32), 0, s>>>(group_list, group_list_type, static_cast<int>(E), static_cast<int>(M),
-                                         goff, gtp, gexp, slabs, valid + 1, valid, status);
+  WeightList wl{};
+  if (listed) {
+    wl.wq = list.wq;
+    wl.ws = list.ws;
+    wl.wq_bytes = macaq_weight_code_bytes(1, N, K);
+    wl.ws_bytes = macaq_weight_scale_bytes(1, N, K);
+    wl.y_lo = reinterpret_cast<uint64_t>(y);
+    wl.y_hi = wl.y_lo + static_cast<uint64_t>(M) * N * 2;
+  }
+  group_tables_kernel<<<1, static_cast<unsigned>((E + 31) / 32 * 32), 0, s>>>(
+      group_list, group_list_type, static_cast<int>(E), static_cast<int>(M), goff, gtp, gexp, slabs, valid + 1, valid,
+      status, wl);
   if (cudaPeekAtLastError() != cudaSuccess) return MACAQ_ERR_CUDA;
   const int KT = static_cast<int>(K / 256);
   QuantParams qp{};
@@ -2008,15 +2157,17 @@ static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, co
   gp.Wq = Wq; gp.Ws = Ws; gp.Aq = qp.Aq; gp.y = y;
   gp.M = static_cast<int>(M); gp.N = static_cast<int>(N); gp.K = static_cast<int>(K);
   gp.NT = static_cast<int>(pad128(N) / 128); gp.KT = KT; gp.E = static_cast<int>(E);
-  gp.NT2 = (gp.NT + 1) / 2; gp.stages = gemm::stages_for(static_cast<int>(E));
+  gp.NT2 = (gp.NT + 1) / 2; gp.stages = gemm::stages_for(static_cast<int>(E), listed);
   gp.goff = goff; gp.gtp = gtp; gp.gexp = gexp; gp.valid = valid;
   gp.out_scale = plain ? 1.0f : 0.03125f;
   gp.bias = ep.bias;
   gp.act = ep.act;
   gp.status = status;
-  const cudaError_t e = launch_ex(gp.bias != nullptr || gp.act != 0 ? gemm_kernel<true> : gemm_kernel<false>,
+  gp.wq_list = list.wq;
+  gp.ws_list = list.ws;
+  const cudaError_t e = launch_ex(gemm_for(gp.bias, gp.act),
                                   dim3(sms), dim3(gemm::kThreads),
-                                  gemm::smem_bytes(static_cast<int>(E)), s, true, 1, gp);
+                                  gemm::smem_bytes(static_cast<int>(E), listed), s, true, 1, gp);
   return e == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
@@ -2043,6 +2194,20 @@ int macaq_grouped_mm_ex(const uint16_t* x, const float* D, const uint8_t* Wq, co
   ep.act = act_type;
   return grouped_impl(x, D, Wq, Ws, group_list, group_list_type, E, y, M, N, K, workspace, workspace_bytes, status,
                       stream, false, ep);
+}
+
+int macaq_grouped_mm_list(const uint16_t* x, const float* D, const uint64_t* Wq_list, const uint64_t* Ws_list,
+                          const int64_t* group_list, int group_list_type, int64_t E, const float* bias, int act_type,
+                          uint16_t* y, int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                          int32_t* status, void* stream) {
+  Epilogue ep;
+  ep.bias = bias;
+  ep.act = act_type;
+  ListArg list;
+  list.wq = Wq_list;
+  list.ws = Ws_list;
+  return grouped_impl(x, D, nullptr, nullptr, group_list, group_list_type, E, y, M, N, K, workspace, workspace_bytes,
+                      status, stream, false, ep, list);
 }
 
 int macaq_calibrate_d(const uint16_t* x, int64_t T, const float* W, int64_t E, int64_t N, int64_t K,
@@ -2177,6 +2342,69 @@ int macaq_dense_mm_noalloc(const uint16_t* x, const float* D, const uint8_t* Wq,
   if (st != MACAQ_OK) return st;
   return run_dense_two_kernel(x, D, Wq, Ws, y, M, N, K, scratch, status, static_cast<cudaStream_t>(stream), sms,
                               true);
+}
+
+int macaq_fused_plan(int64_t M, int64_t N, int64_t K, int* token_tile, int* k_split) {
+  if (M < 1 || M > kSmallM || !valid_nk(N, K)) return MACAQ_ERR_SHAPE;
+  if (!token_tile || !k_split) return MACAQ_ERR_NULL;
+  int dev, sms;
+  const int st = current_device(dev, sms);
+  if (st != MACAQ_OK) return st;
+  const FusedPlan plan = plan_fused(dev, M, N, K);
+  *token_tile = plan.bt;
+  *k_split = plan.S;
+  return MACAQ_OK;
+}
+
+int macaq_fused_probe(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M,
+                      int64_t N, int64_t K, int token_tile, int k_split, int plain, uint8_t* codes, uint8_t* scales,
+                      int32_t* status, void* stream) {
+  const bool pl = plain != 0;
+  int st = check_mm_args(x, D, Wq, Ws, y, M, N, K, 1, pl);
+  if (st != MACAQ_OK || M == 0) return st;
+  const int KT = static_cast<int>(K / 256);
+  if (M > kSmallM || (token_tile != 16 && token_tile != 32 && token_tile != 64 && token_tile != 128) ||
+      k_split < 1 || k_split > 8 || KT % k_split != 0)
+    return MACAQ_ERR_SHAPE;
+  if ((codes == nullptr) != (scales == nullptr)) return MACAQ_ERR_NULL;
+  if (codes != nullptr) {
+    if (!aligned16(codes)) return MACAQ_ERR_ALIGN;
+    const size_t cb = static_cast<size_t>(M) * K / 2, sb = static_cast<size_t>(M) * K / 32, yb = static_cast<size_t>(M) * N * 2;
+    if (overlaps(codes, cb, y, yb) || overlaps(scales, sb, y, yb) || overlaps(codes, cb, scales, sb) ||
+        overlaps(codes, cb, x, static_cast<size_t>(M) * K * 2) || overlaps(scales, sb, x, static_cast<size_t>(M) * K * 2))
+      return MACAQ_ERR_ALIAS;
+  }
+  int dev, sms;
+  st = current_device(dev, sms);
+  if (st != MACAQ_OK) return st;
+  const int bi = token_tile == 16 ? 0 : token_tile == 32 ? 1 : token_tile == 64 ? 2 : 3;
+  if (k_split > 1 && max_active_clusters_any(bi, k_split) < 1) return MACAQ_ERR_SHAPE;
+  const FusedPlan plan{token_tile, k_split, static_cast<int>(pad128(N) / 128) * ceil_div(M, token_tile) * k_split};
+  FusedParams p{};
+  p.Wq = Wq; p.Ws = Ws; p.x = x; p.D = D; p.y = y;
+  p.M = static_cast<int>(M); p.N = static_cast<int>(N); p.K = static_cast<int>(K);
+  p.NT = static_cast<int>(pad128(N) / 128); p.KT = KT;
+  p.S = k_split;
+  p.status = status;
+  p.plain = pl ? 1 : 0;
+  p.out_scale = pl ? 1.0f : 0.03125f;
+  p.dump_codes = codes;
+  p.dump_scales = scales;
+  // without a copy the product instantiation runs, exactly as macaq_dense_mm would run this plan
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = codes != nullptr ? launch_fused_kind<false, true>(p, plan, s) : launch_fused_kind<false, false>(p, plan, s);
+  return e == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
+}
+
+int macaq_test_wait_expiry(int64_t timeout_ns, int32_t* status, void* stream) {
+  if (timeout_ns < 1000 || timeout_ns > 1000000000) return MACAQ_ERR_SHAPE;
+  if (!status) return MACAQ_ERR_NULL;
+  if (!aligned16(status)) return MACAQ_ERR_ALIGN;
+  int dev, sms;
+  const int st = current_device(dev, sms);
+  if (st != MACAQ_OK) return st;
+  wait_expiry_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint64_t>(timeout_ns), status);
+  return cudaPeekAtLastError() == cudaSuccess ? MACAQ_OK : MACAQ_ERR_CUDA;
 }
 
 int macaq_unfused_dense_mm(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y,
