@@ -261,9 +261,13 @@ def capture(fn, stream):
 def time_graph(g, flush, stream, reps: int, warm: int = 3, cold: bool = True):
     """Mean (10% trimmed at each end) and IQR of the device time (us) of one graph
     replay, CUDA events on `stream`; the L2 flush (when `cold`) runs before the
-    start event.  Event timestamps on this GPU advance in 2.048 us ticks; each
-    replay starts at an independent phase of the tick, so the mean of the ticked
-    durations is unbiased where a median would snap to the tick grid."""
+    start event.  Event timestamps on this GPU advance in 2.048 us ticks, and a
+    replay that follows the same flush kernel starts at the same phase of the tick
+    every time, so every sample would tick the same way.  A GPU-side spin of a
+    seeded random 0-4,000 cycles (about 0-2 us, outside the timed interval)
+    before each start event spreads the start phase over the tick: the mean of
+    the ticked durations is then unbiased."""
+    rng = np.random.default_rng(12345)
     with torch.cuda.stream(stream):
         for _ in range(warm):
             g.replay()
@@ -271,6 +275,7 @@ def time_graph(g, flush, stream, reps: int, warm: int = 3, cold: bool = True):
         for _ in range(reps):
             if cold:
                 flush()
+            torch.cuda._sleep(int(rng.integers(0, 4000)))
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
@@ -400,6 +405,7 @@ def main():
                     help="CFG or CFG:IDX: only run these problems' calls --iters times (for profilers; no JSON)")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--unfused", action="store_true", help="with --only: the unfused ablation instead")
+    ap.add_argument("--epilogue", action="store_true", help="with --only: the call with bias and GELU_TANH")
     args = ap.parse_args()
     if args.only is not None:
         run_only(args)
@@ -461,9 +467,11 @@ def main():
     sampler.start()
     time.sleep(0.3)
     step_ev = []
+    phase = np.random.default_rng(54321)
     with torch.cuda.stream(stream):
         for _ in range(args.steps):
             flush()
+            torch.cuda._sleep(int(phase.integers(0, 4000)))  # start phase spread over the event tick (time_graph)
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
             a.record(stream)
@@ -577,7 +585,12 @@ def run_only(args):
         pp = Prepared(p, device, mq)
         for _ in range(args.iters):
             flush_buf.fill_(1)
-            pp.run_unfused(mq) if args.unfused else pp.run(mq)
+            if args.unfused:
+                pp.run_unfused(mq)
+            elif args.epilogue:
+                pp.run_epilogue(mq)
+            else:
+                pp.run(mq)
         torch.cuda.synchronize()
         print("ran", p.name, flush=True)
         del pp
