@@ -89,13 +89,14 @@ def test_weight_list_entry_overlapping_y_is_refused_on_the_device():
     y = torch.full((need // (2 * p.N) + 64, p.N), 7.0, dtype=torch.bfloat16, device="cuda")[:p.M]
     fake = y.view(torch.uint8).reshape(-1)  # y's own bytes posing as expert 1's code images
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
-    tables = torch.tensor([[Wq_l[0].data_ptr(), fake.data_ptr(), Wq_l[2].data_ptr()],
-                           [Ws_l[0].data_ptr(), Ws_l[1].data_ptr(), Ws_l[2].data_ptr()]], dtype=torch.int64).cuda()
+    # two separate tables: each must start 16-byte aligned
+    wq_table = torch.tensor([Wq_l[0].data_ptr(), fake.data_ptr(), Wq_l[2].data_ptr()], dtype=torch.int64).cuda()
+    ws_table = torch.tensor([Ws_l[0].data_ptr(), Ws_l[1].data_ptr(), Ws_l[2].data_ptr()], dtype=torch.int64).cuda()
     ws = torch.zeros(mq.workspace_bytes(p.M, p.N, p.K, p.E), dtype=torch.uint8, device="cuda")
     import ctypes
     P = ctypes.c_void_p
-    rc = mq.lib().macaq_grouped_mm_list(P(x.data_ptr()), P(D.data_ptr()), P(tables[0].data_ptr()),
-                                        P(tables[1].data_ptr()), P(glt.data_ptr()), 1, p.E, None, 0,
+    rc = mq.lib().macaq_grouped_mm_list(P(x.data_ptr()), P(D.data_ptr()), P(wq_table.data_ptr()),
+                                        P(ws_table.data_ptr()), P(glt.data_ptr()), 1, p.E, None, 0,
                                         P(y.data_ptr()), p.M, p.N, p.K, P(ws.data_ptr()), ws.numel(),
                                         P(status.data_ptr()), P(torch.cuda.current_stream().cuda_stream))
     torch.cuda.synchronize()
