@@ -200,6 +200,27 @@ int macaq_grouped_mm_ex(const uint16_t *x_dev, const float *D_dev, const uint8_t
                         int act_type, uint16_t *y_dev, int64_t M, int64_t N, int64_t K, void *workspace_dev,
                         size_t workspace_bytes, int32_t *status_dev, void *stream);
 
+/* FP8 output: the _ex calls with the result written as OCP FP8 E4M3 codes (one
+ * byte per element, [M, N] row-major) instead of BF16, for a following layer
+ * that reads FP8 (the npu_grouped_matmul page's output_dtype parameter selects
+ * the output type; this is its FP8 choice):
+ *     y8 = E4M3( v * y_scale ),  v = act(2^-5 * (block-scaled FP32 sum) + bias[n])
+ * with v as in macaq_dense_mm_ex, the product with y_scale rounded to FP32 and
+ * then to E4M3 by round-to-nearest-even with saturation at +-448 (E4M3 has no
+ * infinity; a caller dequantises with y8 / y_scale).  y_scale must be finite
+ * and > 0, else MACAQ_ERR_SHAPE.  The dense call runs the quantise-once path
+ * for every M (one quantisation kernel, then the block-scaled GEMM) and needs
+ * macaq_unfused_workspace_bytes(M, K) bytes of workspace; the grouped call
+ * needs macaq_workspace_bytes(M, N, K, E).  Other arguments, refusals and
+ * device errors as in macaq_dense_mm_ex / macaq_grouped_mm_ex. */
+int macaq_dense_mm_fp8(const uint16_t *x_dev, const float *D_dev, const uint8_t *Wq_dev, const uint8_t *Ws_dev,
+                       const float *bias_dev, int act_type, float y_scale, uint8_t *y8_dev, int64_t M, int64_t N,
+                       int64_t K, void *workspace_dev, size_t workspace_bytes, int32_t *status_dev, void *stream);
+int macaq_grouped_mm_fp8(const uint16_t *x_dev, const float *D_dev, const uint8_t *Wq_dev, const uint8_t *Ws_dev,
+                         const int64_t *group_list_dev, int group_list_type, int64_t E, const float *bias_dev,
+                         int act_type, float y_scale, uint8_t *y8_dev, int64_t M, int64_t N, int64_t K,
+                         void *workspace_dev, size_t workspace_bytes, int32_t *status_dev, void *stream);
+
 /* Grouped MACAQ linear with one weight tensor per expert: npu_grouped_matmul's
  * weight given as a list of tensors (parameter weight, List[Tensor]; the
  * single-x / several-weight / single-y case of its constraints), with its

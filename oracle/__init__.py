@@ -91,6 +91,10 @@ def _L():
             "oracle_quantize_plain": (I, [P, I64, I64, P, P]),
             "oracle_act_rotate_reading": (I, [P, P, I64, I64, I, P]),
             "oracle_num_threads": (I, []),
+            "oracle_e4m3_decode": (ctypes.c_double, [I]),
+            "oracle_f64_to_e4m3": (I, [ctypes.c_double]),
+            "oracle_f64_to_e4m3_array": (None, [P, I64, P]),
+            "oracle_gemm_fp8": (I, [P, P, P, P, I64, I64, I64, P, I, ctypes.c_double, P, I]),
         }
         for name, (res, args) in sig.items():
             f = getattr(lib, name)
@@ -327,6 +331,34 @@ def dense_mm_ex(x_bf16, D, W, bias=None, act_type: int = 0, nthreads: int = 0) -
     qa, sa = quantize_act(x_bf16, D, nthreads)
     qw, sw = quantize_weights(W, D, nthreads)
     return gemm_ex(qa, sa, qw, sw, bias, act_type, nthreads)
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """Values of OCP FP8 E4M3 codes (binary64; NaN for S.1111.111)."""
+    c = np.asarray(codes, dtype=np.int64)
+    f = _L().oracle_e4m3_decode
+    return np.array([f(int(v)) for v in c.ravel()], np.float64).reshape(c.shape)
+
+
+def f64_to_e4m3(v) -> np.ndarray:
+    """binary64 -> E4M3 codes: round to nearest even, saturating at +-448 (the FP8
+    output format; OCP FP8 E4M3)."""
+    v = _c(v, np.float64)
+    out = np.empty(v.shape, np.uint8)
+    _L().oracle_f64_to_e4m3_array(_p(v.ravel()), v.size, _p(out.reshape(-1)))
+    return out
+
+
+def gemm_fp8(qa, sa, qw, sw, bias=None, act_type: int = 0, y_scale: float = 1.0, nthreads: int = 0) -> np.ndarray:
+    """FP8 (E4M3) output of the layer: E4M3(act(2^-5 * exact sum + bias) * y_scale), [M, N] codes."""
+    qa, sa, qw, sw = (_c(a, np.uint8) for a in (qa, sa, qw, sw))
+    M, N, K = qa.shape[0], qw.shape[0], qa.shape[1] * 2
+    y = np.empty((M, N), np.uint8)
+    b, bp = _bias_ptr(bias)
+    st = _L().oracle_gemm_fp8(_p(qa), _p(sa), _p(qw), _p(sw), M, N, K, bp, int(act_type), float(y_scale), _p(y),
+                              nthreads)
+    assert st == OK, st
+    return y
 
 
 def group_offsets(group_list, group_list_type: int, M: int):

@@ -707,6 +707,81 @@ int oracle_gemm_at_ex(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, c
 }
 
 /* ------------------------------------------------------------------ */
+/* FP8 output (E4M3)                                                   */
+/* ------------------------------------------------------------------ */
+
+/* OCP FP8 E4M3 (the "fn" form: no infinities, S.1111.111 is NaN, largest
+ * finite magnitude 448 = 1.75 * 2^8, smallest subnormal 2^-9): the value of a
+ * code.  Exponent bias 7; exponent field 0 holds the subnormals m/8 * 2^-6. */
+double oracle_e4m3_decode(int code)
+{
+    int s = (code >> 7) & 1, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp(8.0 + m, e - 10); /* (1 + m/8) 2^(e-7) */
+    return s ? -v : v;
+}
+
+/* binary64 -> E4M3 code: round to nearest, ties to even (even last mantissa
+ * bit), magnitudes at or above 448 saturate to 448 (the rounding never goes
+ * past it below that), NaN stays NaN; the code's sign bit copies the value's. */
+int oracle_f64_to_e4m3(double v)
+{
+    int sign = signbit(v) ? 0x80 : 0;
+    if (isnan(v))
+        return sign | 0x7f;
+    double a = fabs(v);
+    if (a >= 448.0)
+        return sign | 0x7e;
+    if (a == 0.0)
+        return sign;
+    int e = ilogb(a);                     /* a in [2^e, 2^(e+1)) */
+    int lsb = e >= -6 ? e - 3 : -9;       /* weight of the last mantissa bit */
+    double r = ldexp(nearbyint(ldexp(a, -lsb)), lsb);  /* exact scaling, round half to even */
+    if (r < ldexp(1.0, -6))               /* subnormal: m steps of 2^-9 */
+        return sign | (int)ldexp(r, 9);
+    int er = ilogb(r);                    /* rounding may carry into the next binade */
+    int m = (int)ldexp(r, 3 - er) - 8;
+    return sign | ((er + 7) << 3) | m;
+}
+
+void oracle_f64_to_e4m3_array(const double *v, int64_t n, uint8_t *out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = (uint8_t)oracle_f64_to_e4m3(v[i]);
+}
+
+/* FP8 output of the layer: y8[m, n] = E4M3(act(2^-5 * exact sum + bias[n]) * y_scale),
+ * the epilogue value and its product with the output scale in binary64, one
+ * rounding to E4M3 (bias may be NULL). */
+int oracle_gemm_fp8(const uint8_t *qa, const uint8_t *sa, const uint8_t *qw, const uint8_t *sw, int64_t M,
+                    int64_t N, int64_t K, const float *bias, int act, double y_scale, uint8_t *y8, int nthreads)
+{
+    if (!act_supported(act))
+        return ORACLE_ERR_ACT_TYPE;
+    if (K <= 0 || K % 32 != 0)
+        return ORACLE_ERR_SHAPE;
+#ifdef _OPENMP
+    if (nthreads > 0)
+        omp_set_num_threads(nthreads);
+#pragma omp parallel for collapse(2) schedule(static)
+#endif
+    for (int64_t m = 0; m < M; m++)
+        for (int64_t n = 0; n < N; n++) {
+            double s = exact_dot_f64(qa + m * (K / 2), sa + m * (K / 32), qw + n * (K / 2), sw + n * (K / 32), K, -5);
+            if (bias)
+                s += (double)bias[n];
+            y8[m * N + n] = (uint8_t)oracle_f64_to_e4m3(oracle_act(s, act) * y_scale);
+        }
+    (void)nthreads;
+    return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ */
 /* Grouped form: rows [cum[g-1], cum[g]) use expert g                  */
 /* ------------------------------------------------------------------ */
 

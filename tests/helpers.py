@@ -88,3 +88,28 @@ def assert_mx_equal(codes, scales, ref_codes, ref_scales, label: str = ""):
     bad = np.argwhere((c != r).any(axis=-1) & finite)
     assert bad.size == 0, f"{label}: codes differ from the oracle in {len(bad)} blocks, first {bad[:3].tolist()}"
 
+
+
+def compare_fp8(y8: np.ndarray, ref8: np.ndarray, label: str = "") -> dict:
+    """FP8 (E4M3) outputs against the oracle's correctly rounded codes, with the
+    bound of compare() carried over to the FP8 grid: each decoded value within
+    1e-2 x rms of the oracle's decoded outputs (the kernels' FP32 accumulation
+    order and their half-precision tanh in the gated activations) plus one E4M3
+    step at the oracle's value (the GPU's FP32 result may land on the other side
+    of a rounding boundary; the step is 2^-9 below the normal range), and the
+    decoded outputs keep cosine >= 0.9999."""
+    import oracle
+    a = oracle.e4m3_decode(np.asarray(y8).ravel())
+    b = oracle.e4m3_decode(np.asarray(ref8).ravel())
+    assert not np.isnan(a).any(), f"{label}: NaN output"
+    rms = float(np.sqrt(np.mean(b * b))) if b.size else 0.0
+    step = np.exp2(np.floor(np.log2(np.maximum(np.abs(b), 2.0 ** -6))) - 3)
+    bad = np.flatnonzero(np.abs(a - b) > 1e-2 * rms + step)
+    denom = float(np.linalg.norm(a) * np.linalg.norm(b))
+    cos = float(a @ b / denom) if denom > 0 else 1.0
+    stats = {"cos": cos, "exact_share": float(np.mean(np.asarray(y8).ravel() == np.asarray(ref8).ravel())),
+             "within_one_step_share": float(np.mean(np.abs(a - b) <= step)) if b.size else 1.0,
+             "n": int(a.size)}
+    assert bad.size == 0, (label, stats, bad[:5], a[bad[:5]], b[bad[:5]])
+    assert cos >= 0.9999, (label, stats)
+    return stats

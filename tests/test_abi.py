@@ -227,3 +227,30 @@ def test_weight_list_and_transposed_refusals_by_name(L):
     assert L.macaq_prepare_weights_transposed(None, D, 1, 1024, 1024, Wq, Ws, None) == -1
     assert L.macaq_prepare_weights_transposed(W, P((2 << 32) + 4), 1, 1024, 1024, Wq, Ws, None) == -2
 
+
+
+@hidden_device
+def test_fp8_output_refusals_by_name(L):
+    y8 = P(5 << 32)
+
+    def d(scale=1.0, act=0, y=y8, M=16, N=1024, ws=None, nws=0):
+        return L.macaq_dense_mm_fp8(A, B, C, Dp, None, act, ctypes.c_float(scale), y, M, N, 1024, ws, nws, None,
+                                    None)
+
+    def g(scale=1.0, act=0, E=4):
+        return L.macaq_grouped_mm_fp8(A, B, C, Dp, P(9 << 32), 1, E, None, act, ctypes.c_float(scale), y8, 64, 1024,
+                                      1024, None, 0, None, None)
+
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        assert d(scale=bad) == -3                 # the output scale must be finite and positive
+        assert d(scale=bad, M=0) == -3            # refused even when there is nothing to compute
+        assert g(scale=bad) == -3
+    assert d(act=3) == -13
+    assert g(act=3) == -13
+    assert d(y=None) == -1
+    assert d(y=P((5 << 32) + 8)) == -2            # the FP8 output starts 16-byte aligned like the others
+    assert d(y=P((1 << 32) + 4096)) == -5         # y8 inside x
+    assert d(N=24) == -3
+    assert d() == -11                             # accepted; the missing workspace is the next refusal
+    assert g() == -11
+    assert d(M=0) == 0

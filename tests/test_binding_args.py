@@ -115,3 +115,16 @@ def test_weight_list_and_transposed_refusals():
     with pytest.raises(ValueError, match="W_kn must be torch.float32"):
         mq.prepare_weights_transposed(torch.zeros((K, N), dtype=torch.float64), torch.ones(K))
 
+
+
+def test_fp8_output_refusals():
+    with pytest.raises(ValueError, match="x must be torch.bfloat16"):
+        mq.dense_mm_fp8(**dense_args(x=torch.zeros((M, K))), y_scale=1.0)
+    with pytest.raises(ValueError, match="Wq holds"):
+        mq.dense_mm_fp8(**dense_args(Wq=torch.zeros(100, dtype=torch.uint8)), y_scale=1.0)
+    with pytest.raises(ValueError, match="expected contiguous CUDA tensors"):
+        mq.dense_mm_fp8(**dense_args(), y_scale=1.0)
+    with pytest.raises(ValueError, match="group_list must be torch.int64"):
+        mq.grouped_mm_fp8(**grouped_args(group_list=torch.tensor([5, 5, 6], dtype=torch.int32)), y_scale=1.0)
+    with pytest.raises(ValueError, match="expected contiguous CUDA tensors"):
+        mq.grouped_mm_fp8(**grouped_args(), y_scale=1.0)

@@ -825,3 +825,88 @@ def test_calibration_reproduces_the_generator_factors():
     g = synth.grouped(2048, 32, 512, 64, seed=1, dist="zipf", group_list_type=0)
     st, D = oracle.calibrate_d(g.x, g.W, g.group_list, g.group_list_type)
     assert st == oracle.OK and np.array_equal(D, g.D)
+
+
+# ----------------------------------------------------------------------------
+# FP8 (E4M3) output: OCP FP8 E4M3, round to nearest even, saturating at 448
+# ----------------------------------------------------------------------------
+
+def _e4m3_library_values():
+    import torch
+    return torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+
+
+def test_e4m3_decode_matches_the_library_format_for_every_code():
+    ours = oracle.e4m3_decode(np.arange(256))
+    lib = _e4m3_library_values()
+    nan = np.isnan(lib)
+    assert np.array_equal(nan, np.isnan(ours)) and nan.sum() == 2          # 0x7f and 0xff
+    assert np.array_equal(ours[~nan], lib[~nan])
+    assert ours[0x7e] == 448.0 and ours[1] == 2.0 ** -9 and ours[0x08] == 2.0 ** -6
+
+
+def test_e4m3_encode_round_trips_every_code():
+    vals = oracle.e4m3_decode(np.arange(256))
+    codes = np.arange(256)
+    keep = ~np.isnan(vals)
+    assert np.array_equal(oracle.f64_to_e4m3(vals[keep]), codes[keep])
+
+
+def test_e4m3_encode_is_the_nearest_code_ties_to_even_brute_force():
+    lib = _e4m3_library_values()
+    finite = np.flatnonzero(~np.isnan(lib))
+    rng = np.random.default_rng(0)
+    v = np.concatenate([rng.uniform(-460, 460, 20000), rng.standard_normal(20000) * np.exp2(rng.integers(-12, 6, 20000)),
+                        (lib[finite][:-1] + np.diff(lib[finite])) / 2])   # include midpoints (ties)
+    v = v[np.isfinite(v)]
+    got = oracle.f64_to_e4m3(v)
+    for x, c in zip(v[:6000], got[:6000]):
+        if abs(x) >= 448:
+            assert c & 0x7f == 0x7e and (c >> 7) == int(np.signbit(x)), (x, c)
+            continue
+        d = np.abs(lib[finite] - x)
+        best = finite[d == d.min()]
+        if best.size > 1:                       # a tie: the even mantissa; the sign of zero follows x
+            best = best[(best & 1) == 0]
+            best = best[((best >> 7) == int(np.signbit(x))) | (lib[best] != 0)]
+        assert c in set(best.tolist()) or (lib[c] == 0 and lib[best[0]] == 0), (x, c, best)
+
+
+def test_e4m3_encode_matches_the_library_conversion_in_range():
+    import torch
+    rng = np.random.default_rng(1)
+    v = (rng.standard_normal(50000) * np.exp2(rng.integers(-10, 8, 50000))).astype(np.float32)
+    v = v[np.abs(v) < 440]
+    lib = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(oracle.f64_to_e4m3(v.astype(np.float64)), lib)
+
+
+def test_fp8_gemm_exact_where_the_product_is_representable():
+    # one nonzero element per row of K = 32: activation code 2 (1.0) at scale 127,
+    # weight codes 1..7 and 9..15 at scale 127 + k: y = w * 2^k / 32 * y_scale
+    K, N = 32, 14
+    qa = np.zeros((1, K // 2), np.uint8); qa[0, 0] = 2
+    sa = np.full((1, 1), 127, np.uint8)
+    w = [c for c in range(1, 16) if c != 8]
+    qw = np.zeros((N, K // 2), np.uint8); qw[:, 0] = w
+    sw = np.full((N, 1), 130, np.uint8)                  # 2^3
+    y = oracle.gemm_fp8(qa, sa, qw, sw, y_scale=4.0)     # w * 8 / 32 * 4 = w
+    want = oracle.f64_to_e4m3(np.array([oracle.e2m1_decode(c) for c in w]))
+    assert np.array_equal(y[0], want)
+    assert np.array_equal(oracle.e4m3_decode(y[0]), [oracle.e2m1_decode(c) for c in w])
+    # saturation and RELU on the same values
+    assert np.all(oracle.gemm_fp8(qa, sa, qw, sw, y_scale=1e4)[0] & 0x7f == 0x7e)
+    yr = oracle.gemm_fp8(qa, sa, qw, sw, act_type=1, y_scale=4.0)[0]
+    assert np.all(oracle.e4m3_decode(yr) == np.maximum([oracle.e2m1_decode(c) for c in w], 0.0))
+
+
+def test_fp8_gemm_agrees_with_the_bf16_path_within_one_step():
+    p = synth.dense(24, 256, 64, seed=5)
+    qa, sa = oracle.quantize_act(p.x, p.D[0])
+    qw, sw = oracle.quantize_weights(p.W[0], p.D[0])
+    y16 = synth.bf16_bits_to_f32(oracle.gemm(qa, sa, qw, sw)).astype(np.float64)
+    s = 100.0 / np.abs(y16).max()
+    y8 = oracle.e4m3_decode(oracle.gemm_fp8(qa, sa, qw, sw, y_scale=s))
+    step = np.exp2(np.floor(np.log2(np.maximum(np.abs(y16 * s), 2.0 ** -6))) - 3)
+    assert np.all(np.abs(y8 - y16 * s) <= step)
+

@@ -104,6 +104,10 @@ _SIG = {
     "macaq_prepare_weights_transposed": (ctypes.c_int, [_P, _P, _I64, _I64, _I64, _P, _P, _P]),
     "macaq_grouped_mm_list": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int, _P, _I64,
                                              _I64, _I64, _P, ctypes.c_size_t, _P, _P]),
+    "macaq_dense_mm_fp8": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, ctypes.c_float, _P, _I64, _I64, _I64,
+                                          _P, ctypes.c_size_t, _P, _P]),
+    "macaq_grouped_mm_fp8": (ctypes.c_int, [_P, _P, _P, _P, _P, ctypes.c_int, _I64, _P, ctypes.c_int,
+                                            ctypes.c_float, _P, _I64, _I64, _I64, _P, ctypes.c_size_t, _P, _P]),
 }
 
 
@@ -307,6 +311,47 @@ def grouped_mm_list(x: torch.Tensor, D: torch.Tensor, Wq_list, Ws_list, group_li
                                    int(group_list_type), E, _ptr(bias), int(act_type), _ptr(y), M, N, K, _ptr(ws),
                                    _nbytes(ws), _ptr(status), _stream_ptr(stream)), "macaq_grouped_mm_list")
     return y
+
+
+def dense_mm_fp8(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, N: int, y_scale: float,
+                 bias: torch.Tensor | None = None, act_type: int = ACT_NONE, out: torch.Tensor | None = None,
+                 status: torch.Tensor | None = None, stream=None, ws: torch.Tensor | None = None) -> torch.Tensor:
+    """MACAQ linear with an FP8 output: E4M3 codes (uint8 [M, N]) of act(v + bias) * y_scale."""
+    _dense_args(x, D, Wq, Ws, N, status)
+    _require_cuda(x, D, Wq, Ws, out, status)
+    M, K = x.shape
+    _check_bias(bias, (N,))
+    with _on(stream):
+        y8 = torch.empty((M, N), dtype=torch.uint8, device=x.device) if out is None else out
+    if y8.dtype != torch.uint8 or tuple(y8.shape) != (M, N):
+        raise ValueError(f"out must be uint8 of shape {(M, N)}")
+    L = lib()
+    ws = workspace(int(L.macaq_unfused_workspace_bytes(M, K)), x.device, stream, ws)
+    _check(L.macaq_dense_mm_fp8(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(bias), int(act_type), float(y_scale),
+                                _ptr(y8), M, N, K, _ptr(ws), _nbytes(ws), _ptr(status), _stream_ptr(stream)),
+           "macaq_dense_mm_fp8")
+    return y8
+
+
+def grouped_mm_fp8(x: torch.Tensor, D: torch.Tensor, Wq: torch.Tensor, Ws: torch.Tensor, group_list: torch.Tensor,
+                   group_list_type: int, N: int, y_scale: float, bias: torch.Tensor | None = None,
+                   act_type: int = ACT_NONE, out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                   stream=None, ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Grouped MACAQ linear with an FP8 output (E4M3 codes, uint8 [M, N])."""
+    E = _grouped_args(x, D, Wq, Ws, group_list, group_list_type, N, status)
+    _require_cuda(x, D, Wq, Ws, group_list, out, status)
+    M, K = x.shape
+    _check_bias(bias, (E, N))
+    with _on(stream):
+        y8 = torch.empty((M, N), dtype=torch.uint8, device=x.device) if out is None else out
+    if y8.dtype != torch.uint8 or tuple(y8.shape) != (M, N):
+        raise ValueError(f"out must be uint8 of shape {(M, N)}")
+    L = lib()
+    ws = workspace(int(L.macaq_workspace_bytes(M, N, K, E)), x.device, stream, ws)
+    _check(L.macaq_grouped_mm_fp8(_ptr(x), _ptr(D), _ptr(Wq), _ptr(Ws), _ptr(group_list), int(group_list_type), E,
+                                  _ptr(bias), int(act_type), float(y_scale), _ptr(y8), M, N, K, _ptr(ws),
+                                  _nbytes(ws), _ptr(status), _stream_ptr(stream)), "macaq_grouped_mm_fp8")
+    return y8
 
 
 def _check_bias(bias, shape):

@@ -237,7 +237,9 @@ __global__ void __launch_bounds__(256) quant_canonical_kernel(const uint16_t* __
   if (m >= M) return;
   uint4 cv;
   uint32_t sc;
-  act_block(xv, r + c * kQRcpStride, cv, sc);
+  uint64_t r2[16];
+  load_rcp_block(r + c * kQRcpStride, r2);
+  act_block(xv, r2, cv, sc);
   *reinterpret_cast<uint4*>(codes + static_cast<int64_t>(m) * (K / 2) + (k0 + c * kBlk) / 2) = cv;
   scales[static_cast<int64_t>(m) * (K / kBlk) + k0 / kBlk + c] = static_cast<uint8_t>(sc);
 }
@@ -562,16 +564,25 @@ struct QuantParams {
   int plain;            // plain MXFP4 (no D, no Hadamard; D not read)
 };
 
-constexpr int kQuantStages = 3;                 // ring slots: the current unit and two ahead
-constexpr int kQuantAhead = kQuantStages - 1;
-constexpr int kQuantSlotBytes = 256 * 64;       // one unit: 256 threads x one 32-element block
-// Within a slot, 16-byte chunk j of thread i sits at (j * 256 + i) * 16: a warp's
-// loads of chunk j are 512 consecutive bytes (no bank conflict).
-constexpr int kQuantSmem = kQuantStages * kQuantSlotBytes;
+// Quantise-once prologue over all rows.  A CTA owns one K tile and a contiguous
+// run of 32-row slabs (dense: rows 32 s..; grouped: the slab table, in group
+// order); a thread owns row tr of the slab and the 32-channel block c of the K
+// tile, i.e. one MX block per slab.  The activations go straight from global
+// memory into registers, one slab ahead of the one being encoded; the block's
+// 32 reciprocals stay in registers while consecutive slabs use the same row of
+// D (dense: always; grouped: until the group changes, a CTA-uniform event).  No
+// shared-memory staging and no barrier per slab.
+constexpr int kQuantCtasPerSm = 2;
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.cs.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
 
-__global__ void __launch_bounds__(256, 4) quant_tiles_kernel(const __grid_constant__ QuantParams p) {
-  extern __shared__ __align__(16) uint8_t qsmem[];  // ring [kQuantStages][4 chunks][256 threads][16]
-  __shared__ __align__(16) float r[2][kQRcpTile];
+__global__ void __launch_bounds__(256, kQuantCtasPerSm) quant_tiles_kernel(const __grid_constant__ QuantParams p) {
+  __shared__ __align__(16) float rs[kQRcpTile];
   pdl_trigger();  // the GEMM may start streaming weights; it waits for our results before reading them
   pdl_wait();     // x (and the grouped tables) may come from the preceding kernels
   const int KT = p.K / kKTile;
@@ -580,94 +591,62 @@ __global__ void __launch_bounds__(256, 4) quant_tiles_kernel(const __grid_consta
     if (*p.valid == 0) return;
     L = *p.nslabs;
   }
-  const int units = L * KT;
-  const int G = static_cast<int>(gridDim.x);
-  if (L <= 0 || static_cast<int>(blockIdx.x) >= units) return;
+  // the grid is KT x per_kt CTAs: CTA (kt, j) takes slabs [j q, (j + 1) q)
+  const int per_kt = static_cast<int>(gridDim.x) / KT;
+  const int kt = static_cast<int>(blockIdx.x) % KT, j = static_cast<int>(blockIdx.x) / KT;
+  const int q = (L + per_kt - 1) / per_kt;
+  int s = j * q;
+  const int s_end = min(L, s + q);
+  if (L <= 0 || j >= per_kt || s >= s_end) return;
   const int tr = threadIdx.x >> 3, c = threadIdx.x & 7;
-  const int gq = G / L, gr = G % L;  // one stride of G units: gq K tiles and gr slabs further
-  struct Unit {
-    uint8_t* img;  // the unit's activation image
-    float d;       // D of this thread's channel (loaded with the activations)
-    int t;         // this thread's row in the tile; negative: the row does not exist
+  const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
+  // (group, first row, rows, quarter = 32-row slot in the tile images)
+  auto slab = [&](int sl) -> int4 {
+    if (p.slabs != nullptr) return p.slabs[sl];
+    return make_int4(0, sl * 32, min(32, p.M - sl * 32), sl);
   };
-  // Issues the activation copy of the unit at (slab s, K tile kt) into ring `slot`.
-  auto fetch = [&](int sl, int kt, int slot) {
-    Unit w;
-    int ex = 0, row0, nrows, quarter;
-    if (p.slabs != nullptr) {
-      const int4 e = p.slabs[sl];
-      ex = e.x;
-      row0 = e.y;
-      nrows = e.z;
-      quarter = e.w;
-    } else {
-      row0 = sl * 32;
-      nrows = min(32, p.M - row0);
-      quarter = sl;
-    }
-    const bool live = tr < nrows;
-    w.t = live ? (quarter & 3) * 32 + tr : -1;
-    w.img = p.Aq + (static_cast<size_t>(quarter >> 2) * KT + kt) * kActImageBytes;
-    const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
-    w.d = p.plain ? 1.f : __ldg(p.D + static_cast<int64_t>(ex) * p.K + k0 + threadIdx.x);
-    if (live) {
-      const uint16_t* src = p.x + (static_cast<int64_t>(row0) + tr) * p.K + k0 + c * kBlk;
-      uint8_t* dst = qsmem + slot * kQuantSlotBytes + threadIdx.x * 16;
+  auto load = [&](const int4& e, uint4 (&v)[4]) {
+    if (tr < e.z) {
+      const uint4* src = reinterpret_cast<const uint4*>(p.x + (static_cast<int64_t>(e.y) + tr) * p.K + k0 + c * kBlk);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) cp_async16(dst + 4096 * i, src + 8 * i);
-    }
-    cp_async_commit();  // one group per unit, empty when the row does not exist
-    return w;
-  };
-  // (fs, fk): slab and K tile of the next unit to fetch; fk == KT past the end
-  int fs = static_cast<int>(blockIdx.x) % L, fk = static_cast<int>(blockIdx.x) / L;
-  auto step = [&]() {
-    fs += gr;
-    fk += gq;
-    if (fs >= L) {
-      fs -= L;
-      ++fk;
+      for (int i = 0; i < 4; ++i) v[i] = ld_stream(src + i);
     }
   };
-  Unit ring[kQuantStages];
+  int4 e = slab(s);
+  uint4 xv[4], xn[4];
+  load(e, xv);
+  uint64_t r2[16];
+  int group = -1;  // the D row whose reciprocals r2 holds
+  for (;;) {
+    const bool more = s + 1 < s_end;
+    int4 en = e;
+    if (more) {
+      en = slab(s + 1);
+      load(en, xn);
+    }
+    if (!p.plain && e.x != group) {
+      __syncthreads();  // every thread holds the previous reciprocals in registers already
+      rs[qrcp_index(threadIdx.x)] = __frcp_rn(__ldg(p.D + static_cast<int64_t>(e.x) * p.K + k0 + threadIdx.x));
+      __syncthreads();
+      load_rcp_block(rs + c * kQRcpStride, r2);
+      group = e.x;
+    }
+    if (tr < e.z) {
+      uint4 cv;
+      uint32_t sc;
+      if (p.plain) act_block_plain(xv, cv, sc);
+      else act_block(xv, r2, cv, sc);
+      const int t = (e.w & 3) * 32 + tr;
+      uint8_t* img = p.Aq + (static_cast<size_t>(e.w >> 2) * KT + kt) * kActImageBytes;
+      *reinterpret_cast<uint4*>(img + code_chunk_offset(t, c)) = cv;
+      img[kTileCodeBytes + sf_offset(t, c)] = static_cast<uint8_t>(sc);
+    }
+    if (!more) break;
+    ++s;
+    e = en;
 #pragma unroll
-  for (int s = 0; s < kQuantAhead; ++s) {
-    if (fk < KT) ring[s] = fetch(fs, fk, s);
-    else cp_async_commit();
-    step();
+    for (int i = 0; i < 4; ++i) xv[i] = xn[i];
   }
-  int buf = 0;  // reciprocal buffer of this unit: alternates unit by unit
-  int u = static_cast<int>(blockIdx.x);
-  // unit i of this CTA uses ring slot i % kQuantStages; unrolled so slots are static
-  while (u < units) {
-#pragma unroll
-    for (int k = 0; k < kQuantStages; ++k) {
-      if (u >= units) break;
-      {  // the unit kQuantAhead ahead goes into the slot freed last iteration
-        const int sa = (k + kQuantAhead) % kQuantStages;
-        if (fk < KT) ring[sa] = fetch(fs, fk, sa);
-        else cp_async_commit();
-        step();
-      }
-      const Unit w = ring[k];
-      r[buf][qrcp_index(threadIdx.x)] = __frcp_rn(w.d);
-      cp_async_wait<kQuantAhead>();  // this thread's copy of this unit has landed
-      __syncthreads();               // every reciprocal written; r[buf] of two units back no longer read
-      if (w.t >= 0) {
-        uint4 cv;
-        uint32_t sc;
-        const uint4* xs = reinterpret_cast<const uint4*>(qsmem + k * kQuantSlotBytes) + threadIdx.x;
-        const uint4 xv[4] = {xs[0], xs[256], xs[512], xs[768]};
-        if (p.plain) act_block_plain(xv, cv, sc);
-        else act_block(xv, r[buf] + c * kQRcpStride, cv, sc);
-        *reinterpret_cast<uint4*>(w.img + code_chunk_offset(w.t, c)) = cv;
-        w.img[kTileCodeBytes + sf_offset(w.t, c)] = static_cast<uint8_t>(sc);
-      }
-      u += G;
-      buf ^= 1;
-    }
-  }
-  cp_async_wait<0>();  // no copy may still be writing this CTA's shared memory at exit
 }
 
 // ============================================================================
@@ -692,38 +671,52 @@ struct GemmParams {
   int act;                // act_type: 0 none, 1 RELU, 2 GELU_TANH, 4 FAST_GELU, 5 SILU
   const uint64_t* wq_list;  // weight-list form: [E] addresses of each expert's images (else nullptr)
   const uint64_t* ws_list;
+  uint8_t* y8;              // FP8 output: E4M3 codes [M, N] written instead of y (else nullptr)
+  float y8_scale;           // multiplies the epilogue value before the E4M3 rounding
 };
 
-// Epilogue of the 128 accumulator columns of one thread's row of its half
-// tile, already loaded into registers: v = acc * out_scale (+ bias[n]), then the
-// activation, packed to BF16 pairs.  kEpi < 0: scaling only (no bias, no
-// activation); otherwise act_type kEpi with an optional bias.  Columns n >= N
-// (the zero rows of a ragged weight tile) take no bias.
+// Epilogue of 32 accumulator columns of one thread's row, loaded into
+// registers: v = acc * out_scale (+ bias[n]), then the activation, packed to 16
+// BF16 pairs.  kEpi < 0: scaling only (no bias, no activation); otherwise
+// act_type kEpi with an optional bias, read from the tile's bias staged in
+// shared memory (sb: the 32 values of these columns; zero past N).
 template <int kEpi>
-__device__ __forceinline__ void finish128(const uint32_t (&r)[128], float os, const float* brow, int ncol0, int N,
-                                          uint32_t (&pk)[64]) {
-  const float2 os2 = make_float2(os, os);
+__device__ __forceinline__ float2 epi_pair(const uint32_t (&r)[32], int e, float2 os2, const float* sb) {
+  const float2 a = make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
   if constexpr (kEpi < 0) {
-#pragma unroll
-    for (int e = 0; e < 64; ++e) {
-      const float2 v = fmul2(make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1])), os2);
-      pk[e] = pack_bf16x2(v.x, v.y);
-    }
+    return fmul2(a, os2);
   } else {
-    const int nb = brow != nullptr ? N - ncol0 : 0;  // leading columns that take a bias (a multiple of 16)
+    const float2 b = *reinterpret_cast<const float2*>(sb + 2 * e);  // warp-uniform: a broadcast
+    return act_pair<kEpi>(ffma2(a, os2, b));
+  }
+}
+template <int kEpi>
+__device__ __forceinline__ void finish32(const uint32_t (&r)[32], float os, const float* sb, uint32_t* pk) {
+  const float2 os2 = make_float2(os, os);
 #pragma unroll
-    for (int c0 = 0; c0 < 128; c0 += 16) {
-      const bool inb = c0 + 16 <= nb;
+  for (int e = 0; e < 16; ++e) {
+    const float2 y = epi_pair<kEpi>(r, e, os2, sb);
+    pk[e] = pack_bf16x2(y.x, y.y);
+  }
+}
+// The same 32 columns as FP8 E4M3 codes (8 words, column 0 in the lowest byte):
+// each value times y8_scale in FP32, then rounded to nearest even with saturation
+// at +-448 (cvt.rn.satfinite; NaN stays NaN).
+__device__ __forceinline__ uint32_t e4m3x4(float2 a, float2 b) {
+  uint16_t lo, hi;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(lo) : "f"(a.x), "f"(a.y));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(hi) : "f"(b.x), "f"(b.y));
+  return static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+}
+template <int kEpi>
+__device__ __forceinline__ void finish32_fp8(const uint32_t (&r)[32], float os, const float* sb, float y8s,
+                                             uint32_t* pk) {
+  const float2 os2 = make_float2(os, os), s2 = make_float2(y8s, y8s);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        float2 b = make_float2(0.f, 0.f);
-        if (inb) b = __ldg(reinterpret_cast<const float2*>(brow + ncol0 + c0 + 2 * e));  // warp-uniform: a broadcast
-        const float2 v =
-            ffma2(make_float2(__uint_as_float(r[c0 + 2 * e]), __uint_as_float(r[c0 + 2 * e + 1])), os2, b);
-        const float2 y = act_pair<kEpi>(v);
-        pk[c0 / 2 + e] = pack_bf16x2(y.x, y.y);
-      }
-    }
+  for (int e = 0; e < 16; e += 2) {
+    const float2 y0 = fmul2(epi_pair<kEpi>(r, e, os2, sb), s2);
+    const float2 y1 = fmul2(epi_pair<kEpi>(r, e + 1, os2, sb), s2);
+    pk[e / 2] = e4m3x4(y0, y1);
   }
 }
 
@@ -745,7 +738,8 @@ constexpr int kOffSfa = kOffA + kTileCodeBytes;             // activation scales
 constexpr int kOffSfb = kOffSfa + kTileSfBytes;             // weight scales of the two images
 constexpr int kStageBytes = kOffSfb + 2 * kTileSfBytes;     // 52224
 constexpr int kStagingBytes = kRowsTile * 64 * 2;           // 128 rows x 64 columns of BF16, swizzled
-constexpr int kFixedBytes = kStagingBytes + 256;            // staging, barriers and flags
+constexpr int kBiasBytes = kTileN * 4;                       // the tile's 256 bias values
+constexpr int kFixedBytes = kStagingBytes + 256 + kBiasBytes;  // staging, barriers and flags, bias
 // TMEM: the accumulator in columns 0-255; from column 256, 24 columns of scales per
 // stage (activation scales 8, weight scales 16)
 constexpr int kTmemCols = 512;
@@ -880,7 +874,7 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
   if (p.gtp != nullptr) {
     pdl_wait();  // tables and activation images come from the preceding kernels
     if (*p.valid == 0) return;
-    goff = reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(full) + 256);
+    goff = reinterpret_cast<int64_t*>(reinterpret_cast<uint8_t*>(full) + 256 + kBiasBytes);
     gtp = reinterpret_cast<int*>(goff + p.E + 1);
     gexp = gtp + p.E + 1;
     if (p.wq_list != nullptr) {
@@ -1053,10 +1047,17 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
     const int et = threadIdx.x - 64;
     const float os = p.out_scale;
     const int tl = q * 32 + lane;
+    float* sbias = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 256);  // [256]
     for (int i = 0; i < my_tiles; ++i) {
       const GemmTile t = gemm_tile(p, blockIdx.x + i * gridDim.x, mtiles, goff, gtp, gexp);
+      if constexpr (kEpi >= 0) {
+        // the tile's 256 bias values, one per thread: every later read is a shared-memory
+        // broadcast instead of a global load in the middle of the epilogue's dependency chain
+        const int n = t.nt * kRowsTile + et;
+        sbias[et] = (p.bias != nullptr && n < p.N) ? __ldg(p.bias + static_cast<int64_t>(t.g) * p.N + n) : 0.f;
+      }
       if (et == 0) *epi_flag = mbar_wait(accf, i & 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
-      named_bar_sync(1, 256);  // also: every thread has finished reading the previous tile's staging
+      named_bar_sync(1, 256);  // also: every thread has finished reading the previous tile's staging and bias
       if (!*epi_flag) break;
       tc_fence_after();
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 128;
@@ -1081,30 +1082,46 @@ __global__ void __launch_bounds__(gemm::kThreads, 1) gemm_kernel(const __grid_co
           }
         }
       };
-      // The whole 128-column run of the row is loaded with one wait and the
-      // accumulator handed back at once, so the next tile's MMAs overlap the
-      // scaling (bias, activation), packing and write-out of this one.
-      uint32_t r[128];
-      tmem_ld_32x32b_x32(taddr + 0, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-      tmem_ld_32x32b_x32(taddr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-      tmem_ld_32x32b_x32(taddr + 64, *reinterpret_cast<uint32_t(*)[32]>(&r[64]));
-      tmem_ld_32x32b_x32(taddr + 96, *reinterpret_cast<uint32_t(*)[32]>(&r[96]));
+      // The row's 128 accumulator columns are loaded into registers with one wait
+      // and the accumulator is handed back at once: the next tile's MMAs overlap
+      // the scaling, bias and activation (bias from shared memory) and the write-out.
+      uint32_t r[4][32];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tmem_ld_32x32b_x32(taddr + 32 * j, r[j]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(acce);
       uint32_t pk[64];
-      {
-        const float* brow = nullptr;
-        if constexpr (kEpi >= 0) brow = p.bias != nullptr ? p.bias + static_cast<int64_t>(t.g) * p.N : nullptr;
-        finish128<kEpi>(r, os, brow, t.nt * kRowsTile + h * 128, p.N, pk);
-      }
+      if (p.y8 == nullptr) {
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        if ((ch >> 1) == h) stage_chunk(pk + (ch & 1) * 32);
-        named_bar_sync(1, 256);
-        store_chunk(ch);
-        if (ch < 3) named_bar_sync(1, 256);  // read out before the next chunk overwrites it
+        for (int j = 0; j < 4; ++j) finish32<kEpi>(r[j], os, sbias + h * 128 + 32 * j, pk + 16 * j);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          if ((ch >> 1) == h) stage_chunk(pk + (ch & 1) * 32);
+          named_bar_sync(1, 256);
+          store_chunk(ch);
+          if (ch < 3) named_bar_sync(1, 256);  // read out before the next chunk overwrites it
+        }
+      } else {
+        // FP8 output: a half's 128 columns are 128 bytes of a row, one staged chunk
+        // per half (the same swizzled staging), stored as 16-column pieces
+#pragma unroll
+        for (int j = 0; j < 4; ++j) finish32_fp8<kEpi>(r[j], os, sbias + h * 128 + 32 * j, p.y8_scale, pk + 8 * j);
+#pragma unroll
+        for (int ch = 0; ch < 2; ++ch) {
+          if (ch == h) stage_chunk(pk);
+          named_bar_sync(1, 256);
+          const int n0 = t.nt * kRowsTile + ch * 128;
+          if (n0 + 16 * c < p.N) {
+#pragma unroll 4
+            for (int rr = et >> 3; rr < t.rows; rr += 32) {
+              const uint4 o = *reinterpret_cast<const uint4*>(staging + rr * 128 + ((c ^ (rr & 7)) << 4));
+              *reinterpret_cast<uint4*>(p.y8 + static_cast<int64_t>(t.m0 + rr) * p.N + n0 + 16 * c) = o;
+            }
+          }
+          if (ch < 1) named_bar_sync(1, 256);
+        }
       }
     }
   }
@@ -1655,8 +1672,6 @@ int current_device(int& dev, int& sms) {
               cudaFuncSetAttribute(gemm_kernel<4>, a, gs) == cudaSuccess &&
               cudaFuncSetAttribute(gemm_kernel<5>, a, gs) == cudaSuccess;
     ok = ok && fused_attrs<16>() && fused_attrs<32>() && fused_attrs<64>() && fused_attrs<128>();
-    ok = ok && cudaFuncSetAttribute(quant_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmem) ==
-                   cudaSuccess;
     if (!ok) return MACAQ_ERR_CUDA;
     s.attrs_set = true;
   }
@@ -1845,14 +1860,15 @@ GroupedWs grouped_ws(int64_t M, int64_t K, int64_t E) {
 // plain: plain MXFP4 call, D is not used (and may be null).
 // weight_bytes: bytes of each of Wq and Ws when they are not prepared weights
 // (the weight-list form passes tables of addresses); 0: prepared images of E experts.
-int check_mm_args(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, uint16_t* y, int64_t M,
-                  int64_t N, int64_t K, int64_t E, bool plain = false, size_t weight_bytes = 0) {
+// ybytes: bytes of the output (0: BF16 [M, N]).
+int check_mm_args(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, void* y, int64_t M,
+                  int64_t N, int64_t K, int64_t E, bool plain = false, size_t weight_bytes = 0, size_t ybytes = 0) {
   if (M < 0 || M > INT32_MAX || !valid_nk(N, K)) return MACAQ_ERR_SHAPE;
   if (M == 0) return MACAQ_OK;
   if (!x || (!D && !plain) || !Wq || !Ws || !y) return MACAQ_ERR_NULL;
   if (!aligned16(x) || (!plain && !aligned16(D)) || !aligned16(Wq) || !aligned16(Ws) || !aligned16(y))
     return MACAQ_ERR_ALIGN;
-  const size_t ybytes = static_cast<size_t>(M) * N * 2;
+  if (ybytes == 0) ybytes = static_cast<size_t>(M) * N * 2;
   if (overlaps(y, ybytes, x, static_cast<size_t>(M) * K * 2) ||
       (!plain && overlaps(y, ybytes, D, static_cast<size_t>(E) * K * 4)) ||
       overlaps(y, ybytes, Wq, weight_bytes ? weight_bytes : macaq_weight_code_bytes(E, N, K)) ||
@@ -1867,11 +1883,12 @@ int check_ws(void* ws, size_t ws_bytes, size_t need, const void* y, size_t ybyte
   return MACAQ_OK;
 }
 
-// Persistent quantiser grid: four CTAs per SM at most, no more than the units
-// (32-row slabs x K tiles; for grouped calls an upper bound).
+// Quantiser grid: KT x per_kt CTAs, about kQuantCtasPerSm per SM, per_kt no
+// more than the slabs (for grouped calls an upper bound of them).
 int quant_grid(int64_t slabs, int KT, int sms) {
-  const int64_t units = slabs * KT;
-  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(units, static_cast<int64_t>(sms) * 4)));
+  int64_t per_kt = std::max<int64_t>(1, static_cast<int64_t>(sms) * kQuantCtasPerSm / KT);
+  per_kt = std::min<int64_t>(per_kt, std::max<int64_t>(1, slabs));
+  return static_cast<int>(per_kt * KT);
 }
 
 // Dense quantise-once: the quantiser over all rows, then the GEMM (launched as
@@ -1880,6 +1897,8 @@ int quant_grid(int64_t slabs, int KT, int sms) {
 struct Epilogue {
   const float* bias = nullptr;
   int act = 0;
+  uint8_t* y8 = nullptr;  // FP8 (E4M3) output instead of BF16
+  float y8_scale = 1.0f;
 };
 bool act_supported(int act) { return act == 0 || act == 1 || act == 2 || act == 4 || act == 5; }
 // bias: 16-byte aligned, rows * N floats, not overlapping y.
@@ -1912,7 +1931,7 @@ int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, c
   QuantParams qp{};
   qp.x = x; qp.D = D; qp.Aq = ws + w.act;
   qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.plain = plain ? 1 : 0;
-  if (launch_ex(quant_tiles_kernel, dim3(quant_grid((M + 31) / 32, KT, sms)), dim3(256), kQuantSmem, st, pdl, 1,
+  if (launch_ex(quant_tiles_kernel, dim3(quant_grid((M + 31) / 32, KT, sms)), dim3(256), 0, st, pdl, 1,
                 qp) !=
       cudaSuccess)
     return MACAQ_ERR_CUDA;
@@ -1924,6 +1943,8 @@ int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, c
   gp.out_scale = plain ? 1.0f : 0.03125f;
   gp.bias = ep.bias;
   gp.act = ep.act;
+  gp.y8 = ep.y8;
+  gp.y8_scale = ep.y8_scale;
   gp.status = status;
   gp.wait_for_producer = pdl ? 1 : 0;
   const int tiles = MT * gp.NT2;
@@ -2104,23 +2125,24 @@ static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, co
   if (E < 1 || E > kMaxGroups) return MACAQ_ERR_TOO_MANY_GROUPS;
   if (group_list_type < 0 || group_list_type > 2) return MACAQ_ERR_GROUP_LIST_TYPE;
   const bool listed = list.wq != nullptr || list.ws != nullptr;
+  void* yout = ep.y8 != nullptr ? static_cast<void*>(ep.y8) : static_cast<void*>(y);
+  const size_t ybytes = static_cast<size_t>(M) * N * (ep.y8 != nullptr ? 1 : 2);
   int st;
   if (!listed) {
-    st = check_mm_args(x, D, Wq, Ws, y, M, N, K, E, plain);
+    st = check_mm_args(x, D, Wq, Ws, yout, M, N, K, E, plain, 0, ybytes);
   } else {  // the tables are checked here, the addresses in them on the device (group_tables_kernel)
-    st = check_mm_args(x, D, reinterpret_cast<const uint8_t*>(list.wq), reinterpret_cast<const uint8_t*>(list.ws), y,
-                       M, N, K, E, plain, /*weight_bytes=*/static_cast<size_t>(E) * 8);
+    st = check_mm_args(x, D, reinterpret_cast<const uint8_t*>(list.wq), reinterpret_cast<const uint8_t*>(list.ws),
+                       yout, M, N, K, E, plain, /*weight_bytes=*/static_cast<size_t>(E) * 8, ybytes);
   }
-  if (st == MACAQ_OK) st = check_epilogue(ep, E, N, y, static_cast<size_t>(M) * N * 2);
+  if (st == MACAQ_OK) st = check_epilogue(ep, E, N, yout, ybytes);
   if (st != MACAQ_OK) return st;
   if (M == 0) return MACAQ_OK;
   if (!group_list) return MACAQ_ERR_NULL;
   if (!aligned16(group_list)) return MACAQ_ERR_ALIGN;
   const size_t gl_bytes = static_cast<size_t>(E) * (group_list_type == 2 ? 16 : 8);
-  if (overlaps(y, static_cast<size_t>(M) * N * 2, group_list, gl_bytes)) return MACAQ_ERR_ALIAS;
+  if (overlaps(yout, ybytes, group_list, gl_bytes)) return MACAQ_ERR_ALIAS;
   const GroupedWs w = grouped_ws(M, K, E);
-  st = check_ws(workspace, workspace_bytes, w.total, y, static_cast<size_t>(M) * N * 2, x,
-                static_cast<size_t>(M) * K * 2);
+  st = check_ws(workspace, workspace_bytes, w.total, yout, ybytes, x, static_cast<size_t>(M) * K * 2);
   if (st != MACAQ_OK) return st;
   int dev, sms;
   st = current_device(dev, sms);
@@ -2138,8 +2160,8 @@ static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, co
     wl.ws = list.ws;
     wl.wq_bytes = macaq_weight_code_bytes(1, N, K);
     wl.ws_bytes = macaq_weight_scale_bytes(1, N, K);
-    wl.y_lo = reinterpret_cast<uint64_t>(y);
-    wl.y_hi = wl.y_lo + static_cast<uint64_t>(M) * N * 2;
+    wl.y_lo = reinterpret_cast<uint64_t>(yout);
+    wl.y_hi = wl.y_lo + ybytes;
   }
   group_tables_kernel<<<1, static_cast<unsigned>((E + 31) / 32 * 32), 0, s>>>(
       group_list, group_list_type, static_cast<int>(E), static_cast<int>(M), goff, gtp, gexp, slabs, valid + 1, valid,
@@ -2150,7 +2172,7 @@ static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, co
   qp.x = x; qp.D = D; qp.Aq = ws + w.act;
   qp.M = static_cast<int>(M); qp.K = static_cast<int>(K);
   qp.slabs = slabs; qp.nslabs = valid + 1; qp.valid = valid; qp.plain = plain ? 1 : 0;
-  if (launch_ex(quant_tiles_kernel, dim3(quant_grid((M + 31) / 32 + E, KT, sms)), dim3(256), kQuantSmem, s, true,
+  if (launch_ex(quant_tiles_kernel, dim3(quant_grid((M + 31) / 32 + E, KT, sms)), dim3(256), 0, s, true,
                 1, qp) != cudaSuccess)
     return MACAQ_ERR_CUDA;
   GemmParams gp{};
@@ -2165,6 +2187,8 @@ static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, co
   gp.status = status;
   gp.wq_list = list.wq;
   gp.ws_list = list.ws;
+  gp.y8 = ep.y8;
+  gp.y8_scale = ep.y8_scale;
   const cudaError_t e = launch_ex(gemm_for(gp.bias, gp.act),
                                   dim3(sms), dim3(gemm::kThreads),
                                   gemm::smem_bytes(static_cast<int>(E), listed), s, true, 1, gp);
@@ -2194,6 +2218,42 @@ int macaq_grouped_mm_ex(const uint16_t* x, const float* D, const uint8_t* Wq, co
   ep.act = act_type;
   return grouped_impl(x, D, Wq, Ws, group_list, group_list_type, E, y, M, N, K, workspace, workspace_bytes, status,
                       stream, false, ep);
+}
+
+int macaq_dense_mm_fp8(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws, const float* bias,
+                       int act_type, float y_scale, uint8_t* y8, int64_t M, int64_t N, int64_t K, void* workspace,
+                       size_t workspace_bytes, int32_t* status, void* stream) {
+  Epilogue ep;
+  ep.bias = bias;
+  ep.act = act_type;
+  ep.y8 = y8;
+  ep.y8_scale = y_scale;
+  const size_t ybytes = static_cast<size_t>(M) * N;
+  int st = check_mm_args(x, D, Wq, Ws, y8, M, N, K, 1, false, 0, ybytes);
+  if (st == MACAQ_OK) st = check_epilogue(ep, 1, N, y8, ybytes);
+  if (st == MACAQ_OK && !(std::isfinite(y_scale) && y_scale > 0.0f)) st = MACAQ_ERR_SHAPE;
+  if (st != MACAQ_OK || M == 0) return st;
+  st = check_ws(workspace, workspace_bytes, dense_ws(M, K).total, y8, ybytes, x, static_cast<size_t>(M) * K * 2);
+  if (st != MACAQ_OK) return st;
+  int dev, sms;
+  st = current_device(dev, sms);
+  if (st != MACAQ_OK) return st;
+  return run_dense_two_kernel(x, D, Wq, Ws, nullptr, M, N, K, static_cast<uint8_t*>(workspace), status,
+                              static_cast<cudaStream_t>(stream), sms, true, false, ep);
+}
+
+int macaq_grouped_mm_fp8(const uint16_t* x, const float* D, const uint8_t* Wq, const uint8_t* Ws,
+                         const int64_t* group_list, int group_list_type, int64_t E, const float* bias, int act_type,
+                         float y_scale, uint8_t* y8, int64_t M, int64_t N, int64_t K, void* workspace,
+                         size_t workspace_bytes, int32_t* status, void* stream) {
+  if (!(std::isfinite(y_scale) && y_scale > 0.0f)) return MACAQ_ERR_SHAPE;
+  Epilogue ep;
+  ep.bias = bias;
+  ep.act = act_type;
+  ep.y8 = y8;
+  ep.y8_scale = y_scale;
+  return grouped_impl(x, D, Wq, Ws, group_list, group_list_type, E, nullptr, M, N, K, workspace, workspace_bytes,
+                      status, stream, false, ep);
 }
 
 int macaq_grouped_mm_list(const uint16_t* x, const float* D, const uint64_t* Wq_list, const uint64_t* Ws_list,

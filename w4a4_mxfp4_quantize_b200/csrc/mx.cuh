@@ -162,22 +162,30 @@ __device__ __forceinline__ uint32_t e2m1x8_f2(uint64_t a, uint64_t b, uint64_t c
   return e2m1x8(a0, a1, b0, b1, c0, c1, d0, d1);
 }
 
+// The 32 reciprocals of one block (16-byte aligned, e.g. in shared memory) as
+// 16 lane pairs: pair j holds channels 2j and 2j + 1.
+__device__ __forceinline__ void load_rcp_block(const float* __restrict__ r, uint64_t (&r2)[16]) {
+  const uint4* r4 = reinterpret_cast<const uint4*>(r);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const uint4 rq = r4[i];  // four reciprocals per 16-byte load
+    r2[2 * i] = f2(__uint_as_float(rq.x), __uint_as_float(rq.y));
+    r2[2 * i + 1] = f2(__uint_as_float(rq.z), __uint_as_float(rq.w));
+  }
+}
+
 // Activation block: 32 bf16 values (four 16-byte words) and the 32
-// reciprocals r = RN32(1/D) of their channels (r must be 16-byte aligned).
+// reciprocals r = RN32(1/D) of their channels as lane pairs (load_rcp_block).
 // Same arithmetic as the scalar definition, two lanes per instruction:
 //   xs = RNE_bf16(RN32(x * r)); FP32 butterfly h = 1, 2, 4, 8, 16;
 //   u = RNE_bf16(.); E8M0 from the block amax of |u|; E2M1 of u * 2^(127-c).
-__device__ __forceinline__ void act_block(const uint4 (&xv)[4], const float* __restrict__ r, uint4& codes,
+__device__ __forceinline__ void act_block(const uint4 (&xv)[4], const uint64_t (&r2)[16], uint4& codes,
                                           uint32_t& scale) {
   const uint32_t* w = reinterpret_cast<const uint32_t*>(xv);
-  const uint4* r4 = reinterpret_cast<const uint4*>(r);
   uint64_t P[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    const uint4 rq = r4[j >> 1];  // four reciprocals per 16-byte load
-    const uint64_t r2 = (j & 1) ? f2(__uint_as_float(rq.z), __uint_as_float(rq.w))
-                                : f2(__uint_as_float(rq.x), __uint_as_float(rq.y));
-    const uint32_t xs = f2_to_bf16x2(f2_mul(bf16x2_to_f2(w[j]), r2));  // channel scaling, BF16
+    const uint32_t xs = f2_to_bf16x2(f2_mul(bf16x2_to_f2(w[j]), r2[j]));  // channel scaling, BF16
     // butterfly stage h = 1 inside the pair: (v0 + v1, v0 - v1)
     const float v0 = bf16lo(xs), v1 = bf16hi(xs);
     P[j] = f2(__fadd_rn(v0, v1), __fsub_rn(v0, v1));
