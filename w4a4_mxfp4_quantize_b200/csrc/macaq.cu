@@ -566,28 +566,34 @@ struct QuantParams {
 
 // Quantise-once prologue over all rows.  A CTA owns one K tile and a contiguous
 // run of 32-row slabs (dense: rows 32 s..; grouped: the slab table, in group
-// order); a thread owns row tr of the slab and the 32-channel block c of the K
-// tile, i.e. one MX block per slab.  The activations go straight from global
-// memory into registers, one slab ahead of the one being encoded; the block's
-// 32 reciprocals stay in registers while consecutive slabs use the same row of
-// D (dense: always; grouped: until the group changes, a CTA-uniform event).  No
-// shared-memory staging and no barrier per slab.
+// order, copied into shared memory up front so that no global read sits on the
+// path to the next copy); a thread owns row tr of the slab and the 32-channel
+// block c of the K tile, i.e. one MX block per slab.  Each thread streams its
+// rows kQuantDepth - 1 slabs ahead through a ring in shared memory (cp.async,
+// chunk-major: a warp's 16-byte loads of chunk j are 512 consecutive bytes) and
+// reads back only what it copied itself, so the ring needs no barrier.  The
+// block's 32 reciprocals stay in registers while consecutive slabs use the same
+// row of D (dense: always; grouped: until the group changes, a CTA-uniform
+// event); the D values of a grouped slab travel in the ring with its
+// activations, so a change of group costs no global round trip.
 constexpr int kQuantCtasPerSm = 2;
-__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
-  uint4 v;
-  asm volatile("ld.global.cs.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
-  return v;
-}
+constexpr int kQuantDepth = 4;             // ring slots: the slab being encoded and three ahead
+constexpr int kQuantSlotBytes = 256 * 64;  // one slab: 256 threads x one 32-element block
+constexpr int kQuantDOff = kQuantDepth * kQuantSlotBytes;          // then [kQuantDepth][256] D values
+constexpr int kQuantSmem = kQuantDOff + kQuantDepth * 256 * 4;
+constexpr int kQuantTab = 256;             // slab-table entries a CTA keeps in shared memory
 
 __global__ void __launch_bounds__(256, kQuantCtasPerSm) quant_tiles_kernel(const __grid_constant__ QuantParams p) {
+  extern __shared__ __align__(16) uint8_t qsmem[];  // ring [kQuantDepth][4 chunks][256 threads][16], then D
+  float* dring = reinterpret_cast<float*>(qsmem + kQuantDOff);
   __shared__ __align__(16) float rs[kQRcpTile];
+  __shared__ int4 tab[kQuantTab];
   pdl_trigger();  // the GEMM may start streaming weights; it waits for our results before reading them
   pdl_wait();     // x (and the grouped tables) may come from the preceding kernels
   const int KT = p.K / kKTile;
+  const bool grouped = p.slabs != nullptr;
   int L = (p.M + 31) / 32;
-  if (p.slabs != nullptr) {
+  if (grouped) {
     if (*p.valid == 0) return;
     L = *p.nslabs;
   }
@@ -595,43 +601,57 @@ __global__ void __launch_bounds__(256, kQuantCtasPerSm) quant_tiles_kernel(const
   const int per_kt = static_cast<int>(gridDim.x) / KT;
   const int kt = static_cast<int>(blockIdx.x) % KT, j = static_cast<int>(blockIdx.x) / KT;
   const int q = (L + per_kt - 1) / per_kt;
-  int s = j * q;
-  const int s_end = min(L, s + q);
-  if (L <= 0 || j >= per_kt || s >= s_end) return;
-  const int tr = threadIdx.x >> 3, c = threadIdx.x & 7;
-  const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
-  // (group, first row, rows, quarter = 32-row slot in the tile images)
-  auto slab = [&](int sl) -> int4 {
-    if (p.slabs != nullptr) return p.slabs[sl];
+  const int s0 = j * q;
+  const int n = min(L, s0 + q) - s0;  // slabs of this CTA
+  if (L <= 0 || j >= per_kt || n <= 0) return;
+  if (grouped) {
+    for (int i = threadIdx.x; i < min(n, kQuantTab); i += blockDim.x) tab[i] = p.slabs[s0 + i];
+    __syncthreads();
+  }
+  // slab i of the run: (group, first row, rows, quarter = 32-row slot in the tile images)
+  auto slab = [&](int i) -> int4 {
+    if (grouped) return i < kQuantTab ? tab[i] : p.slabs[s0 + i];
+    const int sl = s0 + i;
     return make_int4(0, sl * 32, min(32, p.M - sl * 32), sl);
   };
-  auto load = [&](const int4& e, uint4 (&v)[4]) {
-    if (tr < e.z) {
-      const uint4* src = reinterpret_cast<const uint4*>(p.x + (static_cast<int64_t>(e.y) + tr) * p.K + k0 + c * kBlk);
+  const int tr = threadIdx.x >> 3, c = threadIdx.x & 7;
+  const int64_t k0 = static_cast<int64_t>(kt) * kKTile;
+  // copies this thread's 64 bytes of slab i (grouped: and the D value of channel
+  // k0 + threadIdx.x of its group) into ring slot `slot`; one group per slab
+  auto fetch = [&](int i, int slot) {
+    if (i < n) {
+      const int4 e = slab(i);
+      if (grouped && !p.plain)
+        cp_async4(dring + slot * 256 + threadIdx.x, p.D + static_cast<int64_t>(e.x) * p.K + k0 + threadIdx.x);
+      if (tr < e.z) {
+        const uint16_t* src = p.x + (static_cast<int64_t>(e.y) + tr) * p.K + k0 + c * kBlk;
+        uint8_t* dst = qsmem + slot * kQuantSlotBytes + threadIdx.x * 16;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) v[i] = ld_stream(src + i);
+        for (int ii = 0; ii < 4; ++ii) cp_async16(dst + 4096 * ii, src + 8 * ii);
+      }
     }
+    cp_async_commit();
   };
-  int4 e = slab(s);
-  uint4 xv[4], xn[4];
-  load(e, xv);
+#pragma unroll
+  for (int i = 0; i < kQuantDepth - 1; ++i) fetch(i, i);
   uint64_t r2[16];
   int group = -1;  // the D row whose reciprocals r2 holds
-  for (;;) {
-    const bool more = s + 1 < s_end;
-    int4 en = e;
-    if (more) {
-      en = slab(s + 1);
-      load(en, xn);
-    }
+  int slot = 0;    // ring slot of slab i
+  for (int i = 0; i < n; ++i) {
+    fetch(i + kQuantDepth - 1, slot == 0 ? kQuantDepth - 1 : slot - 1);  // the slot slab i - 1 freed
+    const int4 e = slab(i);
+    cp_async_wait<kQuantDepth - 1>();  // this thread's copies of slab i have landed
     if (!p.plain && e.x != group) {
       __syncthreads();  // every thread holds the previous reciprocals in registers already
-      rs[qrcp_index(threadIdx.x)] = __frcp_rn(__ldg(p.D + static_cast<int64_t>(e.x) * p.K + k0 + threadIdx.x));
+      const float d = grouped ? dring[slot * 256 + threadIdx.x] : __ldg(p.D + k0 + threadIdx.x);
+      rs[qrcp_index(threadIdx.x)] = __frcp_rn(d);
       __syncthreads();
       load_rcp_block(rs + c * kQRcpStride, r2);
       group = e.x;
     }
     if (tr < e.z) {
+      const uint4* xs = reinterpret_cast<const uint4*>(qsmem + slot * kQuantSlotBytes) + threadIdx.x;
+      const uint4 xv[4] = {xs[0], xs[256], xs[512], xs[768]};
       uint4 cv;
       uint32_t sc;
       if (p.plain) act_block_plain(xv, cv, sc);
@@ -641,12 +661,9 @@ __global__ void __launch_bounds__(256, kQuantCtasPerSm) quant_tiles_kernel(const
       *reinterpret_cast<uint4*>(img + code_chunk_offset(t, c)) = cv;
       img[kTileCodeBytes + sf_offset(t, c)] = static_cast<uint8_t>(sc);
     }
-    if (!more) break;
-    ++s;
-    e = en;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) xv[i] = xn[i];
+    if (++slot == kQuantDepth) slot = 0;
   }
+  cp_async_wait<0>();  // no copy may still be writing this CTA's shared memory at exit
 }
 
 // ============================================================================
@@ -1175,13 +1192,13 @@ struct Cfg {
   static constexpr int kGroups = BT <= 16 ? 2 : 1;
   static constexpr int kGroupThreads = kProWarps * 32 / kGroups;
   static constexpr int kRbufOff = kBarOff + 256;  // per group, two K tiles of reciprocals
-  static constexpr int kSmemBytes = 1024 + kRbufOff + kGroups * 2 * kRcpTile * 4;
+  static constexpr int kSmemBytes = 1024 + kRbufOff + kGroups * 2 * kQRcpTile * 4;
   // scale factors from kSfCol, 16 columns per stage
   static constexpr int kSfCol = BT < 32 ? 32 : BT;
   static constexpr int kTmemCols = kSfCol + 16 * kStages <= 64 ? 64 : kSfCol + 16 * kStages <= 128 ? 128 : 256;
-  // half-blocks (16 elements, one lane of a pair) per prologue thread and per K tile
-  static constexpr int kTasks = BT * 16 / kGroupThreads;
-  static_assert(BT * 16 % kGroupThreads == 0, "whole pairs of lanes per thread");
+  // 32-element blocks per prologue thread and per K tile
+  static constexpr int kTasks = BT * 8 / kGroupThreads;
+  static_assert(BT * 8 % kGroupThreads == 0, "whole blocks per thread");
   // reciprocals 1/D of a K tile per prologue thread
   static constexpr int kRcp = kKTile / kGroupThreads;
   static_assert(kKTile % kGroupThreads == 0, "whole reciprocals per thread");
@@ -1283,28 +1300,28 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
     __syncwarp();  // lane 0 initialised the barriers
     first_copies(0, 1);
   }
-  // Activation prologue set-up.  Each 32-element block is computed by a pair of
-  // adjacent lanes (16 elements each), so every prologue warp is busy even for the
-  // smallest token tile.  Rows past the tile's end are computed on zeros, which
-  // encode to zero codes and a zero scale (the lane pairs must stay converged).
-  // Group g of the prologue warps takes the CTA's K tiles g, g + kGroups, ...; the
-  // activation loads of its first kAhead K tiles are issued as soon as x may be
-  // read, so they land while the rest of the CTA sets up.
+  // Activation prologue set-up.  Each thread computes whole 32-element blocks (the
+  // rotation and the block maximum stay in its registers: no exchange between
+  // lanes); a K tile of the smallest token tile is one block per thread of its
+  // group.  Rows past the tile's end are computed on zeros, which encode to zero
+  // codes and a zero scale.  Group g of the prologue warps takes the CTA's K tiles
+  // g, g + kGroups, ...; the activation loads of its first kAhead K tiles are
+  // issued as soon as x may be read, so they land while the rest of the CTA sets up.
   constexpr int kGT = C::kGroupThreads, kG = C::kGroups;
-  constexpr int kAhead = C::kTasks <= 2 ? 2 : 1;
+  constexpr int kAhead = C::kTasks <= 1 ? 2 : 1;
   const int pt = static_cast<int>(threadIdx.x) - 6 * 32;
   const int grp = pt / kGT, gt = pt % kGT;
-  auto load = [&](int kt, uint4 (&xv)[C::kTasks][2], float (&d)[C::kRcp]) {
+  auto load = [&](int kt, uint4 (&xv)[C::kTasks][4], float (&d)[C::kRcp]) {
 #pragma unroll
     for (int u = 0; u < C::kTasks; ++u) {
-      const int task = gt + u * kGT, t = task >> 4, c = (task >> 1) & 7, half = task & 1;
-      xv[u][0] = make_uint4(0, 0, 0, 0);
-      xv[u][1] = make_uint4(0, 0, 0, 0);
+      const int task = gt + u * kGT, t = task >> 3, c = task & 7;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) xv[u][i] = make_uint4(0, 0, 0, 0);
       if (t < rows) {
-        const uint4* src = reinterpret_cast<const uint4*>(
-            p.x + static_cast<int64_t>(m0 + t) * p.K + static_cast<int64_t>(kt) * kKTile + c * kBlk + half * 16);
-        xv[u][0] = __ldg(src);
-        xv[u][1] = __ldg(src + 1);
+        const uint4* src = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(m0 + t) * p.K +
+                                                          static_cast<int64_t>(kt) * kKTile + c * kBlk);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xv[u][i] = __ldg(src + i);
       }
     }
 #pragma unroll
@@ -1312,7 +1329,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   };
   const int gst = nst > grp ? (nst - grp + kG - 1) / kG : 0;  // this group's K tiles
   auto kt_of = [&](int jj) { return kt0 + grp + kG * jj; };
-  uint4 xpre[kAhead][C::kTasks][2];
+  uint4 xpre[kAhead][C::kTasks][4];
   float dpre[kAhead][C::kRcp];
   if (warp >= 6) {
     pdl_wait();  // x and D may come from the previous kernel on the stream
@@ -1480,38 +1497,31 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
   } else {
     // ---- activation prologue: x/D, FWHT32, BF16, E8M0, E2M1 -> swizzled B tile ----
     // the group's jj-th K tile: CTA-local index j = grp + kG * jj
-    auto stage_body = [&](int jj, uint4 (&xv)[C::kTasks][2], const float (&d)[C::kRcp]) -> bool {
+    auto stage_body = [&](int jj, uint4 (&xv)[C::kTasks][4], const float (&d)[C::kRcp]) -> bool {
       const int j = grp + kG * jj, stage = j % kStages;
       const int slot = grp * 2 + (jj & 1);
-      float* r = rbuf + slot * kRcpTile;
+      float* r = rbuf + slot * kQRcpTile;
 #pragma unroll
-      for (int e = 0; e < C::kRcp; ++e) r[rcp_index(gt + e * kGT)] = __frcp_rn(d[e]);
+      for (int e = 0; e < C::kRcp; ++e) r[qrcp_index(gt + e * kGT)] = __frcp_rn(d[e]);
       if (gt == 0) pro_flag[slot] = mbar_wait(&empty[stage], ((j / kStages) & 1) ^ 1, abort_flag, kWaitTimeoutNs) ? 1 : 0;
       named_bar_sync(2 + grp, kGT);
       if (!pro_flag[slot]) return false;
       uint8_t* bcode = smem + stage * C::kStageBytes + C::kOffB;
       uint8_t* bsf = smem + stage * C::kStageBytes + C::kOffSfb;
-      // two tasks at a time, interleaved (two dependency chains per thread), where
-      // the registers allow
-      constexpr int kIlp = C::kTasks == 2 ? 2 : 1;
 #pragma unroll
-      for (int u0 = 0; u0 < C::kTasks; u0 += kIlp) {
-        const float* rr[kIlp];
-        uint2 cv[kIlp];
-        uint32_t sc[kIlp];
-#pragma unroll
-        for (int v = 0; v < kIlp; ++v) {
-          const int task = gt + (u0 + v) * kGT, c = (task >> 1) & 7, half = task & 1;
-          rr[v] = r + c * kRcpStride + half * 16;
+      for (int u = 0; u < C::kTasks; ++u) {
+        const int task = gt + u * kGT, t = task >> 3, c = task & 7;
+        uint4 cv;
+        uint32_t sc;
+        if (p.plain) {
+          act_block_plain(xv[u], cv, sc);
+        } else {
+          uint64_t r2[16];
+          load_rcp_block(r + c * kQRcpStride, r2);
+          act_block(xv[u], r2, cv, sc);
         }
-        if (p.plain) act_half_blocks_plain<kIlp>(*reinterpret_cast<const uint4(*)[kIlp][2]>(&xv[u0]), cv, sc);
-        else act_half_blocks<kIlp>(*reinterpret_cast<const uint4(*)[kIlp][2]>(&xv[u0]), rr, cv, sc);
-#pragma unroll
-        for (int v = 0; v < kIlp; ++v) {
-          const int task = gt + (u0 + v) * kGT, t = task >> 4, c = (task >> 1) & 7, half = task & 1;
-          *reinterpret_cast<uint2*>(bcode + code_chunk_offset(t, c) + half * 8) = cv[v];
-          if (half == 0) bsf[sf_offset(t, c)] = static_cast<uint8_t>(sc[v]);
-        }
+        *reinterpret_cast<uint4*>(bcode + code_chunk_offset(t, c)) = cv;
+        bsf[sf_offset(t, c)] = static_cast<uint8_t>(sc);
       }
       fence_proxy_async_smem();
       __syncwarp();
@@ -1524,10 +1534,10 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
         if (jj >= gst) break;
         if (!stage_body(jj, xpre[jj], dpre[jj])) break;
       }
-    } else if constexpr (C::kTasks >= 8) {
+    } else if constexpr (C::kTasks >= 4) {
       // the largest token tile: registers hold one K tile of loads
       if (stage_body(0, xpre[0], dpre[0])) {
-        uint4 xa[C::kTasks][2];
+        uint4 xa[C::kTasks][4];
         float da[C::kRcp];
         for (int jj = 1; jj < gst; ++jj) {
           load(kt_of(jj), xa, da);
@@ -1536,15 +1546,19 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
       }
     } else {
       // deeper K ranges: one K tile of loads ahead
-      uint4 xa[C::kTasks][2], xb[C::kTasks][2];
+      uint4 xa[C::kTasks][4], xb[C::kTasks][4];
       float da[C::kRcp], db[C::kRcp];
 #pragma unroll
-      for (int u = 0; u < C::kTasks; ++u) xa[u][0] = xpre[0][u][0], xa[u][1] = xpre[0][u][1];
+      for (int u = 0; u < C::kTasks; ++u)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) xa[u][i] = xpre[0][u][i];
 #pragma unroll
       for (int e = 0; e < C::kRcp; ++e) da[e] = dpre[0][e];
       if constexpr (kAhead >= 2) {
 #pragma unroll
-        for (int u = 0; u < C::kTasks; ++u) xb[u][0] = xpre[1][u][0], xb[u][1] = xpre[1][u][1];
+        for (int u = 0; u < C::kTasks; ++u)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) xb[u][i] = xpre[1][u][i];
 #pragma unroll
         for (int e = 0; e < C::kRcp; ++e) db[e] = dpre[1][e];
       }
@@ -1672,6 +1686,8 @@ int current_device(int& dev, int& sms) {
               cudaFuncSetAttribute(gemm_kernel<4>, a, gs) == cudaSuccess &&
               cudaFuncSetAttribute(gemm_kernel<5>, a, gs) == cudaSuccess;
     ok = ok && fused_attrs<16>() && fused_attrs<32>() && fused_attrs<64>() && fused_attrs<128>();
+    ok = ok && cudaFuncSetAttribute(quant_tiles_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kQuantSmem) ==
+                   cudaSuccess;
     if (!ok) return MACAQ_ERR_CUDA;
     s.attrs_set = true;
   }
@@ -1931,7 +1947,7 @@ int run_dense_two_kernel(const uint16_t* x, const float* D, const uint8_t* Wq, c
   QuantParams qp{};
   qp.x = x; qp.D = D; qp.Aq = ws + w.act;
   qp.M = static_cast<int>(M); qp.K = static_cast<int>(K); qp.plain = plain ? 1 : 0;
-  if (launch_ex(quant_tiles_kernel, dim3(quant_grid((M + 31) / 32, KT, sms)), dim3(256), 0, st, pdl, 1,
+  if (launch_ex(quant_tiles_kernel, dim3(quant_grid((M + 31) / 32, KT, sms)), dim3(256), kQuantSmem, st, pdl, 1,
                 qp) !=
       cudaSuccess)
     return MACAQ_ERR_CUDA;
@@ -2172,7 +2188,7 @@ static int grouped_impl(const uint16_t* x, const float* D, const uint8_t* Wq, co
   qp.x = x; qp.D = D; qp.Aq = ws + w.act;
   qp.M = static_cast<int>(M); qp.K = static_cast<int>(K);
   qp.slabs = slabs; qp.nslabs = valid + 1; qp.valid = valid; qp.plain = plain ? 1 : 0;
-  if (launch_ex(quant_tiles_kernel, dim3(quant_grid((M + 31) / 32 + E, KT, sms)), dim3(256), 0, s, true,
+  if (launch_ex(quant_tiles_kernel, dim3(quant_grid((M + 31) / 32 + E, KT, sms)), dim3(256), kQuantSmem, s, true,
                 1, qp) != cudaSuccess)
     return MACAQ_ERR_CUDA;
   GemmParams gp{};
