@@ -266,11 +266,11 @@ int macaq_grouped_mm_plain(const uint16_t *x_dev, const uint8_t *Wq_dev, const u
 /* ------------------------------------------------------------------ */
 
 /* The activation prologue alone, writing canonical codes [M, K/2] (element
- * 2j in the low nibble of byte j) and scales [M, K/32].  It runs the
- * one-block-per-thread form of the prologue, the form of the quantise-once
- * path (dense M > 128 and grouped calls); the fused small-M kernel computes the
- * same values with each block split over a lane pair, and its own codes and
- * scales are read out by macaq_fused_probe. */
+ * 2j in the low nibble of byte j) and scales [M, K/32], with the same
+ * per-block arithmetic (act_block) as the quantise-once path (dense M > 128
+ * and grouped calls) and the fused small-M kernel; the fused kernel's own
+ * codes and scales, as its tensor core reads them, are read out by
+ * macaq_fused_probe. */
 int macaq_quantize_activations(const uint16_t *x_dev, const float *D_dev, uint8_t *codes_dev,
                                uint8_t *scales_dev, int64_t M, int64_t K, void *stream);
 

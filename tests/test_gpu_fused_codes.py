@@ -1,8 +1,8 @@
 """The activation codes and scales of the fused small-M kernel itself, bit-exact.
 
 The fused kernel (dense M <= 128) quantises its activation tile straight into
-shared memory with each 32-element block split over a lane pair, so its codes
-never reach global memory on the product path.  macaq_fused_probe runs that
+shared memory, one 32-element block per prologue thread, so its codes never
+reach global memory on the product path.  macaq_fused_probe runs that
 kernel with a chosen plan (token tile, K split) and copies each activation
 operand tile out of shared memory just before the tensor core reads it.  These
 tests compare those tiles with the oracle's codes and E8M0 scales (MACAQ page,
@@ -88,7 +88,7 @@ def test_fused_kernel_codes_ragged_rows(M, K, N):
 
 
 def test_fused_kernel_codes_adversarial():
-    # the adversarial blocks of the quantiser test, in the fused kernel's lane-pair form
+    # the adversarial blocks of the quantiser test, through the fused kernel's prologue
     rng = np.random.default_rng(2)
     M, K, N = 100, 512, 128
     x = rng.standard_normal((M, K)).astype(np.float32)

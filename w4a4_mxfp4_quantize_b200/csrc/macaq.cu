@@ -237,7 +237,7 @@ __global__ void __launch_bounds__(256) quant_canonical_kernel(const uint16_t* __
   if (m >= M) return;
   uint4 cv;
   uint32_t sc;
-  uint64_t r2[16];
+  float2 r2[16];
   load_rcp_block(r + c * kQRcpStride, r2);
   act_block(xv, r2, cv, sc);
   *reinterpret_cast<uint4*>(codes + static_cast<int64_t>(m) * (K / 2) + (k0 + c * kBlk) / 2) = cv;
@@ -634,7 +634,7 @@ __global__ void __launch_bounds__(256, kQuantCtasPerSm) quant_tiles_kernel(const
   };
 #pragma unroll
   for (int i = 0; i < kQuantDepth - 1; ++i) fetch(i, i);
-  uint64_t r2[16];
+  float2 r2[16];
   int group = -1;  // the D row whose reciprocals r2 holds
   int slot = 0;    // ring slot of slab i
   for (int i = 0; i < n; ++i) {
@@ -1516,7 +1516,7 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
         if (p.plain) {
           act_block_plain(xv[u], cv, sc);
         } else {
-          uint64_t r2[16];
+          float2 r2[16];
           load_rcp_block(r + c * kQRcpStride, r2);
           act_block(xv[u], r2, cv, sc);
         }

@@ -8,11 +8,8 @@
 //   both:        E8M0 scale = floor(log2 amax) - 2 + 127 clamped at 0
 //                (OCP MX scale_alg = 0); E2M1 code = RNE with saturation of
 //                value * 2^(127 - scale); sign bit copied from the value.
-// The quantisers give each thread one whole 32-element block (act_block: the
-// rotation and the block amax stay in its registers); the fused kernel splits a
-// block across a lane pair (act_half_block(s): 16 elements per lane, the last
-// butterfly stage and the amax through one exchange each).  Both compute the
-// same values in the same order.
+// Every kernel gives each thread whole 32-element blocks (act_block: the
+// rotation and the block amax stay in its registers).
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -114,57 +111,33 @@ __device__ __forceinline__ void mx_encode_block(const float (&u)[32], uint4& cod
   scale = c;
 }
 
-// ---- packed two-lane FP32 arithmetic (sm_100 f32x2): each lane one IEEE rounding ----
-__device__ __forceinline__ uint64_t f2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
+// ---- packed two-lane FP32 arithmetic (sm_100 f32x2 through CUDA's float2
+// intrinsics): each lane one IEEE rounding to nearest, never contracted ----
+__device__ __forceinline__ float2 f2(float lo, float hi) { return make_float2(lo, hi); }
+__device__ __forceinline__ float2 f2_add(float2 a, float2 b) { return __fadd2_rn(a, b); }
+// a - b as a + (-b): the negation is exact, so the sum is the IEEE difference
+__device__ __forceinline__ float2 f2_sub(float2 a, float2 b) { return __fadd2_rn(a, make_float2(-b.x, -b.y)); }
+__device__ __forceinline__ float2 f2_mul(float2 a, float2 b) { return __fmul2_rn(a, b); }
 // Round both lanes to bf16 (nearest-even); low lane in the low half.
-__device__ __forceinline__ uint32_t f2_to_bf16x2(uint64_t v) {
-  float lo, hi;
-  f2_split(v, lo, hi);
+__device__ __forceinline__ uint32_t f2_to_bf16x2(float2 v) {
   uint32_t r;
-  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(v.y), "f"(v.x));
   return r;
 }
-__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t w) { return f2(bf16lo(w), bf16hi(w)); }
+__device__ __forceinline__ float2 bf16x2_to_f2(uint32_t w) { return make_float2(bf16lo(w), bf16hi(w)); }
 __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("max.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
 // Four lane pairs -> eight E2M1 codes in one word, element 0 in the lowest nibble.
-__device__ __forceinline__ uint32_t e2m1x8_f2(uint64_t a, uint64_t b, uint64_t c, uint64_t d) {
-  float a0, a1, b0, b1, c0, c1, d0, d1;
-  f2_split(a, a0, a1);
-  f2_split(b, b0, b1);
-  f2_split(c, c0, c1);
-  f2_split(d, d0, d1);
-  return e2m1x8(a0, a1, b0, b1, c0, c1, d0, d1);
+__device__ __forceinline__ uint32_t e2m1x8_f2(float2 a, float2 b, float2 c, float2 d) {
+  return e2m1x8(a.x, a.y, b.x, b.y, c.x, c.y, d.x, d.y);
 }
 
 // The 32 reciprocals of one block (16-byte aligned, e.g. in shared memory) as
 // 16 lane pairs: pair j holds channels 2j and 2j + 1.
-__device__ __forceinline__ void load_rcp_block(const float* __restrict__ r, uint64_t (&r2)[16]) {
+__device__ __forceinline__ void load_rcp_block(const float* __restrict__ r, float2 (&r2)[16]) {
   const uint4* r4 = reinterpret_cast<const uint4*>(r);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -179,10 +152,10 @@ __device__ __forceinline__ void load_rcp_block(const float* __restrict__ r, uint
 // Same arithmetic as the scalar definition, two lanes per instruction:
 //   xs = RNE_bf16(RN32(x * r)); FP32 butterfly h = 1, 2, 4, 8, 16;
 //   u = RNE_bf16(.); E8M0 from the block amax of |u|; E2M1 of u * 2^(127-c).
-__device__ __forceinline__ void act_block(const uint4 (&xv)[4], const uint64_t (&r2)[16], uint4& codes,
+__device__ __forceinline__ void act_block(const uint4 (&xv)[4], const float2 (&r2)[16], uint4& codes,
                                           uint32_t& scale) {
   const uint32_t* w = reinterpret_cast<const uint32_t*>(xv);
-  uint64_t P[16];
+  float2 P[16];
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
     const uint32_t xs = f2_to_bf16x2(f2_mul(bf16x2_to_f2(w[j]), r2[j]));  // channel scaling, BF16
@@ -196,7 +169,7 @@ __device__ __forceinline__ void act_block(const uint4 (&xv)[4], const uint64_t (
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       if (i & hp) continue;
-      const uint64_t a = P[i], b = P[i + hp];
+      const float2 a = P[i], b = P[i + hp];
       P[i] = f2_add(a, b);
       P[i + hp] = f2_sub(a, b);
     }
@@ -211,68 +184,13 @@ __device__ __forceinline__ void act_block(const uint4 (&xv)[4], const uint64_t (
   const uint32_t amax16 = max(m & 0xFFFFu, m >> 16);
   const uint32_t c = e8m0_from_amax_bits(amax16 << 16);
   const float s = __uint_as_float((254u - min(c, 253u)) << 23);
-  const uint64_t s2 = f2(s, s);
+  const float2 s2 = f2(s, s);
   uint32_t out[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q)
     out[q] = e2m1x8_f2(f2_mul(bf16x2_to_f2(u[4 * q]), s2), f2_mul(bf16x2_to_f2(u[4 * q + 1]), s2),
                        f2_mul(bf16x2_to_f2(u[4 * q + 2]), s2), f2_mul(bf16x2_to_f2(u[4 * q + 3]), s2));
   codes = make_uint4(out[0], out[1], out[2], out[3]);
-  scale = c;
-}
-
-// The same block computed by two adjacent lanes (lane parity = half): each lane
-// holds 16 of the 32 values (half 0: elements 0-15, half 1: 16-31), does the
-// butterfly stages h = 1..8 in registers and stage h = 16 with one exchange
-// of its partner's values.  Both lanes of a pair must call it together (the
-// whole warp converged).  Output: this lane's 8 code bytes (element 2j of its
-// half in the low nibble of byte j) and the block scale (same in both lanes).
-__device__ __forceinline__ void act_half_block(const uint4 (&xv)[2], const float* __restrict__ r, uint2& codes,
-                                               uint32_t& scale) {
-  const uint32_t half = threadIdx.x & 1u;
-  const uint32_t* w = reinterpret_cast<const uint32_t*>(xv);
-  const uint64_t* r2 = reinterpret_cast<const uint64_t*>(r);
-  uint64_t P[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t xs = f2_to_bf16x2(f2_mul(bf16x2_to_f2(w[j]), r2[j]));
-    const float v0 = bf16lo(xs), v1 = bf16hi(xs);
-    P[j] = f2(__fadd_rn(v0, v1), __fsub_rn(v0, v1));  // stage h = 1
-  }
-#pragma unroll
-  for (int hp = 1; hp < 8; hp <<= 1) {  // stages h = 2, 4, 8
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (i & hp) continue;
-      const uint64_t a = P[i], b = P[i + hp];
-      P[i] = f2_add(a, b);
-      P[i + hp] = f2_sub(a, b);
-    }
-  }
-  // stage h = 16 across the pair: half 0 keeps v[i] + v[i+16], half 1 keeps
-  // v[i] - v[i+16] = partner + (-mine); IEEE a - b == a + (-b) exactly.
-  const uint64_t neg = half ? 0x8000000080000000ull : 0ull;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint64_t q = __shfl_xor_sync(0xffffffffu, P[j], 1);
-    P[j] = f2_add(q, P[j] ^ neg);
-  }
-  uint32_t u[8];
-  uint32_t m = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    u[j] = f2_to_bf16x2(P[j]);
-    m = max_u16x2(m, u[j] & 0x7FFF7FFFu);
-  }
-  m = max_u16x2(m, __shfl_xor_sync(0xffffffffu, m, 1));
-  const uint32_t amax16 = max(m & 0xFFFFu, m >> 16);
-  const uint32_t c = e8m0_from_amax_bits(amax16 << 16);
-  const float s = __uint_as_float((254u - min(c, 253u)) << 23);
-  const uint64_t s2 = f2(s, s);
-  codes.x = e2m1x8_f2(f2_mul(bf16x2_to_f2(u[0]), s2), f2_mul(bf16x2_to_f2(u[1]), s2),
-                      f2_mul(bf16x2_to_f2(u[2]), s2), f2_mul(bf16x2_to_f2(u[3]), s2));
-  codes.y = e2m1x8_f2(f2_mul(bf16x2_to_f2(u[4]), s2), f2_mul(bf16x2_to_f2(u[5]), s2),
-                      f2_mul(bf16x2_to_f2(u[6]), s2), f2_mul(bf16x2_to_f2(u[7]), s2));
   scale = c;
 }
 
@@ -286,7 +204,7 @@ __device__ __forceinline__ void act_block_plain(const uint4 (&xv)[4], uint4& cod
   const uint32_t amax16 = max(m & 0xFFFFu, m >> 16);
   const uint32_t c = e8m0_from_amax_bits(amax16 << 16);
   const float s = __uint_as_float((254u - min(c, 253u)) << 23);
-  const uint64_t s2 = f2(s, s);
+  const float2 s2 = f2(s, s);
   uint32_t out[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q)
@@ -294,103 +212,6 @@ __device__ __forceinline__ void act_block_plain(const uint4 (&xv)[4], uint4& cod
                        f2_mul(bf16x2_to_f2(w[4 * q + 2]), s2), f2_mul(bf16x2_to_f2(w[4 * q + 3]), s2));
   codes = make_uint4(out[0], out[1], out[2], out[3]);
   scale = c;
-}
-
-// Plain MXFP4 of T half-blocks held by lane pairs (the partner holds the other
-// 16 values of each block; the block amax is combined across the pair).
-template <int T>
-__device__ __forceinline__ void act_half_blocks_plain(const uint4 (&xv)[T][2], uint2 (&codes)[T],
-                                                      uint32_t (&scale)[T]) {
-  uint32_t m[T];
-#pragma unroll
-  for (int t = 0; t < T; ++t) {
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(xv[t]);
-    m[t] = 0;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) m[t] = max_u16x2(m[t], w[j] & 0x7FFF7FFFu);
-  }
-#pragma unroll
-  for (int t = 0; t < T; ++t) m[t] = max_u16x2(m[t], __shfl_xor_sync(0xffffffffu, m[t], 1));
-#pragma unroll
-  for (int t = 0; t < T; ++t) {
-    const uint32_t* w = reinterpret_cast<const uint32_t*>(xv[t]);
-    const uint32_t amax16 = max(m[t] & 0xFFFFu, m[t] >> 16);
-    const uint32_t c = e8m0_from_amax_bits(amax16 << 16);
-    const float s = __uint_as_float((254u - min(c, 253u)) << 23);
-    const uint64_t s2 = f2(s, s);
-    codes[t].x = e2m1x8_f2(f2_mul(bf16x2_to_f2(w[0]), s2), f2_mul(bf16x2_to_f2(w[1]), s2),
-                           f2_mul(bf16x2_to_f2(w[2]), s2), f2_mul(bf16x2_to_f2(w[3]), s2));
-    codes[t].y = e2m1x8_f2(f2_mul(bf16x2_to_f2(w[4]), s2), f2_mul(bf16x2_to_f2(w[5]), s2),
-                           f2_mul(bf16x2_to_f2(w[6]), s2), f2_mul(bf16x2_to_f2(w[7]), s2));
-    scale[t] = c;
-  }
-}
-
-// T independent half-blocks, each step done for all T before the next step, so
-// that one thread keeps T dependency chains in flight.  Same arithmetic as
-// act_half_block; lane pairs as there.
-template <int T>
-__device__ __forceinline__ void act_half_blocks(const uint4 (&xv)[T][2], const float* const (&r)[T],
-                                                uint2 (&codes)[T], uint32_t (&scale)[T]) {
-  const uint64_t neg = (threadIdx.x & 1u) ? 0x8000000080000000ull : 0ull;
-  uint64_t P[T][8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-#pragma unroll
-    for (int t = 0; t < T; ++t) {
-      const uint32_t w = reinterpret_cast<const uint32_t*>(xv[t])[j];
-      const uint64_t r2 = reinterpret_cast<const uint64_t*>(r[t])[j];
-      const uint32_t xs = f2_to_bf16x2(f2_mul(bf16x2_to_f2(w), r2));
-      const float v0 = bf16lo(xs), v1 = bf16hi(xs);
-      P[t][j] = f2(__fadd_rn(v0, v1), __fsub_rn(v0, v1));  // stage h = 1
-    }
-  }
-#pragma unroll
-  for (int hp = 1; hp < 8; hp <<= 1) {  // stages h = 2, 4, 8
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (i & hp) continue;
-#pragma unroll
-      for (int t = 0; t < T; ++t) {
-        const uint64_t a = P[t][i], b = P[t][i + hp];
-        P[t][i] = f2_add(a, b);
-        P[t][i + hp] = f2_sub(a, b);
-      }
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {  // stage h = 16 across the pair
-#pragma unroll
-    for (int t = 0; t < T; ++t) {
-      const uint64_t q = __shfl_xor_sync(0xffffffffu, P[t][j], 1);
-      P[t][j] = f2_add(q, P[t][j] ^ neg);
-    }
-  }
-  uint32_t u[T][8], m[T];
-#pragma unroll
-  for (int t = 0; t < T; ++t) m[t] = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-#pragma unroll
-    for (int t = 0; t < T; ++t) {
-      u[t][j] = f2_to_bf16x2(P[t][j]);
-      m[t] = max_u16x2(m[t], u[t][j] & 0x7FFF7FFFu);
-    }
-  }
-#pragma unroll
-  for (int t = 0; t < T; ++t) m[t] = max_u16x2(m[t], __shfl_xor_sync(0xffffffffu, m[t], 1));
-#pragma unroll
-  for (int t = 0; t < T; ++t) {
-    const uint32_t amax16 = max(m[t] & 0xFFFFu, m[t] >> 16);
-    const uint32_t c = e8m0_from_amax_bits(amax16 << 16);
-    const float s = __uint_as_float((254u - min(c, 253u)) << 23);
-    const uint64_t s2 = f2(s, s);
-    codes[t].x = e2m1x8_f2(f2_mul(bf16x2_to_f2(u[t][0]), s2), f2_mul(bf16x2_to_f2(u[t][1]), s2),
-                           f2_mul(bf16x2_to_f2(u[t][2]), s2), f2_mul(bf16x2_to_f2(u[t][3]), s2));
-    codes[t].y = e2m1x8_f2(f2_mul(bf16x2_to_f2(u[t][4]), s2), f2_mul(bf16x2_to_f2(u[t][5]), s2),
-                           f2_mul(bf16x2_to_f2(u[t][6]), s2), f2_mul(bf16x2_to_f2(u[t][7]), s2));
-    scale[t] = c;
-  }
 }
 
 // Weight block: 32 fp32 weights and their 32 channel factors D (offline).

@@ -265,29 +265,8 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
 namespace macaq {
 // Packed FP32 pair arithmetic (sm_100 .f32x2 forms): one instruction for two
 // lanes, each lane rounded exactly as the scalar fma / mul.
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  float2 d;
-  asm("{.reg .b64 a, b, c, d;\n\t"
-      "mov.b64 a, {%2, %3};\n\t"
-      "mov.b64 b, {%4, %5};\n\t"
-      "mov.b64 c, {%6, %7};\n\t"
-      "fma.rn.f32x2 d, a, b, c;\n\t"
-      "mov.b64 {%0, %1}, d;}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-  return d;
-}
-__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
-  float2 d;
-  asm("{.reg .b64 a, b, d;\n\t"
-      "mov.b64 a, {%2, %3};\n\t"
-      "mov.b64 b, {%4, %5};\n\t"
-      "mul.rn.f32x2 d, a, b;\n\t"
-      "mov.b64 {%0, %1}, d;}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return d;
-}
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
 
 // Hardware tanh in half precision: the FP32 argument rounded to FP16 (RN), one
 // special-function-unit operation (tanh.approx.f16), the result widened exactly
