@@ -388,7 +388,8 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * statistics.median(el for _, el in steps), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "mxfp4(e2m1,e8m0)->exact->bf16", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "global_batch": 128, "l2": "n/a (CPU)"},
+        "config": {"workload": WORKLOAD, "global_batch": 128 * world, "per_gpu_batch": 128,
+                   "parallelism": f"replicas x{world}", "l2": "n/a (CPU)"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }

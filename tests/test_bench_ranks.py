@@ -65,3 +65,25 @@ def test_reference_arm_runs_on_rank_zero_only(capsys):
 
     bench.run_reference(Args, rank=1, world=2)        # returns at once, prints nothing
     assert capsys.readouterr().out == ""
+
+
+def test_reference_arm_reports_the_same_config_keys(capsys, monkeypatch):
+    # the driver compares the two arms' lines: the reference arm names the same
+    # workload with the same config keys as ours (the CPU oracle itself is stubbed out)
+    sys.path.insert(0, ROOT)
+    import json
+
+    import bench
+
+    monkeypatch.setattr(bench, "cpu_oracle_sample",
+                        lambda problems, budget_s=0.0, rows=1, prepared=None, nthreads=0: (1.0, 0.01, 4, "stub", None))
+
+    class Args:
+        gpus, steps, warmup = 2, 2, 1
+
+    bench.run_reference(Args, rank=0, world=2)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert set(line["config"]) == {"workload", "global_batch", "per_gpu_batch", "parallelism", "l2"}
+    assert line["config"]["workload"] == bench.WORKLOAD
+    assert line["config"]["global_batch"] == 256 and line["config"]["parallelism"] == "replicas x2"
