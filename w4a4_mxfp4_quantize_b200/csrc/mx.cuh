@@ -69,22 +69,16 @@ __device__ __forceinline__ uint32_t e2m1x8(float v0, float v1, float v2, float v
   return out;
 }
 
-// E8M0 code from the bit pattern of a non-negative float amax:
-// floor(log2 amax) + 127 is the biased exponent field e (0 for zero and
-// subnormals, which clamp to 0 anyway); minus emax(E2M1) = 2.
-// Reciprocals 1/D of one 256-wide K tile in shared memory: block c's 32 values
-// start at c * kRcpStride.  The padding puts the eight blocks on different banks
-// (threads of a warp read the same element of different blocks together).
-constexpr int kRcpStride = kBlk + 2;
-constexpr int kRcpTile = 8 * kRcpStride;  // floats per K tile
-__host__ __device__ constexpr int rcp_index(int k) { return (k >> 5) * kRcpStride + (k & 31); }
-// The quantisers' layout: blocks 36 floats apart, so each block starts on a 16-byte
-// boundary and a warp's 16-byte loads of the same element of the eight blocks
-// cover all 32 banks once.
+// Reciprocals 1/D of one 256-wide K tile in shared memory: blocks 36 floats
+// apart, so each block starts on a 16-byte boundary and a warp's 16-byte loads of
+// the same element of the eight blocks cover all 32 banks once.
 constexpr int kQRcpStride = kBlk + 4;
 constexpr int kQRcpTile = 8 * kQRcpStride;
 __host__ __device__ constexpr int qrcp_index(int k) { return (k >> 5) * kQRcpStride + (k & 31); }
 
+// E8M0 code from the bit pattern of a non-negative float amax:
+// floor(log2 amax) + 127 is the biased exponent field e (0 for zero and
+// subnormals, which clamp to 0 anyway); minus emax(E2M1) = 2.
 __device__ __forceinline__ uint32_t e8m0_from_amax_bits(uint32_t amax_bits) {
   const uint32_t e = amax_bits >> 23;  // sign is clear
   if (e == 0xFFu) return 0xFFu;        // non-finite input (precondition violated)
