@@ -215,6 +215,18 @@ class Prepared:
             mq.grouped_mm(self.x, self.D, self.Wq, self.Ws, self.gl, self.p.group_list_type, self.p.N,
                           out=self.y, stream=stream, ws=self.ws, bias=self.bias, act_type=mq.ACT_GELU_TANH)
 
+    def run_fp8(self, mq, stream=None):
+        """The same call with the FP8 (E4M3) output (per-tensor output scale 1)."""
+        if getattr(self, "y8", None) is None:
+            self.y8 = torch.empty((self.p.M, self.p.N), dtype=torch.uint8, device=self.y.device)
+            nu = mq.unfused_workspace_bytes(self.p.M, self.p.K) if self.gl is None else 0
+            self.ws8 = torch.zeros(nu, dtype=torch.uint8, device=self.y.device) if nu else self.ws
+        if self.gl is None:
+            mq.dense_mm_fp8(self.x, self.D, self.Wq, self.Ws, self.p.N, 1.0, out=self.y8, stream=stream, ws=self.ws8)
+        else:
+            mq.grouped_mm_fp8(self.x, self.D, self.Wq, self.Ws, self.gl, self.p.group_list_type, self.p.N, 1.0,
+                              out=self.y8, stream=stream, ws=self.ws8)
+
     def run_unfused(self, mq, stream=None):
         mq.unfused_dense_mm(self.x, self.D, self.Wq, self.Ws, self.p.N, out=self.y, stream=stream,
                             ws=self.ws_unfused)
@@ -657,9 +669,10 @@ def time_eager(fn, stream, calls: int = 20, trials: int = 15, warm: int = 20) ->
 def workload_table(mq, device, stream, flush, hbm_gbs, reps):
     """us/call (trimmed mean, cold L2), TFLOPS and roofline fraction for every
     problem of the five workloads, fused and unfused (CUDA graph per call), the
-    plain MXFP4 baseline's time, and both paths' error against the unquantised
-    layer on sampled rows; also eager calls that allocate y on every call, and
-    the ALU bound of the activation prologue."""
+    plain MXFP4 baseline's time, the calls with bias + GELU_TANH and with the FP8
+    output, and both paths' error against the unquantised layer on sampled rows;
+    also eager calls that allocate y on every call, and the ALU bound of the
+    activation prologue."""
     rows = []
     sms = torch.cuda.get_device_properties(device).multi_processor_count
     for cfg in range(5):
@@ -691,6 +704,12 @@ def workload_table(mq, device, stream, flush, hbm_gbs, reps):
             ge = capture(lambda: pp.run_epilogue(mq), stream)
             epi_us, _ = time_graph(ge, flush, stream, reps)
             del ge
+            try:  # supplementary: its failure must not cost the table
+                g8 = capture(lambda: pp.run_fp8(mq), stream)
+                fp8_us, _ = time_graph(g8, flush, stream, reps)
+                del g8
+            except Exception:  # noqa: BLE001
+                fp8_us = None
             # accuracy against the unquantised layer on sampled rows, then the plain MXFP4 baseline
             rows_s = np.unique(np.random.default_rng(cfg).integers(0, p.M, min(p.M, 16)))
             pp.run(mq, stream)
@@ -710,7 +729,8 @@ def workload_table(mq, device, stream, flush, hbm_gbs, reps):
                 "tflops": p.flops() / (us * 1e-6) / 1e12, "gbs": p.algorithmic_bytes() / (us * 1e-6) / 1e9,
                 "roofline_us": t_roof * 1e6, "frac_roofline": t_roof / (us * 1e-6), "unfused_us": un,
                 "plain_us": plain_us, "plain_over_macaq_time": plain_us / us,
-                "bias_gelu_tanh_us": epi_us, "eager_alloc_us": eager_alloc_us, "group_list_type2_us": type2_us,
+                "bias_gelu_tanh_us": epi_us, "fp8_out_us": fp8_us, "eager_alloc_us": eager_alloc_us,
+                "group_list_type2_us": type2_us,
                 **({"eager_alloc_error": eager_err} if eager_err else {}),
                 "alu_bound_us": alu_bound_us(p.M, p.K, sms),
                 "nmse": nmse, "nmse_plain": nmse_plain, "nmse_plain_over_macaq": nmse_plain / nmse if nmse else None,
