@@ -208,11 +208,12 @@ int macaq_grouped_mm_ex(const uint16_t *x_dev, const float *D_dev, const uint8_t
  * with v as in macaq_dense_mm_ex, the product with y_scale rounded to FP32 and
  * then to E4M3 by round-to-nearest-even with saturation at +-448 (E4M3 has no
  * infinity; a caller dequantises with y8 / y_scale).  y_scale must be finite
- * and > 0, else MACAQ_ERR_SHAPE.  The dense call runs the quantise-once path
- * for every M (one quantisation kernel, then the block-scaled GEMM) and needs
- * macaq_unfused_workspace_bytes(M, K) bytes of workspace; the grouped call
- * needs macaq_workspace_bytes(M, N, K, E).  Other arguments, refusals and
- * device errors as in macaq_dense_mm_ex / macaq_grouped_mm_ex. */
+ * and > 0, else MACAQ_ERR_SHAPE.  The dense call runs the kernels of
+ * macaq_dense_mm_ex (the fused kernel for M <= 128, the quantise-once pair
+ * above) and takes macaq_unfused_workspace_bytes(M, K) bytes of workspace at
+ * every M (used above M = 128); the grouped call needs
+ * macaq_workspace_bytes(M, N, K, E).  Other arguments, refusals and device
+ * errors as in macaq_dense_mm_ex / macaq_grouped_mm_ex. */
 int macaq_dense_mm_fp8(const uint16_t *x_dev, const float *D_dev, const uint8_t *Wq_dev, const uint8_t *Ws_dev,
                        const float *bias_dev, int act_type, float y_scale, uint8_t *y8_dev, int64_t M, int64_t N,
                        int64_t K, void *workspace_dev, size_t workspace_bytes, int32_t *status_dev, void *stream);

@@ -32,7 +32,8 @@ def _oracle_fp8(p, x_rows, D, W, bias, act, y_scale):
     return oracle.gemm_fp8(qa, sa, qw, sw, bias=bias, act_type=act, y_scale=y_scale)
 
 
-@pytest.mark.parametrize("M,K,N,act", [(16, 1024, 256, 0), (300, 512, 272, 2), (129, 768, 144, 5), (64, 256, 48, 1)])
+@pytest.mark.parametrize("M,K,N,act", [(16, 1024, 256, 0), (300, 512, 272, 2), (129, 768, 144, 5), (64, 256, 48, 1),
+                                        (32, 2048, 512, 2), (128, 1024, 384, 0)])
 def test_dense_fp8_output_against_the_oracle(M, K, N, act):
     p = synth.dense(M, K, N, seed=M + N)
     bias = (np.random.default_rng(M).standard_normal(N) * 0.3).astype(np.float32) if act else None
@@ -99,6 +100,25 @@ def test_fp8_refusals():
     with pytest.raises(mq.MacaqError) as e:
         mq.dense_mm_fp8(x_to_dev(p.x), f32_dev(p.D[0]), Wq, Ws, p.N, 1.0, act_type=3)
     assert e.value.status == -13
+
+
+@pytest.mark.parametrize("M,K,N", [(16, 1024, 256), (96, 2048, 384)])
+def test_fused_fp8_equals_the_e4m3_of_the_fused_bf16_values(M, K, N):
+    # M <= 128 runs the fused kernel for both outputs (the same plan and summation
+    # order): with y_scale = 1 the FP8 codes are the E4M3 rounding of the FP32 values
+    # whose BF16 rounding the BF16 call returns, so decoding both and comparing them
+    # within the larger of the two rounding steps must agree everywhere
+    p = synth.dense(M, K, N, seed=M + 5)
+    Wq, Ws = mq.prepare_weights(f32_dev(p.W), f32_dev(p.D))
+    x, D = x_to_dev(p.x), f32_dev(p.D[0])
+    y16 = mq.dense_mm(x, D, Wq, Ws, N).float().cpu().numpy().astype(np.float64).ravel()
+    y8 = mq.dense_mm_fp8(x, D, Wq, Ws, N, 1.0).cpu().numpy().ravel()
+    torch.cuda.synchronize()
+    dec = oracle.e4m3_decode(y8)
+    big = np.abs(y16) >= 464.0
+    assert np.all((y8[big] & 0x7F) == 0x7E)
+    step = np.exp2(np.floor(np.log2(np.maximum(np.abs(y16[~big]), 2.0 ** -6))) - 3)
+    assert np.all(np.abs(dec[~big] - y16[~big]) <= step)
 
 
 def test_bf16_path_unchanged_next_to_fp8():

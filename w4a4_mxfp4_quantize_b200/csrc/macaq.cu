@@ -719,6 +719,11 @@ __device__ __forceinline__ void finish32(const uint32_t (&r)[32], float os, cons
 // The same 32 columns as FP8 E4M3 codes (8 words, column 0 in the lowest byte):
 // each value times y8_scale in FP32, then rounded to nearest even with saturation
 // at +-448 (cvt.rn.satfinite; NaN stays NaN).
+__device__ __forceinline__ uint8_t e4m3_1(float v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(v));
+  return static_cast<uint8_t>(r & 0xFFu);
+}
 __device__ __forceinline__ uint32_t e4m3x4(float2 a, float2 b) {
   uint16_t lo, hi;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(lo) : "f"(a.x), "f"(a.y));
@@ -1167,6 +1172,8 @@ struct FusedParams {
   int act;                 // act_type (act_value)
   uint8_t* dump_codes;     // test instantiation only: canonical [M, K/2] codes of the operand tiles
   uint8_t* dump_scales;    // and [M, K/32] scales, copied out of shared memory before each MMA
+  uint8_t* y8;             // FP8 (E4M3) output instead of y (nullptr: BF16 into y)
+  float y8_scale;
 };
 
 namespace fused {
@@ -1457,7 +1464,9 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
             if (c0 + jj >= rows) break;
             float v = __uint_as_float(r0[jj]) * os;
             if constexpr (kEpilogue) v = act_value_rt(v + b, p.act);
-            p.y[static_cast<int64_t>(m0 + c0 + jj) * p.N + n] = bf16_bits(v);
+            const int64_t o = static_cast<int64_t>(m0 + c0 + jj) * p.N + n;
+            if (p.y8 != nullptr) p.y8[o] = e4m3_1(v * p.y8_scale);
+            else p.y[o] = bf16_bits(v);
           }
         }
       }
@@ -1608,12 +1617,21 @@ __global__ void __launch_bounds__(fused::kThreads, 1) fused_small_kernel(const _
           for (int i = 0; i < 8; ++i) s[i] = act_value_rt(s[i], p.act);
         }
       }
-      uint4 o;
-      o.x = pack_bf16x2(s[0], s[1]);
-      o.y = pack_bf16x2(s[2], s[3]);
-      o.z = pack_bf16x2(s[4], s[5]);
-      o.w = pack_bf16x2(s[6], s[7]);
-      *reinterpret_cast<uint4*>(p.y + static_cast<int64_t>(m0 + t) * p.N + n0 + n) = o;
+      const int64_t off = static_cast<int64_t>(m0 + t) * p.N + n0 + n;
+      if (p.y8 != nullptr) {
+        const float2 sc = make_float2(p.y8_scale, p.y8_scale);
+        uint2 o8;
+        o8.x = e4m3x4(fmul2(make_float2(s[0], s[1]), sc), fmul2(make_float2(s[2], s[3]), sc));
+        o8.y = e4m3x4(fmul2(make_float2(s[4], s[5]), sc), fmul2(make_float2(s[6], s[7]), sc));
+        *reinterpret_cast<uint2*>(p.y8 + off) = o8;
+      } else {
+        uint4 o;
+        o.x = pack_bf16x2(s[0], s[1]);
+        o.y = pack_bf16x2(s[2], s[3]);
+        o.z = pack_bf16x2(s[4], s[5]);
+        o.w = pack_bf16x2(s[6], s[7]);
+        *reinterpret_cast<uint4*>(p.y + off) = o;
+      }
     }
   }
   // no CTA may leave while a copy it sent can still be reading its shared memory:
@@ -2254,6 +2272,21 @@ int macaq_dense_mm_fp8(const uint16_t* x, const float* D, const uint8_t* Wq, con
   int dev, sms;
   st = current_device(dev, sms);
   if (st != MACAQ_OK) return st;
+  if (M <= kSmallM) {  // the fused kernel, as macaq_dense_mm_ex, storing E4M3 codes
+    FusedParams p{};
+    p.Wq = Wq; p.Ws = Ws; p.x = x; p.D = D; p.y = nullptr;
+    p.M = static_cast<int>(M); p.N = static_cast<int>(N); p.K = static_cast<int>(K);
+    p.NT = static_cast<int>(pad128(N) / 128); p.KT = static_cast<int>(K / 256);
+    const FusedPlan plan = plan_fused(dev, M, N, K);
+    p.S = plan.S;
+    p.status = status;
+    p.out_scale = 0.03125f;
+    p.bias = bias;
+    p.act = act_type;
+    p.y8 = y8;
+    p.y8_scale = y_scale;
+    return launch_fused(p, plan, static_cast<cudaStream_t>(stream));
+  }
   return run_dense_two_kernel(x, D, Wq, Ws, nullptr, M, N, K, static_cast<uint8_t*>(workspace), status,
                               static_cast<cudaStream_t>(stream), sms, true, false, ep);
 }
