@@ -54,7 +54,7 @@
 extern "C" {
 #endif
 
-#define MACAQ_ABI_VERSION 4
+#define MACAQ_ABI_VERSION 5  /* 5: the FP8-output calls */
 
 #define MACAQ_OK 0
 #define MACAQ_ERR_NULL (-1)               /* a required pointer is NULL */

@@ -48,7 +48,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_abi_version_and_status_strings(L):
-    assert L.macaq_abi_version() == 4
+    assert L.macaq_abi_version() == 5
     for code, name in mq.STATUS.items():
         assert L.macaq_status_string(code).decode() == name
     assert L.macaq_status_string(-99).decode() == "MACAQ_ERR_UNKNOWN"
