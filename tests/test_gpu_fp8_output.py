@@ -5,7 +5,9 @@ output_dtype parameter; here its FP8 choice): y8 = E4M3(act(v + bias) * y_scale)
 round to nearest even with saturation at +-448.  Compared with the oracle's
 correctly rounded codes (the exact sum in binary64) with the BF16 tests' bound
 carried over to the FP8 grid (tests/helpers.compare_fp8); without an activation
-the codes themselves agree almost everywhere and lie within one E4M3 step.
+the codes themselves agree almost everywhere and lie within one E4M3 step.  The
+dense call runs the fused kernel for M <= 128 (with and without a K split) and
+the quantise-once pair above; the grouped call always the latter.
 """
 import numpy as np
 import pytest
